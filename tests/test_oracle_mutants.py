@@ -1,0 +1,61 @@
+"""Mutation check of the oracle's pins (CPU only).
+
+Each case plants one plausible mistake in a copy of the oracle's C source
+(a dropped term, an off-by-one, a wrong index, a flipped sign, a swapped
+operand), builds it, and runs the pin suite against that build.  The pins
+must reject every mutant.  Mistakes are planted only in the oracle copy,
+never in the CUDA library.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "nsa_oracle.c")
+
+MUTANTS = {
+    "mean_divides_by_l_minus_1": ("round_store(sk / l, c->kv_round)",
+                                  "round_store(sk / (l - 1), c->kv_round)"),
+    "incomplete_block_visible": ("if (t < c->cmp_block - 1) return 0;\n  int n = (t - c->cmp_block + 1) / c->cmp_stride + 1;",
+                                 "if (t < 0) return 0;\n  int n = t / c->cmp_stride + 1;"),
+    "score_wrong_group": ("score_tok[(size_t)(h / G) * nc + j] += p_row[j];",
+                          "score_tok[(size_t)(h % c->Hkv) * nc + j] += p_row[j];"),
+    "tie_goes_to_higher_block": ("(sr == sb && cand[r] < cand[best])",
+                                 "(sr == sb && cand[r] > cand[best])"),
+    "first_block_not_forced": ("for (int i = 0; i < m; ++i) cand[i] = i + 1;",
+                               "for (int i = 0; i < m; ++i) cand[i] = i + 1;\n  if (m > 0) cand[0] = 0;"),
+    "sel_sees_next_token": ("if (p <= t && p < c->T) pos[n++] = p;",
+                            "if (p <= t + 1 && p < c->T) pos[n++] = p;"),
+    "window_one_too_long": ("int lo = t - c->window + 1;", "int lo = t - c->window;"),
+    "lse_drops_max": ("*lse = mx + log(sum);", "*lse = log(sum);"),
+    "bwd_delta_sign": ("double ds = p[s] * (dp - delta);", "double ds = p[s] * (dp + delta);"),
+    "combine_swaps_gates": ("if (c->branch_mask & ORC_SWA) acc += g3[2] * ow[d];",
+                            "if (c->branch_mask & ORC_SWA) acc += g3[1] * ow[d];"),
+    "pool_bwd_not_spread": ("dk[KI(c, b, j * dstr + i, g) + d] += dkc[(size_t)j * D + d] / l;",
+                            "dk[KI(c, b, j * dstr + i, g) + d] += dkc[(size_t)j * D + d];"),
+    "dv_without_prob": ("dvrows[s][d] += p[s] * dO[d];", "dvrows[s][d] += dO[d];"),
+    "dk_uses_key_not_query": ("dkrows[s][d] += scale * ds * qrow[d];",
+                              "dkrows[s][d] += scale * ds * krows[s][d];"),
+    "softmax_scale_dropped": ("logit[s] = scale * dot(qrow, krows[s], D);",
+                              "logit[s] = dot(qrow, krows[s], D);"),
+    "bf16_round_truncates": ("double r = nearbyint(ldexp(m, 8));", "double r = trunc(ldexp(m, 8));"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_reject_mutant(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
+    mut = tmp_path / "mutant.c"
+    mut.write_text(src.replace(old, new))
+    lib = tmp_path / "libmutant.so"
+    subprocess.run(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-o",
+                    str(lib), str(mut), "-lm"], check=True)
+    env = dict(os.environ, NSA_ORACLE_LIB=str(lib), OMP_NUM_THREADS="2")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, f"pins accepted mutant {name}:\n{r.stdout[-2000:]}"
