@@ -1,0 +1,401 @@
+"""Benchmark of the NSA hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl nsa|reference]
+
+One step = one NSA forward (compression + block scores, top-k, selection,
+sliding window, gated combination) over the 340M-shape workload: B=1,
+T=8192, 16 query heads, 4 KV heads (GQA-4), head dim 64, block 64, top-k 16,
+window 512, bf16, with inputs resident in HBM.  L2 is flushed (256 MiB
+write) between timed steps; each step is timed with CUDA events on the
+launching stream.  Rank 0 prints one JSON line.
+
+With N > 1 (torchrun), every rank runs its own independent copy of the
+workload (NSA has no cross-sequence exchange: weak scaling, no data-path
+collective); the reported time is the max over ranks and the value sums the
+tokens of all ranks.
+
+--impl reference times the fp64 CPU oracle on the host cores on a bounded
+sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import sparse_attention_nsa_b200 as nsa  # noqa: E402
+from sparse_attention_nsa_b200 import inputs as W  # noqa: E402
+
+METRIC = "NSA fwd tokens/s & TFLOP/s (frac of bf16 peak) @8192 GQA-4; decode HBM GB/s"
+WORK = W.NSA_340M
+DECODE = W.DECODE_32K
+KERNELS_PER_FORWARD = 6  # compress, cmp+scores, top-k, selection, window, combine
+
+
+# ------------------------------------------------------------------ work model
+def fwd_flops(w, branch_mask=None) -> dict:
+    """Algorithmic FLOPs of one forward: 4*D per (query row, attended key)
+    (QK^T and PV); the compression branch counts 2*D per key when only its
+    scores are needed."""
+    m = w.branch_mask if branch_mask is None else branch_mask
+    l, n, win, D = w.sel_block, w.topk, w.window, w.D
+    sel = swa = cmp = 0
+    for t in range(w.T):
+        sel += min(t + 1, (n - 1) * l + t % l + 1)
+        swa += min(t + 1, win)
+        cmp += min((t + 1) // w.cmp_block, w.Nc)
+    rows = w.B * w.Hq
+    out = {"sel": 4 * D * sel * rows if m & 2 else 0,
+           "swa": 4 * D * swa * rows if m & 4 else 0,
+           "cmp": (4 if m & 1 else 2) * D * cmp * rows if m & 3 else 0}
+    out["total"] = sum(out.values())
+    return out
+
+
+def load_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML (read only)."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            try:  # NVML indexes every GPU of the host; match ours by UUID
+                uuid = str(torch.cuda.get_device_properties(index).uuid)
+                uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+                self._h = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode())
+            except Exception:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def __enter__(self):
+        if self._nv:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def summary(self) -> dict:
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ timing helpers
+class Flusher:
+    def __init__(self, dev):
+        self.buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def __call__(self):
+        self.buf.fill_(1)
+
+
+def timed_steps(fn, steps: int, flush, stream) -> list[float]:
+    """Per-step device time (ms) of fn, with an L2 flush outside each timing."""
+    times = []
+    for _ in range(steps):
+        flush()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        times.append((a, b))
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in times]
+
+
+def barrier_sync(dist_on):
+    torch.cuda.synchronize()
+    if dist_on:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(x: float, dist_on: bool) -> float:
+    if not dist_on:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ CPU oracle leg
+def oracle_tokens_per_s(budget_s: float, seed: int = 0) -> dict:
+    """Time the fp64 CPU oracle on a bounded sample of the bench workload:
+    whole tokens (all heads, all branches), spread over the sequence."""
+    import numpy as np
+
+    import oracle as orc
+    w = WORK
+    inp = W.make_inputs(w, seed=seed)
+    c = orc.Cfg(B=w.B, T=w.T, Hq=w.Hq, Hkv=w.Hkv, D=w.D, cmp_block=w.cmp_block,
+                cmp_stride=w.cmp_stride, sel_block=w.sel_block, topk=w.topk,
+                window=w.window, scale=w.scale, kv_round=orc.KV_BF16,
+                branch_mask=w.branch_mask)
+    q, k, v, g = (inp[n].double().numpy() for n in ("q", "k", "v", "gates"))
+    kc, vc = orc.compress(c, k, v)
+    rng = np.random.default_rng(seed)
+    # calibrate on a small sample, then size the timed sample to the budget
+    n = 64
+    while True:
+        rows = np.stack([np.zeros(n, dtype=int), rng.integers(0, w.T, n)], 1)
+        t0 = time.perf_counter()
+        orc.forward_rows(c, q, k, v, g, rows, kc, vc)
+        dt = time.perf_counter() - t0
+        if dt >= budget_s or n >= w.B * w.T:
+            break
+        n = int(min(w.B * w.T, max(2 * n, n * budget_s / max(dt, 1e-3) * 1.05)))
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return {"value": n / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} whole tokens (16 heads, 3 branches) drawn uniformly from the "
+                      f"T=8192 sequence of {w.name}; compression of the full sequence "
+                      f"precomputed; {dt:.1f} s"}
+
+
+# ------------------------------------------------------------------ main legs
+def run_reference(args, rank: int) -> None:
+    if rank != 0:
+        return
+    budget = max(2.0, min(20.0, 25.0 / max(args.steps, 1)))
+    vals = []
+    cb = None
+    for i in range(args.warmup + args.steps):
+        r = oracle_tokens_per_s(budget if i >= args.warmup else 1.0, seed=0)
+        if i >= args.warmup:
+            vals.append(r["value"])
+            cb = r
+    v = statistics.median(vals)
+    cb["value"] = v
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": WORK.B * WORK.T / v * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORK.name, "B": WORK.B, "T": WORK.T, "Hq": WORK.Hq,
+                       "Hkv": WORK.Hkv, "D": WORK.D, "block": WORK.sel_block,
+                       "topk": WORK.topk, "window": WORK.window},
+            "cpu_baseline": cb,
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_gpu(args, rank: int, world: int, dist_on: bool) -> None:
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    nsa.load()
+    stream = torch.cuda.current_stream()
+    flush = Flusher(dev)
+    w = WORK
+    p = nsa.params_for(w)
+    inp = W.make_inputs(w, seed=rank)
+    q, k, v, g = (inp[n].to(dev) for n in ("q", "k", "v", "gates"))
+    out = torch.empty_like(q)
+    ws = nsa.alloc_workspace(p, dev)
+    saved = {"idx": torch.empty((w.B, w.T, w.Hkv, w.topk), dtype=torch.int32, device=dev)}
+
+    def step():
+        nsa.nsa_forward(p, q, k, v, g, out, saved, ws)
+
+    for _ in range(args.warmup):
+        flush()
+        step()
+    if nsa.nsa_last_device_error() != 0:
+        raise RuntimeError("device-side check failed during warm-up")
+    sampler = ClockSampler(local)
+    barrier_sync(dist_on)
+    with sampler:
+        times = timed_steps(step, args.steps, flush, stream)
+        barrier_sync(dist_on)
+    ms = max_over_ranks(sum(times) / len(times), dist_on)
+    flops = fwd_flops(w)
+    tokens_per_step = w.B * w.T
+    value = tokens_per_step * world / (ms * 1e-3)
+
+    # dominant kernel alone (selection branch), same inputs, same flushing
+    o_sel = torch.empty_like(q)
+    for _ in range(2):
+        nsa.nsa_sel_attn_fwd(p, q, k, v, saved["idx"], o_sel, None)
+    sel_ms = statistics.mean(timed_steps(
+        lambda: nsa.nsa_sel_attn_fwd(p, q, k, v, saved["idx"], o_sel, None),
+        args.steps, flush, stream))
+    peaks = load_peaks()
+    sel_tflops = flops["sel"] / (sel_ms * 1e-3) / 1e12
+
+    # end to end through the C ABI with host buffers (pinned), copies timed
+    hq, hk, hv, hg = (x.cpu().pin_memory() for x in (q, k, v, g))
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        g.copy_(hg, non_blocking=True)
+        step()
+        hout.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    e2e_ms = max_over_ranks(statistics.mean(timed_steps(e2e_step, args.steps, flush, stream)),
+                            dist_on)
+    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hg))
+    d2h = hout.numel() * hout.element_size()
+
+    # decode (B=64 sequences, 32768-token caches): HBM GB/s
+    dec = run_decode(dev, flush, stream, args.steps, peaks)
+
+    barrier_sync(dist_on)
+    if rank != 0:
+        return
+    clocks = sampler.summary()
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv,
+                   "D": w.D, "block": w.sel_block, "topk": w.topk, "window": w.window,
+                   "l2": "flushed between steps (256 MiB write)",
+                   "parallelism": f"replicas x{world}"},
+        "tflops": flops["total"] * world / (ms * 1e-3) / 1e12,
+        "frac_bf16_peak": flops["total"] / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+        "flops_per_step": flops,
+        "roofline": {"bound": "tensor", "kernel": "selection attention (nsa_sel_attn_fwd)",
+                     "achieved": sel_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": sel_tflops / peaks["bf16_tflops"], "traffic": None,
+                     "ms_per_launch": sel_ms, "peak_source": peaks["source"] + " burst bf16"},
+        "decode": dec,
+        "e2e": {"value": tokens_per_step * world / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": KERNELS_PER_FORWARD * args.steps,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_tokens_per_s(budget_s=12.0)
+    print(json.dumps(line), flush=True)
+
+
+def run_decode(dev, flush, stream, steps, peaks) -> dict:
+    w = DECODE
+    inp = W.make_decode_inputs(w, seed=0)
+    kcache, vcache = inp["k_cache"].to(dev), inp["v_cache"].to(dev)
+    pk = nsa.params_for(w)
+    kc = torch.empty((w.B, w.Nc, w.Hkv, w.D), dtype=w.dtype, device=dev)
+    vc = torch.empty_like(kc)
+    nsa.nsa_compress(pk, kcache, vcache, kc, vc)
+    p = nsa.params_for(w, Tq=1)
+    q = inp["q"].to(dev).unsqueeze(1).contiguous()
+    g = inp["gates"].to(dev).unsqueeze(1).contiguous()
+    out = torch.empty_like(q)
+    idx = torch.empty((w.B, 1, w.Hkv, w.topk), dtype=torch.int32, device=dev)
+    ws = nsa.alloc_workspace(p, dev)
+
+    def step():
+        nsa.nsa_decode(p, q, kcache, vcache, kc, vc, g, out, idx, ws)
+
+    for _ in range(3):
+        step()
+    us = statistics.mean(timed_steps(step, steps, flush, stream)) * 1e3
+    # algorithmic bytes: q, gates, out, the whole compressed cache, and the
+    # union of selected-block keys and window keys (K and V) per sequence
+    ii = idx.cpu().numpy()
+    t = w.T - 1
+    keys = 0
+    for b in range(w.B):
+        for g_ in range(w.Hkv):
+            s = set()
+            for j in ii[b, 0, g_]:
+                if j >= 0:
+                    s.update(range(j * w.sel_block, min(j * w.sel_block + w.sel_block, t + 1)))
+            s.update(range(max(0, t - w.window + 1), t + 1))
+            keys += len(s)
+    es = 2
+    bytes_ = (w.B * w.Hq * w.D * es * 2 + w.B * w.Hq * 3 * 4
+              + w.B * w.Nc * w.Hkv * w.D * es * 2 + keys * w.D * es * 2)
+    gbs = bytes_ / (us * 1e-6) / 1e9
+    return {"workload": w.name, "us_per_step": us, "algorithmic_bytes": bytes_,
+            "gbs": gbs, "peak_gbs": peaks["hbm_gbs"], "frac": gbs / peaks["hbm_gbs"],
+            "tokens_per_s": w.B / (us * 1e-6)}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="nsa", choices=["nsa", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    dist_on = world > 1
+    if dist_on:
+        import datetime
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_gpu(args, rank, world, dist_on)
+    finally:
+        if dist_on:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

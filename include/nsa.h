@@ -1,0 +1,218 @@
+/*
+ * nsa.h -- C ABI of libnsa, a B200 (sm_100a) implementation of Native
+ * Sparse Attention (NSA) with mean-pooled compression.
+ *
+ * The method: "DeepSeek's Native Sparse Attention" (bycloud newsletter #44,
+ * section "How Does Native Sparse Attention Work?") describes three
+ * attention branches per query -- COMPRESSION (attend to one summary
+ * key/value per block of tokens), SELECTION (score the blocks, keep the most
+ * important ones in raw form and attend to them) and SLIDING WINDOW (attend
+ * to the most recent tokens) -- whose outputs are merged by learned gates.
+ * "Sparsity is Cool: Reverse-Engineering MoBA and NSA" (sections TL;DR,
+ * Method, Key claims) fixes the variant built here: mean-pooling instead of
+ * an MLP for compression, block 64, top-k 16, window 512, GQA/MQA KV
+ * sharing with one selection per KV group, the first block always selected,
+ * and branch pruning at inference.
+ *
+ * ------------------------------------------------------------------------
+ * Conventions shared by every entry point
+ * ------------------------------------------------------------------------
+ * Pointers.  Every tensor argument is a DEVICE pointer owned by the caller,
+ *   contiguous in the layout stated, 16-byte aligned.  The library keeps no
+ *   reference after the call returns and allocates no device memory:
+ *   scratch space comes from a caller-provided workspace.
+ * Stream.  `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *   stream).  Every entry point only enqueues work on that stream and
+ *   returns without synchronising, except nsa_last_device_error.
+ * Shapes.  B batch, T keys per sequence, Tq queries per sequence (the
+ *   queries are the LAST Tq positions of the T-key sequence: query i sits at
+ *   position T - Tq + i; prefill has Tq = T, decode Tq = 1), Hq query heads,
+ *   Hkv key/value heads, G = Hq / Hkv query heads per KV group (query head h
+ *   reads KV head h / G), D head dim (64).  l = block size.
+ *   Nc = number of compressed blocks = floor(T / l) (complete blocks only).
+ * Layouts (row-major):
+ *   q, o_*, out          [B, Tq, Hq, D]   dtype
+ *   k, v                 [B, T, Hkv, D]   dtype
+ *   kc, vc               [B, Nc, Hkv, D]  dtype
+ *   gates                [B, Tq, Hq, 3]   float32, branch order (cmp, sel, swa)
+ *   lse_*                [B, Tq, Hq]      float32, natural-log sum-exp
+ *   score                [B, Tq, Hkv, Nc] float32
+ *   idx                  [B, Tq, Hkv, topk] int32, ascending, -1 padded
+ *   dtype is float32 (NSA_F32) or bfloat16 (NSA_BF16) for the whole call.
+ * Errors.  Arguments are validated before anything is enqueued; a bad
+ *   argument returns NSA_ERR_INVALID_ARG and a valid but unimplemented
+ *   geometry NSA_ERR_UNSUPPORTED, with nothing launched.  A failed launch
+ *   returns NSA_ERR_CUDA.  Device-side bounded waits and checks never trap:
+ *   they record a code read back by nsa_last_device_error.
+ */
+#ifndef NSA_H_
+#define NSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  NSA_OK = 0,
+  NSA_ERR_INVALID_ARG = 1,  /* null pointer, bad shape or parameter        */
+  NSA_ERR_UNSUPPORTED = 2,  /* valid NSA geometry this build does not run  */
+  NSA_ERR_CUDA = 3,         /* a CUDA call or launch failed                */
+  NSA_ERR_TIMEOUT = 4,      /* a bounded device-side wait expired          */
+  NSA_ERR_DEVICE_CHECK = 5, /* a device-side consistency check failed      */
+  NSA_ERR_WORKSPACE = 6     /* workspace missing or smaller than required  */
+} nsa_status;
+
+typedef enum { NSA_F32 = 0, NSA_BF16 = 1 } nsa_dtype;
+
+enum {
+  NSA_BRANCH_CMP = 1, /* compression branch  */
+  NSA_BRANCH_SEL = 2, /* selection branch    */
+  NSA_BRANCH_SWA = 4, /* sliding window      */
+  NSA_BRANCH_ALL = 7
+};
+
+/* Problem description.  The block geometry follows the pages' problem
+ * statement: compression block size l and stride d, selection block size l',
+ * top-k n, window w.  This build runs l = d = l' (the geometry used in
+ * "Sparsity is Cool", Method: block 64 for both, stride = block); other
+ * combinations return NSA_ERR_UNSUPPORTED. */
+typedef struct {
+  int B, T, Tq, Hq, Hkv, D;
+  int cmp_block;   /* l  : tokens per compressed block              */
+  int cmp_stride;  /* d  : stride between compressed blocks (= l)   */
+  int sel_block;   /* l' : tokens per selection block (= l)         */
+  int topk;        /* n  : selected blocks per (query, KV group), >= 2 */
+  int window;      /* w  : sliding-window length in keys, >= 1      */
+  float scale;     /* softmax scale, normally 1/sqrt(D)             */
+  int dtype;       /* nsa_dtype of q/k/v/kc/vc/o_*                   */
+  int branch_mask; /* NSA_BRANCH_* bits of the branches to combine   */
+} nsa_params;
+
+/* Optional intermediate tensors of nsa_forward.  A non-NULL pointer makes
+ * nsa_forward write that tensor there (layouts above); a NULL pointer puts
+ * it in the workspace.  nsa_sel_attn_bwd needs idx, o_sel and lse_sel. */
+typedef struct {
+  void* kc;
+  void* vc;
+  void* o_cmp;
+  float* lse_cmp;
+  float* score;
+  int32_t* idx;
+  void* o_sel;
+  float* lse_sel;
+  void* o_swa;
+  float* lse_swa;
+} nsa_saved;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* nsa_status_string(nsa_status s);
+
+/* Validate a parameter block without launching anything.  Returns NSA_OK,
+ * NSA_ERR_INVALID_ARG or NSA_ERR_UNSUPPORTED. */
+nsa_status nsa_check_params(const nsa_params* p);
+
+/* Bytes of workspace nsa_forward / nsa_decode need for parameters p (with
+ * every nsa_saved pointer NULL; passing buffers never increases it). */
+nsa_status nsa_workspace_size(const nsa_params* p, size_t* bytes);
+
+/* Synchronise `stream`, then read and clear the library's device error
+ * word: NSA_OK, NSA_ERR_TIMEOUT or NSA_ERR_DEVICE_CHECK (NSA_ERR_CUDA if
+ * the synchronisation itself failed). */
+nsa_status nsa_last_device_error(void* stream);
+
+/* ---- compression: mean-pool consecutive blocks --------------------------
+ * kc[b, j, g, :] = (1/l) * sum_{i<l} k[b, j*l + i, g, :], same for vc.
+ * Passage: "Sparsity is Cool", Method and Key claims (mean-pooling replaces
+ * NSA's MLP); "DeepSeek's Native Sparse Attention", COMPRESSION.
+ * k, v [B, T, Hkv, D] -> kc, vc [B, Nc, Hkv, D].  The sum is exact (fp64)
+ * and rounded once to dtype (round-to-nearest-even).  Tq is ignored. */
+nsa_status nsa_compress(const nsa_params* p, const void* k, const void* v,
+                        void* kc, void* vc, void* stream);
+
+/* ---- compression branch and block importance ----------------------------
+ * For query position t: compressed block j is visible iff its last token
+ * j*l + l - 1 <= t.  P[t,h,:] = softmax over visible j of scale*q.kc_j;
+ * o_cmp = sum_j P v c_j (0 and lse = -inf when nothing is visible);
+ * score[t,g,j] = sum over the G heads h of group g of P[t,h,j] (0 for
+ * invisible j).  Passage: "DeepSeek's Native Sparse Attention", COMPRESSION
+ * and SELECTION (importance reuses the compression attention scores).
+ * o_cmp and lse_cmp may be NULL (scores only: the branch-pruned case of
+ * "Sparsity is Cool", Key claims). */
+nsa_status nsa_cmp_attn_scores(const nsa_params* p, const void* q,
+                               const void* kc, const void* vc, void* o_cmp,
+                               float* lse_cmp, float* score, void* stream);
+
+/* ---- top-k block selection per (query, KV group) ------------------------
+ * cur = t / l'.  If cur + 1 <= topk, idx = 0..cur then -1 padding.  Else
+ * blocks 0 and cur are forced and the topk - 2 highest-scoring blocks of
+ * 1..cur-1 are added (equal scores: lower block index first); idx is
+ * ascending.  Passage: "DeepSeek's Native Sparse Attention", SELECTION;
+ * "Sparsity is Cool", Method (block 64 / top-k 16) and Key claims (always
+ * include the first block).  score [B,Tq,Hkv,Nc] -> idx [B,Tq,Hkv,topk]. */
+nsa_status nsa_select_topk(const nsa_params* p, const float* score,
+                           int32_t* idx, void* stream);
+
+/* ---- selection branch ----------------------------------------------------
+ * o_sel[t,h] = softmax-weighted sum of v over the keys s <= t that lie in
+ * the blocks idx[t, h/G, :] (entries < 0 ignored); lse_sel its log-sum-exp.
+ * Passage: "DeepSeek's Native Sparse Attention", SELECTION and the kernel
+ * paragraph (queries sharing the same blocks are grouped: one selection per
+ * KV group, all G heads read the same blocks).  Block indices must be
+ * ascending, distinct and causal (<= t / l'); the kernel checks this and
+ * records NSA_ERR_DEVICE_CHECK instead of reading out of bounds. */
+nsa_status nsa_sel_attn_fwd(const nsa_params* p, const void* q, const void* k,
+                            const void* v, const int32_t* idx, void* o_sel,
+                            float* lse_sel, void* stream);
+
+/* ---- sliding-window branch -----------------------------------------------
+ * o_swa[t,h] attends to keys max(0, t-w+1) <= s <= t.
+ * Passage: "DeepSeek's Native Sparse Attention", SLIDING WINDOW;
+ * "Sparsity is Cool", Method (window 512). */
+nsa_status nsa_swa_fwd(const nsa_params* p, const void* q, const void* k,
+                       const void* v, void* o_swa, float* lse_swa,
+                       void* stream);
+
+/* ---- gated combination ---------------------------------------------------
+ * out = g_cmp*o_cmp + g_sel*o_sel + g_swa*o_swa over the branches enabled
+ * in branch_mask (a disabled branch's pointer may be NULL).  Gates are
+ * post-sigmoid values.  Passage: "DeepSeek's Native Sparse Attention"
+ * (outputs merged by gates from a small network); "Sparsity is Cool",
+ * TL;DR and Key claims (unused branches pruned at inference). */
+nsa_status nsa_gate_combine(const nsa_params* p, const float* gates,
+                            const void* o_cmp, const void* o_sel,
+                            const void* o_swa, void* out, void* stream);
+
+/* ---- whole forward ---------------------------------------------------------
+ * compress -> compression branch + scores -> top-k -> selection branch ->
+ * window branch -> gated combination, in one call.  With NSA_BRANCH_CMP
+ * off, the scores are still computed (selection needs them) but the
+ * compression output is not.  With NSA_BRANCH_SEL off the selection path
+ * (scores, top-k, selection) is skipped entirely, and so is the compression
+ * branch if it is off too.  `saved` may be NULL.  workspace must hold at
+ * least nsa_workspace_size(p) bytes (256-byte aligned). */
+nsa_status nsa_forward(const nsa_params* p, const void* q, const void* k,
+                       const void* v, const float* gates, void* out,
+                       const nsa_saved* saved, void* workspace,
+                       size_t workspace_bytes, void* stream);
+
+/* ---- decode ----------------------------------------------------------------
+ * One query per sequence at position T-1 (p->Tq must be 1) against caches
+ * k_cache/v_cache [B, T, Hkv, D] that already hold that position, and the
+ * compressed caches kc_cache/vc_cache [B, Nc, Hkv, D] (nsa_compress of the
+ * caches).  q [B, 1, Hq, D], gates [B, 1, Hq, 3], out [B, 1, Hq, D];
+ * idx_out [B, 1, Hkv, topk] may be NULL.  Same arithmetic as nsa_forward
+ * for that one position. */
+nsa_status nsa_decode(const nsa_params* p, const void* q, const void* k_cache,
+                      const void* v_cache, const void* kc_cache,
+                      const void* vc_cache, const float* gates, void* out,
+                      int32_t* idx_out, void* workspace, size_t workspace_bytes,
+                      void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NSA_H_ */

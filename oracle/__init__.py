@@ -286,18 +286,22 @@ def backward(cfg: Cfg, q, k, v, gates, dout):
     return dq, dk, dv, dg
 
 
-def decode(cfg: Cfg, q_last, kcache, vcache, kc, vc, gates_last):
+def decode(cfg: Cfg, q_last, kcache, vcache, kc, vc, gates_last, with_score=False):
     """One query per sequence at position T-1 (cfg.T = cache length).
 
     q_last [B, Hq, D], caches [B, T, Hkv, D], kc/vc [B, Nc, Hkv, D],
-    gates_last [B, Hq, 3].  Returns (out [B, Hq, D], idx [B, Hkv, topk]).
+    gates_last [B, Hq, 3].  Returns (out [B, Hq, D], idx [B, Hkv, topk]),
+    plus the block scores [B, Hkv, Nc] when with_score=True.
     """
     lib = _load()
     q_last, kcache, vcache = _f64(q_last), _f64(kcache), _f64(vcache)
     kc, vc, gates_last = _f64(kc), _f64(vc), _f64(gates_last)
     out = np.zeros((cfg.B, cfg.Hq, cfg.D))
     idx = np.zeros((cfg.B, cfg.Hkv, cfg.topk), dtype=np.int32)
+    score = np.zeros((cfg.B, cfg.Hkv, max(cfg.Nc, 1)))
     cc = cfg.c()
     lib.orc_decode(C.byref(cc), _p(q_last), _p(kcache), _p(vcache), _p(kc), _p(vc),
-                   _p(gates_last), _p(out), _p(idx))
+                   _p(gates_last), _p(out), _p(idx), _p(score))
+    if with_score:
+        return out, idx, score[..., :cfg.Nc]
     return out, idx

@@ -708,12 +708,14 @@ void orc_backward(const orc_cfg* c, const double* q, const double* k,
 /* L keys/values (its own already appended) and the compressed cache  */
 /* of the same sequence.  Same per-row math as the forward.            */
 /* q [B, Hq, D]; kcache/vcache [B, L, Hkv, D]; kc/vc [B, Nc, Hkv, D];  */
-/* gates [B, Hq, 3]; out [B, Hq, D]; idx [B, Hkv, topk].               */
+/* gates [B, Hq, 3]; out [B, Hq, D]; idx [B, Hkv, topk];               */
+/* score_out (optional) [B, Hkv, Nc].                                  */
 /* The cfg's T is the cache length L.                                  */
 /* ================================================================== */
 void orc_decode(const orc_cfg* c, const double* q_last, const double* kcache,
                 const double* vcache, const double* kc, const double* vc,
-                const double* gates_last, double* out, int* idx_out) {
+                const double* gates_last, double* out, int* idx_out,
+                double* score_out) {
   const int nc = orc_num_cmp_blocks(c);
   const int L = c->T;
   const size_t HD = (size_t)c->Hq * c->D;
@@ -728,6 +730,8 @@ void orc_decode(const orc_cfg* c, const double* q_last, const double* kcache,
                       gates_last + (size_t)b * c->Hq * 3, b, L - 1, oc, lse, sc,
                       idx_out + (size_t)b * c->Hkv * c->topk, os, lse + c->Hq,
                       ow, lse + 2 * c->Hq, out + (size_t)b * HD);
+    if (score_out)
+      memcpy(score_out + (size_t)b * c->Hkv * nc, sc, (size_t)c->Hkv * nc * sizeof(double));
     free(oc);
     free(os);
     free(ow);

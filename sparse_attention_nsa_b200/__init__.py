@@ -1,1 +1,17 @@
-"""B200-native Native Sparse Attention (placeholder until the binding lands)."""
+"""B200-native Native Sparse Attention (NSA).
+
+The compute path is libnsa.so (C ABI in include/nsa.h): hand-written sm_100a
+CUDA kernels for mean-pool compression, the compression branch with block
+scores, per-KV-group top-k selection, selection and sliding-window
+attention, the gated combination, the whole forward and decode.  This
+package is its thin ctypes binding (``abi``) plus seeded synthetic workloads
+(``inputs``).  Build the library with ``python -m sparse_attention_nsa_b200.build``.
+"""
+from .abi import (EXPORTS, NSA_BF16, NSA_BRANCH_ALL, NSA_BRANCH_CMP, NSA_BRANCH_SEL,
+                  NSA_BRANCH_SWA, NSA_F32, NsaError, Params, Saved, alloc_workspace,
+                  forward, load, make_params, nsa_check_params, nsa_cmp_attn_scores,
+                  nsa_compress, nsa_decode, nsa_forward, nsa_gate_combine,
+                  nsa_last_device_error, nsa_sel_attn_fwd, nsa_select_topk,
+                  nsa_status_string, nsa_swa_fwd, nsa_workspace_size, params_for)
+
+__all__ = [n for n in dir() if not n.startswith("_")]

@@ -1,0 +1,302 @@
+"""ctypes binding of libnsa (include/nsa.h), one function per C entry point.
+
+Argument marshalling only: every function checks that its torch tensors
+live on the current CUDA device with the dtype, shape and contiguity the C
+ABI documents, passes their device pointers and the current CUDA stream to
+the library, and raises NsaError on a non-OK status.  All arithmetic runs in
+libnsa's CUDA kernels; there is no fallback path.  PyTorch only provides
+device memory and streams.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libnsa.so")
+
+NSA_F32, NSA_BF16 = 0, 1
+NSA_BRANCH_CMP, NSA_BRANCH_SEL, NSA_BRANCH_SWA = 1, 2, 4
+NSA_BRANCH_ALL = 7
+
+STATUS = {0: "NSA_OK", 1: "NSA_ERR_INVALID_ARG", 2: "NSA_ERR_UNSUPPORTED",
+          3: "NSA_ERR_CUDA", 4: "NSA_ERR_TIMEOUT", 5: "NSA_ERR_DEVICE_CHECK",
+          6: "NSA_ERR_WORKSPACE"}
+
+# every symbol include/nsa.h declares
+EXPORTS = ("nsa_status_string", "nsa_check_params", "nsa_workspace_size",
+           "nsa_last_device_error", "nsa_compress", "nsa_cmp_attn_scores",
+           "nsa_select_topk", "nsa_sel_attn_fwd", "nsa_swa_fwd", "nsa_gate_combine",
+           "nsa_forward", "nsa_decode")
+
+
+class NsaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+
+
+class Params(C.Structure):
+    """Mirror of nsa_params."""
+    _fields_ = [("B", C.c_int), ("T", C.c_int), ("Tq", C.c_int), ("Hq", C.c_int),
+                ("Hkv", C.c_int), ("D", C.c_int), ("cmp_block", C.c_int),
+                ("cmp_stride", C.c_int), ("sel_block", C.c_int), ("topk", C.c_int),
+                ("window", C.c_int), ("scale", C.c_float), ("dtype", C.c_int),
+                ("branch_mask", C.c_int)]
+
+    @property
+    def Nc(self) -> int:
+        return self.T // self.cmp_block
+
+    @property
+    def G(self) -> int:
+        return self.Hq // self.Hkv
+
+    @property
+    def torch_dtype(self) -> torch.dtype:
+        return torch.bfloat16 if self.dtype == NSA_BF16 else torch.float32
+
+
+class Saved(C.Structure):
+    """Mirror of nsa_saved (device pointers, 0 = put it in the workspace)."""
+    _fields_ = [("kc", C.c_void_p), ("vc", C.c_void_p), ("o_cmp", C.c_void_p),
+                ("lse_cmp", C.c_void_p), ("score", C.c_void_p), ("idx", C.c_void_p),
+                ("o_sel", C.c_void_p), ("lse_sel", C.c_void_p), ("o_swa", C.c_void_p),
+                ("lse_swa", C.c_void_p)]
+
+
+_lib = None
+
+
+def load():
+    """Load libnsa.so; raise if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m sparse_attention_nsa_b200.build`")
+        lib = C.CDLL(LIB_PATH)
+        vp, P = C.c_void_p, C.POINTER(Params)
+        sig = {
+            "nsa_status_string": ([C.c_int], C.c_char_p),
+            "nsa_check_params": ([P], C.c_int),
+            "nsa_workspace_size": ([P, C.POINTER(C.c_size_t)], C.c_int),
+            "nsa_last_device_error": ([vp], C.c_int),
+            "nsa_compress": ([P, vp, vp, vp, vp, vp], C.c_int),
+            "nsa_cmp_attn_scores": ([P, vp, vp, vp, vp, vp, vp, vp], C.c_int),
+            "nsa_select_topk": ([P, vp, vp, vp], C.c_int),
+            "nsa_sel_attn_fwd": ([P, vp, vp, vp, vp, vp, vp, vp], C.c_int),
+            "nsa_swa_fwd": ([P, vp, vp, vp, vp, vp, vp], C.c_int),
+            "nsa_gate_combine": ([P, vp, vp, vp, vp, vp, vp], C.c_int),
+            "nsa_forward": ([P, vp, vp, vp, vp, vp, C.POINTER(Saved), vp, C.c_size_t, vp],
+                            C.c_int),
+            "nsa_decode": ([P, vp, vp, vp, vp, vp, vp, vp, vp, vp, C.c_size_t, vp], C.c_int),
+        }
+        for name, (args, res) in sig.items():
+            f = getattr(lib, name)
+            f.argtypes = args
+            f.restype = res
+        _lib = lib
+    return _lib
+
+
+def make_params(B, T, Hq, Hkv, D=64, *, Tq=None, cmp_block=64, cmp_stride=None,
+                sel_block=None, topk=16, window=512, scale=None, dtype=NSA_BF16,
+                branch_mask=NSA_BRANCH_ALL) -> Params:
+    if isinstance(dtype, torch.dtype):
+        dtype = NSA_BF16 if dtype == torch.bfloat16 else NSA_F32
+    return Params(B, T, T if Tq is None else Tq, Hq, Hkv, D, cmp_block,
+                  cmp_block if cmp_stride is None else cmp_stride,
+                  cmp_block if sel_block is None else sel_block, topk, window,
+                  float(D ** -0.5 if scale is None else scale), dtype, branch_mask)
+
+
+def params_for(w, Tq=None) -> Params:
+    """Params of a sparse_attention_nsa_b200.inputs.Workload."""
+    return make_params(w.B, w.T, w.Hq, w.Hkv, w.D, Tq=Tq, cmp_block=w.cmp_block,
+                       cmp_stride=w.cmp_stride, sel_block=w.sel_block, topk=w.topk,
+                       window=w.window, scale=w.scale, dtype=w.dtype,
+                       branch_mask=w.branch_mask)
+
+
+# ------------------------------------------------------------------ helpers
+def _stream(stream):
+    if stream is None:
+        return C.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return C.c_void_p(stream.cuda_stream)
+    return C.c_void_p(int(stream))
+
+
+def _ptr(t, shape=None, dtype=None, name="tensor", nullable=False):
+    if t is None:
+        if nullable:
+            return None
+        raise ValueError(f"{name} is required")
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return C.c_void_p(t.data_ptr())
+
+
+def _check(st: int, where: str):
+    if st != 0:
+        raise NsaError(st, where)
+
+
+def _shapes(p: Params):
+    B, T, Tq, Hq, Hkv, D = p.B, p.T, p.Tq, p.Hq, p.Hkv, p.D
+    return {"q": (B, Tq, Hq, D), "k": (B, T, Hkv, D), "kc": (B, p.Nc, Hkv, D),
+            "o": (B, Tq, Hq, D), "lse": (B, Tq, Hq), "score": (B, Tq, Hkv, p.Nc),
+            "idx": (B, Tq, Hkv, p.topk), "gates": (B, Tq, Hq, 3)}
+
+
+# ------------------------------------------------------------------ entry points
+def nsa_status_string(status: int) -> str:
+    return load().nsa_status_string(status).decode()
+
+
+def nsa_check_params(p: Params) -> int:
+    return load().nsa_check_params(C.byref(p))
+
+
+def nsa_workspace_size(p: Params) -> int:
+    n = C.c_size_t(0)
+    _check(load().nsa_workspace_size(C.byref(p), C.byref(n)), "nsa_workspace_size")
+    return n.value
+
+
+def nsa_last_device_error(stream=None) -> int:
+    return load().nsa_last_device_error(_stream(stream))
+
+
+def nsa_compress(p: Params, k, v, kc, vc, stream=None):
+    s, dt = _shapes(p), p.torch_dtype
+    _check(load().nsa_compress(C.byref(p), _ptr(k, s["k"], dt, "k"), _ptr(v, s["k"], dt, "v"),
+                               _ptr(kc, s["kc"], dt, "kc"), _ptr(vc, s["kc"], dt, "vc"),
+                               _stream(stream)), "nsa_compress")
+
+
+def nsa_cmp_attn_scores(p: Params, q, kc, vc, o_cmp, lse_cmp, score, stream=None):
+    s, dt = _shapes(p), p.torch_dtype
+    _check(load().nsa_cmp_attn_scores(
+        C.byref(p), _ptr(q, s["q"], dt, "q"), _ptr(kc, s["kc"], dt, "kc"),
+        _ptr(vc, s["kc"], dt, "vc"), _ptr(o_cmp, s["o"], dt, "o_cmp", True),
+        _ptr(lse_cmp, s["lse"], torch.float32, "lse_cmp", True),
+        _ptr(score, s["score"], torch.float32, "score"), _stream(stream)),
+        "nsa_cmp_attn_scores")
+
+
+def nsa_select_topk(p: Params, score, idx, stream=None):
+    s = _shapes(p)
+    _check(load().nsa_select_topk(C.byref(p), _ptr(score, s["score"], torch.float32, "score"),
+                                  _ptr(idx, s["idx"], torch.int32, "idx"), _stream(stream)),
+           "nsa_select_topk")
+
+
+def nsa_sel_attn_fwd(p: Params, q, k, v, idx, o_sel, lse_sel, stream=None):
+    s, dt = _shapes(p), p.torch_dtype
+    _check(load().nsa_sel_attn_fwd(
+        C.byref(p), _ptr(q, s["q"], dt, "q"), _ptr(k, s["k"], dt, "k"),
+        _ptr(v, s["k"], dt, "v"), _ptr(idx, s["idx"], torch.int32, "idx"),
+        _ptr(o_sel, s["o"], dt, "o_sel"), _ptr(lse_sel, s["lse"], torch.float32, "lse_sel", True),
+        _stream(stream)), "nsa_sel_attn_fwd")
+
+
+def nsa_swa_fwd(p: Params, q, k, v, o_swa, lse_swa, stream=None):
+    s, dt = _shapes(p), p.torch_dtype
+    _check(load().nsa_swa_fwd(
+        C.byref(p), _ptr(q, s["q"], dt, "q"), _ptr(k, s["k"], dt, "k"),
+        _ptr(v, s["k"], dt, "v"), _ptr(o_swa, s["o"], dt, "o_swa"),
+        _ptr(lse_swa, s["lse"], torch.float32, "lse_swa", True), _stream(stream)),
+        "nsa_swa_fwd")
+
+
+def nsa_gate_combine(p: Params, gates, o_cmp, o_sel, o_swa, out, stream=None):
+    s, dt = _shapes(p), p.torch_dtype
+    m = p.branch_mask
+    _check(load().nsa_gate_combine(
+        C.byref(p), _ptr(gates, s["gates"], torch.float32, "gates"),
+        _ptr(o_cmp, s["o"], dt, "o_cmp", not m & 1), _ptr(o_sel, s["o"], dt, "o_sel", not m & 2),
+        _ptr(o_swa, s["o"], dt, "o_swa", not m & 4), _ptr(out, s["o"], dt, "out"),
+        _stream(stream)), "nsa_gate_combine")
+
+
+def nsa_forward(p: Params, q, k, v, gates, out, saved: dict | None = None,
+                workspace=None, stream=None):
+    """saved: optional dict of tensors named like nsa_saved's fields."""
+    s, dt = _shapes(p), p.torch_dtype
+    sv = Saved()
+    if saved:
+        want = {"kc": (s["kc"], dt), "vc": (s["kc"], dt), "o_cmp": (s["o"], dt),
+                "lse_cmp": (s["lse"], torch.float32), "score": (s["score"], torch.float32),
+                "idx": (s["idx"], torch.int32), "o_sel": (s["o"], dt),
+                "lse_sel": (s["lse"], torch.float32), "o_swa": (s["o"], dt),
+                "lse_swa": (s["lse"], torch.float32)}
+        for name, t in saved.items():
+            shp, tdt = want[name]
+            setattr(sv, name, _ptr(t, shp, tdt, name).value)
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr, ws_bytes = _ptr(workspace, name="workspace"), workspace.numel() * workspace.element_size()
+    _check(load().nsa_forward(
+        C.byref(p), _ptr(q, s["q"], dt, "q"), _ptr(k, s["k"], dt, "k"), _ptr(v, s["k"], dt, "v"),
+        _ptr(gates, s["gates"], torch.float32, "gates"), _ptr(out, s["o"], dt, "out"),
+        C.byref(sv), ws_ptr, ws_bytes, _stream(stream)), "nsa_forward")
+
+
+def nsa_decode(p: Params, q, k_cache, v_cache, kc_cache, vc_cache, gates, out,
+               idx_out=None, workspace=None, stream=None):
+    s, dt = _shapes(p), p.torch_dtype
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr, ws_bytes = _ptr(workspace, name="workspace"), workspace.numel() * workspace.element_size()
+    _check(load().nsa_decode(
+        C.byref(p), _ptr(q, s["q"], dt, "q"), _ptr(k_cache, s["k"], dt, "k_cache"),
+        _ptr(v_cache, s["k"], dt, "v_cache"), _ptr(kc_cache, s["kc"], dt, "kc_cache", p.Nc == 0),
+        _ptr(vc_cache, s["kc"], dt, "vc_cache", p.Nc == 0),
+        _ptr(gates, s["gates"], torch.float32, "gates"), _ptr(out, s["o"], dt, "out"),
+        _ptr(idx_out, s["idx"], torch.int32, "idx_out", True), ws_ptr, ws_bytes,
+        _stream(stream)), "nsa_decode")
+
+
+# ------------------------------------------------------------------ conveniences
+def alloc_workspace(p: Params, device=None) -> torch.Tensor:
+    n = nsa_workspace_size(p)
+    return torch.empty(max(n, 1), dtype=torch.uint8, device=device or "cuda")
+
+
+def forward(p: Params, q, k, v, gates, keep: bool = False, workspace=None, stream=None):
+    """Allocate outputs with torch and run nsa_forward.
+
+    Returns out, or (out, saved-dict) with every intermediate when keep=True.
+    """
+    s, dt = _shapes(p), p.torch_dtype
+    dev = q.device
+    out = torch.empty(s["o"], dtype=dt, device=dev)
+    saved = None
+    if keep:
+        saved = {"kc": torch.empty(s["kc"], dtype=dt, device=dev),
+                 "vc": torch.empty(s["kc"], dtype=dt, device=dev),
+                 "o_cmp": torch.zeros(s["o"], dtype=dt, device=dev),
+                 "lse_cmp": torch.zeros(s["lse"], dtype=torch.float32, device=dev),
+                 "score": torch.zeros(s["score"], dtype=torch.float32, device=dev),
+                 "idx": torch.zeros(s["idx"], dtype=torch.int32, device=dev),
+                 "o_sel": torch.zeros(s["o"], dtype=dt, device=dev),
+                 "lse_sel": torch.zeros(s["lse"], dtype=torch.float32, device=dev),
+                 "o_swa": torch.zeros(s["o"], dtype=dt, device=dev),
+                 "lse_swa": torch.zeros(s["lse"], dtype=torch.float32, device=dev)}
+        saved = {k_: t for k_, t in saved.items() if t.numel() > 0}
+    if workspace is None:
+        workspace = alloc_workspace(p, dev)
+    nsa_forward(p, q, k, v, gates, out, saved, workspace, stream)
+    return (out, saved) if keep else out

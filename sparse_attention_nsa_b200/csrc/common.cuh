@@ -1,0 +1,73 @@
+// common.cuh -- device helpers shared by the libnsa kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace nsa {
+
+using bf16 = __nv_bfloat16;
+
+// Codes written to the library's device error word (first writer wins).
+enum : int {
+  kDevOk = 0,
+  kDevTimeout = 1,   // a bounded wait gave up
+  kDevBadIndex = 2,  // a block index was out of range / not causal / unsorted
+};
+
+__device__ __forceinline__ void record_error(int* err, int code) {
+  if (err) atomicCAS(err, 0, code);
+}
+
+// ---- scalar load/store in the path dtype, arithmetic in fp32 -------------
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(bf16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ bf16 from_f32<bf16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// Round a double to bfloat16, nearest-even, on the binary64 bit pattern:
+// bfloat16 keeps 7 of the 52 fraction bits, so the low 45 bits are rounded
+// away (add half an ulp minus one, plus the kept lsb for ties-to-even) and
+// the result, which has 8 significant bits, converts to float exactly.
+__device__ __forceinline__ bf16 f64_to_bf16_rne(double x) {
+  unsigned long long u = (unsigned long long)__double_as_longlong(x);
+  const unsigned long long lsb = (u >> 45) & 1ull;
+  u += 0x00000FFFFFFFFFFFull + lsb;
+  u &= ~0x00001FFFFFFFFFFFull;
+  const float f = (float)__longlong_as_double((long long)u);
+  return __float2bfloat16_rz(f);  // exact: f is a bfloat16 value
+}
+
+template <typename T> __device__ __forceinline__ T from_f64(double x);
+template <> __device__ __forceinline__ float from_f64<float>(double x) {
+  return __double2float_rn(x);
+}
+template <> __device__ __forceinline__ bf16 from_f64<bf16>(double x) {
+  return f64_to_bf16_rne(x);
+}
+
+// ---- warp reductions -------------------------------------------------------
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+// Load 64 consecutive path-dtype elements as fp32 into smem/regs helpers.
+template <typename T>
+__device__ __forceinline__ float ldf(const T* p) { return to_f32(*p); }
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+}  // namespace nsa

@@ -1,0 +1,42 @@
+// internal.h -- launch interface between the C ABI layer and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace nsa {
+
+// Validated, derived problem sizes (see nsa.h for the meaning of each).
+struct Dims {
+  int B, T, Tq, Hq, Hkv, D, G;
+  int l;       // block size (compression = selection = stride)
+  int Nc;      // complete compressed blocks: T / l
+  int Nb;      // selection blocks: ceil(T / l)
+  int topk;
+  int window;
+  float scale;
+  int dtype;   // 0 f32, 1 bf16
+  int branch_mask;
+  int q_off;   // position of query 0: T - Tq
+};
+
+// Each launcher enqueues on `s` and returns the launch status.  `err` is
+// the device error word (may be NULL).
+cudaError_t launch_compress(const Dims& d, const void* k, const void* v,
+                            void* kc, void* vc, cudaStream_t s);
+cudaError_t launch_cmp_scores(const Dims& d, const void* q, const void* kc,
+                              const void* vc, void* o_cmp, float* lse_cmp,
+                              float* score, cudaStream_t s);
+cudaError_t launch_topk(const Dims& d, const float* score, int32_t* idx,
+                        cudaStream_t s);
+cudaError_t launch_sel_fwd(const Dims& d, const void* q, const void* k,
+                           const void* v, const int32_t* idx, void* o,
+                           float* lse, int* err, cudaStream_t s);
+cudaError_t launch_swa_fwd(const Dims& d, const void* q, const void* k,
+                           const void* v, void* o, float* lse, cudaStream_t s);
+cudaError_t launch_combine(const Dims& d, const float* gates, const void* o_cmp,
+                           const void* o_sel, const void* o_swa, void* out,
+                           cudaStream_t s);
+
+}  // namespace nsa

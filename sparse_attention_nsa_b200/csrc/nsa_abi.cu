@@ -1,0 +1,363 @@
+// nsa_abi.cu -- the extern "C" entry points of libnsa (declared in nsa.h).
+//
+// This layer validates arguments, derives sizes, carves the caller's
+// workspace, and enqueues kernels on the caller's stream.  It allocates no
+// device memory and never synchronises except in nsa_last_device_error.
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+#include "nsa.h"
+
+namespace nsa {
+cudaError_t launch_sel_fwd_simt(const Dims& d, const void* q, const void* k,
+                                const void* v, const int32_t* idx, void* o,
+                                float* lse, int* err, cudaStream_t s);
+cudaError_t launch_swa_fwd_simt(const Dims& d, const void* q, const void* k,
+                                const void* v, void* o, float* lse, cudaStream_t s);
+
+cudaError_t launch_sel_fwd(const Dims& d, const void* q, const void* k, const void* v,
+                           const int32_t* idx, void* o, float* lse, int* err,
+                           cudaStream_t s) {
+  return launch_sel_fwd_simt(d, q, k, v, idx, o, lse, err, s);
+}
+cudaError_t launch_swa_fwd(const Dims& d, const void* q, const void* k, const void* v,
+                           void* o, float* lse, cudaStream_t s) {
+  return launch_swa_fwd_simt(d, q, k, v, o, lse, s);
+}
+}  // namespace nsa
+
+using nsa::Dims;
+
+// The device error word: kernels record the first failing check here.
+__device__ int g_nsa_error_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+int* g_err_ptr[kMaxDevices] = {};
+
+// Device address of the error word on the current device (looked up once
+// per device, with that device current).
+int* err_word() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_err_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_nsa_error_word) != cudaSuccess) return nullptr;
+    g_err_ptr[dev] = (int*)p;
+  }
+  return g_err_ptr[dev];
+}
+
+bool aligned16(const void* p) { return p && (((uintptr_t)p) & 15u) == 0; }
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+nsa_status fill_dims(const nsa_params* p, Dims* d) {
+  if (!p) return NSA_ERR_INVALID_ARG;
+  if (p->B < 1 || p->T < 1 || p->Tq < 1 || p->Tq > p->T || p->Hq < 1 || p->Hkv < 1 ||
+      p->D < 1 || p->cmp_block < 1 || p->cmp_stride < 1 || p->sel_block < 1 ||
+      p->topk < 2 || p->window < 1)
+    return NSA_ERR_INVALID_ARG;
+  if (p->Hq % p->Hkv != 0) return NSA_ERR_INVALID_ARG;
+  if (p->dtype != NSA_F32 && p->dtype != NSA_BF16) return NSA_ERR_INVALID_ARG;
+  if (p->branch_mask < 1 || p->branch_mask > NSA_BRANCH_ALL) return NSA_ERR_INVALID_ARG;
+  if (!(p->scale == p->scale) || p->scale == INFINITY || p->scale == -INFINITY)
+    return NSA_ERR_INVALID_ARG;
+  // valid NSA geometry, but outside what this build runs
+  if (p->D != 64) return NSA_ERR_UNSUPPORTED;
+  if (p->cmp_stride != p->cmp_block || p->sel_block != p->cmp_block)
+    return NSA_ERR_UNSUPPORTED;
+  const int G = p->Hq / p->Hkv;
+  if (G > 32 || (G & (G - 1)) != 0) return NSA_ERR_UNSUPPORTED;
+  if (p->Hkv > 64 || p->topk > 64) return NSA_ERR_UNSUPPORTED;
+  const int l = p->cmp_block;
+  const int Nb = (p->T + l - 1) / l;
+  if (Nb > 1024) return NSA_ERR_UNSUPPORTED;
+  d->B = p->B;
+  d->T = p->T;
+  d->Tq = p->Tq;
+  d->Hq = p->Hq;
+  d->Hkv = p->Hkv;
+  d->D = p->D;
+  d->G = G;
+  d->l = l;
+  d->Nc = p->T / l;
+  d->Nb = Nb;
+  d->topk = p->topk;
+  d->window = p->window;
+  d->scale = p->scale;
+  d->dtype = p->dtype;
+  d->branch_mask = p->branch_mask;
+  d->q_off = p->T - p->Tq;
+  return NSA_OK;
+}
+
+size_t esize(const Dims& d) { return d.dtype == NSA_BF16 ? 2 : 4; }
+
+// Workspace layout of nsa_forward / nsa_decode: every intermediate the
+// caller did not supply, each 256-byte aligned, in this order.
+struct Carve {
+  size_t off[10];
+  size_t total;
+};
+
+enum { W_KC, W_VC, W_OCMP, W_LSECMP, W_SCORE, W_IDX, W_OSEL, W_LSESEL, W_OSWA, W_LSESWA };
+
+void tensor_bytes(const Dims& d, size_t out[10]) {
+  const size_t es = esize(d);
+  const size_t kcb = (size_t)d.B * d.Nc * d.Hkv * 64 * es;
+  const size_t ob = (size_t)d.B * d.Tq * d.Hq * 64 * es;
+  const size_t lb = (size_t)d.B * d.Tq * d.Hq * 4;
+  out[W_KC] = kcb;
+  out[W_VC] = kcb;
+  out[W_OCMP] = ob;
+  out[W_LSECMP] = lb;
+  out[W_SCORE] = (size_t)d.B * d.Tq * d.Hkv * d.Nc * 4;
+  out[W_IDX] = (size_t)d.B * d.Tq * d.Hkv * d.topk * 4;
+  out[W_OSEL] = ob;
+  out[W_LSESEL] = lb;
+  out[W_OSWA] = ob;
+  out[W_LSESWA] = lb;
+}
+
+Carve carve(const Dims& d, const nsa_saved* sv) {
+  size_t bytes[10];
+  tensor_bytes(d, bytes);
+  const void* given[10] = {};
+  if (sv) {
+    given[W_KC] = sv->kc;
+    given[W_VC] = sv->vc;
+    given[W_OCMP] = sv->o_cmp;
+    given[W_LSECMP] = sv->lse_cmp;
+    given[W_SCORE] = sv->score;
+    given[W_IDX] = sv->idx;
+    given[W_OSEL] = sv->o_sel;
+    given[W_LSESEL] = sv->lse_sel;
+    given[W_OSWA] = sv->o_swa;
+    given[W_LSESWA] = sv->lse_swa;
+  }
+  Carve c{};
+  size_t at = 0;
+  for (int i = 0; i < 10; ++i) {
+    c.off[i] = at;
+    if (!given[i]) at += align256(bytes[i]);
+  }
+  c.total = at;
+  return c;
+}
+
+#define NSA_TRY_CUDA(expr)                           \
+  do {                                               \
+    if ((expr) != cudaSuccess) return NSA_ERR_CUDA;  \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+const char* nsa_status_string(nsa_status s) {
+  switch (s) {
+    case NSA_OK: return "NSA_OK";
+    case NSA_ERR_INVALID_ARG: return "NSA_ERR_INVALID_ARG";
+    case NSA_ERR_UNSUPPORTED: return "NSA_ERR_UNSUPPORTED";
+    case NSA_ERR_CUDA: return "NSA_ERR_CUDA";
+    case NSA_ERR_TIMEOUT: return "NSA_ERR_TIMEOUT";
+    case NSA_ERR_DEVICE_CHECK: return "NSA_ERR_DEVICE_CHECK";
+    case NSA_ERR_WORKSPACE: return "NSA_ERR_WORKSPACE";
+  }
+  return "NSA_ERR_UNKNOWN";
+}
+
+nsa_status nsa_check_params(const nsa_params* p) {
+  Dims d;
+  return fill_dims(p, &d);
+}
+
+nsa_status nsa_workspace_size(const nsa_params* p, size_t* bytes) {
+  Dims d;
+  nsa_status st = fill_dims(p, &d);
+  if (st != NSA_OK) return st;
+  if (!bytes) return NSA_ERR_INVALID_ARG;
+  *bytes = carve(d, nullptr).total;
+  return NSA_OK;
+}
+
+nsa_status nsa_last_device_error(void* stream) {
+  int* ew = err_word();
+  if (!ew) return NSA_ERR_CUDA;
+  NSA_TRY_CUDA(cudaStreamSynchronize((cudaStream_t)stream));
+  int v = 0;
+  NSA_TRY_CUDA(cudaMemcpy(&v, ew, sizeof(int), cudaMemcpyDeviceToHost));
+  if (v != 0) {
+    const int zero = 0;
+    NSA_TRY_CUDA(cudaMemcpy(ew, &zero, sizeof(int), cudaMemcpyHostToDevice));
+  }
+  if (v == nsa::kDevTimeout) return NSA_ERR_TIMEOUT;
+  if (v != 0) return NSA_ERR_DEVICE_CHECK;
+  return NSA_OK;
+}
+
+nsa_status nsa_compress(const nsa_params* p, const void* k, const void* v, void* kc,
+                        void* vc, void* stream) {
+  Dims d;
+  nsa_status st = fill_dims(p, &d);
+  if (st != NSA_OK) return st;
+  if (!aligned16(k) || !aligned16(v)) return NSA_ERR_INVALID_ARG;
+  if (d.Nc > 0 && (!aligned16(kc) || !aligned16(vc))) return NSA_ERR_INVALID_ARG;
+  NSA_TRY_CUDA(nsa::launch_compress(d, k, v, kc, vc, (cudaStream_t)stream));
+  return NSA_OK;
+}
+
+nsa_status nsa_cmp_attn_scores(const nsa_params* p, const void* q, const void* kc,
+                               const void* vc, void* o_cmp, float* lse_cmp,
+                               float* score, void* stream) {
+  Dims d;
+  nsa_status st = fill_dims(p, &d);
+  if (st != NSA_OK) return st;
+  if (!aligned16(q) || (d.Nc > 0 && (!aligned16(kc) || !aligned16(vc))))
+    return NSA_ERR_INVALID_ARG;
+  if (d.Nc > 0 && !aligned16(score)) return NSA_ERR_INVALID_ARG;
+  if (o_cmp && !aligned16(o_cmp)) return NSA_ERR_INVALID_ARG;
+  NSA_TRY_CUDA(nsa::launch_cmp_scores(d, q, kc, vc, o_cmp, lse_cmp, score,
+                                      (cudaStream_t)stream));
+  return NSA_OK;
+}
+
+nsa_status nsa_select_topk(const nsa_params* p, const float* score, int32_t* idx,
+                           void* stream) {
+  Dims d;
+  nsa_status st = fill_dims(p, &d);
+  if (st != NSA_OK) return st;
+  if ((d.Nc > 0 && !aligned16(score)) || !aligned16(idx)) return NSA_ERR_INVALID_ARG;
+  NSA_TRY_CUDA(nsa::launch_topk(d, score, idx, (cudaStream_t)stream));
+  return NSA_OK;
+}
+
+nsa_status nsa_sel_attn_fwd(const nsa_params* p, const void* q, const void* k,
+                            const void* v, const int32_t* idx, void* o_sel,
+                            float* lse_sel, void* stream) {
+  Dims d;
+  nsa_status st = fill_dims(p, &d);
+  if (st != NSA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(idx) ||
+      !aligned16(o_sel))
+    return NSA_ERR_INVALID_ARG;
+  NSA_TRY_CUDA(nsa::launch_sel_fwd(d, q, k, v, idx, o_sel, lse_sel, err_word(),
+                                   (cudaStream_t)stream));
+  return NSA_OK;
+}
+
+nsa_status nsa_swa_fwd(const nsa_params* p, const void* q, const void* k, const void* v,
+                       void* o_swa, float* lse_swa, void* stream) {
+  Dims d;
+  nsa_status st = fill_dims(p, &d);
+  if (st != NSA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o_swa))
+    return NSA_ERR_INVALID_ARG;
+  NSA_TRY_CUDA(nsa::launch_swa_fwd(d, q, k, v, o_swa, lse_swa, (cudaStream_t)stream));
+  return NSA_OK;
+}
+
+nsa_status nsa_gate_combine(const nsa_params* p, const float* gates, const void* o_cmp,
+                            const void* o_sel, const void* o_swa, void* out,
+                            void* stream) {
+  Dims d;
+  nsa_status st = fill_dims(p, &d);
+  if (st != NSA_OK) return st;
+  if (!aligned16(gates) || !aligned16(out)) return NSA_ERR_INVALID_ARG;
+  if ((d.branch_mask & NSA_BRANCH_CMP) && !aligned16(o_cmp)) return NSA_ERR_INVALID_ARG;
+  if ((d.branch_mask & NSA_BRANCH_SEL) && !aligned16(o_sel)) return NSA_ERR_INVALID_ARG;
+  if ((d.branch_mask & NSA_BRANCH_SWA) && !aligned16(o_swa)) return NSA_ERR_INVALID_ARG;
+  NSA_TRY_CUDA(nsa::launch_combine(d, gates, o_cmp, o_sel, o_swa, out,
+                                   (cudaStream_t)stream));
+  return NSA_OK;
+}
+
+// Shared body of nsa_forward and nsa_decode.  kc_given means the compressed
+// tensors in sv->kc / sv->vc are inputs (decode) and compression is skipped.
+static nsa_status run_forward(const Dims& d, const void* q, const void* k, const void* v,
+                              bool kc_given, const float* gates, void* out,
+                              const nsa_saved* sv, void* ws, size_t ws_bytes,
+                              cudaStream_t s) {
+  const Carve c = carve(d, sv);
+  if (c.total > 0 && (!ws || ws_bytes < c.total || (((uintptr_t)ws) & 255u) != 0))
+    return NSA_ERR_WORKSPACE;
+  char* w = (char*)ws;
+  auto pick = [&](void* given, int slot) -> void* {
+    return given ? given : (void*)(w + c.off[slot]);
+  };
+  const nsa_saved z{};
+  const nsa_saved& S = sv ? *sv : z;
+  void* kc = kc_given ? S.kc : pick(S.kc, W_KC);
+  void* vc = kc_given ? S.vc : pick(S.vc, W_VC);
+  void* o_cmp = pick(S.o_cmp, W_OCMP);
+  float* lse_cmp = (float*)pick(S.lse_cmp, W_LSECMP);
+  float* score = (float*)pick(S.score, W_SCORE);
+  int32_t* idx = (int32_t*)pick(S.idx, W_IDX);
+  void* o_sel = pick(S.o_sel, W_OSEL);
+  float* lse_sel = (float*)pick(S.lse_sel, W_LSESEL);
+  void* o_swa = pick(S.o_swa, W_OSWA);
+  float* lse_swa = (float*)pick(S.lse_swa, W_LSESWA);
+  const bool cmp = d.branch_mask & NSA_BRANCH_CMP;
+  const bool sel = d.branch_mask & NSA_BRANCH_SEL;
+  const bool swa = d.branch_mask & NSA_BRANCH_SWA;
+  if (cmp || sel) {
+    if (!kc_given) NSA_TRY_CUDA(nsa::launch_compress(d, k, v, kc, vc, s));
+    NSA_TRY_CUDA(nsa::launch_cmp_scores(d, q, kc, vc, cmp ? o_cmp : nullptr,
+                                        cmp ? lse_cmp : nullptr, score, s));
+  }
+  if (sel) {
+    NSA_TRY_CUDA(nsa::launch_topk(d, score, idx, s));
+    NSA_TRY_CUDA(nsa::launch_sel_fwd(d, q, k, v, idx, o_sel, lse_sel, err_word(), s));
+  }
+  if (swa) NSA_TRY_CUDA(nsa::launch_swa_fwd(d, q, k, v, o_swa, lse_swa, s));
+  NSA_TRY_CUDA(nsa::launch_combine(d, gates, o_cmp, o_sel, o_swa, out, s));
+  return NSA_OK;
+}
+
+nsa_status nsa_forward(const nsa_params* p, const void* q, const void* k, const void* v,
+                       const float* gates, void* out, const nsa_saved* saved,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+  Dims d;
+  nsa_status st = fill_dims(p, &d);
+  if (st != NSA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(gates) ||
+      !aligned16(out))
+    return NSA_ERR_INVALID_ARG;
+  if (saved) {
+    const void* ptrs[10] = {saved->kc, saved->vc, saved->o_cmp, saved->lse_cmp,
+                            saved->score, saved->idx, saved->o_sel, saved->lse_sel,
+                            saved->o_swa, saved->lse_swa};
+    for (const void* ptr : ptrs)
+      if (ptr && (((uintptr_t)ptr) & 15u)) return NSA_ERR_INVALID_ARG;
+  }
+  return run_forward(d, q, k, v, false, gates, out, saved, workspace, workspace_bytes,
+                     (cudaStream_t)stream);
+}
+
+nsa_status nsa_decode(const nsa_params* p, const void* q, const void* k_cache,
+                      const void* v_cache, const void* kc_cache, const void* vc_cache,
+                      const float* gates, void* out, int32_t* idx_out, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  Dims d;
+  nsa_status st = fill_dims(p, &d);
+  if (st != NSA_OK) return st;
+  if (d.Tq != 1) return NSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(gates) ||
+      !aligned16(out))
+    return NSA_ERR_INVALID_ARG;
+  if (d.Nc > 0 && (!aligned16(kc_cache) || !aligned16(vc_cache))) return NSA_ERR_INVALID_ARG;
+  if (idx_out && (((uintptr_t)idx_out) & 15u)) return NSA_ERR_INVALID_ARG;
+  nsa_saved sv{};
+  sv.idx = idx_out;
+  sv.kc = (void*)kc_cache;  // inputs here; NULL only when Nc == 0 (never read)
+  sv.vc = (void*)vc_cache;
+  return run_forward(d, q, k_cache, v_cache, true, gates, out, &sv, workspace,
+                     workspace_bytes, (cudaStream_t)stream);
+}
+
+}  // extern "C"

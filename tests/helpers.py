@@ -1,0 +1,82 @@
+"""Shared helpers for the GPU parity tests: oracle configs, comparisons.
+
+Tolerances (from the method's stated targets, applied on the same
+bf16-rounded inputs):
+  fp32 path  : 1e-4 max-abs on every floating-point output
+  bf16 path  : 2e-2 max-abs on every floating-point output
+  block idx  : bit-exact, except rows where the oracle's k-th and (k+1)-th
+               candidate scores differ by less than 1e-5 (relative); such a
+               row must still hold a valid selection.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle as orc
+from sparse_attention_nsa_b200 import inputs as W
+
+TOL = {torch.float32: 1e-4, torch.bfloat16: 2e-2}
+LSE_TOL = {torch.float32: 1e-4, torch.bfloat16: 2e-3}
+NEAR_TIE = 1e-5
+
+
+def ocfg(w: W.Workload, **kw) -> orc.Cfg:
+    """Oracle config for a workload; compressed keys/values are stored in the
+    path's dtype, exactly as the library stores them."""
+    c = orc.Cfg(B=w.B, T=w.T, Hq=w.Hq, Hkv=w.Hkv, D=w.D, cmp_block=w.cmp_block,
+                cmp_stride=w.cmp_stride, sel_block=w.sel_block, topk=w.topk,
+                window=w.window, scale=w.scale,
+                kv_round=orc.KV_BF16 if w.dtype == torch.bfloat16 else orc.KV_F32,
+                branch_mask=w.branch_mask)
+    for k, v in kw.items():
+        setattr(c, k, v)
+    return c
+
+
+def to_np(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().double().numpy() if t.dtype != torch.int32 \
+        else t.detach().cpu().numpy()
+
+
+def max_abs(a, b) -> float:
+    a, b = np.asarray(a, dtype=np.float64), np.asarray(b, dtype=np.float64)
+    both_inf = np.isinf(a) & np.isinf(b) & (np.sign(a) == np.sign(b))
+    d = np.where(both_inf, 0.0, np.abs(a - b))
+    return float(np.nanmax(d)) if d.size else 0.0
+
+
+def assert_close(got, want, tol, what=""):
+    err = max_abs(got, want)
+    assert np.all(np.isfinite(got) == np.isfinite(want)), f"{what}: finiteness differs"
+    assert err <= tol, f"{what}: max-abs error {err:.3e} > {tol:.1e}"
+    return err
+
+
+def candidate_ranking(score_row: np.ndarray, cur: int) -> list[int]:
+    return sorted(range(1, cur), key=lambda j: (-score_row[j], j))
+
+
+def idx_mismatch_rows(gpu_idx, orc_idx, orc_score, t_of_row, topk, l):
+    """Compare selections row by row.  Returns the boolean mask of rows that
+    differ; asserts that every differing row is a near-tie of the oracle's
+    scores and that the GPU's selection is a valid one for that row."""
+    g = gpu_idx.reshape(-1, topk)
+    o = orc_idx.reshape(-1, topk)
+    s = orc_score.reshape(g.shape[0], -1)
+    t = np.asarray(t_of_row).reshape(-1)
+    diff = np.any(g != o, axis=1)
+    for r in np.nonzero(diff)[0]:
+        cur = int(t[r]) // l
+        assert cur + 1 > topk, f"row {r}: all-causal selection differs"
+        gs = set(int(x) for x in g[r] if x >= 0)
+        assert len(gs) == topk and 0 in gs and cur in gs, f"row {r}: invalid selection {g[r]}"
+        assert list(g[r]) == sorted(g[r]), f"row {r}: not ascending"
+        rank = candidate_ranking(s[r], cur)
+        kth, nxt = s[r][rank[topk - 3]], s[r][rank[topk - 2]]
+        assert abs(kth - nxt) <= NEAR_TIE * max(abs(kth), 1e-30), \
+            f"row {r}: selections differ without a near-tie ({kth} vs {nxt})"
+        # every GPU pick must score within the near-tie band of the k-th score
+        for j in gs - {0, cur}:
+            assert s[r][j] >= kth - NEAR_TIE * abs(kth) * 2, f"row {r}: block {j} not a top pick"
+    return diff

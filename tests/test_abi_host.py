@@ -1,0 +1,90 @@
+"""Host-side checks of the C-ABI library (CPU only, no kernel launches).
+
+The library must load, export every symbol include/nsa.h declares, and
+reject bad parameter blocks before launching anything.
+"""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+import sparse_attention_nsa_b200 as nsa
+from sparse_attention_nsa_b200 import abi
+from sparse_attention_nsa_b200 import inputs as W
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(nsa_[a-z0-9_]+)\s*\(", text))
+    return names
+
+
+def test_header_and_binding_agree():
+    assert declared_symbols() == set(abi.EXPORTS)
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    lib = nsa.load()
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    assert isinstance(C.CDLL(abi.LIB_PATH).nsa_forward, C._CFuncPtr)
+
+
+def test_status_strings():
+    for code, name in abi.STATUS.items():
+        assert nsa.nsa_status_string(code) == name
+
+
+@pytest.mark.parametrize("w", list(W.WORKLOADS.values()), ids=lambda w: w.name)
+def test_workload_params_are_accepted(w):
+    p = nsa.params_for(w, Tq=1 if "decode" in w.name else None)
+    assert nsa.nsa_check_params(p) == 0
+    assert nsa.nsa_workspace_size(p) > 0
+
+
+BAD = [
+    (dict(B=0), 1), (dict(T=0), 1), (dict(Tq=5000), 1), (dict(Hkv=3), 1),
+    (dict(topk=1), 1), (dict(window=0), 1), (dict(dtype=7), 1), (dict(branch_mask=0), 1),
+    (dict(branch_mask=9), 1), (dict(scale=float("nan")), 1),
+    (dict(D=128), 2), (dict(cmp_stride=32), 2), (dict(sel_block=32), 2),
+    (dict(Hq=24, Hkv=4), 2), (dict(topk=65), 2), (dict(T=200000), 2),
+]
+
+
+@pytest.mark.parametrize("change,code", BAD)
+def test_bad_params_rejected(change, code):
+    base = dict(B=1, T=4096, Hq=16, Hkv=4)
+    kw = {k: change.pop(k) for k in list(change) if k in base}
+    base.update(kw)
+    p = nsa.make_params(**base)
+    for k, v in change.items():
+        setattr(p, k, v)
+    assert nsa.nsa_check_params(p) == code
+    n = C.c_size_t(0)
+    assert nsa.load().nsa_workspace_size(C.byref(p), C.byref(n)) == code
+
+
+def test_null_pointers_rejected_before_launch():
+    lib = nsa.load()
+    p = nsa.make_params(1, 256, 4, 1, cmp_block=32, topk=4, window=64, dtype=nsa.NSA_F32)
+    assert lib.nsa_compress(C.byref(p), None, None, None, None, None) == 1
+    assert lib.nsa_swa_fwd(C.byref(p), None, None, None, None, None, None) == 1
+    assert lib.nsa_forward(C.byref(p), None, None, None, None, None, None, None, 0, None) == 1
+    assert lib.nsa_sel_attn_fwd(C.byref(p), C.c_void_p(16), C.c_void_p(32), C.c_void_p(48),
+                                C.c_void_p(64), C.c_void_p(8), None, None) == 1  # misaligned o
+    p.Tq = 2
+    assert lib.nsa_decode(C.byref(p), *([C.c_void_p(256)] * 7), None, None, 0, None) == 1
+
+
+def test_forward_without_workspace_is_rejected():
+    lib = nsa.load()
+    p = nsa.make_params(1, 256, 4, 1, cmp_block=32, topk=4, window=64, dtype=nsa.NSA_F32)
+    ptr = C.c_void_p(4096)
+    assert lib.nsa_forward(C.byref(p), ptr, ptr, ptr, ptr, ptr, None, None, 0, None) == 6
