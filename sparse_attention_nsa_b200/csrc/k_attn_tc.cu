@@ -1,0 +1,451 @@
+// k_attn_tc.cu -- selection and sliding-window attention on the sm_100a
+// tensor cores (tcgen05 + TMEM, TMA-staged K/V blocks), bf16 in, fp32
+// softmax and accumulation.
+//
+// "DeepSeek's Native Sparse Attention", How Does Native Sparse Attention
+// Work?: SELECTION attends to the top-scoring blocks in raw form, SLIDING
+// WINDOW to the most recent tokens; the kernel paragraph groups the queries
+// that share a sparse selection so reads stay contiguous.  Here the queries
+// of one KV group are the unit: a CTA owns 128 query rows = 128/G
+// consecutive tokens x the G heads of one KV group (head-stacking gives the
+// MMA its M = 128), and walks a list of 64-key blocks:
+//   selection: the ascending union of the blocks its tokens selected; a row
+//              whose token did not select a block gets P = 0 for it;
+//   window   : the contiguous blocks that intersect any row's window.
+// The K and V tile of a block is loaded once per CTA by TMA and serves all
+// 128 rows.
+//
+// Per block:  S = Q K^T   (tcgen05, M=128 N=64 K=64, into TMEM)
+//             softmax rows in fp32 (one thread per row, online max/sum)
+//             P (bf16, swizzled smem) ;  O_blk = P V  (tcgen05, into TMEM)
+//             o += o * alpha + O_blk in registers.
+// Warp roles (192 threads): warps 0-3 softmax/epilogue, warp 4 MMA issue and
+// TMEM owner, warp 5 TMA producer.  S and O_blk are double-buffered in TMEM
+// (256 columns), P in smem, K/V in a 3-stage ring, so the MMAs of block i+1
+// and the P*V of block i overlap the softmax of block i.  Two CTAs fit per
+// SM, and their softmax and MMA phases interleave.
+#include <cudaTypedefs.h>
+
+#include <climits>
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace nsa {
+
+cudaError_t launch_sel_fwd_simt(const Dims& d, const void* q, const void* k,
+                                const void* v, const int32_t* idx, void* o,
+                                float* lse, int* err, cudaStream_t s);
+cudaError_t launch_swa_fwd_simt(const Dims& d, const void* q, const void* k,
+                                const void* v, void* o, float* lse, cudaStream_t s);
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kRows = 128;   // query rows per CTA (M)
+constexpr int kKeys = 64;    // keys per block (N of S, K of P*V)
+constexpr int kStages = 3;   // K/V ring depth
+constexpr int kThreads = 192;
+constexpr uint32_t kTileBytes = kKeys * 64 * 2;  // one K or V block, bf16
+constexpr uint32_t kQBytes = kRows * 64 * 2;
+constexpr uint32_t kPBytes = kRows * kKeys * 2;
+
+constexpr uint32_t OFF_Q = 0;
+constexpr uint32_t OFF_KV = OFF_Q + kQBytes;                      // stage s: K, then V
+constexpr uint32_t OFF_P = OFF_KV + kStages * 2 * kTileBytes;    // two P buffers
+constexpr uint32_t OFF_BAR = OFF_P + 2 * kPBytes;
+
+struct Bars {
+  uint64_t q;
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t s[2];
+  uint64_t p[2];
+  uint64_t o[2];
+  uint64_t fin;
+};
+constexpr uint32_t OFF_MISC = OFF_BAR + ((sizeof(Bars) + 15) / 16) * 16;  // tmem, abort, nblk
+constexpr uint32_t OFF_LIST = OFF_MISC + 16;
+
+__host__ __device__ inline int tokens_per_tile(int G) { return kRows / G; }
+
+__host__ __device__ inline size_t list_ints(const Dims& d) {
+  const int words = (d.Nb + 31) / 32;
+  return (size_t)d.Nb + words + (size_t)tokens_per_tile(d.G) * (d.topk + 1);
+}
+
+template <bool SEL>
+__global__ void __launch_bounds__(kThreads, 2)
+attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, bf16* __restrict__ o,
+               float* __restrict__ lse, const int32_t* __restrict__ idx, Dims d, int* err) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  Bars* bars = (Bars*)(smem + OFF_BAR);
+  uint32_t* tmem_slot = (uint32_t*)(smem + OFF_MISC);
+  volatile int* abort_flag = (volatile int*)(smem + OFF_MISC + 4);
+  int* nblk_s = (int*)(smem + OFF_MISC + 8);
+  int* blk = (int*)(smem + OFF_LIST);
+  const int words = (d.Nb + 31) / 32;
+  uint32_t* bits = (uint32_t*)(blk + d.Nb);
+  int* toks = (int*)(bits + words);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
+  const int TQ = tokens_per_tile(d.G);
+  const int tile = gridDim.x - 1 - blockIdx.x;  // heavy (late) tiles first
+  const int t0 = tile * TQ;
+  const int g = blockIdx.y, b = blockIdx.z;
+  const int nvalid = min(TQ, d.Tq - t0);
+  const int pos0 = d.q_off + t0;  // key position of the tile's first query
+
+  if (tid == 0) {
+    mbar_init(&bars->q, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bars->full[s], 1);
+      mbar_init(&bars->empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars->s[i], 1);
+      mbar_init(&bars->p[i], 128);
+      mbar_init(&bars->o[i], 1);
+    }
+    mbar_init(&bars->fin, 1);
+    fence_barrier_init();
+    fence_proxy_async_smem();
+    *abort_flag = 0;
+  }
+  if (warp == 4) tmem_alloc(tmem_slot, 256);
+  if (warp == 5 && lane == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+  }
+
+  // ---- block list ------------------------------------------------------------
+  if (SEL) {
+    for (int w = tid; w < words; w += kThreads) bits[w] = 0u;
+    __syncthreads();
+    // one thread per token: validate and copy its selection, mark the union
+    for (int tl = tid; tl < TQ; tl += kThreads) {
+      int* lst = toks + tl * (d.topk + 1);
+      int cnt = 0;
+      if (tl < nvalid) {
+        const int t = pos0 + tl;
+        const int cur = t / d.l;
+        const int32_t* ir = idx + (((size_t)b * d.Tq + t0 + tl) * d.Hkv + g) * d.topk;
+        int prev = -1;
+        for (int s = 0; s < d.topk; ++s) {
+          const int j = ir[s];
+          if (j == -1) continue;
+          if (j < -1 || j <= prev || j > cur) {  // never read a non-causal block
+            record_error(err, kDevBadIndex);
+            continue;
+          }
+          prev = j;
+          lst[cnt++] = j;
+          atomicOr(&bits[j >> 5], 1u << (j & 31));
+        }
+      }
+      lst[cnt] = INT_MAX;
+    }
+    __syncthreads();
+    if (warp == 0) {  // compact the bitmap into an ascending list
+      int base = 0;
+      for (int w0 = 0; w0 < words; w0 += 32) {
+        const int w = w0 + lane;
+        uint32_t m = w < words ? bits[w] : 0u;
+        const int c = __popc(m);
+        int incl = c;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, off);
+          if (lane >= off) incl += y;
+        }
+        int pos = base + incl - c;
+        while (m) {
+          const int bit = __ffs(m) - 1;
+          m &= m - 1;
+          blk[pos++] = w * 32 + bit;
+        }
+        base += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      if (lane == 0) *nblk_s = base;
+    }
+  } else if (tid == 0) {
+    const int tlast = pos0 + nvalid - 1;
+    const int jlo = max(0, pos0 - d.window + 1) / d.l;
+    const int jhi = tlast / d.l;
+    blk[0] = jlo;
+    *nblk_s = jhi - jlo + 1;
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int n = *nblk_s;
+  const int blk0 = blk[0];
+
+  if (warp == 5) {
+    // ---- TMA producer -----------------------------------------------------------
+    if (lane == 0) {
+      mbar_expect_tx(&bars->q, kQBytes);
+      tma_load_3d(smem + OFF_Q, &tm_q, &bars->q, 0, g * d.G, b * d.Tq + t0);
+      int issued = 0;
+      for (int i = 0; i < n; ++i) {
+        const int st = i % kStages;
+        if (i >= kStages &&
+            !wait_bar(&bars->empty[st], ((i / kStages) & 1) ^ 1, abort_flag, err))
+          break;
+        const int j = SEL ? blk[i] : blk0 + i;
+        const int row = b * d.T + j * kKeys;
+        uint8_t* kv = smem + OFF_KV + st * 2 * kTileBytes;
+        mbar_expect_tx(&bars->full[st], 2 * kTileBytes);
+        tma_load_3d(kv, &tm_k, &bars->full[st], 0, g, row);
+        tma_load_3d(kv + kTileBytes, &tm_v, &bars->full[st], 0, g, row);
+        issued = i + 1;
+      }
+      if (*abort_flag) {  // let the copies already issued land before exit
+        drain_bar(&bars->q, 0);
+        for (int i = max(0, issued - kStages); i < issued; ++i)
+          drain_bar(&bars->full[i % kStages], (i / kStages) & 1);
+      }
+    }
+  } else if (warp == 4) {
+    // ---- MMA issue ------------------------------------------------------------------
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16(kRows, kKeys, false, false);
+      constexpr uint32_t idesc_o = idesc_bf16(kRows, 64, false, true);
+      const uint32_t q_addr = smem_u32(smem + OFF_Q);
+      bool ok = wait_bar(&bars->q, 0, abort_flag, err);
+      auto issue_s = [&](int i) -> bool {
+        const int st = i % kStages;
+        if (!wait_bar(&bars->full[st], (i / kStages) & 1, abort_flag, err)) return false;
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(smem + OFF_KV + st * 2 * kTileBytes);
+        const uint32_t d_tmem = tmem + (uint32_t)(i & 1) * 64u;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(d_tmem, desc_sw128(q_addr + kk * 32, 16), desc_sw128(k_addr + kk * 32, 16),
+                   idesc_s, kk > 0);
+        mma_commit(&bars->s[i & 1]);
+        return true;
+      };
+      if (ok && n > 0) ok = issue_s(0);
+      for (int i = 0; ok && i < n; ++i) {
+        if (i + 1 < n && !issue_s(i + 1)) break;
+        if (!wait_bar(&bars->p[i & 1], (i >> 1) & 1, abort_flag, err)) break;
+        tc_fence_after();
+        const int st = i % kStages;
+        const uint32_t v_addr = smem_u32(smem + OFF_KV + st * 2 * kTileBytes + kTileBytes);
+        const uint32_t p_addr = smem_u32(smem + OFF_P + (i & 1) * kPBytes);
+        const uint32_t d_tmem = tmem + 128u + (uint32_t)(i & 1) * 64u;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(d_tmem, desc_sw128(p_addr + kk * 32, 16),
+                   desc_sw128(v_addr + kk * 2048, 8192), idesc_o, kk > 0);
+        mma_commit(&bars->o[i & 1]);
+        mma_commit(&bars->empty[st]);
+      }
+      // every MMA issued must finish before TMEM is released
+      mma_commit(&bars->fin);
+      drain_bar(&bars->fin, 0);
+    }
+  } else {
+    // ---- softmax and epilogue: thread r owns query row r -------------------------
+    const int r = tid;
+    const int tl = r / d.G, hh = r % d.G;
+    const bool valid = tl < nvalid;
+    const int t = pos0 + tl;
+    const int lo = SEL ? 0 : max(0, t - d.window + 1);  // first key of the row
+    const int* lst = SEL ? toks + tl * (d.topk + 1) : nullptr;
+    int ptr = 0;
+    float m = -INFINITY, lsum = 0.f, alpha_prev = 1.f;
+    float acc[64];
+#pragma unroll
+    for (int c = 0; c < 64; ++c) acc[c] = 0.f;
+    const float sl2 = d.scale * kLog2e;
+    const uint32_t lane_tmem = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t prow = smem_u32(smem + OFF_P) + (uint32_t)(r >> 3) * 1024u + (uint32_t)(r & 7) * 128u;
+    bool ok = true;
+    for (int i = 0; i < n; ++i) {
+      const int j = SEL ? blk[i] : blk0 + i;
+      const int k0 = j * kKeys;
+      bool rowsel = valid && k0 <= t;
+      if (SEL) {
+        if (valid) {
+          while (lst[ptr] < j) ++ptr;
+          const bool hit = lst[ptr] == j;
+          if (hit) ++ptr;
+          rowsel = rowsel && hit;
+        }
+      } else {
+        rowsel = rowsel && (k0 + kKeys - 1 >= lo);
+      }
+      if (!wait_bar_warp(&bars->s[i & 1], (i >> 1) & 1, abort_flag, err)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float sv[64];
+      tmem_ld32(lane_tmem + (uint32_t)(i & 1) * 64u, sv);
+      tmem_ld32(lane_tmem + (uint32_t)(i & 1) * 64u + 32u, sv + 32);
+      tmem_wait_ld();
+      float alpha = 1.f;
+      uint32_t pk[32];
+      if (rowsel) {
+        const bool full = (k0 + kKeys - 1 <= t) && (k0 >= lo);
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          float x = sv[c] * sl2;
+          if (!full && (k0 + c > t || k0 + c < lo)) x = -INFINITY;
+          sv[c] = x;
+          mx = fmaxf(mx, x);
+        }
+        const float mn = fmaxf(m, mx);
+        alpha = exp2f(m - mn);
+        float rs = 0.f;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const float p = exp2f(sv[c] - mn);
+          sv[c] = p;
+          rs += p;
+        }
+        lsum = lsum * alpha + rs;
+        m = mn;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(sv[2 * c], sv[2 * c + 1]);
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) pk[c] = 0u;
+      }
+      const uint32_t pb = prow + (uint32_t)(i & 1) * kPBytes;
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        st_shared_v4(pb + ((uint32_t)(c ^ (r & 7)) << 4), pk[4 * c], pk[4 * c + 1],
+                     pk[4 * c + 2], pk[4 * c + 3]);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bars->p[i & 1]);
+      if (i > 0) {
+        if (!wait_bar_warp(&bars->o[(i - 1) & 1], ((i - 1) >> 1) & 1, abort_flag, err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        float ov[64];
+        tmem_ld32(lane_tmem + 128u + (uint32_t)((i - 1) & 1) * 64u, ov);
+        tmem_ld32(lane_tmem + 128u + (uint32_t)((i - 1) & 1) * 64u + 32u, ov + 32);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 64; ++c) acc[c] = fmaf(acc[c], alpha_prev, ov[c]);
+      }
+      alpha_prev = alpha;
+    }
+    if (ok && n > 0) {
+      if (wait_bar_warp(&bars->o[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag, err)) {
+        tc_fence_after();
+        float ov[64];
+        tmem_ld32(lane_tmem + 128u + (uint32_t)((n - 1) & 1) * 64u, ov);
+        tmem_ld32(lane_tmem + 128u + (uint32_t)((n - 1) & 1) * 64u + 32u, ov + 32);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 64; ++c) acc[c] = fmaf(acc[c], alpha_prev, ov[c]);
+      }
+    }
+    tc_fence_before();
+    if (valid) {
+      const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+      const int h = g * d.G + hh;
+      const size_t row = ((size_t)b * d.Tq + t0 + tl) * d.Hq + h;
+      uint4* dst = reinterpret_cast<uint4*>(o + row * 64);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint4 u;
+        u.x = pack_bf16(acc[8 * c + 0] * inv, acc[8 * c + 1] * inv);
+        u.y = pack_bf16(acc[8 * c + 2] * inv, acc[8 * c + 3] * inv);
+        u.z = pack_bf16(acc[8 * c + 4] * inv, acc[8 * c + 5] * inv);
+        u.w = pack_bf16(acc[8 * c + 6] * inv, acc[8 * c + 7] * inv);
+        dst[c] = u;
+      }
+      if (lse) lse[row] = lsum > 0.f ? (m + log2f(lsum)) * kLn2 : -INFINITY;
+    }
+  }
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+// ---- host side ------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (PFN_cuTensorMapEncodeTiled_v12000)p;
+  });
+  return fn;
+}
+
+// 3-D bf16 view (64 head dims, heads, rows) with a (64, box_h, box_rows) box,
+// 128-byte swizzle, zero fill outside the tensor.
+bool make_map(CUtensorMap* map, const void* base, int heads, long rows, int box_h,
+              int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {64, (cuuint64_t)heads, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {128, (cuuint64_t)heads * 128};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_h, (cuuint32_t)box_rows};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+            box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool tc_eligible(const Dims& d) {
+  return d.dtype == 1 && d.l == kKeys && d.D == 64 && d.G >= 1 && kRows % d.G == 0 &&
+         d.Nb <= 4096 && encode_fn() != nullptr;
+}
+
+template <bool SEL>
+cudaError_t launch_tc(const Dims& d, const void* q, const void* k, const void* v,
+                      const int32_t* idx, void* o, float* lse, int* err, cudaStream_t s) {
+  const int TQ = tokens_per_tile(d.G);
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, d.Hq, (long)d.B * d.Tq, d.G, TQ) ||
+      !make_map(&mk, k, d.Hkv, (long)d.B * d.T, 1, kKeys) ||
+      !make_map(&mv, v, d.Hkv, (long)d.B * d.T, 1, kKeys))
+    return cudaErrorInvalidValue;
+  const size_t smem = OFF_LIST + list_ints(d) * sizeof(int) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<SEL>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((d.Tq + TQ - 1) / TQ, d.Hkv, d.B);
+  attn_tc_kernel<SEL><<<grid, kThreads, smem, s>>>(mq, mk, mv, (bf16*)o, lse, idx, d, err);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_sel_fwd(const Dims& d, const void* q, const void* k, const void* v,
+                           const int32_t* idx, void* o, float* lse, int* err,
+                           cudaStream_t s) {
+  if (tc_eligible(d)) return launch_tc<true>(d, q, k, v, idx, o, lse, err, s);
+  return launch_sel_fwd_simt(d, q, k, v, idx, o, lse, err, s);
+}
+
+cudaError_t launch_swa_fwd(const Dims& d, const void* q, const void* k, const void* v,
+                           void* o, float* lse, cudaStream_t s) {
+  if (tc_eligible(d)) return launch_tc<false>(d, q, k, v, nullptr, o, lse, nullptr, s);
+  return launch_swa_fwd_simt(d, q, k, v, o, lse, s);
+}
+
+}  // namespace nsa

@@ -9,24 +9,6 @@
 #include "internal.h"
 #include "nsa.h"
 
-namespace nsa {
-cudaError_t launch_sel_fwd_simt(const Dims& d, const void* q, const void* k,
-                                const void* v, const int32_t* idx, void* o,
-                                float* lse, int* err, cudaStream_t s);
-cudaError_t launch_swa_fwd_simt(const Dims& d, const void* q, const void* k,
-                                const void* v, void* o, float* lse, cudaStream_t s);
-
-cudaError_t launch_sel_fwd(const Dims& d, const void* q, const void* k, const void* v,
-                           const int32_t* idx, void* o, float* lse, int* err,
-                           cudaStream_t s) {
-  return launch_sel_fwd_simt(d, q, k, v, idx, o, lse, err, s);
-}
-cudaError_t launch_swa_fwd(const Dims& d, const void* q, const void* k, const void* v,
-                           void* o, float* lse, cudaStream_t s) {
-  return launch_swa_fwd_simt(d, q, k, v, o, lse, s);
-}
-}  // namespace nsa
-
 using nsa::Dims;
 
 // The device error word: kernels record the first failing check here.
