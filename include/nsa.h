@@ -62,7 +62,9 @@ typedef enum {
   NSA_ERR_CUDA = 3,         /* a CUDA call or launch failed                */
   NSA_ERR_TIMEOUT = 4,      /* a bounded device-side wait expired          */
   NSA_ERR_DEVICE_CHECK = 5, /* a device-side consistency check failed      */
-  NSA_ERR_WORKSPACE = 6     /* workspace missing or smaller than required  */
+  NSA_ERR_WORKSPACE = 6,    /* workspace missing or smaller than required  */
+  NSA_ERR_SCRATCH_TOO_SMALL = 7 /* problem needs more than the fixed scratch
+                                   of nsa_decode_noalloc                    */
 } nsa_status;
 
 typedef enum { NSA_F32 = 0, NSA_BF16 = 1 } nsa_dtype;
@@ -210,6 +212,33 @@ nsa_status nsa_decode(const nsa_params* p, const void* q, const void* k_cache,
                       const void* vc_cache, const float* gates, void* out,
                       int32_t* idx_out, void* workspace, size_t workspace_bytes,
                       void* stream);
+
+/* ---- decode without any allocation by the caller ---------------------------
+ * No counterpart in the paper: this is a deployment variant of nsa_decode.
+ * Some callers cannot allocate device memory -- for example a plugin that
+ * its host framework hands only input and output buffers, or a runtime that
+ * serves from a fixed memory pool with no allocation hook -- so they cannot
+ * provide nsa_decode's workspace.  This entry point takes the same
+ * arguments as nsa_decode minus the workspace and runs the same kernels,
+ * with the scratch taken from a fixed array inside the library's device
+ * memory (nsa_decode_noalloc_max_scratch() bytes, 4 MiB, held on every GPU
+ * that loads the library until the process exits).  It allocates nothing.
+ * A problem whose scratch would not fit returns NSA_ERR_SCRATCH_TOO_SMALL
+ * before anything is launched (B=64, 16 heads, 32768-token caches need
+ * about 0.5 MiB).  The first call on a device looks up the array's device
+ * address (with that device current) and caches it; make that first call
+ * before any stream capture.  All calls on a device share the array and it
+ * keeps the previous call's contents (every element is written before it
+ * is read, so nothing needs clearing); calls that overlap on the GPU race
+ * on it, so order them on one stream. */
+nsa_status nsa_decode_noalloc(const nsa_params* p, const void* q,
+                              const void* k_cache, const void* v_cache,
+                              const void* kc_cache, const void* vc_cache,
+                              const float* gates, void* out, int32_t* idx_out,
+                              void* stream);
+
+/* Size in bytes of nsa_decode_noalloc's fixed scratch array. */
+size_t nsa_decode_noalloc_max_scratch(void);
 
 #ifdef __cplusplus
 }

@@ -10,7 +10,8 @@ package is its thin ctypes binding (``abi``) plus seeded synthetic workloads
 from .abi import (EXPORTS, NSA_BF16, NSA_BRANCH_ALL, NSA_BRANCH_CMP, NSA_BRANCH_SEL,
                   NSA_BRANCH_SWA, NSA_F32, NsaError, Params, Saved, alloc_workspace,
                   forward, load, make_params, nsa_check_params, nsa_cmp_attn_scores,
-                  nsa_compress, nsa_decode, nsa_forward, nsa_gate_combine,
+                  nsa_compress, nsa_decode, nsa_decode_noalloc,
+                  nsa_decode_noalloc_max_scratch, nsa_forward, nsa_gate_combine,
                   nsa_last_device_error, nsa_sel_attn_fwd, nsa_select_topk,
                   nsa_status_string, nsa_swa_fwd, nsa_workspace_size, params_for)
 

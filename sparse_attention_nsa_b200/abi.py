@@ -23,13 +23,14 @@ NSA_BRANCH_ALL = 7
 
 STATUS = {0: "NSA_OK", 1: "NSA_ERR_INVALID_ARG", 2: "NSA_ERR_UNSUPPORTED",
           3: "NSA_ERR_CUDA", 4: "NSA_ERR_TIMEOUT", 5: "NSA_ERR_DEVICE_CHECK",
-          6: "NSA_ERR_WORKSPACE"}
+          6: "NSA_ERR_WORKSPACE", 7: "NSA_ERR_SCRATCH_TOO_SMALL"}
 
 # every symbol include/nsa.h declares
 EXPORTS = ("nsa_status_string", "nsa_check_params", "nsa_workspace_size",
            "nsa_last_device_error", "nsa_compress", "nsa_cmp_attn_scores",
            "nsa_select_topk", "nsa_sel_attn_fwd", "nsa_swa_fwd", "nsa_gate_combine",
-           "nsa_forward", "nsa_decode")
+           "nsa_forward", "nsa_decode", "nsa_decode_noalloc",
+           "nsa_decode_noalloc_max_scratch")
 
 
 class NsaError(RuntimeError):
@@ -93,6 +94,8 @@ def load():
             "nsa_forward": ([P, vp, vp, vp, vp, vp, C.POINTER(Saved), vp, C.c_size_t, vp],
                             C.c_int),
             "nsa_decode": ([P, vp, vp, vp, vp, vp, vp, vp, vp, vp, C.c_size_t, vp], C.c_int),
+            "nsa_decode_noalloc": ([P, vp, vp, vp, vp, vp, vp, vp, vp, vp], C.c_int),
+            "nsa_decode_noalloc_max_scratch": ([], C.c_size_t),
         }
         for name, (args, res) in sig.items():
             f = getattr(lib, name)
@@ -267,6 +270,24 @@ def nsa_decode(p: Params, q, k_cache, v_cache, kc_cache, vc_cache, gates, out,
         _ptr(gates, s["gates"], torch.float32, "gates"), _ptr(out, s["o"], dt, "out"),
         _ptr(idx_out, s["idx"], torch.int32, "idx_out", True), ws_ptr, ws_bytes,
         _stream(stream)), "nsa_decode")
+
+
+def nsa_decode_noalloc(p: Params, q, k_cache, v_cache, kc_cache, vc_cache, gates, out,
+                       idx_out=None, stream=None):
+    """nsa_decode without a workspace: the library's fixed device scratch is
+    used instead (for callers that cannot allocate; see include/nsa.h)."""
+    s, dt = _shapes(p), p.torch_dtype
+    _check(load().nsa_decode_noalloc(
+        C.byref(p), _ptr(q, s["q"], dt, "q"), _ptr(k_cache, s["k"], dt, "k_cache"),
+        _ptr(v_cache, s["k"], dt, "v_cache"), _ptr(kc_cache, s["kc"], dt, "kc_cache", p.Nc == 0),
+        _ptr(vc_cache, s["kc"], dt, "vc_cache", p.Nc == 0),
+        _ptr(gates, s["gates"], torch.float32, "gates"), _ptr(out, s["o"], dt, "out"),
+        _ptr(idx_out, s["idx"], torch.int32, "idx_out", True), _stream(stream)),
+        "nsa_decode_noalloc")
+
+
+def nsa_decode_noalloc_max_scratch() -> int:
+    return int(load().nsa_decode_noalloc_max_scratch())
 
 
 # ------------------------------------------------------------------ conveniences

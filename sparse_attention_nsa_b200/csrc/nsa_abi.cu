@@ -150,6 +150,7 @@ const char* nsa_status_string(nsa_status s) {
     case NSA_ERR_TIMEOUT: return "NSA_ERR_TIMEOUT";
     case NSA_ERR_DEVICE_CHECK: return "NSA_ERR_DEVICE_CHECK";
     case NSA_ERR_WORKSPACE: return "NSA_ERR_WORKSPACE";
+    case NSA_ERR_SCRATCH_TOO_SMALL: return "NSA_ERR_SCRATCH_TOO_SMALL";
   }
   return "NSA_ERR_UNKNOWN";
 }
@@ -343,3 +344,20 @@ nsa_status nsa_decode(const nsa_params* p, const void* q, const void* k_cache,
 }
 
 }  // extern "C"
+
+namespace nsa {
+// Workspace bytes nsa_decode carves when the compressed caches are inputs,
+// with or without a caller-provided idx_out (used by the no-alloc variant).
+nsa_status decode_scratch_bytes(const nsa_params* p, bool idx_given, size_t* bytes) {
+  Dims d;
+  nsa_status st = fill_dims(p, &d);
+  if (st != NSA_OK) return st;
+  if (!bytes) return NSA_ERR_INVALID_ARG;
+  nsa_saved sv{};
+  sv.kc = (void*)1;  // marks the slot as supplied; never dereferenced
+  sv.vc = (void*)1;
+  if (idx_given) sv.idx = (int32_t*)1;
+  *bytes = carve(d, &sv).total;
+  return NSA_OK;
+}
+}  // namespace nsa

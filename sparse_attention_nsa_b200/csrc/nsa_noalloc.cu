@@ -1,0 +1,74 @@
+// nsa_noalloc.cu -- nsa_decode_noalloc: decode for callers that cannot
+// allocate device memory.
+//
+// nsa_decode needs a scratch workspace for its intermediate branch outputs,
+// block scores and indices, which the caller normally allocates and passes
+// in.  Some callers have no way to do that: a plugin that a host framework
+// hands only its input and output buffers, or a runtime whose memory is a
+// fixed pool with no allocation hook.  This variant takes its scratch from
+// a fixed array in the library's own device memory instead, so the caller
+// passes inputs and outputs only, and nothing is allocated at call time.
+//
+// The array (kNoAllocScratchBytes) is a file-scope __device__ object: every
+// GPU that loads the library holds it until the process exits.  All calls
+// on a device share it and it keeps the previous call's contents; decode
+// writes every scratch element before reading it, so nothing needs
+// clearing.  Calls whose executions overlap on the GPU (different streams,
+// or different host threads without ordering) race on the array.
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+#include "nsa.h"
+
+namespace nsa {
+nsa_status decode_scratch_bytes(const nsa_params* p, bool idx_given, size_t* bytes);
+}
+
+// Fixed scratch for nsa_decode_noalloc: 4 MiB per device.
+static constexpr size_t kNoAllocScratchBytes = (size_t)4 << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+constexpr int kMaxDev = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDev] = {};
+
+// Device address of the scratch array on the current device.  In host code
+// the array's name only stands for it; the real address is looked up once
+// per device, with that device current, and cached.
+nsa_status scratch_ptr(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return NSA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return NSA_ERR_CUDA;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return NSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t nsa_decode_noalloc_max_scratch(void) { return kNoAllocScratchBytes; }
+
+nsa_status nsa_decode_noalloc(const nsa_params* p, const void* q, const void* k_cache,
+                              const void* v_cache, const void* kc_cache, const void* vc_cache,
+                              const float* gates, void* out, int32_t* idx_out, void* stream) {
+  size_t need = 0;
+  nsa_status st = nsa::decode_scratch_bytes(p, idx_out != nullptr, &need);
+  if (st != NSA_OK) return st;
+  if (need > kNoAllocScratchBytes) return NSA_ERR_SCRATCH_TOO_SMALL;
+  void* scratch = nullptr;
+  st = scratch_ptr(&scratch);
+  if (st != NSA_OK) return st;
+  return nsa_decode(p, q, k_cache, v_cache, kc_cache, vc_cache, gates, out, idx_out, scratch,
+                    kNoAllocScratchBytes, stream);
+}
+
+}  // extern "C"
