@@ -27,7 +27,7 @@ cudaError_t launch_compress(const Dims& d, const void* k, const void* v,
                             void* kc, void* vc, cudaStream_t s);
 cudaError_t launch_cmp_scores(const Dims& d, const void* q, const void* kc,
                               const void* vc, void* o_cmp, float* lse_cmp,
-                              float* score, cudaStream_t s);
+                              float* score, int* err, cudaStream_t s);
 cudaError_t launch_topk(const Dims& d, const float* score, int32_t* idx,
                         cudaStream_t s);
 cudaError_t launch_sel_fwd(const Dims& d, const void* q, const void* k,

@@ -24,14 +24,12 @@
 // (256 columns), P in smem, K/V in a 3-stage ring, so the MMAs of block i+1
 // and the P*V of block i overlap the softmax of block i.  Two CTAs fit per
 // SM, and their softmax and MMA phases interleave.
-#include <cudaTypedefs.h>
-
 #include <climits>
-#include <mutex>
 
 #include "common.cuh"
 #include "internal.h"
 #include "sm100.cuh"
+#include "tmap.h"
 
 namespace nsa {
 
@@ -381,38 +379,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 }
 
 // ---- host side ------------------------------------------------------------------------
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = (PFN_cuTensorMapEncodeTiled_v12000)p;
-  });
-  return fn;
-}
-
-// 3-D bf16 view (64 head dims, heads, rows) with a (64, box_h, box_rows) box,
-// 128-byte swizzle, zero fill outside the tensor.
-bool make_map(CUtensorMap* map, const void* base, int heads, long rows, int box_h,
-              int box_rows) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[3] = {64, (cuuint64_t)heads, (cuuint64_t)rows};
-  cuuint64_t strides[2] = {128, (cuuint64_t)heads * 128};
-  cuuint32_t box[3] = {64, (cuuint32_t)box_h, (cuuint32_t)box_rows};
-  cuuint32_t es[3] = {1, 1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
-            box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 bool tc_eligible(const Dims& d) {
   return d.dtype == 1 && d.l == kKeys && d.D == 64 && d.G >= 1 && kRows % d.G == 0 &&
-         d.Nb <= 4096 && encode_fn() != nullptr;
+         d.Nb <= 4096 && tmap_encode_fn() != nullptr;
 }
 
 template <bool SEL>
@@ -420,9 +389,9 @@ cudaError_t launch_tc(const Dims& d, const void* q, const void* k, const void* v
                       const int32_t* idx, void* o, float* lse, int* err, cudaStream_t s) {
   const int TQ = tokens_per_tile(d.G);
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, q, d.Hq, (long)d.B * d.Tq, d.G, TQ) ||
-      !make_map(&mk, k, d.Hkv, (long)d.B * d.T, 1, kKeys) ||
-      !make_map(&mv, v, d.Hkv, (long)d.B * d.T, 1, kKeys))
+  if (!make_tmap_bf16(&mq, q, d.Hq, (long)d.B * d.Tq, d.G, TQ) ||
+      !make_tmap_bf16(&mk, k, d.Hkv, (long)d.B * d.T, 1, kKeys) ||
+      !make_tmap_bf16(&mv, v, d.Hkv, (long)d.B * d.T, 1, kKeys))
     return cudaErrorInvalidValue;
   const size_t smem = OFF_LIST + list_ints(d) * sizeof(int) + 1024;
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<SEL>,

@@ -7,7 +7,8 @@
 // importance of block j for KV group g is the compression softmax
 // probability summed over the G query heads that share the group.
 //
-// One warp per (sequence, query, KV group).  For each of the G heads the
+// This is the fp32 path (and the path for geometries the tensor-core kernel
+// in k_cmp_tc.cu does not tile).  One warp per (sequence, query, KV group).  For each of the G heads the
 // warp computes the logits of all visible blocks (lanes over blocks), keeps
 // them in shared memory, normalises them in fp32, adds them into the
 // group's score row, and forms o_cmp with lanes over the head dimension.
@@ -102,9 +103,9 @@ static cudaError_t launch_t(const Dims& d, const void* q, const void* kc, const 
   return cudaGetLastError();
 }
 
-cudaError_t launch_cmp_scores(const Dims& d, const void* q, const void* kc,
-                              const void* vc, void* o_cmp, float* lse_cmp,
-                              float* score, cudaStream_t s) {
+cudaError_t launch_cmp_scores_simt(const Dims& d, const void* q, const void* kc,
+                                   const void* vc, void* o_cmp, float* lse_cmp,
+                                   float* score, cudaStream_t s) {
   return d.dtype == 1 ? launch_t<bf16>(d, q, kc, vc, o_cmp, lse_cmp, score, s)
                       : launch_t<float>(d, q, kc, vc, o_cmp, lse_cmp, score, s);
 }

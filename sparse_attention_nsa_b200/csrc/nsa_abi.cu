@@ -205,7 +205,7 @@ nsa_status nsa_cmp_attn_scores(const nsa_params* p, const void* q, const void* k
     return NSA_ERR_INVALID_ARG;
   if (d.Nc > 0 && !aligned16(score)) return NSA_ERR_INVALID_ARG;
   if (o_cmp && !aligned16(o_cmp)) return NSA_ERR_INVALID_ARG;
-  NSA_TRY_CUDA(nsa::launch_cmp_scores(d, q, kc, vc, o_cmp, lse_cmp, score,
+  NSA_TRY_CUDA(nsa::launch_cmp_scores(d, q, kc, vc, o_cmp, lse_cmp, score, err_word(),
                                       (cudaStream_t)stream));
   return NSA_OK;
 }
@@ -291,7 +291,7 @@ static nsa_status run_forward(const Dims& d, const void* q, const void* k, const
   if (cmp || sel) {
     if (!kc_given) NSA_TRY_CUDA(nsa::launch_compress(d, k, v, kc, vc, s));
     NSA_TRY_CUDA(nsa::launch_cmp_scores(d, q, kc, vc, cmp ? o_cmp : nullptr,
-                                        cmp ? lse_cmp : nullptr, score, s));
+                                        cmp ? lse_cmp : nullptr, score, err_word(), s));
   }
   if (sel) {
     NSA_TRY_CUDA(nsa::launch_topk(d, score, idx, s));
