@@ -16,14 +16,15 @@
 // 128 rows.
 //
 // Per block:  S = Q K^T   (tcgen05, M=128 N=64 K=64, into TMEM)
-//             softmax rows in fp32 (one thread per row, online max/sum)
-//             P (bf16, swizzled smem) ;  O_blk = P V  (tcgen05, into TMEM)
-//             o += o * alpha + O_blk in registers.
+//             softmax rows in fp32 (one thread per row, exp2 on MUFU)
+//             P (bf16, swizzled smem) ;  O += P V  (tcgen05, accumulated in TMEM)
+// P is relative to a per-row reference max that moves only when a block's
+// max exceeds it by more than 2^8; then the row's O is rescaled in TMEM.
 // Warp roles (192 threads): warps 0-3 softmax/epilogue, warp 4 MMA issue and
-// TMEM owner, warp 5 TMA producer.  S and O_blk are double-buffered in TMEM
-// (256 columns), P in smem, K/V in a 3-stage ring, so the MMAs of block i+1
-// and the P*V of block i overlap the softmax of block i.  Two CTAs fit per
-// SM, and their softmax and MMA phases interleave.
+// TMEM owner, warp 5 TMA producer.  S is double-buffered in TMEM, P in smem,
+// K/V in a 3-stage ring, so the MMAs of block i+1 and the P*V of block i
+// overlap the softmax of block i.  Two CTAs fit per SM, and their softmax
+// and MMA phases interleave.
 #include <climits>
 
 #include "common.cuh"
@@ -62,7 +63,7 @@ struct Bars {
   uint64_t empty[kStages];
   uint64_t s[2];
   uint64_t p[2];
-  uint64_t o[2];
+  uint64_t pfree[2];  // P*V of the block that used this P buffer is done
   uint64_t fin;
 };
 constexpr uint32_t OFF_MISC = OFF_BAR + ((sizeof(Bars) + 15) / 16) * 16;  // tmem, abort, nblk
@@ -108,7 +109,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->s[i], 1);
       mbar_init(&bars->p[i], 128);
-      mbar_init(&bars->o[i], 1);
+      mbar_init(&bars->pfree[i], 1);
     }
     mbar_init(&bars->fin, 1);
     fence_barrier_init();
@@ -238,12 +239,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int st = i % kStages;
         const uint32_t v_addr = smem_u32(smem + OFF_KV + st * 2 * kTileBytes + kTileBytes);
         const uint32_t p_addr = smem_u32(smem + OFF_P + (i & 1) * kPBytes);
-        const uint32_t d_tmem = tmem + 128u + (uint32_t)(i & 1) * 64u;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(d_tmem, desc_sw128(p_addr + kk * 32, 16),
-                   desc_sw128(v_addr + kk * 2048, 8192), idesc_o, kk > 0);
-        mma_commit(&bars->o[i & 1]);
+          mma_bf16(tmem + 128u, desc_sw128(p_addr + kk * 32, 16),
+                   desc_sw128(v_addr + kk * 2048, 8192), idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&bars->pfree[i & 1]);
         mma_commit(&bars->empty[st]);
       }
       // every MMA issued must finish before TMEM is released
@@ -252,6 +252,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
   } else {
     // ---- softmax and epilogue: thread r owns query row r -------------------------
+    // O accumulates in TMEM (the MMA adds P*V of every block).  P is taken
+    // relative to a per-row reference max `mref` that only moves when the
+    // block max exceeds it by more than 2^8, so P <= 256; when it moves for
+    // some row of a warp, the warp rescales its O rows in TMEM once the
+    // previous P*V has landed.
     const int r = tid;
     const int tl = r / d.G, hh = r % d.G;
     const bool valid = tl < nvalid;
@@ -259,10 +264,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const int lo = SEL ? 0 : max(0, t - d.window + 1);  // first key of the row
     const int* lst = SEL ? toks + tl * (d.topk + 1) : nullptr;
     int ptr = 0;
-    float m = -INFINITY, lsum = 0.f, alpha_prev = 1.f;
-    float acc[64];
-#pragma unroll
-    for (int c = 0; c < 64; ++c) acc[c] = 0.f;
+    float mref = -INFINITY, lsum = 0.f;
     const float sl2 = d.scale * kLog2e;
     const uint32_t lane_tmem = tmem + ((uint32_t)(warp * 32) << 16);
     const uint32_t prow = smem_u32(smem + OFF_P) + (uint32_t)(r >> 3) * 1024u + (uint32_t)(r & 7) * 128u;
@@ -290,34 +292,75 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       tmem_ld32(lane_tmem + (uint32_t)(i & 1) * 64u, sv);
       tmem_ld32(lane_tmem + (uint32_t)(i & 1) * 64u + 32u, sv + 32);
       tmem_wait_ld();
-      float alpha = 1.f;
+      float ms = -INFINITY;  // block max, scaled to log2 units
+      if (rowsel) {
+        if (!((k0 + kKeys - 1 <= t) && (k0 >= lo))) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (k0 + c > t || k0 + c < lo) sv[c] = -INFINITY;
+        }
+        float m0 = sv[0], m1 = sv[1], m2 = sv[2], m3 = sv[3];
+#pragma unroll
+        for (int c = 4; c < 64; c += 4) {
+          m0 = fmaxf(m0, sv[c]);
+          m1 = fmaxf(m1, sv[c + 1]);
+          m2 = fmaxf(m2, sv[c + 2]);
+          m3 = fmaxf(m3, sv[c + 3]);
+        }
+        ms = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)) * sl2;
+      }
+      const bool grow = rowsel && ms > mref + 8.f;
+      const bool resc = grow && mref != -INFINITY;
+      if (i > 0 && __any_sync(0xffffffffu, resc)) {
+        // O holds P*V of blocks 0..i-1: wait for the last one, rescale rows
+        if (!wait_bar_warp(&bars->pfree[(i - 1) & 1], ((i - 1) >> 1) & 1, abort_flag, err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const float f = resc ? fast_exp2(mref - ms) : 1.f;
+        float ov[32];
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          tmem_ld32(lane_tmem + 128u + 32u * h2, ov);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) ov[c] *= f;
+          tmem_st32(lane_tmem + 128u + 32u * h2, ov);
+        }
+        tmem_wait_st();
+      }
+      if (grow) {
+        if (resc) lsum *= fast_exp2(mref - ms);
+        mref = ms;
+      }
       uint32_t pk[32];
       if (rowsel) {
-        const bool full = (k0 + kKeys - 1 <= t) && (k0 >= lo);
-        float mx = -INFINITY;
+        const float nm = -mref;
+        float r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f;
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          float x = sv[c] * sl2;
-          if (!full && (k0 + c > t || k0 + c < lo)) x = -INFINITY;
-          sv[c] = x;
-          mx = fmaxf(mx, x);
+        for (int c = 0; c < 64; c += 4) {
+          const float p0 = fast_exp2(fmaf(sv[c], sl2, nm));
+          const float p1 = fast_exp2(fmaf(sv[c + 1], sl2, nm));
+          const float p2 = fast_exp2(fmaf(sv[c + 2], sl2, nm));
+          const float p3 = fast_exp2(fmaf(sv[c + 3], sl2, nm));
+          r0 += p0;
+          r1 += p1;
+          r2 += p2;
+          r3 += p3;
+          pk[c / 2] = pack_bf16(p0, p1);
+          pk[c / 2 + 1] = pack_bf16(p2, p3);
         }
-        const float mn = fmaxf(m, mx);
-        alpha = exp2f(m - mn);
-        float rs = 0.f;
-#pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const float p = exp2f(sv[c] - mn);
-          sv[c] = p;
-          rs += p;
-        }
-        lsum = lsum * alpha + rs;
-        m = mn;
-#pragma unroll
-        for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(sv[2 * c], sv[2 * c + 1]);
+        lsum += (r0 + r1) + (r2 + r3);
       } else {
 #pragma unroll
         for (int c = 0; c < 32; ++c) pk[c] = 0u;
+      }
+      // the P buffer of this block was last read by the P*V of block i-2
+      if (i >= 2 &&
+          !wait_bar_warp(&bars->pfree[i & 1], ((i - 2) >> 1) & 1, abort_flag, err)) {
+        ok = false;
+        break;
       }
       const uint32_t pb = prow + (uint32_t)(i & 1) * kPBytes;
 #pragma unroll
@@ -327,31 +370,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&bars->p[i & 1]);
-      if (i > 0) {
-        if (!wait_bar_warp(&bars->o[(i - 1) & 1], ((i - 1) >> 1) & 1, abort_flag, err)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        float ov[64];
-        tmem_ld32(lane_tmem + 128u + (uint32_t)((i - 1) & 1) * 64u, ov);
-        tmem_ld32(lane_tmem + 128u + (uint32_t)((i - 1) & 1) * 64u + 32u, ov + 32);
-        tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < 64; ++c) acc[c] = fmaf(acc[c], alpha_prev, ov[c]);
-      }
-      alpha_prev = alpha;
     }
-    if (ok && n > 0) {
-      if (wait_bar_warp(&bars->o[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag, err)) {
-        tc_fence_after();
-        float ov[64];
-        tmem_ld32(lane_tmem + 128u + (uint32_t)((n - 1) & 1) * 64u, ov);
-        tmem_ld32(lane_tmem + 128u + (uint32_t)((n - 1) & 1) * 64u + 32u, ov + 32);
-        tmem_wait_ld();
+    float acc[64];
+    bool have_o = false;
+    if (ok && n > 0)
+      have_o = wait_bar_warp(&bars->pfree[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag, err);
+    if (have_o) {
+      tc_fence_after();
+      tmem_ld32(lane_tmem + 128u, acc);
+      tmem_ld32(lane_tmem + 160u, acc + 32);
+      tmem_wait_ld();
+    } else {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) acc[c] = fmaf(acc[c], alpha_prev, ov[c]);
-      }
+      for (int c = 0; c < 64; ++c) acc[c] = 0.f;
     }
     tc_fence_before();
     if (valid) {
@@ -368,7 +399,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         u.w = pack_bf16(acc[8 * c + 6] * inv, acc[8 * c + 7] * inv);
         dst[c] = u;
       }
-      if (lse) lse[row] = lsum > 0.f ? (m + log2f(lsum)) * kLn2 : -INFINITY;
+      if (lse) lse[row] = lsum > 0.f ? (mref + log2f(lsum)) * kLn2 : -INFINITY;
     }
   }
   __syncthreads();
