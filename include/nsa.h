@@ -213,6 +213,74 @@ nsa_status nsa_decode(const nsa_params* p, const void* q, const void* k_cache,
                       int32_t* idx_out, void* workspace, size_t workspace_bytes,
                       void* stream);
 
+/* ========================================================================
+ * Backward.  Gradients are float32 and ACCUMULATED (+=) by the branch calls
+ * so that branches can be summed; nsa_backward overwrites its outputs.
+ *   dO_* (branch upstream gradients)  [B, Tq, Hq, D]  float32
+ *   dq                                 [B, Tq, Hq, D]  float32
+ *   dk, dv                             [B, T, Hkv, D]  float32
+ *   dgates                             [B, Tq, Hq, 3]  float32
+ * No gradient flows through the discrete top-k: the selection (idx) of the
+ * forward is an input.  Every gradient element is produced by one thread
+ * in a fixed order (no atomics on gradients), so results are deterministic.
+ * ======================================================================== */
+
+/* Bytes of workspace nsa_backward needs (the branch backward calls need no
+ * more than this). */
+nsa_status nsa_backward_workspace_size(const nsa_params* p, size_t* bytes);
+
+/* ---- gated combination backward --------------------------------------------
+ * dgates[.., i] = dout . o_i for enabled branches (0 otherwise) and
+ * dO_i = gate_i * dout (any dO_i may be NULL).  Passage: "DeepSeek's Native
+ * Sparse Attention" (gated merge of the three outputs).  dout, o_* dtype. */
+nsa_status nsa_gate_combine_bwd(const nsa_params* p, const float* gates,
+                                const void* dout, const void* o_cmp,
+                                const void* o_sel, const void* o_swa,
+                                float* dgates, float* dO_cmp, float* dO_sel,
+                                float* dO_swa, void* stream);
+
+/* ---- selection backward, two passes ----------------------------------------
+ * "Sparsity is Cool", Method and Key claims: a query-stationary pass computes
+ * dQ over each query's selected blocks; a reverse block->query map is
+ * rebuilt from idx (counting sort, queries in ascending order, no atomics on
+ * data); a key-stationary pass then computes dK/dV of each block over the
+ * queries that selected it.  o_sel, lse_sel are the forward's outputs.
+ * workspace: at least nsa_backward_workspace_size(p) bytes, 256-aligned. */
+nsa_status nsa_sel_attn_bwd(const nsa_params* p, const void* q, const void* k,
+                            const void* v, const int32_t* idx, const void* o_sel,
+                            const float* lse_sel, const float* dO_sel, float* dq,
+                            float* dk, float* dv, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
+/* ---- sliding-window backward (same two-pass shape; the reverse map of key
+ * s is the query range [s, s + w - 1]).  Passage: "DeepSeek's Native Sparse
+ * Attention", SLIDING WINDOW. */
+nsa_status nsa_swa_bwd(const nsa_params* p, const void* q, const void* k,
+                       const void* v, const void* o_swa, const float* lse_swa,
+                       const float* dO_swa, float* dq, float* dk, float* dv,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---- compression-branch backward: gradients reach kc/vc and, through the
+ * mean pool, each raw row of a block (d kc_j / d k_t = 1/l).  dk, dv are
+ * the RAW key/value gradients [B, T, Hkv, D].  Passage: "Sparsity is Cool",
+ * Key claims (the compression scores receive direct gradient through the
+ * gated combination; mean-pooling as the compressor). */
+nsa_status nsa_cmp_bwd(const nsa_params* p, const void* q, const void* kc,
+                       const void* vc, const void* o_cmp, const float* lse_cmp,
+                       const float* dO_cmp, float* dq, float* dk, float* dv,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---- whole backward ------------------------------------------------------------
+ * Gradient of out = nsa_forward(q, k, v, gates) for upstream dout, with the
+ * forward's saved tensors (kc, vc, o_cmp, lse_cmp for the compression branch;
+ * idx, o_sel, lse_sel for selection; o_swa, lse_swa for the window; entries
+ * of disabled branches may be NULL).  Overwrites dq, dk, dv, dgates. */
+nsa_status nsa_backward(const nsa_params* p, const void* q, const void* k,
+                        const void* v, const float* gates, const void* dout,
+                        const nsa_saved* saved, float* dq, float* dk, float* dv,
+                        float* dgates, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
 /* ---- decode without any allocation by the caller ---------------------------
  * No counterpart in the paper: this is a deployment variant of nsa_decode.
  * Some callers cannot allocate device memory -- for example a plugin that

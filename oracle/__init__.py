@@ -305,3 +305,18 @@ def decode(cfg: Cfg, q_last, kcache, vcache, kc, vc, gates_last, with_score=Fals
     if with_score:
         return out, idx, score[..., :cfg.Nc]
     return out, idx
+
+
+def backward_dq_rows(cfg: Cfg, q, k, v, gates, dout, rows, kc=None, vc=None):
+    """dq [n, Hq, D] of the full backward for a sample of (b, t) tokens."""
+    lib = _load()
+    q, k, v, gates, dout = _f64(q), _f64(k), _f64(v), _f64(gates), _f64(dout)
+    if kc is None or vc is None:
+        kc, vc = compress(cfg, k, v)
+    kc, vc = _f64(kc), _f64(vc)
+    rows = _i32(np.asarray(rows).reshape(-1, 2))
+    dq = np.zeros((rows.shape[0], cfg.Hq, cfg.D))
+    cc = cfg.c()
+    lib.orc_backward_dq_rows(C.byref(cc), _p(q), _p(k), _p(v), _p(gates), _p(dout), _p(kc),
+                             _p(vc), C.c_int(rows.shape[0]), _p(rows), _p(dq))
+    return dq

@@ -703,6 +703,79 @@ void orc_backward(const orc_cfg* c, const double* q, const double* k,
   free(dOb);
 }
 
+/* dq for a sample of query tokens only (dq is local to its row: it needs
+ * the row's own forward and upstream gradient).  rows[2*i] = b,
+ * rows[2*i+1] = t; kc/vc from orc_compress of the full input;
+ * dq_out [n, Hq, D] is overwritten. */
+void orc_backward_dq_rows(const orc_cfg* c, const double* q, const double* k,
+                          const double* v, const double* gates, const double* dout,
+                          const double* kc, const double* vc, int n,
+                          const int* rows, double* dq_out) {
+  const int nc = orc_num_cmp_blocks(c);
+  const int G = c->Hq / c->Hkv;
+  const int D = c->D;
+  const size_t HD = (size_t)c->Hq * D;
+  const int maxk = c->topk * c->sel_block + c->window + nc + 1;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int i = 0; i < n; ++i) {
+    const int b = rows[2 * i], t = rows[2 * i + 1];
+    double* oc = (double*)malloc(HD * sizeof(double));
+    double* os = (double*)malloc(HD * sizeof(double));
+    double* ow = (double*)malloc(HD * sizeof(double));
+    double* out = (double*)malloc(HD * sizeof(double));
+    double* lse = (double*)malloc((size_t)3 * c->Hq * sizeof(double));
+    double* sc = (double*)malloc(((size_t)c->Hkv * nc + 1) * sizeof(double));
+    int* idx = (int*)malloc((size_t)c->Hkv * c->topk * sizeof(int));
+    int* pos = (int*)malloc(sizeof(int) * (size_t)maxk);
+    const double** kr = (const double**)malloc(sizeof(double*) * (size_t)maxk);
+    const double** vr = (const double**)malloc(sizeof(double*) * (size_t)maxk);
+    double** dkr = (double**)malloc(sizeof(double*) * (size_t)maxk);
+    double** dvr = (double**)malloc(sizeof(double*) * (size_t)maxk);
+    double* sink = (double*)calloc((size_t)D, sizeof(double)); /* dk/dv not wanted */
+    double* dO = (double*)malloc((size_t)D * sizeof(double));
+    orc_token_forward(c, q + QI(c, b, t, 0), k, v, kc, vc, gates + RI(c, b, t, 0) * 3, b, t,
+                      oc, lse, sc, idx, os, lse + c->Hq, ow, lse + 2 * c->Hq, out);
+    for (int m = 0; m < maxk; ++m) dkr[m] = dvr[m] = sink;
+    for (int h = 0; h < c->Hq; ++h) {
+      const int g = h / G;
+      const double* qrow = q + QI(c, b, t, h);
+      const double* g3 = gates + RI(c, b, t, h) * 3;
+      const double* dorow = dout + QI(c, b, t, h);
+      double* dq = dq_out + (size_t)i * HD + (size_t)h * D;
+      for (int d = 0; d < D; ++d) dq[d] = 0.0;
+      if (c->branch_mask & ORC_CMP) {
+        const int nv = cmp_visible(c, t);
+        for (int j = 0; j < nv; ++j) {
+          kr[j] = kc + CI(c, nc, b, j, g);
+          vr[j] = vc + CI(c, nc, b, j, g);
+        }
+        for (int d = 0; d < D; ++d) dO[d] = g3[0] * dorow[d];
+        attend_bwd(qrow, D, c->scale, nv, kr, vr, dO, dq, dkr, dvr);
+      }
+      if (c->branch_mask & ORC_SEL) {
+        const int nk = sel_keys(c, idx + (size_t)g * c->topk, t, pos);
+        for (int m = 0; m < nk; ++m) {
+          kr[m] = k + KI(c, b, pos[m], g);
+          vr[m] = v + KI(c, b, pos[m], g);
+        }
+        for (int d = 0; d < D; ++d) dO[d] = g3[1] * dorow[d];
+        attend_bwd(qrow, D, c->scale, nk, kr, vr, dO, dq, dkr, dvr);
+      }
+      if (c->branch_mask & ORC_SWA) {
+        const int nk = swa_keys(c, t, pos);
+        for (int m = 0; m < nk; ++m) {
+          kr[m] = k + KI(c, b, pos[m], g);
+          vr[m] = v + KI(c, b, pos[m], g);
+        }
+        for (int d = 0; d < D; ++d) dO[d] = g3[2] * dorow[d];
+        attend_bwd(qrow, D, c->scale, nk, kr, vr, dO, dq, dkr, dvr);
+      }
+    }
+    free(oc); free(os); free(ow); free(out); free(lse); free(sc); free(idx); free(pos);
+    free(kr); free(vr); free(dkr); free(dvr); free(sink); free(dO);
+  }
+}
+
 /* ================================================================== */
 /* Decode: one query per sequence at position L-1 against a cache of  */
 /* L keys/values (its own already appended) and the compressed cache  */

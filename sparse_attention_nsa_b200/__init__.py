@@ -5,9 +5,10 @@ CUDA kernels for mean-pool compression, the compression branch with block
 scores, per-KV-group top-k selection, selection and sliding-window
 attention, the gated combination, the whole forward and decode.  This
 package is its thin ctypes binding (``abi``) plus seeded synthetic workloads
-(``inputs``).  Build the library with ``python -m sparse_attention_nsa_b200.build``.
+(``inputs``), and the backward of every branch.  Build the library with ``python -m sparse_attention_nsa_b200.build``.
 """
-from .abi import (EXPORTS, NSA_BF16, NSA_BRANCH_ALL, NSA_BRANCH_CMP, NSA_BRANCH_SEL,
+from .abi import (EXPORTS, backward, nsa_backward, nsa_backward_workspace_size,
+                  nsa_cmp_bwd, nsa_gate_combine_bwd, nsa_sel_attn_bwd, nsa_swa_bwd, NSA_BF16, NSA_BRANCH_ALL, NSA_BRANCH_CMP, NSA_BRANCH_SEL,
                   NSA_BRANCH_SWA, NSA_F32, NsaError, Params, Saved, alloc_workspace,
                   forward, load, make_params, nsa_check_params, nsa_cmp_attn_scores,
                   nsa_compress, nsa_decode, nsa_decode_noalloc,

@@ -29,8 +29,9 @@ STATUS = {0: "NSA_OK", 1: "NSA_ERR_INVALID_ARG", 2: "NSA_ERR_UNSUPPORTED",
 EXPORTS = ("nsa_status_string", "nsa_check_params", "nsa_workspace_size",
            "nsa_last_device_error", "nsa_compress", "nsa_cmp_attn_scores",
            "nsa_select_topk", "nsa_sel_attn_fwd", "nsa_swa_fwd", "nsa_gate_combine",
-           "nsa_forward", "nsa_decode", "nsa_decode_noalloc",
-           "nsa_decode_noalloc_max_scratch")
+           "nsa_forward", "nsa_decode", "nsa_backward_workspace_size",
+           "nsa_gate_combine_bwd", "nsa_sel_attn_bwd", "nsa_swa_bwd", "nsa_cmp_bwd",
+           "nsa_backward", "nsa_decode_noalloc", "nsa_decode_noalloc_max_scratch")
 
 
 class NsaError(RuntimeError):
@@ -95,6 +96,13 @@ def load():
                             C.c_int),
             "nsa_decode": ([P, vp, vp, vp, vp, vp, vp, vp, vp, vp, C.c_size_t, vp], C.c_int),
             "nsa_decode_noalloc": ([P, vp, vp, vp, vp, vp, vp, vp, vp, vp], C.c_int),
+            "nsa_backward_workspace_size": ([P, C.POINTER(C.c_size_t)], C.c_int),
+            "nsa_gate_combine_bwd": ([P] + [vp] * 10, C.c_int),
+            "nsa_sel_attn_bwd": ([P] + [vp] * 11 + [C.c_size_t, vp], C.c_int),
+            "nsa_swa_bwd": ([P] + [vp] * 10 + [C.c_size_t, vp], C.c_int),
+            "nsa_cmp_bwd": ([P] + [vp] * 10 + [C.c_size_t, vp], C.c_int),
+            "nsa_backward": ([P, vp, vp, vp, vp, vp, C.POINTER(Saved), vp, vp, vp, vp, vp,
+                              C.c_size_t, vp], C.c_int),
             "nsa_decode_noalloc_max_scratch": ([], C.c_size_t),
         }
         for name, (args, res) in sig.items():
@@ -270,6 +278,97 @@ def nsa_decode(p: Params, q, k_cache, v_cache, kc_cache, vc_cache, gates, out,
         _ptr(gates, s["gates"], torch.float32, "gates"), _ptr(out, s["o"], dt, "out"),
         _ptr(idx_out, s["idx"], torch.int32, "idx_out", True), ws_ptr, ws_bytes,
         _stream(stream)), "nsa_decode")
+
+
+# ------------------------------------------------------------------ backward
+def nsa_backward_workspace_size(p: Params) -> int:
+    n = C.c_size_t(0)
+    _check(load().nsa_backward_workspace_size(C.byref(p), C.byref(n)),
+           "nsa_backward_workspace_size")
+    return n.value
+
+
+def _ws(workspace):
+    if workspace is None:
+        return None, 0
+    return _ptr(workspace, name="workspace"), workspace.numel() * workspace.element_size()
+
+
+def nsa_gate_combine_bwd(p: Params, gates, dout, o_cmp, o_sel, o_swa, dgates,
+                         dO_cmp=None, dO_sel=None, dO_swa=None, stream=None):
+    s, dt, f = _shapes(p), p.torch_dtype, torch.float32
+    m = p.branch_mask
+    _check(load().nsa_gate_combine_bwd(
+        C.byref(p), _ptr(gates, s["gates"], f, "gates"), _ptr(dout, s["o"], dt, "dout"),
+        _ptr(o_cmp, s["o"], dt, "o_cmp", not m & 1), _ptr(o_sel, s["o"], dt, "o_sel", not m & 2),
+        _ptr(o_swa, s["o"], dt, "o_swa", not m & 4), _ptr(dgates, s["gates"], f, "dgates"),
+        _ptr(dO_cmp, s["o"], f, "dO_cmp", True), _ptr(dO_sel, s["o"], f, "dO_sel", True),
+        _ptr(dO_swa, s["o"], f, "dO_swa", True), _stream(stream)), "nsa_gate_combine_bwd")
+
+
+def nsa_sel_attn_bwd(p: Params, q, k, v, idx, o_sel, lse_sel, dO_sel, dq, dk, dv,
+                     workspace, stream=None):
+    s, dt, f = _shapes(p), p.torch_dtype, torch.float32
+    wp, wb = _ws(workspace)
+    _check(load().nsa_sel_attn_bwd(
+        C.byref(p), _ptr(q, s["q"], dt, "q"), _ptr(k, s["k"], dt, "k"), _ptr(v, s["k"], dt, "v"),
+        _ptr(idx, s["idx"], torch.int32, "idx"), _ptr(o_sel, s["o"], dt, "o_sel"),
+        _ptr(lse_sel, s["lse"], f, "lse_sel"), _ptr(dO_sel, s["o"], f, "dO_sel"),
+        _ptr(dq, s["q"], f, "dq"), _ptr(dk, s["k"], f, "dk"), _ptr(dv, s["k"], f, "dv"),
+        wp, wb, _stream(stream)), "nsa_sel_attn_bwd")
+
+
+def nsa_swa_bwd(p: Params, q, k, v, o_swa, lse_swa, dO_swa, dq, dk, dv, workspace,
+                stream=None):
+    s, dt, f = _shapes(p), p.torch_dtype, torch.float32
+    wp, wb = _ws(workspace)
+    _check(load().nsa_swa_bwd(
+        C.byref(p), _ptr(q, s["q"], dt, "q"), _ptr(k, s["k"], dt, "k"), _ptr(v, s["k"], dt, "v"),
+        _ptr(o_swa, s["o"], dt, "o_swa"), _ptr(lse_swa, s["lse"], f, "lse_swa"),
+        _ptr(dO_swa, s["o"], f, "dO_swa"), _ptr(dq, s["q"], f, "dq"), _ptr(dk, s["k"], f, "dk"),
+        _ptr(dv, s["k"], f, "dv"), wp, wb, _stream(stream)), "nsa_swa_bwd")
+
+
+def nsa_cmp_bwd(p: Params, q, kc, vc, o_cmp, lse_cmp, dO_cmp, dq, dk, dv, workspace,
+                stream=None):
+    s, dt, f = _shapes(p), p.torch_dtype, torch.float32
+    wp, wb = _ws(workspace)
+    _check(load().nsa_cmp_bwd(
+        C.byref(p), _ptr(q, s["q"], dt, "q"), _ptr(kc, s["kc"], dt, "kc", p.Nc == 0),
+        _ptr(vc, s["kc"], dt, "vc", p.Nc == 0), _ptr(o_cmp, s["o"], dt, "o_cmp"),
+        _ptr(lse_cmp, s["lse"], f, "lse_cmp"), _ptr(dO_cmp, s["o"], f, "dO_cmp"),
+        _ptr(dq, s["q"], f, "dq"), _ptr(dk, s["k"], f, "dk"), _ptr(dv, s["k"], f, "dv"),
+        wp, wb, _stream(stream)), "nsa_cmp_bwd")
+
+
+def nsa_backward(p: Params, q, k, v, gates, dout, saved: dict, dq, dk, dv, dgates,
+                 workspace, stream=None):
+    """saved: the forward's tensors by nsa_saved field name (see nsa.h)."""
+    s, dt, f = _shapes(p), p.torch_dtype, torch.float32
+    sv = Saved()
+    for name, t in saved.items():
+        if t is not None and t.numel() > 0:
+            setattr(sv, name, _ptr(t, name=name).value)
+    wp, wb = _ws(workspace)
+    _check(load().nsa_backward(
+        C.byref(p), _ptr(q, s["q"], dt, "q"), _ptr(k, s["k"], dt, "k"), _ptr(v, s["k"], dt, "v"),
+        _ptr(gates, s["gates"], f, "gates"), _ptr(dout, s["o"], dt, "dout"), C.byref(sv),
+        _ptr(dq, s["q"], f, "dq"), _ptr(dk, s["k"], f, "dk"), _ptr(dv, s["k"], f, "dv"),
+        _ptr(dgates, s["gates"], f, "dgates"), wp, wb, _stream(stream)), "nsa_backward")
+
+
+def backward(p: Params, q, k, v, gates, dout, saved: dict, workspace=None, stream=None):
+    """Allocate fp32 gradients with torch and run nsa_backward."""
+    s, dev = _shapes(p), q.device
+    dq = torch.empty(s["q"], dtype=torch.float32, device=dev)
+    dk = torch.empty(s["k"], dtype=torch.float32, device=dev)
+    dv = torch.empty(s["k"], dtype=torch.float32, device=dev)
+    dg = torch.empty(s["gates"], dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(max(nsa_backward_workspace_size(p), 1), dtype=torch.uint8,
+                                device=dev)
+    nsa_backward(p, q, k, v, gates, dout, saved, dq, dk, dv, dg, workspace, stream)
+    return dq, dk, dv, dg
 
 
 def nsa_decode_noalloc(p: Params, q, k_cache, v_cache, kc_cache, vc_cache, gates, out,

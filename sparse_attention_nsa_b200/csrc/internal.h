@@ -39,4 +39,20 @@ cudaError_t launch_combine(const Dims& d, const float* gates, const void* o_cmp,
                            const void* o_sel, const void* o_swa, void* out,
                            cudaStream_t s);
 
+// ---- backward (k_bwd.cu); mode 0 selection, 1 window, 2 compression ----
+cudaError_t launch_gate_bwd(const Dims& d, const float* gates, const void* dout,
+                            const void* o_cmp, const void* o_sel, const void* o_swa,
+                            float* dgates, float* dOc, float* dOs, float* dOw, cudaStream_t s);
+cudaError_t launch_dq(const Dims& d, int mode, const void* q, const void* keys,
+                      const void* vals, const int32_t* idx, const void* o, const float* lse,
+                      const float* dO, float* dq, float* delta, int* err, cudaStream_t s);
+cudaError_t launch_revmap(const Dims& d, const int32_t* idx, int* counts, int* offsets,
+                          int* list, cudaStream_t s);
+cudaError_t launch_dkdv(const Dims& d, int mode, const void* q, const void* keys,
+                        const void* vals, const float* lse, const float* delta,
+                        const float* dO, const int* offsets, const int* list, float* dk,
+                        float* dv, cudaStream_t s);
+cudaError_t launch_pool_bwd(const Dims& d, const float* dkc, const float* dvc, float* dk,
+                            float* dv, cudaStream_t s);
+
 }  // namespace nsa

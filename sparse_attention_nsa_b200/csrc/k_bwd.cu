@@ -1,0 +1,439 @@
+// k_bwd.cu -- NSA backward: gated combination, selection (two passes over
+// a reverse block->query map), sliding window and compression branches.
+//
+// "Sparsity is Cool: Reverse-Engineering MoBA and NSA", Method / Key claims:
+// each query attends to its own selected subset of keys, so the usual
+// key-stationary FlashAttention backward does not apply directly; the study
+// runs a query-stationary pass for dQ and then a key-stationary pass for
+// dK/dV over a reconstructed reverse key->query mapping, which beats a
+// single pass with atomics because keys are shared by many queries.  The
+// same two-pass shape serves the window and compression branches, whose
+// reverse maps are plain ranges.  No gradient flows through the top-k.
+//
+// Math per branch (rows r = (token t, head h), keys s):
+//   P = exp(scale q.k_s - lse), delta_r = dO_r . o_r,
+//   dS = P (dO_r . v_s - delta_r),  dq += scale dS k_s,
+//   dk_s += scale dS q_r,  dv_s += P dO_r.
+// Gradients are fp32 and accumulated (+=) so the branches can be summed;
+// every element is written by one thread in a fixed order (deterministic).
+#include "common.cuh"
+#include "internal.h"
+
+namespace nsa {
+
+enum BwdMode { kBwdSel = 0, kBwdSwa = 1, kBwdCmp = 2 };
+
+// ---- gated combination ---------------------------------------------------------
+// dgates[r, i] = dout_r . o_i,r (enabled branches, else 0); dO_i = gate_i dout.
+template <typename T>
+__global__ void gate_bwd_kernel(const float* __restrict__ gates, const T* __restrict__ dout,
+                                const T* __restrict__ oc, const T* __restrict__ os,
+                                const T* __restrict__ ow, float* __restrict__ dgates,
+                                float* __restrict__ dOc, float* __restrict__ dOs,
+                                float* __restrict__ dOw, long nrows, int mask) {
+  const long warp = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= nrows) return;
+  const size_t base = (size_t)warp * 64;
+  const float g0 = to_f32(dout[base + lane]), g1 = to_f32(dout[base + lane + 32]);
+  const T* br[3] = {oc, os, ow};
+  float* dst[3] = {dOc, dOs, dOw};
+#pragma unroll
+  for (int i = 0; i < 3; ++i) {
+    const bool on = (mask >> i) & 1;
+    float dg = 0.f;
+    if (on) dg = warp_sum(g0 * to_f32(br[i][base + lane]) + g1 * to_f32(br[i][base + lane + 32]));
+    const float gi = on ? gates[warp * 3 + i] : 0.f;
+    if (dst[i]) {
+      dst[i][base + lane] = gi * g0;
+      dst[i][base + lane + 32] = gi * g1;
+    }
+    if (lane == 0) dgates[warp * 3 + i] = dg;
+  }
+}
+
+// ---- pass 1: dQ, query-stationary ----------------------------------------------
+// One CTA per (sequence, query, KV group), one warp per head of the group.
+// Also writes delta_r = dO_r . o_r for the key-stationary pass.
+template <typename T, int MODE>
+__global__ void __launch_bounds__(1024)
+dq_kernel(const T* __restrict__ q, const T* __restrict__ keys, const T* __restrict__ vals,
+          const int32_t* __restrict__ idx, const T* __restrict__ o, const float* __restrict__ lse,
+          const float* __restrict__ dO, float* __restrict__ dq, float* __restrict__ delta, Dims d,
+          int* err) {
+  __shared__ float qs_all[32][64];
+  __shared__ float ds_all[32][64];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tq = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int h = g * d.G + warp;
+  const int t = d.q_off + tq;
+  const size_t row = ((size_t)b * d.Tq + tq) * d.Hq + h;
+  float* qs = qs_all[warp];
+  float* dos = ds_all[warp];
+  const float sl2 = d.scale * kLog2e;
+  qs[lane] = to_f32(q[row * 64 + lane]) * sl2;
+  qs[lane + 32] = to_f32(q[row * 64 + lane + 32]) * sl2;
+  const float d0 = dO[row * 64 + lane], d1 = dO[row * 64 + lane + 32];
+  dos[lane] = d0;
+  dos[lane + 32] = d1;
+  const float dl = warp_sum(d0 * to_f32(o[row * 64 + lane]) + d1 * to_f32(o[row * 64 + lane + 32]));
+  if (lane == 0) delta[row] = dl;
+  __syncwarp();
+  const float lse2 = lse[row] * kLog2e;
+  float a0 = 0.f, a1 = 0.f;  // dq / scale, dims lane and lane + 32
+  if (lse2 != -INFINITY) {
+    // key rows of this KV head: raw keys (sel, swa) or compressed keys (cmp)
+    const int nrow_keys = MODE == kBwdCmp ? d.Nc : d.T;
+    const size_t krow = (size_t)d.Hkv * 64;
+    const T* kb = keys + (size_t)b * nrow_keys * krow + (size_t)g * 64;
+    const T* vb = vals + (size_t)b * nrow_keys * krow + (size_t)g * 64;
+    auto fold = [&](int s0, int s1) {
+      for (int base = s0; base < s1; base += 32) {
+        const int s = base + lane;
+        float ds = 0.f;
+        if (s < s1) {
+          const T* kr = kb + (size_t)s * krow;
+          const T* vr = vb + (size_t)s * krow;
+          float qk = 0.f, dv = 0.f;
+#pragma unroll 16
+          for (int e = 0; e < 64; ++e) {
+            qk = fmaf(qs[e], to_f32(kr[e]), qk);
+            dv = fmaf(dos[e], to_f32(vr[e]), dv);
+          }
+          const float p = exp2f(qk - lse2);
+          ds = p * (dv - dl);
+        }
+        const int nk = min(32, s1 - base);
+        for (int i = 0; i < nk; ++i) {
+          const float dsi = __shfl_sync(0xffffffffu, ds, i);
+          const T* kr = kb + (size_t)(base + i) * krow;
+          a0 = fmaf(dsi, to_f32(kr[lane]), a0);
+          a1 = fmaf(dsi, to_f32(kr[lane + 32]), a1);
+        }
+      }
+    };
+    if (MODE == kBwdSel) {
+      const int32_t* ir = idx + (((size_t)b * d.Tq + tq) * d.Hkv + g) * d.topk;
+      const int cur = t / d.l;
+      int prev = -1;
+      for (int sidx = 0; sidx < d.topk; ++sidx) {
+        const int j = ir[sidx];
+        if (j == -1) continue;
+        if (j < -1 || j <= prev || j > cur) {
+          if (lane == 0) record_error(err, kDevBadIndex);
+          continue;
+        }
+        prev = j;
+        fold(j * d.l, min(j * d.l + d.l, t + 1));
+      }
+    } else if (MODE == kBwdSwa) {
+      fold(max(0, t - d.window + 1), t + 1);
+    } else {
+      fold(0, min((t + 1) / d.l, d.Nc));
+    }
+  }
+  dq[row * 64 + lane] += a0 * d.scale;
+  dq[row * 64 + lane + 32] += a1 * d.scale;
+}
+
+// ---- reverse block -> query map (selection) -------------------------------------
+// counts[b, g, j] = number of queries selecting block j; offsets = exclusive
+// scan; list[offsets[j] ..] = those queries' indices tq in ascending order.
+__global__ void rev_count_kernel(const int32_t* __restrict__ idx, int* __restrict__ counts,
+                                 Dims d) {
+  const long e = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long n = (long)d.B * d.Tq * d.Hkv * d.topk;
+  if (e >= n) return;
+  const int j = idx[e];
+  const long r = e / d.topk;  // (b, tq, g)
+  const int slot = (int)(e % d.topk);
+  const int g = (int)(r % d.Hkv);
+  const int tq = (int)((r / d.Hkv) % d.Tq);
+  const int b = (int)(r / ((long)d.Hkv * d.Tq));
+  const int cur = (d.q_off + tq) / d.l;
+  // the same validity rule as the forward: ascending, distinct, causal
+  const bool ok = j >= 0 && j <= cur && (slot == 0 || idx[e - 1] < j);
+  if (ok) atomicAdd(&counts[((size_t)b * d.Hkv + g) * (d.Nb + 1) + j], 1);
+}
+
+// one CTA per (b, g): exclusive scan of Nb counts into Nb + 1 offsets
+__global__ void rev_scan_kernel(const int* __restrict__ counts, int* __restrict__ offsets,
+                                Dims d) {
+  __shared__ int part[1024];
+  const int bg = blockIdx.x;
+  const int* c = counts + (size_t)bg * (d.Nb + 1);
+  int* off = offsets + (size_t)bg * (d.Nb + 1);
+  const int per = (d.Nb + blockDim.x - 1) / blockDim.x;
+  const int lo = threadIdx.x * per, hi = min(lo + per, d.Nb);
+  int s = 0;
+  for (int j = lo; j < hi; ++j) s += c[j];
+  part[threadIdx.x] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int i = 0; i < (int)blockDim.x; ++i) {
+      const int v = part[i];
+      part[i] = acc;
+      acc += v;
+    }
+    off[d.Nb] = acc;
+  }
+  __syncthreads();
+  int acc = part[threadIdx.x];
+  for (int j = lo; j < hi; ++j) {
+    off[j] = acc;
+    acc += c[j];
+  }
+}
+
+// one warp per (b, g, j): scan queries in order, ballot the ones that chose j
+__global__ void rev_fill_kernel(const int32_t* __restrict__ idx, const int* __restrict__ offsets,
+                                int* __restrict__ list, Dims d) {
+  const long w = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const long nw = (long)d.B * d.Hkv * d.Nb;
+  if (w >= nw) return;
+  const int j = (int)(w % d.Nb);
+  const long bg = w / d.Nb;
+  const int g = (int)(bg % d.Hkv), b = (int)(bg / d.Hkv);
+  int pos = offsets[bg * (d.Nb + 1) + j];
+  const size_t list_base = (size_t)bg * d.Tq * d.topk;
+  // a query can choose block j only once it is at or past the block
+  const int tq0 = max(0, j * d.l - d.q_off);
+  for (int base = tq0; base < d.Tq; base += 32) {
+    const int tq = base + lane;
+    bool hit = false;
+    if (tq < d.Tq) {
+      const int32_t* ir = idx + (((size_t)b * d.Tq + tq) * d.Hkv + g) * d.topk;
+      const int cur = (d.q_off + tq) / d.l;
+      if (j <= cur)
+        for (int s = 0; s < d.topk; ++s) hit |= ir[s] == j && (s == 0 || ir[s - 1] < j);
+    }
+    const unsigned m = __ballot_sync(0xffffffffu, hit);
+    if (hit) list[list_base + pos + __popc(m & ((1u << lane) - 1u))] = tq;
+    pos += __popc(m);
+  }
+}
+
+// ---- pass 2: dK, dV, key-stationary ----------------------------------------------
+// One CTA per (sequence, KV group, 64-key block); thread (key, quarter) owns
+// 16 head dims of that key's dk and dv.  Query rows are streamed in batches
+// of 32 through shared memory, in ascending query order.
+constexpr int kKB = 64;     // keys per CTA
+constexpr int kRB = 32;     // query rows per batch
+
+template <typename T, int MODE>
+__global__ void __launch_bounds__(256)
+dkdv_kernel(const T* __restrict__ q, const T* __restrict__ keys, const T* __restrict__ vals,
+            const float* __restrict__ lse, const float* __restrict__ delta,
+            const float* __restrict__ dO, const int* __restrict__ offsets,
+            const int* __restrict__ list, float* __restrict__ dk, float* __restrict__ dv,
+            Dims d) {
+  __shared__ float qsm[kRB][64];
+  __shared__ float dosm[kRB][64];
+  __shared__ float lse_s[kRB], del_s[kRB];
+  __shared__ int pos_s[kRB];
+  const int tid = threadIdx.x;
+  const int kl = tid >> 2, qd = tid & 3;  // key in chunk, quarter of dims
+  const int g = blockIdx.y, b = blockIdx.z;
+  const int nrow_keys = MODE == kBwdCmp ? d.Nc : d.T;
+  // selection: chunk c of selection block j (a block of l keys spans
+  // ceil(l / 64) chunks); window / compression: plain 64-key chunks
+  const int nsub = (d.l + kKB - 1) / kKB;
+  const int j = MODE == kBwdSel ? (int)blockIdx.x / nsub : (int)blockIdx.x;
+  const int csub = MODE == kBwdSel ? (int)blockIdx.x % nsub : 0;
+  const int s = MODE == kBwdSel ? j * d.l + csub * kKB + kl : j * kKB + kl;  // key index
+  const bool key_ok = s < nrow_keys && (MODE != kBwdSel || csub * kKB + kl < d.l);
+  const size_t krow = (size_t)d.Hkv * 64;
+  float kr[16], vr[16], dka[16], dva[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    kr[e] = key_ok ? to_f32(keys[((size_t)b * nrow_keys + s) * krow + g * 64 + qd * 16 + e]) : 0.f;
+    vr[e] = key_ok ? to_f32(vals[((size_t)b * nrow_keys + s) * krow + g * 64 + qd * 16 + e]) : 0.f;
+    dka[e] = 0.f;
+    dva[e] = 0.f;
+  }
+  const float sl2 = d.scale * kLog2e;
+  // query tokens (as query indices tq) contributing to this key block
+  int n_tok = 0, tq_lo = 0;
+  const int* lst = nullptr;
+  if (MODE == kBwdSel) {
+    const size_t bg = (size_t)b * d.Hkv + g;
+    const int o0 = offsets[bg * (d.Nb + 1) + j], o1 = offsets[bg * (d.Nb + 1) + j + 1];
+    n_tok = o1 - o0;
+    lst = list + bg * (size_t)d.Tq * d.topk + o0;
+  } else if (MODE == kBwdSwa) {
+    const int t_lo = j * kKB, t_hi = min(j * kKB + kKB - 1 + d.window - 1, d.T - 1);
+    tq_lo = max(0, t_lo - d.q_off);
+    n_tok = max(0, t_hi - d.q_off - tq_lo + 1);
+  } else {
+    const int t_lo = (j * kKB) * d.l + d.l - 1;  // first query that sees the chunk
+    tq_lo = max(0, t_lo - d.q_off);
+    n_tok = max(0, d.Tq - tq_lo);
+  }
+  const long n_rows = (long)n_tok * d.G;
+  for (long r0 = 0; r0 < n_rows; r0 += kRB) {
+    const int nr = (int)min((long)kRB, n_rows - r0);
+    __syncthreads();
+    // load the batch: row = (token-in-list, head), token-major
+    for (int e = tid; e < nr * 64; e += 256) {
+      const int rr = e >> 6, c = e & 63;
+      const long rix = r0 + rr;
+      const int ti = (int)(rix / d.G), hh = (int)(rix % d.G);
+      int tq = MODE == kBwdSel ? lst[ti] : tq_lo + ti;
+      const bool tq_ok = tq >= 0 && tq < d.Tq;
+      if (!tq_ok) tq = 0;
+      const size_t row = ((size_t)b * d.Tq + tq) * d.Hq + g * d.G + hh;
+      qsm[rr][c] = tq_ok ? to_f32(q[row * 64 + c]) : 0.f;
+      dosm[rr][c] = tq_ok ? dO[row * 64 + c] : 0.f;
+      if (c == 0) {
+        lse_s[rr] = tq_ok ? lse[row] * kLog2e : -INFINITY;
+        del_s[rr] = tq_ok ? delta[row] : 0.f;
+        pos_s[rr] = d.q_off + tq;
+      }
+    }
+    __syncthreads();
+    for (int rr = 0; rr < nr; ++rr) {
+      float qk = 0.f, dp = 0.f;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        qk = fmaf(qsm[rr][qd * 16 + e], kr[e], qk);
+        dp = fmaf(dosm[rr][qd * 16 + e], vr[e], dp);
+      }
+      qk += __shfl_xor_sync(0xffffffffu, qk, 1);
+      qk += __shfl_xor_sync(0xffffffffu, qk, 2);
+      dp += __shfl_xor_sync(0xffffffffu, dp, 1);
+      dp += __shfl_xor_sync(0xffffffffu, dp, 2);
+      const int t = pos_s[rr];
+      bool vis;
+      if (MODE == kBwdSel) vis = s <= t;
+      else if (MODE == kBwdSwa) vis = s <= t && s >= t - d.window + 1;
+      else vis = s * d.l + d.l - 1 <= t;
+      vis = vis && key_ok && lse_s[rr] != -INFINITY;
+      const float p = vis ? exp2f(qk * sl2 - lse_s[rr]) : 0.f;
+      const float ds = p * (dp - del_s[rr]);
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        dva[e] = fmaf(p, dosm[rr][qd * 16 + e], dva[e]);
+        dka[e] = fmaf(ds, qsm[rr][qd * 16 + e], dka[e]);
+      }
+    }
+  }
+  if (key_ok) {
+    float* dkr = dk + ((size_t)b * nrow_keys + s) * krow + g * 64 + qd * 16;
+    float* dvr = dv + ((size_t)b * nrow_keys + s) * krow + g * 64 + qd * 16;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      dkr[e] += dka[e] * d.scale;
+      dvr[e] += dva[e];
+    }
+  }
+}
+
+// dk[t] += dkc[t / l] / l for the tokens of complete blocks (mean-pool backward)
+__global__ void pool_bwd_kernel(const float* __restrict__ dkc, const float* __restrict__ dvc,
+                                float* __restrict__ dk, float* __restrict__ dv, Dims d) {
+  const long e = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long row_elems = (long)d.Hkv * 64;
+  const long n = (long)d.B * d.Nc * d.l * row_elems;
+  if (e >= n) return;
+  const long c = e % row_elems;
+  const long tok = e / row_elems;  // b * (Nc * l) + t
+  const int t = (int)(tok % ((long)d.Nc * d.l));
+  const int b = (int)(tok / ((long)d.Nc * d.l));
+  const int jc = t / d.l;
+  const float inv = 1.f / (float)d.l;
+  const size_t src = ((size_t)b * d.Nc + jc) * row_elems + c;
+  const size_t dst = ((size_t)b * d.T + t) * row_elems + c;
+  dk[dst] += dkc[src] * inv;
+  dv[dst] += dvc[src] * inv;
+}
+
+// ---- launchers ----------------------------------------------------------------------
+cudaError_t launch_gate_bwd(const Dims& d, const float* gates, const void* dout,
+                            const void* o_cmp, const void* o_sel, const void* o_swa,
+                            float* dgates, float* dOc, float* dOs, float* dOw, cudaStream_t s) {
+  const long nrows = (long)d.B * d.Tq * d.Hq;
+  const unsigned blocks = (unsigned)((nrows * 32 + 255) / 256);
+  if (d.dtype == 1)
+    gate_bwd_kernel<bf16><<<blocks, 256, 0, s>>>(gates, (const bf16*)dout, (const bf16*)o_cmp,
+                                                 (const bf16*)o_sel, (const bf16*)o_swa, dgates,
+                                                 dOc, dOs, dOw, nrows, d.branch_mask);
+  else
+    gate_bwd_kernel<float><<<blocks, 256, 0, s>>>(gates, (const float*)dout, (const float*)o_cmp,
+                                                  (const float*)o_sel, (const float*)o_swa,
+                                                  dgates, dOc, dOs, dOw, nrows, d.branch_mask);
+  return cudaGetLastError();
+}
+
+template <typename T, int MODE>
+static cudaError_t dq_t(const Dims& d, const void* q, const void* keys, const void* vals,
+                        const int32_t* idx, const void* o, const float* lse, const float* dO,
+                        float* dq, float* delta, int* err, cudaStream_t s) {
+  dq_kernel<T, MODE><<<dim3(d.Tq, d.Hkv, d.B), d.G * 32, 0, s>>>(
+      (const T*)q, (const T*)keys, (const T*)vals, idx, (const T*)o, lse, dO, dq, delta, d, err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dq(const Dims& d, int mode, const void* q, const void* keys, const void* vals,
+                      const int32_t* idx, const void* o, const float* lse, const float* dO,
+                      float* dq, float* delta, int* err, cudaStream_t s) {
+  if (d.dtype == 1) {
+    if (mode == kBwdSel) return dq_t<bf16, kBwdSel>(d, q, keys, vals, idx, o, lse, dO, dq, delta, err, s);
+    if (mode == kBwdSwa) return dq_t<bf16, kBwdSwa>(d, q, keys, vals, idx, o, lse, dO, dq, delta, err, s);
+    return dq_t<bf16, kBwdCmp>(d, q, keys, vals, idx, o, lse, dO, dq, delta, err, s);
+  }
+  if (mode == kBwdSel) return dq_t<float, kBwdSel>(d, q, keys, vals, idx, o, lse, dO, dq, delta, err, s);
+  if (mode == kBwdSwa) return dq_t<float, kBwdSwa>(d, q, keys, vals, idx, o, lse, dO, dq, delta, err, s);
+  return dq_t<float, kBwdCmp>(d, q, keys, vals, idx, o, lse, dO, dq, delta, err, s);
+}
+
+cudaError_t launch_revmap(const Dims& d, const int32_t* idx, int* counts, int* offsets,
+                          int* list, cudaStream_t s) {
+  const size_t nco = (size_t)d.B * d.Hkv * (d.Nb + 1);
+  cudaError_t e = cudaMemsetAsync(counts, 0, nco * sizeof(int), s);
+  if (e != cudaSuccess) return e;
+  const long n = (long)d.B * d.Tq * d.Hkv * d.topk;
+  rev_count_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(idx, counts, d);
+  rev_scan_kernel<<<d.B * d.Hkv, 256, 0, s>>>(counts, offsets, d);
+  const long nw = (long)d.B * d.Hkv * d.Nb;
+  rev_fill_kernel<<<(unsigned)((nw * 32 + 255) / 256), 256, 0, s>>>(idx, offsets, list, d);
+  return cudaGetLastError();
+}
+
+template <typename T, int MODE>
+static cudaError_t dkdv_t(const Dims& d, const void* q, const void* keys, const void* vals,
+                          const float* lse, const float* delta, const float* dO,
+                          const int* offsets, const int* list, float* dk, float* dv,
+                          cudaStream_t s) {
+  const int nkeys = MODE == kBwdCmp ? d.Nc : d.T;
+  const int nblk = MODE == kBwdSel ? d.Nb * ((d.l + kKB - 1) / kKB) : (nkeys + kKB - 1) / kKB;
+  if (nblk == 0) return cudaSuccess;
+  dkdv_kernel<T, MODE><<<dim3(nblk, d.Hkv, d.B), 256, 0, s>>>(
+      (const T*)q, (const T*)keys, (const T*)vals, lse, delta, dO, offsets, list, dk, dv, d);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dkdv(const Dims& d, int mode, const void* q, const void* keys,
+                        const void* vals, const float* lse, const float* delta, const float* dO,
+                        const int* offsets, const int* list, float* dk, float* dv,
+                        cudaStream_t s) {
+  if (d.dtype == 1) {
+    if (mode == kBwdSel) return dkdv_t<bf16, kBwdSel>(d, q, keys, vals, lse, delta, dO, offsets, list, dk, dv, s);
+    if (mode == kBwdSwa) return dkdv_t<bf16, kBwdSwa>(d, q, keys, vals, lse, delta, dO, offsets, list, dk, dv, s);
+    return dkdv_t<bf16, kBwdCmp>(d, q, keys, vals, lse, delta, dO, offsets, list, dk, dv, s);
+  }
+  if (mode == kBwdSel) return dkdv_t<float, kBwdSel>(d, q, keys, vals, lse, delta, dO, offsets, list, dk, dv, s);
+  if (mode == kBwdSwa) return dkdv_t<float, kBwdSwa>(d, q, keys, vals, lse, delta, dO, offsets, list, dk, dv, s);
+  return dkdv_t<float, kBwdCmp>(d, q, keys, vals, lse, delta, dO, offsets, list, dk, dv, s);
+}
+
+cudaError_t launch_pool_bwd(const Dims& d, const float* dkc, const float* dvc, float* dk,
+                            float* dv, cudaStream_t s) {
+  const long n = (long)d.B * d.Nc * d.l * d.Hkv * 64;
+  if (n == 0) return cudaSuccess;
+  pool_bwd_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(dkc, dvc, dk, dv, d);
+  return cudaGetLastError();
+}
+
+}  // namespace nsa

@@ -361,3 +361,209 @@ nsa_status decode_scratch_bytes(const nsa_params* p, bool idx_given, size_t* byt
   return NSA_OK;
 }
 }  // namespace nsa
+
+// ============================================================================
+// Backward entry points
+// ============================================================================
+namespace {
+
+// Backward workspace layout, each part 256-byte aligned:
+//   delta [B*Tq*Hq] f32 | dO_cmp, dO_sel, dO_swa [B*Tq*Hq*64] f32 |
+//   dkc, dvc [B*Nc*Hkv*64] f32 | counts, offsets [B*Hkv*(Nb+1)] i32 |
+//   list [B*Hkv*Tq*topk] i32
+struct BwdCarve {
+  size_t delta, dO[3], dkc, dvc, counts, offsets, list, total;
+};
+
+BwdCarve bwd_carve(const Dims& d) {
+  BwdCarve c{};
+  size_t at = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = at;
+    at += align256(bytes);
+    return o;
+  };
+  const size_t rows = (size_t)d.B * d.Tq * d.Hq;
+  c.delta = take(rows * 4);
+  for (int i = 0; i < 3; ++i) c.dO[i] = take(rows * 64 * 4);
+  c.dkc = take((size_t)d.B * d.Nc * d.Hkv * 64 * 4);
+  c.dvc = take((size_t)d.B * d.Nc * d.Hkv * 64 * 4);
+  c.counts = take((size_t)d.B * d.Hkv * (d.Nb + 1) * 4);
+  c.offsets = take((size_t)d.B * d.Hkv * (d.Nb + 1) * 4);
+  c.list = take((size_t)d.B * d.Hkv * d.Tq * d.topk * 4);
+  c.total = at;
+  return c;
+}
+
+bool ws_ok(const void* ws, size_t bytes, size_t need) {
+  return ws && bytes >= need && (((uintptr_t)ws) & 255u) == 0;
+}
+
+nsa_status sel_bwd_body(const Dims& d, const void* q, const void* k, const void* v,
+                        const int32_t* idx, const void* o_sel, const float* lse_sel,
+                        const float* dO_sel, float* dq, float* dk, float* dv, char* w,
+                        const BwdCarve& c, cudaStream_t s) {
+  float* delta = (float*)(w + c.delta);
+  int* counts = (int*)(w + c.counts);
+  int* offsets = (int*)(w + c.offsets);
+  int* list = (int*)(w + c.list);
+  NSA_TRY_CUDA(nsa::launch_dq(d, 0, q, k, v, idx, o_sel, lse_sel, dO_sel, dq, delta, err_word(), s));
+  NSA_TRY_CUDA(nsa::launch_revmap(d, idx, counts, offsets, list, s));
+  NSA_TRY_CUDA(nsa::launch_dkdv(d, 0, q, k, v, lse_sel, delta, dO_sel, offsets, list, dk, dv, s));
+  return NSA_OK;
+}
+
+nsa_status swa_bwd_body(const Dims& d, const void* q, const void* k, const void* v,
+                        const void* o_swa, const float* lse_swa, const float* dO_swa,
+                        float* dq, float* dk, float* dv, char* w, const BwdCarve& c,
+                        cudaStream_t s) {
+  float* delta = (float*)(w + c.delta);
+  NSA_TRY_CUDA(nsa::launch_dq(d, 1, q, k, v, nullptr, o_swa, lse_swa, dO_swa, dq, delta, nullptr, s));
+  NSA_TRY_CUDA(nsa::launch_dkdv(d, 1, q, k, v, lse_swa, delta, dO_swa, nullptr, nullptr, dk, dv, s));
+  return NSA_OK;
+}
+
+nsa_status cmp_bwd_body(const Dims& d, const void* q, const void* kc, const void* vc,
+                        const void* o_cmp, const float* lse_cmp, const float* dO_cmp,
+                        float* dq, float* dk, float* dv, char* w, const BwdCarve& c,
+                        cudaStream_t s) {
+  float* delta = (float*)(w + c.delta);
+  float* dkc = (float*)(w + c.dkc);
+  float* dvc = (float*)(w + c.dvc);
+  if (d.Nc == 0) return NSA_OK;  // nothing visible anywhere: no gradient
+  const size_t nkc = (size_t)d.B * d.Nc * d.Hkv * 64 * 4;
+  NSA_TRY_CUDA(cudaMemsetAsync(dkc, 0, nkc, s));
+  NSA_TRY_CUDA(cudaMemsetAsync(dvc, 0, nkc, s));
+  NSA_TRY_CUDA(nsa::launch_dq(d, 2, q, kc, vc, nullptr, o_cmp, lse_cmp, dO_cmp, dq, delta, nullptr, s));
+  NSA_TRY_CUDA(nsa::launch_dkdv(d, 2, q, kc, vc, lse_cmp, delta, dO_cmp, nullptr, nullptr, dkc, dvc, s));
+  NSA_TRY_CUDA(nsa::launch_pool_bwd(d, dkc, dvc, dk, dv, s));
+  return NSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+nsa_status nsa_backward_workspace_size(const nsa_params* p, size_t* bytes) {
+  Dims d;
+  nsa_status st = fill_dims(p, &d);
+  if (st != NSA_OK) return st;
+  if (!bytes) return NSA_ERR_INVALID_ARG;
+  *bytes = bwd_carve(d).total;
+  return NSA_OK;
+}
+
+nsa_status nsa_gate_combine_bwd(const nsa_params* p, const float* gates, const void* dout,
+                                const void* o_cmp, const void* o_sel, const void* o_swa,
+                                float* dgates, float* dO_cmp, float* dO_sel, float* dO_swa,
+                                void* stream) {
+  Dims d;
+  nsa_status st = fill_dims(p, &d);
+  if (st != NSA_OK) return st;
+  if (!aligned16(gates) || !aligned16(dout) || !aligned16(dgates)) return NSA_ERR_INVALID_ARG;
+  if ((d.branch_mask & NSA_BRANCH_CMP) && !aligned16(o_cmp)) return NSA_ERR_INVALID_ARG;
+  if ((d.branch_mask & NSA_BRANCH_SEL) && !aligned16(o_sel)) return NSA_ERR_INVALID_ARG;
+  if ((d.branch_mask & NSA_BRANCH_SWA) && !aligned16(o_swa)) return NSA_ERR_INVALID_ARG;
+  for (const void* ptr : {(const void*)dO_cmp, (const void*)dO_sel, (const void*)dO_swa})
+    if (ptr && (((uintptr_t)ptr) & 15u)) return NSA_ERR_INVALID_ARG;
+  NSA_TRY_CUDA(nsa::launch_gate_bwd(d, gates, dout, o_cmp, o_sel, o_swa, dgates, dO_cmp, dO_sel,
+                                    dO_swa, (cudaStream_t)stream));
+  return NSA_OK;
+}
+
+nsa_status nsa_sel_attn_bwd(const nsa_params* p, const void* q, const void* k, const void* v,
+                            const int32_t* idx, const void* o_sel, const float* lse_sel,
+                            const float* dO_sel, float* dq, float* dk, float* dv, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  Dims d;
+  nsa_status st = fill_dims(p, &d);
+  if (st != NSA_OK) return st;
+  for (const void* ptr : {q, k, v, (const void*)idx, o_sel, (const void*)lse_sel,
+                          (const void*)dO_sel, (const void*)dq, (const void*)dk, (const void*)dv})
+    if (!aligned16(ptr)) return NSA_ERR_INVALID_ARG;
+  const BwdCarve c = bwd_carve(d);
+  if (!ws_ok(workspace, workspace_bytes, c.total)) return NSA_ERR_WORKSPACE;
+  return sel_bwd_body(d, q, k, v, idx, o_sel, lse_sel, dO_sel, dq, dk, dv, (char*)workspace, c,
+                      (cudaStream_t)stream);
+}
+
+nsa_status nsa_swa_bwd(const nsa_params* p, const void* q, const void* k, const void* v,
+                       const void* o_swa, const float* lse_swa, const float* dO_swa, float* dq,
+                       float* dk, float* dv, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  Dims d;
+  nsa_status st = fill_dims(p, &d);
+  if (st != NSA_OK) return st;
+  for (const void* ptr : {q, k, v, o_swa, (const void*)lse_swa, (const void*)dO_swa,
+                          (const void*)dq, (const void*)dk, (const void*)dv})
+    if (!aligned16(ptr)) return NSA_ERR_INVALID_ARG;
+  const BwdCarve c = bwd_carve(d);
+  if (!ws_ok(workspace, workspace_bytes, c.total)) return NSA_ERR_WORKSPACE;
+  return swa_bwd_body(d, q, k, v, o_swa, lse_swa, dO_swa, dq, dk, dv, (char*)workspace, c,
+                      (cudaStream_t)stream);
+}
+
+nsa_status nsa_cmp_bwd(const nsa_params* p, const void* q, const void* kc, const void* vc,
+                       const void* o_cmp, const float* lse_cmp, const float* dO_cmp, float* dq,
+                       float* dk, float* dv, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  Dims d;
+  nsa_status st = fill_dims(p, &d);
+  if (st != NSA_OK) return st;
+  for (const void* ptr : {q, o_cmp, (const void*)lse_cmp, (const void*)dO_cmp, (const void*)dq,
+                          (const void*)dk, (const void*)dv})
+    if (!aligned16(ptr)) return NSA_ERR_INVALID_ARG;
+  if (d.Nc > 0 && (!aligned16(kc) || !aligned16(vc))) return NSA_ERR_INVALID_ARG;
+  const BwdCarve c = bwd_carve(d);
+  if (!ws_ok(workspace, workspace_bytes, c.total)) return NSA_ERR_WORKSPACE;
+  return cmp_bwd_body(d, q, kc, vc, o_cmp, lse_cmp, dO_cmp, dq, dk, dv, (char*)workspace, c,
+                      (cudaStream_t)stream);
+}
+
+nsa_status nsa_backward(const nsa_params* p, const void* q, const void* k, const void* v,
+                        const float* gates, const void* dout, const nsa_saved* sv, float* dq,
+                        float* dk, float* dv, float* dgates, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  Dims d;
+  nsa_status st = fill_dims(p, &d);
+  if (st != NSA_OK) return st;
+  if (!sv) return NSA_ERR_INVALID_ARG;
+  for (const void* ptr : {q, k, v, (const void*)gates, dout, (const void*)dq, (const void*)dk,
+                          (const void*)dv, (const void*)dgates})
+    if (!aligned16(ptr)) return NSA_ERR_INVALID_ARG;
+  const bool cmp = d.branch_mask & NSA_BRANCH_CMP;
+  const bool sel = d.branch_mask & NSA_BRANCH_SEL;
+  const bool swa = d.branch_mask & NSA_BRANCH_SWA;
+  if (cmp && (!aligned16(sv->o_cmp) || !aligned16(sv->lse_cmp) ||
+              (d.Nc > 0 && (!aligned16(sv->kc) || !aligned16(sv->vc)))))
+    return NSA_ERR_INVALID_ARG;
+  if (sel && (!aligned16(sv->idx) || !aligned16(sv->o_sel) || !aligned16(sv->lse_sel)))
+    return NSA_ERR_INVALID_ARG;
+  if (swa && (!aligned16(sv->o_swa) || !aligned16(sv->lse_swa))) return NSA_ERR_INVALID_ARG;
+  const BwdCarve c = bwd_carve(d);
+  if (!ws_ok(workspace, workspace_bytes, c.total)) return NSA_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  char* w = (char*)workspace;
+  float* dO[3] = {(float*)(w + c.dO[0]), (float*)(w + c.dO[1]), (float*)(w + c.dO[2])};
+  NSA_TRY_CUDA(nsa::launch_gate_bwd(d, gates, dout, sv->o_cmp, sv->o_sel, sv->o_swa, dgates,
+                                    cmp ? dO[0] : nullptr, sel ? dO[1] : nullptr,
+                                    swa ? dO[2] : nullptr, s));
+  NSA_TRY_CUDA(cudaMemsetAsync(dq, 0, (size_t)d.B * d.Tq * d.Hq * 64 * 4, s));
+  NSA_TRY_CUDA(cudaMemsetAsync(dk, 0, (size_t)d.B * d.T * d.Hkv * 64 * 4, s));
+  NSA_TRY_CUDA(cudaMemsetAsync(dv, 0, (size_t)d.B * d.T * d.Hkv * 64 * 4, s));
+  if (cmp) {
+    st = cmp_bwd_body(d, q, sv->kc, sv->vc, sv->o_cmp, sv->lse_cmp, dO[0], dq, dk, dv, w, c, s);
+    if (st != NSA_OK) return st;
+  }
+  if (sel) {
+    st = sel_bwd_body(d, q, k, v, sv->idx, sv->o_sel, sv->lse_sel, dO[1], dq, dk, dv, w, c, s);
+    if (st != NSA_OK) return st;
+  }
+  if (swa) {
+    st = swa_bwd_body(d, q, k, v, sv->o_swa, sv->lse_swa, dO[2], dq, dk, dv, w, c, s);
+    if (st != NSA_OK) return st;
+  }
+  return NSA_OK;
+}
+
+}  // extern "C"

@@ -455,3 +455,16 @@ def test_sel_backward_matches_autograd_of_masked_attention():
     np.testing.assert_allclose(dq, qt.grad.numpy(), atol=1e-12)
     np.testing.assert_allclose(dk, kt.grad.numpy(), atol=1e-12)
     np.testing.assert_allclose(dv, vt.grad.numpy(), atol=1e-12)
+
+
+def test_backward_dq_rows_match_full_backward():
+    c = cfg_small(T=40)
+    q, k, v = qkv(c, 131)
+    g = np.random.default_rng(132)
+    gates = g.random((c.B, c.T, c.Hq, 3))
+    dout = g.standard_normal((c.B, c.T, c.Hq, c.D))
+    dq, _, _, _ = orc.backward(c, q, k, v, gates, dout)
+    rows = np.array([[0, 0], [1, 39], [0, 8], [1, 23], [0, 31]])
+    got = orc.backward_dq_rows(c, q, k, v, gates, dout, rows)
+    for i, (b, t) in enumerate(rows):
+        np.testing.assert_allclose(got[i], dq[b, t], rtol=0, atol=1e-13)
