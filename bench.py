@@ -75,6 +75,24 @@ def load_peaks() -> dict:
                 "source": "fallback"}
 
 
+def profiled_traffic(kernel_src: str, profile_md: str):
+    """DRAM bytes per launch recorded in a committed ncu summary, if that
+    summary was taken on the current source of the kernel (its sha1 prefix
+    matches); otherwise None (the counters are stale)."""
+    import hashlib
+    try:
+        sha = hashlib.sha1(open(os.path.join(ROOT, kernel_src), "rb").read()).hexdigest()[:12]
+        rec_sha, traffic = None, None
+        for line in open(os.path.join(ROOT, profile_md)):
+            if line.startswith("source-sha1:"):
+                rec_sha = line.split(":", 1)[1].strip()
+            if line.startswith("| dram_bytes_per_launch"):
+                traffic = int(line.split("|")[2].strip())
+        return traffic if rec_sha == sha else None
+    except Exception:
+        return None
+
+
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
     """Samples SM clock and clock-event reasons through NVML (read only)."""
@@ -295,6 +313,9 @@ def run_gpu(args, rank: int, world: int, dist_on: bool) -> None:
 
     # decode (B=64 sequences, 32768-token caches): HBM GB/s
     dec = run_decode(dev, flush, stream, args.steps, peaks)
+    # training step (B=8 forward + backward)
+    del hq, hk, hv, hg, hout
+    train = run_train(dev, flush, stream, max(3, args.steps // 4), peaks)
 
     barrier_sync(dist_on)
     if rank != 0:
@@ -314,9 +335,12 @@ def run_gpu(args, rank: int, world: int, dist_on: bool) -> None:
         "flops_per_step": flops,
         "roofline": {"bound": "tensor", "kernel": "selection attention (nsa_sel_attn_fwd)",
                      "achieved": sel_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": sel_tflops / peaks["bf16_tflops"], "traffic": None,
+                     "frac": sel_tflops / peaks["bf16_tflops"],
+                     "traffic": profiled_traffic("sparse_attention_nsa_b200/csrc/k_attn_tc.cu",
+                                                 "profiles/attn_tc_sel_340m.md"),
                      "ms_per_launch": sel_ms, "peak_source": peaks["source"] + " burst bf16"},
         "decode": dec,
+        "train": train,
         "e2e": {"value": tokens_per_step * world / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": KERNELS_PER_FORWARD * args.steps,
@@ -325,6 +349,48 @@ def run_gpu(args, rank: int, world: int, dist_on: bool) -> None:
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_tokens_per_s(budget_s=12.0)
     print(json.dumps(line), flush=True)
+
+
+def run_train(dev, flush, stream, steps, peaks) -> dict:
+    """One training step of attention: NSA forward (intermediates kept) and
+    the whole backward, B=8 x 8192 tokens, 340M shape."""
+    w = W.TRAIN_340M
+    inp = W.make_inputs(w, seed=1, with_dout=True)
+    q, k, v, g, dout = (inp[n].to(dev) for n in ("q", "k", "v", "gates", "dout"))
+    p = nsa.params_for(w)
+    out = torch.empty_like(q)
+    ws = nsa.alloc_workspace(p, dev)
+    f32 = torch.float32
+    saved = {"kc": torch.empty((w.B, w.Nc, w.Hkv, w.D), dtype=w.dtype, device=dev),
+             "vc": torch.empty((w.B, w.Nc, w.Hkv, w.D), dtype=w.dtype, device=dev),
+             "o_cmp": torch.empty_like(q), "o_sel": torch.empty_like(q), "o_swa": torch.empty_like(q),
+             "lse_cmp": torch.empty((w.B, w.T, w.Hq), dtype=f32, device=dev),
+             "lse_sel": torch.empty((w.B, w.T, w.Hq), dtype=f32, device=dev),
+             "lse_swa": torch.empty((w.B, w.T, w.Hq), dtype=f32, device=dev),
+             "idx": torch.empty((w.B, w.T, w.Hkv, w.topk), dtype=torch.int32, device=dev)}
+    dq = torch.empty((w.B, w.T, w.Hq, w.D), dtype=f32, device=dev)
+    dk = torch.empty((w.B, w.T, w.Hkv, w.D), dtype=f32, device=dev)
+    dv = torch.empty_like(dk)
+    dg = torch.empty((w.B, w.T, w.Hq, 3), dtype=f32, device=dev)
+    bws = torch.empty(nsa.nsa_backward_workspace_size(p), dtype=torch.uint8, device=dev)
+
+    def fwd():
+        nsa.nsa_forward(p, q, k, v, g, out, saved, ws)
+
+    def bwd():
+        nsa.nsa_backward(p, q, k, v, g, dout, saved, dq, dk, dv, dg, bws)
+
+    for _ in range(2):
+        fwd()
+        bwd()
+    fwd_ms = statistics.mean(timed_steps(fwd, steps, flush, stream))
+    bwd_ms = statistics.mean(timed_steps(bwd, steps, flush, stream))
+    flops = fwd_flops(w)["total"]
+    step_ms = fwd_ms + bwd_ms
+    return {"workload": w.name, "fwd_ms": fwd_ms, "bwd_ms": bwd_ms, "ms_per_step": step_ms,
+            "tokens_per_s": w.B * w.T / (step_ms * 1e-3),
+            "tflops_fwd_plus_bwd": 3.5 * flops / (step_ms * 1e-3) / 1e12,
+            "flops_note": "algorithmic: forward + backward counted as 2.5x forward"}
 
 
 def run_decode(dev, flush, stream, steps, peaks) -> dict:

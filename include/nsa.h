@@ -205,8 +205,13 @@ nsa_status nsa_forward(const nsa_params* p, const void* q, const void* k,
  * k_cache/v_cache [B, T, Hkv, D] that already hold that position, and the
  * compressed caches kc_cache/vc_cache [B, Nc, Hkv, D] (nsa_compress of the
  * caches).  q [B, 1, Hq, D], gates [B, 1, Hq, 3], out [B, 1, Hq, D];
- * idx_out [B, 1, Hkv, topk] may be NULL.  Same arithmetic as nsa_forward
- * for that one position. */
+ * idx_out [B, 1, Hkv, topk] may be NULL (it is written only when the
+ * selection branch is enabled).  Same arithmetic as nsa_forward for that
+ * one position.  For bf16, block 64, at most 16 query heads per KV group
+ * and at most 512 compressed blocks, decode runs as three kernels that
+ * stream the caches across all SMs (compression + scores + top-k per
+ * sequence; one small CTA per selected or window block; a merge); other
+ * shapes reuse the prefill kernels. */
 nsa_status nsa_decode(const nsa_params* p, const void* q, const void* k_cache,
                       const void* v_cache, const void* kc_cache,
                       const void* vc_cache, const float* gates, void* out,
@@ -289,11 +294,11 @@ nsa_status nsa_backward(const nsa_params* p, const void* q, const void* k,
  * provide nsa_decode's workspace.  This entry point takes the same
  * arguments as nsa_decode minus the workspace and runs the same kernels,
  * with the scratch taken from a fixed array inside the library's device
- * memory (nsa_decode_noalloc_max_scratch() bytes, 4 MiB, held on every GPU
+ * memory (nsa_decode_noalloc_max_scratch() bytes, 8 MiB, held on every GPU
  * that loads the library until the process exits).  It allocates nothing.
  * A problem whose scratch would not fit returns NSA_ERR_SCRATCH_TOO_SMALL
- * before anything is launched (B=64, 16 heads, 32768-token caches need
- * about 0.5 MiB).  The first call on a device looks up the array's device
+ * before anything is launched (B=64 sequences, 16 heads on one KV head,
+ * 32768-token caches, top-k 16, window 512 need about 6.8 MiB).  The first call on a device looks up the array's device
  * address (with that device current) and caches it; make that first call
  * before any stream capture.  All calls on a device share the array and it
  * keeps the previous call's contents (every element is written before it

@@ -55,4 +55,12 @@ cudaError_t launch_dkdv(const Dims& d, int mode, const void* q, const void* keys
 cudaError_t launch_pool_bwd(const Dims& d, const float* dkc, const float* dvc, float* dk,
                             float* dv, cudaStream_t s);
 
+// ---- decode split into HBM-streaming kernels (k_decode.cu) ----
+bool decode_split_eligible(const Dims& d);
+size_t decode_split_ws_bytes(const Dims& d);
+cudaError_t launch_decode_split(const Dims& d, const void* q, const void* kcache,
+                                const void* vcache, const void* kc, const void* vc,
+                                const float* gates, void* out, int32_t* idx_out, void* ws,
+                                int* err, cudaStream_t s);
+
 }  // namespace nsa

@@ -52,6 +52,48 @@ __global__ void gate_bwd_kernel(const float* __restrict__ gates, const T* __rest
   }
 }
 
+// Two 64-wide dot products of shared-memory rows a, c with global rows x, y
+// (16-byte loads).
+template <typename T>
+__device__ __forceinline__ void dot2_64(const float* a, const float* c, const T* x, const T* y,
+                                        float& ax, float& cy);
+template <>
+__device__ __forceinline__ void dot2_64<bf16>(const float* a, const float* c, const bf16* x,
+                                              const bf16* y, float& ax, float& cy) {
+  float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint4 ux = __ldg(reinterpret_cast<const uint4*>(x) + k);
+    const uint4 uy = __ldg(reinterpret_cast<const uint4*>(y) + k);
+    const __nv_bfloat162* px = reinterpret_cast<const __nv_bfloat162*>(&ux);
+    const __nv_bfloat162* py = reinterpret_cast<const __nv_bfloat162*>(&uy);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 fx = __bfloat1622float2(px[i]), fy = __bfloat1622float2(py[i]);
+      s0 = fmaf(a[8 * k + 2 * i], fx.x, s0);
+      s0 = fmaf(a[8 * k + 2 * i + 1], fx.y, s0);
+      s1 = fmaf(c[8 * k + 2 * i], fy.x, s1);
+      s1 = fmaf(c[8 * k + 2 * i + 1], fy.y, s1);
+    }
+  }
+  ax = s0;
+  cy = s1;
+}
+template <>
+__device__ __forceinline__ void dot2_64<float>(const float* a, const float* c, const float* x,
+                                               const float* y, float& ax, float& cy) {
+  float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const float4 fx = __ldg(reinterpret_cast<const float4*>(x) + k);
+    const float4 fy = __ldg(reinterpret_cast<const float4*>(y) + k);
+    s0 = fmaf(a[4 * k], fx.x, fmaf(a[4 * k + 1], fx.y, fmaf(a[4 * k + 2], fx.z, fmaf(a[4 * k + 3], fx.w, s0))));
+    s1 = fmaf(c[4 * k], fy.x, fmaf(c[4 * k + 1], fy.y, fmaf(c[4 * k + 2], fy.z, fmaf(c[4 * k + 3], fy.w, s1))));
+  }
+  ax = s0;
+  cy = s1;
+}
+
 // ---- pass 1: dQ, query-stationary ----------------------------------------------
 // One CTA per (sequence, query, KV group), one warp per head of the group.
 // Also writes delta_r = dO_r . o_r for the key-stationary pass.
@@ -92,14 +134,8 @@ dq_kernel(const T* __restrict__ q, const T* __restrict__ keys, const T* __restri
         const int s = base + lane;
         float ds = 0.f;
         if (s < s1) {
-          const T* kr = kb + (size_t)s * krow;
-          const T* vr = vb + (size_t)s * krow;
-          float qk = 0.f, dv = 0.f;
-#pragma unroll 16
-          for (int e = 0; e < 64; ++e) {
-            qk = fmaf(qs[e], to_f32(kr[e]), qk);
-            dv = fmaf(dos[e], to_f32(vr[e]), dv);
-          }
+          float qk, dv;
+          dot2_64<T>(qs, dos, kb + (size_t)s * krow, vb + (size_t)s * krow, qk, dv);
           const float p = exp2f(qk - lse2);
           ds = p * (dv - dl);
         }

@@ -3,6 +3,7 @@
 // This layer validates arguments, derives sizes, carves the caller's
 // workspace, and enqueues kernels on the caller's stream.  It allocates no
 // device memory and never synchronises except in nsa_last_device_error.
+#include <algorithm>
 #include <mutex>
 
 #include "common.cuh"
@@ -166,6 +167,7 @@ nsa_status nsa_workspace_size(const nsa_params* p, size_t* bytes) {
   if (st != NSA_OK) return st;
   if (!bytes) return NSA_ERR_INVALID_ARG;
   *bytes = carve(d, nullptr).total;
+  if (nsa::decode_split_eligible(d)) *bytes = std::max(*bytes, nsa::decode_split_ws_bytes(d));
   return NSA_OK;
 }
 
@@ -335,6 +337,14 @@ nsa_status nsa_decode(const nsa_params* p, const void* q, const void* k_cache,
     return NSA_ERR_INVALID_ARG;
   if (d.Nc > 0 && (!aligned16(kc_cache) || !aligned16(vc_cache))) return NSA_ERR_INVALID_ARG;
   if (idx_out && (((uintptr_t)idx_out) & 15u)) return NSA_ERR_INVALID_ARG;
+  if (nsa::decode_split_eligible(d)) {
+    const size_t need = nsa::decode_split_ws_bytes(d);
+    if (!workspace || workspace_bytes < need || (((uintptr_t)workspace) & 255u) != 0)
+      return NSA_ERR_WORKSPACE;
+    NSA_TRY_CUDA(nsa::launch_decode_split(d, q, k_cache, v_cache, kc_cache, vc_cache, gates, out,
+                                          idx_out, workspace, err_word(), (cudaStream_t)stream));
+    return NSA_OK;
+  }
   nsa_saved sv{};
   sv.idx = idx_out;
   sv.kc = (void*)kc_cache;  // inputs here; NULL only when Nc == 0 (never read)
@@ -353,6 +363,10 @@ nsa_status decode_scratch_bytes(const nsa_params* p, bool idx_given, size_t* byt
   nsa_status st = fill_dims(p, &d);
   if (st != NSA_OK) return st;
   if (!bytes) return NSA_ERR_INVALID_ARG;
+  if (decode_split_eligible(d)) {
+    *bytes = decode_split_ws_bytes(d);
+    return NSA_OK;
+  }
   nsa_saved sv{};
   sv.kc = (void*)1;  // marks the slot as supplied; never dereferenced
   sv.vc = (void*)1;

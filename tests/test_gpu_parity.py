@@ -286,9 +286,12 @@ def check_decode(w, inp, seqs):
     okc, ovc = orc.compress(c, kcache, vcache)
     o_ref, i_ref, s_ref = orc.decode(c, inp["q"][seqs], kcache, vcache, okc, ovc,
                                      inp["gates"][seqs], with_score=True)
-    diff = idx_mismatch_rows(to_np(idx)[seqs], i_ref, s_ref,
-                             np.full(len(seqs) * w.Hkv, w.T - 1), w.topk, w.sel_block)
-    keep = ~diff.reshape(len(seqs), w.Hkv).any(-1)
+    if w.branch_mask & W.BR_SEL:  # idx_out is written when selection runs
+        diff = idx_mismatch_rows(to_np(idx)[seqs], i_ref, s_ref,
+                                 np.full(len(seqs) * w.Hkv, w.T - 1), w.topk, w.sel_block)
+        keep = ~diff.reshape(len(seqs), w.Hkv).any(-1)
+    else:
+        keep = np.ones(len(seqs), dtype=bool)
     assert_close(to_np(out)[seqs][keep], o_ref[keep], TOL[w.dtype], "decode out")
 
 
@@ -296,6 +299,12 @@ def check_decode(w, inp, seqs):
     W.DECODE_32K.replace(name="decode_small", B=3, T=1500),
     W.DECODE_32K.replace(name="decode_gqa_ragged", B=5, T=2049, Hq=16, Hkv=4),
     W.DECODE_32K.replace(name="decode_short", B=2, T=70),
+    W.DECODE_32K.replace(name="decode_pruned_w100_k4", B=4, T=5000, topk=4, window=100,
+                         branch_mask=W.BR_SEL | W.BR_SWA, cmp_gate_zero=True),
+    W.DECODE_32K.replace(name="decode_swa_only_gqa8", B=3, T=3333, Hq=16, Hkv=2, window=200,
+                         branch_mask=W.BR_SWA),
+    W.DECODE_32K.replace(name="decode_cmp_sel_mha", B=2, T=1999, Hq=4, Hkv=4, topk=6,
+                         branch_mask=W.BR_CMP | W.BR_SEL),
 ], ids=lambda w: w.name)
 def test_decode_small(cuda_lib, w):
     inp = W.make_decode_inputs(w, seed=13)
