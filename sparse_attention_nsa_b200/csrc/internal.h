@@ -35,6 +35,13 @@ cudaError_t launch_sel_fwd(const Dims& d, const void* q, const void* k,
                            float* lse, int* err, cudaStream_t s);
 cudaError_t launch_swa_fwd(const Dims& d, const void* q, const void* k,
                            const void* v, void* o, float* lse, cudaStream_t s);
+// window branch with the gated combination fused into its epilogue (bf16
+// tensor-core path); o_swa may be NULL (not stored)
+bool swa_combine_fusable(const Dims& d);
+cudaError_t launch_swa_fwd_combine(const Dims& d, const void* q, const void* k, const void* v,
+                                   void* o_swa, float* lse_swa, const float* gates,
+                                   const void* o_cmp, const void* o_sel, void* out,
+                                   cudaStream_t s);
 cudaError_t launch_combine(const Dims& d, const float* gates, const void* o_cmp,
                            const void* o_sel, const void* o_swa, void* out,
                            cudaStream_t s);

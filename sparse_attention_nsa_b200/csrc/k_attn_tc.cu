@@ -76,11 +76,23 @@ __host__ __device__ inline size_t list_ints(const Dims& d) {
   return (size_t)d.Nb + words + (size_t)tokens_per_tile(d.G) * (d.topk + 1);
 }
 
-template <bool SEL>
+// Gated combination fused into the window branch's epilogue (the last
+// branch of a forward): out = g_cmp o_cmp + g_sel o_sel + g_swa o_swa over
+// the enabled branches, with o_swa unrounded; o_swa itself is stored only
+// when `o` is not null.
+struct Fuse {
+  const float* gates;
+  const bf16* o_cmp;
+  const bf16* o_sel;
+  bf16* out;
+};
+
+template <bool SEL, bool FUSE>
 __global__ void __launch_bounds__(kThreads, 2)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, bf16* __restrict__ o,
-               float* __restrict__ lse, const int32_t* __restrict__ idx, Dims d, int* err) {
+               float* __restrict__ lse, const int32_t* __restrict__ idx, Dims d, int* err,
+               Fuse fz) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   Bars* bars = (Bars*)(smem + OFF_BAR);
@@ -264,6 +276,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const int lo = SEL ? 0 : max(0, t - d.window + 1);  // first key of the row
     const int* lst = SEL ? toks + tl * (d.topk + 1) : nullptr;
     int ptr = 0;
+    int nxt = SEL && valid ? lst[0] : INT_MAX;  // next block this row selected
     float mref = -INFINITY, lsum = 0.f;
     const float sl2 = d.scale * kLog2e;
     const uint32_t lane_tmem = tmem + ((uint32_t)(warp * 32) << 16);
@@ -274,12 +287,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       const int k0 = j * kKeys;
       bool rowsel = valid && k0 <= t;
       if (SEL) {
-        if (valid) {
-          while (lst[ptr] < j) ++ptr;
-          const bool hit = lst[ptr] == j;
-          if (hit) ++ptr;
-          rowsel = rowsel && hit;
-        }
+        // the union list is ascending and contains every block of the row's
+        // list, so the row's next selected block is never below j
+        const bool hit = nxt == j;
+        if (hit) nxt = lst[++ptr];  // consumed only at the next hit
+        rowsel = rowsel && hit;
       } else {
         rowsel = rowsel && (k0 + kKeys - 1 >= lo);
       }
@@ -389,15 +401,52 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
       const int h = g * d.G + hh;
       const size_t row = ((size_t)b * d.Tq + t0 + tl) * d.Hq + h;
-      uint4* dst = reinterpret_cast<uint4*>(o + row * 64);
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint4 u;
-        u.x = pack_bf16(acc[8 * c + 0] * inv, acc[8 * c + 1] * inv);
-        u.y = pack_bf16(acc[8 * c + 2] * inv, acc[8 * c + 3] * inv);
-        u.z = pack_bf16(acc[8 * c + 4] * inv, acc[8 * c + 5] * inv);
-        u.w = pack_bf16(acc[8 * c + 6] * inv, acc[8 * c + 7] * inv);
-        dst[c] = u;
+      for (int c = 0; c < 64; ++c) acc[c] *= inv;
+      if (o) {
+        uint4* dst = reinterpret_cast<uint4*>(o + row * 64);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint4 u;
+          u.x = pack_bf16(acc[8 * c + 0], acc[8 * c + 1]);
+          u.y = pack_bf16(acc[8 * c + 2], acc[8 * c + 3]);
+          u.z = pack_bf16(acc[8 * c + 4], acc[8 * c + 5]);
+          u.w = pack_bf16(acc[8 * c + 6], acc[8 * c + 7]);
+          dst[c] = u;
+        }
+      }
+      if (FUSE) {
+        const float gw = fz.gates[row * 3 + 2];
+#pragma unroll
+        for (int c = 0; c < 64; ++c) acc[c] *= gw;
+        const bf16* srcs[2] = {fz.o_cmp, fz.o_sel};
+#pragma unroll
+        for (int br = 0; br < 2; ++br) {
+          if (!srcs[br]) continue;
+          const float gb = fz.gates[row * 3 + br];
+          const uint4* src = reinterpret_cast<const uint4*>(srcs[br] + row * 64);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint4 u = src[c];
+            const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __bfloat1622float2(pb[e]);
+              acc[8 * c + 2 * e] = fmaf(gb, f.x, acc[8 * c + 2 * e]);
+              acc[8 * c + 2 * e + 1] = fmaf(gb, f.y, acc[8 * c + 2 * e + 1]);
+            }
+          }
+        }
+        uint4* dst = reinterpret_cast<uint4*>(fz.out + row * 64);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint4 u;
+          u.x = pack_bf16(acc[8 * c + 0], acc[8 * c + 1]);
+          u.y = pack_bf16(acc[8 * c + 2], acc[8 * c + 3]);
+          u.z = pack_bf16(acc[8 * c + 4], acc[8 * c + 5]);
+          u.w = pack_bf16(acc[8 * c + 6], acc[8 * c + 7]);
+          dst[c] = u;
+        }
       }
       if (lse) lse[row] = lsum > 0.f ? (mref + log2f(lsum)) * kLn2 : -INFINITY;
     }
@@ -415,9 +464,10 @@ bool tc_eligible(const Dims& d) {
          d.Nb <= 4096 && tmap_encode_fn() != nullptr;
 }
 
-template <bool SEL>
+template <bool SEL, bool FUSE>
 cudaError_t launch_tc(const Dims& d, const void* q, const void* k, const void* v,
-                      const int32_t* idx, void* o, float* lse, int* err, cudaStream_t s) {
+                      const int32_t* idx, void* o, float* lse, int* err, const Fuse& fz,
+                      cudaStream_t s) {
   const int TQ = tokens_per_tile(d.G);
   CUtensorMap mq, mk, mv;
   if (!make_tmap_bf16(&mq, q, d.Hq, (long)d.B * d.Tq, d.G, TQ) ||
@@ -425,11 +475,12 @@ cudaError_t launch_tc(const Dims& d, const void* q, const void* k, const void* v
       !make_tmap_bf16(&mv, v, d.Hkv, (long)d.B * d.T, 1, kKeys))
     return cudaErrorInvalidValue;
   const size_t smem = OFF_LIST + list_ints(d) * sizeof(int) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<SEL>,
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<SEL, FUSE>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((d.Tq + TQ - 1) / TQ, d.Hkv, d.B);
-  attn_tc_kernel<SEL><<<grid, kThreads, smem, s>>>(mq, mk, mv, (bf16*)o, lse, idx, d, err);
+  attn_tc_kernel<SEL, FUSE><<<grid, kThreads, smem, s>>>(mq, mk, mv, (bf16*)o, lse, idx, d, err,
+                                                        fz);
   return cudaGetLastError();
 }
 
@@ -438,14 +489,25 @@ cudaError_t launch_tc(const Dims& d, const void* q, const void* k, const void* v
 cudaError_t launch_sel_fwd(const Dims& d, const void* q, const void* k, const void* v,
                            const int32_t* idx, void* o, float* lse, int* err,
                            cudaStream_t s) {
-  if (tc_eligible(d)) return launch_tc<true>(d, q, k, v, idx, o, lse, err, s);
+  if (tc_eligible(d)) return launch_tc<true, false>(d, q, k, v, idx, o, lse, err, Fuse{}, s);
   return launch_sel_fwd_simt(d, q, k, v, idx, o, lse, err, s);
 }
 
 cudaError_t launch_swa_fwd(const Dims& d, const void* q, const void* k, const void* v,
                            void* o, float* lse, cudaStream_t s) {
-  if (tc_eligible(d)) return launch_tc<false>(d, q, k, v, nullptr, o, lse, nullptr, s);
+  if (tc_eligible(d)) return launch_tc<false, false>(d, q, k, v, nullptr, o, lse, nullptr, Fuse{}, s);
   return launch_swa_fwd_simt(d, q, k, v, o, lse, s);
+}
+
+bool swa_combine_fusable(const Dims& d) { return tc_eligible(d); }
+
+cudaError_t launch_swa_fwd_combine(const Dims& d, const void* q, const void* k, const void* v,
+                                   void* o_swa, float* lse_swa, const float* gates,
+                                   const void* o_cmp, const void* o_sel, void* out,
+                                   cudaStream_t s) {
+  Fuse fz{gates, (d.branch_mask & 1) ? (const bf16*)o_cmp : nullptr,
+          (d.branch_mask & 2) ? (const bf16*)o_sel : nullptr, (bf16*)out};
+  return launch_tc<false, true>(d, q, k, v, nullptr, o_swa, lse_swa, nullptr, fz, s);
 }
 
 }  // namespace nsa

@@ -120,6 +120,19 @@ __device__ __forceinline__ void pv_tile(float o[8][4], const float p[8][4], uint
   }
 }
 
+// Programmatic dependent launch: the next kernel in the stream may start its
+// prologue early; it waits for this grid's completion (and memory) with
+// griddepcontrol.wait before touching this grid's outputs.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// (score desc, block asc): does (va, ia) come before (vb, ib)?
+__device__ __forceinline__ bool goes_first(float va, int ia, float vb, int ib) {
+  return va > vb || (va == vb && ia < ib);
+}
+
 __device__ __forceinline__ float quad_max(float x) {
   x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 1));
   return fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 2));
@@ -176,6 +189,7 @@ decode_cmp_topk_kernel(const __grid_constant__ CUtensorMap tm_kc,
     fence_barrier_init();
     *abort_flag = 0;
   }
+  pdl_launch_dependents();
   __syncthreads();
   if (threadIdx.x == 0 && nchunks > 0) {
     mbar_expect_tx(&bar[0], (uint32_t)nchunks * 8192u);
@@ -307,56 +321,99 @@ decode_cmp_topk_kernel(const __grid_constant__ CUtensorMap tm_kc,
   } else {
     __syncthreads();
   }
-  // top-k over blocks 1..cur-1 (forced: 0 and cur): the whole CTA sorts the
-  // candidates by (score desc, block asc) with a bitonic network, and the
-  // first topk - 2 win.
+  // top-k over blocks 1..cur-1 (forced: 0 and cur).  Each warp sorts the
+  // candidates among its 64 blocks by (score desc, block asc) with a bitonic
+  // network in registers and shuffles; warp 0 then merges the eight sorted
+  // lists, taking the best head topk - 2 times.
   if (need_idx) {
     int* out = ws.idx + (size_t)bg * d.topk;
     int32_t* out2 = idx_out ? idx_out + (size_t)bg * d.topk : nullptr;
     const int cur = t / d.l;
+    const int K2 = d.topk - 2;
     if (cur + 1 <= d.topk) {
       for (int k = threadIdx.x; k < d.topk; k += kK1Threads) {
         out[k] = k <= cur ? k : -1;
         if (out2) out2[k] = out[k];
       }
     } else {
-      const int ncand = cur - 1;  // blocks 1 .. cur-1, at most 510
-      int n2 = 1;
-      while (n2 < ncand) n2 <<= 1;
-      for (int e = threadIdx.x; e < n2; e += kK1Threads) {
-        const bool c = e < ncand;
-        sort_v[e] = c ? score[e + 1] : -INFINITY;
-        sort_i[e] = c ? e + 1 : INT_MAX;
+      float v[2];
+      int ix[2];
+#pragma unroll
+      for (int sl = 0; sl < 2; ++sl) {
+        const int j = key0 + lane + 32 * sl;
+        const bool c = j >= 1 && j < cur && j < ncp;
+        v[sl] = c ? score[j] : -INFINITY;
+        ix[sl] = c ? j : INT_MAX;
       }
-      __syncthreads();
-      // "a goes first" = larger score, or equal score and lower block
-      for (int size = 2; size <= n2; size <<= 1) {
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-          for (int e = threadIdx.x; e < n2; e += kK1Threads) {
-            const int p = e ^ stride;
-            if (p > e) {
-              const float va = sort_v[e], vb = sort_v[p];
-              const int ia = sort_i[e], ib = sort_i[p];
-              const bool a_first = va > vb || (va == vb && ia < ib);
-              const bool want_a_first = (e & size) == 0;
-              if (a_first != want_a_first) {
-                sort_v[e] = vb;
-                sort_v[p] = va;
-                sort_i[e] = ib;
-                sort_i[p] = ia;
+      for (int size = 2; size <= 64; size <<= 1) {
+        for (int jj = size >> 1; jj > 0; jj >>= 1) {
+          if (jj == 32) {  // the pair is held by one lane: (lane, lane + 32)
+            const bool dir = (lane & size) == 0;
+            const bool f = goes_first(v[0], ix[0], v[1], ix[1]);
+            if (f != dir) {
+              const float tv = v[0];
+              const int ti = ix[0];
+              v[0] = v[1];
+              ix[0] = ix[1];
+              v[1] = tv;
+              ix[1] = ti;
+            }
+          } else {
+#pragma unroll
+            for (int sl = 0; sl < 2; ++sl) {
+              const int e = lane + 32 * sl;
+              const float pv = __shfl_xor_sync(0xffffffffu, v[sl], jj);
+              const int pi = __shfl_xor_sync(0xffffffffu, ix[sl], jj);
+              const bool lower = (e & jj) == 0;
+              const bool dir = (e & size) == 0;
+              const bool self_first = goes_first(v[sl], ix[sl], pv, pi);
+              const bool keep = lower ? (dir == self_first) : (dir != self_first);
+              if (!keep) {
+                v[sl] = pv;
+                ix[sl] = pi;
               }
             }
           }
-          __syncthreads();
         }
       }
+      float* cand_v = sort_v + warp * 64;
+      int* cand_i = sort_i + warp * 64;
+      cand_v[lane] = v[0];
+      cand_i[lane] = ix[0];
+      cand_v[lane + 32] = v[1];
+      cand_i[lane + 32] = ix[1];
+      __syncthreads();
       if (warp == 0) {
         const int words = (d.Nb + 31) / 32;
         for (int w = lane; w < words; w += 32) bits[w] = 0u;
         __syncwarp();
-        for (int k = lane; k < d.topk - 2; k += 32) {
-          const int j = sort_i[k];
-          if (j != INT_MAX) atomicOr(&bits[j >> 5], 1u << (j & 31));
+        int head = 0;  // lanes 0..7: position in warp `lane`'s sorted list
+        for (int k = 0; k < K2; ++k) {
+          float hv = -INFINITY;
+          int hi = INT_MAX;
+          if (lane < 8 && head < 64) {
+            hv = sort_v[lane * 64 + head];
+            hi = sort_i[lane * 64 + head];
+          }
+          float wv = hv;
+          int wi = hi, wl = lane;
+#pragma unroll
+          for (int off = 4; off > 0; off >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, wv, off);
+            const int oi = __shfl_xor_sync(0xffffffffu, wi, off);
+            const int ol = __shfl_xor_sync(0xffffffffu, wl, off);
+            if (goes_first(ov, oi, wv, wi)) {
+              wv = ov;
+              wi = oi;
+              wl = ol;
+            }
+          }
+          wv = __shfl_sync(0xffffffffu, wv, 0);
+          wi = __shfl_sync(0xffffffffu, wi, 0);
+          wl = __shfl_sync(0xffffffffu, wl, 0);
+          if (wi == INT_MAX) break;
+          if (lane == wl) ++head;
+          if (lane == 0) bits[wi >> 5] |= 1u << (wi & 31);
         }
         __syncwarp();
         if (lane == 0) {
@@ -412,18 +469,18 @@ decode_block_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
   const int t = d.T - 1;
   const int cur = t / d.l;
   const int* sel = ws.idx + (size_t)bg * d.topk;
-  // which block, and which branches it serves here
+  pdl_launch_dependents();
+  // which block, and which branches it serves here; window blocks are known
+  // before the selection, so their loads start before K1 has finished
   int j, sel_slot = -1;
   bool win = false;
   if (u < ws.nwin) {
     if (!do_swa) return;
     j = ws.jlo + u;
     win = true;
-    if (do_sel)
-      for (int m = 0; m < d.topk; ++m)
-        if (sel[m] == j) sel_slot = m;
   } else {
     if (!do_sel) return;
+    pdl_wait();
     const int m = u - ws.nwin;
     j = sel[m];
     if (j < 0) return;
@@ -446,6 +503,11 @@ decode_block_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     tma_load_3d(kv + 8192, &tm_v, &bar, 0, g, b * d.T + j * 64);
   }
   stage_q(qs, q + ((size_t)b * d.Hq + (size_t)g * d.G) * 64, d.G, lane);
+  if (win && do_sel) {  // is this window block also selected?
+    pdl_wait();
+    for (int m = 0; m < d.topk; ++m)
+      if (sel[m] == j) sel_slot = m;
+  }
   fence_proxy_async_smem();
   __syncwarp();
   uint32_t qa[4][4];
@@ -520,6 +582,7 @@ __global__ void decode_merge_kernel(const float* __restrict__ gates, bf16* __res
                                     Dims d, DecodeWs ws) {
   const int bg = blockIdx.x;
   const int row = threadIdx.x >> 5, lane = threadIdx.x & 31;  // one warp per head
+  pdl_wait();
   if (row >= d.G) return;
   const int b = bg / d.Hkv, g = bg % d.Hkv;
   const int h = g * d.G + row;
@@ -552,13 +615,16 @@ __global__ void decode_merge_kernel(const float* __restrict__ gates, bf16* __res
         L += f * base[(size_t)m * 16 * kPartStride + 65];
       }
       const int cnt = min(32, n - m0);
+      // loads of every slot are issued together (all addresses are inside
+      // the workspace); slots without a partial get weight 0 and their
+      // (possibly stale) values are discarded by the select
+#pragma unroll 8
       for (int i = 0; i < cnt; ++i) {
         const float fi = __shfl_sync(0xffffffffu, f, i);
-        if (fi != 0.f) {
-          const float* pr = base + (size_t)(m0 + i) * 16 * kPartStride;
-          o0 = fmaf(fi, pr[lane], o0);
-          o1 = fmaf(fi, pr[lane + 32], o1);
-        }
+        const float* pr = base + (size_t)(m0 + i) * 16 * kPartStride;
+        const float x0 = pr[lane], x1 = pr[lane + 32];
+        o0 = fi != 0.f ? fmaf(fi, x0, o0) : o0;
+        o1 = fi != 0.f ? fmaf(fi, x1, o1) : o1;
       }
     }
     L = warp_sum(L);
@@ -643,15 +709,29 @@ cudaError_t launch_decode_split(const Dims& d, const void* q, const void* kcache
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
   if (sel || swa) {
-    dim3 grid(ws.nwin + d.topk, d.Hkv, d.B);
-    decode_block_kernel<<<grid, 32, 0, s>>>(mk, mv, (const bf16*)q, d, ws, sel ? 1 : 0,
-                                             swa ? 1 : 0, err);
-    cudaError_t e = cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(ws.nwin + d.topk, d.Hkv, d.B);
+    cfg.blockDim = dim3(32);
+    cfg.stream = s;
+    cfg.attrs = pdl;
+    cfg.numAttrs = 1;
+    const bf16* qb = (const bf16*)q;
+    const int ds = sel ? 1 : 0, dw = swa ? 1 : 0;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, decode_block_kernel, mk, mv, qb, d, ws, ds, dw, err);
     if (e != cudaSuccess) return e;
   }
-  decode_merge_kernel<<<(unsigned)bgn, d.G * 32, 0, s>>>(gates, (bf16*)out, d, ws);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)bgn);
+  cfg.blockDim = dim3(d.G * 32);
+  cfg.stream = s;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  bf16* ob = (bf16*)out;
+  return cudaLaunchKernelEx(&cfg, decode_merge_kernel, gates, ob, d, ws);
 }
 
 }  // namespace nsa

@@ -299,6 +299,13 @@ static nsa_status run_forward(const Dims& d, const void* q, const void* k, const
     NSA_TRY_CUDA(nsa::launch_topk(d, score, idx, s));
     NSA_TRY_CUDA(nsa::launch_sel_fwd(d, q, k, v, idx, o_sel, lse_sel, err_word(), s));
   }
+  if (swa && nsa::swa_combine_fusable(d)) {
+    // the window branch runs last and writes `out` itself; its own output
+    // and lse are stored only when the caller asked for them
+    NSA_TRY_CUDA(nsa::launch_swa_fwd_combine(d, q, k, v, S.o_swa, S.lse_swa, gates, o_cmp, o_sel,
+                                             out, s));
+    return NSA_OK;
+  }
   if (swa) NSA_TRY_CUDA(nsa::launch_swa_fwd(d, q, k, v, o_swa, lse_swa, s));
   NSA_TRY_CUDA(nsa::launch_combine(d, gates, o_cmp, o_sel, o_swa, out, s));
   return NSA_OK;
