@@ -181,12 +181,19 @@ def barrier_sync(dist_on):
     torch.cuda.synchronize()
 
 
-def max_over_ranks(x: float, dist_on: bool) -> float:
+def max_over_ranks(x: float, dist_on: bool, device: str = "cuda") -> float:
+    """Job time = the slowest rank's time (all ranks must call this)."""
     if not dist_on:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_tokens_per_s(tokens_per_rank_step: int, world: int, job_ms: float) -> float:
+    """Weak scaling: every rank processes its own copy of the workload, so
+    the job processes world x tokens per step in the slowest rank's time."""
+    return tokens_per_rank_step * world / (job_ms * 1e-3)
 
 
 # ------------------------------------------------------------------ CPU oracle leg
@@ -280,7 +287,7 @@ def run_gpu(args, rank: int, world: int, dist_on: bool) -> None:
     ms = max_over_ranks(sum(times) / len(times), dist_on)
     flops = fwd_flops(w)
     tokens_per_step = w.B * w.T
-    value = tokens_per_step * world / (ms * 1e-3)
+    value = job_tokens_per_s(tokens_per_step, world, ms)
 
     # dominant kernel alone (selection branch), same inputs, same flushing
     o_sel = torch.empty_like(q)
@@ -341,7 +348,7 @@ def run_gpu(args, rank: int, world: int, dist_on: bool) -> None:
                      "ms_per_launch": sel_ms, "peak_source": peaks["source"] + " burst bf16"},
         "decode": dec,
         "train": train,
-        "e2e": {"value": tokens_per_step * world / (e2e_ms * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": job_tokens_per_s(tokens_per_step, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": KERNELS_PER_FORWARD * args.steps,
         "clocks": clocks,
