@@ -42,6 +42,12 @@ cudaError_t launch_swa_fwd_combine(const Dims& d, const void* q, const void* k, 
                                    void* o_swa, float* lse_swa, const float* gates,
                                    const void* o_cmp, const void* o_sel, void* out,
                                    cudaStream_t s);
+// selection branch with the gated combination fused into its epilogue;
+// o_sel may be NULL (not stored)
+cudaError_t launch_sel_fwd_combine(const Dims& d, const void* q, const void* k, const void* v,
+                                   const int32_t* idx, void* o_sel, float* lse_sel, int* err,
+                                   const float* gates, const void* o_cmp, const void* o_swa,
+                                   void* out, cudaStream_t s);
 cudaError_t launch_combine(const Dims& d, const float* gates, const void* o_cmp,
                            const void* o_sel, const void* o_swa, void* out,
                            cudaStream_t s);

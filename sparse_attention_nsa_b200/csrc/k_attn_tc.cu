@@ -76,14 +76,16 @@ __host__ __device__ inline size_t list_ints(const Dims& d) {
   return (size_t)d.Nb + words + (size_t)tokens_per_tile(d.G) * (d.topk + 1);
 }
 
-// Gated combination fused into the window branch's epilogue (the last
-// branch of a forward): out = g_cmp o_cmp + g_sel o_sel + g_swa o_swa over
-// the enabled branches, with o_swa unrounded; o_swa itself is stored only
-// when `o` is not null.
+// Gated combination fused into the epilogue of the branch that runs last
+// in a forward: out = g_own o_own + sum of g_i o_i over the other enabled
+// branches (stored bf16 outputs), with o_own unrounded; o_own itself is
+// stored only when `o` is not null.  Gate i is gates[row * 3 + i] in the
+// order (cmp, sel, swa).
 struct Fuse {
   const float* gates;
-  const bf16* o_cmp;
-  const bf16* o_sel;
+  const bf16* other[2];  // NULL when that branch is disabled
+  int other_gate[2];
+  int own_gate;
   bf16* out;
 };
 
@@ -416,15 +418,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
       }
       if (FUSE) {
-        const float gw = fz.gates[row * 3 + 2];
+        const float gw = fz.gates[row * 3 + fz.own_gate];
 #pragma unroll
         for (int c = 0; c < 64; ++c) acc[c] *= gw;
-        const bf16* srcs[2] = {fz.o_cmp, fz.o_sel};
 #pragma unroll
         for (int br = 0; br < 2; ++br) {
-          if (!srcs[br]) continue;
-          const float gb = fz.gates[row * 3 + br];
-          const uint4* src = reinterpret_cast<const uint4*>(srcs[br] + row * 64);
+          if (!fz.other[br]) continue;
+          const float gb = fz.gates[row * 3 + fz.other_gate[br]];
+          const uint4* src = reinterpret_cast<const uint4*>(fz.other[br] + row * 64);
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             const uint4 u = src[c];
@@ -505,9 +506,26 @@ cudaError_t launch_swa_fwd_combine(const Dims& d, const void* q, const void* k, 
                                    void* o_swa, float* lse_swa, const float* gates,
                                    const void* o_cmp, const void* o_sel, void* out,
                                    cudaStream_t s) {
-  Fuse fz{gates, (d.branch_mask & 1) ? (const bf16*)o_cmp : nullptr,
-          (d.branch_mask & 2) ? (const bf16*)o_sel : nullptr, (bf16*)out};
+  Fuse fz{gates,
+          {(d.branch_mask & 1) ? (const bf16*)o_cmp : nullptr,
+           (d.branch_mask & 2) ? (const bf16*)o_sel : nullptr},
+          {0, 1},
+          2,
+          (bf16*)out};
   return launch_tc<false, true>(d, q, k, v, nullptr, o_swa, lse_swa, nullptr, fz, s);
+}
+
+cudaError_t launch_sel_fwd_combine(const Dims& d, const void* q, const void* k, const void* v,
+                                   const int32_t* idx, void* o_sel, float* lse_sel, int* err,
+                                   const float* gates, const void* o_cmp, const void* o_swa,
+                                   void* out, cudaStream_t s) {
+  Fuse fz{gates,
+          {(d.branch_mask & 1) ? (const bf16*)o_cmp : nullptr,
+           (d.branch_mask & 4) ? (const bf16*)o_swa : nullptr},
+          {0, 2},
+          1,
+          (bf16*)out};
+  return launch_tc<true, true>(d, q, k, v, idx, o_sel, lse_sel, err, fz, s);
 }
 
 }  // namespace nsa

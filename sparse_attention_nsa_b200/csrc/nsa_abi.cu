@@ -262,6 +262,29 @@ nsa_status nsa_gate_combine(const nsa_params* p, const float* gates, const void*
   return NSA_OK;
 }
 
+// Library-owned side stream per device for running the window branch
+// concurrently with compression -> top-k -> selection inside one forward.
+// Created on first use (with that device current) and kept until exit.
+struct SideStream {
+  cudaStream_t s2 = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+static std::mutex g_side_mu;  // also held across each fork ... join enqueue
+static SideStream g_side[64];
+
+static SideStream* side_stream_locked() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  SideStream& ss = g_side[dev];
+  if (!ss.s2) {
+    if (cudaStreamCreateWithFlags(&ss.s2, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    if (cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess)
+      return nullptr;
+  }
+  return &ss;
+}
+
 // Shared body of nsa_forward and nsa_decode.  kc_given means the compressed
 // tensors in sv->kc / sv->vc are inputs (decode) and compression is skipped.
 static nsa_status run_forward(const Dims& d, const void* q, const void* k, const void* v,
@@ -290,6 +313,34 @@ static nsa_status run_forward(const Dims& d, const void* q, const void* k, const
   const bool cmp = d.branch_mask & NSA_BRANCH_CMP;
   const bool sel = d.branch_mask & NSA_BRANCH_SEL;
   const bool swa = d.branch_mask & NSA_BRANCH_SWA;
+  if (sel && swa && nsa::swa_combine_fusable(d)) {
+    // The window branch does not depend on compression, top-k or selection:
+    // it runs on the side stream while those run here, and the selection
+    // kernel, last on this stream, applies the gates in its epilogue.
+    std::lock_guard<std::mutex> lock(g_side_mu);
+    SideStream* ss = side_stream_locked();
+    if (ss) {
+      if (cudaEventRecord(ss->fork, s) != cudaSuccess ||
+          cudaStreamWaitEvent(ss->s2, ss->fork, 0) != cudaSuccess)
+        return NSA_ERR_CUDA;
+      const cudaError_t ew = nsa::launch_swa_fwd(d, q, k, v, o_swa, S.lse_swa, ss->s2);
+      // the join is enqueued whatever happens, so no side-stream work can
+      // outlive this call's ordering on the caller's stream
+      const cudaError_t ej = cudaEventRecord(ss->join, ss->s2);
+      cudaError_t em = cudaSuccess;
+      if (!kc_given) em = nsa::launch_compress(d, k, v, kc, vc, s);
+      if (em == cudaSuccess)
+        em = nsa::launch_cmp_scores(d, q, kc, vc, cmp ? o_cmp : nullptr, cmp ? lse_cmp : nullptr,
+                                    score, err_word(), s);
+      if (em == cudaSuccess) em = nsa::launch_topk(d, score, idx, s);
+      const cudaError_t ewait = cudaStreamWaitEvent(s, ss->join, 0);
+      if (ew != cudaSuccess || ej != cudaSuccess || em != cudaSuccess || ewait != cudaSuccess)
+        return NSA_ERR_CUDA;
+      NSA_TRY_CUDA(nsa::launch_sel_fwd_combine(d, q, k, v, idx, S.o_sel, S.lse_sel, err_word(),
+                                               gates, o_cmp, o_swa, out, s));
+      return NSA_OK;
+    }
+  }
   if (cmp || sel) {
     if (!kc_given) NSA_TRY_CUDA(nsa::launch_compress(d, k, v, kc, vc, s));
     NSA_TRY_CUDA(nsa::launch_cmp_scores(d, q, kc, vc, cmp ? o_cmp : nullptr,
