@@ -9,12 +9,13 @@
 // 1..cur-1 are added, equal scores going to the lower block index.  The
 // output is ascending and padded with -1.
 //
-// One warp per row.  The row's candidate scores are staged in shared
-// memory; each lane keeps the best of its own candidates (blocks
-// 1 + lane + 32q), each of the topk - 2 rounds is a warp arg-max over those
-// lane bests ordered by (score desc, index asc), and only the winning lane
-// rescans its candidates.  A per-warp bitmap records the winners and the
-// ascending list is read back from it.
+// One warp per row, no shared memory.  Lane `lane` holds the candidates
+// 1 + lane + 32 q in registers as order-preserving integer keys.  A radix
+// select finds tau, the (topk-2)-th largest key, bit by bit from the top
+// (each step one warp-wide count with redux.sync).  The winners are every
+// key above tau plus, among keys equal to tau, the lowest block indices
+// (ballots in ascending block order); they are written out in ascending
+// order between the forced blocks 0 and cur.
 #include "common.cuh"
 #include "internal.h"
 
@@ -22,30 +23,17 @@ namespace nsa {
 
 constexpr int kTopkWarps = 8;
 
-// Best not-yet-taken candidate of this lane: blocks 1 + lane + 32 q, q < 32,
-// below cur, ordered by (score desc, index asc).
-__device__ __forceinline__ void lane_best(const float* row, int cur, int lane, uint32_t taken,
-                                          float& bv, int& bj) {
-  bv = -INFINITY;
-  bj = 0x7fffffff;
-  for (int q = 0; q < 32; ++q) {
-    const int j = 1 + lane + 32 * q;
-    if (j >= cur) break;
-    if ((taken >> q) & 1u) continue;
-    const float v = row[j];
-    if (v > bv || (v == bv && j < bj)) {
-      bv = v;
-      bj = j;
-    }
-  }
+// Monotone map of a float to uint32 (larger float -> larger key); NaN -> 0.
+__device__ __forceinline__ uint32_t order_key(float x) {
+  if (x != x) return 0u;
+  const uint32_t u = __float_as_uint(x);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+template <int QMAX>
 __global__ void __launch_bounds__(kTopkWarps * 32)
-topk_kernel(const float* __restrict__ score, int32_t* __restrict__ idx, Dims d, int words) {
-  extern __shared__ uint32_t sm_all[];
+topk_kernel(const float* __restrict__ score, int32_t* __restrict__ idx, Dims d) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float* row = reinterpret_cast<float*>(sm_all) + (size_t)warp * (d.Nc + words);
-  uint32_t* bits = reinterpret_cast<uint32_t*>(row + d.Nc);
   const long r = (long)blockIdx.x * kTopkWarps + warp;
   const long nrows = (long)d.B * d.Tq * d.Hkv;
   if (r >= nrows) return;
@@ -59,70 +47,56 @@ topk_kernel(const float* __restrict__ score, int32_t* __restrict__ idx, Dims d, 
   }
   // candidates are blocks 1..cur-1 (all complete, so all have scores)
   const float* sr = score + r * d.Nc;
-  for (int j = lane; j < cur; j += 32) row[j] = sr[j];
-  for (int w = lane; w < words; w += 32) bits[w] = 0u;
-  __syncwarp();
-  uint32_t taken = 0;
-  float bv;
-  int bj;
-  lane_best(row, cur, lane, taken, bv, bj);
-  for (int k = 0; k < d.topk - 2; ++k) {
-    float wv = bv;
-    int wj = bj;
+  uint32_t key[QMAX];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, wv, o);
-      const int oj = __shfl_xor_sync(0xffffffffu, wj, o);
-      if (ov > wv || (ov == wv && oj < wj)) {
-        wv = ov;
-        wj = oj;
-      }
-    }
-    if (wj == 0x7fffffff) break;  // only NaN scores left
-    if (lane == ((wj - 1) & 31)) {
-      taken |= 1u << ((wj - 1) >> 5);
-      lane_best(row, cur, lane, taken, bv, bj);
-    }
-    if (lane == 0) bits[wj >> 5] |= 1u << (wj & 31);
+  for (int q = 0; q < QMAX; ++q) {
+    const int j = 1 + lane + 32 * q;
+    key[q] = j < cur ? order_key(__ldg(sr + j)) : 0u;
   }
-  __syncwarp();
+  const int K2 = d.topk - 2;
+  // tau = the largest value with at least K2 keys >= tau (absent slots are
+  // excluded from the counts)
+  uint32_t tau = 0u;
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t tc = tau | (1u << bit);
+    unsigned c = 0;
+#pragma unroll
+    for (int q = 0; q < QMAX; ++q) c += (1 + lane + 32 * q < cur && key[q] >= tc) ? 1u : 0u;
+    if ((int)__reduce_add_sync(0xffffffffu, c) >= K2) tau = tc;
+  }
+  unsigned cg = 0;
+#pragma unroll
+  for (int q = 0; q < QMAX; ++q) cg += (1 + lane + 32 * q < cur && key[q] > tau) ? 1u : 0u;
+  const int need = K2 - (int)__reduce_add_sync(0xffffffffu, cg);  // >= 1 keys equal to tau
+  int eq_before = 0, pos = 1;
+  const unsigned lt = (1u << lane) - 1u;
+#pragma unroll
+  for (int q = 0; q < QMAX; ++q) {
+    const int j = 1 + lane + 32 * q;
+    const bool ok = j < cur;
+    const bool eq = ok && key[q] == tau;
+    const unsigned em = __ballot_sync(0xffffffffu, eq);
+    const bool win = ok && (key[q] > tau || (eq && eq_before + __popc(em & lt) < need));
+    const unsigned wm = __ballot_sync(0xffffffffu, win);
+    if (win) out[pos + __popc(wm & lt)] = j;
+    pos += __popc(wm);
+    eq_before += __popc(em);
+  }
   if (lane == 0) {
-    bits[0] |= 1u;
-    bits[cur >> 5] |= 1u << (cur & 31);
+    out[0] = 0;
+    out[K2 + 1] = cur;
   }
-  __syncwarp();
-  // ascending write-out: lanes own 32-block words, prefix count over lanes
-  int base = 0;
-  for (int w0 = 0; w0 <= (cur >> 5); w0 += 32) {
-    const int w = w0 + lane;
-    const uint32_t m = w <= (cur >> 5) ? bits[w] : 0u;
-    const int c = __popc(m);
-    int incl = c;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    int pos = base + incl - c;
-    uint32_t mm = m;
-    while (mm) {
-      const int bit = __ffs(mm) - 1;
-      mm &= mm - 1;
-      if (pos < d.topk) out[pos] = w * 32 + bit;
-      ++pos;
-    }
-    base += __shfl_sync(0xffffffffu, incl, 31);
-  }
-  for (int p = base + lane; p < d.topk; p += 32) out[p] = -1;
 }
 
 cudaError_t launch_topk(const Dims& d, const float* score, int32_t* idx,
                         cudaStream_t s) {
   const long nrows = (long)d.B * d.Tq * d.Hkv;
-  const int words = (d.Nb + 31) / 32;
-  const size_t smem = (size_t)kTopkWarps * (d.Nc + words) * sizeof(uint32_t);
-  const long blocks = (nrows + kTopkWarps - 1) / kTopkWarps;
-  topk_kernel<<<(unsigned)blocks, kTopkWarps * 32, smem, s>>>(score, idx, d, words);
+  const unsigned blocks = (unsigned)((nrows + kTopkWarps - 1) / kTopkWarps);
+  const int q = (d.Nb + 31) / 32;  // candidate slots per lane
+  if (q <= 4) topk_kernel<4><<<blocks, kTopkWarps * 32, 0, s>>>(score, idx, d);
+  else if (q <= 8) topk_kernel<8><<<blocks, kTopkWarps * 32, 0, s>>>(score, idx, d);
+  else if (q <= 16) topk_kernel<16><<<blocks, kTopkWarps * 32, 0, s>>>(score, idx, d);
+  else topk_kernel<32><<<blocks, kTopkWarps * 32, 0, s>>>(score, idx, d);
   return cudaGetLastError();
 }
 
