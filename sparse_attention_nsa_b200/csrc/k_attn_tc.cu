@@ -17,14 +17,24 @@
 //
 // Per block:  S = Q K^T   (tcgen05, M=128 N=64 K=64, into TMEM)
 //             softmax rows in fp32 (one thread per row, exp2 on MUFU)
-//             P (bf16, swizzled smem) ;  O += P V  (tcgen05, accumulated in TMEM)
+//             P (bf16, into TMEM) ;  O += P V  (tcgen05, accumulated in TMEM)
 // P is relative to a per-row reference max that moves only when a block's
 // max exceeds it by more than 2^8; then the row's O is rescaled in TMEM.
-// Warp roles (192 threads): warps 0-3 softmax/epilogue, warp 4 MMA issue and
-// TMEM owner, warp 5 TMA producer.  S is double-buffered in TMEM, P in smem,
-// K/V in a 3-stage ring, so the MMAs of block i+1 and the P*V of block i
-// overlap the softmax of block i.  Two CTAs fit per SM, and their softmax
-// and MMA phases interleave.
+// Q and P are A operands read from TMEM, so the only shared-memory traffic
+// per block is the TMA write of K and V and the MMAs' reads of them: with
+// N = 64 tiles, A operands in shared memory would make the MMAs wait on
+// shared-memory bandwidth rather than on the tensor pipe.
+// TMEM columns (256 per CTA): S double buffer [0,128), O [128,192),
+// Q [192,224) (bf16 pairs per 32-bit column).  P of block i overwrites the
+// first 32 columns of the S buffer it was computed from, so writing P never
+// waits for an earlier P*V; instead the MMA thread issues the S MMA that
+// next fills that buffer only once the P*V reading it has completed (MMAs
+// issued in order may still overlap in the pipe).
+// Warp roles (192 threads): warps 0-3 load Q, softmax and epilogue, warp 4
+// MMA issue and TMEM owner, warp 5 TMA producer.  S is double-buffered, K/V
+// sit in a 6-stage ring, so the MMAs of block i+1 and the P*V of block i
+// overlap the softmax of block i.  Two CTAs fit per SM (TMEM), and their
+// softmax and MMA phases interleave.
 #include <climits>
 
 #include "common.cuh"
@@ -46,24 +56,27 @@ using namespace sm100;
 
 constexpr int kRows = 128;   // query rows per CTA (M)
 constexpr int kKeys = 64;    // keys per block (N of S, K of P*V)
-constexpr int kStages = 3;   // K/V ring depth
+constexpr int kStages = 6;   // K/V ring depth
 constexpr int kThreads = 192;
 constexpr uint32_t kTileBytes = kKeys * 64 * 2;  // one K or V block, bf16
-constexpr uint32_t kQBytes = kRows * 64 * 2;
-constexpr uint32_t kPBytes = kRows * kKeys * 2;
 
-constexpr uint32_t OFF_Q = 0;
-constexpr uint32_t OFF_KV = OFF_Q + kQBytes;                      // stage s: K, then V
-constexpr uint32_t OFF_P = OFF_KV + kStages * 2 * kTileBytes;    // two P buffers
-constexpr uint32_t OFF_BAR = OFF_P + 2 * kPBytes;
+// TMEM column map
+constexpr uint32_t kColS = 0;    // two S buffers of 64 fp32 columns
+constexpr uint32_t kColO = 128;  // O, 64 fp32 columns
+constexpr uint32_t kColQ = 192;  // Q rows, 64 bf16 in 32 columns
+
+constexpr uint32_t OFF_KV = 0;  // stage s: K, then V
+constexpr uint32_t OFF_BAR = OFF_KV + kStages * 2 * kTileBytes;
 
 struct Bars {
-  uint64_t q;
+  uint64_t q;      // the 128 row threads have written Q into TMEM
   uint64_t full[kStages];
   uint64_t empty[kStages];
   uint64_t s[2];
+  // p[i & 1]: the 128 row threads have written P of block i.  Two barriers,
+  // because a warp may finish block i+1 before another finishes block i.
   uint64_t p[2];
-  uint64_t pfree[2];  // P*V of the block that used this P buffer is done
+  uint64_t pfree;  // P*V of a block is done (O holds every block so far)
   uint64_t fin;
 };
 constexpr uint32_t OFF_MISC = OFF_BAR + ((sizeof(Bars) + 15) / 16) * 16;  // tmem, abort, nblk
@@ -91,7 +104,7 @@ struct Fuse {
 
 template <bool SEL, bool FUSE>
 __global__ void __launch_bounds__(kThreads, 2)
-attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+attn_tc_kernel(const bf16* __restrict__ qg, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, bf16* __restrict__ o,
                float* __restrict__ lse, const int32_t* __restrict__ idx, Dims d, int* err,
                Fuse fz) {
@@ -115,7 +128,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   const int pos0 = d.q_off + t0;  // key position of the tile's first query
 
   if (tid == 0) {
-    mbar_init(&bars->q, 1);
+    mbar_init(&bars->q, 128);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bars->full[s], 1);
       mbar_init(&bars->empty[s], 1);
@@ -123,8 +136,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->s[i], 1);
       mbar_init(&bars->p[i], 128);
-      mbar_init(&bars->pfree[i], 1);
     }
+    mbar_init(&bars->pfree, 1);
     mbar_init(&bars->fin, 1);
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -132,7 +145,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   }
   if (warp == 4) tmem_alloc(tmem_slot, 256);
   if (warp == 5 && lane == 0) {
-    prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
   }
@@ -203,8 +215,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   if (warp == 5) {
     // ---- TMA producer -----------------------------------------------------------
     if (lane == 0) {
-      mbar_expect_tx(&bars->q, kQBytes);
-      tma_load_3d(smem + OFF_Q, &tm_q, &bars->q, 0, g * d.G, b * d.Tq + t0);
       int issued = 0;
       for (int i = 0; i < n; ++i) {
         const int st = i % kStages;
@@ -220,7 +230,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         issued = i + 1;
       }
       if (*abort_flag) {  // let the copies already issued land before exit
-        drain_bar(&bars->q, 0);
         for (int i = max(0, issued - kStages); i < issued; ++i)
           drain_bar(&bars->full[i % kStages], (i / kStages) & 1);
       }
@@ -230,34 +239,38 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16(kRows, kKeys, false, false);
       constexpr uint32_t idesc_o = idesc_bf16(kRows, 64, false, true);
-      const uint32_t q_addr = smem_u32(smem + OFF_Q);
       bool ok = wait_bar(&bars->q, 0, abort_flag, err);
+      tc_fence_after();
       auto issue_s = [&](int i) -> bool {
         const int st = i % kStages;
         if (!wait_bar(&bars->full[st], (i / kStages) & 1, abort_flag, err)) return false;
         tc_fence_after();
         const uint32_t k_addr = smem_u32(smem + OFF_KV + st * 2 * kTileBytes);
-        const uint32_t d_tmem = tmem + (uint32_t)(i & 1) * 64u;
+        const uint32_t d_tmem = tmem + kColS + (uint32_t)(i & 1) * 64u;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(d_tmem, desc_sw128(q_addr + kk * 32, 16), desc_sw128(k_addr + kk * 32, 16),
-                   idesc_s, kk > 0);
+          mma_bf16_ts(d_tmem, tmem + kColQ + kk * 8, desc_sw128(k_addr + kk * 32, 16), idesc_s,
+                      kk > 0);
         mma_commit(&bars->s[i & 1]);
         return true;
       };
       if (ok && n > 0) ok = issue_s(0);
       for (int i = 0; ok && i < n; ++i) {
+        // S buffer (i+1)&1 holds P of block i-1: its P*V must be complete
+        if (i >= 1 && i + 1 < n) {
+          if (!wait_bar(&bars->pfree, (i - 1) & 1, abort_flag, err)) break;
+          tc_fence_after();
+        }
         if (i + 1 < n && !issue_s(i + 1)) break;
         if (!wait_bar(&bars->p[i & 1], (i >> 1) & 1, abort_flag, err)) break;
         tc_fence_after();
         const int st = i % kStages;
         const uint32_t v_addr = smem_u32(smem + OFF_KV + st * 2 * kTileBytes + kTileBytes);
-        const uint32_t p_addr = smem_u32(smem + OFF_P + (i & 1) * kPBytes);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + 128u, desc_sw128(p_addr + kk * 32, 16),
-                   desc_sw128(v_addr + kk * 2048, 8192), idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&bars->pfree[i & 1]);
+          mma_bf16_ts(tmem + kColO, tmem + kColS + (uint32_t)(i & 1) * 64u + kk * 8,
+                      desc_sw128(v_addr + kk * 2048, 8192), idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&bars->pfree);
         mma_commit(&bars->empty[st]);
       }
       // every MMA issued must finish before TMEM is released
@@ -275,14 +288,35 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const int tl = r / d.G, hh = r % d.G;
     const bool valid = tl < nvalid;
     const int t = pos0 + tl;
+    const uint32_t lane_tmem = tmem + ((uint32_t)(warp * 32) << 16);
+    {  // this row of Q into TMEM (zeros past the last query)
+      uint32_t qv[32];
+      if (valid) {
+        const uint4* src = reinterpret_cast<const uint4*>(
+            qg + (((size_t)b * d.Tq + t0 + tl) * d.Hq + (size_t)g * d.G + hh) * 64);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 u = __ldg(src + c);
+          qv[4 * c] = u.x;
+          qv[4 * c + 1] = u.y;
+          qv[4 * c + 2] = u.z;
+          qv[4 * c + 3] = u.w;
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) qv[c] = 0u;
+      }
+      tmem_st32u(lane_tmem + kColQ, qv);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars->q);
+    }
     const int lo = SEL ? 0 : max(0, t - d.window + 1);  // first key of the row
     const int* lst = SEL ? toks + tl * (d.topk + 1) : nullptr;
     int ptr = 0;
     int nxt = SEL && valid ? lst[0] : INT_MAX;  // next block this row selected
     float mref = -INFINITY, lsum = 0.f;
     const float sl2 = d.scale * kLog2e;
-    const uint32_t lane_tmem = tmem + ((uint32_t)(warp * 32) << 16);
-    const uint32_t prow = smem_u32(smem + OFF_P) + (uint32_t)(r >> 3) * 1024u + (uint32_t)(r & 7) * 128u;
     bool ok = true;
     for (int i = 0; i < n; ++i) {
       const int j = SEL ? blk[i] : blk0 + i;
@@ -303,8 +337,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       }
       tc_fence_after();
       float sv[64];
-      tmem_ld32(lane_tmem + (uint32_t)(i & 1) * 64u, sv);
-      tmem_ld32(lane_tmem + (uint32_t)(i & 1) * 64u + 32u, sv + 32);
+      tmem_ld32(lane_tmem + kColS + (uint32_t)(i & 1) * 64u, sv);
+      tmem_ld32(lane_tmem + kColS + (uint32_t)(i & 1) * 64u + 32u, sv + 32);
       tmem_wait_ld();
       float ms = -INFINITY;  // block max, scaled to log2 units
       if (rowsel) {
@@ -325,27 +359,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       }
       const bool grow = rowsel && ms > mref + 8.f;
       const bool resc = grow && mref != -INFINITY;
-      if (i > 0 && __any_sync(0xffffffffu, resc)) {
-        // O holds P*V of blocks 0..i-1: wait for the last one, rescale rows
-        if (!wait_bar_warp(&bars->pfree[(i - 1) & 1], ((i - 1) >> 1) & 1, abort_flag, err)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const float f = resc ? fast_exp2(mref - ms) : 1.f;
-        float ov[32];
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          tmem_ld32(lane_tmem + 128u + 32u * h2, ov);
-          tmem_wait_ld();
-#pragma unroll
-          for (int c = 0; c < 32; ++c) ov[c] *= f;
-          tmem_st32(lane_tmem + 128u + 32u * h2, ov);
-        }
-        tmem_wait_st();
-      }
+      float f = 1.f;  // factor for this row's O (blocks before i)
       if (grow) {
-        if (resc) lsum *= fast_exp2(mref - ms);
+        if (resc) {
+          f = fast_exp2(mref - ms);
+          lsum *= f;
+        }
         mref = ms;
       }
       uint32_t pk[32];
@@ -370,29 +389,40 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
         for (int c = 0; c < 32; ++c) pk[c] = 0u;
       }
-      // the P buffer of this block was last read by the P*V of block i-2
-      if (i >= 2 &&
-          !wait_bar_warp(&bars->pfree[i & 1], ((i - 2) >> 1) & 1, abort_flag, err)) {
-        ok = false;
-        break;
-      }
-      const uint32_t pb = prow + (uint32_t)(i & 1) * kPBytes;
+      if (__any_sync(0xffffffffu, resc)) {  // resc implies i > 0
+        // O holds P*V of blocks 0..i-1: wait for the last one, rescale rows.
+        // The S wait of this block already covered every P*V before i-1,
+        // so the parity below cannot alias an older phase.
+        if (!wait_bar_warp(&bars->pfree, (i - 1) & 1, abort_flag, err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        float ov[32];
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        st_shared_v4(pb + ((uint32_t)(c ^ (r & 7)) << 4), pk[4 * c], pk[4 * c + 1],
-                     pk[4 * c + 2], pk[4 * c + 3]);
-      fence_proxy_async_smem();
+        for (int h2 = 0; h2 < 2; ++h2) {
+          tmem_ld32(lane_tmem + kColO + 32u * h2, ov);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) ov[c] *= f;
+          tmem_st32(lane_tmem + kColO + 32u * h2, ov);
+        }
+      }
+      tmem_st32u(lane_tmem + kColS + (uint32_t)(i & 1) * 64u, pk);
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars->p[i & 1]);
     }
     float acc[64];
     bool have_o = false;
-    if (ok && n > 0)
-      have_o = wait_bar_warp(&bars->pfree[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag, err);
+    // every MMA of this CTA has completed once `fin` (committed after the
+    // last P*V) fires; a parity wait on pfree could alias an older phase
+    // here, since no P*V after block n-3 was waited for
+    if (ok && n > 0) have_o = wait_bar_warp(&bars->fin, 0, abort_flag, err);
     if (have_o) {
       tc_fence_after();
-      tmem_ld32(lane_tmem + 128u, acc);
-      tmem_ld32(lane_tmem + 160u, acc + 32);
+      tmem_ld32(lane_tmem + kColO, acc);
+      tmem_ld32(lane_tmem + kColO + 32u, acc + 32);
       tmem_wait_ld();
     } else {
 #pragma unroll
@@ -470,9 +500,8 @@ cudaError_t launch_tc(const Dims& d, const void* q, const void* k, const void* v
                       const int32_t* idx, void* o, float* lse, int* err, const Fuse& fz,
                       cudaStream_t s) {
   const int TQ = tokens_per_tile(d.G);
-  CUtensorMap mq, mk, mv;
-  if (!make_tmap_bf16(&mq, q, d.Hq, (long)d.B * d.Tq, d.G, TQ) ||
-      !make_tmap_bf16(&mk, k, d.Hkv, (long)d.B * d.T, 1, kKeys) ||
+  CUtensorMap mk, mv;
+  if (!make_tmap_bf16(&mk, k, d.Hkv, (long)d.B * d.T, 1, kKeys) ||
       !make_tmap_bf16(&mv, v, d.Hkv, (long)d.B * d.T, 1, kKeys))
     return cudaErrorInvalidValue;
   const size_t smem = OFF_LIST + list_ints(d) * sizeof(int) + 1024;
@@ -480,7 +509,8 @@ cudaError_t launch_tc(const Dims& d, const void* q, const void* k, const void* v
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((d.Tq + TQ - 1) / TQ, d.Hkv, d.B);
-  attn_tc_kernel<SEL, FUSE><<<grid, kThreads, smem, s>>>(mq, mk, mv, (bf16*)o, lse, idx, d, err,
+  attn_tc_kernel<SEL, FUSE><<<grid, kThreads, smem, s>>>((const bf16*)q, mk, mv, (bf16*)o, lse,
+                                                        idx, d, err,
                                                         fz);
   return cudaGetLastError();
 }
