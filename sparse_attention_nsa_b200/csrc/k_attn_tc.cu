@@ -27,14 +27,16 @@
 // TMEM columns (256 per CTA): S double buffer [0,128), O [128,192),
 // Q [192,224) (bf16 pairs per 32-bit column).  P of block i overwrites the
 // first 32 columns of the S buffer it was computed from, so writing P never
-// waits for an earlier P*V; instead the MMA thread issues the S MMA that
-// next fills that buffer only once the P*V reading it has completed (MMAs
-// issued in order may still overlap in the pipe).
-// Warp roles (192 threads): warps 0-3 load Q, softmax and epilogue, warp 4
-// MMA issue and TMEM owner, warp 5 TMA producer.  S is double-buffered, K/V
-// sit in a 6-stage ring, so the MMAs of block i+1 and the P*V of block i
-// overlap the softmax of block i.  Two CTAs fit per SM (TMEM), and their
-// softmax and MMA phases interleave.
+// waits for an earlier P*V; instead the S MMA that next fills that buffer is
+// issued only once the P*V reading it has completed (MMAs of different
+// accumulators may overlap in the pipe).
+// Warp roles (224 threads): warps 0-3 load Q, softmax and epilogue; warp 4
+// issues the S MMAs and owns TMEM; warp 6 issues the P*V MMAs; warp 5 is the
+// TMA producer.  Each tcgen05.mma, commit and barrier wait costs its issuing
+// thread tens of cycles (measured in place: about 80 per MMA, 100 per
+// commit or satisfied wait), so one thread issuing both kinds is the
+// critical path once the softmax is short.  S is double-buffered, K/V sit
+// in a 6-stage ring.  Two CTAs fit per SM (TMEM).
 #include <climits>
 
 #include "common.cuh"
@@ -57,7 +59,7 @@ using namespace sm100;
 constexpr int kRows = 128;   // query rows per CTA (M)
 constexpr int kKeys = 64;    // keys per block (N of S, K of P*V)
 constexpr int kStages = 6;   // K/V ring depth
-constexpr int kThreads = 192;
+constexpr int kThreads = 224;
 constexpr uint32_t kTileBytes = kKeys * 64 * 2;  // one K or V block, bf16
 
 // TMEM column map
@@ -76,7 +78,6 @@ struct Bars {
   // p[i & 1]: the 128 row threads have written P of block i.  Two barriers,
   // because a warp may finish block i+1 before another finishes block i.
   uint64_t p[2];
-  uint64_t pfree;  // P*V of a block is done (O holds every block so far)
   uint64_t fin;
 };
 constexpr uint32_t OFF_MISC = OFF_BAR + ((sizeof(Bars) + 15) / 16) * 16;  // tmem, abort, nblk
@@ -137,7 +138,6 @@ attn_tc_kernel(const bf16* __restrict__ qg, const __grid_constant__ CUtensorMap 
       mbar_init(&bars->s[i], 1);
       mbar_init(&bars->p[i], 128);
     }
-    mbar_init(&bars->pfree, 1);
     mbar_init(&bars->fin, 1);
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -235,15 +235,19 @@ attn_tc_kernel(const bf16* __restrict__ qg, const __grid_constant__ CUtensorMap 
       }
     }
   } else if (warp == 4) {
-    // ---- MMA issue ------------------------------------------------------------------
+    // ---- S = Q K^T issue --------------------------------------------------------------
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16(kRows, kKeys, false, false);
-      constexpr uint32_t idesc_o = idesc_bf16(kRows, 64, false, true);
       bool ok = wait_bar(&bars->q, 0, abort_flag, err);
       tc_fence_after();
-      auto issue_s = [&](int i) -> bool {
+      for (int i = 0; ok && i < n; ++i) {
         const int st = i % kStages;
-        if (!wait_bar(&bars->full[st], (i / kStages) & 1, abort_flag, err)) return false;
+        // S buffer i&1 holds P of block i-2: its P*V (hence its softmax) must
+        // be complete; the commit that frees that block's K/V stage says so
+        if (i >= 2 &&
+            !wait_bar(&bars->empty[(i - 2) % kStages], ((i - 2) / kStages) & 1, abort_flag, err))
+          break;
+        if (!wait_bar(&bars->full[st], (i / kStages) & 1, abort_flag, err)) break;
         tc_fence_after();
         const uint32_t k_addr = smem_u32(smem + OFF_KV + st * 2 * kTileBytes);
         const uint32_t d_tmem = tmem + kColS + (uint32_t)(i & 1) * 64u;
@@ -252,16 +256,13 @@ attn_tc_kernel(const bf16* __restrict__ qg, const __grid_constant__ CUtensorMap 
           mma_bf16_ts(d_tmem, tmem + kColQ + kk * 8, desc_sw128(k_addr + kk * 32, 16), idesc_s,
                       kk > 0);
         mma_commit(&bars->s[i & 1]);
-        return true;
-      };
-      if (ok && n > 0) ok = issue_s(0);
-      for (int i = 0; ok && i < n; ++i) {
-        // S buffer (i+1)&1 holds P of block i-1: its P*V must be complete
-        if (i >= 1 && i + 1 < n) {
-          if (!wait_bar(&bars->pfree, (i - 1) & 1, abort_flag, err)) break;
-          tc_fence_after();
-        }
-        if (i + 1 < n && !issue_s(i + 1)) break;
+      }
+    }
+  } else if (warp == 6) {
+    // ---- O += P V issue -----------------------------------------------------------------
+    if (lane == 0) {
+      constexpr uint32_t idesc_o = idesc_bf16(kRows, 64, false, true);
+      for (int i = 0; i < n; ++i) {
         if (!wait_bar(&bars->p[i & 1], (i >> 1) & 1, abort_flag, err)) break;
         tc_fence_after();
         const int st = i % kStages;
@@ -270,10 +271,11 @@ attn_tc_kernel(const bf16* __restrict__ qg, const __grid_constant__ CUtensorMap 
         for (int kk = 0; kk < 4; ++kk)
           mma_bf16_ts(tmem + kColO, tmem + kColS + (uint32_t)(i & 1) * 64u + kk * 8,
                       desc_sw128(v_addr + kk * 2048, 8192), idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&bars->pfree);
+        // frees the K/V stage and the P columns; O is complete up to block i
         mma_commit(&bars->empty[st]);
       }
-      // every MMA issued must finish before TMEM is released
+      // every P*V must finish before the epilogue reads O; every S MMA has
+      // finished before the P it fed was written
       mma_commit(&bars->fin);
       drain_bar(&bars->fin, 0);
     }
@@ -390,10 +392,12 @@ attn_tc_kernel(const bf16* __restrict__ qg, const __grid_constant__ CUtensorMap 
         for (int c = 0; c < 32; ++c) pk[c] = 0u;
       }
       if (__any_sync(0xffffffffu, resc)) {  // resc implies i > 0
-        // O holds P*V of blocks 0..i-1: wait for the last one, rescale rows.
-        // The S wait of this block already covered every P*V before i-1,
-        // so the parity below cannot alias an older phase.
-        if (!wait_bar_warp(&bars->pfree, (i - 1) & 1, abort_flag, err)) {
+        // O holds P*V of blocks 0..i-1: wait for the last one (its commit
+        // frees that block's K/V stage), then rescale rows.  The next phase
+        // of that barrier needs the P*V of block i-1+kStages, so the parity
+        // below cannot alias.
+        if (!wait_bar_warp(&bars->empty[(i - 1) % kStages], ((i - 1) / kStages) & 1, abort_flag,
+                           err)) {
           ok = false;
           break;
         }
@@ -416,8 +420,7 @@ attn_tc_kernel(const bf16* __restrict__ qg, const __grid_constant__ CUtensorMap 
     float acc[64];
     bool have_o = false;
     // every MMA of this CTA has completed once `fin` (committed after the
-    // last P*V) fires; a parity wait on pfree could alias an older phase
-    // here, since no P*V after block n-3 was waited for
+    // last P*V) fires
     if (ok && n > 0) have_o = wait_bar_warp(&bars->fin, 0, abort_flag, err);
     if (have_o) {
       tc_fence_after();
