@@ -39,7 +39,7 @@ from sparse_attention_nsa_b200 import inputs as W  # noqa: E402
 METRIC = "NSA fwd tokens/s & TFLOP/s (frac of bf16 peak) @8192 GQA-4; decode HBM GB/s"
 WORK = W.NSA_340M
 DECODE = W.DECODE_32K
-KERNELS_PER_FORWARD = 6  # compress, cmp+scores, top-k, selection, window, combine
+KERNELS_PER_FORWARD = 5  # compress, cmp+scores, top-k, window (side stream), selection+combine
 
 
 # ------------------------------------------------------------------ work model
