@@ -131,7 +131,7 @@ class ClockSampler:
                         self.reasons.add(name)
             except Exception:
                 pass
-            time.sleep(0.01)
+            time.sleep(0.002)
 
     def __enter__(self):
         if self._nv:
@@ -279,11 +279,13 @@ def run_gpu(args, rank: int, world: int, dist_on: bool) -> None:
         step()
     if nsa.nsa_last_device_error() != 0:
         raise RuntimeError("device-side check failed during warm-up")
+    # clocks are sampled across every timed region of this run (forward,
+    # selection alone, end to end, decode, training step)
     sampler = ClockSampler(local)
     barrier_sync(dist_on)
-    with sampler:
-        times = timed_steps(step, args.steps, flush, stream)
-        barrier_sync(dist_on)
+    sampler.__enter__()
+    times = timed_steps(step, args.steps, flush, stream)
+    barrier_sync(dist_on)
     ms = max_over_ranks(sum(times) / len(times), dist_on)
     flops = fwd_flops(w)
     tokens_per_step = w.B * w.T
@@ -323,6 +325,7 @@ def run_gpu(args, rank: int, world: int, dist_on: bool) -> None:
     # training step (B=8 forward + backward)
     del hq, hk, hv, hg, hout
     train = run_train(dev, flush, stream, max(3, args.steps // 4), peaks)
+    sampler.__exit__(None, None, None)
 
     barrier_sync(dist_on)
     if rank != 0:

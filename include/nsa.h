@@ -294,11 +294,12 @@ nsa_status nsa_backward(const nsa_params* p, const void* q, const void* k,
  * provide nsa_decode's workspace.  This entry point takes the same
  * arguments as nsa_decode minus the workspace and runs the same kernels,
  * with the scratch taken from a fixed array inside the library's device
- * memory (nsa_decode_noalloc_max_scratch() bytes, 8 MiB, held on every GPU
+ * memory (nsa_decode_noalloc_max_scratch() bytes, 16 MiB, held on every GPU
  * that loads the library until the process exits).  It allocates nothing.
  * A problem whose scratch would not fit returns NSA_ERR_SCRATCH_TOO_SMALL
  * before anything is launched (B=64 sequences, 16 heads on one KV head,
- * 32768-token caches, top-k 16, window 512 need about 6.8 MiB).  The first call on a device looks up the array's device
+ * 32768-token caches, top-k 16, window 512 need about 11 MiB).  The first
+ * call on a device looks up the array's device
  * address (with that device current) and caches it; make that first call
  * before any stream capture.  All calls on a device share the array and it
  * keeps the previous call's contents (every element is written before it

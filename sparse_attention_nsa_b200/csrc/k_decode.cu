@@ -24,6 +24,7 @@
 #include "internal.h"
 #include "sm100.cuh"
 #include "tmap.h"
+#include "topk.cuh"
 
 namespace nsa {
 namespace {
@@ -31,6 +32,7 @@ namespace {
 using namespace sm100;
 
 constexpr int kPartStride = 66;  // o[64], m (log2 units), l per row
+constexpr int kMaxChunks = 16;   // 64-block chunks of the compressed cache (Nc <= 1024)
 
 __device__ __forceinline__ uint32_t swz(uint32_t base, int row, int chunk) {
   return base + (uint32_t)row * 128u + ((uint32_t)(chunk ^ (row & 7)) << 4);
@@ -128,11 +130,6 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
-// (score desc, block asc): does (va, ia) come before (vb, ib)?
-__device__ __forceinline__ bool goes_first(float va, int ia, float vb, int ib) {
-  return va > vb || (va == vb && ia < ib);
-}
-
 __device__ __forceinline__ float quad_max(float x) {
   x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 1));
   return fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 2));
@@ -143,314 +140,177 @@ __device__ __forceinline__ float quad_sum(float x) {
 }
 
 struct DecodeWs {
-  float* ocmp;   // [B*Hkv][16][64]
+  float* pcmp;   // [B*Hkv][nchunk][16][66]  compression-branch partials
+  float* logit;  // [B*Hkv][16][Nc]          compression logits (log2 units)
   int* idx;      // [B*Hkv][topk]
   float* psel;   // [B*Hkv][topk][16][66]
   float* pswa;   // [B*Hkv][nwin][16][66]
   int nwin;      // window blocks of the decoded position
   int jlo;       // first window block
+  int nchunk;    // 64-block chunks of the compressed cache
 };
 
-// ---- K1: compression branch, block scores, top-k --------------------------------------
-constexpr int kK1Threads = 256;
-
-__global__ void __launch_bounds__(kK1Threads, 1)
-decode_cmp_topk_kernel(const __grid_constant__ CUtensorMap tm_kc,
-                       const __grid_constant__ CUtensorMap tm_vc, const bf16* __restrict__ q,
-                       Dims d, DecodeWs ws, int32_t* __restrict__ idx_out, int need_o,
-                       int need_idx, int* err) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  const int ncp = (d.Nc + 63) & ~63;  // compressed rows staged (64-row TMA boxes)
-  // region 0 holds the staged Kc and Vc, later the per-warp o_cmp partials
-  const size_t r0_bytes = max((size_t)ncp * 256, (size_t)8 * 16 * 64 * 4);
-  uint8_t* kcs = smem;
-  uint8_t* vcs = kcs + (size_t)ncp * 128;
-  uint8_t* qs = smem + r0_bytes;
-  float* red = (float*)(qs + 2048);             // [8 warps][16 rows]
-  float* rowM = red + 8 * 16;                   // [16]
-  float* rowL = rowM + 16;                      // [16]
-  float* score = rowL + 16;                     // [ncp]
-  uint32_t* bits = (uint32_t*)(score + ncp);    // [(Nb+31)/32]
-  float* sort_v = (float*)(bits + (d.Nb + 31) / 32 + 2);  // [512]
-  int* sort_i = (int*)(sort_v + 512);                      // [512]
-  uint64_t* bar = (uint64_t*)(((uintptr_t)(sort_i + 512) + 7) & ~(uintptr_t)7);
-  volatile int* abort_flag = (volatile int*)(bar + 2);
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bg = blockIdx.x;
-  const int b = bg / d.Hkv, g = bg % d.Hkv;
-  const int t = d.T - 1;
-  const int nvis = min((t + 1) / d.l, d.Nc);
-  const int nchunks = ncp / 64;
-  if (threadIdx.x == 0) {
-    mbar_init(&bar[0], 1);
-    mbar_init(&bar[1], 1);
-    fence_barrier_init();
-    *abort_flag = 0;
-  }
-  pdl_launch_dependents();
-  __syncthreads();
-  if (threadIdx.x == 0 && nchunks > 0) {
-    mbar_expect_tx(&bar[0], (uint32_t)nchunks * 8192u);
-    for (int c = 0; c < nchunks; ++c)
-      tma_load_3d(kcs + c * 8192, &tm_kc, &bar[0], 0, g, b * d.Nc + c * 64);
-    if (need_o) {
-      mbar_expect_tx(&bar[1], (uint32_t)nchunks * 8192u);
-      for (int c = 0; c < nchunks; ++c)
-        tma_load_3d(vcs + c * 8192, &tm_vc, &bar[1], 0, g, b * d.Nc + c * 64);
-    }
-  }
-  if (warp == 0) stage_q(qs, q + ((size_t)b * d.Hq + (size_t)g * d.G) * 64, d.G, lane);
-  fence_proxy_async_smem();
-  __syncthreads();
-  const uint32_t qbase = smem_u32(qs);
-  const int r0 = lane >> 2, cq = lane & 3;  // fragment row (and r0 + 8), column pair
-  const float sl2 = d.scale * kLog2e;
-  const int key0 = warp * 64;               // this warp's 64 compressed blocks
-  const bool active = key0 < ncp && nvis > 0;
-  float s[8][4];
-  bool ok = true;
-  if (nchunks > 0) ok = wait_bar_warp(&bar[0], 0, abort_flag, err);
-  if (active && ok) {
-    uint32_t qa[4][4];
-    load_qa(qa, qbase, lane);
-    qk_tile(s, qa, smem_u32(kcs), key0, lane);
-  } else {
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) s[nt][e] = 0.f;
-  }
-  // scale, mask (block visible, row is a real head), row max
+// Softmax partial of one 64-key tile for the 16 MMA rows (rows >= G and
+// invisible keys are -inf in p on entry): writes (P V, max, sum) to part in
+// the [16][kPartStride] layout; p is replaced by its exponentials.
+__device__ __forceinline__ void tile_partial(float p[8][4], uint32_t vbase, float* part,
+                                             bool need_o, int lane) {
+  const int r0 = lane >> 2, cq = lane & 3;
   float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-  for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int j = key0 + nt * 8 + 2 * cq + (e & 1);
-      const int row = r0 + (e >> 1) * 8;
-      const bool vis = active && j < nvis && row < d.G;
-      s[nt][e] = vis ? s[nt][e] * sl2 : -INFINITY;
-      if (e < 2) mx0 = fmaxf(mx0, s[nt][e]);
-      else mx1 = fmaxf(mx1, s[nt][e]);
-    }
+  for (int nt = 0; nt < 8; ++nt) {
+    mx0 = fmaxf(mx0, fmaxf(p[nt][0], p[nt][1]));
+    mx1 = fmaxf(mx1, fmaxf(p[nt][2], p[nt][3]));
+  }
   mx0 = quad_max(mx0);
   mx1 = quad_max(mx1);
-  if (cq == 0) {
-    red[warp * 16 + r0] = mx0;
-    red[warp * 16 + r0 + 8] = mx1;
-  }
-  __syncthreads();
-  if (threadIdx.x < 16) {
-    float m = -INFINITY;
-    for (int w = 0; w < 8; ++w) m = fmaxf(m, red[w * 16 + threadIdx.x]);
-    rowM[threadIdx.x] = m;
-  }
-  __syncthreads();
-  const float M0 = rowM[r0], M1 = rowM[r0 + 8];
-  const float b0 = M0 == -INFINITY ? 0.f : M0, b1 = M1 == -INFINITY ? 0.f : M1;
-  float sm0 = 0.f, sm1 = 0.f;
+  const float b0 = mx0 == -INFINITY ? 0.f : mx0, b1 = mx1 == -INFINITY ? 0.f : mx1;
+  float l0 = 0.f, l1 = 0.f;
 #pragma unroll
   for (int nt = 0; nt < 8; ++nt) {
-    s[nt][0] = fast_exp2(s[nt][0] - b0);
-    s[nt][1] = fast_exp2(s[nt][1] - b0);
-    s[nt][2] = fast_exp2(s[nt][2] - b1);
-    s[nt][3] = fast_exp2(s[nt][3] - b1);
-    sm0 += s[nt][0] + s[nt][1];
-    sm1 += s[nt][2] + s[nt][3];
+    p[nt][0] = fast_exp2(p[nt][0] - b0);
+    p[nt][1] = fast_exp2(p[nt][1] - b0);
+    p[nt][2] = fast_exp2(p[nt][2] - b1);
+    p[nt][3] = fast_exp2(p[nt][3] - b1);
+    l0 += p[nt][0] + p[nt][1];
+    l1 += p[nt][2] + p[nt][3];
   }
-  sm0 = quad_sum(sm0);
-  sm1 = quad_sum(sm1);
-  if (cq == 0) {
-    red[warp * 16 + r0] = sm0;
-    red[warp * 16 + r0 + 8] = sm1;
-  }
-  __syncthreads();
-  if (threadIdx.x < 16) {
-    float l = 0.f;
-    for (int w = 0; w < 8; ++w) l += red[w * 16 + threadIdx.x];
-    rowL[threadIdx.x] = l;
-  }
-  __syncthreads();
-  const float i0 = rowL[r0] > 0.f ? 1.f / rowL[r0] : 0.f;
-  const float i1 = rowL[r0 + 8] > 0.f ? 1.f / rowL[r0 + 8] : 0.f;
-  // normalised probabilities; block scores = sum over the group's heads
-#pragma unroll
-  for (int nt = 0; nt < 8; ++nt) {
-    s[nt][0] *= i0;
-    s[nt][1] *= i0;
-    s[nt][2] *= i1;
-    s[nt][3] *= i1;
-    float c0 = s[nt][0] + s[nt][2], c1 = s[nt][1] + s[nt][3];
-#pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-      c0 += __shfl_xor_sync(0xffffffffu, c0, off);
-      c1 += __shfl_xor_sync(0xffffffffu, c1, off);
-    }
-    if (r0 == 0 && key0 < ncp) {
-      score[key0 + nt * 8 + 2 * cq] = c0;
-      score[key0 + nt * 8 + 2 * cq + 1] = c1;
-    }
-  }
-  // o_cmp = P Vc: each warp its 64 blocks, then a sum over warps
+  l0 = quad_sum(l0);
+  l1 = quad_sum(l1);
   if (need_o) {
     float o[8][4];
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
-    const bool okv = nchunks > 0 && wait_bar_warp(&bar[1], 0, abort_flag, err);
-    if (active && okv) pv_tile(o, s, smem_u32(vcs), key0, lane);
-    __syncthreads();  // every warp is done with Kc and Vc: reuse region 0
-    float* part = (float*)smem;  // [8 warps][16][64]
+    pv_tile(o, p, vbase, 0, lane);
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt) {
-      part[(warp * 16 + r0) * 64 + nt * 8 + 2 * cq] = o[nt][0];
-      part[(warp * 16 + r0) * 64 + nt * 8 + 2 * cq + 1] = o[nt][1];
-      part[(warp * 16 + r0 + 8) * 64 + nt * 8 + 2 * cq] = o[nt][2];
-      part[(warp * 16 + r0 + 8) * 64 + nt * 8 + 2 * cq + 1] = o[nt][3];
+      part[r0 * kPartStride + nt * 8 + 2 * cq] = o[nt][0];
+      part[r0 * kPartStride + nt * 8 + 2 * cq + 1] = o[nt][1];
+      part[(r0 + 8) * kPartStride + nt * 8 + 2 * cq] = o[nt][2];
+      part[(r0 + 8) * kPartStride + nt * 8 + 2 * cq + 1] = o[nt][3];
     }
-    __syncthreads();
-    float* dst = ws.ocmp + (size_t)bg * 16 * 64;
-    for (int e = threadIdx.x; e < 16 * 64; e += kK1Threads) {
-      float acc = 0.f;
-      for (int w = 0; w < 8; ++w) acc += part[w * 16 * 64 + e];
-      dst[e] = acc;
-    }
-  } else {
-    __syncthreads();
   }
-  // top-k over blocks 1..cur-1 (forced: 0 and cur).  Each warp sorts the
-  // candidates among its 64 blocks by (score desc, block asc) with a bitonic
-  // network in registers and shuffles; warp 0 then merges the eight sorted
-  // lists, taking the best head topk - 2 times.
-  if (need_idx) {
-    int* out = ws.idx + (size_t)bg * d.topk;
-    int32_t* out2 = idx_out ? idx_out + (size_t)bg * d.topk : nullptr;
-    const int cur = t / d.l;
-    const int K2 = d.topk - 2;
-    if (cur + 1 <= d.topk) {
-      for (int k = threadIdx.x; k < d.topk; k += kK1Threads) {
-        out[k] = k <= cur ? k : -1;
-        if (out2) out2[k] = out[k];
-      }
-    } else {
-      float v[2];
-      int ix[2];
+  if (cq == 0) {
+    part[r0 * kPartStride + 64] = mx0;
+    part[r0 * kPartStride + 65] = l0;
+    part[(r0 + 8) * kPartStride + 64] = mx1;
+    part[(r0 + 8) * kPartStride + 65] = l1;
+  }
+}
+
+// ---- K1a: compression branch over one 64-block chunk of the compressed cache --------
+// One single-warp CTA per (chunk, group, sequence), so every SM streams the
+// compressed cache: S = Q Kc^T for the G heads of the group (rows of the
+// m16n8k16 MMA), the chunk's softmax partial (max, sum, P Vc) for the
+// compression branch, and the scaled logits for the block scores.
+__global__ void __launch_bounds__(32)
+decode_cmp_chunk_kernel(const __grid_constant__ CUtensorMap tm_kc,
+                        const __grid_constant__ CUtensorMap tm_vc, const bf16* __restrict__ q,
+                        Dims d, DecodeWs ws, int need_o, int* err) {
+  __shared__ __align__(1024) uint8_t kv[2 * 8192];
+  __shared__ __align__(1024) uint8_t qs[2048];
+  __shared__ uint64_t bar;
+  __shared__ int abort_s;
+  const int lane = threadIdx.x;
+  const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int bg = b * d.Hkv + g;
+  const int t = d.T - 1;
+  const int nvis = min((t + 1) / d.l, d.Nc);  // complete blocks
+  pdl_launch_dependents();
+  if (lane == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+    abort_s = 0;
+  }
+  __syncwarp();
+  if (lane == 0) {
+    mbar_expect_tx(&bar, (need_o ? 2u : 1u) * 8192u);
+    tma_load_3d(kv, &tm_kc, &bar, 0, g, b * d.Nc + c * 64);
+    if (need_o) tma_load_3d(kv + 8192, &tm_vc, &bar, 0, g, b * d.Nc + c * 64);
+  }
+  stage_q(qs, q + ((size_t)b * d.Hq + (size_t)g * d.G) * 64, d.G, lane);
+  fence_proxy_async_smem();
+  __syncwarp();
+  uint32_t qa[4][4];
+  load_qa(qa, smem_u32(qs), lane);
+  if (!wait_bar(&bar, 0, (volatile int*)&abort_s, err)) {
+    drain_bar(&bar, 0);  // let the copies land before the CTA exits
+    return;
+  }
+  float s[8][4];
+  qk_tile(s, qa, smem_u32(kv), 0, lane);
+  const int r0 = lane >> 2, cq = lane & 3;
+  const float sl2 = d.scale * kLog2e;
+  float* lg = ws.logit + (size_t)bg * 16 * d.Nc;
 #pragma unroll
-      for (int sl = 0; sl < 2; ++sl) {
-        const int j = key0 + lane + 32 * sl;
-        const bool c = j >= 1 && j < cur && j < ncp;
-        v[sl] = c ? score[j] : -INFINITY;
-        ix[sl] = c ? j : INT_MAX;
-      }
-      for (int size = 2; size <= 64; size <<= 1) {
-        for (int jj = size >> 1; jj > 0; jj >>= 1) {
-          if (jj == 32) {  // the pair is held by one lane: (lane, lane + 32)
-            const bool dir = (lane & size) == 0;
-            const bool f = goes_first(v[0], ix[0], v[1], ix[1]);
-            if (f != dir) {
-              const float tv = v[0];
-              const int ti = ix[0];
-              v[0] = v[1];
-              ix[0] = ix[1];
-              v[1] = tv;
-              ix[1] = ti;
-            }
-          } else {
+  for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
-            for (int sl = 0; sl < 2; ++sl) {
-              const int e = lane + 32 * sl;
-              const float pv = __shfl_xor_sync(0xffffffffu, v[sl], jj);
-              const int pi = __shfl_xor_sync(0xffffffffu, ix[sl], jj);
-              const bool lower = (e & jj) == 0;
-              const bool dir = (e & size) == 0;
-              const bool self_first = goes_first(v[sl], ix[sl], pv, pi);
-              const bool keep = lower ? (dir == self_first) : (dir != self_first);
-              if (!keep) {
-                v[sl] = pv;
-                ix[sl] = pi;
-              }
-            }
-          }
-        }
-      }
-      float* cand_v = sort_v + warp * 64;
-      int* cand_i = sort_i + warp * 64;
-      cand_v[lane] = v[0];
-      cand_i[lane] = ix[0];
-      cand_v[lane + 32] = v[1];
-      cand_i[lane + 32] = ix[1];
-      __syncthreads();
-      if (warp == 0) {
-        const int words = (d.Nb + 31) / 32;
-        for (int w = lane; w < words; w += 32) bits[w] = 0u;
-        __syncwarp();
-        int head = 0;  // lanes 0..7: position in warp `lane`'s sorted list
-        for (int k = 0; k < K2; ++k) {
-          float hv = -INFINITY;
-          int hi = INT_MAX;
-          if (lane < 8 && head < 64) {
-            hv = sort_v[lane * 64 + head];
-            hi = sort_i[lane * 64 + head];
-          }
-          float wv = hv;
-          int wi = hi, wl = lane;
-#pragma unroll
-          for (int off = 4; off > 0; off >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, wv, off);
-            const int oi = __shfl_xor_sync(0xffffffffu, wi, off);
-            const int ol = __shfl_xor_sync(0xffffffffu, wl, off);
-            if (goes_first(ov, oi, wv, wi)) {
-              wv = ov;
-              wi = oi;
-              wl = ol;
-            }
-          }
-          wv = __shfl_sync(0xffffffffu, wv, 0);
-          wi = __shfl_sync(0xffffffffu, wi, 0);
-          wl = __shfl_sync(0xffffffffu, wl, 0);
-          if (wi == INT_MAX) break;
-          if (lane == wl) ++head;
-          if (lane == 0) bits[wi >> 5] |= 1u << (wi & 31);
-        }
-        __syncwarp();
-        if (lane == 0) {
-          bits[0] |= 1u;
-          bits[cur >> 5] |= 1u << (cur & 31);
-        }
-        __syncwarp();
-        int base = 0;
-        for (int w0 = 0; w0 <= (cur >> 5); w0 += 32) {
-          const int w = w0 + lane;
-          const uint32_t m = w <= (cur >> 5) ? bits[w] : 0u;
-          const int c = __popc(m);
-          int incl = c;
-#pragma unroll
-          for (int off = 1; off < 32; off <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, incl, off);
-            if (lane >= off) incl += y;
-          }
-          int pos = base + incl - c;
-          uint32_t mm = m;
-          while (mm) {
-            const int bit = __ffs(mm) - 1;
-            mm &= mm - 1;
-            if (pos < d.topk) {
-              out[pos] = w * 32 + bit;
-              if (out2) out2[pos] = w * 32 + bit;
-            }
-            ++pos;
-          }
-          base += __shfl_sync(0xffffffffu, incl, 31);
-        }
-        for (int p = base + lane; p < d.topk; p += 32) {
-          out[p] = -1;
-          if (out2) out2[p] = -1;
-        }
-      }
+    for (int e = 0; e < 4; ++e) {
+      const int j = c * 64 + nt * 8 + 2 * cq + (e & 1);
+      const int row = r0 + (e >> 1) * 8;
+      const bool vis = j < nvis && row < d.G;
+      s[nt][e] = vis ? s[nt][e] * sl2 : -INFINITY;
+      if (row < d.G && j < d.Nc) lg[(size_t)row * d.Nc + j] = s[nt][e];
     }
+  tile_partial(s, smem_u32(kv + 8192), ws.pcmp + ((size_t)bg * ws.nchunk + c) * 16 * kPartStride,
+               need_o != 0, lane);
+}
+
+// ---- K1b: block scores and top-k per (sequence, group) -----------------------------------
+// score_j = sum over the group's heads of exp2(logit - lse2), lse2 from the
+// chunk partials; then the warp radix select of topk.cuh.
+template <int QMAX>
+__global__ void __launch_bounds__(256)
+decode_topk_kernel(Dims d, DecodeWs ws, int32_t* __restrict__ idx_out) {
+  __shared__ float lse2[16];
+  __shared__ float score[QMAX * 32];
+  const int bg = blockIdx.x;
+  const int t = d.T - 1;
+  const int cur = t / d.l;
+  const int nvis = min((t + 1) / d.l, d.Nc);
+  pdl_launch_dependents();
+  pdl_wait();
+  // every load of a step is issued before any is used (fixed trip counts,
+  // predicated), so each step costs one memory round trip
+  if (threadIdx.x < d.G) {
+    const float* part = ws.pcmp + (size_t)bg * ws.nchunk * 16 * kPartStride + threadIdx.x * kPartStride;
+    float m[kMaxChunks], l[kMaxChunks];
+#pragma unroll
+    for (int c = 0; c < kMaxChunks; ++c) {
+      const bool ok = c < ws.nchunk;
+      m[c] = ok ? part[(size_t)c * 16 * kPartStride + 64] : -INFINITY;
+      l[c] = ok ? part[(size_t)c * 16 * kPartStride + 65] : 0.f;
+    }
+    float M = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < kMaxChunks; ++c) M = fmaxf(M, m[c]);
+    float L = 0.f;
+#pragma unroll
+    for (int c = 0; c < kMaxChunks; ++c)
+      if (m[c] != -INFINITY) L += fast_exp2(m[c] - M) * l[c];
+    lse2[threadIdx.x] = L > 0.f ? M + __log2f(L) : INFINITY;  // no visible block: scores 0
+  }
+  __syncthreads();
+  const float* lg = ws.logit + (size_t)bg * 16 * d.Nc;
+  for (int j = threadIdx.x; j < QMAX * 32; j += blockDim.x) {
+    float x[16];
+#pragma unroll
+    for (int r = 0; r < 16; ++r) x[r] = (r < d.G && j < nvis) ? lg[(size_t)r * d.Nc + j] : -INFINITY;
+    float sc = 0.f;
+#pragma unroll
+    for (int r = 0; r < 16; ++r)
+      if (r < d.G) sc += fast_exp2(x[r] - lse2[r]);
+    score[j] = sc;
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    int* out = ws.idx + (size_t)bg * d.topk;
+    warp_select_blocks<QMAX>(score, cur, d.topk, out, threadIdx.x);
+    __syncwarp();
+    if (idx_out)
+      for (int m = threadIdx.x; m < d.topk; m += 32) idx_out[(size_t)bg * d.topk + m] = out[m];
   }
 }
 
@@ -475,7 +335,10 @@ decode_block_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
   int j, sel_slot = -1;
   bool win = false;
   if (u < ws.nwin) {
-    if (!do_swa) return;
+    if (!do_swa) {
+      pdl_wait();  // completion of this grid implies completion of the ones before
+      return;
+    }
     j = ws.jlo + u;
     win = true;
   } else {
@@ -573,11 +436,15 @@ decode_block_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
       part[(r0 + 8) * kPartStride + 65] = l1;
     }
   }
+  if (win && !do_sel) pdl_wait();  // see the early return above
 }
 
 // ---- K3: merge the partials of each branch and apply the gates ------------------------
-// One warp per query head: lanes read the slots' (max, sum) in parallel, the
-// warp reduces them, then every slot's 64-wide partial output is folded in.
+// One warp per query head.  The slots of all three branches (compression
+// chunks, selected blocks, window blocks) are one list: lanes read the
+// slots' (max, sum) in parallel, the warp reduces them per branch, then the
+// slots' 64-wide partial outputs are folded in 16 at a time with every load
+// of a batch issued before any is used.
 __global__ void decode_merge_kernel(const float* __restrict__ gates, bf16* __restrict__ out,
                                     Dims d, DecodeWs ws) {
   const int bg = blockIdx.x;
@@ -590,56 +457,89 @@ __global__ void decode_merge_kernel(const float* __restrict__ gates, bf16* __res
   const int cur = t / d.l;
   const int* sel = ws.idx + (size_t)bg * d.topk;
   const float* grow = gates + ((size_t)b * d.Hq + h) * 3;
-  float acc0 = 0.f, acc1 = 0.f;
-  for (int br = 0; br < 2; ++br) {
-    const bool is_sel = br == 0;
-    if (!(d.branch_mask & (is_sel ? 2 : 4))) continue;
-    const int n = is_sel ? d.topk : ws.nwin;
-    const float* base = (is_sel ? ws.psel + (size_t)bg * d.topk * 16 * kPartStride
-                                : ws.pswa + (size_t)bg * ws.nwin * 16 * kPartStride) +
-                        row * kPartStride;
-    float M = -INFINITY;
-    for (int m = lane; m < n; m += 32) {
-      const bool ok = !is_sel || (sel[m] >= 0 && sel[m] <= cur);
-      if (ok) M = fmaxf(M, base[(size_t)m * 16 * kPartStride + 64]);
+  const int nc = (d.branch_mask & 1) ? ws.nchunk : 0;
+  const int nsel = (d.branch_mask & 2) ? d.topk : 0;
+  const int nw = (d.branch_mask & 4) ? ws.nwin : 0;
+  const int ns = nc + nsel + nw;
+  auto slot_ptr = [&](int s) -> const float* {
+    if (s < nc) return ws.pcmp + ((size_t)bg * ws.nchunk + s) * 16 * kPartStride + row * kPartStride;
+    s -= nc;
+    if (s < nsel) return ws.psel + ((size_t)bg * d.topk + s) * 16 * kPartStride + row * kPartStride;
+    s -= nsel;
+    return ws.pswa + ((size_t)bg * ws.nwin + s) * 16 * kPartStride + row * kPartStride;
+  };
+  auto slot_branch = [&](int s) { return s < nc ? 0 : s < nc + nsel ? 1 : 2; };
+  auto slot_valid = [&](int s) {  // a selected slot holds a partial only for a real block
+    if (s < nc || s >= nc + nsel) return true;
+    const int j = sel[s - nc];
+    return j >= 0 && j <= cur;
+  };
+  float M0 = -INFINITY, M1 = -INFINITY, M2 = -INFINITY;
+  for (int s0 = 0; s0 < ns; s0 += 32) {
+    const int s = s0 + lane;
+    float m = -INFINITY;
+    int br = 3;
+    if (s < ns) {
+      br = slot_branch(s);
+      if (slot_valid(s)) m = slot_ptr(s)[64];
     }
-    M = warp_max(M);
-    float L = 0.f, o0 = 0.f, o1 = 0.f;
-    for (int m0 = 0; m0 < n; m0 += 32) {
-      const int m = m0 + lane;
-      float f = 0.f;
-      if (m < n) {
-        const bool ok = !is_sel || (sel[m] >= 0 && sel[m] <= cur);
-        const float mm = ok ? base[(size_t)m * 16 * kPartStride + 64] : -INFINITY;
-        f = mm == -INFINITY ? 0.f : fast_exp2(mm - M);
-        L += f * base[(size_t)m * 16 * kPartStride + 65];
-      }
-      const int cnt = min(32, n - m0);
-      // loads of every slot are issued together (all addresses are inside
-      // the workspace); slots without a partial get weight 0 and their
-      // (possibly stale) values are discarded by the select
-#pragma unroll 8
-      for (int i = 0; i < cnt; ++i) {
-        const float fi = __shfl_sync(0xffffffffu, f, i);
-        const float* pr = base + (size_t)(m0 + i) * 16 * kPartStride;
-        const float x0 = pr[lane], x1 = pr[lane + 32];
-        o0 = fi != 0.f ? fmaf(fi, x0, o0) : o0;
-        o1 = fi != 0.f ? fmaf(fi, x1, o1) : o1;
+    M0 = fmaxf(M0, warp_max(br == 0 ? m : -INFINITY));
+    M1 = fmaxf(M1, warp_max(br == 1 ? m : -INFINITY));
+    M2 = fmaxf(M2, warp_max(br == 2 ? m : -INFINITY));
+  }
+  float L0 = 0.f, L1 = 0.f, L2 = 0.f;
+  float a00 = 0.f, a01 = 0.f, a10 = 0.f, a11 = 0.f, a20 = 0.f, a21 = 0.f;
+  for (int s0 = 0; s0 < ns; s0 += 32) {
+    const int s = s0 + lane;
+    float f = 0.f;
+    int br = 3;
+    if (s < ns) {
+      br = slot_branch(s);
+      if (slot_valid(s)) {
+        const float* pr = slot_ptr(s);
+        const float m = pr[64], l = pr[65];
+        const float Mb = br == 0 ? M0 : br == 1 ? M1 : M2;
+        f = m == -INFINITY ? 0.f : fast_exp2(m - Mb);
+        if (br == 0) L0 += f * l;
+        else if (br == 1) L1 += f * l;
+        else L2 += f * l;
       }
     }
-    L = warp_sum(L);
-    const float gi = grow[is_sel ? 1 : 2] * (L > 0.f ? 1.f / L : 0.f);
-    acc0 = fmaf(gi, o0, acc0);
-    acc1 = fmaf(gi, o1, acc1);
+    const int cnt = min(32, ns - s0);
+    for (int i0 = 0; i0 < cnt; i0 += 16) {
+      float fs[16], x0[16], x1[16];
+      int bs[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        const int i = i0 + k;
+        fs[k] = __shfl_sync(0xffffffffu, f, i & 31);
+        bs[k] = __shfl_sync(0xffffffffu, br, i & 31);
+        const bool use = i < cnt && fs[k] != 0.f;
+        const float* pr = slot_ptr(s0 + i);  // inside the workspace for every i < cnt
+        x0[k] = use ? pr[lane] : 0.f;
+        x1[k] = use ? pr[lane + 32] : 0.f;
+      }
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        const float w0 = bs[k] == 0 ? fs[k] : 0.f, w1 = bs[k] == 1 ? fs[k] : 0.f,
+                    w2 = bs[k] == 2 ? fs[k] : 0.f;
+        a00 = fmaf(w0, x0[k], a00);
+        a01 = fmaf(w0, x1[k], a01);
+        a10 = fmaf(w1, x0[k], a10);
+        a11 = fmaf(w1, x1[k], a11);
+        a20 = fmaf(w2, x0[k], a20);
+        a21 = fmaf(w2, x1[k], a21);
+      }
+    }
   }
-  if (d.branch_mask & 1) {
-    const float* oc = ws.ocmp + ((size_t)bg * 16 + row) * 64;
-    acc0 = fmaf(grow[0], oc[lane], acc0);
-    acc1 = fmaf(grow[0], oc[lane + 32], acc1);
-  }
+  L0 = warp_sum(L0);
+  L1 = warp_sum(L1);
+  L2 = warp_sum(L2);
+  const float g0 = L0 > 0.f ? grow[0] / L0 : 0.f, g1 = L1 > 0.f ? grow[1] / L1 : 0.f,
+              g2 = L2 > 0.f ? grow[2] / L2 : 0.f;
   bf16* o = out + ((size_t)b * d.Hq + h) * 64;
-  o[lane] = __float2bfloat16_rn(acc0);
-  o[lane + 32] = __float2bfloat16_rn(acc1);
+  o[lane] = __float2bfloat16_rn(g0 * a00 + g1 * a10 + g2 * a20);
+  o[lane + 32] = __float2bfloat16_rn(g0 * a01 + g1 * a11 + g2 * a21);
 }
 
 int window_blocks(const Dims& d, int* jlo) {
@@ -648,50 +548,57 @@ int window_blocks(const Dims& d, int* jlo) {
   return t / d.l - *jlo + 1;
 }
 
-size_t k1_smem(const Dims& d) {
-  const int ncp = (d.Nc + 63) & ~63;
-  const size_t r0_bytes = ((size_t)ncp * 256 > 32768) ? (size_t)ncp * 256 : 32768;
-  return r0_bytes + 2048 + (8 * 16 + 32) * 4 + (size_t)ncp * 4 + ((d.Nb + 31) / 32 + 2) * 4 +
-         512 * 8 + 64 + 1024 + 64;
-}
-
 }  // namespace
 
 // Decode with the split kernels applies to bf16, block 64, G <= 16 heads per
-// group, up to 512 compressed blocks (the K1 tile) and one query.
+// group (the 16 MMA rows), up to 1024 compressed blocks (the top-k warp's
+// registers) and one query.
 bool decode_split_eligible(const Dims& d) {
-  return d.Tq == 1 && d.dtype == 1 && d.l == 64 && d.D == 64 && d.G <= 16 && d.Nc <= 512 &&
+  return d.Tq == 1 && d.dtype == 1 && d.l == 64 && d.D == 64 && d.G <= 16 && d.Nc <= 1024 &&
          tmap_encode_fn() != nullptr;
 }
+
+namespace {
+size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
+}  // namespace
 
 size_t decode_split_ws_bytes(const Dims& d) {
   int jlo;
   const int nwin = window_blocks(d, &jlo);
   const size_t bgn = (size_t)d.B * d.Hkv;
-  auto a = [](size_t x) { return (x + 255) & ~(size_t)255; };
-  return a(bgn * 16 * 64 * 4) + a(bgn * d.topk * 4) + a(bgn * d.topk * 16 * kPartStride * 4) +
-         a(bgn * nwin * 16 * kPartStride * 4);
+  const size_t nchunk = (size_t)(d.Nc + 63) / 64;
+  return al256(bgn * nchunk * 16 * kPartStride * 4) + al256(bgn * 16 * (size_t)d.Nc * 4) +
+         al256(bgn * d.topk * 4) + al256(bgn * d.topk * 16 * kPartStride * 4) +
+         al256(bgn * nwin * 16 * kPartStride * 4);
 }
 
+// K1a (chunks of the compressed cache) -> K1b (block scores, top-k) -> K2
+// (selected and window blocks) -> K3 (merge, gates), chained with
+// programmatic dependent launch: each kernel's prologue overlaps the tail of
+// the previous one, and every CTA of a dependent kernel waits for its
+// predecessor before it exits, so completion is transitive.
 cudaError_t launch_decode_split(const Dims& d, const void* q, const void* kcache,
                                 const void* vcache, const void* kc, const void* vc,
                                 const float* gates, void* out, int32_t* idx_out, void* ws_ptr,
                                 int* err, cudaStream_t s) {
   DecodeWs ws;
   ws.nwin = window_blocks(d, &ws.jlo);
+  ws.nchunk = (d.Nc + 63) / 64;
   const size_t bgn = (size_t)d.B * d.Hkv;
-  auto a = [](size_t x) { return (x + 255) & ~(size_t)255; };
   char* w = (char*)ws_ptr;
-  ws.ocmp = (float*)w;
-  w += a(bgn * 16 * 64 * 4);
+  ws.pcmp = (float*)w;
+  w += al256(bgn * ws.nchunk * 16 * kPartStride * 4);
+  ws.logit = (float*)w;
+  w += al256(bgn * 16 * (size_t)d.Nc * 4);
   ws.idx = (int*)w;
-  w += a(bgn * d.topk * 4);
+  w += al256(bgn * d.topk * 4);
   ws.psel = (float*)w;
-  w += a(bgn * d.topk * 16 * kPartStride * 4);
+  w += al256(bgn * d.topk * 16 * kPartStride * 4);
   ws.pswa = (float*)w;
   const bool cmp = d.branch_mask & 1, sel = d.branch_mask & 2, swa = d.branch_mask & 4;
   CUtensorMap mkc{}, mvc{}, mk, mv;
-  if (d.Nc > 0 && (cmp || sel)) {
+  const bool k1 = d.Nc > 0 && (cmp || sel);
+  if (k1) {
     if (!make_tmap_bf16(&mkc, kc, d.Hkv, (long)d.B * d.Nc, 1, 64) ||
         !make_tmap_bf16(&mvc, vc, d.Hkv, (long)d.B * d.Nc, 1, 64))
       return cudaErrorInvalidValue;
@@ -699,19 +606,27 @@ cudaError_t launch_decode_split(const Dims& d, const void* q, const void* kcache
   if (!make_tmap_bf16(&mk, kcache, d.Hkv, (long)d.B * d.T, 1, 64) ||
       !make_tmap_bf16(&mv, vcache, d.Hkv, (long)d.B * d.T, 1, 64))
     return cudaErrorInvalidValue;
-  if (cmp || sel) {
-    const size_t smem = k1_smem(d);
-    cudaError_t e = cudaFuncSetAttribute(decode_cmp_topk_kernel,
-                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    decode_cmp_topk_kernel<<<(unsigned)bgn, kK1Threads, smem, s>>>(
-        mkc, mvc, (const bf16*)q, d, ws, idx_out, cmp ? 1 : 0, sel ? 1 : 0, err);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
   cudaLaunchAttribute pdl[1];
   pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  const bf16* qb = (const bf16*)q;
+  if (k1) {
+    decode_cmp_chunk_kernel<<<dim3(ws.nchunk, d.Hkv, d.B), 32, 0, s>>>(mkc, mvc, qb, d, ws,
+                                                                      cmp ? 1 : 0, err);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if (sel) {  // also when no block is complete yet: the forced blocks still go out
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)bgn);
+    cfg.blockDim = dim3(256);
+    cfg.stream = s;
+    cfg.attrs = pdl;
+    cfg.numAttrs = 1;
+    cudaError_t e = d.Nc <= 512 ? cudaLaunchKernelEx(&cfg, decode_topk_kernel<16>, d, ws, idx_out)
+                                : cudaLaunchKernelEx(&cfg, decode_topk_kernel<32>, d, ws, idx_out);
+    if (e != cudaSuccess) return e;
+  }
   if (sel || swa) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(ws.nwin + d.topk, d.Hkv, d.B);
@@ -719,7 +634,6 @@ cudaError_t launch_decode_split(const Dims& d, const void* q, const void* kcache
     cfg.stream = s;
     cfg.attrs = pdl;
     cfg.numAttrs = 1;
-    const bf16* qb = (const bf16*)q;
     const int ds = sel ? 1 : 0, dw = swa ? 1 : 0;
     cudaError_t e = cudaLaunchKernelEx(&cfg, decode_block_kernel, mk, mv, qb, d, ws, ds, dw, err);
     if (e != cudaSuccess) return e;

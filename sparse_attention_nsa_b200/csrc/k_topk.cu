@@ -9,26 +9,15 @@
 // 1..cur-1 are added, equal scores going to the lower block index.  The
 // output is ascending and padded with -1.
 //
-// One warp per row, no shared memory.  Lane `lane` holds the candidates
-// 1 + lane + 32 q in registers as order-preserving integer keys.  A radix
-// select finds tau, the (topk-2)-th largest key, bit by bit from the top
-// (each step one warp-wide count with redux.sync).  The winners are every
-// key above tau plus, among keys equal to tau, the lowest block indices
-// (ballots in ascending block order); they are written out in ascending
-// order between the forced blocks 0 and cur.
+// One warp per row, no shared memory: the radix select of topk.cuh over the
+// row's fp32 scores read straight from global memory.
 #include "common.cuh"
 #include "internal.h"
+#include "topk.cuh"
 
 namespace nsa {
 
 constexpr int kTopkWarps = 8;
-
-// Monotone map of a float to uint32 (larger float -> larger key); NaN -> 0.
-__device__ __forceinline__ uint32_t order_key(float x) {
-  if (x != x) return 0u;
-  const uint32_t u = __float_as_uint(x);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
 
 template <int QMAX>
 __global__ void __launch_bounds__(kTopkWarps * 32)
@@ -39,53 +28,8 @@ topk_kernel(const float* __restrict__ score, int32_t* __restrict__ idx, Dims d) 
   if (r >= nrows) return;
   const int tq = (int)((r / d.Hkv) % d.Tq);
   const int t = d.q_off + tq;
-  const int cur = t / d.l;
-  int32_t* out = idx + r * d.topk;
-  if (cur + 1 <= d.topk) {
-    for (int s = lane; s < d.topk; s += 32) out[s] = s <= cur ? s : -1;
-    return;
-  }
   // candidates are blocks 1..cur-1 (all complete, so all have scores)
-  const float* sr = score + r * d.Nc;
-  uint32_t key[QMAX];
-#pragma unroll
-  for (int q = 0; q < QMAX; ++q) {
-    const int j = 1 + lane + 32 * q;
-    key[q] = j < cur ? order_key(__ldg(sr + j)) : 0u;
-  }
-  const int K2 = d.topk - 2;
-  // tau = the largest value with at least K2 keys >= tau (absent slots are
-  // excluded from the counts)
-  uint32_t tau = 0u;
-  for (int bit = 31; bit >= 0; --bit) {
-    const uint32_t tc = tau | (1u << bit);
-    unsigned c = 0;
-#pragma unroll
-    for (int q = 0; q < QMAX; ++q) c += (1 + lane + 32 * q < cur && key[q] >= tc) ? 1u : 0u;
-    if ((int)__reduce_add_sync(0xffffffffu, c) >= K2) tau = tc;
-  }
-  unsigned cg = 0;
-#pragma unroll
-  for (int q = 0; q < QMAX; ++q) cg += (1 + lane + 32 * q < cur && key[q] > tau) ? 1u : 0u;
-  const int need = K2 - (int)__reduce_add_sync(0xffffffffu, cg);  // >= 1 keys equal to tau
-  int eq_before = 0, pos = 1;
-  const unsigned lt = (1u << lane) - 1u;
-#pragma unroll
-  for (int q = 0; q < QMAX; ++q) {
-    const int j = 1 + lane + 32 * q;
-    const bool ok = j < cur;
-    const bool eq = ok && key[q] == tau;
-    const unsigned em = __ballot_sync(0xffffffffu, eq);
-    const bool win = ok && (key[q] > tau || (eq && eq_before + __popc(em & lt) < need));
-    const unsigned wm = __ballot_sync(0xffffffffu, win);
-    if (win) out[pos + __popc(wm & lt)] = j;
-    pos += __popc(wm);
-    eq_before += __popc(em);
-  }
-  if (lane == 0) {
-    out[0] = 0;
-    out[K2 + 1] = cur;
-  }
+  warp_select_blocks<QMAX>(score + r * d.Nc, t / d.l, d.topk, idx + r * d.topk, lane);
 }
 
 cudaError_t launch_topk(const Dims& d, const float* score, int32_t* idx,

@@ -25,8 +25,8 @@ namespace nsa {
 nsa_status decode_scratch_bytes(const nsa_params* p, bool idx_given, size_t* bytes);
 }
 
-// Fixed scratch for nsa_decode_noalloc: 8 MiB per device.
-static constexpr size_t kNoAllocScratchBytes = (size_t)8 << 20;
+// Fixed scratch for nsa_decode_noalloc: 16 MiB per device.
+static constexpr size_t kNoAllocScratchBytes = (size_t)16 << 20;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 namespace {

@@ -52,8 +52,8 @@ def test_noalloc_decode_matches_workspace_decode(cuda_lib, w):
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch(cuda_lib):
-    assert nsa.nsa_decode_noalloc_max_scratch() == 8 << 20
-    # 4096 sequences x 16 heads: the per-block partials alone exceed 8 MiB
+    assert nsa.nsa_decode_noalloc_max_scratch() == 16 << 20
+    # 4096 sequences x 16 heads: the per-block partials alone exceed 16 MiB
     p = nsa.make_params(4096, 32768, 16, 1, Tq=1)
     ptr = C.c_void_p(1 << 20)  # never dereferenced: rejected before launch
     st = nsa.load().nsa_decode_noalloc(C.byref(p), ptr, ptr, ptr, ptr, ptr, ptr, ptr, None, None)
