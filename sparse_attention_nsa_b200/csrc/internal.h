@@ -59,6 +59,11 @@ cudaError_t launch_gate_bwd(const Dims& d, const float* gates, const void* dout,
 cudaError_t launch_dq(const Dims& d, int mode, const void* q, const void* keys,
                       const void* vals, const int32_t* idx, const void* o, const float* lse,
                       const float* dO, float* dq, float* delta, int* err, cudaStream_t s);
+// tensor-core dQ pass (k_bwd_tc.cu); modes 0 selection, 1 window
+bool dq_tc_eligible(const Dims& d, int mode);
+cudaError_t launch_dq_tc(const Dims& d, int mode, const void* q, const void* keys,
+                         const void* vals, const int32_t* idx, const void* o, const float* lse,
+                         const float* dO, float* dq, float* delta, int* err, cudaStream_t s);
 cudaError_t launch_revmap(const Dims& d, const int32_t* idx, int* counts, int* offsets,
                           int* list, cudaStream_t s);
 cudaError_t launch_dkdv(const Dims& d, int mode, const void* q, const void* keys,

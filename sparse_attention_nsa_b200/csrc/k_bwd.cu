@@ -414,6 +414,8 @@ static cudaError_t dq_t(const Dims& d, const void* q, const void* keys, const vo
 cudaError_t launch_dq(const Dims& d, int mode, const void* q, const void* keys, const void* vals,
                       const int32_t* idx, const void* o, const float* lse, const float* dO,
                       float* dq, float* delta, int* err, cudaStream_t s) {
+  if (dq_tc_eligible(d, mode))
+    return launch_dq_tc(d, mode, q, keys, vals, idx, o, lse, dO, dq, delta, err, s);
   if (d.dtype == 1) {
     if (mode == kBwdSel) return dq_t<bf16, kBwdSel>(d, q, keys, vals, idx, o, lse, dO, dq, delta, err, s);
     if (mode == kBwdSwa) return dq_t<bf16, kBwdSwa>(d, q, keys, vals, idx, o, lse, dO, dq, delta, err, s);
