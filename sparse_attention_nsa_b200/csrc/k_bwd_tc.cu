@@ -386,6 +386,393 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   }
 }
 
+// ---- pass 2: dK, dV, key-stationary, on tensor cores --------------------------------
+// One CTA per (pair of 64-key blocks j0 = 2p, j1 = 2p+1, KV group, sequence):
+// M = 128 keys.  The query rows that attend those keys are streamed in
+// tiles of 128 rows (128/G tokens x G heads), gathered by four producer
+// warps into a double-buffered, 128-byte-swizzled Q tile and dO tile (dO
+// rounded to bf16).  Selection: the reverse-map lists of j0 and then of j1
+// (a row of j0's list only reaches the first 64 keys, and so on); window:
+// the contiguous range of tokens whose windows reach the pair.  Per tile:
+//   S^T = K Q^T, dP^T = V dO^T   (M128 N128 K64, fp32 in TMEM)
+//   key threads: P^T, dS^T into TMEM (one thread per key)
+//   dV += P^T dO, dK += dS^T Q   (M128 N64 K128, A from TMEM, B = the
+//                                 gathered tiles read MN-major)
+// Precision: dK and dV sum over many query rows, so the bf16 rounding of a
+// single operand (2^-9 relative) would show in them.  dO enters dP^T as a
+// bf16 pair hi + lo (two MMAs), dS enters dK as hi (TMEM) + lo (shared
+// memory), and dV takes P and dO in fp16 (2^-11): the products keep about
+// fp32 accuracy for dK and four times bf16's for dV, with operands whose
+// range is bounded (P in [0, 1]; dO a gradient).
+// TMEM (512 columns, one CTA per SM): S^T [0,128), dP^T [128,256),
+// dV [256,320), dK [320,384), P^T (fp16) [384,448), dS^T hi [448,512).
+// Warps: 0-3 key threads and epilogue, 4 MMA issue and TMEM owner (and the
+// K/V TMA), 5-8 row gather.
+constexpr int kKvThreads = 288;
+constexpr uint32_t kKTile2 = 128 * 64 * 2;  // 128 keys x 64 dims, bf16
+constexpr uint32_t kRowTile = 128 * 64 * 2;
+
+constexpr uint32_t kvColS = 0, kvColDP = 128, kvColDV = 256, kvColDK = 320, kvColP = 384,
+                   kvColDS = 448;
+
+struct KvRowInfo {
+  float lse2[128];
+  float delta[128];
+  int tpos[128];   // key position of the row's query
+  int blkmask[128];  // selection: 1 << (block - j0) the row's list belongs to; 0 = no row
+};
+
+constexpr uint32_t KV_OFF_K = 0;
+constexpr uint32_t KV_OFF_V = KV_OFF_K + kKTile2;
+constexpr uint32_t KV_OFF_Q = KV_OFF_V + kKTile2;           // 2 buffers each:
+constexpr uint32_t KV_OFF_DO = KV_OFF_Q + 2 * kRowTile;     //   dO hi (bf16)
+constexpr uint32_t KV_OFF_DOL = KV_OFF_DO + 2 * kRowTile;   //   dO lo (bf16)
+constexpr uint32_t KV_OFF_DOH = KV_OFF_DOL + 2 * kRowTile;  //   dO (fp16)
+constexpr uint32_t KV_OFF_DSL = KV_OFF_DOH + 2 * kRowTile;  // dS^T lo, 128 keys x 128 rows
+constexpr uint32_t KV_OFF_INFO = KV_OFF_DSL + 2 * kKTile2;  // 2 x KvRowInfo
+constexpr uint32_t KV_OFF_BAR = KV_OFF_INFO + 2 * sizeof(KvRowInfo);
+
+struct KvBars {
+  uint64_t kv;          // K and V of the pair landed (TMA)
+  uint64_t gathered[2]; // 128 gather threads filled row buffer u & 1
+  uint64_t s;           // S^T and dP^T of the current tile are in TMEM
+  uint64_t sfree;       // 128 key threads loaded them
+  uint64_t p;           // 128 key threads wrote P^T and dS^T
+  uint64_t bfree[2];    // dV / dK MMAs of the tile in row buffer u & 1 done
+  uint64_t fin;
+};
+constexpr uint32_t KV_OFF_MISC = KV_OFF_BAR + ((sizeof(KvBars) + 15) / 16) * 16;
+constexpr uint32_t KV_SMEM = KV_OFF_MISC + 16;
+
+// Rows of one tile: row index within the CTA's row list -> (query index tq
+// or -1, list bit).  Selection lists: j0's tokens then j1's, G rows each.
+__device__ __forceinline__ int kv_row_token(bool sel, long rix, int G, int n0, int n1,
+                                           const int* l0, const int* l1, int tq_lo, int ntok,
+                                           int* bit) {
+  const long ti = rix / G;
+  if (sel) {
+    if (ti < n0) {
+      *bit = 1;
+      return l0[ti];
+    }
+    if (ti < (long)n0 + n1) {
+      *bit = 2;
+      return l1[ti - n0];
+    }
+    *bit = 0;
+    return -1;
+  }
+  *bit = 3;
+  return ti < ntok ? tq_lo + (int)ti : -1;
+}
+
+template <bool SEL>
+__global__ void __launch_bounds__(kKvThreads, 1)
+bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                   const bf16* __restrict__ q, const float* __restrict__ lse,
+                   const float* __restrict__ delta, const float* __restrict__ dO,
+                   const int* __restrict__ offsets, const int* __restrict__ list,
+                   float* __restrict__ dk, float* __restrict__ dv, Dims d, int* err) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  KvBars* bars = (KvBars*)(smem + KV_OFF_BAR);
+  KvRowInfo* info = (KvRowInfo*)(smem + KV_OFF_INFO);
+  uint32_t* tmem_slot = (uint32_t*)(smem + KV_OFF_MISC);
+  volatile int* abort_flag = (volatile int*)(smem + KV_OFF_MISC + 4);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
+  const int pr = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int j0 = 2 * pr;
+  const int kbase = j0 * kKeys;  // first key of the pair
+
+  // the rows of this CTA
+  int n0 = 0, n1 = 0, tq_lo = 0, ntok = 0;
+  const int* l0 = nullptr;
+  const int* l1 = nullptr;
+  if (SEL) {
+    const size_t bg = (size_t)b * d.Hkv + g;
+    const int* off = offsets + bg * (d.Nb + 1);
+    l0 = list + bg * (size_t)d.Tq * d.topk + off[j0];
+    n0 = off[j0 + 1] - off[j0];
+    if (j0 + 1 < d.Nb) {
+      l1 = list + bg * (size_t)d.Tq * d.topk + off[j0 + 1];
+      n1 = off[j0 + 2] - off[j0 + 1];
+    }
+  } else {
+    const int t_lo = kbase, t_hi = min(kbase + 2 * kKeys - 1 + d.window - 1, d.T - 1);
+    tq_lo = max(0, t_lo - d.q_off);
+    ntok = max(0, t_hi - d.q_off - tq_lo + 1);
+  }
+  const long nrows = SEL ? ((long)n0 + n1) * d.G : (long)ntok * d.G;
+  const int ntiles = (int)((nrows + 127) / 128);
+
+  if (tid == 0) {
+    mbar_init(&bars->kv, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars->gathered[i], 128);
+      mbar_init(&bars->bfree[i], 1);
+    }
+    mbar_init(&bars->s, 1);
+    mbar_init(&bars->sfree, 128);
+    mbar_init(&bars->p, 128);
+    mbar_init(&bars->fin, 1);
+    fence_barrier_init();
+    fence_proxy_async_smem();
+    *abort_flag = 0;
+  }
+  if (warp == 4) tmem_alloc(tmem_slot, 512);
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp >= 5) {
+    // ---- row gather: thread gr fills row gr of each tile ------------------------------
+    const int gr = tid - 160;
+    for (int u = 0; u < ntiles; ++u) {
+      const int bu = u & 1;
+      if (u >= 2 && !wait_bar(&bars->bfree[bu], ((u - 2) >> 1) & 1, abort_flag, err)) break;
+      const long rix = (long)u * 128 + gr;
+      int bit = 0;
+      const int tq =
+          rix < nrows ? kv_row_token(SEL, rix, d.G, n0, n1, l0, l1, tq_lo, ntok, &bit) : -1;
+      const int hh = (int)(rix % d.G);
+      const bool ok = tq >= 0 && tq < d.Tq;
+      const size_t row = ((size_t)b * d.Tq + (ok ? tq : 0)) * d.Hq + (size_t)g * d.G + hh;
+      const uint32_t off = (uint32_t)(gr >> 3) * 1024u + (uint32_t)(gr & 7) * 128u;
+      const uint32_t qrow = smem_u32(smem + KV_OFF_Q + bu * kRowTile) + off;
+      const uint32_t drow = smem_u32(smem + KV_OFF_DO + bu * kRowTile) + off;
+      const uint32_t lrow = smem_u32(smem + KV_OFF_DOL + bu * kRowTile) + off;
+      const uint32_t hrow = smem_u32(smem + KV_OFF_DOH + bu * kRowTile) + off;
+      float l2 = -INFINITY;
+      if (ok) l2 = lse[row] * kLog2e;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint4 qv = make_uint4(0u, 0u, 0u, 0u);
+        uint32_t w[4] = {0u, 0u, 0u, 0u}, wl[4] = {0u, 0u, 0u, 0u}, wh[4] = {0u, 0u, 0u, 0u};
+        if (ok) {
+          qv = __ldg(reinterpret_cast<const uint4*>(q + row * 64) + c);
+          const float4 a = __ldg(reinterpret_cast<const float4*>(dO + row * 64) + 2 * c);
+          const float4 a2 = __ldg(reinterpret_cast<const float4*>(dO + row * 64) + 2 * c + 1);
+          const float x[8] = {a.x, a.y, a.z, a.w, a2.x, a2.y, a2.z, a2.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float h0 = __bfloat162float(__float2bfloat16_rn(x[2 * e]));
+            const float h1 = __bfloat162float(__float2bfloat16_rn(x[2 * e + 1]));
+            w[e] = pack_bf16(h0, h1);
+            wl[e] = pack_bf16(x[2 * e] - h0, x[2 * e + 1] - h1);
+            wh[e] = pack_f16(x[2 * e], x[2 * e + 1]);
+          }
+        }
+        const uint32_t sw = (uint32_t)(c ^ (gr & 7)) << 4;
+        st_shared_v4(qrow + sw, qv.x, qv.y, qv.z, qv.w);
+        st_shared_v4(drow + sw, w[0], w[1], w[2], w[3]);
+        st_shared_v4(lrow + sw, wl[0], wl[1], wl[2], wl[3]);
+        st_shared_v4(hrow + sw, wh[0], wh[1], wh[2], wh[3]);
+      }
+      KvRowInfo& in = info[bu];
+      in.lse2[gr] = l2;
+      in.delta[gr] = ok ? delta[row] : 0.f;
+      in.tpos[gr] = d.q_off + (ok ? tq : 0);
+      in.blkmask[gr] = (ok && l2 != -INFINITY) ? bit : 0;
+      fence_proxy_async_smem();
+      mbar_arrive(&bars->gathered[bu]);
+    }
+  } else if (warp == 4) {
+    // ---- MMA issue (and the pair's K/V by TMA) ----------------------------------------
+    if (lane == 0) {
+      constexpr uint32_t idesc_st = idesc_bf16(128, 128, false, false);  // S^T, dP^T
+      constexpr uint32_t idesc_kv = idesc_bf16(128, 64, false, true);    // dK (hi)
+      constexpr uint32_t idesc_kl = idesc_bf16(128, 64, false, true);    // dK (lo, A from smem)
+      constexpr uint32_t idesc_v16 = idesc_f16(128, 64, false, true);    // dV (fp16)
+      const uint32_t dsl_addr = smem_u32(smem + KV_OFF_DSL);
+      const uint32_t k_addr = smem_u32(smem + KV_OFF_K), v_addr = smem_u32(smem + KV_OFF_V);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      mbar_expect_tx(&bars->kv, 2 * kKTile2);
+      for (int h = 0; h < 2; ++h) {
+        tma_load_3d(smem + KV_OFF_K + h * kTileBytes, &tm_k, &bars->kv, 0, g, b * d.T + kbase + h * kKeys);
+        tma_load_3d(smem + KV_OFF_V + h * kTileBytes, &tm_v, &bars->kv, 0, g, b * d.T + kbase + h * kKeys);
+      }
+      bool ok = wait_bar(&bars->kv, 0, abort_flag, err);
+      auto issue_kv = [&](int u) -> bool {
+        // dV += P^T dO and dK += dS^T Q of tile u (A operands in TMEM, the
+        // gathered tiles read MN-major: K dimension = rows)
+        if (!wait_bar(&bars->p, u & 1, abort_flag, err)) return false;
+        tc_fence_after();
+        const int bu = u & 1;
+        const uint32_t q_addr = smem_u32(smem + KV_OFF_Q + bu * kRowTile);
+        const uint32_t doh_addr = smem_u32(smem + KV_OFF_DOH + bu * kRowTile);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t acc = (u > 0 || kk > 0) ? 1u : 0u;
+          const uint64_t qb = desc_sw128(q_addr + kk * 2048, 8192);
+          mma_bf16_ts(tmem + kvColDV, tmem + kvColP + kk * 8,
+                      desc_sw128(doh_addr + kk * 2048, 8192), idesc_v16, acc);
+          mma_bf16_ts(tmem + kvColDK, tmem + kvColDS + kk * 8, qb, idesc_kv, acc);
+          // dS^T lo: 128 keys x 128 rows, K-major, two 64-row swizzle atoms
+          mma_bf16(tmem + kvColDK, desc_sw128(dsl_addr + (kk >> 2) * kKTile2 + (kk & 3) * 32, 16),
+                   qb, idesc_kl, 1u);
+        }
+        mma_commit(&bars->bfree[bu]);  // frees the row buffer and the P^T / dS^T columns
+        return true;
+      };
+      for (int u = 0; ok && u < ntiles; ++u) {
+        const int bu = u & 1;
+        if (!wait_bar(&bars->gathered[bu], (u >> 1) & 1, abort_flag, err)) break;
+        // S^T / dP^T are single-buffered: the key threads must have loaded tile u-1's
+        if (u >= 1 && !wait_bar(&bars->sfree, (u - 1) & 1, abort_flag, err)) break;
+        tc_fence_after();
+        const uint32_t q_addr = smem_u32(smem + KV_OFF_Q + bu * kRowTile);
+        const uint32_t do_addr = smem_u32(smem + KV_OFF_DO + bu * kRowTile);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmem + kvColS, desc_sw128(k_addr + kk * 32, 16), desc_sw128(q_addr + kk * 32, 16),
+                   idesc_st, kk > 0);
+        const uint32_t dol_addr = smem_u32(smem + KV_OFF_DOL + bu * kRowTile);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmem + kvColDP, desc_sw128(v_addr + kk * 32, 16), desc_sw128(do_addr + kk * 32, 16),
+                   idesc_st, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)  // dO lo: dP^T keeps about fp32 accuracy
+          mma_bf16(tmem + kvColDP, desc_sw128(v_addr + kk * 32, 16), desc_sw128(dol_addr + kk * 32, 16),
+                   idesc_st, 1u);
+        mma_commit(&bars->s);
+        if (u >= 1 && !issue_kv(u - 1)) break;
+        if (u == ntiles - 1) issue_kv(u);
+      }
+      mma_commit(&bars->fin);
+      drain_bar(&bars->fin, 0);
+      if (!ok) drain_bar(&bars->kv, 0);
+    }
+  } else {
+    // ---- key threads: thread k owns key kbase + k (TMEM lane k) -------------------------
+    const int k = tid;
+    const int key = kbase + k;
+    const int kbit = 1 << (k >> 6);  // which block of the pair
+    const uint32_t lane_tmem = tmem + ((uint32_t)(warp * 32) << 16);
+    const float sl2 = d.scale * kLog2e;
+    bool ok = true;
+    for (int u = 0; u < ntiles; ++u) {
+      const KvRowInfo& in = info[u & 1];
+      if (!wait_bar_warp(&bars->s, u & 1, abort_flag, err)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      // P^T / dS^T (TMEM and the dS lo tile): the dV/dK MMAs of tile u-1 must have read them
+      if (u >= 1) {
+        if (!wait_bar_warp(&bars->bfree[(u - 1) & 1], ((u - 1) >> 1) & 1, abort_flag, err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+      }
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {  // 32 rows at a time
+        float sv[32], pv[32];
+        tmem_ld32(lane_tmem + kvColS + 32u * c, sv);
+        tmem_ld32(lane_tmem + kvColDP + 32u * c, pv);
+        tmem_wait_ld();
+        if (c == 3) {  // S^T and dP^T of this tile are in registers: release them
+          tc_fence_before();
+          mbar_arrive(&bars->sfree);
+        }
+        uint32_t pp[16], dd[16], dl[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float p2[2], d2[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int r = 32 * c + e + h;
+            const int t = in.tpos[r];
+            bool vis = (in.blkmask[r] & kbit) && key <= t;
+            if (!SEL) vis = vis && key >= t - d.window + 1;
+            const float pr = vis ? fast_exp2(fmaf(sv[e + h], sl2, -in.lse2[r])) : 0.f;
+            p2[h] = pr;
+            d2[h] = pr * (pv[e + h] - in.delta[r]);
+          }
+          const float h0 = __bfloat162float(__float2bfloat16_rn(d2[0]));
+          const float h1 = __bfloat162float(__float2bfloat16_rn(d2[1]));
+          pp[e / 2] = pack_f16(p2[0], p2[1]);
+          dd[e / 2] = pack_bf16(h0, h1);
+          dl[e / 2] = pack_bf16(d2[0] - h0, d2[1] - h1);
+        }
+        tmem_st16u(lane_tmem + kvColP + 16u * c, pp);
+        tmem_st16u(lane_tmem + kvColDS + 16u * c, dd);
+        // dS lo into the K-major smem tile: row k, rows 32c .. 32c+31 of the
+        // tile are 16-byte chunks 4(c&1) .. 4(c&1)+3 of swizzle atom c >> 1
+        const uint32_t lrow = smem_u32(smem + KV_OFF_DSL) + (uint32_t)(c >> 1) * kKTile2 +
+                              (uint32_t)(k >> 3) * 1024u + (uint32_t)(k & 7) * 128u;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const int cc = 4 * (c & 1) + q4;
+          st_shared_v4(lrow + ((uint32_t)(cc ^ (k & 7)) << 4), dl[4 * q4], dl[4 * q4 + 1],
+                       dl[4 * q4 + 2], dl[4 * q4 + 3]);
+        }
+      }
+      fence_proxy_async_smem();  // dS lo is read by the MMA (async proxy)
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars->p);
+    }
+    // epilogue: dk += scale * dK, dv += dV for this key (fp32, accumulated)
+    bool have = false;
+    if (ok && ntiles > 0) have = wait_bar_warp(&bars->fin, 0, abort_flag, err);
+    float a[32];
+    const size_t krow = ((size_t)b * d.T + key) * d.Hkv * 64 + (size_t)g * 64;
+    const bool kin = key < d.T;
+#pragma unroll 1
+    for (int h = 0; h < 4; ++h) {  // dV [0,64), dK [64,128) in halves of 32
+      if (have) {
+        tc_fence_after();
+        tmem_ld32(lane_tmem + kvColDV + 32u * h, a);
+        tmem_wait_ld();
+      }
+      if (have && kin) {
+        float* dst = (h < 2 ? dv : dk) + krow + 32 * (h & 1);
+        const float sc = h < 2 ? 1.f : d.scale;
+#pragma unroll
+        for (int c = 0; c < 32; c += 4) {
+          float4 x = *reinterpret_cast<float4*>(dst + c);
+          x.x = fmaf(a[c], sc, x.x);
+          x.y = fmaf(a[c + 1], sc, x.y);
+          x.z = fmaf(a[c + 2], sc, x.z);
+          x.w = fmaf(a[c + 3], sc, x.w);
+          *reinterpret_cast<float4*>(dst + c) = x;
+        }
+      }
+    }
+    tc_fence_before();
+  }
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <bool SEL>
+cudaError_t launch_dkdv_tc_t(const Dims& d, const void* q, const void* k, const void* v,
+                             const float* lse, const float* delta, const float* dO,
+                             const int* offsets, const int* list, float* dk, float* dv, int* err,
+                             cudaStream_t s) {
+  const int npairs = (d.Nb + 1) / 2;
+  if (npairs == 0) return cudaSuccess;
+  CUtensorMap mk, mv;
+  if (!make_tmap_bf16(&mk, k, d.Hkv, (long)d.B * d.T, 1, kKeys) ||
+      !make_tmap_bf16(&mv, v, d.Hkv, (long)d.B * d.T, 1, kKeys))
+    return cudaErrorInvalidValue;
+  // 512 TMEM columns per CTA: ask for enough shared memory that a second CTA
+  // never shares the SM (it would wait in tcgen05.alloc)
+  const size_t smem = KV_SMEM + 1024 > 120 * 1024 ? KV_SMEM + 1024 : 120 * 1024;
+  cudaError_t e = cudaFuncSetAttribute(bwd_dkdv_tc_kernel<SEL>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  bwd_dkdv_tc_kernel<SEL><<<dim3(npairs, d.Hkv, d.B), kKvThreads, smem, s>>>(
+      mk, mv, (const bf16*)q, lse, delta, dO, offsets, list, dk, dv, d, err);
+  return cudaGetLastError();
+}
+
 template <bool SEL>
 cudaError_t launch_dq_tc_t(const Dims& d, const void* q, const void* k, const void* v,
                            const int32_t* idx, const void* o, const float* lse, const float* dO,
@@ -412,6 +799,18 @@ cudaError_t launch_dq_tc_t(const Dims& d, const void* q, const void* k, const vo
 bool dq_tc_eligible(const Dims& d, int mode) {
   return mode != 2 && d.dtype == 1 && d.l == kKeys && d.D == 64 && d.G >= 1 &&
          kRows % d.G == 0 && d.Nb <= 4096 && tmap_encode_fn() != nullptr;
+}
+
+// Tensor-core dK/dV: the same geometry (key-stationary over pairs of blocks).
+bool dkdv_tc_eligible(const Dims& d, int mode) { return dq_tc_eligible(d, mode); }
+
+cudaError_t launch_dkdv_tc(const Dims& d, int mode, const void* q, const void* k, const void* v,
+                           const float* lse, const float* delta, const float* dO,
+                           const int* offsets, const int* list, float* dk, float* dv, int* err,
+                           cudaStream_t s) {
+  return mode == 0
+             ? launch_dkdv_tc_t<true>(d, q, k, v, lse, delta, dO, offsets, list, dk, dv, err, s)
+             : launch_dkdv_tc_t<false>(d, q, k, v, lse, delta, dO, offsets, list, dk, dv, err, s);
 }
 
 cudaError_t launch_dq_tc(const Dims& d, int mode, const void* q, const void* k, const void* v,

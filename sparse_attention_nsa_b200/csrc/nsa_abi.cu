@@ -481,7 +481,7 @@ nsa_status sel_bwd_body(const Dims& d, const void* q, const void* k, const void*
   int* list = (int*)(w + c.list);
   NSA_TRY_CUDA(nsa::launch_dq(d, 0, q, k, v, idx, o_sel, lse_sel, dO_sel, dq, delta, err_word(), s));
   NSA_TRY_CUDA(nsa::launch_revmap(d, idx, counts, offsets, list, s));
-  NSA_TRY_CUDA(nsa::launch_dkdv(d, 0, q, k, v, lse_sel, delta, dO_sel, offsets, list, dk, dv, s));
+  NSA_TRY_CUDA(nsa::launch_dkdv(d, 0, q, k, v, lse_sel, delta, dO_sel, offsets, list, dk, dv, err_word(), s));
   return NSA_OK;
 }
 
@@ -491,7 +491,7 @@ nsa_status swa_bwd_body(const Dims& d, const void* q, const void* k, const void*
                         cudaStream_t s) {
   float* delta = (float*)(w + c.delta);
   NSA_TRY_CUDA(nsa::launch_dq(d, 1, q, k, v, nullptr, o_swa, lse_swa, dO_swa, dq, delta, nullptr, s));
-  NSA_TRY_CUDA(nsa::launch_dkdv(d, 1, q, k, v, lse_swa, delta, dO_swa, nullptr, nullptr, dk, dv, s));
+  NSA_TRY_CUDA(nsa::launch_dkdv(d, 1, q, k, v, lse_swa, delta, dO_swa, nullptr, nullptr, dk, dv, err_word(), s));
   return NSA_OK;
 }
 
@@ -507,7 +507,7 @@ nsa_status cmp_bwd_body(const Dims& d, const void* q, const void* kc, const void
   NSA_TRY_CUDA(cudaMemsetAsync(dkc, 0, nkc, s));
   NSA_TRY_CUDA(cudaMemsetAsync(dvc, 0, nkc, s));
   NSA_TRY_CUDA(nsa::launch_dq(d, 2, q, kc, vc, nullptr, o_cmp, lse_cmp, dO_cmp, dq, delta, nullptr, s));
-  NSA_TRY_CUDA(nsa::launch_dkdv(d, 2, q, kc, vc, lse_cmp, delta, dO_cmp, nullptr, nullptr, dkc, dvc, s));
+  NSA_TRY_CUDA(nsa::launch_dkdv(d, 2, q, kc, vc, lse_cmp, delta, dO_cmp, nullptr, nullptr, dkc, dvc, err_word(), s));
   NSA_TRY_CUDA(nsa::launch_pool_bwd(d, dkc, dvc, dk, dv, s));
   return NSA_OK;
 }
