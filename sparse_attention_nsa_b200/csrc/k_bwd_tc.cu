@@ -70,16 +70,21 @@ __host__ __device__ inline size_t list_ints(const Dims& d) {
   return (size_t)d.Nb + words + (size_t)tokens_per_tile(d.G) * (d.topk + 1);
 }
 
-template <bool SEL>
+// MODE 0 selection, 1 window, 2 compression (keys = the compressed cache;
+// key c is visible to the query at t when its block is complete:
+// (c + 1) l - 1 <= t).
+template <int MODE>
 __global__ void __launch_bounds__(kThreads, 2)
 bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const bf16* __restrict__ o,
                  const float* __restrict__ lse, const float* __restrict__ dO,
                  const int32_t* __restrict__ idx, float* __restrict__ dq,
                  float* __restrict__ delta, Dims d, int* err) {
+  constexpr bool SEL = MODE == 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   Bars* bars = (Bars*)(smem + OFF_BAR);
+  const int nkeys = MODE == 2 ? d.Nc : d.T;  // key rows per sequence
   uint32_t* tmem_slot = (uint32_t*)(smem + OFF_MISC);
   volatile int* abort_flag = (volatile int*)(smem + OFF_MISC + 4);
   int* nblk_s = (int*)(smem + OFF_MISC + 8);
@@ -169,10 +174,15 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
   } else if (tid == 0) {
     const int tlast = pos0 + nvalid - 1;
-    const int jlo = max(0, pos0 - d.window + 1) / d.l;
-    const int jhi = tlast / d.l;
-    blk[0] = jlo;
-    *nblk_s = jhi - jlo + 1;
+    if (MODE == 1) {
+      const int jlo = max(0, pos0 - d.window + 1) / d.l;
+      blk[0] = jlo;
+      *nblk_s = tlast / d.l - jlo + 1;
+    } else {  // compressed keys 0 .. (tlast + 1) / l - 1, in 64-key chunks
+      const int cmax = min((tlast + 1) / d.l, d.Nc) - 1;
+      blk[0] = 0;
+      *nblk_s = cmax < 0 ? 0 : cmax / kKeys + 1;
+    }
   }
   __syncthreads();
   tc_fence_after();
@@ -192,7 +202,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             !wait_bar(&bars->empty[st], ((i / kStages) & 1) ^ 1, abort_flag, err))
           break;
         const int j = SEL ? blk[i] : blk0 + i;
-        const int row = b * d.T + j * kKeys;
+        const int row = b * nkeys + j * kKeys;
         uint8_t* kv = smem + OFF_KV + st * 2 * kTileBytes;
         mbar_expect_tx(&bars->full[st], 2 * kTileBytes);
         tma_load_3d(kv, &tm_k, &bars->full[st], 0, g, row);
@@ -287,7 +297,8 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       fence_proxy_async_smem();
       mbar_arrive(&bars->dorows);
     }
-    const int lo = SEL ? 0 : max(0, t - d.window + 1);
+    const int lo = MODE == 1 ? max(0, t - d.window + 1) : 0;
+    const int khi = MODE == 2 ? min((t + 1) / d.l, d.Nc) - 1 : t;  // last visible key
     const int* lst = SEL ? toks + tl * (d.topk + 1) : nullptr;
     int ptr = 0;
     int nxt = SEL && valid ? lst[0] : INT_MAX;
@@ -296,7 +307,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     for (int i = 0; i < n; ++i) {
       const int j = SEL ? blk[i] : blk0 + i;
       const int k0 = j * kKeys;
-      bool rowsel = valid && k0 <= t && lse2 != -INFINITY;
+      bool rowsel = valid && k0 <= khi && lse2 != -INFINITY;
       if (SEL) {
         const bool hit = nxt == j;
         if (hit) nxt = lst[++ptr];
@@ -321,15 +332,15 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           mbar_arrive(&bars->sfree);
         }
         if (rowsel) {
-          const bool part = !((k0 + kKeys - 1 <= t) && (k0 >= lo));
+          const bool part = !((k0 + kKeys - 1 <= khi) && (k0 >= lo));
 #pragma unroll
           for (int c = 0; c < 32; c += 2) {
             const int key = k0 + 32 * h2 + c;
             float p0 = fast_exp2(fmaf(sv[c], sl2, -lse2));
             float p1 = fast_exp2(fmaf(sv[c + 1], sl2, -lse2));
             if (part) {
-              if (key > t || key < lo) p0 = 0.f;
-              if (key + 1 > t || key + 1 < lo) p1 = 0.f;
+              if (key > khi || key < lo) p0 = 0.f;
+              if (key + 1 > khi || key + 1 < lo) p1 = 0.f;
             }
             dsk[16 * h2 + c / 2] = pack_bf16(p0 * (pv[c] - dl), p1 * (pv[c + 1] - dl));
           }
@@ -409,6 +420,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 // Warps: 0-3 key threads and epilogue, 4 MMA issue and TMEM owner (and the
 // K/V TMA), 5-8 row gather.
 constexpr int kKvThreads = 288;
+constexpr int kCmpShares = 16;  // row shares of a compression-branch key pair
 constexpr uint32_t kKTile2 = 128 * 64 * 2;  // 128 keys x 64 dims, bf16
 constexpr uint32_t kRowTile = 128 * 64 * 2;
 
@@ -466,13 +478,20 @@ __device__ __forceinline__ int kv_row_token(bool sel, long rix, int G, int n0, i
   return ti < ntok ? tq_lo + (int)ti : -1;
 }
 
-template <bool SEL>
+// MODE 0 selection, 1 window, 2 compression.  With nseg > 1 (compression:
+// every later query sees a compressed key, so one pair has all the rows)
+// the CTA blockIdx.x = pair * nseg + seg takes the seg-th share of the
+// pair's row tiles and stores its partial dK/dV in part[seg] instead of
+// accumulating; a reduction kernel sums the shares in order.
+template <int MODE>
 __global__ void __launch_bounds__(kKvThreads, 1)
 bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                    const bf16* __restrict__ q, const float* __restrict__ lse,
                    const float* __restrict__ delta, const float* __restrict__ dO,
                    const int* __restrict__ offsets, const int* __restrict__ list,
-                   float* __restrict__ dk, float* __restrict__ dv, Dims d, int* err) {
+                   float* __restrict__ dk, float* __restrict__ dv, float* __restrict__ part,
+                   int nseg, Dims d, int* err) {
+  constexpr bool SEL = MODE == 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   KvBars* bars = (KvBars*)(smem + KV_OFF_BAR);
@@ -480,7 +499,8 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
   uint32_t* tmem_slot = (uint32_t*)(smem + KV_OFF_MISC);
   volatile int* abort_flag = (volatile int*)(smem + KV_OFF_MISC + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
-  const int pr = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int pr = blockIdx.x / nseg, seg = blockIdx.x % nseg, g = blockIdx.y, b = blockIdx.z;
+  const int nkeys = MODE == 2 ? d.Nc : d.T;
   const int j0 = 2 * pr;
   const int kbase = j0 * kKeys;  // first key of the pair
 
@@ -497,13 +517,19 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
       l1 = list + bg * (size_t)d.Tq * d.topk + off[j0 + 1];
       n1 = off[j0 + 2] - off[j0 + 1];
     }
-  } else {
+  } else if (MODE == 1) {
     const int t_lo = kbase, t_hi = min(kbase + 2 * kKeys - 1 + d.window - 1, d.T - 1);
     tq_lo = max(0, t_lo - d.q_off);
     ntok = max(0, t_hi - d.q_off - tq_lo + 1);
+  } else {  // every query from the one that completes compressed block kbase on
+    tq_lo = max(0, (kbase + 1) * d.l - 1 - d.q_off);
+    ntok = max(0, d.Tq - tq_lo);
   }
   const long nrows = SEL ? ((long)n0 + n1) * d.G : (long)ntok * d.G;
-  const int ntiles = (int)((nrows + 127) / 128);
+  const int ntiles_all = (int)((nrows + 127) / 128);
+  const int tps = (ntiles_all + nseg - 1) / nseg;  // tiles per share
+  const int u0 = seg * tps;
+  const int ntiles = max(0, min(tps, ntiles_all - u0));
 
   if (tid == 0) {
     mbar_init(&bars->kv, 1);
@@ -530,7 +556,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     for (int u = 0; u < ntiles; ++u) {
       const int bu = u & 1;
       if (u >= 2 && !wait_bar(&bars->bfree[bu], ((u - 2) >> 1) & 1, abort_flag, err)) break;
-      const long rix = (long)u * 128 + gr;
+      const long rix = (long)(u0 + u) * 128 + gr;
       int bit = 0;
       const int tq =
           rix < nrows ? kv_row_token(SEL, rix, d.G, n0, n1, l0, l1, tq_lo, ntok, &bit) : -1;
@@ -589,8 +615,8 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
       prefetch_tmap(&tm_v);
       mbar_expect_tx(&bars->kv, 2 * kKTile2);
       for (int h = 0; h < 2; ++h) {
-        tma_load_3d(smem + KV_OFF_K + h * kTileBytes, &tm_k, &bars->kv, 0, g, b * d.T + kbase + h * kKeys);
-        tma_load_3d(smem + KV_OFF_V + h * kTileBytes, &tm_v, &bars->kv, 0, g, b * d.T + kbase + h * kKeys);
+        tma_load_3d(smem + KV_OFF_K + h * kTileBytes, &tm_k, &bars->kv, 0, g, b * nkeys + kbase + h * kKeys);
+        tma_load_3d(smem + KV_OFF_V + h * kTileBytes, &tm_v, &bars->kv, 0, g, b * nkeys + kbase + h * kKeys);
       }
       bool ok = wait_bar(&bars->kv, 0, abort_flag, err);
       auto issue_kv = [&](int u) -> bool {
@@ -685,8 +711,9 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
           for (int h = 0; h < 2; ++h) {
             const int r = 32 * c + e + h;
             const int t = in.tpos[r];
-            bool vis = (in.blkmask[r] & kbit) && key <= t;
-            if (!SEL) vis = vis && key >= t - d.window + 1;
+            bool vis = (in.blkmask[r] & kbit) &&
+                       (MODE == 2 ? key * d.l + d.l - 1 <= t : key <= t);
+            if (MODE == 1) vis = vis && key >= t - d.window + 1;
             const float pr = vis ? fast_exp2(fmaf(sv[e + h], sl2, -in.lse2[r])) : 0.f;
             p2[h] = pr;
             d2[h] = pr * (pv[e + h] - in.delta[r]);
@@ -719,8 +746,9 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     bool have = false;
     if (ok && ntiles > 0) have = wait_bar_warp(&bars->fin, 0, abort_flag, err);
     float a[32];
-    const size_t krow = ((size_t)b * d.T + key) * d.Hkv * 64 + (size_t)g * 64;
-    const bool kin = key < d.T;
+    const size_t krow = ((size_t)b * nkeys + key) * d.Hkv * 64 + (size_t)g * 64;
+    const bool kin = key < nkeys;
+    const size_t nk_all = (size_t)d.B * nkeys * d.Hkv * 64;  // one share of dK (or dV)
 #pragma unroll 1
     for (int h = 0; h < 4; ++h) {  // dV [0,64), dK [64,128) in halves of 32
       if (have) {
@@ -728,9 +756,16 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         tmem_ld32(lane_tmem + kvColDV + 32u * h, a);
         tmem_wait_ld();
       }
-      if (have && kin) {
+      const float sc = h < 2 ? 1.f : d.scale;
+      if (MODE == 2 && kin) {  // this share's partial (zeros when it had no rows)
+        float* dst = part + ((size_t)seg * 2 + (h < 2 ? 1 : 0)) * nk_all + krow + 32 * (h & 1);
+#pragma unroll
+        for (int c = 0; c < 32; c += 4)
+          *reinterpret_cast<float4*>(dst + c) =
+              have ? make_float4(a[c] * sc, a[c + 1] * sc, a[c + 2] * sc, a[c + 3] * sc)
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
+      } else if (have && kin) {
         float* dst = (h < 2 ? dv : dk) + krow + 32 * (h & 1);
-        const float sc = h < 2 ? 1.f : d.scale;
 #pragma unroll
         for (int c = 0; c < 32; c += 4) {
           float4 x = *reinterpret_cast<float4*>(dst + c);
@@ -751,45 +786,75 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
   }
 }
 
-template <bool SEL>
+// dk += sum over shares of part[s][0], dv += sum of part[s][1], in share order.
+__global__ void dkdv_share_sum_kernel(const float* __restrict__ part, float* __restrict__ dk,
+                                      float* __restrict__ dv, size_t n, int nseg) {
+  const size_t e = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) * 4;
+  if (e >= n) return;
+  float4 sk = make_float4(0.f, 0.f, 0.f, 0.f), sv = sk;
+  for (int s = 0; s < nseg; ++s) {
+    const float4 x = *reinterpret_cast<const float4*>(part + (size_t)(2 * s) * n + e);
+    const float4 y = *reinterpret_cast<const float4*>(part + (size_t)(2 * s + 1) * n + e);
+    sk.x += x.x; sk.y += x.y; sk.z += x.z; sk.w += x.w;
+    sv.x += y.x; sv.y += y.y; sv.z += y.z; sv.w += y.w;
+  }
+  float4* pk = reinterpret_cast<float4*>(dk + e);
+  float4* pv = reinterpret_cast<float4*>(dv + e);
+  float4 a = *pk, c = *pv;
+  a.x += sk.x; a.y += sk.y; a.z += sk.z; a.w += sk.w;
+  c.x += sv.x; c.y += sv.y; c.z += sv.z; c.w += sv.w;
+  *pk = a;
+  *pv = c;
+}
+
+template <int MODE>
 cudaError_t launch_dkdv_tc_t(const Dims& d, const void* q, const void* k, const void* v,
                              const float* lse, const float* delta, const float* dO,
-                             const int* offsets, const int* list, float* dk, float* dv, int* err,
-                             cudaStream_t s) {
-  const int npairs = (d.Nb + 1) / 2;
+                             const int* offsets, const int* list, float* dk, float* dv,
+                             float* part, int* err, cudaStream_t s) {
+  const int nkeys = MODE == 2 ? d.Nc : d.T;
+  const int nchunk = (nkeys + kKeys - 1) / kKeys;
+  const int npairs = (nchunk + 1) / 2;
   if (npairs == 0) return cudaSuccess;
+  const int nseg = MODE == 2 ? kCmpShares : 1;
   CUtensorMap mk, mv;
-  if (!make_tmap_bf16(&mk, k, d.Hkv, (long)d.B * d.T, 1, kKeys) ||
-      !make_tmap_bf16(&mv, v, d.Hkv, (long)d.B * d.T, 1, kKeys))
+  if (!make_tmap_bf16(&mk, k, d.Hkv, (long)d.B * nkeys, 1, kKeys) ||
+      !make_tmap_bf16(&mv, v, d.Hkv, (long)d.B * nkeys, 1, kKeys))
     return cudaErrorInvalidValue;
   // 512 TMEM columns per CTA: ask for enough shared memory that a second CTA
   // never shares the SM (it would wait in tcgen05.alloc)
   const size_t smem = KV_SMEM + 1024 > 120 * 1024 ? KV_SMEM + 1024 : 120 * 1024;
-  cudaError_t e = cudaFuncSetAttribute(bwd_dkdv_tc_kernel<SEL>,
+  cudaError_t e = cudaFuncSetAttribute(bwd_dkdv_tc_kernel<MODE>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  bwd_dkdv_tc_kernel<SEL><<<dim3(npairs, d.Hkv, d.B), kKvThreads, smem, s>>>(
-      mk, mv, (const bf16*)q, lse, delta, dO, offsets, list, dk, dv, d, err);
+  bwd_dkdv_tc_kernel<MODE><<<dim3(npairs * nseg, d.Hkv, d.B), kKvThreads, smem, s>>>(
+      mk, mv, (const bf16*)q, lse, delta, dO, offsets, list, dk, dv, part, nseg, d, err);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || MODE != 2) return e;
+  const size_t n = (size_t)d.B * nkeys * d.Hkv * 64;
+  dkdv_share_sum_kernel<<<(unsigned)((n / 4 + 255) / 256), 256, 0, s>>>(part, dk, dv, n, nseg);
   return cudaGetLastError();
 }
 
-template <bool SEL>
+template <int MODE>
 cudaError_t launch_dq_tc_t(const Dims& d, const void* q, const void* k, const void* v,
                            const int32_t* idx, const void* o, const float* lse, const float* dO,
                            float* dq, float* delta, int* err, cudaStream_t s) {
   const int TQ = tokens_per_tile(d.G);
+  const long key_rows = (long)d.B * (MODE == 2 ? d.Nc : d.T);
+  if (key_rows == 0) return cudaSuccess;
   CUtensorMap mq, mk, mv;
   if (!make_tmap_bf16(&mq, q, d.Hq, (long)d.B * d.Tq, d.G, TQ) ||
-      !make_tmap_bf16(&mk, k, d.Hkv, (long)d.B * d.T, 1, kKeys) ||
-      !make_tmap_bf16(&mv, v, d.Hkv, (long)d.B * d.T, 1, kKeys))
+      !make_tmap_bf16(&mk, k, d.Hkv, key_rows, 1, kKeys) ||
+      !make_tmap_bf16(&mv, v, d.Hkv, key_rows, 1, kKeys))
     return cudaErrorInvalidValue;
   const size_t smem = OFF_LIST + list_ints(d) * sizeof(int) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(bwd_dq_tc_kernel<SEL>,
+  cudaError_t e = cudaFuncSetAttribute(bwd_dq_tc_kernel<MODE>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((d.Tq + TQ - 1) / TQ, d.Hkv, d.B);
-  bwd_dq_tc_kernel<SEL><<<grid, kThreads, smem, s>>>(mq, mk, mv, (const bf16*)o, lse, dO, idx, dq,
-                                                     delta, d, err);
+  bwd_dq_tc_kernel<MODE><<<grid, kThreads, smem, s>>>(mq, mk, mv, (const bf16*)o, lse, dO, idx,
+                                                      dq, delta, d, err);
   return cudaGetLastError();
 }
 
@@ -797,27 +862,34 @@ cudaError_t launch_dq_tc_t(const Dims& d, const void* q, const void* k, const vo
 
 // Tensor-core dQ applies to bf16, 64-key blocks, head dim 64, G dividing 128.
 bool dq_tc_eligible(const Dims& d, int mode) {
-  return mode != 2 && d.dtype == 1 && d.l == kKeys && d.D == 64 && d.G >= 1 &&
-         kRows % d.G == 0 && d.Nb <= 4096 && tmap_encode_fn() != nullptr;
+  return d.dtype == 1 && d.l == kKeys && d.D == 64 && d.G >= 1 && kRows % d.G == 0 &&
+         d.Nb <= 4096 && tmap_encode_fn() != nullptr;
 }
 
 // Tensor-core dK/dV: the same geometry (key-stationary over pairs of blocks).
 bool dkdv_tc_eligible(const Dims& d, int mode) { return dq_tc_eligible(d, mode); }
 
+size_t dkdv_cmp_part_bytes(const Dims& d) {
+  return (size_t)kCmpShares * 2 * d.B * d.Nc * d.Hkv * 64 * sizeof(float);
+}
+
 cudaError_t launch_dkdv_tc(const Dims& d, int mode, const void* q, const void* k, const void* v,
                            const float* lse, const float* delta, const float* dO,
-                           const int* offsets, const int* list, float* dk, float* dv, int* err,
-                           cudaStream_t s) {
-  return mode == 0
-             ? launch_dkdv_tc_t<true>(d, q, k, v, lse, delta, dO, offsets, list, dk, dv, err, s)
-             : launch_dkdv_tc_t<false>(d, q, k, v, lse, delta, dO, offsets, list, dk, dv, err, s);
+                           const int* offsets, const int* list, float* dk, float* dv, float* part,
+                           int* err, cudaStream_t s) {
+  if (mode == 0)
+    return launch_dkdv_tc_t<0>(d, q, k, v, lse, delta, dO, offsets, list, dk, dv, part, err, s);
+  if (mode == 1)
+    return launch_dkdv_tc_t<1>(d, q, k, v, lse, delta, dO, offsets, list, dk, dv, part, err, s);
+  return launch_dkdv_tc_t<2>(d, q, k, v, lse, delta, dO, offsets, list, dk, dv, part, err, s);
 }
 
 cudaError_t launch_dq_tc(const Dims& d, int mode, const void* q, const void* k, const void* v,
                          const int32_t* idx, const void* o, const float* lse, const float* dO,
                          float* dq, float* delta, int* err, cudaStream_t s) {
-  return mode == 0 ? launch_dq_tc_t<true>(d, q, k, v, idx, o, lse, dO, dq, delta, err, s)
-                   : launch_dq_tc_t<false>(d, q, k, v, idx, o, lse, dO, dq, delta, err, s);
+  return mode == 0   ? launch_dq_tc_t<0>(d, q, k, v, idx, o, lse, dO, dq, delta, err, s)
+         : mode == 1 ? launch_dq_tc_t<1>(d, q, k, v, idx, o, lse, dO, dq, delta, err, s)
+                     : launch_dq_tc_t<2>(d, q, k, v, idx, o, lse, dO, dq, delta, err, s);
 }
 
 }  // namespace nsa
