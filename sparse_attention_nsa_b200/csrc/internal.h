@@ -64,7 +64,9 @@ bool dq_tc_eligible(const Dims& d, int mode);
 cudaError_t launch_dq_tc(const Dims& d, int mode, const void* q, const void* keys,
                          const void* vals, const int32_t* idx, const void* o, const float* lse,
                          const float* dO, float* dq, float* delta, int* err, cudaStream_t s);
-cudaError_t launch_revmap(const Dims& d, const int32_t* idx, int* counts, int* offsets,
+// chunk: workspace of revmap_chunk_ints(d) ints
+size_t revmap_chunk_ints(const Dims& d);
+cudaError_t launch_revmap(const Dims& d, const int32_t* idx, int* chunk, int* offsets,
                           int* list, cudaStream_t s);
 cudaError_t launch_dkdv(const Dims& d, int mode, const void* q, const void* keys,
                         const void* vals, const float* lse, const float* delta,

@@ -173,81 +173,143 @@ dq_kernel(const T* __restrict__ q, const T* __restrict__ keys, const T* __restri
 }
 
 // ---- reverse block -> query map (selection) -------------------------------------
-// counts[b, g, j] = number of queries selecting block j; offsets = exclusive
-// scan; list[offsets[j] ..] = those queries' indices tq in ascending order.
-__global__ void rev_count_kernel(const int32_t* __restrict__ idx, int* __restrict__ counts,
-                                 Dims d) {
-  const long e = (long)blockIdx.x * blockDim.x + threadIdx.x;
-  const long n = (long)d.B * d.Tq * d.Hkv * d.topk;
-  if (e >= n) return;
-  const int j = idx[e];
-  const long r = e / d.topk;  // (b, tq, g)
-  const int slot = (int)(e % d.topk);
-  const int g = (int)(r % d.Hkv);
-  const int tq = (int)((r / d.Hkv) % d.Tq);
-  const int b = (int)(r / ((long)d.Hkv * d.Tq));
-  const int cur = (d.q_off + tq) / d.l;
-  // the same validity rule as the forward: ascending, distinct, causal
-  const bool ok = j >= 0 && j <= cur && (slot == 0 || idx[e - 1] < j);
-  if (ok) atomicAdd(&counts[((size_t)b * d.Hkv + g) * (d.Nb + 1) + j], 1);
+// For each (sequence, KV group) and block j: offsets[j] .. offsets[j+1] index
+// the ascending list of the queries tq that selected j.  Built without
+// global atomics in three steps over chunks of kRevChunk consecutive
+// queries: (1) per chunk, a shared-memory histogram of the blocks chosen;
+// (2) per (sequence, group), the per-block totals, their exclusive scan
+// (offsets) and each chunk's first position per block; (3) per chunk, one
+// warp walks the queries in ascending order, 32 at a time, and places each
+// selection at its block's running position plus its rank among the lanes
+// that chose the same block.  A selection counts when it is a real,
+// causal block that does not repeat or go back (the forward's rule).
+constexpr int kRevChunk = 256;
+
+__device__ __forceinline__ bool rev_valid(const int32_t* ir, int s, int cur) {
+  const int j = ir[s];
+  return j >= 0 && j <= cur && (s == 0 || ir[s - 1] < j);
 }
 
-// one CTA per (b, g): exclusive scan of Nb counts into Nb + 1 offsets
-__global__ void rev_scan_kernel(const int* __restrict__ counts, int* __restrict__ offsets,
-                                Dims d) {
-  __shared__ int part[1024];
+__global__ void __launch_bounds__(kRevChunk)
+rev_chunk_count_kernel(const int32_t* __restrict__ idx, int* __restrict__ chunk, Dims d) {
+  extern __shared__ int hist[];  // [Nb]
+  const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int nchunk = gridDim.x;
+  for (int j = threadIdx.x; j < d.Nb; j += blockDim.x) hist[j] = 0;
+  __syncthreads();
+  const int tq = c * kRevChunk + threadIdx.x;
+  if (tq < d.Tq) {
+    const int32_t* ir = idx + (((size_t)b * d.Tq + tq) * d.Hkv + g) * d.topk;
+    const int cur = (d.q_off + tq) / d.l;
+    for (int s = 0; s < d.topk; ++s)
+      if (rev_valid(ir, s, cur)) atomicAdd(&hist[ir[s]], 1);
+  }
+  __syncthreads();
+  int* out = chunk + (((size_t)b * d.Hkv + g) * nchunk + c) * d.Nb;
+  for (int j = threadIdx.x; j < d.Nb; j += blockDim.x) out[j] = hist[j];
+}
+
+// one CTA per (sequence, group); chunk[c][j] becomes chunk c's first list
+// position for block j
+__global__ void __launch_bounds__(1024)
+rev_chunk_scan_kernel(int* __restrict__ chunk, int* __restrict__ offsets, Dims d, int nchunk) {
+  extern __shared__ int tot[];  // [Nb]
+  __shared__ int wsum[32];
   const int bg = blockIdx.x;
-  const int* c = counts + (size_t)bg * (d.Nb + 1);
-  int* off = offsets + (size_t)bg * (d.Nb + 1);
+  int* cc = chunk + (size_t)bg * nchunk * d.Nb;
+  for (int j = threadIdx.x; j < d.Nb; j += blockDim.x) {
+    int run = 0;
+    for (int c = 0; c < nchunk; ++c) {
+      const int v = cc[(size_t)c * d.Nb + j];
+      cc[(size_t)c * d.Nb + j] = run;
+      run += v;
+    }
+    tot[j] = run;
+  }
+  __syncthreads();
+  // exclusive scan of tot over j: each thread a contiguous range
   const int per = (d.Nb + blockDim.x - 1) / blockDim.x;
   const int lo = threadIdx.x * per, hi = min(lo + per, d.Nb);
-  int s = 0;
-  for (int j = lo; j < hi; ++j) s += c[j];
-  part[threadIdx.x] = s;
+  int sum = 0;
+  for (int j = lo; j < hi; ++j) sum += tot[j];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = sum;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += y;
+  }
+  if (lane == 31) wsum[warp] = incl;
   __syncthreads();
-  if (threadIdx.x == 0) {
-    int acc = 0;
-    for (int i = 0; i < (int)blockDim.x; ++i) {
-      const int v = part[i];
-      part[i] = acc;
-      acc += v;
+  if (warp == 0) {
+    const int nw = (blockDim.x + 31) / 32;
+    int w = lane < nw ? wsum[lane] : 0;
+    int wi = w;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, wi, off);
+      if (lane >= off) wi += y;
     }
-    off[d.Nb] = acc;
+    wsum[lane] = wi - w;  // exclusive over warps
   }
   __syncthreads();
-  int acc = part[threadIdx.x];
+  int run = wsum[warp] + incl - sum;
+  int* off = offsets + (size_t)bg * (d.Nb + 1);
   for (int j = lo; j < hi; ++j) {
-    off[j] = acc;
-    acc += c[j];
+    const int t = tot[j];
+    tot[j] = run;
+    off[j] = run;
+    run += t;
   }
+  if (threadIdx.x == blockDim.x - 1) off[d.Nb] = run;
+  __syncthreads();
+  for (int j = threadIdx.x; j < d.Nb; j += blockDim.x)
+    for (int c = 0; c < nchunk; ++c) cc[(size_t)c * d.Nb + j] += tot[j];
 }
 
-// one warp per (b, g, j): scan queries in order, ballot the ones that chose j
-__global__ void rev_fill_kernel(const int32_t* __restrict__ idx, const int* __restrict__ offsets,
-                                int* __restrict__ list, Dims d) {
-  const long w = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  const long nw = (long)d.B * d.Hkv * d.Nb;
-  if (w >= nw) return;
-  const int j = (int)(w % d.Nb);
-  const long bg = w / d.Nb;
-  const int g = (int)(bg % d.Hkv), b = (int)(bg / d.Hkv);
-  int pos = offsets[bg * (d.Nb + 1) + j];
-  const size_t list_base = (size_t)bg * d.Tq * d.topk;
-  // a query can choose block j only once it is at or past the block
-  const int tq0 = max(0, j * d.l - d.q_off);
-  for (int base = tq0; base < d.Tq; base += 32) {
-    const int tq = base + lane;
-    bool hit = false;
-    if (tq < d.Tq) {
-      const int32_t* ir = idx + (((size_t)b * d.Tq + tq) * d.Hkv + g) * d.topk;
-      const int cur = (d.q_off + tq) / d.l;
-      if (j <= cur)
-        for (int s = 0; s < d.topk; ++s) hit |= ir[s] == j && (s == 0 || ir[s - 1] < j);
-    }
-    const unsigned m = __ballot_sync(0xffffffffu, hit);
-    if (hit) list[list_base + pos + __popc(m & ((1u << lane) - 1u))] = tq;
-    pos += __popc(m);
+// one warp per (chunk, group, sequence)
+__global__ void __launch_bounds__(32)
+rev_chunk_fill_kernel(const int32_t* __restrict__ idx, const int* __restrict__ chunk,
+                      int* __restrict__ list, Dims d) {
+  extern __shared__ int sm[];  // run[Nb], bits[Nb]
+  int* run = sm;
+  unsigned* bits = (unsigned*)(sm + d.Nb);
+  const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int nchunk = gridDim.x;
+  const int lane = threadIdx.x;
+  const size_t bg = (size_t)b * d.Hkv + g;
+  const int* base = chunk + (bg * nchunk + c) * d.Nb;
+  for (int j = lane; j < d.Nb; j += 32) {
+    run[j] = base[j];
+    bits[j] = 0u;
+  }
+  __syncwarp();
+  int* lst = list + bg * (size_t)d.Tq * d.topk;
+  const unsigned lt = (1u << lane) - 1u;
+  for (int grp = 0; grp < kRevChunk / 32; ++grp) {
+    const int tq = c * kRevChunk + grp * 32 + lane;
+    const bool q_ok = tq < d.Tq;
+    const int32_t* ir = idx + (((size_t)b * d.Tq + (q_ok ? tq : 0)) * d.Hkv + g) * d.topk;
+    const int cur = (d.q_off + tq) / d.l;
+    for (int s = 0; s < d.topk; ++s)
+      if (q_ok && rev_valid(ir, s, cur)) atomicOr(&bits[ir[s]], 1u << lane);
+    __syncwarp();
+    for (int s = 0; s < d.topk; ++s)
+      if (q_ok && rev_valid(ir, s, cur)) {
+        const int j = ir[s];
+        lst[run[j] + __popc(bits[j] & lt)] = tq;
+      }
+    __syncwarp();
+    for (int s = 0; s < d.topk; ++s)
+      if (q_ok && rev_valid(ir, s, cur)) {
+        const int j = ir[s];
+        const unsigned m = bits[j];
+        if ((m & lt) == 0u) {  // the lowest lane that chose j advances its position
+          run[j] += __popc(m);
+          bits[j] = 0u;
+        }
+      }
+    __syncwarp();
   }
 }
 
@@ -426,16 +488,18 @@ cudaError_t launch_dq(const Dims& d, int mode, const void* q, const void* keys, 
   return dq_t<float, kBwdCmp>(d, q, keys, vals, idx, o, lse, dO, dq, delta, err, s);
 }
 
-cudaError_t launch_revmap(const Dims& d, const int32_t* idx, int* counts, int* offsets,
+size_t revmap_chunk_ints(const Dims& d) {
+  return (size_t)d.B * d.Hkv * ((d.Tq + kRevChunk - 1) / kRevChunk) * d.Nb;
+}
+
+cudaError_t launch_revmap(const Dims& d, const int32_t* idx, int* chunk, int* offsets,
                           int* list, cudaStream_t s) {
-  const size_t nco = (size_t)d.B * d.Hkv * (d.Nb + 1);
-  cudaError_t e = cudaMemsetAsync(counts, 0, nco * sizeof(int), s);
-  if (e != cudaSuccess) return e;
-  const long n = (long)d.B * d.Tq * d.Hkv * d.topk;
-  rev_count_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(idx, counts, d);
-  rev_scan_kernel<<<d.B * d.Hkv, 256, 0, s>>>(counts, offsets, d);
-  const long nw = (long)d.B * d.Hkv * d.Nb;
-  rev_fill_kernel<<<(unsigned)((nw * 32 + 255) / 256), 256, 0, s>>>(idx, offsets, list, d);
+  const int nchunk = (d.Tq + kRevChunk - 1) / kRevChunk;
+  if (nchunk == 0 || d.Nb == 0) return cudaSuccess;
+  const size_t nb_bytes = (size_t)d.Nb * sizeof(int);
+  rev_chunk_count_kernel<<<dim3(nchunk, d.Hkv, d.B), kRevChunk, nb_bytes, s>>>(idx, chunk, d);
+  rev_chunk_scan_kernel<<<d.B * d.Hkv, 1024, nb_bytes, s>>>(chunk, offsets, d, nchunk);
+  rev_chunk_fill_kernel<<<dim3(nchunk, d.Hkv, d.B), 32, 2 * nb_bytes, s>>>(idx, chunk, list, d);
   return cudaGetLastError();
 }
 

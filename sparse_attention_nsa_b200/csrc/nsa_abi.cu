@@ -441,7 +441,8 @@ namespace {
 
 // Backward workspace layout, each part 256-byte aligned:
 //   delta [B*Tq*Hq] f32 | dO_cmp, dO_sel, dO_swa [B*Tq*Hq*64] f32 |
-//   dkc, dvc [B*Nc*Hkv*64] f32 | counts, offsets [B*Hkv*(Nb+1)] i32 |
+//   dkc, dvc [B*Nc*Hkv*64] f32 | reverse-map chunk positions
+//   [B*Hkv*ceil(Tq/256)*Nb] i32 | offsets [B*Hkv*(Nb+1)] i32 |
 //   list [B*Hkv*Tq*topk] i32 | compression dK/dV row shares (tensor-core path)
 struct BwdCarve {
   size_t delta, dO[3], dkc, dvc, counts, offsets, list, part, total;
@@ -460,7 +461,7 @@ BwdCarve bwd_carve(const Dims& d) {
   for (int i = 0; i < 3; ++i) c.dO[i] = take(rows * 64 * 4);
   c.dkc = take((size_t)d.B * d.Nc * d.Hkv * 64 * 4);
   c.dvc = take((size_t)d.B * d.Nc * d.Hkv * 64 * 4);
-  c.counts = take((size_t)d.B * d.Hkv * (d.Nb + 1) * 4);
+  c.counts = take(nsa::revmap_chunk_ints(d) * 4);
   c.offsets = take((size_t)d.B * d.Hkv * (d.Nb + 1) * 4);
   c.list = take((size_t)d.B * d.Hkv * d.Tq * d.topk * 4);
   c.part = take(nsa::dkdv_tc_eligible(d, 2) ? nsa::dkdv_cmp_part_bytes(d) : 0);
