@@ -62,6 +62,23 @@ def fwd_flops(w, branch_mask=None) -> dict:
     return out
 
 
+def executed_sel_flops(w, idx) -> float:
+    """MMA FLOPs the selection kernel actually issues: each 128-row tile
+    (128/G tokens x G heads of one group) runs S = QK^T and O += PV over the
+    union of its tokens' selected 64-key blocks (2 x 2*128*64*64 FLOP per
+    union block), whatever fraction of its rows selected each block."""
+    import numpy as np
+    ii = idx.cpu().numpy()  # [B, T, Hkv, topk]
+    tq = 128 // (w.Hq // w.Hkv)
+    blocks = 0
+    for b in range(w.B):
+        for g in range(w.Hkv):
+            for t0 in range(0, w.T, tq):
+                sel = ii[b, t0:t0 + tq, g].ravel()
+                blocks += len(np.unique(sel[sel >= 0]))
+    return blocks * 2 * 2.0 * 128 * 64 * 64
+
+
 def load_peaks() -> dict:
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -300,6 +317,7 @@ def run_gpu(args, rank: int, world: int, dist_on: bool) -> None:
         args.steps, flush, stream))
     peaks = load_peaks()
     sel_tflops = flops["sel"] / (sel_ms * 1e-3) / 1e12
+    sel_exec_flops = executed_sel_flops(w, saved["idx"])
 
     # end to end through the C ABI with host buffers (pinned), copies timed
     hq, hk, hv, hg = (x.cpu().pin_memory() for x in (q, k, v, g))
@@ -348,7 +366,12 @@ def run_gpu(args, rank: int, world: int, dist_on: bool) -> None:
                      "frac": sel_tflops / peaks["bf16_tflops"],
                      "traffic": profiled_traffic("sparse_attention_nsa_b200/csrc/k_attn_tc.cu",
                                                  "profiles/attn_tc_sel_340m.md"),
-                     "ms_per_launch": sel_ms, "peak_source": peaks["source"] + " burst bf16"},
+                     "ms_per_launch": sel_ms, "peak_source": peaks["source"] + " burst bf16",
+                     # context, not the roofline figure: on structure-free selections the
+                     # union of a tile's blocks is near dense, so the tensor pipe runs
+                     # more MMA work than the algorithmic count
+                     "executed_tflops": sel_exec_flops / (sel_ms * 1e-3) / 1e12,
+                     "executed_over_algorithmic": sel_exec_flops / flops["sel"]},
         "decode": dec,
         "train": train,
         "e2e": {"value": job_tokens_per_s(tokens_per_step, world, e2e_ms), "unit": "tokens/s",

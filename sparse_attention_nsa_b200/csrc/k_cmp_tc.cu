@@ -10,7 +10,8 @@
 // compressed keys of its 128 rows (128/G tokens x the G heads of one group):
 //   pass 1  S = Q Kc^T chunk by chunk (64 compressed blocks per chunk),
 //           running row max and sum of exponentials;
-//   pass 2  S again, P = exp(S - m) / l exactly normalised, the G heads of
+//   pass 2  S again (with at most two chunks, re-read from TMEM rather than
+//           recomputed), P = exp(S - m) / l exactly normalised, the G heads of
 //           each token summed with warp shuffles into the block scores, and
 //           (unless only scores are wanted) P in bf16 through swizzled smem
 //           into O += P Vc, accumulated directly in TMEM.
@@ -78,6 +79,10 @@ cmp_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   const int pos0 = d.q_off + t0;
   const int nvis_max = min((pos0 + nvalid) / d.l, d.Nc);  // of the tile's last token
   const int n = (nvis_max + kChunk - 1) / kChunk;
+  // with at most two chunks both S tiles stay in TMEM: pass 2 re-reads them
+  // instead of recomputing, and each chunk's Kc and Vc are loaded once
+  const bool res = n <= 2;
+  const int nload = res ? n : 2 * n;
 
   if (tid == 0) {
     mbar_init(&bars->q, 1);
@@ -108,12 +113,12 @@ cmp_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       mbar_expect_tx(&bars->q, kQBytes);
       tma_load_3d(smem + OFF_Q, &tm_q, &bars->q, 0, g * d.G, b * d.Tq + t0);
       int issued = 0;
-      for (int u = 0; u < 2 * n; ++u) {
+      for (int u = 0; u < nload; ++u) {
         const int st = u % kStages;
         if (u >= kStages && !wait_bar(&bars->empty[st], ((u / kStages) & 1) ^ 1, abort_flag, err))
           break;
         const int i = u < n ? u : u - n;
-        const bool with_v = WITH_O && u >= n;
+        const bool with_v = WITH_O && (res || u >= n);
         uint8_t* kv = smem + OFF_KV + st * 2 * kTileBytes;
         const int row = b * d.Nc + i * kChunk;
         mbar_expect_tx(&bars->full[st], with_v ? 2 * kTileBytes : kTileBytes);
@@ -136,7 +141,7 @@ cmp_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       auto do_pv = [&](int i) -> bool {
         if (!wait_bar(&bars->p[i & 1], (i >> 1) & 1, abort_flag, err)) return false;
         tc_fence_after();
-        const int st = (n + i) % kStages;
+        const int st = (res ? i : n + i) % kStages;
         const uint32_t v_addr = smem_u32(smem + OFF_KV + st * 2 * kTileBytes + kTileBytes);
         const uint32_t p_addr = smem_u32(smem + OFF_P + (i & 1) * kPBytes);
 #pragma unroll
@@ -147,7 +152,7 @@ cmp_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         mma_commit(&bars->empty[st]);
         return true;
       };
-      for (int u = 0; ok && u < 2 * n; ++u) {
+      for (int u = 0; ok && u < nload; ++u) {
         const int st = u % kStages;
         if (!wait_bar(&bars->full[st], (u / kStages) & 1, abort_flag, err)) break;
         if (u >= 2 && !wait_bar(&bars->sfree[u & 1], ((u - 2) >> 1) & 1, abort_flag, err)) break;
@@ -158,12 +163,14 @@ cmp_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           mma_bf16(tmem + (uint32_t)(u & 1) * 64u, desc_sw128(q_addr + kk * 32, 16),
                    desc_sw128(k_addr + kk * 32, 16), idesc_s, kk > 0);
         mma_commit(&bars->s[u & 1]);
-        if (u < n || !WITH_O) mma_commit(&bars->empty[st]);
-        if (WITH_O && u - 1 >= n && !do_pv(u - 1 - n)) {
+        if ((u < n && !res) || !WITH_O) mma_commit(&bars->empty[st]);
+        if (WITH_O && !res && u - 1 >= n && !do_pv(u - 1 - n)) {
           ok = false;
           break;
         }
       }
+      if (ok && WITH_O && res)
+        for (int i = 0; ok && i + 1 < n; ++i) ok = do_pv(i);
       if (ok && WITH_O && n > 0) ok = do_pv(n - 1);
       mma_commit(&bars->odone);  // fires when every MMA above has completed
       drain_bar(&bars->odone, 0);
@@ -190,8 +197,10 @@ cmp_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       tmem_ld32(lane_tmem + (uint32_t)(u & 1) * 64u, sv);
       tmem_ld32(lane_tmem + (uint32_t)(u & 1) * 64u + 32u, sv + 32);
       tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&bars->sfree[u & 1]);
+      if (!res) {
+        tc_fence_before();
+        mbar_arrive(&bars->sfree[u & 1]);
+      }
       const int j0 = u * kChunk;
       if (j0 < nvis) {
         float mx = -INFINITY;
@@ -204,8 +213,8 @@ cmp_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const float mn = fmaxf(m, mx);
         float rs = 0.f;
 #pragma unroll
-        for (int c = 0; c < 64; ++c) rs += exp2f(sv[c] - mn);
-        lsum = lsum * exp2f(m - mn) + rs;
+        for (int c = 0; c < 64; ++c) rs += fast_exp2(sv[c] - mn);
+        lsum = lsum * fast_exp2(m - mn) + rs;
         m = mn;
       }
     }
@@ -214,8 +223,8 @@ cmp_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const int per = 64 / d.G;  // score columns written by each head-lane of a token
     // pass 2: normalised probabilities, block scores, P for the value MMA
     for (int i = 0; ok && i < n; ++i) {
-      const int u = n + i;
-      if (!wait_bar_warp(&bars->s[u & 1], (u >> 1) & 1, abort_flag, err)) {
+      const int u = res ? i : n + i;
+      if (!res && !wait_bar_warp(&bars->s[u & 1], (u >> 1) & 1, abort_flag, err)) {
         ok = false;
         break;
       }
@@ -223,12 +232,14 @@ cmp_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       tmem_ld32(lane_tmem + (uint32_t)(u & 1) * 64u, sv);
       tmem_ld32(lane_tmem + (uint32_t)(u & 1) * 64u + 32u, sv + 32);
       tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&bars->sfree[u & 1]);
+      if (!res) {
+        tc_fence_before();
+        mbar_arrive(&bars->sfree[u & 1]);
+      }
       const int j0 = i * kChunk;
 #pragma unroll
       for (int c = 0; c < 64; ++c)
-        sv[c] = j0 + c < nvis ? exp2f(fmaf(sv[c], sl2, -m)) * inv : 0.f;
+        sv[c] = j0 + c < nvis ? fast_exp2(fmaf(sv[c], sl2, -m)) * inv : 0.f;
       if (WITH_O) {
         if (i >= 2 && !wait_bar_warp(&bars->pfree[i & 1], ((i - 2) >> 1) & 1, abort_flag, err)) {
           ok = false;
