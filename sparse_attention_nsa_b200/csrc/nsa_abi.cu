@@ -348,6 +348,12 @@ static nsa_status run_forward(const Dims& d, const void* q, const void* k, const
   }
   if (sel) {
     NSA_TRY_CUDA(nsa::launch_topk(d, score, idx, s));
+    if (!swa && nsa::swa_combine_fusable(d)) {
+      // no window branch: the selection kernel runs last and applies the gates
+      NSA_TRY_CUDA(nsa::launch_sel_fwd_combine(d, q, k, v, idx, S.o_sel, S.lse_sel, err_word(),
+                                               gates, o_cmp, nullptr, out, s));
+      return NSA_OK;
+    }
     NSA_TRY_CUDA(nsa::launch_sel_fwd(d, q, k, v, idx, o_sel, lse_sel, err_word(), s));
   }
   if (swa && nsa::swa_combine_fusable(d)) {

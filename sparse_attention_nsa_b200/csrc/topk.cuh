@@ -11,7 +11,8 @@
 // Lane `lane` holds the candidates 1 + lane + 32 q in registers as
 // order-preserving integer keys.  A radix select finds tau, the (topk-2)-th
 // largest key, bit by bit from the top (each step one warp-wide count with
-// redux.sync).  The winners are every key above tau plus, among keys equal
+// redux.sync), stopping early once exactly topk-2 keys lie at or above the
+// prefix found so far.  The winners are every key above tau plus, among keys equal
 // to tau, the lowest block indices (ballots in ascending block order).
 #pragma once
 
@@ -43,14 +44,17 @@ __device__ __forceinline__ void warp_select_blocks(const float* score, int cur, 
   }
   const int K2 = topk - 2;
   // tau = the largest value with at least K2 keys >= tau (absent slots are
-  // excluded from the counts)
+  // excluded from the counts).  The search stops as soon as exactly K2 keys
+  // are >= tau: those are the winners whatever the lower bits of tau.
   uint32_t tau = 0u;
   for (int bit = 31; bit >= 0; --bit) {
     const uint32_t tc = tau | (1u << bit);
     unsigned c = 0;
 #pragma unroll
     for (int q = 0; q < QMAX; ++q) c += (1 + lane + 32 * q < cur && key[q] >= tc) ? 1u : 0u;
-    if ((int)__reduce_add_sync(0xffffffffu, c) >= K2) tau = tc;
+    const int cnt = (int)__reduce_add_sync(0xffffffffu, c);
+    if (cnt >= K2) tau = tc;
+    if (cnt == K2) break;
   }
   unsigned cg = 0;
 #pragma unroll
