@@ -59,6 +59,19 @@ struct Bars {
 constexpr uint32_t OFF_MISC = OFF_BAR + ((sizeof(Bars) + 15) / 16) * 16;
 constexpr uint32_t kSmemBytes = OFF_MISC + 16 + 1024;
 
+// One reduce-scatter step over v[0, 2H): a lane with `upper` set keeps
+// columns [H, 2H), its partner (lane ^ off) the lower ones; each adds the
+// partner's copy of the half it keeps, leaving it in v[0, H).
+template <int H>
+__device__ __forceinline__ void reduce_half(float* v, int upper, int off) {
+#pragma unroll
+  for (int c = 0; c < H; ++c) {
+    const float send = upper ? v[c] : v[c + H];
+    const float keep = upper ? v[c + H] : v[c];
+    v[c] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+  }
+}
+
 template <bool WITH_O>
 __global__ void __launch_bounds__(kThreads, 2)
 cmp_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kc,
@@ -257,15 +270,19 @@ cmp_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         tc_fence_before();
         mbar_arrive(&bars->p[i & 1]);
       }
-      // sum the G heads of each token (consecutive lanes) in fp32
-      for (int off = 1; off < d.G; off <<= 1) {
-#pragma unroll
-        for (int c = 0; c < 64; ++c) sv[c] += __shfl_xor_sync(0xffffffffu, sv[c], off);
-      }
+      // sum the G heads of each token (consecutive lanes) in fp32 with a
+      // reduce-scatter: each step halves the columns a lane keeps and adds
+      // the partner lane's copy of them, so head hh ends with the sums of
+      // columns [hh*per, (hh+1)*per) in sv[0, per)
+      if (d.G >= 2) reduce_half<32>(sv, hh & (32 / per), 32 / per);
+      if (d.G >= 4) reduce_half<16>(sv, hh & (16 / per), 16 / per);
+      if (d.G >= 8) reduce_half<8>(sv, hh & (8 / per), 8 / per);
+      if (d.G >= 16) reduce_half<4>(sv, hh & (4 / per), 4 / per);
+      if (d.G >= 32) reduce_half<2>(sv, hh & (2 / per), 2 / per);
       if (valid) {
 #pragma unroll
         for (int c = 0; c < 64; ++c)
-          if (c / per == hh && j0 + c < d.Nc) srow[j0 + c] = sv[c];
+          if (c < per && j0 + hh * per + c < d.Nc) srow[j0 + hh * per + c] = sv[c];
       }
     }
     if (valid)  // blocks beyond the last chunk are not visible to this tile
