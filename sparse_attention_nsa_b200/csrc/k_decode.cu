@@ -5,16 +5,18 @@
 // Sparse Attention Work? -- compression, selection, sliding window, gated
 // merge).  Decode reads each cached byte once, so it is bound by HBM; the
 // work is split so that all SMs stream:
-//   K1  one CTA per (sequence, KV group): the compressed keys/values of the
-//       sequence (TMA), S = Q Kc^T for the G query heads stacked as MMA rows,
-//       softmax, block scores (summed over the group), o_cmp = P Vc, and the
-//       top-k selection with forced first/current blocks;
+//   K1  one single-warp CTA per (64-block chunk of the compressed cache,
+//       group, sequence): S = Q Kc^T for the G query heads stacked as MMA
+//       rows, the chunk's softmax partial (max, sum, P Vc) and the scaled
+//       logits for the block scores;
 //   K2  one single-warp CTA per (sequence, group, 64-key block) of the
-//       window or the selection: TMA-loads that block's K and V, computes
-//       the block's unnormalised softmax partial (max, sum, P V) for each
-//       branch the block belongs to;
-//   K3  per (sequence, group): merges the partials of each branch and applies
-//       the gates.
+//       window or the selection: TMA-loads that block's K and V and computes
+//       the block's unnormalised softmax partial (max, sum, P V).  Window
+//       blocks are known up front and start before K1 ends; every selection
+//       CTA first computes the group's block scores from K1's logits and the
+//       top-k (the same in each), then takes its own slot's block;
+//   K3  per (sequence, group): merges the partials of the three branches and
+//       applies the gates.
 // The head dimension contractions use warp-level mma.sync (m16n8k16, bf16 in,
 // fp32 accumulate): with G <= 16 heads per group the row count is 16, below
 // the 64/128-row tcgen05 tiles, and the kernel is bandwidth-bound anyway.
@@ -200,7 +202,7 @@ __device__ __forceinline__ void tile_partial(float p[8][4], uint32_t vbase, floa
   }
 }
 
-// ---- K1a: compression branch over one 64-block chunk of the compressed cache --------
+// ---- K1: compression branch over one 64-block chunk of the compressed cache --------
 // One single-warp CTA per (chunk, group, sequence), so every SM streams the
 // compressed cache: S = Q Kc^T for the G heads of the group (rows of the
 // m16n8k16 MMA), the chunk's softmax partial (max, sum, P Vc) for the
@@ -258,69 +260,73 @@ decode_cmp_chunk_kernel(const __grid_constant__ CUtensorMap tm_kc,
                need_o != 0, lane);
 }
 
-// ---- K1b: block scores and top-k per (sequence, group) -----------------------------------
-// score_j = sum over the group's heads of exp2(logit - lse2), lse2 from the
-// chunk partials; then the warp radix select of topk.cuh.
+// ---- the block selection of one (sequence, group), by one warp ----------------------
+// lse of each head row from the compression chunk partials, block scores
+// score_j = sum over the group's heads of exp2(logit - lse2), then the warp
+// radix select of topk.cuh.  Every load of a step is issued before any is
+// used (fixed trip counts, predicated).
 template <int QMAX>
-__global__ void __launch_bounds__(256)
-decode_topk_kernel(Dims d, DecodeWs ws, int32_t* __restrict__ idx_out) {
-  __shared__ float lse2[16];
-  __shared__ float score[QMAX * 32];
-  const int bg = blockIdx.x;
+__device__ __forceinline__ void decode_select(const Dims& d, const DecodeWs& ws, int bg, int lane,
+                                              float* score, int* idx, float* lse2s) {
   const int t = d.T - 1;
   const int cur = t / d.l;
   const int nvis = min((t + 1) / d.l, d.Nc);
-  pdl_launch_dependents();
-  pdl_wait();
-  // every load of a step is issued before any is used (fixed trip counts,
-  // predicated), so each step costs one memory round trip
-  if (threadIdx.x < d.G) {
-    const float* part = ws.pcmp + (size_t)bg * ws.nchunk * 16 * kPartStride + threadIdx.x * kPartStride;
-    float m[kMaxChunks], l[kMaxChunks];
+  if (lane < 16) {
+    float M = -INFINITY, L = 0.f;
+    if (lane < d.G) {
+      const float* part =
+          ws.pcmp + (size_t)bg * ws.nchunk * 16 * kPartStride + lane * kPartStride;
+      float m[kMaxChunks], l[kMaxChunks];
 #pragma unroll
-    for (int c = 0; c < kMaxChunks; ++c) {
-      const bool ok = c < ws.nchunk;
-      m[c] = ok ? part[(size_t)c * 16 * kPartStride + 64] : -INFINITY;
-      l[c] = ok ? part[(size_t)c * 16 * kPartStride + 65] : 0.f;
+      for (int c = 0; c < kMaxChunks; ++c) {
+        const bool ok = c < ws.nchunk;
+        m[c] = ok ? part[(size_t)c * 16 * kPartStride + 64] : -INFINITY;
+        l[c] = ok ? part[(size_t)c * 16 * kPartStride + 65] : 0.f;
+      }
+#pragma unroll
+      for (int c = 0; c < kMaxChunks; ++c) M = fmaxf(M, m[c]);
+#pragma unroll
+      for (int c = 0; c < kMaxChunks; ++c)
+        if (m[c] != -INFINITY) L += fast_exp2(m[c] - M) * l[c];
     }
-    float M = -INFINITY;
-#pragma unroll
-    for (int c = 0; c < kMaxChunks; ++c) M = fmaxf(M, m[c]);
-    float L = 0.f;
-#pragma unroll
-    for (int c = 0; c < kMaxChunks; ++c)
-      if (m[c] != -INFINITY) L += fast_exp2(m[c] - M) * l[c];
-    lse2[threadIdx.x] = L > 0.f ? M + __log2f(L) : INFINITY;  // no visible block: scores 0
+    lse2s[lane] = L > 0.f ? M + __log2f(L) : INFINITY;  // no visible block: scores 0
   }
-  __syncthreads();
+  __syncwarp();
   const float* lg = ws.logit + (size_t)bg * 16 * d.Nc;
-  for (int j = threadIdx.x; j < QMAX * 32; j += blockDim.x) {
-    float x[16];
+  for (int j0 = 0; j0 < QMAX * 32; j0 += 128) {
+    float x[4][16];
 #pragma unroll
-    for (int r = 0; r < 16; ++r) x[r] = (r < d.G && j < nvis) ? lg[(size_t)r * d.Nc + j] : -INFINITY;
-    float sc = 0.f;
+    for (int q = 0; q < 4; ++q) {
+      const int j = j0 + 32 * q + lane;
 #pragma unroll
-    for (int r = 0; r < 16; ++r)
-      if (r < d.G) sc += fast_exp2(x[r] - lse2[r]);
-    score[j] = sc;
+      for (int r = 0; r < 16; ++r)
+        x[q][r] = (r < d.G && j < nvis) ? lg[(size_t)r * d.Nc + j] : -INFINITY;
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float sc = 0.f;
+#pragma unroll
+      for (int r = 0; r < 16; ++r)
+        if (r < d.G) sc += fast_exp2(x[q][r] - lse2s[r]);
+      if (j0 + 32 * q < QMAX * 32) score[j0 + 32 * q + lane] = sc;
+    }
   }
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    int* out = ws.idx + (size_t)bg * d.topk;
-    warp_select_blocks<QMAX>(score, cur, d.topk, out, threadIdx.x);
-    __syncwarp();
-    if (idx_out)
-      for (int m = threadIdx.x; m < d.topk; m += 32) idx_out[(size_t)bg * d.topk + m] = out[m];
-  }
+  __syncwarp();
+  warp_select_blocks<QMAX>(score, cur, d.topk, idx, lane);
+  __syncwarp();
 }
 
 // ---- K2: one 64-key block of the window or the selection ------------------------------
+template <int QMAX>
 __global__ void __launch_bounds__(32)
 decode_block_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                    const bf16* __restrict__ q, Dims d, DecodeWs ws, int do_sel, int do_swa,
-                    int* err) {
+                    const bf16* __restrict__ q, Dims d, DecodeWs ws, int32_t* __restrict__ idx_out,
+                    int do_sel, int do_swa, int* err) {
   __shared__ __align__(1024) uint8_t kv[2 * 8192];
   __shared__ __align__(1024) uint8_t qs[2048];
+  __shared__ float score_s[QMAX * 32];
+  __shared__ int idx_s[64];
+  __shared__ float lse2_s[16];
   __shared__ uint64_t bar;
   __shared__ int abort_s;
   const int lane = threadIdx.x;
@@ -328,10 +334,10 @@ decode_block_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
   const int bg = b * d.Hkv + g;
   const int t = d.T - 1;
   const int cur = t / d.l;
-  const int* sel = ws.idx + (size_t)bg * d.topk;
   pdl_launch_dependents();
-  // which block, and which branches it serves here; window blocks are known
-  // before the selection, so their loads start before K1 has finished
+  // which block and branch: window blocks are known before the selection, so
+  // their loads start before K1 has finished; a selected block inside the
+  // window gets its own CTA (the two branches mask it differently)
   int j, sel_slot = -1;
   bool win = false;
   if (u < ws.nwin) {
@@ -342,16 +348,23 @@ decode_block_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     j = ws.jlo + u;
     win = true;
   } else {
-    if (!do_sel) return;
     pdl_wait();
+    if (!do_sel) return;
+    // every selection CTA of the (sequence, group) runs the same selection
+    // (no kernel boundary between the scores and their use); slot 0 stores it
     const int m = u - ws.nwin;
-    j = sel[m];
+    decode_select<QMAX>(d, ws, bg, lane, score_s, idx_s, lse2_s);
+    if (m == 0)
+      for (int s = lane; s < d.topk; s += 32) {
+        ws.idx[(size_t)bg * d.topk + s] = idx_s[s];
+        if (idx_out) idx_out[(size_t)bg * d.topk + s] = idx_s[s];
+      }
+    j = idx_s[m];
     if (j < 0) return;
     if (j > cur) {  // never read a non-causal block
       if (lane == 0) record_error(err, kDevBadIndex);
       return;
     }
-    if (do_swa && j >= ws.jlo) return;  // its window CTA covers the selection too
     sel_slot = m;
   }
   if (lane == 0) {
@@ -366,11 +379,6 @@ decode_block_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     tma_load_3d(kv + 8192, &tm_v, &bar, 0, g, b * d.T + j * 64);
   }
   stage_q(qs, q + ((size_t)b * d.Hq + (size_t)g * d.G) * 64, d.G, lane);
-  if (win && do_sel) {  // is this window block also selected?
-    pdl_wait();
-    for (int m = 0; m < d.topk; ++m)
-      if (sel[m] == j) sel_slot = m;
-  }
   fence_proxy_async_smem();
   __syncwarp();
   uint32_t qa[4][4];
@@ -436,7 +444,7 @@ decode_block_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
       part[(r0 + 8) * kPartStride + 65] = l1;
     }
   }
-  if (win && !do_sel) pdl_wait();  // see the early return above
+  if (win) pdl_wait();  // completion of this grid implies completion of the ones before
 }
 
 // ---- K3: merge the partials of each branch and apply the gates ------------------------
@@ -572,8 +580,8 @@ size_t decode_split_ws_bytes(const Dims& d) {
          al256(bgn * nwin * 16 * kPartStride * 4);
 }
 
-// K1a (chunks of the compressed cache) -> K1b (block scores, top-k) -> K2
-// (selected and window blocks) -> K3 (merge, gates), chained with
+// K1 (chunks of the compressed cache) -> K2 (block scores and top-k, then
+// the selected and window blocks) -> K3 (merge, gates), chained with
 // programmatic dependent launch: each kernel's prologue overlaps the tail of
 // the previous one, and every CTA of a dependent kernel waits for its
 // predecessor before it exits, so completion is transitive.
@@ -616,17 +624,6 @@ cudaError_t launch_decode_split(const Dims& d, const void* q, const void* kcache
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  if (sel) {  // also when no block is complete yet: the forced blocks still go out
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)bgn);
-    cfg.blockDim = dim3(256);
-    cfg.stream = s;
-    cfg.attrs = pdl;
-    cfg.numAttrs = 1;
-    cudaError_t e = d.Nc <= 512 ? cudaLaunchKernelEx(&cfg, decode_topk_kernel<16>, d, ws, idx_out)
-                                : cudaLaunchKernelEx(&cfg, decode_topk_kernel<32>, d, ws, idx_out);
-    if (e != cudaSuccess) return e;
-  }
   if (sel || swa) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(ws.nwin + d.topk, d.Hkv, d.B);
@@ -635,7 +632,10 @@ cudaError_t launch_decode_split(const Dims& d, const void* q, const void* kcache
     cfg.attrs = pdl;
     cfg.numAttrs = 1;
     const int ds = sel ? 1 : 0, dw = swa ? 1 : 0;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, decode_block_kernel, mk, mv, qb, d, ws, ds, dw, err);
+    cudaError_t e =
+        d.Nc <= 512
+            ? cudaLaunchKernelEx(&cfg, decode_block_kernel<16>, mk, mv, qb, d, ws, idx_out, ds, dw, err)
+            : cudaLaunchKernelEx(&cfg, decode_block_kernel<32>, mk, mv, qb, d, ws, idx_out, ds, dw, err);
     if (e != cudaSuccess) return e;
   }
   cudaLaunchConfig_t cfg = {};
