@@ -476,6 +476,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="nsa", choices=["nsa", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--leg", default="all", choices=["all", "decode", "train"],
+                    help="decode / train: run only that leg on one GPU and print its "
+                         "numbers (for profiling that leg alone); all: the benchmark")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -483,6 +486,16 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args, rank)
+        return
+    if args.leg != "all":
+        dev = torch.device("cuda", 0)
+        torch.cuda.set_device(dev)
+        nsa.load()
+        flush, stream, peaks = Flusher(dev), torch.cuda.current_stream(), load_peaks()
+        if args.leg == "decode":
+            print(json.dumps({"decode": run_decode(dev, flush, stream, args.steps, peaks)}))
+        else:
+            print(json.dumps({"train": run_train(dev, flush, stream, args.steps, peaks)}))
         return
     dist_on = world > 1
     if dist_on:
