@@ -299,6 +299,8 @@ def check_decode(w, inp, seqs):
     W.DECODE_32K.replace(name="decode_small", B=3, T=1500),
     W.DECODE_32K.replace(name="decode_gqa_ragged", B=5, T=2049, Hq=16, Hkv=4),
     W.DECODE_32K.replace(name="decode_short", B=2, T=70),
+    # 625 compressed blocks: ten K1 chunks and the 32-slot-per-lane top-k
+    W.DECODE_32K.replace(name="decode_long_nc625", B=2, T=40000),
     W.DECODE_32K.replace(name="decode_pruned_w100_k4", B=4, T=5000, topk=4, window=100,
                          branch_mask=W.BR_SEL | W.BR_SWA, cmp_gate_zero=True),
     W.DECODE_32K.replace(name="decode_swa_only_gqa8", B=3, T=3333, Hq=16, Hkv=2, window=200,
@@ -320,7 +322,10 @@ def sample_rows(w, n, seed):
     return np.array([[int(g.integers(0, w.B)), t] for t in ts])
 
 
-@pytest.mark.parametrize("w", [W.NSA_340M, W.PRUNED_32K, W.NSA_1P3B], ids=lambda w: w.name)
+@pytest.mark.parametrize("w", [W.NSA_340M, W.PRUNED_32K, W.NSA_1P3B,
+                               # 625 selection blocks: the 32-slot-per-lane top-k
+                               W.NSA_340M.replace(name="gqa4_t40000_nb625", T=40000)],
+                         ids=lambda w: w.name)
 def test_forward_full_size_sampled(cuda_lib, w):
     inp = W.make_inputs(w, seed=0)
     out, saved = gpu_forward(w, inp)
