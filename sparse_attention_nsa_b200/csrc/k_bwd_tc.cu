@@ -417,9 +417,10 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 // range is bounded (P in [0, 1]; dO a gradient).
 // TMEM (512 columns, one CTA per SM): S^T [0,128), dP^T [128,256),
 // dV [256,320), dK [320,384), P^T (fp16) [384,448), dS^T hi [448,512).
-// Warps: 0-3 key threads and epilogue, 4 MMA issue and TMEM owner (and the
-// K/V TMA), 5-8 row gather.
-constexpr int kKvThreads = 288;
+// Warps: 0-3 key threads and epilogue, 4 S^T/dP^T issue and TMEM owner (and
+// the K/V TMA), 5-8 row gather, 9 dV/dK issue (its 24 MMAs per tile overlap
+// the next tile's S^T/dP^T and key-thread work).
+constexpr int kKvThreads = 320;
 constexpr int kCmpShares = 16;  // row shares of a compression-branch key pair
 constexpr uint32_t kKTile2 = 128 * 64 * 2;  // 128 keys x 64 dims, bf16
 constexpr uint32_t kRowTile = 128 * 64 * 2;
@@ -451,6 +452,7 @@ struct KvBars {
   uint64_t sfree;       // 128 key threads loaded them
   uint64_t p;           // 128 key threads wrote P^T and dS^T
   uint64_t bfree[2];    // dV / dK MMAs of the tile in row buffer u & 1 done
+  uint64_t sdone;       // every S^T / dP^T MMA done (unwinding)
   uint64_t fin;
 };
 constexpr uint32_t KV_OFF_MISC = KV_OFF_BAR + ((sizeof(KvBars) + 15) / 16) * 16;
@@ -540,6 +542,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     mbar_init(&bars->s, 1);
     mbar_init(&bars->sfree, 128);
     mbar_init(&bars->p, 128);
+    mbar_init(&bars->sdone, 1);
     mbar_init(&bars->fin, 1);
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -550,7 +553,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp >= 5) {
+  if (warp >= 5 && warp <= 8) {
     // ---- row gather: thread gr fills row gr of each tile ------------------------------
     const int gr = tid - 160;
     for (int u = 0; u < ntiles; ++u) {
@@ -603,13 +606,9 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
       mbar_arrive(&bars->gathered[bu]);
     }
   } else if (warp == 4) {
-    // ---- MMA issue (and the pair's K/V by TMA) ----------------------------------------
+    // ---- S^T / dP^T issue (and the pair's K/V by TMA) ---------------------------------
     if (lane == 0) {
-      constexpr uint32_t idesc_st = idesc_bf16(128, 128, false, false);  // S^T, dP^T
-      constexpr uint32_t idesc_kv = idesc_bf16(128, 64, false, true);    // dK (hi)
-      constexpr uint32_t idesc_kl = idesc_bf16(128, 64, false, true);    // dK (lo, A from smem)
-      constexpr uint32_t idesc_v16 = idesc_f16(128, 64, false, true);    // dV (fp16)
-      const uint32_t dsl_addr = smem_u32(smem + KV_OFF_DSL);
+      constexpr uint32_t idesc_st = idesc_bf16(128, 128, false, false);
       const uint32_t k_addr = smem_u32(smem + KV_OFF_K), v_addr = smem_u32(smem + KV_OFF_V);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
@@ -618,11 +617,45 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         tma_load_3d(smem + KV_OFF_K + h * kTileBytes, &tm_k, &bars->kv, 0, g, b * nkeys + kbase + h * kKeys);
         tma_load_3d(smem + KV_OFF_V + h * kTileBytes, &tm_v, &bars->kv, 0, g, b * nkeys + kbase + h * kKeys);
       }
-      bool ok = wait_bar(&bars->kv, 0, abort_flag, err);
-      auto issue_kv = [&](int u) -> bool {
-        // dV += P^T dO and dK += dS^T Q of tile u (A operands in TMEM, the
-        // gathered tiles read MN-major: K dimension = rows)
-        if (!wait_bar(&bars->p, u & 1, abort_flag, err)) return false;
+      const bool ok = wait_bar(&bars->kv, 0, abort_flag, err);
+      for (int u = 0; ok && u < ntiles; ++u) {
+        const int bu = u & 1;
+        if (!wait_bar(&bars->gathered[bu], (u >> 1) & 1, abort_flag, err)) break;
+        // S^T / dP^T are single-buffered: the key threads must have loaded tile u-1's
+        if (u >= 1 && !wait_bar(&bars->sfree, (u - 1) & 1, abort_flag, err)) break;
+        tc_fence_after();
+        const uint32_t q_addr = smem_u32(smem + KV_OFF_Q + bu * kRowTile);
+        const uint32_t do_addr = smem_u32(smem + KV_OFF_DO + bu * kRowTile);
+        const uint32_t dol_addr = smem_u32(smem + KV_OFF_DOL + bu * kRowTile);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmem + kvColS, desc_sw128(k_addr + kk * 32, 16), desc_sw128(q_addr + kk * 32, 16),
+                   idesc_st, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmem + kvColDP, desc_sw128(v_addr + kk * 32, 16), desc_sw128(do_addr + kk * 32, 16),
+                   idesc_st, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)  // dO lo: dP^T keeps about fp32 accuracy
+          mma_bf16(tmem + kvColDP, desc_sw128(v_addr + kk * 32, 16), desc_sw128(dol_addr + kk * 32, 16),
+                   idesc_st, 1u);
+        mma_commit(&bars->s);
+      }
+      mma_commit(&bars->sdone);
+      drain_bar(&bars->sdone, 0);
+      if (!ok) drain_bar(&bars->kv, 0);
+    }
+  } else if (warp == 9) {
+    // ---- dV += P^T dO, dK += dS^T Q issue ----------------------------------------------
+    if (lane == 0) {
+      constexpr uint32_t idesc_kv = idesc_bf16(128, 64, false, true);  // dK (hi, A in TMEM)
+      constexpr uint32_t idesc_kl = idesc_bf16(128, 64, false, true);  // dK (lo, A from smem)
+      constexpr uint32_t idesc_v16 = idesc_f16(128, 64, false, true);  // dV (fp16)
+      const uint32_t dsl_addr = smem_u32(smem + KV_OFF_DSL);
+      for (int u = 0; u < ntiles; ++u) {
+        // A operands in TMEM (and dS^T lo in smem); the gathered tiles read
+        // MN-major: K dimension = rows
+        if (!wait_bar(&bars->p, u & 1, abort_flag, err)) break;
         tc_fence_after();
         const int bu = u & 1;
         const uint32_t q_addr = smem_u32(smem + KV_OFF_Q + bu * kRowTile);
@@ -639,36 +672,9 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                    qb, idesc_kl, 1u);
         }
         mma_commit(&bars->bfree[bu]);  // frees the row buffer and the P^T / dS^T columns
-        return true;
-      };
-      for (int u = 0; ok && u < ntiles; ++u) {
-        const int bu = u & 1;
-        if (!wait_bar(&bars->gathered[bu], (u >> 1) & 1, abort_flag, err)) break;
-        // S^T / dP^T are single-buffered: the key threads must have loaded tile u-1's
-        if (u >= 1 && !wait_bar(&bars->sfree, (u - 1) & 1, abort_flag, err)) break;
-        tc_fence_after();
-        const uint32_t q_addr = smem_u32(smem + KV_OFF_Q + bu * kRowTile);
-        const uint32_t do_addr = smem_u32(smem + KV_OFF_DO + bu * kRowTile);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + kvColS, desc_sw128(k_addr + kk * 32, 16), desc_sw128(q_addr + kk * 32, 16),
-                   idesc_st, kk > 0);
-        const uint32_t dol_addr = smem_u32(smem + KV_OFF_DOL + bu * kRowTile);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + kvColDP, desc_sw128(v_addr + kk * 32, 16), desc_sw128(do_addr + kk * 32, 16),
-                   idesc_st, kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)  // dO lo: dP^T keeps about fp32 accuracy
-          mma_bf16(tmem + kvColDP, desc_sw128(v_addr + kk * 32, 16), desc_sw128(dol_addr + kk * 32, 16),
-                   idesc_st, 1u);
-        mma_commit(&bars->s);
-        if (u >= 1 && !issue_kv(u - 1)) break;
-        if (u == ntiles - 1) issue_kv(u);
       }
       mma_commit(&bars->fin);
       drain_bar(&bars->fin, 0);
-      if (!ok) drain_bar(&bars->kv, 0);
     }
   } else {
     // ---- key threads: thread k owns key kbase + k (TMEM lane k) -------------------------
@@ -685,14 +691,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         break;
       }
       tc_fence_after();
-      // P^T / dS^T (TMEM and the dS lo tile): the dV/dK MMAs of tile u-1 must have read them
-      if (u >= 1) {
-        if (!wait_bar_warp(&bars->bfree[(u - 1) & 1], ((u - 1) >> 1) & 1, abort_flag, err)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-      }
+      bool stop = false;
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {  // 32 rows at a time
         float sv[32], pv[32];
@@ -724,6 +723,15 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
           dd[e / 2] = pack_bf16(h0, h1);
           dl[e / 2] = pack_bf16(d2[0] - h0, d2[1] - h1);
         }
+        if (c == 0 && u >= 1) {
+          // P^T / dS^T (TMEM and the dS lo tile): the dV/dK MMAs of tile u-1
+          // must have read them (waited for only now, after the first 32 rows)
+          if (!wait_bar_warp(&bars->bfree[(u - 1) & 1], ((u - 1) >> 1) & 1, abort_flag, err)) {
+            stop = true;
+            break;
+          }
+          tc_fence_after();
+        }
         tmem_st16u(lane_tmem + kvColP + 16u * c, pp);
         tmem_st16u(lane_tmem + kvColDS + 16u * c, dd);
         // dS lo into the K-major smem tile: row k, rows 32c .. 32c+31 of the
@@ -736,6 +744,10 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
           st_shared_v4(lrow + ((uint32_t)(cc ^ (k & 7)) << 4), dl[4 * q4], dl[4 * q4 + 1],
                        dl[4 * q4 + 2], dl[4 * q4 + 3]);
         }
+      }
+      if (stop) {
+        ok = false;
+        break;
       }
       fence_proxy_async_smem();  // dS lo is read by the MMA (async proxy)
       tmem_wait_st();
