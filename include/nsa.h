@@ -169,6 +169,27 @@ nsa_status nsa_sel_attn_fwd(const nsa_params* p, const void* q, const void* k,
                             const void* v, const int32_t* idx, void* o_sel,
                             float* lse_sel, void* stream);
 
+/* The same selection branch, block-major, with a caller workspace of at
+ * least nsa_sel_workspace_size(p) bytes (256-byte aligned).  The queries
+ * that chose each block are gathered from a reverse map (block -> queries),
+ * each (query, head, block) pair gets its own softmax over the block's keys,
+ * and each row's partials are merged exactly with their log-sum-exps (the
+ * split-softmax identity); results match nsa_sel_attn_fwd up to rounding.
+ * nsa_forward takes this path itself when Tq >= 64 and Nb >= 16 topk (the
+ * query-tiled kernel's union of blocks grows with Nb / topk).  Passage: as for
+ * nsa_sel_attn_fwd, plus the kernel paragraph (each block is loaded once for
+ * all the queries that selected it).  o_sel may be NULL (not
+ * stored), as may lse_sel.  Index errors are recorded as in nsa_sel_attn_fwd;
+ * the per-block partial outputs are held in fp16, and a value beyond its
+ * range (|v| > 65504) is recorded as NSA_ERR_DEVICE_CHECK.
+ * Returns NSA_ERR_UNSUPPORTED for shapes the block-major kernels do not
+ * cover (fp32, block size != 64, D != 64, 128 % G != 0). */
+nsa_status nsa_sel_workspace_size(const nsa_params* p, size_t* bytes);
+nsa_status nsa_sel_attn_fwd_ws(const nsa_params* p, const void* q, const void* k,
+                               const void* v, const int32_t* idx, void* o_sel,
+                               float* lse_sel, void* workspace, size_t workspace_bytes,
+                               void* stream);
+
 /* ---- sliding-window branch -----------------------------------------------
  * o_swa[t,h] attends to keys max(0, t-w+1) <= s <= t.
  * Passage: "DeepSeek's Native Sparse Attention", SLIDING WINDOW;

@@ -31,7 +31,8 @@ EXPORTS = ("nsa_status_string", "nsa_check_params", "nsa_workspace_size",
            "nsa_select_topk", "nsa_sel_attn_fwd", "nsa_swa_fwd", "nsa_gate_combine",
            "nsa_forward", "nsa_decode", "nsa_backward_workspace_size",
            "nsa_gate_combine_bwd", "nsa_sel_attn_bwd", "nsa_swa_bwd", "nsa_cmp_bwd",
-           "nsa_backward", "nsa_decode_noalloc", "nsa_decode_noalloc_max_scratch")
+           "nsa_backward", "nsa_decode_noalloc", "nsa_decode_noalloc_max_scratch",
+           "nsa_sel_workspace_size", "nsa_sel_attn_fwd_ws")
 
 
 class NsaError(RuntimeError):
@@ -104,6 +105,8 @@ def load():
             "nsa_backward": ([P, vp, vp, vp, vp, vp, C.POINTER(Saved), vp, vp, vp, vp, vp,
                               C.c_size_t, vp], C.c_int),
             "nsa_decode_noalloc_max_scratch": ([], C.c_size_t),
+            "nsa_sel_workspace_size": ([P, C.POINTER(C.c_size_t)], C.c_int),
+            "nsa_sel_attn_fwd_ws": ([P, vp, vp, vp, vp, vp, vp, vp, C.c_size_t, vp], C.c_int),
         }
         for name, (args, res) in sig.items():
             f = getattr(lib, name)
@@ -221,6 +224,23 @@ def nsa_sel_attn_fwd(p: Params, q, k, v, idx, o_sel, lse_sel, stream=None):
         _ptr(v, s["k"], dt, "v"), _ptr(idx, s["idx"], torch.int32, "idx"),
         _ptr(o_sel, s["o"], dt, "o_sel"), _ptr(lse_sel, s["lse"], torch.float32, "lse_sel", True),
         _stream(stream)), "nsa_sel_attn_fwd")
+
+
+def nsa_sel_workspace_size(p: Params) -> int:
+    n = C.c_size_t(0)
+    _check(load().nsa_sel_workspace_size(C.byref(p), C.byref(n)), "nsa_sel_workspace_size")
+    return n.value
+
+
+def nsa_sel_attn_fwd_ws(p: Params, q, k, v, idx, o_sel, lse_sel, workspace, stream=None):
+    s, dt = _shapes(p), p.torch_dtype
+    _check(load().nsa_sel_attn_fwd_ws(
+        C.byref(p), _ptr(q, s["q"], dt, "q"), _ptr(k, s["k"], dt, "k"),
+        _ptr(v, s["k"], dt, "v"), _ptr(idx, s["idx"], torch.int32, "idx"),
+        _ptr(o_sel, s["o"], dt, "o_sel", True),
+        _ptr(lse_sel, s["lse"], torch.float32, "lse_sel", True),
+        _ptr(workspace, None, torch.uint8, "workspace"), C.c_size_t(workspace.numel()),
+        _stream(stream)), "nsa_sel_attn_fwd_ws")
 
 
 def nsa_swa_fwd(p: Params, q, k, v, o_swa, lse_swa, stream=None):

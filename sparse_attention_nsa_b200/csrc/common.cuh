@@ -15,6 +15,7 @@ enum : int {
   kDevOk = 0,
   kDevTimeout = 1,   // a bounded wait gave up
   kDevBadIndex = 2,  // a block index was out of range / not causal / unsorted
+  kDevRange = 3,     // a value exceeded an intermediate format's range
 };
 
 __device__ __forceinline__ void record_error(int* err, int code) {

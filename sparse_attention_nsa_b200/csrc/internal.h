@@ -48,6 +48,25 @@ cudaError_t launch_sel_fwd_combine(const Dims& d, const void* q, const void* k, 
                                    const int32_t* idx, void* o_sel, float* lse_sel, int* err,
                                    const float* gates, const void* o_cmp, const void* o_swa,
                                    void* out, cudaStream_t s);
+// Gated combination fused into an attention epilogue: out = gate_own * o +
+// sum over the non-NULL other[i] of gate(other_gate[i]) * other[i]; gate i of
+// a row is gates[row * 3 + i] in the order (cmp, sel, swa); bf16 rows of 64.
+struct EpilogueFuse {
+  const float* gates;
+  const void* other[2];
+  int other_gate[2];
+  int own_gate;
+  void* out;
+};
+// block-major selection (k_sel_bm.cu): reverse map, per-(query, slot)
+// partials, merge; fz (may be NULL) fuses the gated combination into the
+// merge.  ws: sel_bm_ws_bytes(d) bytes, 256-byte aligned.  o_sel and
+// lse_sel may be NULL (not stored).
+bool sel_bm_eligible(const Dims& d);
+size_t sel_bm_ws_bytes(const Dims& d);
+cudaError_t launch_sel_bm(const Dims& d, const void* q, const void* k, const void* v,
+                          const int32_t* idx, void* o_sel, float* lse_sel, int* err,
+                          const EpilogueFuse* fz, void* ws, cudaStream_t s);
 cudaError_t launch_combine(const Dims& d, const float* gates, const void* o_cmp,
                            const void* o_sel, const void* o_swa, void* out,
                            cudaStream_t s);
@@ -68,6 +87,15 @@ cudaError_t launch_dq_tc(const Dims& d, int mode, const void* q, const void* key
 size_t revmap_chunk_ints(const Dims& d);
 cudaError_t launch_revmap(const Dims& d, const int32_t* idx, int* chunk, int* offsets,
                           int* list, cudaStream_t s);
+// the same map for the block-major selection forward: entries are
+// query << 6 | slot in no particular order within a block's list, indices
+// that break the forward's rule are reported in err, and per (sequence,
+// group) the lists are cut into work units of at most tpu entries
+// (units[bg * umax + u] = (block, first, end) for u < ucount[bg]).
+// cursor: B * Hkv * Nb ints.
+cudaError_t launch_revmap_units(const Dims& d, const int32_t* idx, int* chunk, int* offsets,
+                                int* cursor, int* list, int4* units, int* ucount, int tpu,
+                                int umax, int* err, cudaStream_t s);
 cudaError_t launch_dkdv(const Dims& d, int mode, const void* q, const void* keys,
                         const void* vals, const float* lse, const float* delta,
                         const float* dO, const int* offsets, const int* list, float* dk,

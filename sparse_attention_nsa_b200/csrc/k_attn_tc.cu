@@ -90,18 +90,10 @@ __host__ __device__ inline size_t list_ints(const Dims& d) {
   return (size_t)d.Nb + words + (size_t)tokens_per_tile(d.G) * (d.topk + 1);
 }
 
-// Gated combination fused into the epilogue of the branch that runs last
-// in a forward: out = g_own o_own + sum of g_i o_i over the other enabled
-// branches (stored bf16 outputs), with o_own unrounded; o_own itself is
-// stored only when `o` is not null.  Gate i is gates[row * 3 + i] in the
-// order (cmp, sel, swa).
-struct Fuse {
-  const float* gates;
-  const bf16* other[2];  // NULL when that branch is disabled
-  int other_gate[2];
-  int own_gate;
-  bf16* out;
-};
+// The gated combination (EpilogueFuse) is fused into the epilogue of the
+// branch that runs last in a forward, with o_own unrounded; o_own itself is
+// stored only when `o` is not null.
+using Fuse = EpilogueFuse;
 
 template <bool SEL, bool FUSE>
 __global__ void __launch_bounds__(kThreads, 2)
@@ -458,7 +450,7 @@ attn_tc_kernel(const bf16* __restrict__ qg, const __grid_constant__ CUtensorMap 
         for (int br = 0; br < 2; ++br) {
           if (!fz.other[br]) continue;
           const float gb = fz.gates[row * 3 + fz.other_gate[br]];
-          const uint4* src = reinterpret_cast<const uint4*>(fz.other[br] + row * 64);
+          const uint4* src = reinterpret_cast<const uint4*>((const bf16*)fz.other[br] + row * 64);
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             const uint4 u = src[c];
@@ -471,7 +463,7 @@ attn_tc_kernel(const bf16* __restrict__ qg, const __grid_constant__ CUtensorMap 
             }
           }
         }
-        uint4* dst = reinterpret_cast<uint4*>(fz.out + row * 64);
+        uint4* dst = reinterpret_cast<uint4*>((bf16*)fz.out + row * 64);
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           uint4 u;
@@ -540,11 +532,10 @@ cudaError_t launch_swa_fwd_combine(const Dims& d, const void* q, const void* k, 
                                    const void* o_cmp, const void* o_sel, void* out,
                                    cudaStream_t s) {
   Fuse fz{gates,
-          {(d.branch_mask & 1) ? (const bf16*)o_cmp : nullptr,
-           (d.branch_mask & 2) ? (const bf16*)o_sel : nullptr},
+          {(d.branch_mask & 1) ? o_cmp : nullptr, (d.branch_mask & 2) ? o_sel : nullptr},
           {0, 1},
           2,
-          (bf16*)out};
+          out};
   return launch_tc<false, true>(d, q, k, v, nullptr, o_swa, lse_swa, nullptr, fz, s);
 }
 
@@ -553,11 +544,10 @@ cudaError_t launch_sel_fwd_combine(const Dims& d, const void* q, const void* k, 
                                    const float* gates, const void* o_cmp, const void* o_swa,
                                    void* out, cudaStream_t s) {
   Fuse fz{gates,
-          {(d.branch_mask & 1) ? (const bf16*)o_cmp : nullptr,
-           (d.branch_mask & 4) ? (const bf16*)o_swa : nullptr},
+          {(d.branch_mask & 1) ? o_cmp : nullptr, (d.branch_mask & 4) ? o_swa : nullptr},
           {0, 2},
           1,
-          (bf16*)out};
+          out};
   return launch_tc<true, true>(d, q, k, v, idx, o_sel, lse_sel, err, fz, s);
 }
 

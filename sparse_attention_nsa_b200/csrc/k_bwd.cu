@@ -191,7 +191,8 @@ __device__ __forceinline__ bool rev_valid(const int32_t* ir, int s, int cur) {
 }
 
 __global__ void __launch_bounds__(kRevChunk)
-rev_chunk_count_kernel(const int32_t* __restrict__ idx, int* __restrict__ chunk, Dims d) {
+rev_chunk_count_kernel(const int32_t* __restrict__ idx, int* __restrict__ chunk, Dims d,
+                       int* err) {
   extern __shared__ int hist[];  // [Nb]
   const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int nchunk = gridDim.x;
@@ -201,8 +202,16 @@ rev_chunk_count_kernel(const int32_t* __restrict__ idx, int* __restrict__ chunk,
   if (tq < d.Tq) {
     const int32_t* ir = idx + (((size_t)b * d.Tq + tq) * d.Hkv + g) * d.topk;
     const int cur = (d.q_off + tq) / d.l;
-    for (int s = 0; s < d.topk; ++s)
+    int prev = -1;
+    for (int s = 0; s < d.topk; ++s) {
       if (rev_valid(ir, s, cur)) atomicAdd(&hist[ir[s]], 1);
+      if (err) {  // the forward's rule: -1 or a causal block above the last one
+        const int j = ir[s];
+        if (j == -1) continue;
+        if (j < -1 || j <= prev || j > cur) record_error(err, kDevBadIndex);
+        else prev = j;
+      }
+    }
   }
   __syncthreads();
   int* out = chunk + (((size_t)b * d.Hkv + g) * nchunk + c) * d.Nb;
@@ -212,7 +221,9 @@ rev_chunk_count_kernel(const int32_t* __restrict__ idx, int* __restrict__ chunk,
 // one CTA per (sequence, group); chunk[c][j] becomes chunk c's first list
 // position for block j
 __global__ void __launch_bounds__(1024)
-rev_chunk_scan_kernel(int* __restrict__ chunk, int* __restrict__ offsets, Dims d, int nchunk) {
+rev_chunk_scan_kernel(int* __restrict__ chunk, int* __restrict__ offsets, Dims d, int nchunk,
+                      int4* __restrict__ units, int* __restrict__ ucount, int* __restrict__ cursor,
+                      int tpu, int umax) {
   extern __shared__ int tot[];  // [Nb]
   __shared__ int wsum[32];
   const int bg = blockIdx.x;
@@ -265,6 +276,40 @@ rev_chunk_scan_kernel(int* __restrict__ chunk, int* __restrict__ offsets, Dims d
   __syncthreads();
   for (int j = threadIdx.x; j < d.Nb; j += blockDim.x)
     for (int c = 0; c < nchunk; ++c) cc[(size_t)c * d.Nb + j] += tot[j];
+  if (!units) return;
+  // work units of at most tpu list entries: block j's list [off[j], off[j+1])
+  // split into ceil(len / tpu) consecutive pieces, blocks in ascending order
+  int nu = 0;
+  for (int j = lo; j < hi; ++j) nu += (off[j + 1] - off[j] + tpu - 1) / tpu;
+  int ui = nu;
+#pragma unroll
+  for (int o2 = 1; o2 < 32; o2 <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, ui, o2);
+    if (lane >= o2) ui += y;
+  }
+  __syncthreads();  // wsum is reused
+  if (lane == 31) wsum[warp] = ui;
+  __syncthreads();
+  if (warp == 0) {
+    const int nw = (blockDim.x + 31) / 32;
+    int w = lane < nw ? wsum[lane] : 0;
+    int wi = w;
+#pragma unroll
+    for (int o2 = 1; o2 < 32; o2 <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, wi, o2);
+      if (lane >= o2) wi += y;
+    }
+    wsum[lane] = wi - w;
+    if (lane == 31) ucount[bg] = wi;
+  }
+  __syncthreads();
+  int at = wsum[warp] + ui - nu;
+  int4* ub = units + (size_t)bg * umax;
+  for (int j = lo; j < hi; ++j) {
+    cursor[(size_t)bg * d.Nb + j] = off[j];
+    for (int p0 = off[j]; p0 < off[j + 1]; p0 += tpu)
+      ub[at++] = make_int4(j, p0, min(p0 + tpu, off[j + 1]), 0);
+  }
 }
 
 // one warp per (chunk, group, sequence)
@@ -310,6 +355,38 @@ rev_chunk_fill_kernel(const int32_t* __restrict__ idx, const int* __restrict__ c
         }
       }
     __syncwarp();
+  }
+}
+
+// The forward's fill, entries query << 6 | slot (topk <= 64).  The order
+// inside a block's list is free (each (query, slot) pair is computed on its
+// own), so positions come from one atomic cursor per (sequence, group,
+// block), started at the block's scanned offset, the lanes of a warp that
+// chose the same block sharing one atomic.  One thread per query.
+__global__ void __launch_bounds__(256)
+rev_atomic_fill_kernel(const int32_t* __restrict__ idx, int* __restrict__ cursor,
+                       int* __restrict__ list, Dims d) {
+  const int tq = blockIdx.x * blockDim.x + threadIdx.x;
+  const int g = blockIdx.y, b = blockIdx.z;
+  const int lane = threadIdx.x & 31;
+  const bool q_ok = tq < d.Tq;
+  const size_t bg = (size_t)b * d.Hkv + g;
+  const int32_t* ir = idx + (((size_t)b * d.Tq + (q_ok ? tq : 0)) * d.Hkv + g) * d.topk;
+  const int cur = (d.q_off + tq) / d.l;
+  int* cb = cursor + bg * d.Nb;
+  int* lst = list + bg * (size_t)d.Tq * d.topk;
+  for (int s = 0; s < d.topk; ++s) {
+    const bool v = q_ok && rev_valid(ir, s, cur);
+    const unsigned act = __ballot_sync(0xffffffffu, v);
+    if (v) {
+      const int j = ir[s];
+      const unsigned peers = __match_any_sync(act, j);
+      const int leader = __ffs(peers) - 1;
+      int base = 0;
+      if (lane == leader) base = atomicAdd(cb + j, __popc(peers));
+      base = __shfl_sync(peers, base, leader);
+      lst[base + __popc(peers & ((1u << lane) - 1u))] = (tq << 6) | s;
+    }
   }
 }
 
@@ -497,9 +574,27 @@ cudaError_t launch_revmap(const Dims& d, const int32_t* idx, int* chunk, int* of
   const int nchunk = (d.Tq + kRevChunk - 1) / kRevChunk;
   if (nchunk == 0 || d.Nb == 0) return cudaSuccess;
   const size_t nb_bytes = (size_t)d.Nb * sizeof(int);
-  rev_chunk_count_kernel<<<dim3(nchunk, d.Hkv, d.B), kRevChunk, nb_bytes, s>>>(idx, chunk, d);
-  rev_chunk_scan_kernel<<<d.B * d.Hkv, 1024, nb_bytes, s>>>(chunk, offsets, d, nchunk);
-  rev_chunk_fill_kernel<<<dim3(nchunk, d.Hkv, d.B), 32, 2 * nb_bytes, s>>>(idx, chunk, list, d);
+  rev_chunk_count_kernel<<<dim3(nchunk, d.Hkv, d.B), kRevChunk, nb_bytes, s>>>(idx, chunk, d,
+                                                                              nullptr);
+  rev_chunk_scan_kernel<<<d.B * d.Hkv, 1024, nb_bytes, s>>>(chunk, offsets, d, nchunk, nullptr,
+                                                           nullptr, nullptr, 0, 0);
+  rev_chunk_fill_kernel<<<dim3(nchunk, d.Hkv, d.B), 32, 2 * nb_bytes, s>>>(idx, chunk,
+                                                                                  list, d);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_revmap_units(const Dims& d, const int32_t* idx, int* chunk, int* offsets,
+                                int* cursor, int* list, int4* units, int* ucount, int tpu,
+                                int umax, int* err, cudaStream_t s) {
+  const int nchunk = (d.Tq + kRevChunk - 1) / kRevChunk;
+  if (nchunk == 0 || d.Nb == 0) return cudaSuccess;
+  const size_t nb_bytes = (size_t)d.Nb * sizeof(int);
+  rev_chunk_count_kernel<<<dim3(nchunk, d.Hkv, d.B), kRevChunk, nb_bytes, s>>>(idx, chunk, d,
+                                                                              err);
+  rev_chunk_scan_kernel<<<d.B * d.Hkv, 1024, nb_bytes, s>>>(chunk, offsets, d, nchunk, units,
+                                                           ucount, cursor, tpu, umax);
+  rev_atomic_fill_kernel<<<dim3((d.Tq + 255) / 256, d.Hkv, d.B), 256, 0, s>>>(idx, cursor,
+                                                                             list, d);
   return cudaGetLastError();
 }
 
