@@ -453,12 +453,14 @@ decode_block_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 // slots' (max, sum) in parallel, the warp reduces them per branch, then the
 // slots' 64-wide partial outputs are folded in 16 at a time with every load
 // of a batch issued before any is used.
-__global__ void decode_merge_kernel(const float* __restrict__ gates, bf16* __restrict__ out,
-                                    Dims d, DecodeWs ws) {
+__global__ void __launch_bounds__(32)
+decode_merge_kernel(const float* __restrict__ gates, bf16* __restrict__ out, Dims d,
+                    DecodeWs ws) {
+  // one single-warp CTA per (sequence and group, head): small enough to be
+  // resident beside the block kernel's CTAs and wait there (PDL)
   const int bg = blockIdx.x;
-  const int row = threadIdx.x >> 5, lane = threadIdx.x & 31;  // one warp per head
+  const int row = blockIdx.y, lane = threadIdx.x;
   pdl_wait();
-  if (row >= d.G) return;
   const int b = bg / d.Hkv, g = bg % d.Hkv;
   const int h = g * d.G + row;
   const int t = d.T - 1;
@@ -482,61 +484,72 @@ __global__ void decode_merge_kernel(const float* __restrict__ gates, bf16* __res
     const int j = sel[s - nc];
     return j >= 0 && j <= cur;
   };
-  float M0 = -INFINITY, M1 = -INFINITY, M2 = -INFINITY;
-  for (int s0 = 0; s0 < ns; s0 += 32) {
-    const int s = s0 + lane;
-    float m = -INFINITY;
-    int br = 3;
-    if (s < ns) {
-      br = slot_branch(s);
-      if (slot_valid(s)) m = slot_ptr(s)[64];
-    }
-    M0 = fmaxf(M0, warp_max(br == 0 ? m : -INFINITY));
-    M1 = fmaxf(M1, warp_max(br == 1 ? m : -INFINITY));
-    M2 = fmaxf(M2, warp_max(br == 2 ? m : -INFINITY));
+  // Two rounds of loads: every slot's (m, l) and the selected indices at
+  // once (lane L holds slots L + 32 k), then the partial rows 16 slots at a
+  // time.  Slots past ns or not holding a partial get weight 0.
+  constexpr int kMaxSlots = 128;
+  float m[kMaxSlots / 32], l[kMaxSlots / 32];
+  int br[kMaxSlots / 32];
+#pragma unroll
+  for (int k = 0; k < kMaxSlots / 32; ++k) {
+    const int sl = lane + 32 * k;
+    const bool in = sl < ns;
+    const float* pr = slot_ptr(in ? sl : 0);  // inside the workspace
+    br[k] = in ? slot_branch(sl) : 3;
+    m[k] = in ? pr[64] : -INFINITY;
+    l[k] = in ? pr[65] : 0.f;
   }
+#pragma unroll
+  for (int k = 0; k < kMaxSlots / 32; ++k)
+    if (br[k] < 3 && !slot_valid(lane + 32 * k)) m[k] = -INFINITY;
+  float M0 = -INFINITY, M1 = -INFINITY, M2 = -INFINITY;
+#pragma unroll
+  for (int k = 0; k < kMaxSlots / 32; ++k) {
+    M0 = fmaxf(M0, br[k] == 0 ? m[k] : -INFINITY);
+    M1 = fmaxf(M1, br[k] == 1 ? m[k] : -INFINITY);
+    M2 = fmaxf(M2, br[k] == 2 ? m[k] : -INFINITY);
+  }
+  M0 = warp_max(M0);
+  M1 = warp_max(M1);
+  M2 = warp_max(M2);
   float L0 = 0.f, L1 = 0.f, L2 = 0.f;
+  float fw[kMaxSlots / 32];
+#pragma unroll
+  for (int k = 0; k < kMaxSlots / 32; ++k) {
+    const float Mb = br[k] == 0 ? M0 : br[k] == 1 ? M1 : M2;
+    fw[k] = (br[k] < 3 && m[k] != -INFINITY) ? fast_exp2(m[k] - Mb) : 0.f;
+    if (br[k] == 0) L0 += fw[k] * l[k];
+    else if (br[k] == 1) L1 += fw[k] * l[k];
+    else if (br[k] == 2) L2 += fw[k] * l[k];
+  }
   float a00 = 0.f, a01 = 0.f, a10 = 0.f, a11 = 0.f, a20 = 0.f, a21 = 0.f;
-  for (int s0 = 0; s0 < ns; s0 += 32) {
-    const int s = s0 + lane;
-    float f = 0.f;
-    int br = 3;
-    if (s < ns) {
-      br = slot_branch(s);
-      if (slot_valid(s)) {
-        const float* pr = slot_ptr(s);
-        const float m = pr[64], l = pr[65];
-        const float Mb = br == 0 ? M0 : br == 1 ? M1 : M2;
-        f = m == -INFINITY ? 0.f : fast_exp2(m - Mb);
-        if (br == 0) L0 += f * l;
-        else if (br == 1) L1 += f * l;
-        else L2 += f * l;
-      }
-    }
-    const int cnt = min(32, ns - s0);
-    for (int i0 = 0; i0 < cnt; i0 += 16) {
-      float fs[16], x0[16], x1[16];
-      int bs[16];
 #pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        const int i = i0 + k;
-        fs[k] = __shfl_sync(0xffffffffu, f, i & 31);
-        bs[k] = __shfl_sync(0xffffffffu, br, i & 31);
-        const bool use = i < cnt && fs[k] != 0.f;
-        const float* pr = slot_ptr(s0 + i);  // inside the workspace for every i < cnt
-        x0[k] = use ? pr[lane] : 0.f;
-        x1[k] = use ? pr[lane + 32] : 0.f;
+  for (int k = 0; k < kMaxSlots / 32; ++k) {
+    if (32 * k >= ns) break;
+    {
+      constexpr int i0 = 0;  // all 32 slots of this group of loads in flight together
+      float fs[32], x0[32], x1[32];
+      int bs[32];
+#pragma unroll
+      for (int q = 0; q < 32; ++q) {
+        const int i = i0 + q;
+        fs[q] = __shfl_sync(0xffffffffu, fw[k], i);
+        bs[q] = __shfl_sync(0xffffffffu, br[k], i);
+        const bool use = 32 * k + i < ns && fs[q] != 0.f;
+        const float* pr = slot_ptr(use ? 32 * k + i : 0);
+        x0[q] = use ? pr[lane] : 0.f;
+        x1[q] = use ? pr[lane + 32] : 0.f;
       }
 #pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        const float w0 = bs[k] == 0 ? fs[k] : 0.f, w1 = bs[k] == 1 ? fs[k] : 0.f,
-                    w2 = bs[k] == 2 ? fs[k] : 0.f;
-        a00 = fmaf(w0, x0[k], a00);
-        a01 = fmaf(w0, x1[k], a01);
-        a10 = fmaf(w1, x0[k], a10);
-        a11 = fmaf(w1, x1[k], a11);
-        a20 = fmaf(w2, x0[k], a20);
-        a21 = fmaf(w2, x1[k], a21);
+      for (int q = 0; q < 32; ++q) {
+        const float w0 = bs[q] == 0 ? fs[q] : 0.f, w1 = bs[q] == 1 ? fs[q] : 0.f,
+                    w2 = bs[q] == 2 ? fs[q] : 0.f;
+        a00 = fmaf(w0, x0[q], a00);
+        a01 = fmaf(w0, x1[q], a01);
+        a10 = fmaf(w1, x0[q], a10);
+        a11 = fmaf(w1, x1[q], a11);
+        a20 = fmaf(w2, x0[q], a20);
+        a21 = fmaf(w2, x1[q], a21);
       }
     }
   }
@@ -562,8 +575,12 @@ int window_blocks(const Dims& d, int* jlo) {
 // group (the 16 MMA rows), up to 1024 compressed blocks (the top-k warp's
 // registers) and one query.
 bool decode_split_eligible(const Dims& d) {
-  return d.Tq == 1 && d.dtype == 1 && d.l == 64 && d.D == 64 && d.G <= 16 && d.Nc <= 1024 &&
-         tmap_encode_fn() != nullptr;
+  if (!(d.Tq == 1 && d.dtype == 1 && d.l == 64 && d.D == 64 && d.G <= 16 && d.Nc <= 1024 &&
+        tmap_encode_fn() != nullptr))
+    return false;
+  int jlo = 0;
+  const int slots = (d.Nc + 63) / 64 + d.topk + window_blocks(d, &jlo);
+  return slots <= 128;  // the merge holds up to 128 partial slots per row
 }
 
 namespace {
@@ -639,8 +656,8 @@ cudaError_t launch_decode_split(const Dims& d, const void* q, const void* kcache
     if (e != cudaSuccess) return e;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)bgn);
-  cfg.blockDim = dim3(d.G * 32);
+  cfg.gridDim = dim3((unsigned)bgn, (unsigned)d.G);
+  cfg.blockDim = dim3(32);
   cfg.stream = s;
   cfg.attrs = pdl;
   cfg.numAttrs = 1;
