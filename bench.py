@@ -343,6 +343,8 @@ def run_gpu(args, rank: int, world: int, dist_on: bool) -> None:
     # training step (B=8 forward + backward)
     del hq, hk, hv, hg, hout
     train = run_train(dev, flush, stream, max(3, args.steps // 4), peaks)
+    # long context (32768 tokens, block-major selection)
+    long_ctx = run_long(dev, flush, stream, max(3, args.steps // 4), peaks)
     sampler.__exit__(None, None, None)
 
     barrier_sync(dist_on)
@@ -374,6 +376,7 @@ def run_gpu(args, rank: int, world: int, dist_on: bool) -> None:
                      "executed_over_algorithmic": sel_exec_flops / flops["sel"]},
         "decode": dec,
         "train": train,
+        "long_context": long_ctx,
         "e2e": {"value": job_tokens_per_s(tokens_per_step, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": KERNELS_PER_FORWARD * args.steps,
@@ -426,6 +429,45 @@ def run_train(dev, flush, stream, steps, peaks) -> dict:
             "flops_note": "algorithmic: forward + backward counted as 2.5x forward"}
 
 
+def run_long(dev, flush, stream, steps, peaks) -> dict:
+    """Long-context forward: the pruned MQA workload (B=1, 32768 tokens,
+    selection + window).  Its selection runs block-major (Nb = 32 top-k);
+    the query-tiled kernel is timed beside it on the same indices."""
+    w = W.PRUNED_32K
+    inp = W.make_inputs(w, seed=2)
+    q, k, v, g = (inp[n].to(dev) for n in ("q", "k", "v", "gates"))
+    p = nsa.params_for(w)
+    out = torch.empty_like(q)
+    ws = nsa.alloc_workspace(p, dev)
+    saved = {"idx": torch.empty((w.B, w.T, w.Hkv, w.topk), dtype=torch.int32, device=dev)}
+
+    def fwd():
+        nsa.nsa_forward(p, q, k, v, g, out, saved, ws)
+
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.T, w.Hq), dtype=torch.float32, device=dev)
+    sws = torch.empty(nsa.nsa_sel_workspace_size(p), dtype=torch.uint8, device=dev)
+
+    def sel_bm():
+        nsa.nsa_sel_attn_fwd_ws(p, q, k, v, saved["idx"], o, lse, sws)
+
+    def sel_tiled():
+        nsa.nsa_sel_attn_fwd(p, q, k, v, saved["idx"], o, lse)
+
+    for _ in range(2):
+        fwd()
+    fwd_ms = statistics.mean(timed_steps(fwd, steps, flush, stream))
+    bm_ms = statistics.mean(timed_steps(sel_bm, steps, flush, stream))
+    tiled_ms = statistics.mean(timed_steps(sel_tiled, steps, flush, stream))
+    if nsa.nsa_last_device_error() != 0:
+        raise RuntimeError("device-side check failed in the long-context leg")
+    flops = fwd_flops(w)
+    return {"workload": w.name, "fwd_ms": fwd_ms, "tokens_per_s": w.B * w.T / (fwd_ms * 1e-3),
+            "tflops": flops["total"] / (fwd_ms * 1e-3) / 1e12,
+            "sel_block_major_ms": bm_ms, "sel_query_tiled_ms": tiled_ms,
+            "sel_block_major_tflops": flops["sel"] / (bm_ms * 1e-3) / 1e12}
+
+
 def run_decode(dev, flush, stream, steps, peaks) -> dict:
     w = DECODE
     inp = W.make_decode_inputs(w, seed=0)
@@ -476,9 +518,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="nsa", choices=["nsa", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--leg", default="all", choices=["all", "decode", "train"],
-                    help="decode / train: run only that leg on one GPU and print its "
-                         "numbers (for profiling that leg alone); all: the benchmark")
+    ap.add_argument("--leg", default="all", choices=["all", "decode", "train", "long"],
+                    help="decode / train / long: run only that leg on one GPU and print "
+                         "its numbers (for profiling that leg alone); all: the benchmark")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -494,6 +536,8 @@ def main():
         flush, stream, peaks = Flusher(dev), torch.cuda.current_stream(), load_peaks()
         if args.leg == "decode":
             print(json.dumps({"decode": run_decode(dev, flush, stream, args.steps, peaks)}))
+        elif args.leg == "long":
+            print(json.dumps({"long_context": run_long(dev, flush, stream, args.steps, peaks)}))
         else:
             print(json.dumps({"train": run_train(dev, flush, stream, args.steps, peaks)}))
         return
