@@ -192,7 +192,7 @@ __device__ __forceinline__ bool rev_valid(const int32_t* ir, int s, int cur) {
 
 __global__ void __launch_bounds__(kRevChunk)
 rev_chunk_count_kernel(const int32_t* __restrict__ idx, int* __restrict__ chunk, Dims d,
-                       int* err) {
+                       int* err, int* __restrict__ totals) {
   extern __shared__ int hist[];  // [Nb]
   const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int nchunk = gridDim.x;
@@ -214,6 +214,12 @@ rev_chunk_count_kernel(const int32_t* __restrict__ idx, int* __restrict__ chunk,
     }
   }
   __syncthreads();
+  if (totals) {  // per-(sequence, group) totals only: the order inside a list is free
+    int* tot = totals + ((size_t)b * d.Hkv + g) * d.Nb;
+    for (int j = threadIdx.x; j < d.Nb; j += blockDim.x)
+      if (hist[j]) atomicAdd(tot + j, hist[j]);
+    return;
+  }
   int* out = chunk + (((size_t)b * d.Hkv + g) * nchunk + c) * d.Nb;
   for (int j = threadIdx.x; j < d.Nb; j += blockDim.x) out[j] = hist[j];
 }
@@ -360,34 +366,42 @@ rev_chunk_fill_kernel(const int32_t* __restrict__ idx, const int* __restrict__ c
 
 // The forward's fill, entries query << 6 | slot (topk <= 64).  The order
 // inside a block's list is free (each (query, slot) pair is computed on its
-// own), so positions come from one atomic cursor per (sequence, group,
-// block), started at the block's scanned offset, the lanes of a warp that
-// chose the same block sharing one atomic.  One thread per query.
-__global__ void __launch_bounds__(256)
+// own), so a CTA of kRevChunk queries counts its pairs per block in shared
+// memory, reserves each block's range with one global atomic on the block's
+// cursor (started at its scanned offset), and places its pairs with shared
+// atomics.  One thread per query.
+__global__ void __launch_bounds__(kRevChunk)
 rev_atomic_fill_kernel(const int32_t* __restrict__ idx, int* __restrict__ cursor,
                        int* __restrict__ list, Dims d) {
-  const int tq = blockIdx.x * blockDim.x + threadIdx.x;
+  extern __shared__ int sh[];  // count[Nb], base[Nb]
+  int* cnt = sh;
+  int* base = sh + d.Nb;
+  const int tq = blockIdx.x * kRevChunk + threadIdx.x;
   const int g = blockIdx.y, b = blockIdx.z;
-  const int lane = threadIdx.x & 31;
   const bool q_ok = tq < d.Tq;
   const size_t bg = (size_t)b * d.Hkv + g;
   const int32_t* ir = idx + (((size_t)b * d.Tq + (q_ok ? tq : 0)) * d.Hkv + g) * d.topk;
   const int cur = (d.q_off + tq) / d.l;
+  for (int j = threadIdx.x; j < d.Nb; j += blockDim.x) cnt[j] = 0;
+  __syncthreads();
+  if (q_ok)
+    for (int s = 0; s < d.topk; ++s)
+      if (rev_valid(ir, s, cur)) atomicAdd(&cnt[ir[s]], 1);
+  __syncthreads();
   int* cb = cursor + bg * d.Nb;
-  int* lst = list + bg * (size_t)d.Tq * d.topk;
-  for (int s = 0; s < d.topk; ++s) {
-    const bool v = q_ok && rev_valid(ir, s, cur);
-    const unsigned act = __ballot_sync(0xffffffffu, v);
-    if (v) {
-      const int j = ir[s];
-      const unsigned peers = __match_any_sync(act, j);
-      const int leader = __ffs(peers) - 1;
-      int base = 0;
-      if (lane == leader) base = atomicAdd(cb + j, __popc(peers));
-      base = __shfl_sync(peers, base, leader);
-      lst[base + __popc(peers & ((1u << lane) - 1u))] = (tq << 6) | s;
-    }
+  for (int j = threadIdx.x; j < d.Nb; j += blockDim.x) {
+    const int c = cnt[j];
+    base[j] = c ? atomicAdd(cb + j, c) : 0;
+    cnt[j] = 0;
   }
+  __syncthreads();
+  int* lst = list + bg * (size_t)d.Tq * d.topk;
+  if (q_ok)
+    for (int s = 0; s < d.topk; ++s)
+      if (rev_valid(ir, s, cur)) {
+        const int j = ir[s];
+        lst[base[j] + atomicAdd(&cnt[j], 1)] = (tq << 6) | s;
+      }
 }
 
 // ---- pass 2: dK, dV, key-stationary ----------------------------------------------
@@ -575,7 +589,7 @@ cudaError_t launch_revmap(const Dims& d, const int32_t* idx, int* chunk, int* of
   if (nchunk == 0 || d.Nb == 0) return cudaSuccess;
   const size_t nb_bytes = (size_t)d.Nb * sizeof(int);
   rev_chunk_count_kernel<<<dim3(nchunk, d.Hkv, d.B), kRevChunk, nb_bytes, s>>>(idx, chunk, d,
-                                                                              nullptr);
+                                                                              nullptr, nullptr);
   rev_chunk_scan_kernel<<<d.B * d.Hkv, 1024, nb_bytes, s>>>(chunk, offsets, d, nchunk, nullptr,
                                                            nullptr, nullptr, 0, 0);
   rev_chunk_fill_kernel<<<dim3(nchunk, d.Hkv, d.B), 32, 2 * nb_bytes, s>>>(idx, chunk,
@@ -589,12 +603,15 @@ cudaError_t launch_revmap_units(const Dims& d, const int32_t* idx, int* chunk, i
   const int nchunk = (d.Tq + kRevChunk - 1) / kRevChunk;
   if (nchunk == 0 || d.Nb == 0) return cudaSuccess;
   const size_t nb_bytes = (size_t)d.Nb * sizeof(int);
+  // per-(sequence, group, block) totals (chunk holds them: B * Hkv * Nb ints)
+  cudaError_t e = cudaMemsetAsync(chunk, 0, (size_t)d.B * d.Hkv * nb_bytes, s);
+  if (e != cudaSuccess) return e;
   rev_chunk_count_kernel<<<dim3(nchunk, d.Hkv, d.B), kRevChunk, nb_bytes, s>>>(idx, chunk, d,
-                                                                              err);
-  rev_chunk_scan_kernel<<<d.B * d.Hkv, 1024, nb_bytes, s>>>(chunk, offsets, d, nchunk, units,
+                                                                              err, chunk);
+  rev_chunk_scan_kernel<<<d.B * d.Hkv, 1024, nb_bytes, s>>>(chunk, offsets, d, 1, units,
                                                            ucount, cursor, tpu, umax);
-  rev_atomic_fill_kernel<<<dim3((d.Tq + 255) / 256, d.Hkv, d.B), 256, 0, s>>>(idx, cursor,
-                                                                             list, d);
+  rev_atomic_fill_kernel<<<dim3(nchunk, d.Hkv, d.B), kRevChunk, 2 * nb_bytes, s>>>(idx, cursor,
+                                                                                   list, d);
   return cudaGetLastError();
 }
 

@@ -73,7 +73,9 @@ constexpr uint32_t OFF_STG = OFF_Q + kQBufs * kQBytes;            // 4 KB per ep
 constexpr uint32_t OFF_ERING = OFF_STG + kRows * 128;             // kERing x 128 list entries
 constexpr uint32_t OFF_MRING = OFF_ERING + kERing * kRows * 4;    // kMRing x 128 x (m, l, slot)
 constexpr uint32_t OFF_UNITS = OFF_MRING + kMRing * kRows * 16;   // kMaxUnits int4
-constexpr uint32_t OFF_BAR = OFF_UNITS + kMaxUnits * 16;
+constexpr int kMaxTiles = kMaxUnits * kSeg;
+constexpr uint32_t OFF_TLIST = OFF_UNITS + kMaxUnits * 16;       // kMaxTiles uint16: unit << 2 | tile
+constexpr uint32_t OFF_BAR = OFF_TLIST + kMaxTiles * 2;
 
 struct Bars {
   uint64_t kvfull[kKvStages];
@@ -90,7 +92,7 @@ struct Bars {
   uint64_t fin;                // every P*V of the CTA is done
   uint64_t sfin;               // every S MMA of the CTA is done
 };
-constexpr uint32_t OFF_MISC = OFF_BAR + ((sizeof(Bars) + 15) / 16) * 16;  // tmem slot, abort
+constexpr uint32_t OFF_MISC = OFF_BAR + ((sizeof(Bars) + 15) / 16) * 16;  // tmem, abort, ntiles
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 16;
 
 __host__ __device__ inline int tile_tokens(int G) { return kRows / G; }
@@ -101,27 +103,6 @@ __host__ __device__ inline int tile_tokens(int G) { return kRows / G; }
 __device__ __forceinline__ int u_b(int4 u) { return u.x >> 20; }
 __device__ __forceinline__ int u_g(int4 u) { return (u.x >> 13) & 127; }
 __device__ __forceinline__ int u_j(int4 u) { return u.x & 8191; }
-
-// Position (unit k, first list entry p) of the CTA's tiles in order; k ==
-// nk once past the last one.
-struct TilePos {
-  int k, p;
-};
-__device__ __forceinline__ void tp_skip(TilePos& t, const int4* us, int nk) {
-  while (t.k < nk && t.p >= us[t.k].z) {
-    ++t.k;
-    if (t.k < nk) t.p = us[t.k].y;
-  }
-}
-__device__ __forceinline__ void tp_first(TilePos& t, const int4* us, int nk) {
-  t.k = 0;
-  t.p = nk > 0 ? us[0].y : 0;
-  tp_skip(t, us, nk);
-}
-__device__ __forceinline__ void tp_next(TilePos& t, int TQ, const int4* us, int nk) {
-  t.p += TQ;
-  tp_skip(t, us, nk);
-}
 
 __global__ void __launch_bounds__(kThreads, 1)
 sel_bm_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -187,6 +168,35 @@ sel_bm_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     prefetch_tmap(&tm_v);
   }
   __syncthreads();
+  // The CTA's tiles in order (tile i = entry i: unit k, tile t of it), so
+  // the roles index tiles instead of walking the unit list: thread k < nk
+  // counts unit k's tiles, a block scan places them.
+  uint16_t* tl = (uint16_t*)(smem + OFF_TLIST);
+  int* ntiles_s = (int*)(smem + OFF_MISC + 8);
+  {
+    int* wsum = (int*)(smem + OFF_ERING);  // scratch before the ring is used
+    const int4 u = tid < nk ? us[tid] : make_int4(0, 0, 0, 0);
+    const int cnt = u.z > u.y ? (u.z - u.y + TQ - 1) / TQ : 0;
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    int base = 0;
+    for (int w2 = 0; w2 < warp; ++w2) base += wsum[w2];
+    if (tid == kThreads - 1) *ntiles_s = base + incl;
+    for (int t2 = 0; t2 < cnt; ++t2) tl[base + incl - cnt + t2] = (uint16_t)((tid << 2) | t2);
+    __syncthreads();
+  }
+  const int ntiles = *ntiles_s;
+  auto tile_pos = [&](int it, int4& u, int& p) {  // unit and first list position of tile it
+    const int e = tl[it];
+    u = us[e >> 2];
+    p = u.y + (e & 3) * TQ;
+  };
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
@@ -198,17 +208,19 @@ sel_bm_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     constexpr int kEAhead = 4;
     const int h = warp - kWarpGather;
     const uint32_t ering_s = smem_u32(ering);
-    auto fetch = [&](const TilePos& tt, int it) {  // one cp.async group
+    auto fetch = [&](int it) {  // one cp.async group
       const uint32_t dst = ering_s + (uint32_t)(((it & (kERing - 1)) * kRows + 64 * h + lane) * 4);
-      if (tt.k >= nk) {
+      if (it >= ntiles) {
         st_shared_u32(dst, (uint32_t)-2);
         st_shared_u32(dst + 128, (uint32_t)-2);
       } else {
-        const int4 u = us[tt.k];
+        int4 u;
+        int p0;
+        tile_pos(it, u, p0);
         const int* lst = list + (size_t)(u_b(u) * d.Hkv + u_g(u)) * list_stride;
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
-          const int pos = tt.p + ((64 * h + lane + 32 * k) >> lgG);
+          const int pos = p0 + ((64 * h + lane + 32 * k) >> lgG);
           if (pos < u.z)
             cp_async4(dst + 128 * k, lst + pos);
           else
@@ -217,25 +229,17 @@ sel_bm_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
       }
       cp_async_commit();
     };
-    TilePos t, ta;  // tiles i, i + kEAhead
-    tp_first(t, us, nk);
-    ta = t;
-    for (int j = 0; j < kEAhead; ++j) {
-      fetch(ta, j);
-      tp_next(ta, TQ, us, nk);
-    }
-    for (int i = 0; t.k < nk; ++i) {
+    for (int j = 0; j < kEAhead; ++j) fetch(j);
+    for (int i = 0; i < ntiles; ++i) {
       const int ia = i + kEAhead;
       // ring slot ia % kERing held tile ia - kERing's entries
       if (ia >= kERing && !wait_bar_warp(&bars->efree[ia & (kERing - 1)],
                                          ((ia / kERing) - 1) & 1, abort_flag, err))
         break;
-      fetch(ta, ia);
-      tp_next(ta, TQ, us, nk);
+      fetch(ia);
       cp_async_wait<kEAhead>();  // tile i's group has landed
       __syncwarp();
       mbar_arrive(&bars->efull[i & (kERing - 1)]);
-      tp_next(t, TQ, us, nk);
     }
     cp_async_wait<0>();  // no copy outlives the CTA
   } else if (warp == kWarpS) {
@@ -347,11 +351,13 @@ sel_bm_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     const uint32_t lane_tmem = tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(x * 256);
     const float sl2 = d.scale * kLog2e;
     const int hh = r & (d.G - 1);
-    auto copy_q = [&](const TilePos& tt, int it) -> bool {  // one cp.async group
-      if (tt.k < nk) {
+    auto copy_q = [&](int it) -> bool {  // one cp.async group
+      if (it < ntiles) {
         if (!wait_bar_warp(&bars->efull[it & (kERing - 1)], (it / kERing) & 1, abort_flag, err))
           return false;
-        const int4 u = us[tt.k];
+        int4 u;
+        int p0;
+        tile_pos(it, u, p0);
         const int* er = ering + (it & (kERing - 1)) * kRows + (warp & 3) * 32;
         int ev[8];
 #pragma unroll
@@ -376,38 +382,22 @@ sel_bm_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
       fence_proxy_async_smem();  // the MMA reads the tile through the async proxy
       mbar_arrive(&bars->qfull[it % kQBufs]);
     };
-    TilePos t, t2, t8;  // tiles i, i+2, i+kQBufs
-    tp_first(t, us, nk);
-    t2 = t;
-    tp_next(t2, TQ, us, nk);
-    tp_next(t2, TQ, us, nk);
     {  // this warpgroup's first kQBufs / 2 tiles: x, x + 2, ...
-      TilePos f = t;
-      if (x == 1) tp_next(f, TQ, us, nk);
-      const TilePos f0 = f;
       bool ok0 = true;
-      for (int j = 0; ok0 && j < kQBufs / 2; ++j) {
-        ok0 = copy_q(f, x + 2 * j);
-        tp_next(f, TQ, us, nk);
-        tp_next(f, TQ, us, nk);
-      }
-      if (ok0 && f0.k < nk) {  // tile x: all but the kQBufs/2 - 1 newer groups
+      for (int j = 0; ok0 && j < kQBufs / 2; ++j) ok0 = copy_q(x + 2 * j);
+      if (ok0 && x < ntiles) {  // tile x: all but the kQBufs/2 - 1 newer groups
         cp_async_wait<kQBufs / 2 - 1>();
         fence_proxy_async_smem();
         mbar_arrive(&bars->qfull[x % kQBufs]);
       }
     }
-    t8 = t;
-    for (int j = 0; j < kQBufs; ++j) tp_next(t8, TQ, us, nk);
-    for (int i = 0; t.k < nk;
-         ++i, tp_next(t, TQ, us, nk), tp_next(t2, TQ, us, nk), tp_next(t8, TQ, us, nk)) {
-      if ((i & 1) != x) continue;
+    for (int i = x; i < ntiles; i += 2) {
       const int bf = (i >> 1) & 1;
       if (!wait_bar_warp(&bars->efull[i & (kERing - 1)], (i / kERing) & 1, abort_flag, err)) break;
       const int e = ering[(i & (kERing - 1)) * kRows + r];
       if (!wait_bar_warp(&bars->s[x][bf], (i >> 2) & 1, abort_flag, err)) break;
-      if (t2.k < nk) publish_q(i + 2);
-      const int4 u = us[t.k];
+      if (i + 2 < ntiles) publish_q(i + 2);
+      const int4 u = us[tl[i] >> 2];
       const bool valid = e >= 0;
       const int tq = max(e, 0) >> 6;
       const int tpos = d.q_off + tq;
@@ -461,7 +451,7 @@ sel_bm_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
       tc_fence_before();
       mbar_arrive(&bars->p[x][bf]);
       // tile i+kQBufs's Q into the buffer tile i's S MMA has finished reading
-      if (!copy_q(t8, i + kQBufs)) break;
+      if (!copy_q(i + kQBufs)) break;
       // the row's statistics and partial slot for the epilogue
       uint32_t slot = UINT_MAX;
       if (valid)
@@ -479,9 +469,7 @@ sel_bm_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     const uint32_t lane_tmem = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const uint32_t stg = smem_u32(smem + OFF_STG) + (uint32_t)(warp - kWarpEpi) * 4096u;
     const uint32_t mine = stg + (uint32_t)lane * 128u;
-    TilePos t;
-    tp_first(t, us, nk);
-    for (int i = 0; t.k < nk; ++i, tp_next(t, TQ, us, nk)) {
+    for (int i = 0; i < ntiles; ++i) {
       const int x = i & 1, bf = (i >> 1) & 1;
       if (!wait_bar_warp(&bars->mfull[i & (kMRing - 1)], (i / kMRing) & 1, abort_flag, err)) break;
       const float4 st = mring[(i & (kMRing - 1)) * kRows + r];

@@ -96,7 +96,7 @@ enum { W_KC, W_VC, W_OCMP, W_LSECMP, W_SCORE, W_IDX, W_OSEL, W_LSESEL, W_OSWA, W
 // kernel's does not (measured on B200: equal at Nb = 8 topk, 1.6x faster at
 // Nb = 32 topk).
 bool use_sel_bm(const Dims& d) {
-  return (d.branch_mask & NSA_BRANCH_SEL) && d.Tq >= 64 && d.Nb >= 16 * d.topk &&
+  return (d.branch_mask & NSA_BRANCH_SEL) && d.Tq >= 64 && d.Nb >= 8 * d.topk &&
          nsa::sel_bm_eligible(d);
 }
 
