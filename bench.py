@@ -191,6 +191,39 @@ def timed_steps(fn, steps: int, flush, stream) -> list[float]:
     return [a.elapsed_time(b) for a, b in times]
 
 
+def kernel_event_times(fn, steps: int, flush, stream) -> list[float]:
+    """Device time (ms) of the block-major selection kernel inside fn: the
+    library records a CUDA event pair around it on the launching stream."""
+    times = []
+    for _ in range(steps):
+        flush()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)  # creates the events; the library records them again
+        b.record(stream)
+        nsa.nsa_set_kernel_events(a, b)
+        fn()
+        times.append((a, b))
+    nsa.nsa_set_kernel_events(None, None)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in times]
+
+
+def sel_bm_algorithmic_bytes(w, idx) -> int:
+    """HBM bytes the block-major selection kernel must move: one fp16 partial
+    row (128 B) and one float lse per (query row, used slot) written, plus Q,
+    K and V read once and the reverse-map list entries (4 B per used slot)."""
+    import numpy as np
+    ii = idx.cpu().numpy()  # [B, T, Hkv, topk]
+    t = np.arange(w.T)[None, :, None, None]
+    used = (ii >= 0) & (ii <= t // w.sel_block)
+    slots = int(used.sum())  # (token, group, slot) triples
+    G = w.Hq // w.Hkv
+    es = 2
+    return (slots * G * (128 + 4) + slots * 4
+            + w.B * w.T * w.Hq * w.D * es + 2 * w.B * w.T * w.Hkv * w.D * es)
+
+
 def barrier_sync(dist_on):
     torch.cuda.synchronize()
     if dist_on:
@@ -308,7 +341,12 @@ def run_gpu(args, rank: int, world: int, dist_on: bool) -> None:
     tokens_per_step = w.B * w.T
     value = job_tokens_per_s(tokens_per_step, world, ms)
 
-    # dominant kernel alone (selection branch), same inputs, same flushing
+    # the forward's dominant kernel (block-major selection, sel_bm_kernel):
+    # CUDA events the library records around that kernel on this stream,
+    # inside the same forward call, flushed as above
+    bm_ms = statistics.mean(kernel_event_times(step, args.steps, flush, stream))
+    bm_bytes = sel_bm_algorithmic_bytes(w, saved["idx"])
+    # context: the query-tiled selection kernel on the same indices
     o_sel = torch.empty_like(q)
     for _ in range(2):
         nsa.nsa_sel_attn_fwd(p, q, k, v, saved["idx"], o_sel, None)
@@ -338,10 +376,16 @@ def run_gpu(args, rank: int, world: int, dist_on: bool) -> None:
     h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hg))
     d2h = hout.numel() * hout.element_size()
 
+    del hq, hk, hv, hg, hout
+    if args.leg == "forward":  # the forward alone (for profiling it)
+        sampler.__exit__(None, None, None)
+        print(json.dumps({"forward": {"ms_per_step": ms, "tokens_per_s": value,
+                                      "sel_bm_kernel_ms": bm_ms,
+                                      "sel_bm_kernel_gbs": bm_bytes / (bm_ms * 1e-3) / 1e9}}))
+        return
     # decode (B=64 sequences, 32768-token caches): HBM GB/s
     dec = run_decode(dev, flush, stream, args.steps, peaks)
     # training step (B=8 forward + backward)
-    del hq, hk, hv, hg, hout
     train = run_train(dev, flush, stream, max(3, args.steps // 4), peaks)
     # long context (32768 tokens, block-major selection)
     long_ctx = run_long(dev, flush, stream, max(3, args.steps // 4), peaks)
@@ -363,17 +407,27 @@ def run_gpu(args, rank: int, world: int, dist_on: bool) -> None:
         "tflops": flops["total"] * world / (ms * 1e-3) / 1e12,
         "frac_bf16_peak": flops["total"] / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
         "flops_per_step": flops,
-        "roofline": {"bound": "tensor", "kernel": "selection attention (nsa_sel_attn_fwd)",
-                     "achieved": sel_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": sel_tflops / peaks["bf16_tflops"],
-                     "traffic": profiled_traffic("sparse_attention_nsa_b200/csrc/k_attn_tc.cu",
-                                                 "profiles/attn_tc_sel_340m.md"),
-                     "ms_per_launch": sel_ms, "peak_source": peaks["source"] + " burst bf16",
-                     # context, not the roofline figure: on structure-free selections the
-                     # union of a tile's blocks is near dense, so the tensor pipe runs
-                     # more MMA work than the algorithmic count
-                     "executed_tflops": sel_exec_flops / (sel_ms * 1e-3) / 1e12,
-                     "executed_over_algorithmic": sel_exec_flops / flops["sel"]},
+        # dominant kernel of the timed forward: the block-major selection
+        # kernel; its design minimum is the HBM time of the per-(row, slot)
+        # partials it must write plus its compulsory reads (46 us here) against
+        # 19 us of tensor time, so it is rated against HBM bandwidth
+        "roofline": {"bound": "hbm", "kernel": "block-major selection (sel_bm_kernel)",
+                     "achieved": bm_bytes / (bm_ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": bm_bytes / (bm_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                     "traffic": profiled_traffic("sparse_attention_nsa_b200/csrc/k_sel_bm.cu",
+                                                 "profiles/sel_bm_340m.md"),
+                     "algorithmic_bytes": bm_bytes, "ms_per_launch": bm_ms,
+                     "peak_source": peaks["source"] + " HBM copy",
+                     "tensor_tflops": flops["sel"] / (bm_ms * 1e-3) / 1e12,
+                     "tensor_frac": flops["sel"] / (bm_ms * 1e-3) / 1e12 / peaks["bf16_tflops"]},
+        # context: the query-tiled selection kernel (the forward's path for
+        # Nb < 8 top-k) on the same indices; on structure-free selections the
+        # union of a tile's blocks is near dense, so it issues more MMA work
+        # than the algorithmic count
+        "selection_query_tiled": {"ms_per_launch": sel_ms, "tflops": sel_tflops,
+                                  "frac_bf16_peak": sel_tflops / peaks["bf16_tflops"],
+                                  "executed_tflops": sel_exec_flops / (sel_ms * 1e-3) / 1e12,
+                                  "executed_over_algorithmic": sel_exec_flops / flops["sel"]},
         "decode": dec,
         "train": train,
         "long_context": long_ctx,
@@ -518,9 +572,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="nsa", choices=["nsa", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--leg", default="all", choices=["all", "decode", "train", "long"],
-                    help="decode / train / long: run only that leg on one GPU and print "
-                         "its numbers (for profiling that leg alone); all: the benchmark")
+    ap.add_argument("--leg", default="all",
+                    choices=["all", "forward", "decode", "train", "long"],
+                    help="forward / decode / train / long: run only that leg on one GPU "
+                         "and print its numbers (for profiling that leg alone); all: the "
+                         "benchmark")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -529,7 +585,7 @@ def main():
     if args.impl == "reference":
         run_reference(args, rank)
         return
-    if args.leg != "all":
+    if args.leg not in ("all", "forward"):
         dev = torch.device("cuda", 0)
         torch.cuda.set_device(dev)
         nsa.load()

@@ -185,6 +185,14 @@ nsa_status nsa_sel_attn_fwd(const nsa_params* p, const void* q, const void* k,
  * Returns NSA_ERR_UNSUPPORTED for shapes the block-major kernels do not
  * cover (fp32, block size != 64, D != 64, 128 % G != 0). */
 nsa_status nsa_sel_workspace_size(const nsa_params* p, size_t* bytes);
+
+/* Profiling aid: record the CUDA events `start` and `stop` (cudaEvent_t,
+ * owned by the caller) on the launching stream immediately before and after
+ * the block-major selection kernel of every later call that runs it, so a
+ * caller can time that kernel alone with cudaEventElapsedTime.  Both NULL
+ * turns it off (the default); one NULL is NSA_ERR_INVALID_ARG.
+ * Process-wide; not for concurrent use from several threads. */
+nsa_status nsa_set_kernel_events(void* start, void* stop);
 nsa_status nsa_sel_attn_fwd_ws(const nsa_params* p, const void* q, const void* k,
                                const void* v, const int32_t* idx, void* o_sel,
                                float* lse_sel, void* workspace, size_t workspace_bytes,

@@ -14,7 +14,7 @@ from .abi import (EXPORTS, backward, nsa_backward, nsa_backward_workspace_size,
                   nsa_compress, nsa_decode, nsa_decode_noalloc,
                   nsa_decode_noalloc_max_scratch, nsa_forward, nsa_gate_combine,
                   nsa_last_device_error, nsa_sel_attn_fwd, nsa_sel_attn_fwd_ws,
-                  nsa_sel_workspace_size, nsa_select_topk,
+                  nsa_sel_workspace_size, nsa_select_topk, nsa_set_kernel_events,
                   nsa_status_string, nsa_swa_fwd, nsa_workspace_size, params_for)
 
 __all__ = [n for n in dir() if not n.startswith("_")]

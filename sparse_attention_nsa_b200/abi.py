@@ -32,7 +32,7 @@ EXPORTS = ("nsa_status_string", "nsa_check_params", "nsa_workspace_size",
            "nsa_forward", "nsa_decode", "nsa_backward_workspace_size",
            "nsa_gate_combine_bwd", "nsa_sel_attn_bwd", "nsa_swa_bwd", "nsa_cmp_bwd",
            "nsa_backward", "nsa_decode_noalloc", "nsa_decode_noalloc_max_scratch",
-           "nsa_sel_workspace_size", "nsa_sel_attn_fwd_ws")
+           "nsa_sel_workspace_size", "nsa_sel_attn_fwd_ws", "nsa_set_kernel_events")
 
 
 class NsaError(RuntimeError):
@@ -107,6 +107,7 @@ def load():
             "nsa_decode_noalloc_max_scratch": ([], C.c_size_t),
             "nsa_sel_workspace_size": ([P, C.POINTER(C.c_size_t)], C.c_int),
             "nsa_sel_attn_fwd_ws": ([P, vp, vp, vp, vp, vp, vp, vp, C.c_size_t, vp], C.c_int),
+            "nsa_set_kernel_events": ([vp, vp], C.c_int),
         }
         for name, (args, res) in sig.items():
             f = getattr(lib, name)
@@ -224,6 +225,13 @@ def nsa_sel_attn_fwd(p: Params, q, k, v, idx, o_sel, lse_sel, stream=None):
         _ptr(v, s["k"], dt, "v"), _ptr(idx, s["idx"], torch.int32, "idx"),
         _ptr(o_sel, s["o"], dt, "o_sel"), _ptr(lse_sel, s["lse"], torch.float32, "lse_sel", True),
         _stream(stream)), "nsa_sel_attn_fwd")
+
+
+def nsa_set_kernel_events(start=None, stop=None):
+    """Record torch.cuda.Event pair (start, stop) around the block-major
+    selection kernel of later calls; None, None turns it off."""
+    ptr = lambda e: None if e is None else C.c_void_p(e.cuda_event)
+    _check(load().nsa_set_kernel_events(ptr(start), ptr(stop)), "nsa_set_kernel_events")
 
 
 def nsa_sel_workspace_size(p: Params) -> int:

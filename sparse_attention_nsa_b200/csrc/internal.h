@@ -63,6 +63,9 @@ struct EpilogueFuse {
 // merge.  ws: sel_bm_ws_bytes(d) bytes, 256-byte aligned.  o_sel and
 // lse_sel may be NULL (not stored).
 bool sel_bm_eligible(const Dims& d);
+// CUDA events recorded on the launching stream right before and after the
+// block-major selection kernel of every later call (profiling; null: off)
+void set_sel_bm_events(cudaEvent_t start, cudaEvent_t stop);
 size_t sel_bm_ws_bytes(const Dims& d);
 cudaError_t launch_sel_bm(const Dims& d, const void* q, const void* k, const void* v,
                           const int32_t* idx, void* o_sel, float* lse_sel, int* err,

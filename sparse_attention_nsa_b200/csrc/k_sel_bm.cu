@@ -38,6 +38,7 @@
 // the S MMAs (and the K/V TMA) and the P*V MMAs.
 // TMEM (512 columns): softmax warpgroup x owns [256 x, 256 x + 256): two
 // S/P buffers of 64 columns, then two O buffers of 64.
+#include <atomic>
 #include <climits>
 
 #include "common.cuh"
@@ -683,6 +684,15 @@ int sm_count() {
 
 }  // namespace
 
+namespace {
+std::atomic<cudaEvent_t> g_ev_start{nullptr}, g_ev_stop{nullptr};
+}  // namespace
+
+void set_sel_bm_events(cudaEvent_t start, cudaEvent_t stop) {
+  g_ev_start.store(start);
+  g_ev_stop.store(stop);
+}
+
 bool sel_bm_eligible(const Dims& d) {
   return d.dtype == 1 && d.l == kKeys && d.D == 64 && d.G >= 1 && kRows % d.G == 0 &&
          d.Tq >= 1 && d.Nb >= 1 && d.Nb <= 8192 && d.B < 2048 && d.Hkv <= 128 &&
@@ -717,10 +727,13 @@ cudaError_t launch_sel_bm(const Dims& d, const void* q, const void* k, const voi
   if (e != cudaSuccess) return e;
   const long nU = (long)d.B * d.Hkv * umax;
   const long grid = std::max(std::min(nU, (long)sm_count()), (nU + kMaxUnits - 1) / kMaxUnits);
+  const cudaEvent_t ev0 = g_ev_start.load(), ev1 = g_ev_stop.load();
+  if (ev0 && (e = cudaEventRecord(ev0, s)) != cudaSuccess) return e;
   sel_bm_kernel<<<(unsigned)grid, kThreads, smem, s>>>(mk, mv, (const bf16*)q, list, units, ucount,
                                                        umax, part_o, part_lse, d, err);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  if (ev1 && (e = cudaEventRecord(ev1, s)) != cudaSuccess) return e;
   const size_t nrows = (size_t)d.B * d.Tq * d.Hq;
   const unsigned mgrid = (unsigned)((nrows + 31) / 32);
   if (fz)

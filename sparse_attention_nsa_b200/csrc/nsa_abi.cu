@@ -247,6 +247,12 @@ nsa_status nsa_sel_attn_fwd(const nsa_params* p, const void* q, const void* k,
   return NSA_OK;
 }
 
+nsa_status nsa_set_kernel_events(void* start, void* stop) {
+  if ((start == nullptr) != (stop == nullptr)) return NSA_ERR_INVALID_ARG;
+  nsa::set_sel_bm_events((cudaEvent_t)start, (cudaEvent_t)stop);
+  return NSA_OK;
+}
+
 nsa_status nsa_sel_workspace_size(const nsa_params* p, size_t* bytes) {
   Dims d;
   nsa_status st = fill_dims(p, &d);

@@ -88,3 +88,11 @@ def test_forward_without_workspace_is_rejected():
     p = nsa.make_params(1, 256, 4, 1, cmp_block=32, topk=4, window=64, dtype=nsa.NSA_F32)
     ptr = C.c_void_p(4096)
     assert lib.nsa_forward(C.byref(p), ptr, ptr, ptr, ptr, ptr, None, None, 0, None) == 6
+
+
+def test_kernel_event_hook_arguments():
+    """The profiling hook takes both events or neither; it touches no device."""
+    lib = nsa.load()
+    assert lib.nsa_set_kernel_events(C.c_void_p(64), None) == 1  # NSA_ERR_INVALID_ARG
+    assert lib.nsa_set_kernel_events(None, C.c_void_p(64)) == 1
+    assert lib.nsa_set_kernel_events(None, None) == 0

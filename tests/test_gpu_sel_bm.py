@@ -194,3 +194,25 @@ def test_sel_bm_partial_range_is_reported(cuda_lib):
     o, _ = run_ws(w, inp["q"], inp["k"], v, idx)
     assert nsa.nsa_last_device_error() == 0
     assert torch.all(o.float() == torch.tensor(6.0e4).bfloat16().float())
+
+
+def test_kernel_event_hook_times_the_kernel(cuda_lib):
+    """Events handed to nsa_set_kernel_events bracket the block-major kernel
+    of the next call on its stream; the hook is off again afterwards."""
+    w = small("events_g4_t900", T=900, topk=4)
+    inp = W.make_inputs(w, seed=30)
+    r = orc.forward(ocfg(w), inp["q"], inp["k"], inp["v"], inp["gates"])
+    q, k, v = (inp[n].to(DEV) for n in ("q", "k", "v"))
+    idx = torch.from_numpy(r["idx"]).to(DEV)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    b.record()
+    nsa.nsa_set_kernel_events(a, b)
+    try:
+        o, _ = run_ws(w, q, k, v, idx)
+    finally:
+        nsa.nsa_set_kernel_events(None, None)
+    torch.cuda.synchronize()
+    assert 0.0 < a.elapsed_time(b) < 1000.0
+    assert_close(to_np(o), r["o_sel"], TOL[w.dtype], "o_sel")
