@@ -175,7 +175,7 @@ nsa_status nsa_sel_attn_fwd(const nsa_params* p, const void* q, const void* k,
  * each (query, head, block) pair gets its own softmax over the block's keys,
  * and each row's partials are merged exactly with their log-sum-exps (the
  * split-softmax identity); results match nsa_sel_attn_fwd up to rounding.
- * nsa_forward takes this path itself when Tq >= 64 and Nb >= 16 topk (the
+ * nsa_forward takes this path itself when Tq >= 64 and Nb >= 8 topk (the
  * query-tiled kernel's union of blocks grows with Nb / topk).  Passage: as for
  * nsa_sel_attn_fwd, plus the kernel paragraph (each block is loaded once for
  * all the queries that selected it).  o_sel may be NULL (not

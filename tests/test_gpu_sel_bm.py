@@ -169,7 +169,7 @@ def test_sel_bm_workspace_checks(cuda_lib):
                                      cmp_gate_zero=True, qk_norm=False)],
                          ids=lambda w: w.name)
 def test_forward_takes_block_major_path(cuda_lib, w):
-    """nsa_forward with Nb >= 16 topk runs the selection block-major (the merge
+    """nsa_forward with Nb >= 8 topk runs the selection block-major (the merge
     applies the gates); the whole forward still matches the oracle."""
     from test_gpu_parity import compare_forward, gpu_forward
     assert -(-w.T // w.sel_block) >= 16 * w.topk  # Nb
