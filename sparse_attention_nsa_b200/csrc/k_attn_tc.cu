@@ -341,15 +341,16 @@ attn_tc_kernel(const bf16* __restrict__ qg, const __grid_constant__ CUtensorMap 
           for (int c = 0; c < 64; ++c)
             if (k0 + c > t || k0 + c < lo) sv[c] = -INFINITY;
         }
+        // instruction-bound: three-input max, scale and sums on fp32 pairs
         float m0 = sv[0], m1 = sv[1], m2 = sv[2], m3 = sv[3];
 #pragma unroll
-        for (int c = 4; c < 64; c += 4) {
-          m0 = fmaxf(m0, sv[c]);
-          m1 = fmaxf(m1, sv[c + 1]);
-          m2 = fmaxf(m2, sv[c + 2]);
-          m3 = fmaxf(m3, sv[c + 3]);
+        for (int c = 4; c < 64; c += 8) {
+          m0 = fmax3(m0, sv[c], sv[c + 4]);
+          m1 = fmax3(m1, sv[c + 1], sv[c + 5]);
+          m2 = fmax3(m2, sv[c + 2], sv[c + 6]);
+          m3 = fmax3(m3, sv[c + 3], sv[c + 7]);
         }
-        ms = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)) * sl2;
+        ms = fmaxf(fmax3(m0, m1, m2), m3) * sl2;
       }
       const bool grow = rowsel && ms > mref + 8.f;
       const bool resc = grow && mref != -INFINITY;
@@ -363,22 +364,21 @@ attn_tc_kernel(const bf16* __restrict__ qg, const __grid_constant__ CUtensorMap 
       }
       uint32_t pk[32];
       if (rowsel) {
-        const float nm = -mref;
-        float r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f;
+        const uint64_t sc2 = f2_pack(sl2, sl2), nm2 = f2_pack(-mref, -mref);
+        uint64_t r01 = f2_pack(0.f, 0.f), r23 = r01;
 #pragma unroll
         for (int c = 0; c < 64; c += 4) {
-          const float p0 = fast_exp2(fmaf(sv[c], sl2, nm));
-          const float p1 = fast_exp2(fmaf(sv[c + 1], sl2, nm));
-          const float p2 = fast_exp2(fmaf(sv[c + 2], sl2, nm));
-          const float p3 = fast_exp2(fmaf(sv[c + 3], sl2, nm));
-          r0 += p0;
-          r1 += p1;
-          r2 += p2;
-          r3 += p3;
+          const float2 x01 = f2_unpack(f2_fma(f2_pack(sv[c], sv[c + 1]), sc2, nm2));
+          const float2 x23 = f2_unpack(f2_fma(f2_pack(sv[c + 2], sv[c + 3]), sc2, nm2));
+          const float p0 = fast_exp2(x01.x), p1 = fast_exp2(x01.y);
+          const float p2 = fast_exp2(x23.x), p3 = fast_exp2(x23.y);
+          r01 = f2_add(r01, f2_pack(p0, p1));
+          r23 = f2_add(r23, f2_pack(p2, p3));
           pk[c / 2] = pack_bf16(p0, p1);
           pk[c / 2 + 1] = pack_bf16(p2, p3);
         }
-        lsum += (r0 + r1) + (r2 + r3);
+        const float2 a01 = f2_unpack(r01), a23 = f2_unpack(r23);
+        lsum += (a01.x + a01.y) + (a23.x + a23.y);
       } else {
 #pragma unroll
         for (int c = 0; c < 32; ++c) pk[c] = 0u;

@@ -39,6 +39,7 @@
 // TMEM (512 columns): softmax warpgroup x owns [256 x, 256 x + 256): two
 // S/P buffers of 64 columns, then two O buffers of 64.
 #include <atomic>
+#include <cfloat>
 #include <climits>
 
 #include "common.cuh"
@@ -418,31 +419,32 @@ sel_bm_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
 #pragma unroll
           for (int c = 0; c < 64; ++c) sv[c] = c > lim ? -INFINITY : sv[c];
         }
+        // the row is instruction-bound: three-input max, and the scale and
+        // the running sums on fp32 pairs (one instruction per two columns)
         float m0 = sv[0], m1 = sv[1], m2 = sv[2], m3 = sv[3];
 #pragma unroll
-        for (int c = 4; c < 64; c += 4) {
-          m0 = fmaxf(m0, sv[c]);
-          m1 = fmaxf(m1, sv[c + 1]);
-          m2 = fmaxf(m2, sv[c + 2]);
-          m3 = fmaxf(m3, sv[c + 3]);
+        for (int c = 4; c < 64; c += 8) {
+          m0 = fmax3(m0, sv[c], sv[c + 4]);
+          m1 = fmax3(m1, sv[c + 1], sv[c + 5]);
+          m2 = fmax3(m2, sv[c + 2], sv[c + 6]);
+          m3 = fmax3(m3, sv[c + 3], sv[c + 7]);
         }
-        mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)) * sl2;  // key k0 <= t: finite
-        const float nm = -mx;
-        float r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f;
+        mx = fmaxf(fmax3(m0, m1, m2), m3) * sl2;  // key k0 <= t: finite
+        const uint64_t sc2 = f2_pack(sl2, sl2), nm2 = f2_pack(-mx, -mx);
+        uint64_t r01 = f2_pack(0.f, 0.f), r23 = r01;
 #pragma unroll
         for (int c = 0; c < 64; c += 4) {
-          const float p0 = fast_exp2(fmaf(sv[c], sl2, nm));
-          const float p1 = fast_exp2(fmaf(sv[c + 1], sl2, nm));
-          const float p2 = fast_exp2(fmaf(sv[c + 2], sl2, nm));
-          const float p3 = fast_exp2(fmaf(sv[c + 3], sl2, nm));
-          r0 += p0;
-          r1 += p1;
-          r2 += p2;
-          r3 += p3;
+          const float2 x01 = f2_unpack(f2_fma(f2_pack(sv[c], sv[c + 1]), sc2, nm2));
+          const float2 x23 = f2_unpack(f2_fma(f2_pack(sv[c + 2], sv[c + 3]), sc2, nm2));
+          const float p0 = fast_exp2(x01.x), p1 = fast_exp2(x01.y);
+          const float p2 = fast_exp2(x23.x), p3 = fast_exp2(x23.y);
+          r01 = f2_add(r01, f2_pack(p0, p1));
+          r23 = f2_add(r23, f2_pack(p2, p3));
           pk[c / 2] = pack_bf16(p0, p1);
           pk[c / 2 + 1] = pack_bf16(p2, p3);
         }
-        l = (r0 + r1) + (r2 + r3);
+        const float2 a01 = f2_unpack(r01), a23 = f2_unpack(r23);
+        l = (a01.x + a01.y) + (a23.x + a23.y);
       } else {
 #pragma unroll
         for (int c = 0; c < 32; ++c) pk[c] = 0u;
@@ -477,7 +479,7 @@ sel_bm_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
       const uint32_t slot = __float_as_uint(st.z);
       if (!wait_bar_warp(&bars->o[x][bf], (i >> 2) & 1, abort_flag, err)) break;
       tc_fence_after();
-      const float inv = slot != UINT_MAX ? 1.f / st.y : 0.f;
+      const float inv = slot != UINT_MAX ? __fdividef(1.f, st.y) : 0.f;  // l in [1, 64]
       float ov[64];
       tmem_ld32(lane_tmem + (uint32_t)(x * 256 + 128 + bf * 64), ov);
       tmem_ld32(lane_tmem + (uint32_t)(x * 256 + 128 + bf * 64 + 32), ov + 32);
@@ -485,22 +487,22 @@ sel_bm_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
       tc_fence_before();
       mbar_arrive(&bars->ofree[x][bf]);
       // fp16 partials: 11 significant bits, so the merge of up to topk of
-      // them adds well under the output's own bf16 rounding; a partial
-      // beyond fp16's range (|v| > 65504) is reported, not stored silently
-      float amax = 0.f;
+      // them adds well under the output's own bf16 rounding.  A partial
+      // beyond fp16's range (|v| > 65504) becomes inf, which the merge
+      // reports (its output is then not finite).
+      const uint64_t inv2 = f2_pack(inv, inv);
+      uint32_t hv[32];
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        ov[c] *= inv;
-        amax = fmaxf(amax, fabsf(ov[c]));
+      for (int c = 0; c < 64; c += 2) {
+        const float2 v = f2_unpack(f2_mul(f2_pack(ov[c], ov[c + 1]), inv2));
+        hv[c / 2] = pack_f16(v.x, v.y);
       }
-      if (!(amax <= 65504.f) && slot != UINT_MAX) record_error(err, kDevRange);
       __syncwarp();  // the previous tile's staging reads are done
 #pragma unroll
       for (int c = 0; c < 8; ++c)  // fp16 into the staging row, chunks XOR-swizzled by row
-        st_shared_v4(mine + ((uint32_t)(c ^ (lane & 7)) << 4),
-                     pack_f16(ov[8 * c + 0], ov[8 * c + 1]), pack_f16(ov[8 * c + 2], ov[8 * c + 3]),
-                     pack_f16(ov[8 * c + 4], ov[8 * c + 5]), pack_f16(ov[8 * c + 6], ov[8 * c + 7]));
-      if (slot != UINT_MAX) __stcs(part_lse + slot, (st.x + log2f(st.y)) * kLn2);
+        st_shared_v4(mine + ((uint32_t)(c ^ (lane & 7)) << 4), hv[4 * c], hv[4 * c + 1],
+                     hv[4 * c + 2], hv[4 * c + 3]);
+      if (slot != UINT_MAX) __stcs(part_lse + slot, (st.x + __log2f(st.y)) * kLn2);
       __syncwarp();
       // four whole rows per store instruction; loads first so their latencies overlap
       const int c = lane & 7;
@@ -543,7 +545,7 @@ template <bool FUSE>
 __global__ void __launch_bounds__(256)
 sel_merge_kernel(const int32_t* __restrict__ idx, const __half* __restrict__ part_o,
                  const float* __restrict__ part_lse, bf16* __restrict__ o_sel,
-                 float* __restrict__ lse_sel, Dims d, EpilogueFuse fz) {
+                 float* __restrict__ lse_sel, Dims d, EpilogueFuse fz, int* err) {
   const size_t nrows = (size_t)d.B * d.Tq * d.Hq;
   const size_t row0 = (size_t)blockIdx.x * 32 + (threadIdx.x >> 3);
   const bool live = row0 < nrows;  // every lane stays for the shuffles
@@ -601,6 +603,12 @@ sel_merge_kernel(const int32_t* __restrict__ idx, const __half* __restrict__ par
     }
   }
   if (!live) return;
+  // the weights are at most 1, so the sum is finite unless a partial that
+  // contributes to it overflowed fp16 (or the inputs were not finite)
+  bool finite = true;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) finite = finite && fabsf(acc[c]) <= FLT_MAX;
+  if (!finite) record_error(err, kDevRange);
   const float inv = L > 0.f ? 1.f / L : 0.f;
 #pragma unroll
   for (int c = 0; c < 8; ++c) acc[c] *= inv;
@@ -738,10 +746,10 @@ cudaError_t launch_sel_bm(const Dims& d, const void* q, const void* k, const voi
   const unsigned mgrid = (unsigned)((nrows + 31) / 32);
   if (fz)
     sel_merge_kernel<true><<<mgrid, 256, 0, s>>>(idx, part_o, part_lse, (bf16*)o_sel, lse_sel, d,
-                                                 *fz);
+                                                 *fz, err);
   else
     sel_merge_kernel<false><<<mgrid, 256, 0, s>>>(idx, part_o, part_lse, (bf16*)o_sel, lse_sel,
-                                                  d, EpilogueFuse{});
+                                                  d, EpilogueFuse{}, err);
   return cudaGetLastError();
 }
 

@@ -11,6 +11,8 @@
 //
 // One warp per row, no shared memory: the radix select of topk.cuh over the
 // row's fp32 scores read straight from global memory.
+#include <climits>
+
 #include "common.cuh"
 #include "internal.h"
 #include "topk.cuh"
@@ -23,19 +25,22 @@ template <int QMAX>
 __global__ void __launch_bounds__(kTopkWarps * 32)
 topk_kernel(const float* __restrict__ score, int32_t* __restrict__ idx, Dims d) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long r = (long)blockIdx.x * kTopkWarps + warp;
-  const long nrows = (long)d.B * d.Tq * d.Hkv;
-  if (r >= nrows) return;
-  const int tq = (int)((r / d.Hkv) % d.Tq);
-  const int t = d.q_off + tq;
-  // candidates are blocks 1..cur-1 (all complete, so all have scores)
-  warp_select_blocks<QMAX>(score + r * d.Nc, t / d.l, d.topk, idx + r * d.topk, lane);
+  const int rb = blockIdx.x * kTopkWarps + warp;  // row within the sequence: tq * Hkv + g
+  if (rb >= d.Tq * d.Hkv) return;
+  const int t = d.q_off + rb / d.Hkv;
+  for (int b = blockIdx.y; b < d.B; b += gridDim.y) {
+    const size_t r = (size_t)b * d.Tq * d.Hkv + rb;
+    // candidates are blocks 1..cur-1 (all complete, so all have scores)
+    warp_select_blocks<QMAX>(score + r * d.Nc, t / d.l, d.topk, idx + r * d.topk, lane);
+  }
 }
 
 cudaError_t launch_topk(const Dims& d, const float* score, int32_t* idx,
                         cudaStream_t s) {
-  const long nrows = (long)d.B * d.Tq * d.Hkv;
-  const unsigned blocks = (unsigned)((nrows + kTopkWarps - 1) / kTopkWarps);
+  const long rows = (long)d.Tq * d.Hkv;  // per sequence (< 2^31: Tq < 2^24, Hkv <= 128)
+  if (rows == 0 || d.B == 0) return cudaSuccess;
+  if (rows > INT_MAX - kTopkWarps) return cudaErrorInvalidValue;
+  const dim3 blocks((unsigned)((rows + kTopkWarps - 1) / kTopkWarps), (unsigned)min(d.B, 65535));
   const int q = (d.Nb + 31) / 32;  // candidate slots per lane
   if (q <= 4) topk_kernel<4><<<blocks, kTopkWarps * 32, 0, s>>>(score, idx, d);
   else if (q <= 8) topk_kernel<8><<<blocks, kTopkWarps * 32, 0, s>>>(score, idx, d);

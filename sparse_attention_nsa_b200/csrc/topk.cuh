@@ -43,15 +43,29 @@ __device__ __forceinline__ void warp_select_blocks(const float* score, int cur, 
     key[q] = j < cur ? order_key(score[j]) : 0u;
   }
   const int K2 = topk - 2;
-  // tau = the largest value with at least K2 keys >= tau (absent slots are
-  // excluded from the counts).  The search stops as soon as exactly K2 keys
-  // are >= tau: those are the winners whatever the lower bits of tau.
-  uint32_t tau = 0u;
-  for (int bit = 31; bit >= 0; --bit) {
+  // tau = the largest value with at least K2 keys >= tau.  Absent slots hold
+  // key 0 and every threshold tried is >= 1, so they never count.  The bits
+  // all candidates share are tau's from the start (every key is >= that
+  // prefix); the search walks down from the highest bit in which two
+  // candidates differ and stops as soon as exactly K2 keys are >= tau:
+  // those are the winners whatever the lower bits of tau.
+  uint32_t kand = 0xffffffffu, kor = 0u;
+#pragma unroll
+  for (int q = 0; q < QMAX; ++q)
+    if (1 + lane + 32 * q < cur) {
+      kand &= key[q];
+      kor |= key[q];
+    }
+  kand = __reduce_and_sync(0xffffffffu, kand);
+  kor = __reduce_or_sync(0xffffffffu, kor);
+  const uint32_t diff = kand ^ kor;
+  int bit = diff ? 31 - __clz(diff) : -1;
+  uint32_t tau = bit >= 0 ? kand & ~((2u << bit) - 1u) : kand;  // bit 31: 2u << 31 == 0
+  for (; bit >= 0; --bit) {
     const uint32_t tc = tau | (1u << bit);
     unsigned c = 0;
 #pragma unroll
-    for (int q = 0; q < QMAX; ++q) c += (1 + lane + 32 * q < cur && key[q] >= tc) ? 1u : 0u;
+    for (int q = 0; q < QMAX; ++q) c += key[q] >= tc ? 1u : 0u;
     const int cnt = (int)__reduce_add_sync(0xffffffffu, c);
     if (cnt >= K2) tau = tc;
     if (cnt == K2) break;
