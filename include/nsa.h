@@ -88,7 +88,7 @@ typedef struct {
   int sel_block;   /* l' : tokens per selection block (= l)         */
   int topk;        /* n  : selected blocks per (query, KV group), >= 2 */
   int window;      /* w  : sliding-window length in keys, >= 1      */
-  float scale;     /* softmax scale, normally 1/sqrt(D)             */
+  float scale;     /* softmax scale, finite and > 0, normally 1/sqrt(D) */
   int dtype;       /* nsa_dtype of q/k/v/kc/vc/o_*                   */
   int branch_mask; /* NSA_BRANCH_* bits of the branches to combine   */
 } nsa_params;

@@ -76,7 +76,7 @@ template <bool WITH_O>
 __global__ void __launch_bounds__(kThreads, 2)
 cmp_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kc,
               const __grid_constant__ CUtensorMap tm_vc, bf16* __restrict__ o_cmp,
-              float* __restrict__ lse, float* __restrict__ score, Dims d, int* err) {
+              float* __restrict__ lse, float* __restrict__ score, Dims d, int* err, bool vec4) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   Bars* bars = (Bars*)(smem + OFF_BAR);
@@ -198,9 +198,12 @@ cmp_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const float sl2 = d.scale * kLog2e;
     const uint32_t lane_tmem = tmem + ((uint32_t)(warp * 32) << 16);
     float m = -INFINITY, lsum = 0.f;
+    float mu0 = -INFINITY, mu1 = -INFINITY;  // with both chunks resident: their reference maxima
     bool ok = true;
     float sv[64];
-    // pass 1: row statistics
+    // pass 1: row statistics.  With both chunks resident in TMEM the
+    // exponentials (relative to the running max m_u after chunk u) are
+    // written back over S, so pass 2 only rescales them by 2^(m_u - m) / l.
     for (int u = 0; u < n; ++u) {
       if (!wait_bar_warp(&bars->s[u & 1], (u >> 1) & 1, abort_flag, err)) {
         ok = false;
@@ -216,21 +219,42 @@ cmp_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       }
       const int j0 = u * kChunk;
       if (j0 < nvis) {
-        float mx = -INFINITY;
+        if (j0 + kChunk > nvis) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const float x = j0 + c < nvis ? sv[c] * sl2 : -INFINITY;
-          sv[c] = x;
-          mx = fmaxf(mx, x);
+          for (int c = 0; c < 64; ++c) sv[c] = j0 + c < nvis ? sv[c] : -INFINITY;
         }
-        const float mn = fmaxf(m, mx);
-        float rs = 0.f;
+        float m0 = sv[0], m1 = sv[1], m2 = sv[2], m3 = sv[3];
 #pragma unroll
-        for (int c = 0; c < 64; ++c) rs += fast_exp2(sv[c] - mn);
-        lsum = lsum * fast_exp2(m - mn) + rs;
+        for (int c = 4; c < 64; c += 8) {
+          m0 = fmax3(m0, sv[c], sv[c + 4]);
+          m1 = fmax3(m1, sv[c + 1], sv[c + 5]);
+          m2 = fmax3(m2, sv[c + 2], sv[c + 6]);
+          m3 = fmax3(m3, sv[c + 3], sv[c + 7]);
+        }
+        const float mn = fmaxf(m, fmaxf(fmax3(m0, m1, m2), m3) * sl2);  // column 0 is visible
+        const uint64_t sc2 = f2_pack(sl2, sl2), nm2 = f2_pack(-mn, -mn);
+        uint64_t r2 = f2_pack(0.f, 0.f);
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          const float2 x = f2_unpack(f2_fma(f2_pack(sv[c], sv[c + 1]), sc2, nm2));
+          sv[c] = fast_exp2(x.x);
+          sv[c + 1] = fast_exp2(x.y);
+          r2 = f2_add(r2, f2_pack(sv[c], sv[c + 1]));
+        }
+        const float2 rs = f2_unpack(r2);
+        lsum = lsum * fast_exp2(m - mn) + (rs.x + rs.y);
         m = mn;
+        if (u == 0) mu0 = mn;
+        else mu1 = mn;
+      }
+      // tcgen05.st is warp-collective: every lane stores (a row that sees
+      // none of this chunk stores its raw S, which pass 2 never reads)
+      if (res) {
+        tmem_st32(lane_tmem + (uint32_t)u * 64u, sv);
+        tmem_st32(lane_tmem + (uint32_t)u * 64u + 32u, sv + 32);
       }
     }
+    if (res) tmem_wait_st();
     const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
     float* srow = score + (((size_t)b * d.Tq + t0 + tl) * d.Hkv + g) * d.Nc;
     const int per = 64 / d.G;  // score columns written by each head-lane of a token
@@ -250,9 +274,23 @@ cmp_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         mbar_arrive(&bars->sfree[u & 1]);
       }
       const int j0 = i * kChunk;
+      if (j0 >= nvis) {
 #pragma unroll
-      for (int c = 0; c < 64; ++c)
-        sv[c] = j0 + c < nvis ? fast_exp2(fmaf(sv[c], sl2, -m)) * inv : 0.f;
+        for (int c = 0; c < 64; ++c) sv[c] = 0.f;
+      } else if (res) {  // stored 2^(s - m_i): masked columns are already 0
+        const float fac = fast_exp2((i == 0 ? mu0 : mu1) - m) * inv;
+        const uint64_t f2 = f2_pack(fac, fac);
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          const float2 x = f2_unpack(f2_mul(f2_pack(sv[c], sv[c + 1]), f2));
+          sv[c] = x.x;
+          sv[c + 1] = x.y;
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          sv[c] = j0 + c < nvis ? fast_exp2(fmaf(sv[c], sl2, -m)) * inv : 0.f;
+      }
       if (WITH_O) {
         if (i >= 2 && !wait_bar_warp(&bars->pfree[i & 1], ((i - 2) >> 1) & 1, abort_flag, err)) {
           ok = false;
@@ -280,13 +318,27 @@ cmp_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       if (d.G >= 16) reduce_half<4>(sv, hh & (4 / per), 4 / per);
       if (d.G >= 32) reduce_half<2>(sv, hh & (2 / per), 2 / per);
       if (valid) {
+        const int jb = j0 + hh * per;
+        if (vec4) {  // 16-byte groups, each wholly inside or outside [0, Nc)
 #pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (c < per && j0 + hh * per + c < d.Nc) srow[j0 + hh * per + c] = sv[c];
+          for (int c = 0; c < 64; c += 4)
+            if (c < per && jb + c < d.Nc)
+              *reinterpret_cast<float4*>(srow + jb + c) =
+                  make_float4(sv[c], sv[c + 1], sv[c + 2], sv[c + 3]);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (c < per && jb + c < d.Nc) srow[jb + c] = sv[c];
+        }
       }
     }
-    if (valid)  // blocks beyond the last chunk are not visible to this tile
-      for (int j = n * kChunk + hh; j < d.Nc; j += d.G) srow[j] = 0.f;
+    if (valid) {  // blocks beyond the last chunk are not visible to this tile
+      if (vec4)
+        for (int j = n * kChunk + 4 * hh; j < d.Nc; j += 4 * d.G)
+          *reinterpret_cast<float4*>(srow + j) = make_float4(0.f, 0.f, 0.f, 0.f);
+      else
+        for (int j = n * kChunk + hh; j < d.Nc; j += d.G) srow[j] = 0.f;
+    }
     float ov[64];
     const bool have_o = WITH_O && ok && n > 0 &&
                         wait_bar_warp(&bars->odone, 0, abort_flag, err);
@@ -341,8 +393,11 @@ cudaError_t launch_cmp_tc(const Dims& d, const void* q, const void* kc, const vo
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid((d.Tq + TQ - 1) / TQ, d.Hkv, d.B);
+  // score rows in 16-byte groups when every group is aligned: Nc % 4 == 0,
+  // a head-lane's run of 64 / G columns a multiple of 4, an aligned base
+  const bool vec4 = d.Nc % 4 == 0 && d.G <= 16 && ((uintptr_t)score & 15) == 0;
   cmp_tc_kernel<WITH_O><<<grid, kThreads, kSmemBytes, s>>>(mq, mk, mv, (bf16*)o_cmp, lse, score,
-                                                          d, err);
+                                                          d, err, vec4);
   return cudaGetLastError();
 }
 

@@ -48,8 +48,8 @@ nsa_status fill_dims(const nsa_params* p, Dims* d) {
   if (p->Hq % p->Hkv != 0) return NSA_ERR_INVALID_ARG;
   if (p->dtype != NSA_F32 && p->dtype != NSA_BF16) return NSA_ERR_INVALID_ARG;
   if (p->branch_mask < 1 || p->branch_mask > NSA_BRANCH_ALL) return NSA_ERR_INVALID_ARG;
-  if (!(p->scale == p->scale) || p->scale == INFINITY || p->scale == -INFINITY)
-    return NSA_ERR_INVALID_ARG;
+  // a positive finite scale: the kernels take each row's max before scaling
+  if (!(p->scale > 0.f) || p->scale == INFINITY) return NSA_ERR_INVALID_ARG;
   // valid NSA geometry, but outside what this build runs
   if (p->D != 64) return NSA_ERR_UNSUPPORTED;
   if (p->cmp_stride != p->cmp_block || p->sel_block != p->cmp_block)

@@ -52,7 +52,8 @@ def test_workload_params_are_accepted(w):
 BAD = [
     (dict(B=0), 1), (dict(T=0), 1), (dict(Tq=5000), 1), (dict(Hkv=3), 1),
     (dict(topk=1), 1), (dict(window=0), 1), (dict(dtype=7), 1), (dict(branch_mask=0), 1),
-    (dict(branch_mask=9), 1), (dict(scale=float("nan")), 1),
+    (dict(branch_mask=9), 1), (dict(scale=float("nan")), 1), (dict(scale=-0.125), 1), (dict(scale=0.0), 1),
+    (dict(scale=float("inf")), 1),
     (dict(D=128), 2), (dict(cmp_stride=32), 2), (dict(sel_block=32), 2),
     (dict(Hq=24, Hkv=4), 2), (dict(topk=65), 2), (dict(T=200000), 2),
 ]
