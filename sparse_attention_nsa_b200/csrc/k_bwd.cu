@@ -232,6 +232,7 @@ rev_chunk_scan_kernel(int* __restrict__ chunk, int* __restrict__ offsets, Dims d
                       int tpu, int umax) {
   extern __shared__ int tot[];  // [Nb]
   __shared__ int wsum[32];
+  __shared__ int utotal;
   const int bg = blockIdx.x;
   int* cc = chunk + (size_t)bg * nchunk * d.Nb;
   for (int j = threadIdx.x; j < d.Nb; j += blockDim.x) {
@@ -306,15 +307,33 @@ rev_chunk_scan_kernel(int* __restrict__ chunk, int* __restrict__ offsets, Dims d
       if (lane >= o2) wi += y;
     }
     wsum[lane] = wi - w;
-    if (lane == 31) ucount[bg] = wi;
+    if (lane == 31) {
+      ucount[bg] = wi;
+      utotal = wi;
+    }
   }
   __syncthreads();
+  // tot[j] = block j's first unit; then unit u belongs to the last block j
+  // with tot[j] <= u (a block with no units shares its tot with the next),
+  // so the units are written by all threads, not by the owner of a block
+  // whose list is long (block 0 is in every query's selection)
   int at = wsum[warp] + ui - nu;
-  int4* ub = units + (size_t)bg * umax;
   for (int j = lo; j < hi; ++j) {
     cursor[(size_t)bg * d.Nb + j] = off[j];
-    for (int p0 = off[j]; p0 < off[j + 1]; p0 += tpu)
-      ub[at++] = make_int4(j, p0, min(p0 + tpu, off[j + 1]), 0);
+    tot[j] = at;
+    at += (off[j + 1] - off[j] + tpu - 1) / tpu;
+  }
+  __syncthreads();
+  int4* ub = units + (size_t)bg * umax;
+  for (int u = threadIdx.x; u < utotal; u += blockDim.x) {
+    int a = 0, z = d.Nb - 1;  // tot[0] = 0 <= u
+    while (a < z) {
+      const int mid = (a + z + 1) >> 1;
+      if (tot[mid] <= u) a = mid;
+      else z = mid - 1;
+    }
+    const int p0 = off[a] + (u - tot[a]) * tpu;
+    ub[u] = make_int4(a, p0, min(p0 + tpu, off[a + 1]), 0);
   }
 }
 

@@ -399,6 +399,9 @@ sel_bm_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
       const int e = ering[(i & (kERing - 1)) * kRows + r];
       if (!wait_bar_warp(&bars->s[x][bf], (i >> 2) & 1, abort_flag, err)) break;
       if (i + 2 < ntiles) publish_q(i + 2);
+      // tile i+kQBufs's Q into the buffer tile i's S MMA has finished
+      // reading; the copies are in flight under this tile's softmax
+      if (!copy_q(i + kQBufs)) break;
       const int4 u = us[tl[i] >> 2];
       const bool valid = e >= 0;
       const int tq = max(e, 0) >> 6;
@@ -453,8 +456,6 @@ sel_bm_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars->p[x][bf]);
-      // tile i+kQBufs's Q into the buffer tile i's S MMA has finished reading
-      if (!copy_q(i + kQBufs)) break;
       // the row's statistics and partial slot for the epilogue
       uint32_t slot = UINT_MAX;
       if (valid)
