@@ -96,8 +96,13 @@ cudaError_t launch_revmap(const Dims& d, const int32_t* idx, int* chunk, int* of
 // group) the lists are cut into work units of at most tpu entries
 // (units[bg * umax + u] = (block, first, end) for u < ucount[bg]).
 // cursor: B * Hkv * Nb ints.
+// Reverse map of the forward's selection plus its work units: per (sequence,
+// group) at most umax units of at most tpu = k * tq list entries (k <= 4
+// tiles of tq entries), written sorted by size (units of k tiles first, then
+// tails of k - 1, ..., 1 tiles, each class in block order); ucount holds the
+// four class sizes of each (sequence, group) as an int4.
 cudaError_t launch_revmap_units(const Dims& d, const int32_t* idx, int* chunk, int* offsets,
-                                int* cursor, int* list, int4* units, int* ucount, int tpu,
+                                int* cursor, int* list, int4* units, int* ucount, int tpu, int tq,
                                 int umax, int* err, cudaStream_t s);
 cudaError_t launch_dkdv(const Dims& d, int mode, const void* q, const void* keys,
                         const void* vals, const float* lse, const float* delta,

@@ -184,6 +184,7 @@ dq_kernel(const T* __restrict__ q, const T* __restrict__ keys, const T* __restri
 // that chose the same block.  A selection counts when it is a real,
 // causal block that does not repeat or go back (the forward's rule).
 constexpr int kRevChunk = 256;
+constexpr int kMaxUnitClasses = 4;  // work-unit sizes of 1 .. 4 tiles
 
 __device__ __forceinline__ bool rev_valid(const int32_t* ir, int s, int cur) {
   const int j = ir[s];
@@ -229,9 +230,11 @@ rev_chunk_count_kernel(const int32_t* __restrict__ idx, int* __restrict__ chunk,
 __global__ void __launch_bounds__(1024)
 rev_chunk_scan_kernel(int* __restrict__ chunk, int* __restrict__ offsets, Dims d, int nchunk,
                       int4* __restrict__ units, int* __restrict__ ucount, int* __restrict__ cursor,
-                      int tpu, int umax) {
-  extern __shared__ int tot[];  // [Nb]
+                      int tpu, int tq, int umax) {
+  extern __shared__ int tot[];  // [Nb]; with units [Nb + 1] offsets, then [kMaxUnitClasses][Nb]
   __shared__ int wsum[32];
+  __shared__ int4 wsum4[32];
+  __shared__ int cbase[kMaxUnitClasses];
   __shared__ int utotal;
   const int bg = blockIdx.x;
   int* cc = chunk + (size_t)bg * nchunk * d.Nb;
@@ -279,61 +282,125 @@ rev_chunk_scan_kernel(int* __restrict__ chunk, int* __restrict__ offsets, Dims d
     off[j] = run;
     run += t;
   }
-  if (threadIdx.x == blockDim.x - 1) off[d.Nb] = run;
+  if (threadIdx.x == blockDim.x - 1) {
+    off[d.Nb] = run;
+    if (units) tot[d.Nb] = run;  // with units tot holds Nb + 1 offsets
+  }
   __syncthreads();
   for (int j = threadIdx.x; j < d.Nb; j += blockDim.x)
     for (int c = 0; c < nchunk; ++c) cc[(size_t)c * d.Nb + j] += tot[j];
   if (!units) return;
-  // work units of at most tpu list entries: block j's list [off[j], off[j+1])
-  // split into ceil(len / tpu) consecutive pieces, blocks in ascending order
-  int nu = 0;
-  for (int j = lo; j < hi; ++j) nu += (off[j + 1] - off[j] + tpu - 1) / tpu;
-  int ui = nu;
+  // Work units of at most tpu list entries (tpu = kseg tiles of tq entries):
+  // block j's list [off[j], off[j+1]) in consecutive pieces.  The group's
+  // units are written sorted by size, so that the kernel can deal them out
+  // evenly: class 0 = units of kseg tiles (block order; a block's full units,
+  // then its tail if that also has kseg tiles), class c = the tails of
+  // kseg - c tiles (block order).  ucls[bg][c] = the class sizes.
+  // tq and tpu are powers of two (shifts, not divisions); the offsets are
+  // read from shared memory (tot[0 .. Nb])
+  const int lq = __ffs(tq) - 1, lpu = __ffs(tpu) - 1;
+  const int kseg = tpu >> lq;  // <= kMaxUnitClasses
+  const int* offs = tot;
+  auto block_counts = [&](int j, int4& n) {
+    const int len = offs[j + 1] - offs[j];
+    const int nf = len >> lpu, rem = len - (nf << lpu);
+    const int tc = rem ? (rem + tq - 1) >> lq : 0;  // tail tiles, 0 = no tail
+    int a[kMaxUnitClasses] = {nf + (tc == kseg ? 1 : 0), 0, 0, 0};
+    if (tc > 0 && tc < kseg) a[kseg - tc] = 1;
+    n = make_int4(a[0], a[1], a[2], a[3]);
+  };
+  int4 mine = make_int4(0, 0, 0, 0);
+  for (int j = lo; j < hi; ++j) {
+    int4 n;
+    block_counts(j, n);
+    mine.x += n.x;
+    mine.y += n.y;
+    mine.z += n.z;
+    mine.w += n.w;
+  }
+  int4 incl4 = mine;
 #pragma unroll
   for (int o2 = 1; o2 < 32; o2 <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, ui, o2);
-    if (lane >= o2) ui += y;
+    const int ax = __shfl_up_sync(0xffffffffu, incl4.x, o2);
+    const int ay = __shfl_up_sync(0xffffffffu, incl4.y, o2);
+    const int az = __shfl_up_sync(0xffffffffu, incl4.z, o2);
+    const int aw = __shfl_up_sync(0xffffffffu, incl4.w, o2);
+    if (lane >= o2) {
+      incl4.x += ax;
+      incl4.y += ay;
+      incl4.z += az;
+      incl4.w += aw;
+    }
   }
-  __syncthreads();  // wsum is reused
-  if (lane == 31) wsum[warp] = ui;
+  __syncthreads();  // wsum and tot are reused below
+  if (lane == 31) wsum4[warp] = incl4;
   __syncthreads();
   if (warp == 0) {
     const int nw = (blockDim.x + 31) / 32;
-    int w = lane < nw ? wsum[lane] : 0;
-    int wi = w;
+    const int4 w = lane < nw ? wsum4[lane] : make_int4(0, 0, 0, 0);
+    int4 wi = w;
 #pragma unroll
     for (int o2 = 1; o2 < 32; o2 <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, wi, o2);
-      if (lane >= o2) wi += y;
+      const int ax = __shfl_up_sync(0xffffffffu, wi.x, o2);
+      const int ay = __shfl_up_sync(0xffffffffu, wi.y, o2);
+      const int az = __shfl_up_sync(0xffffffffu, wi.z, o2);
+      const int aw = __shfl_up_sync(0xffffffffu, wi.w, o2);
+      if (lane >= o2) {
+        wi.x += ax;
+        wi.y += ay;
+        wi.z += az;
+        wi.w += aw;
+      }
     }
-    wsum[lane] = wi - w;
+    wsum4[lane] = make_int4(wi.x - w.x, wi.y - w.y, wi.z - w.z, wi.w - w.w);  // exclusive
     if (lane == 31) {
-      ucount[bg] = wi;
-      utotal = wi;
+      reinterpret_cast<int4*>(ucount)[bg] = wi;  // class sizes
+      cbase[0] = 0;
+      cbase[1] = wi.x;
+      cbase[2] = wi.x + wi.y;
+      cbase[3] = wi.x + wi.y + wi.z;
+      utotal = wi.x + wi.y + wi.z + wi.w;
     }
   }
   __syncthreads();
-  // tot[j] = block j's first unit; then unit u belongs to the last block j
-  // with tot[j] <= u (a block with no units shares its tot with the next),
-  // so the units are written by all threads, not by the owner of a block
-  // whose list is long (block 0 is in every query's selection)
-  int at = wsum[warp] + ui - nu;
-  for (int j = lo; j < hi; ++j) {
-    cursor[(size_t)bg * d.Nb + j] = off[j];
-    tot[j] = at;
-    at += (off[j + 1] - off[j] + tpu - 1) / tpu;
+  // pre[c][j] = the units of class c before block j
+  int* pre = tot + d.Nb + 1;  // [kMaxUnitClasses][Nb]
+  {
+    const int4 w = wsum4[warp];
+    int4 at = make_int4(w.x + incl4.x - mine.x, w.y + incl4.y - mine.y, w.z + incl4.z - mine.z,
+                        w.w + incl4.w - mine.w);
+    for (int j = lo; j < hi; ++j) {
+      cursor[(size_t)bg * d.Nb + j] = offs[j];
+      pre[j] = at.x;
+      pre[d.Nb + j] = at.y;
+      pre[2 * d.Nb + j] = at.z;
+      pre[3 * d.Nb + j] = at.w;
+      int4 n;
+      block_counts(j, n);
+      at.x += n.x;
+      at.y += n.y;
+      at.z += n.z;
+      at.w += n.w;
+    }
   }
   __syncthreads();
+  // unit p of class c, rank r in its class, belongs to the last block j
+  // with pre[c][j] <= r (a block with none shares its prefix with the next)
   int4* ub = units + (size_t)bg * umax;
-  for (int u = threadIdx.x; u < utotal; u += blockDim.x) {
-    int a = 0, z = d.Nb - 1;  // tot[0] = 0 <= u
+  for (int p = threadIdx.x; p < utotal; p += blockDim.x) {
+    const int c = p < cbase[1] ? 0 : p < cbase[2] ? 1 : p < cbase[3] ? 2 : 3;
+    const int r = p - cbase[c];
+    const int* pc = pre + c * d.Nb;
+    int a = 0, z = d.Nb - 1;
     while (a < z) {
       const int mid = (a + z + 1) >> 1;
-      if (tot[mid] <= u) a = mid;
+      if (pc[mid] <= r) a = mid;
       else z = mid - 1;
     }
-    const int p0 = off[a] + (u - tot[a]) * tpu;
-    ub[u] = make_int4(a, p0, min(p0 + tpu, off[a + 1]), 0);
+    const int nf = (offs[a + 1] - offs[a]) >> lpu;
+    const int k = c == 0 ? r - pc[a] : nf;  // the tail follows the full units
+    const int p0 = offs[a] + (k << lpu);
+    ub[p] = make_int4(a, p0, min(p0 + tpu, offs[a + 1]), 0);
   }
 }
 
@@ -610,15 +677,17 @@ cudaError_t launch_revmap(const Dims& d, const int32_t* idx, int* chunk, int* of
   rev_chunk_count_kernel<<<dim3(nchunk, d.Hkv, d.B), kRevChunk, nb_bytes, s>>>(idx, chunk, d,
                                                                               nullptr, nullptr);
   rev_chunk_scan_kernel<<<d.B * d.Hkv, 1024, nb_bytes, s>>>(chunk, offsets, d, nchunk, nullptr,
-                                                           nullptr, nullptr, 0, 0);
+                                                           nullptr, nullptr, 0, 1, 0);
   rev_chunk_fill_kernel<<<dim3(nchunk, d.Hkv, d.B), 32, 2 * nb_bytes, s>>>(idx, chunk,
                                                                                   list, d);
   return cudaGetLastError();
 }
 
 cudaError_t launch_revmap_units(const Dims& d, const int32_t* idx, int* chunk, int* offsets,
-                                int* cursor, int* list, int4* units, int* ucount, int tpu,
+                                int* cursor, int* list, int4* units, int* ucount, int tpu, int tq,
                                 int umax, int* err, cudaStream_t s) {
+  if (tq < 1 || (tq & (tq - 1)) || (tpu & (tpu - 1)) || tpu < tq || tpu / tq > kMaxUnitClasses)
+    return cudaErrorInvalidValue;  // powers of two, at most four tiles a unit
   const int nchunk = (d.Tq + kRevChunk - 1) / kRevChunk;
   if (nchunk == 0 || d.Nb == 0) return cudaSuccess;
   const size_t nb_bytes = (size_t)d.Nb * sizeof(int);
@@ -627,8 +696,8 @@ cudaError_t launch_revmap_units(const Dims& d, const int32_t* idx, int* chunk, i
   if (e != cudaSuccess) return e;
   rev_chunk_count_kernel<<<dim3(nchunk, d.Hkv, d.B), kRevChunk, nb_bytes, s>>>(idx, chunk, d,
                                                                               err, chunk);
-  rev_chunk_scan_kernel<<<d.B * d.Hkv, 1024, nb_bytes, s>>>(chunk, offsets, d, 1, units,
-                                                           ucount, cursor, tpu, umax);
+  rev_chunk_scan_kernel<<<d.B * d.Hkv, 1024, (kMaxUnitClasses + 1) * nb_bytes + sizeof(int), s>>>(
+      chunk, offsets, d, 1, units, ucount, cursor, tpu, tq, umax);
   rev_atomic_fill_kernel<<<dim3(nchunk, d.Hkv, d.B), kRevChunk, 2 * nb_bytes, s>>>(idx, cursor,
                                                                                    list, d);
   return cudaGetLastError();

@@ -54,12 +54,13 @@ using namespace sm100;
 
 constexpr int kRows = 128;       // rows per tile (M)
 constexpr int kKeys = 64;        // keys per block
-constexpr int kSeg = 4;          // tiles per work unit
+constexpr int kSeg = 4;          // tiles per work unit (unit sizes 1 .. kSeg: four classes)
 constexpr int kThreads = 512;
 constexpr int kQBufs = 8;        // Q tiles in shared memory (copied kQBufs tiles ahead)
 constexpr int kERing = 16;       // list-entry ring (tiles)
 constexpr int kMRing = 8;        // row-statistics ring (tiles)
 constexpr int kMaxUnits = 256;   // units per CTA (the grid grows past that)
+constexpr int kMaxSortedGroups = 1024;  // (sequence, group) pairs whose units are dealt by size
 constexpr uint32_t kTileBytes = kKeys * 64 * 2;  // one K or V block, bf16
 constexpr uint32_t kQBytes = kRows * 64 * 2;
 
@@ -94,8 +95,12 @@ struct Bars {
   uint64_t fin;                // every P*V of the CTA is done
   uint64_t sfin;               // every S MMA of the CTA is done
 };
-constexpr uint32_t OFF_MISC = OFF_BAR + ((sizeof(Bars) + 15) / 16) * 16;  // tmem, abort, ntiles
-constexpr uint32_t SMEM_BYTES = OFF_MISC + 16;
+// tmem, abort, ntiles, units, four class bases, unit total
+constexpr uint32_t OFF_MISC = OFF_BAR + ((sizeof(Bars) + 15) / 16) * 16;
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 48;
+static_assert(kSeg == 4, "four unit-size classes");
+static_assert(kMRing * kRows * 16 >= 4 * kMaxSortedGroups * 4, "class prefixes fit the row ring");
+static_assert(kERing * kRows * 4 >= 16 * 4 * 4, "scan scratch fits the entry ring");
 
 __host__ __device__ inline int tile_tokens(int G) { return kRows / G; }
 
@@ -122,9 +127,9 @@ sel_bm_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
   const int TQ = tile_tokens(d.G);
   const int lgG = __ffs(d.G) - 1;  // G is a power of two (it divides 128)
-  const int nU = d.B * d.Hkv * umax;
-  const int nk = (int)blockIdx.x < nU ? (nU - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x
-                                      : 0;  // <= kMaxUnits (host sizes the grid)
+  const int BG = d.B * d.Hkv;
+  const int nU = BG * umax;
+  const int4* ucls = reinterpret_cast<const int4*>(ucount);  // class sizes per (sequence, group)
   const size_t list_stride = (size_t)d.Tq * d.topk;  // list entries per (sequence, group)
 
   if (tid == 0) {
@@ -153,14 +158,100 @@ sel_bm_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     fence_proxy_async_smem();
     *abort_flag = 0;
   }
-  for (int k = tid; k < nk; k += kThreads) {  // this CTA's units
-    const int U = (int)blockIdx.x + k * (int)gridDim.x;
-    const int bg = U / umax;
-    int4 e = make_int4(0, 0, 0, U);
-    if (U - bg * umax < __ldg(ucount + bg)) {
-      const int4 x = __ldg(units + U);
+  // This CTA's units.  Each group's units come sorted by size (kSeg tiles,
+  // then tails of kSeg-1 .. 1 tiles); with at most kMaxSortedGroups groups
+  // the CTAs deal the globally sorted sequence (class by class, groups in
+  // order) in a snake: CTA c takes positions c, 2 grid - 1 - c, 2 grid + c,
+  // ..., so every CTA gets nearly the same number of tiles.  With more
+  // groups, CTA c takes unit slots c, c + grid, ... of the groups' arrays.
+  int* misc = (int*)(smem + OFF_MISC);  // [3] units of this CTA, [4..7] class bases, [8] total
+  const bool dealt = BG <= kMaxSortedGroups;
+  const int bid = (int)blockIdx.x, grid = (int)gridDim.x;
+  int* pre = (int*)(smem + OFF_MRING);  // [4][BG] per class: its units in the groups before
+  if (dealt) {
+    // exclusive scan over the groups of the four class sizes (two groups a thread)
+    int* wsum = (int*)(smem + OFF_ERING);  // 16 warps x 4, scratch before the ring is used
+    const int g0 = 2 * tid, g1 = 2 * tid + 1;
+    const int4 v0 = g0 < BG ? __ldg(ucls + g0) : make_int4(0, 0, 0, 0);
+    const int4 v1 = g1 < BG ? __ldg(ucls + g1) : make_int4(0, 0, 0, 0);
+    int inc[4] = {v0.x + v1.x, v0.y + v1.y, v0.z + v1.z, v0.w + v1.w};
+    const int own[4] = {inc[0], inc[1], inc[2], inc[3]};
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int y = __shfl_up_sync(0xffffffffu, inc[c], o);
+        if (lane >= o) inc[c] += y;
+      }
+    if (lane == 31)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) wsum[warp * 4 + c] = inc[c];
+    __syncthreads();
+    int ex[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      int base = 0, all = 0;
+      for (int w2 = 0; w2 < kThreads / 32; ++w2) {
+        const int x = wsum[w2 * 4 + c];
+        base += w2 < warp ? x : 0;
+        all += x;
+      }
+      ex[c] = base + inc[c] - own[c];
+      if (tid == 0) misc[4 + c] = all;  // class total, turned into bases below
+    }
+    const int v0c[4] = {v0.x, v0.y, v0.z, v0.w};
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      if (g0 < BG) pre[c * BG + g0] = ex[c];
+      if (g1 < BG) pre[c * BG + g1] = ex[c] + v0c[c];
+    }
+    __syncthreads();
+    if (tid == 0) {
+      int at = 0;
+      for (int c = 0; c < 4; ++c) {
+        const int n = misc[4 + c];
+        misc[4 + c] = at;
+        at += n;
+      }
+      misc[8] = at;
+      const int F = at / grid, rem = at - F * grid;
+      const int posF = (F & 1) ? grid - 1 - bid : bid;
+      misc[3] = F + (posF < rem ? 1 : 0);  // <= ceil(nU / grid) <= kMaxUnits
+    }
+  } else if (tid == 0) {
+    misc[3] = bid < nU ? (nU - bid + grid - 1) / grid : 0;  // <= kMaxUnits (host sizes the grid)
+  }
+  __syncthreads();
+  const int nk = misc[3];
+  for (int k = tid; k < nk; k += kThreads) {
+    int bg, local;
+    bool live = true;
+    if (dealt) {
+      const int sp = k * grid + ((k & 1) ? grid - 1 - bid : bid);
+      const int c = sp < misc[5] ? 0 : sp < misc[6] ? 1 : sp < misc[7] ? 2 : 3;
+      const int r = sp - misc[4 + c];
+      const int* pc = pre + c * BG;
+      int a = 0, z = BG - 1;  // the last group with pc[a] <= r
+      while (a < z) {
+        const int mid = (a + z + 1) >> 1;
+        if (pc[mid] <= r) a = mid;
+        else z = mid - 1;
+      }
+      bg = a;
+      const int4 n = __ldg(ucls + bg);  // the group's units of the classes before c come first
+      local = (c > 0 ? n.x : 0) + (c > 1 ? n.y : 0) + (c > 2 ? n.z : 0) + (r - pc[a]);
+    } else {
+      const int U = bid + k * grid;
+      bg = U / umax;
+      local = U - bg * umax;
+      const int4 n = __ldg(ucls + bg);
+      live = local < n.x + n.y + n.z + n.w;
+    }
+    int4 e = make_int4(0, 0, 0, 0);
+    if (live) {
+      const int4 x = __ldg(units + (size_t)bg * umax + local);
       const int b = bg / d.Hkv;
-      e = make_int4((b << 20) | ((bg - b * d.Hkv) << 13) | x.x, x.y, x.z, U);
+      e = make_int4((b << 20) | ((bg - b * d.Hkv) << 13) | x.x, x.y, x.z, 0);
     }
     us[k] = e;
   }
@@ -673,7 +764,7 @@ BmCarve bm_carve(const Dims& d) {
   c.cursor = take(bg * d.Nb * 4);
   c.list = take(bg * d.Tq * d.topk * 4);
   c.units = take(bg * units_per_group(d) * sizeof(int4));
-  c.ucount = take(bg * 4);
+  c.ucount = take(bg * sizeof(int4));  // four unit-class sizes per (sequence, group)
   c.part_o = take(slots * 64 * 2);
   c.part_lse = take(slots * 4);
   c.total = at;
@@ -725,7 +816,7 @@ cudaError_t launch_sel_bm(const Dims& d, const void* q, const void* k, const voi
   const int umax = units_per_group(d);
   cudaError_t e = launch_revmap_units(d, idx, (int*)(w + c.chunk), (int*)(w + c.offsets),
                                       (int*)(w + c.cursor), list, units, ucount,
-                                      kSeg * tile_tokens(d.G), umax, err, s);
+                                      kSeg * tile_tokens(d.G), tile_tokens(d.G), umax, err, s);
   if (e != cudaSuccess) return e;
   CUtensorMap mk, mv;
   if (!make_tmap_bf16(&mk, k, d.Hkv, (long)d.B * d.T, 1, kKeys) ||
