@@ -216,3 +216,22 @@ def test_kernel_event_hook_times_the_kernel(cuda_lib):
     torch.cuda.synchronize()
     assert 0.0 < a.elapsed_time(b) < 1000.0
     assert_close(to_np(o), r["o_sel"], TOL[w.dtype], "o_sel")
+
+
+@pytest.mark.parametrize("w", [
+    # 576 (sequence, group) pairs: the units are dealt by size, two groups per
+    # scanning thread
+    small("dealt_b9_mha64_t200_k3", B=9, T=200, Hq=64, Hkv=64, topk=3),
+    # 1040 pairs, beyond the groups whose units are dealt by size: round-robin slots
+    small("roundrobin_b260_g2_t130_k2", B=260, T=130, Hq=8, Hkv=4, topk=2, window=64),
+], ids=lambda w: w.name)
+def test_sel_bm_many_groups(cuda_lib, w):
+    inp = W.make_inputs(w, seed=31)
+    rng = np.random.default_rng(32)
+    idx = random_idx(w, rng)
+    o_ref, lse_ref = orc.sel_attn_fwd(ocfg(w), inp["q"], inp["k"], inp["v"], idx)
+    q, k, v = (inp[n].to(DEV) for n in ("q", "k", "v"))
+    o, lse = run_ws(w, q, k, v, torch.from_numpy(idx).to(DEV))
+    assert nsa.nsa_last_device_error() == 0
+    assert_close(to_np(o), o_ref, TOL[w.dtype], "o_sel")
+    assert_close(to_np(lse), lse_ref, LSE_TOL[w.dtype], "lse_sel")
