@@ -33,9 +33,11 @@
  *     visible block gets output 0, lse -inf, no gradient      [orc_cmp_row]
  *   - compression is the plain mean of the raw rows           [orc_compress]
  *   - block importance = compression softmax probabilities summed over the
- *     query heads of one KV group; compression and selection share the
- *     block geometry (l = d = selection block), so compressed block j
- *     scores selection block j                                 [orc_scores]
+ *     query heads of one KV group                              [orc_scores]
+ *   - a selection block's importance is the sum of the importances of the
+ *     compressed blocks whose tokens overlap it: compressed block i covers
+ *     [i*d, i*d + l), selection block j covers [j*l', (j+1)*l'); with
+ *     l = d = l' that is compressed block j alone              [orc_topk_row]
  *   - block 0 and the query's own block are always selected and count
  *     toward topk; if a query has at most topk causal blocks it takes all
  *     of them; ties go to the lower block index; the list is ascending and
@@ -258,7 +260,7 @@ static void orc_scores_token(const orc_cfg* c, const double* q_tok,
 /* (always include the first block); "DeepSeek's Native Sparse         */
 /* Attention", SELECTION.                                              */
 /* ------------------------------------------------------------------ */
-static void orc_topk_row(const orc_cfg* c, const double* score_row, int t,
+static void orc_topk_row(const orc_cfg* c, const double* cmp_score_row, int t,
                          int* idx_row) {
   const int n = c->topk;
   const int cur = t / c->sel_block;
@@ -266,6 +268,19 @@ static void orc_topk_row(const orc_cfg* c, const double* score_row, int t,
   if (cur + 1 <= n) { /* all causal blocks fit */
     for (int j = 0; j <= cur; ++j) idx_row[j] = j;
     return;
+  }
+  /* selection-block importances from the compressed blocks that overlap
+     each selection block (blocks not yet complete have importance 0) */
+  const int nc = orc_num_cmp_blocks(c);
+  double* score_row = (double*)malloc(sizeof(double) * (size_t)(cur + 1));
+  for (int j = 0; j <= cur; ++j) {
+    const long lo = (long)j * c->sel_block, hi = lo + c->sel_block; /* [lo, hi) */
+    double acc = 0.0;
+    for (int i = 0; i < nc; ++i) {
+      const long clo = (long)i * c->cmp_stride, chi = clo + c->cmp_block;
+      if (clo < hi && chi > lo) acc += cmp_score_row[i];
+    }
+    score_row[j] = acc;
   }
   /* rank the non-forced causal blocks 1..cur-1 by (score desc, index asc)
      with a plain selection sort; keep the first n-2. */
@@ -294,6 +309,7 @@ static void orc_topk_row(const orc_cfg* c, const double* score_row, int t,
       idx_row[r - 1] = tmp;
     }
   free(cand);
+  free(score_row);
 }
 
 /* key positions attended by the selection branch at query t */

@@ -200,6 +200,70 @@ def test_topk_brute_force():
                 assert idx[b, t, h].tolist() == want
 
 
+# Compression and selection with different block geometry (compressed
+# blocks of l tokens every d tokens, selection blocks of l' tokens): a
+# selection block's importance is the sum over the compressed blocks whose
+# tokens overlap it.
+@pytest.mark.parametrize("l,d,ls", [(4, 2, 8), (8, 8, 16), (6, 4, 8), (4, 2, 4)])
+def test_topk_general_geometry_brute_force(l, d, ls):
+    """Overlap written as a token-set intersection, ranking as in the
+    equal-geometry brute force."""
+    c = cfg_small(T=96, cmp_block=l, cmp_stride=d, sel_block=ls, topk=4, Hkv=2)
+    g = np.random.default_rng(7)
+    score = np.round(g.random((c.B, c.T, c.Hkv, c.Nc)) * 20) / 20  # ties occur
+    idx = orc.select_topk(c, score)
+    cmp_tokens = [set(range(i * d, i * d + l)) for i in range(c.Nc)]
+    for b in range(c.B):
+        for t in range(c.T):
+            for h in range(c.Hkv):
+                cur = t // ls
+                if cur + 1 <= c.topk:
+                    want = list(range(cur + 1)) + [-1] * (c.topk - cur - 1)
+                else:
+                    sel = [sum(score[b, t, h, i] for i in range(c.Nc)
+                               if cmp_tokens[i] & set(range(j * ls, (j + 1) * ls)))
+                           for j in range(cur + 1)]
+                    cands = sorted(range(1, cur), key=lambda j: (-sel[j], j))
+                    want = sorted([0, cur] + cands[:c.topk - 2])
+                assert idx[b, t, h].tolist() == want, (b, t, h)
+
+
+def test_topk_general_geometry_hand_cases():
+    """Hand-derived: with l = 4, d = 2 a compressed block i covers tokens
+    [2i, 2i + 4), so for selection blocks of 4 tokens block j collects the
+    compressed blocks 2j - 1, 2j and 2j + 1; a lone importance on an odd
+    compressed block 2m + 1 lifts selection blocks m and m + 1 alike (the
+    tie goes to m).  With l = d = 4 and selection blocks of 8 tokens, block j
+    collects compressed blocks 2j and 2j + 1."""
+    c = cfg_small(B=1, T=64, Hkv=1, Hq=1, cmp_block=4, cmp_stride=2, sel_block=4, topk=3)
+    t = 63  # cur = 15: candidates 1 .. 14, one winner besides 0 and 15
+    score = np.zeros((1, c.T, 1, c.Nc))
+    score[0, t, 0, 2 * 6 + 1] = 1.0  # blocks 6 and 7 tie: 6 wins
+    assert orc.select_topk(c, score)[0, t, 0].tolist() == [0, 6, 15]
+    score[0, t, 0, 2 * 7] = 0.5      # block 7 alone gets 1.5 (13 and 14)
+    assert orc.select_topk(c, score)[0, t, 0].tolist() == [0, 7, 15]
+    c2 = cfg_small(B=1, T=64, Hkv=1, Hq=1, cmp_block=4, cmp_stride=4, sel_block=8, topk=3)
+    t = 63  # cur = 7
+    score = np.zeros((1, c2.T, 1, c2.Nc))
+    score[0, t, 0, 2 * 3] = 0.6       # selection block 3: 0.6 + 0.0
+    score[0, t, 0, 2 * 5 + 1] = 0.4   # block 5: 0.0 + 0.4 + the next one
+    score[0, t, 0, 2 * 5] = 0.3       #          = 0.7 > 0.6
+    assert orc.select_topk(c2, score)[0, t, 0].tolist() == [0, 5, 7]
+
+
+def test_forward_general_geometry_selection_and_compression():
+    """With every selection block selected the selection branch is dense
+    causal attention whatever the scores; with l = d = 1 the compression
+    branch is dense causal attention (selection blocks of 4 tokens)."""
+    c = cfg_small(T=48, Hq=4, Hkv=2, cmp_block=1, cmp_stride=1, sel_block=4, topk=12,
+                  branch_mask=orc.BR_ALL)
+    q, k, v = qkv(c, 61)
+    r = orc.forward(c, q, k, v, rand((c.B, c.T, c.Hq, 3), 62))
+    o_ref, lse_ref = sdpa(q, k, v, causal(c.T), 1 / math.sqrt(c.D))
+    np.testing.assert_allclose(r["o_sel"], o_ref, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(r["o_cmp"], o_ref, rtol=0, atol=1e-12)
+
+
 # ---------------------------------------------------------------- sel branch
 def test_sel_covering_every_block_is_full_causal_attention():
     c = cfg_small(T=64, sel_block=8, topk=8)  # 8 blocks, all selected
