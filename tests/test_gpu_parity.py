@@ -324,7 +324,12 @@ def sample_rows(w, n, seed):
 
 @pytest.mark.parametrize("w", [W.NSA_340M, W.PRUNED_32K, W.NSA_1P3B,
                                # 625 selection blocks: the 32-slot-per-lane top-k
-                               W.NSA_340M.replace(name="gqa4_t40000_nb625", T=40000)],
+                               W.NSA_340M.replace(name="gqa4_t40000_nb625", T=40000),
+                               # the limits: 1024 blocks per sequence, top-k 64 (the
+                               # block-major path's 6-bit slot numbers), 32 heads a group
+                               W.NSA_340M.replace(name="gqa4_t65536_nb1024", T=65536),
+                               W.PRUNED_32K.replace(name="mqa_t32768_k64", topk=64),
+                               W.NSA_340M.replace(name="mqa_g32_t8192", Hq=32, Hkv=1)],
                          ids=lambda w: w.name)
 def test_forward_full_size_sampled(cuda_lib, w):
     inp = W.make_inputs(w, seed=0)
