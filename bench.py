@@ -357,17 +357,14 @@ def run_gpu(args, rank: int, world: int, dist_on: bool) -> None:
     sel_tflops = flops["sel"] / (sel_ms * 1e-3) / 1e12
     sel_exec_flops = executed_sel_flops(w, saved["idx"])
 
-    # end to end through the C ABI with host buffers (pinned), copies timed
+    # end to end through the C ABI with host buffers (pinned): nsa_forward_host
+    # copies the inputs in, runs the forward and copies out back, all timed
     hq, hk, hv, hg = (x.cpu().pin_memory() for x in (q, k, v, g))
     hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    hws = torch.empty(nsa.nsa_forward_host_workspace_size(p), dtype=torch.uint8, device=dev)
 
     def e2e_step():
-        q.copy_(hq, non_blocking=True)
-        k.copy_(hk, non_blocking=True)
-        v.copy_(hv, non_blocking=True)
-        g.copy_(hg, non_blocking=True)
-        step()
-        hout.copy_(out, non_blocking=True)
+        nsa.nsa_forward_host(p, hq, hk, hv, hg, hout, hws, stream)
 
     for _ in range(2):
         e2e_step()
@@ -376,7 +373,7 @@ def run_gpu(args, rank: int, world: int, dist_on: bool) -> None:
     h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hg))
     d2h = hout.numel() * hout.element_size()
 
-    del hq, hk, hv, hg, hout
+    del hq, hk, hv, hg, hout, hws
     if args.leg == "forward":  # the forward alone (for profiling it)
         sampler.__exit__(None, None, None)
         print(json.dumps({"forward": {"ms_per_step": ms, "tokens_per_s": value,

@@ -229,6 +229,23 @@ nsa_status nsa_forward(const nsa_params* p, const void* q, const void* k,
                        const nsa_saved* saved, void* workspace,
                        size_t workspace_bytes, void* stream);
 
+/* ---- whole forward from host memory ------------------------------------------
+ * nsa_forward for a caller whose q, k, v, gates and out live in host memory
+ * (same layouts): on `stream`, one host-to-device copy per input into the
+ * workspace, the forward, one device-to-host copy of out.  The call returns
+ * once everything is enqueued; out is valid after the stream has been
+ * synchronised, and the host buffers must stay untouched until then.  Page-
+ * locked host memory makes the copies asynchronous (pageable memory works,
+ * with copies staged by the driver).  workspace is device memory of at least
+ * nsa_forward_host_workspace_size(p) bytes, 256-byte aligned: the device
+ * copies of the five tensors, then nsa_forward's own workspace.  Errors as
+ * nsa_forward, plus NSA_ERR_INVALID_ARG for a NULL host pointer and
+ * NSA_ERR_CUDA if a copy cannot be enqueued. */
+nsa_status nsa_forward_host_workspace_size(const nsa_params* p, size_t* bytes);
+nsa_status nsa_forward_host(const nsa_params* p, const void* q, const void* k,
+                            const void* v, const float* gates, void* out,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
 /* ---- decode ----------------------------------------------------------------
  * One query per sequence at position T-1 (p->Tq must be 1) against caches
  * k_cache/v_cache [B, T, Hkv, D] that already hold that position, and the

@@ -11,6 +11,7 @@ from .abi import (EXPORTS, backward, nsa_backward, nsa_backward_workspace_size,
                   nsa_cmp_bwd, nsa_gate_combine_bwd, nsa_sel_attn_bwd, nsa_swa_bwd, NSA_BF16, NSA_BRANCH_ALL, NSA_BRANCH_CMP, NSA_BRANCH_SEL,
                   NSA_BRANCH_SWA, NSA_F32, NsaError, Params, Saved, alloc_workspace,
                   forward, load, make_params, nsa_check_params, nsa_cmp_attn_scores,
+                  nsa_forward_host, nsa_forward_host_workspace_size,
                   nsa_compress, nsa_decode, nsa_decode_noalloc,
                   nsa_decode_noalloc_max_scratch, nsa_forward, nsa_gate_combine,
                   nsa_last_device_error, nsa_sel_attn_fwd, nsa_sel_attn_fwd_ws,

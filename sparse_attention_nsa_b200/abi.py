@@ -32,7 +32,8 @@ EXPORTS = ("nsa_status_string", "nsa_check_params", "nsa_workspace_size",
            "nsa_forward", "nsa_decode", "nsa_backward_workspace_size",
            "nsa_gate_combine_bwd", "nsa_sel_attn_bwd", "nsa_swa_bwd", "nsa_cmp_bwd",
            "nsa_backward", "nsa_decode_noalloc", "nsa_decode_noalloc_max_scratch",
-           "nsa_sel_workspace_size", "nsa_sel_attn_fwd_ws", "nsa_set_kernel_events")
+           "nsa_sel_workspace_size", "nsa_sel_attn_fwd_ws", "nsa_set_kernel_events",
+           "nsa_forward_host_workspace_size", "nsa_forward_host")
 
 
 class NsaError(RuntimeError):
@@ -96,6 +97,8 @@ def load():
             "nsa_forward": ([P, vp, vp, vp, vp, vp, C.POINTER(Saved), vp, C.c_size_t, vp],
                             C.c_int),
             "nsa_decode": ([P, vp, vp, vp, vp, vp, vp, vp, vp, vp, C.c_size_t, vp], C.c_int),
+            "nsa_forward_host_workspace_size": ([P, C.POINTER(C.c_size_t)], C.c_int),
+            "nsa_forward_host": ([P, vp, vp, vp, vp, vp, vp, C.c_size_t, vp], C.c_int),
             "nsa_decode_noalloc": ([P, vp, vp, vp, vp, vp, vp, vp, vp, vp], C.c_int),
             "nsa_backward_workspace_size": ([P, C.POINTER(C.c_size_t)], C.c_int),
             "nsa_gate_combine_bwd": ([P] + [vp] * 10, C.c_int),
@@ -291,6 +294,39 @@ def nsa_forward(p: Params, q, k, v, gates, out, saved: dict | None = None,
         C.byref(p), _ptr(q, s["q"], dt, "q"), _ptr(k, s["k"], dt, "k"), _ptr(v, s["k"], dt, "v"),
         _ptr(gates, s["gates"], torch.float32, "gates"), _ptr(out, s["o"], dt, "out"),
         C.byref(sv), ws_ptr, ws_bytes, _stream(stream)), "nsa_forward")
+
+
+def _host_ptr(t, shape, dtype, name):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch tensor")
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host (CPU) tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return C.c_void_p(t.data_ptr())
+
+
+def nsa_forward_host_workspace_size(p: Params) -> int:
+    n = C.c_size_t(0)
+    _check(load().nsa_forward_host_workspace_size(C.byref(p), C.byref(n)),
+           "nsa_forward_host_workspace_size")
+    return n.value
+
+
+def nsa_forward_host(p: Params, q, k, v, gates, out, workspace, stream=None):
+    """nsa_forward on host (CPU, ideally pinned) tensors: the library copies
+    them in, runs the forward and copies out back, all enqueued on the
+    stream; out is valid once the stream has been synchronised."""
+    s, dt = _shapes(p), p.torch_dtype
+    _check(load().nsa_forward_host(
+        C.byref(p), _host_ptr(q, s["q"], dt, "q"), _host_ptr(k, s["k"], dt, "k"),
+        _host_ptr(v, s["k"], dt, "v"), _host_ptr(gates, s["gates"], torch.float32, "gates"),
+        _host_ptr(out, s["o"], dt, "out"), _ptr(workspace, name="workspace"),
+        workspace.numel() * workspace.element_size(), _stream(stream)), "nsa_forward_host")
 
 
 def nsa_decode(p: Params, q, k_cache, v_cache, kc_cache, vc_cache, gates, out,

@@ -455,6 +455,76 @@ nsa_status nsa_forward(const nsa_params* p, const void* q, const void* k, const 
                      (cudaStream_t)stream);
 }
 
+}  // extern "C"
+
+namespace {
+// device copies of nsa_forward_host's inputs and output, then the forward's
+// own workspace, each 256-byte aligned
+struct HostCarve {
+  size_t q, k, v, gates, out, fwd, total, qb, kb, gb;
+};
+HostCarve host_carve(const Dims& d, size_t fwd_bytes) {
+  HostCarve c{};
+  const size_t es = d.dtype == 1 ? 2 : 4;
+  c.qb = (size_t)d.B * d.Tq * d.Hq * d.D * es;   // q and out
+  c.kb = (size_t)d.B * d.T * d.Hkv * d.D * es;   // k and v
+  c.gb = (size_t)d.B * d.Tq * d.Hq * 3 * sizeof(float);
+  size_t at = 0;
+  auto take = [&](size_t b) {
+    const size_t o = at;
+    at += align256(b);
+    return o;
+  };
+  c.q = take(c.qb);
+  c.k = take(c.kb);
+  c.v = take(c.kb);
+  c.gates = take(c.gb);
+  c.out = take(c.qb);
+  c.fwd = take(fwd_bytes);
+  c.total = at;
+  return c;
+}
+}  // namespace
+
+extern "C" {
+
+nsa_status nsa_forward_host_workspace_size(const nsa_params* p, size_t* bytes) {
+  if (!bytes) return NSA_ERR_INVALID_ARG;
+  size_t fwd = 0;
+  nsa_status st = nsa_workspace_size(p, &fwd);
+  if (st != NSA_OK) return st;
+  Dims d;
+  fill_dims(p, &d);
+  *bytes = host_carve(d, fwd).total;
+  return NSA_OK;
+}
+
+nsa_status nsa_forward_host(const nsa_params* p, const void* q, const void* k, const void* v,
+                            const float* gates, void* out, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  Dims d;
+  nsa_status st = fill_dims(p, &d);
+  if (st != NSA_OK) return st;
+  if (!q || !k || !v || !gates || !out) return NSA_ERR_INVALID_ARG;
+  size_t fwd = 0;
+  if ((st = nsa_workspace_size(p, &fwd)) != NSA_OK) return st;
+  const HostCarve c = host_carve(d, fwd);
+  if (!workspace || workspace_bytes < c.total || (((uintptr_t)workspace) & 255u) != 0)
+    return NSA_ERR_WORKSPACE;
+  char* w = (char*)workspace;
+  const cudaStream_t s = (cudaStream_t)stream;
+  // one copy per tensor, in order on the caller's stream
+  NSA_TRY_CUDA(cudaMemcpyAsync(w + c.q, q, c.qb, cudaMemcpyHostToDevice, s));
+  NSA_TRY_CUDA(cudaMemcpyAsync(w + c.k, k, c.kb, cudaMemcpyHostToDevice, s));
+  NSA_TRY_CUDA(cudaMemcpyAsync(w + c.v, v, c.kb, cudaMemcpyHostToDevice, s));
+  NSA_TRY_CUDA(cudaMemcpyAsync(w + c.gates, gates, c.gb, cudaMemcpyHostToDevice, s));
+  st = run_forward(d, w + c.q, w + c.k, w + c.v, false, (const float*)(w + c.gates), w + c.out,
+                   nullptr, w + c.fwd, workspace_bytes - c.fwd, s);
+  if (st != NSA_OK) return st;
+  NSA_TRY_CUDA(cudaMemcpyAsync(out, w + c.out, c.qb, cudaMemcpyDeviceToHost, s));
+  return NSA_OK;
+}
+
 nsa_status nsa_decode(const nsa_params* p, const void* q, const void* k_cache,
                       const void* v_cache, const void* kc_cache, const void* vc_cache,
                       const float* gates, void* out, int32_t* idx_out, void* workspace,

@@ -97,3 +97,25 @@ def test_kernel_event_hook_arguments():
     assert lib.nsa_set_kernel_events(C.c_void_p(64), None) == 1  # NSA_ERR_INVALID_ARG
     assert lib.nsa_set_kernel_events(None, C.c_void_p(64)) == 1
     assert lib.nsa_set_kernel_events(None, None) == 0
+
+
+def test_forward_host_workspace_and_argument_checks():
+    """The host-buffer forward needs nsa_forward's workspace plus device room
+    for q, k, v, gates and out; NULL host pointers and a missing workspace
+    are rejected before anything is enqueued."""
+    p = nsa.make_params(2, 1000, 16, 4, topk=5, window=200)
+    fwd = nsa.nsa_workspace_size(p)
+    need = nsa.nsa_forward_host_workspace_size(p)
+    al = lambda n: (n + 255) // 256 * 256
+    tens = 2 * al(2 * 1000 * 16 * 64 * 2) + 2 * al(2 * 1000 * 4 * 64 * 2) + al(2 * 1000 * 16 * 3 * 4)
+    assert need == tens + al(fwd)
+    lib = nsa.load()
+    host = C.c_void_p(4096)  # never dereferenced: the checks come first
+    assert lib.nsa_forward_host(C.byref(p), None, host, host, host, host, host, need, None) == 1
+    assert lib.nsa_forward_host(C.byref(p), host, host, host, host, None, host, need, None) == 1
+    assert lib.nsa_forward_host(C.byref(p), host, host, host, host, host, None, need, None) == 6
+    assert lib.nsa_forward_host(C.byref(p), host, host, host, host, host, host, need - 1,
+                                None) == 6  # NSA_ERR_WORKSPACE
+    bad = nsa.make_params(2, 1000, 16, 4, scale=-1.0)
+    assert lib.nsa_forward_host(C.byref(bad), host, host, host, host, host, host, need,
+                                None) == 1

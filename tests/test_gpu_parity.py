@@ -356,3 +356,23 @@ def test_decode_full_size_sampled(cuda_lib):
     w = W.DECODE_32K
     inp = W.make_decode_inputs(w, seed=0)
     check_decode(w, inp, [0, 17, 42, 63])
+
+
+@pytest.mark.parametrize("w", [small("host_fwd_gqa4_t1000", T=1000, topk=5, window=200),
+                               small("host_fwd_bm_t4200_k4", T=4200, topk=4, window=150)],
+                         ids=lambda w: w.name)
+def test_forward_host_buffers_match_device_forward(cuda_lib, w):
+    """nsa_forward_host (pinned host tensors in and out) gives the device
+    forward's output bit for bit."""
+    inp = W.make_inputs(w, seed=33)
+    p = nsa.params_for(w)
+    d = {n: inp[n].to(DEV) for n in ("q", "k", "v", "gates")}
+    out_d = torch.empty_like(d["q"])
+    nsa.nsa_forward(p, d["q"], d["k"], d["v"], d["gates"], out_d, None, nsa.alloc_workspace(p))
+    h = {n: inp[n].contiguous().pin_memory() for n in ("q", "k", "v", "gates")}
+    out_h = torch.full(tuple(out_d.shape), float("nan"), dtype=out_d.dtype).pin_memory()
+    ws = torch.empty(nsa.nsa_forward_host_workspace_size(p), dtype=torch.uint8, device=DEV)
+    nsa.nsa_forward_host(p, h["q"], h["k"], h["v"], h["gates"], out_h, ws)
+    torch.cuda.synchronize()
+    assert nsa.nsa_last_device_error() == 0
+    assert torch.equal(out_h, out_d.cpu())
