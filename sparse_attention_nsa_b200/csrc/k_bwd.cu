@@ -694,7 +694,8 @@ cudaError_t launch_revmap_units(const Dims& d, const int32_t* idx, int* chunk, i
   // per-(sequence, group, block) totals (chunk holds them: B * Hkv * Nb ints)
   cudaError_t e = cudaMemsetAsync(chunk, 0, (size_t)d.B * d.Hkv * nb_bytes, s);
   if (e != cudaSuccess) return e;
-  rev_chunk_count_kernel<<<dim3(nchunk, d.Hkv, d.B), kRevChunk, nb_bytes, s>>>(idx, chunk, d,
+  // with totals given the count kernel writes only them (its chunk output is unused)
+  rev_chunk_count_kernel<<<dim3(nchunk, d.Hkv, d.B), kRevChunk, nb_bytes, s>>>(idx, nullptr, d,
                                                                               err, chunk);
   rev_chunk_scan_kernel<<<d.B * d.Hkv, 1024, (kMaxUnitClasses + 1) * nb_bytes + sizeof(int), s>>>(
       chunk, offsets, d, 1, units, ucount, cursor, tpu, tq, umax);

@@ -493,8 +493,8 @@ nsa_status nsa_forward_host_workspace_size(const nsa_params* p, size_t* bytes) {
   size_t fwd = 0;
   nsa_status st = nsa_workspace_size(p, &fwd);
   if (st != NSA_OK) return st;
-  Dims d;
-  fill_dims(p, &d);
+  Dims d{};
+  if ((st = fill_dims(p, &d)) != NSA_OK) return st;
   *bytes = host_carve(d, fwd).total;
   return NSA_OK;
 }
