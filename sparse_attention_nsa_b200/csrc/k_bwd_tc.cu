@@ -872,8 +872,9 @@ cudaError_t launch_dq_tc_t(const Dims& d, const void* q, const void* k, const vo
 
 }  // namespace
 
-// Tensor-core dQ applies to bf16, 64-key blocks, head dim 64, G dividing 128.
-bool dq_tc_eligible(const Dims& d, int mode) {
+// Tensor-core dQ applies to bf16, 64-key blocks, head dim 64, G dividing 128,
+// for every branch alike.
+bool dq_tc_eligible(const Dims& d, int /*mode*/) {
   return d.dtype == 1 && d.l == kKeys && d.D == 64 && d.G >= 1 && kRows % d.G == 0 &&
          d.Nb <= 4096 && tmap_encode_fn() != nullptr;
 }
