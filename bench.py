@@ -39,7 +39,17 @@ from sparse_attention_nsa_b200 import inputs as W  # noqa: E402
 METRIC = "NSA fwd tokens/s & TFLOP/s (frac of bf16 peak) @8192 GQA-4; decode HBM GB/s"
 WORK = W.NSA_340M
 DECODE = W.DECODE_32K
-KERNELS_PER_FORWARD = 5  # compress, cmp+scores, top-k, window (side stream), selection+combine
+
+
+def kernels_per_forward(w) -> int:
+    """Kernels one nsa_forward of workload w launches (as its ncu launch list
+    shows): pooling, compression branch + scores, top-k, window (side
+    stream), then either the query-tiled selection with the combination, or
+    (block-major, from Nb >= 8 top-k and Tq >= 64) the reverse map's count,
+    scan and fill, the selection kernel and the merge with the combination."""
+    nb = -(-w.T // w.sel_block)
+    block_major = w.dtype == torch.bfloat16 and nb >= 8 * w.topk and w.T >= 64
+    return 4 + (5 if block_major else 1)
 
 
 # ------------------------------------------------------------------ work model
@@ -430,7 +440,7 @@ def run_gpu(args, rank: int, world: int, dist_on: bool) -> None:
         "long_context": long_ctx,
         "e2e": {"value": job_tokens_per_s(tokens_per_step, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": KERNELS_PER_FORWARD * args.steps,
+        "gpu_launches": kernels_per_forward(w) * args.steps,
         "clocks": clocks,
     }
     if world == 1 and not args.no_cpu_baseline:
