@@ -7,7 +7,9 @@ sliding window, gated combination) over the 340M-shape workload: B=1,
 T=8192, 16 query heads, 4 KV heads (GQA-4), head dim 64, block 64, top-k 16,
 window 512, bf16, with inputs resident in HBM.  L2 is flushed (256 MiB
 write) between timed steps; each step is timed with CUDA events on the
-launching stream.  Rank 0 prints one JSON line.
+launching stream.  Rank 0 prints one JSON line.  Its `e2e` figure times the
+same forward through nsa_forward_host from page-locked host buffers, the
+copies in and out inside each timed step.
 
 With N > 1 (torchrun), every rank runs its own independent copy of the
 workload (NSA has no cross-sequence exchange: weak scaling, no data-path
