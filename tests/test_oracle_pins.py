@@ -411,8 +411,10 @@ def test_forward_rows_matches_forward():
             np.testing.assert_array_equal(s[key][i], r[key][b, t])
 
 
-def test_decode_is_last_row_of_forward():
-    c = cfg_small(B=3, T=48)
+@pytest.mark.parametrize("geom", [dict(), dict(cmp_block=4, cmp_stride=2, sel_block=8, T=50)],
+                         ids=["equal_blocks", "overlapping_cmp_blocks"])
+def test_decode_is_last_row_of_forward(geom):
+    c = cfg_small(**{"B": 3, "T": 48, **geom})
     q, k, v = qkv(c, 97)
     gates = np.random.default_rng(8).random((c.B, c.T, c.Hq, 3))
     r = orc.forward(c, q, k, v, gates)
