@@ -445,6 +445,10 @@ def _loss(c, q, k, v, gates, dout):
          topk=3, window=4),
     dict(B=2, T=12, Hq=4, Hkv=2, D=3, cmp_block=3, cmp_stride=3, sel_block=3,
          topk=2, window=5),
+    # overlapping compressed blocks (a token in two of them), selection blocks
+    # of another size: the pooling backward spreads over both blocks
+    dict(B=1, T=16, Hq=2, Hkv=1, D=3, cmp_block=4, cmp_stride=2, sel_block=4,
+         topk=2, window=5),
 ])
 def test_backward_matches_central_differences(shape):
     c = orc.Cfg(**shape)
