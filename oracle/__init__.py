@@ -35,7 +35,7 @@ class _CCfg(C.Structure):
                 ("cmp_stride", C.c_int), ("sel_block", C.c_int),
                 ("topk", C.c_int), ("window", C.c_int),
                 ("scale", C.c_double), ("kv_round", C.c_int),
-                ("branch_mask", C.c_int)]
+                ("branch_mask", C.c_int), ("o_round", C.c_int)]
 
 
 @dataclasses.dataclass
@@ -54,12 +54,13 @@ class Cfg:
     scale: float | None = None
     kv_round: int = KV_KEEP
     branch_mask: int = BR_ALL
+    o_round: int = KV_KEEP  # precision of the stored branch outputs the gate gradient reads
 
     def c(self) -> _CCfg:
         s = self.scale if self.scale is not None else 1.0 / math.sqrt(self.D)
         return _CCfg(self.B, self.T, self.Hq, self.Hkv, self.D, self.cmp_block,
                      self.cmp_stride, self.sel_block, self.topk, self.window,
-                     float(s), self.kv_round, self.branch_mask)
+                     float(s), self.kv_round, self.branch_mask, self.o_round)
 
     @property
     def Nc(self) -> int:

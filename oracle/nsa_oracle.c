@@ -50,6 +50,10 @@
  *   - in a low-precision path the compressed keys/values are stored in that
  *     precision (round-to-nearest-even) before anything reads them, so the
  *     oracle rounds them the same way when asked              [orc_compress]
+ *   - likewise the three branch outputs are stored in the path's precision
+ *     and the gate gradient dL/dg_i = dO . o_i reads the stored values; the
+ *     oracle rounds o_i the same way when asked (the other gradients use
+ *     the exact outputs)                                      [orc_backward]
  */
 #include <math.h>
 #include <stdint.h>
@@ -66,6 +70,9 @@ typedef struct {
   double scale;    /* softmax scale                               */
   int kv_round;    /* 0 keep fp64, 1 round kc/vc to fp32, 2 to bf16 */
   int branch_mask; /* bit 0 cmp, bit 1 sel, bit 2 swa              */
+  int o_round;     /* 0 keep fp64, 1 fp32, 2 bf16: precision in which the
+                      branch outputs are stored before the gate gradient
+                      reads them (orc_backward only)                 */
 } orc_cfg;
 
 #define ORC_CMP 1
@@ -698,6 +705,12 @@ void orc_backward(const orc_cfg* c, const double* q, const double* k,
   double* dOb = (double*)malloc(3 * nq * sizeof(double));
   orc_forward(c, q, k, v, gates, kc, vc, o_cmp, lse, score, idx, o_sel,
               lse + nr, o_swa, lse + 2 * nr, out);
+  /* the gate gradient reads the branch outputs as stored (reading R15) */
+  for (size_t i = 0; i < nq; ++i) {
+    o_cmp[i] = round_store(o_cmp[i], c->o_round);
+    o_sel[i] = round_store(o_sel[i], c->o_round);
+    o_swa[i] = round_store(o_swa[i], c->o_round);
+  }
   orc_gate_combine_bwd(c, gates, dout, o_cmp, o_sel, o_swa, dgates, dOb,
                        dOb + nq, dOb + 2 * nq);
   memset(dq, 0, nq * sizeof(double));

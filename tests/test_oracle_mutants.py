@@ -41,6 +41,8 @@ MUTANTS = {
     "softmax_scale_dropped": ("logit[s] = scale * dot(qrow, krows[s], D);",
                               "logit[s] = dot(qrow, krows[s], D);"),
     "bf16_round_truncates": ("double r = nearbyint(ldexp(m, 8));", "double r = trunc(ldexp(m, 8));"),
+    "gate_grad_reads_exact_outputs": ("    o_sel[i] = round_store(o_sel[i], c->o_round);\n",
+                                      "    o_sel[i] = o_sel[i];\n"),
     "remap_overlap_off_by_one": ("if (clo < hi && chi > lo) acc += cmp_score_row[i];",
                                  "if (clo <= hi && chi > lo) acc += cmp_score_row[i];"),
     "remap_first_block_only": ("if (clo < hi && chi > lo) acc += cmp_score_row[i];",

@@ -538,3 +538,49 @@ def test_backward_dq_rows_match_full_backward():
     got = orc.backward_dq_rows(c, q, k, v, gates, dout, rows)
     for i, (b, t) in enumerate(rows):
         np.testing.assert_allclose(got[i], dq[b, t], rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("mode", [orc.KV_BF16, orc.KV_F32])
+def test_backward_gate_gradient_reads_stored_outputs(mode):
+    """Reading R15: with the branch outputs stored in a lower precision, the
+    gate gradient is dout . o_i of the STORED o_i (rounded here by torch's
+    own cast, independent of the oracle's rounding), while dq, dk and dv
+    keep using the exact outputs."""
+    c = cfg_small(T=40)
+    q, k, v = qkv(c, 141)
+    g = np.random.default_rng(142)
+    gates = g.random((c.B, c.T, c.Hq, 3))
+    dout = g.standard_normal((c.B, c.T, c.Hq, c.D))
+    r = orc.forward(c, q, k, v, gates)
+    exact = orc.backward(c, q, k, v, gates, dout)
+    c.o_round = mode
+    stored = orc.backward(c, q, k, v, gates, dout)
+    to = torch.bfloat16 if mode == orc.KV_BF16 else torch.float32
+    for i, name in enumerate(("o_cmp", "o_sel", "o_swa")):
+        o_st = torch.from_numpy(r[name]).to(to).double().numpy()
+        np.testing.assert_allclose(stored[3][..., i], np.sum(dout * o_st, -1), rtol=0,
+                                   atol=1e-13)
+        if mode == orc.KV_BF16:  # the rounding must actually move dgates
+            assert np.abs(stored[3][..., i] - exact[3][..., i]).max() > 1e-6
+    for a, b in zip(stored[:3], exact[:3]):
+        np.testing.assert_array_equal(a, b)
+
+
+def test_backward_composed_on_own_selection_equals_backward():
+    """The GPU tests' composition of the oracle's branch backwards on a given
+    selection reproduces orc_backward exactly when given the oracle's own
+    selection (with the stored-output rounding of reading R15)."""
+    import torch as _t
+
+    from helpers import oracle_backward_given_idx
+    from sparse_attention_nsa_b200 import inputs as W
+    w = W.Workload("compose_check", B=2, T=40, Hq=4, Hkv=2, D=8, cmp_block=8, cmp_stride=8,
+                   sel_block=8, topk=3, window=12, dtype=_t.bfloat16)
+    inp = {n: x.double().numpy() for n, x in W.make_inputs(w, seed=151, with_dout=True).items()}
+    c = orc.Cfg(B=w.B, T=w.T, Hq=w.Hq, Hkv=w.Hkv, D=w.D, cmp_block=8, cmp_stride=8,
+                sel_block=8, topk=3, window=12, kv_round=orc.KV_BF16, o_round=orc.KV_BF16)
+    r = orc.forward(c, inp["q"], inp["k"], inp["v"], inp["gates"])
+    got = oracle_backward_given_idx(c, w, inp, inp["dout"], r["idx"])
+    want = orc.backward(c, inp["q"], inp["k"], inp["v"], inp["gates"], inp["dout"])
+    for a, b in zip(got, want):
+        np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
