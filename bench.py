@@ -104,22 +104,29 @@ def load_peaks() -> dict:
                 "source": "fallback"}
 
 
-def profiled_traffic(kernel_src: str, profile_md: str):
-    """DRAM bytes per launch recorded in a committed ncu summary, if that
-    summary was taken on the current source of the kernel (its sha1 prefix
-    matches); otherwise None (the counters are stale)."""
+def profiled_traffic(kernel_src: str, profile_json: str):
+    """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum)
+    recorded in a committed machine-readable ncu summary, if that summary was
+    taken on the current source of the kernel (its sha1 prefix matches);
+    otherwise None (the counters are stale)."""
     import hashlib
     try:
         sha = hashlib.sha1(open(os.path.join(ROOT, kernel_src), "rb").read()).hexdigest()[:12]
-        rec_sha, traffic = None, None
-        for line in open(os.path.join(ROOT, profile_md)):
-            if line.startswith("source-sha1:"):
-                rec_sha = line.split(":", 1)[1].strip()
-            if line.startswith("| dram_bytes_per_launch"):
-                traffic = int(line.split("|")[2].strip())
-        return traffic if rec_sha == sha else None
+        with open(os.path.join(ROOT, profile_json)) as f:
+            rec = json.load(f)
+        if rec.get("source_sha1") != sha:
+            return None
+        return int(rec["dram_bytes_per_launch"])
     except Exception:
         return None
+
+
+def sel_compulsory_bytes(w) -> int:
+    """HBM bytes the selection branch must move at the least: q, k, v and
+    the block indices read once; o_sel (path dtype) and lse_sel written."""
+    es = 2 if w.dtype == torch.bfloat16 else 4
+    return (w.B * w.T * w.Hq * w.D * es + 2 * w.B * w.T * w.Hkv * w.D * es
+            + w.B * w.T * w.Hkv * w.topk * 4 + w.B * w.T * w.Hq * w.D * es + w.B * w.T * w.Hq * 4)
 
 
 # ------------------------------------------------------------------ clocks
@@ -234,6 +241,23 @@ def sel_bm_algorithmic_bytes(w, idx) -> int:
     es = 2
     return (slots * G * (128 + 4) + slots * 4
             + w.B * w.T * w.Hq * w.D * es + 2 * w.B * w.T * w.Hkv * w.D * es)
+
+
+def roofline_line(kernel: str, flops: float, ms: float, peaks: dict, traffic, compulsory: int,
+                  design: dict | None = None) -> dict:
+    """Roofline record of a tensor-bound kernel: algorithmic TFLOP/s per
+    launch against the measured bf16 peak."""
+    achieved = flops / (ms * 1e-3) / 1e12
+    r = {"bound": "tensor", "kernel": kernel, "achieved": achieved,
+         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+         "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
+         "peak_source": f"{peaks['source']} bf16 dense GEMM (burst)",
+         "algorithmic_flops": flops, "ms_per_launch": ms,
+         "compulsory_bytes": compulsory,
+         "traffic_over_algorithmic": (traffic / compulsory) if traffic else None}
+    if design:
+        r["design_min_bytes"] = design
+    return r
 
 
 def barrier_sync(dist_on):
@@ -398,6 +422,8 @@ def run_gpu(args, rank: int, world: int, dist_on: bool) -> None:
     train = run_train(dev, flush, stream, max(3, args.steps // 4), peaks)
     # long context (32768 tokens, block-major selection)
     long_ctx = run_long(dev, flush, stream, max(3, args.steps // 4), peaks)
+    # the 1.3B-shape forward (B=4, GQA-4 with 8 KV heads)
+    onep3b = run_1p3b(dev, flush, stream, max(3, args.steps // 2), peaks)
     sampler.__exit__(None, None, None)
 
     barrier_sync(dist_on)
@@ -417,18 +443,22 @@ def run_gpu(args, rank: int, world: int, dist_on: bool) -> None:
         "frac_bf16_peak": flops["total"] / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
         "flops_per_step": flops,
         # dominant kernel of the timed forward: the block-major selection
-        # kernel; its design minimum is the HBM time of the per-(row, slot)
-        # partials it must write plus its compulsory reads (46 us here) against
-        # 19 us of tensor time, so it is rated against HBM bandwidth
-        "roofline": {"bound": "hbm", "kernel": "block-major selection (sel_bm_kernel)",
-                     "achieved": bm_bytes / (bm_ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
-                     "unit": "GB/s", "frac": bm_bytes / (bm_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                     "traffic": profiled_traffic("sparse_attention_nsa_b200/csrc/k_sel_bm.cu",
-                                                 "profiles/sel_bm_340m.md"),
-                     "algorithmic_bytes": bm_bytes, "ms_per_launch": bm_ms,
-                     "peak_source": peaks["source"] + " HBM copy",
-                     "tensor_tflops": flops["sel"] / (bm_ms * 1e-3) / 1e12,
-                     "tensor_frac": flops["sel"] / (bm_ms * 1e-3) / 1e12 / peaks["bf16_tflops"]},
+        # kernel, rated on the selection branch's algorithmic FLOPs (4 D per
+        # selected (query row, key)) against the measured bf16 peak (burst:
+        # the kernel is timed inside a 0.3 ms forward).  traffic is its ncu
+        # DRAM bytes per launch; traffic_over_algorithmic divides that by the
+        # branch's compulsory bytes (q, k, v, indices in; o_sel, lse out).
+        # The design's own minimum bytes (the per-(row, slot) partials it
+        # writes) are given as a labelled extra.
+        "roofline": roofline_line(
+            "block-major selection (sel_bm_kernel)", flops["sel"], bm_ms, peaks,
+            profiled_traffic("sparse_attention_nsa_b200/csrc/k_sel_bm.cu",
+                             "profiles/sel_bm_340m.json"),
+            sel_compulsory_bytes(w),
+            design={"bytes": bm_bytes, "what": "fp16 partial row + lse per used (row, slot), "
+                    "list entries, q/k/v once",
+                    "gbs": bm_bytes / (bm_ms * 1e-3) / 1e9,
+                    "frac_of_hbm": bm_bytes / (bm_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}),
         # context: the query-tiled selection kernel (the forward's path for
         # Nb < 8 top-k) on the same indices; on structure-free selections the
         # union of a tile's blocks is near dense, so it issues more MMA work
@@ -440,6 +470,7 @@ def run_gpu(args, rank: int, world: int, dist_on: bool) -> None:
         "decode": dec,
         "train": train,
         "long_context": long_ctx,
+        "nsa_1p3b": onep3b,
         "e2e": {"value": job_tokens_per_s(tokens_per_step, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": kernels_per_forward(w) * args.steps,
@@ -450,10 +481,11 @@ def run_gpu(args, rank: int, world: int, dist_on: bool) -> None:
     print(json.dumps(line), flush=True)
 
 
-def run_train(dev, flush, stream, steps, peaks) -> dict:
+def run_train(dev, flush, stream, steps, peaks, batch=None) -> dict:
     """One training step of attention: NSA forward (intermediates kept) and
-    the whole backward, B=8 x 8192 tokens, 340M shape."""
-    w = W.TRAIN_340M
+    the whole backward, B=8 x 8192 tokens, 340M shape (batch overrides B, to
+    profile a smaller case of the same kernels)."""
+    w = W.TRAIN_340M if batch is None else W.TRAIN_340M.replace(B=batch)
     inp = W.make_inputs(w, seed=1, with_dout=True)
     q, k, v, g, dout = (inp[n].to(dev) for n in ("q", "k", "v", "gates", "dout"))
     p = nsa.params_for(w)
@@ -490,6 +522,31 @@ def run_train(dev, flush, stream, steps, peaks) -> dict:
             "tokens_per_s": w.B * w.T / (step_ms * 1e-3),
             "tflops_fwd_plus_bwd": 3.5 * flops / (step_ms * 1e-3) / 1e12,
             "flops_note": "algorithmic: forward + backward counted as 2.5x forward"}
+
+
+def run_1p3b(dev, flush, stream, steps, peaks) -> dict:
+    """The 1.3B-shape forward: B=4 x 8192 tokens, 32 query heads on 8 KV
+    heads (GQA-4), block 64, top-k 16, window 512, bf16."""
+    w = W.NSA_1P3B
+    inp = W.make_inputs(w, seed=4)
+    q, k, v, g = (inp[n].to(dev) for n in ("q", "k", "v", "gates"))
+    p = nsa.params_for(w)
+    out = torch.empty_like(q)
+    ws = nsa.alloc_workspace(p, dev)
+
+    def fwd():
+        nsa.nsa_forward(p, q, k, v, g, out, None, ws)
+
+    for _ in range(3):
+        fwd()
+    ms = statistics.mean(timed_steps(fwd, steps, flush, stream))
+    if nsa.nsa_last_device_error() != 0:
+        raise RuntimeError("device-side check failed in the 1.3B-shape leg")
+    flops = fwd_flops(w)
+    tf = flops["total"] / (ms * 1e-3) / 1e12
+    return {"workload": w.name, "fwd_ms": ms, "tokens_per_s": w.B * w.T / (ms * 1e-3),
+            "tflops": tf, "frac_bf16_peak": tf / peaks["bf16_tflops"],
+            "flops_per_step": flops}
 
 
 def run_long(dev, flush, stream, steps, peaks) -> dict:
@@ -582,10 +639,13 @@ def main():
     ap.add_argument("--impl", default="nsa", choices=["nsa", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--leg", default="all",
-                    choices=["all", "forward", "decode", "train", "long"],
-                    help="forward / decode / train / long: run only that leg on one GPU "
+                    choices=["all", "forward", "decode", "train", "long", "onep3b"],
+                    help="forward / decode / train / long / onep3b: run only that leg on one GPU "
                          "and print its numbers (for profiling that leg alone); all: the "
                          "benchmark")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="--leg train only: batch size instead of 8 (a smaller case of the "
+                         "same kernels, for profiling)")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -603,8 +663,11 @@ def main():
             print(json.dumps({"decode": run_decode(dev, flush, stream, args.steps, peaks)}))
         elif args.leg == "long":
             print(json.dumps({"long_context": run_long(dev, flush, stream, args.steps, peaks)}))
+        elif args.leg == "onep3b":
+            print(json.dumps({"nsa_1p3b": run_1p3b(dev, flush, stream, args.steps, peaks)}))
         else:
-            print(json.dumps({"train": run_train(dev, flush, stream, args.steps, peaks)}))
+            print(json.dumps({"train": run_train(dev, flush, stream, args.steps, peaks,
+                                                 batch=args.batch)}))
         return
     dist_on = world > 1
     if dist_on:

@@ -223,7 +223,12 @@ nsa_status nsa_gate_combine(const nsa_params* p, const float* gates,
  * compression output is not.  With NSA_BRANCH_SEL off the selection path
  * (scores, top-k, selection) is skipped entirely, and so is the compression
  * branch if it is off too.  `saved` may be NULL.  workspace must hold at
- * least nsa_workspace_size(p) bytes (256-byte aligned). */
+ * least nsa_workspace_size(p) bytes (256-byte aligned).
+ * Passage: "DeepSeek's Native Sparse Attention", How Does Native Sparse
+ * Attention Work? (three key/value sets per query, three attention outputs
+ * merged by gates); "Sparsity is Cool", Method (mean-pool compression,
+ * block 64, top-k 16, window 512) and Key claims (later layers pruned to
+ * fewer branches at inference: the branch mask). */
 nsa_status nsa_forward(const nsa_params* p, const void* q, const void* k,
                        const void* v, const float* gates, void* out,
                        const nsa_saved* saved, void* workspace,
@@ -257,7 +262,12 @@ nsa_status nsa_forward_host(const nsa_params* p, const void* q, const void* k,
  * and at most 512 compressed blocks, decode runs as three kernels that
  * stream the caches across all SMs (compression + scores + top-k per
  * sequence; one small CTA per selected or window block; a merge); other
- * shapes reuse the prefill kernels. */
+ * shapes reuse the prefill kernels.  Passage: as nsa_forward, for the one
+ * query a generation step adds ("DeepSeek's Native Sparse Attention",
+ * kernel paragraph: the same block-grouped reads serve training and
+ * inference; "Sparsity is Cool", TL;DR and Key claims: branch pruning at
+ * inference).  idx_out is an addition of this ABI: the decode's block
+ * selection, returned so a caller can inspect or reuse it. */
 nsa_status nsa_decode(const nsa_params* p, const void* q, const void* k_cache,
                       const void* v_cache, const void* kc_cache,
                       const void* vc_cache, const float* gates, void* out,
@@ -325,7 +335,13 @@ nsa_status nsa_cmp_bwd(const nsa_params* p, const void* q, const void* kc,
  * Gradient of out = nsa_forward(q, k, v, gates) for upstream dout, with the
  * forward's saved tensors (kc, vc, o_cmp, lse_cmp for the compression branch;
  * idx, o_sel, lse_sel for selection; o_swa, lse_swa for the window; entries
- * of disabled branches may be NULL).  Overwrites dq, dk, dv, dgates. */
+ * of disabled branches may be NULL).  Overwrites dq, dk, dv, dgates.
+ * Passage: "Sparsity is Cool", Method (the selection backward in two
+ * passes, query-stationary dQ then key-stationary dK/dV over the reverse
+ * block->query map) and Key claims (the compression branch's scores get
+ * direct gradient through the gated combination; no gradient through the
+ * discrete top-k); "DeepSeek's Native Sparse Attention", How Does Native
+ * Sparse Attention Work? (the gated merge whose gradient gives dgates). */
 nsa_status nsa_backward(const nsa_params* p, const void* q, const void* k,
                         const void* v, const float* gates, const void* dout,
                         const nsa_saved* saved, float* dq, float* dk, float* dv,

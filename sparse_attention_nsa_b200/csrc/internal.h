@@ -104,17 +104,19 @@ cudaError_t launch_revmap(const Dims& d, const int32_t* idx, int* chunk, int* of
 cudaError_t launch_revmap_units(const Dims& d, const int32_t* idx, int* chunk, int* offsets,
                                 int* cursor, int* list, int4* units, int* ucount, int tpu, int tq,
                                 int umax, int* err, cudaStream_t s);
+// dO16: scratch of 2*B*Tq*Hq*64 16-bit values (the tensor-core path splits
+// dO into an fp16 pair hi, lo there)
 cudaError_t launch_dkdv(const Dims& d, int mode, const void* q, const void* keys,
                         const void* vals, const float* lse, const float* delta,
-                        const float* dO, const int* offsets, const int* list, float* dk,
-                        float* dv, float* part, int* err, cudaStream_t s);
+                        const float* dO, void* dO16, const int* offsets, const int* list,
+                        float* dk, float* dv, float* part, int* err, cudaStream_t s);
 bool dkdv_tc_eligible(const Dims& d, int mode);
 // workspace of the compression branch's row shares (tensor-core dK/dV)
 size_t dkdv_cmp_part_bytes(const Dims& d);
 cudaError_t launch_dkdv_tc(const Dims& d, int mode, const void* q, const void* keys,
                            const void* vals, const float* lse, const float* delta,
-                           const float* dO, const int* offsets, const int* list, float* dk,
-                           float* dv, float* part, int* err, cudaStream_t s);
+                           const float* dO, void* dO16, const int* offsets, const int* list,
+                           float* dk, float* dv, float* part, int* err, cudaStream_t s);
 cudaError_t launch_pool_bwd(const Dims& d, const float* dkc, const float* dvc, float* dk,
                             float* dv, cudaStream_t s);
 

@@ -719,11 +719,11 @@ static cudaError_t dkdv_t(const Dims& d, const void* q, const void* keys, const 
 
 cudaError_t launch_dkdv(const Dims& d, int mode, const void* q, const void* keys,
                         const void* vals, const float* lse, const float* delta, const float* dO,
-                        const int* offsets, const int* list, float* dk, float* dv, float* part,
-                        int* err, cudaStream_t s) {
+                        void* dO16, const int* offsets, const int* list, float* dk, float* dv,
+                        float* part, int* err, cudaStream_t s) {
   if (dkdv_tc_eligible(d, mode))
-    return launch_dkdv_tc(d, mode, q, keys, vals, lse, delta, dO, offsets, list, dk, dv, part,
-                          err, s);
+    return launch_dkdv_tc(d, mode, q, keys, vals, lse, delta, dO, dO16, offsets, list, dk, dv,
+                          part, err, s);
   if (d.dtype == 1) {
     if (mode == kBwdSel) return dkdv_t<bf16, kBwdSel>(d, q, keys, vals, lse, delta, dO, offsets, list, dk, dv, s);
     if (mode == kBwdSwa) return dkdv_t<bf16, kBwdSwa>(d, q, keys, vals, lse, delta, dO, offsets, list, dk, dv, s);

@@ -400,84 +400,95 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 // ---- pass 2: dK, dV, key-stationary, on tensor cores --------------------------------
 // One CTA per (pair of 64-key blocks j0 = 2p, j1 = 2p+1, KV group, sequence):
 // M = 128 keys.  The query rows that attend those keys are streamed in
-// tiles of 128 rows (128/G tokens x G heads), gathered by four producer
-// warps into a double-buffered, 128-byte-swizzled Q tile and dO tile (dO
-// rounded to bf16).  Selection: the reverse-map lists of j0 and then of j1
-// (a row of j0's list only reaches the first 64 keys, and so on); window:
-// the contiguous range of tokens whose windows reach the pair.  Per tile:
-//   S^T = K Q^T, dP^T = V dO^T   (M128 N128 K64, fp32 in TMEM)
-//   key threads: P^T, dS^T into TMEM (one thread per key)
-//   dV += P^T dO, dK += dS^T Q   (M128 N64 K128, A from TMEM, B = the
-//                                 gathered tiles read MN-major)
-// Precision: dK and dV sum over many query rows, so the bf16 rounding of a
-// single operand (2^-9 relative) would show in them.  dO enters dP^T as a
-// bf16 pair hi + lo (two MMAs), dS enters dK as hi (TMEM) + lo (shared
-// memory), and dV takes P and dO in fp16 (2^-11): the products keep about
-// fp32 accuracy for dK and four times bf16's for dV, with operands whose
-// range is bounded (P in [0, 1]; dO a gradient).
+// tiles of 128 rows, copied by four gather warps with cp.async straight into
+// 128-byte-swizzled Q and dO tiles (dO already split into fp16 hi + lo in
+// memory), kNBuf tiles deep.  Selection: while both blocks' reverse-map
+// lists have rows, a tile takes 64 rows of j0's list (they reach only the
+// first 64 keys) and 64 of j1's (the last 64), so each key warp has 64 rows
+// of work per tile; the rest of the longer list follows in full tiles.
+// Window: the contiguous range of tokens whose windows reach the pair.  Per
+// tile:
+//   S^T = K Q^T                    (bf16, M128 N128 K64, fp32 in TMEM)
+//   dP^T = V (dO_hi + dO_lo)^T     (fp16, M128 N128 K64, fp32 in TMEM)
+//   key threads: P^T (fp16), dS^T (bf16) into TMEM (one thread per key)
+//   dV += P^T dO_hi                (fp16, M128 N64 K128, A from TMEM, B the
+//                                   gathered dO tile read MN-major)
+//   dK += dS^T Q                   (bf16, likewise)
+// Precision: dS = P (dP - delta) subtracts two nearly equal numbers when the
+// softmax is peaked, so dP must keep about fp32 accuracy: dO enters it as an
+// fp16 pair hi + lo (dO = hi + lo to 2^-22), against V converted exactly
+// from bf16 to fp16 in shared memory.  dV sums P dO over many rows, so both
+// factors are fp16 (2^-11); dK takes dS in bf16 (2^-9; the rounding errors
+// of independent rows add in quadrature).  A V or dO element beyond fp16's
+// range (|x| > 65504) is recorded as a range error.  The sums over rows
+// accumulate in fp32 in TMEM.
 // TMEM (512 columns, one CTA per SM): S^T [0,128), dP^T [128,256),
-// dV [256,320), dK [320,384), P^T (fp16) [384,448), dS^T hi [448,512).
-// Warps: 0-3 key threads and epilogue, 4 S^T/dP^T issue and TMEM owner (and
-// the K/V TMA), 5-8 row gather, 9 dV/dK issue (its 24 MMAs per tile overlap
-// the next tile's S^T/dP^T and key-thread work).
-constexpr int kKvThreads = 320;
+// dV [256,320), dK [320,384), P^T [384,448), dS^T [448,512).
+// Warps: 0-7 key threads and epilogue (warps w and w + 4 share TMEM lane
+// quarter w: keys 32w .. 32w+31; warp w takes the 32-row chunks 0 and 2 of
+// every tile, warp w + 4 chunks 1 and 3, so that an interleaved tile gives
+// each warp one chunk of work), 8 S^T/dP^T issue and TMEM owner (and the
+// K/V TMA), 9 dV/dK issue (its 16 MMAs per tile overlap the next tile's
+// S^T/dP^T and key-thread work), 10-13 row gather (warp 10 + c fills rows
+// 32c .. 32c+31).
+constexpr int kKvThreads = 448;
+constexpr int kKeyThreads = 256;
 constexpr int kCmpShares = 16;  // row shares of a compression-branch key pair
+constexpr int kNBuf = 3;        // row-tile buffers
 constexpr uint32_t kKTile2 = 128 * 64 * 2;  // 128 keys x 64 dims, bf16
 constexpr uint32_t kRowTile = 128 * 64 * 2;
+constexpr int kNoKey = 0x40000000;  // first visible key of a row that reaches none
 
 constexpr uint32_t kvColS = 0, kvColDP = 128, kvColDV = 256, kvColDK = 320, kvColP = 384,
                    kvColDS = 448;
 
+// Per tile row r: the keys it reaches among the pair's first 64 (h = 0) and
+// last 64 (h = 1) are those with absolute index in [klo[h][r], klo[h][r] +
+// span[h][r]]; nlse2 = -lse * log2(e), ndelta = -delta.
 struct KvRowInfo {
-  float lse2[128];
-  float delta[128];
-  int tpos[128];   // key position of the row's query
-  int blkmask[128];  // selection: 1 << (block - j0) the row's list belongs to; 0 = no row
+  float nlse2[128];
+  float ndelta[128];
+  int klo[2][128];
+  int span[2][128];
+  int chunk[4];  // bit h: some row of rows 32c .. 32c+31 reaches a key of half h
 };
 
 constexpr uint32_t KV_OFF_K = 0;
 constexpr uint32_t KV_OFF_V = KV_OFF_K + kKTile2;
-constexpr uint32_t KV_OFF_Q = KV_OFF_V + kKTile2;           // 2 buffers each:
-constexpr uint32_t KV_OFF_DO = KV_OFF_Q + 2 * kRowTile;     //   dO hi (bf16)
-constexpr uint32_t KV_OFF_DOL = KV_OFF_DO + 2 * kRowTile;   //   dO lo (bf16)
-constexpr uint32_t KV_OFF_DOH = KV_OFF_DOL + 2 * kRowTile;  //   dO (fp16)
-constexpr uint32_t KV_OFF_DSL = KV_OFF_DOH + 2 * kRowTile;  // dS^T lo, 128 keys x 128 rows
-constexpr uint32_t KV_OFF_INFO = KV_OFF_DSL + 2 * kKTile2;  // 2 x KvRowInfo
-constexpr uint32_t KV_OFF_BAR = KV_OFF_INFO + 2 * sizeof(KvRowInfo);
+constexpr uint32_t KV_OFF_Q = KV_OFF_V + kKTile2;                // kNBuf buffers each:
+constexpr uint32_t KV_OFF_DO = KV_OFF_Q + kNBuf * kRowTile;      //   Q, dO hi, dO lo (bf16)
+constexpr uint32_t KV_OFF_DOL = KV_OFF_DO + kNBuf * kRowTile;
+constexpr uint32_t KV_OFF_INFO = KV_OFF_DOL + kNBuf * kRowTile;  // kNBuf x KvRowInfo
+constexpr uint32_t KV_OFF_BAR = KV_OFF_INFO + ((kNBuf * sizeof(KvRowInfo) + 15) / 16) * 16;
 
 struct KvBars {
-  uint64_t kv;          // K and V of the pair landed (TMA)
-  uint64_t gathered[2]; // 128 gather threads filled row buffer u & 1
-  uint64_t s;           // S^T and dP^T of the current tile are in TMEM
-  uint64_t sfree;       // 128 key threads loaded them
-  uint64_t p;           // 128 key threads wrote P^T and dS^T
-  uint64_t bfree[2];    // dV / dK MMAs of the tile in row buffer u & 1 done
-  uint64_t sdone;       // every S^T / dP^T MMA done (unwinding)
+  uint64_t kv;                 // K and V of the pair landed (TMA)
+  uint64_t vready;             // 256 key threads converted V to fp16
+  uint64_t gathered[kNBuf];    // 128 gather threads filled row buffer u % kNBuf
+  uint64_t s;                  // S^T and dP^T of the current tile are in TMEM
+  uint64_t sfree;              // 128 key threads loaded them
+  uint64_t p;                  // 128 key threads wrote P^T and dS^T
+  uint64_t bfree[kNBuf];       // dV / dK MMAs of the tile in row buffer u % kNBuf done
+  uint64_t sdone;              // every S^T / dP^T MMA done (unwinding)
   uint64_t fin;
 };
 constexpr uint32_t KV_OFF_MISC = KV_OFF_BAR + ((sizeof(KvBars) + 15) / 16) * 16;
 constexpr uint32_t KV_SMEM = KV_OFF_MISC + 16;
+static_assert(KV_SMEM + 1024 <= 227 * 1024, "dK/dV kernel shared memory");
 
-// Rows of one tile: row index within the CTA's row list -> (query index tq
-// or -1, list bit).  Selection lists: j0's tokens then j1's, G rows each.
-__device__ __forceinline__ int kv_row_token(bool sel, long rix, int G, int n0, int n1,
-                                           const int* l0, const int* l1, int tq_lo, int ntok,
-                                           int* bit) {
-  const long ti = rix / G;
-  if (sel) {
-    if (ti < n0) {
-      *bit = 1;
-      return l0[ti];
-    }
-    if (ti < (long)n0 + n1) {
-      *bit = 2;
-      return l1[ti - n0];
-    }
-    *bit = 0;
-    return -1;
+// Row r of tile u of a CTA's row sequence -> (list, index within that list's
+// rows) for the selection branch.  R0, R1: rows (tokens x G) of j0's and
+// j1's lists; nI = tiles that take 64 rows of each.
+__device__ __forceinline__ long sel_tile_row(int u, int r, long R0, long R1, int nI, int* which) {
+  if (u < nI) {
+    *which = r >> 6;
+    const long rix = (long)u * 64 + (r & 63);
+    return rix < (r < 64 ? R0 : R1) ? rix : -1;
   }
-  *bit = 3;
-  return ti < ntok ? tq_lo + (int)ti : -1;
+  const bool first = R0 > R1;  // the longer list continues in full tiles
+  *which = first ? 0 : 1;
+  const long rix = (long)nI * 64 + (long)(u - nI) * 128 + r;
+  return rix < (first ? R0 : R1) ? rix : -1;
 }
 
 // MODE 0 selection, 1 window, 2 compression.  With nseg > 1 (compression:
@@ -489,10 +500,10 @@ template <int MODE>
 __global__ void __launch_bounds__(kKvThreads, 1)
 bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                    const bf16* __restrict__ q, const float* __restrict__ lse,
-                   const float* __restrict__ delta, const float* __restrict__ dO,
-                   const int* __restrict__ offsets, const int* __restrict__ list,
-                   float* __restrict__ dk, float* __restrict__ dv, float* __restrict__ part,
-                   int nseg, Dims d, int* err) {
+                   const float* __restrict__ delta, const __half* __restrict__ dO_hi,
+                   const __half* __restrict__ dO_lo, const int* __restrict__ offsets,
+                   const int* __restrict__ list, float* __restrict__ dk, float* __restrict__ dv,
+                   float* __restrict__ part, int nseg, Dims d, int* err) {
   constexpr bool SEL = MODE == 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -507,108 +518,176 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
   const int kbase = j0 * kKeys;  // first key of the pair
 
   // the rows of this CTA
-  int n0 = 0, n1 = 0, tq_lo = 0, ntok = 0;
+  long R0 = 0, R1 = 0;
+  int nI = 0, tq_lo = 0, ntok = 0;
   const int* l0 = nullptr;
   const int* l1 = nullptr;
+  int ntiles_all;
   if (SEL) {
     const size_t bg = (size_t)b * d.Hkv + g;
     const int* off = offsets + bg * (d.Nb + 1);
     l0 = list + bg * (size_t)d.Tq * d.topk + off[j0];
-    n0 = off[j0 + 1] - off[j0];
+    R0 = (long)(off[j0 + 1] - off[j0]) * d.G;
     if (j0 + 1 < d.Nb) {
       l1 = list + bg * (size_t)d.Tq * d.topk + off[j0 + 1];
-      n1 = off[j0 + 2] - off[j0 + 1];
+      R1 = (long)(off[j0 + 2] - off[j0 + 1]) * d.G;
     }
-  } else if (MODE == 1) {
-    const int t_lo = kbase, t_hi = min(kbase + 2 * kKeys - 1 + d.window - 1, d.T - 1);
-    tq_lo = max(0, t_lo - d.q_off);
-    ntok = max(0, t_hi - d.q_off - tq_lo + 1);
-  } else {  // every query from the one that completes compressed block kbase on
-    tq_lo = max(0, (kbase + 1) * d.l - 1 - d.q_off);
-    ntok = max(0, d.Tq - tq_lo);
+    const long h0 = (R0 + 63) / 64, h1 = (R1 + 63) / 64;
+    nI = (int)min(h0, h1);
+    const long rest = (R0 > R1 ? R0 : R1) - (long)nI * 64;
+    ntiles_all = nI + (int)((max(rest, 0L) + 127) / 128);
+  } else {
+    if (MODE == 1) {
+      const int t_lo = kbase, t_hi = min(kbase + 2 * kKeys - 1 + d.window - 1, d.T - 1);
+      tq_lo = max(0, t_lo - d.q_off);
+      ntok = max(0, t_hi - d.q_off - tq_lo + 1);
+    } else {  // every query from the one that completes compressed block kbase on
+      tq_lo = max(0, (kbase + 1) * d.l - 1 - d.q_off);
+      ntok = max(0, d.Tq - tq_lo);
+    }
+    ntiles_all = (int)(((long)ntok * d.G + 127) / 128);
   }
-  const long nrows = SEL ? ((long)n0 + n1) * d.G : (long)ntok * d.G;
-  const int ntiles_all = (int)((nrows + 127) / 128);
   const int tps = (ntiles_all + nseg - 1) / nseg;  // tiles per share
   const int u0 = seg * tps;
   const int ntiles = max(0, min(tps, ntiles_all - u0));
 
   if (tid == 0) {
     mbar_init(&bars->kv, 1);
-    for (int i = 0; i < 2; ++i) {
+    mbar_init(&bars->vready, kKeyThreads);
+    for (int i = 0; i < kNBuf; ++i) {
       mbar_init(&bars->gathered[i], 128);
       mbar_init(&bars->bfree[i], 1);
     }
     mbar_init(&bars->s, 1);
-    mbar_init(&bars->sfree, 128);
-    mbar_init(&bars->p, 128);
+    mbar_init(&bars->sfree, kKeyThreads);
+    mbar_init(&bars->p, kKeyThreads);
     mbar_init(&bars->sdone, 1);
     mbar_init(&bars->fin, 1);
     fence_barrier_init();
     fence_proxy_async_smem();
     *abort_flag = 0;
   }
-  if (warp == 4) tmem_alloc(tmem_slot, 512);
+  if (warp == 8) tmem_alloc(tmem_slot, 512);
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp >= 5 && warp <= 8) {
-    // ---- row gather: thread gr fills row gr of each tile ------------------------------
-    const int gr = tid - 160;
+  if (warp >= 10) {
+    // ---- row gather: warp 10 + w fills rows 32w .. 32w+31 of each tile ------------------
+    // Thread gr looks up row gr's token (one iteration ahead: the list entry
+    // of the next tile is loaded while this tile's copies go out).  The Q and
+    // dO rows go by cp.async (16 bytes each, zero-filled for an absent row),
+    // lane L copying 16-byte chunk L % 8 of rows 4i + L / 8 of the warp's 32,
+    // so each instruction covers four whole 128-byte rows; a tile is handed
+    // to the MMA side one iteration after its copies were issued, once they
+    // have landed.
+    const int gr = tid - 320;
+    const int ch = lane & 7;
+    auto row_of = [&](int u, int* which, int* hh) -> int {  // query index or -1
+      const int uu = u0 + u;
+      if (SEL) {
+        const long rix = sel_tile_row(uu, gr, R0, R1, nI, which);
+        if (rix < 0) return -1;
+        *hh = (int)(rix % d.G);
+        return (*which ? l1 : l0)[rix / d.G];
+      }
+      *which = 0;
+      const long rix = (long)uu * 128 + gr;
+      *hh = (int)(rix % d.G);
+      const long ti = rix / d.G;
+      return ti < ntok ? tq_lo + (int)ti : -1;
+    };
+    int wh_n = 0, hh_n = 0;
+    int tq_n = ntiles > 0 ? row_of(0, &wh_n, &hh_n) : -1;
+    bool ok = true;
     for (int u = 0; u < ntiles; ++u) {
-      const int bu = u & 1;
-      if (u >= 2 && !wait_bar(&bars->bfree[bu], ((u - 2) >> 1) & 1, abort_flag, err)) break;
-      const long rix = (long)(u0 + u) * 128 + gr;
-      int bit = 0;
-      const int tq =
-          rix < nrows ? kv_row_token(SEL, rix, d.G, n0, n1, l0, l1, tq_lo, ntok, &bit) : -1;
-      const int hh = (int)(rix % d.G);
-      const bool ok = tq >= 0 && tq < d.Tq;
-      const size_t row = ((size_t)b * d.Tq + (ok ? tq : 0)) * d.Hq + (size_t)g * d.G + hh;
-      const uint32_t off = (uint32_t)(gr >> 3) * 1024u + (uint32_t)(gr & 7) * 128u;
-      const uint32_t qrow = smem_u32(smem + KV_OFF_Q + bu * kRowTile) + off;
-      const uint32_t drow = smem_u32(smem + KV_OFF_DO + bu * kRowTile) + off;
-      const uint32_t lrow = smem_u32(smem + KV_OFF_DOL + bu * kRowTile) + off;
-      const uint32_t hrow = smem_u32(smem + KV_OFF_DOH + bu * kRowTile) + off;
-      float l2 = -INFINITY;
-      if (ok) l2 = lse[row] * kLog2e;
+      const int bu = u % kNBuf;
+      if (u >= kNBuf &&
+          !wait_bar(&bars->bfree[bu], ((u - kNBuf) / kNBuf) & 1, abort_flag, err)) {
+        ok = false;
+        break;
+      }
+      const int tq = tq_n, which = wh_n, hh = hh_n;
+      if (u + 1 < ntiles) tq_n = row_of(u + 1, &wh_n, &hh_n);  // issued now, used next iteration
+      const bool okr = tq >= 0 && tq < d.Tq;
+      const size_t row = ((size_t)b * d.Tq + (okr ? tq : 0)) * d.Hq + (size_t)g * d.G + hh;
+      const uint32_t qb = smem_u32(smem + KV_OFF_Q + bu * kRowTile);
+      const uint32_t hb = smem_u32(smem + KV_OFF_DO + bu * kRowTile);
+      const uint32_t lb = smem_u32(smem + KV_OFF_DOL + bu * kRowTile);
+      const unsigned long long rowc = okr ? (unsigned long long)row : ~0ull;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint4 qv = make_uint4(0u, 0u, 0u, 0u);
-        uint32_t w[4] = {0u, 0u, 0u, 0u}, wl[4] = {0u, 0u, 0u, 0u}, wh[4] = {0u, 0u, 0u, 0u};
-        if (ok) {
-          qv = __ldg(reinterpret_cast<const uint4*>(q + row * 64) + c);
-          const float4 a = __ldg(reinterpret_cast<const float4*>(dO + row * 64) + 2 * c);
-          const float4 a2 = __ldg(reinterpret_cast<const float4*>(dO + row * 64) + 2 * c + 1);
-          const float x[8] = {a.x, a.y, a.z, a.w, a2.x, a2.y, a2.z, a2.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float h0 = __bfloat162float(__float2bfloat16_rn(x[2 * e]));
-            const float h1 = __bfloat162float(__float2bfloat16_rn(x[2 * e + 1]));
-            w[e] = pack_bf16(h0, h1);
-            wl[e] = pack_bf16(x[2 * e] - h0, x[2 * e + 1] - h1);
-            wh[e] = pack_f16(x[2 * e], x[2 * e + 1]);
+      for (int i = 0; i < 8; ++i) {
+        const int rr = 4 * i + (lane >> 3);  // row of the warp's 32
+        const unsigned long long rw = __shfl_sync(0xffffffffu, rowc, rr);
+        const int r = 32 * (warp - 10) + rr;  // row of the tile
+        const uint32_t off = (uint32_t)(r >> 3) * 1024u + (uint32_t)(r & 7) * 128u +
+                             ((uint32_t)(ch ^ (r & 7)) << 4);
+        const bool present = rw != ~0ull;
+        const size_t src = (present ? (size_t)rw : 0) * 64 + 8 * ch;
+        const uint32_t nb = present ? 16u : 0u;
+        cp_async16(qb + off, q + src, nb);
+        cp_async16(hb + off, dO_hi + src, nb);
+        cp_async16(lb + off, dO_lo + src, nb);
+      }
+      cp_async_commit();
+      float l2 = -INFINITY, dl = 0.f;
+      if (okr) {
+        l2 = __ldg(lse + row) * kLog2e;
+        dl = __ldg(delta + row);
+      }
+      // visible keys of this row among the pair's two halves
+      const int t = d.q_off + (okr ? tq : 0);
+      const bool live = okr && l2 != -INFINITY;
+      int lo0 = kNoKey, lo1 = kNoKey, sp0 = 0, sp1 = 0;
+      if (live) {
+        if (SEL) {
+          if (which == 0) {
+            lo0 = 0;
+            sp0 = t;
+          } else {
+            lo1 = 0;
+            sp1 = t;
+          }
+        } else if (MODE == 1) {
+          lo0 = lo1 = max(0, t - d.window + 1);
+          sp0 = sp1 = t - lo0;
+        } else {
+          const int khi = (t + 1) / d.l - 1;  // last complete compressed block
+          if (khi >= 0) {
+            lo0 = lo1 = 0;
+            sp0 = sp1 = khi;
           }
         }
-        const uint32_t sw = (uint32_t)(c ^ (gr & 7)) << 4;
-        st_shared_v4(qrow + sw, qv.x, qv.y, qv.z, qv.w);
-        st_shared_v4(drow + sw, w[0], w[1], w[2], w[3]);
-        st_shared_v4(lrow + sw, wl[0], wl[1], wl[2], wl[3]);
-        st_shared_v4(hrow + sw, wh[0], wh[1], wh[2], wh[3]);
       }
       KvRowInfo& in = info[bu];
-      in.lse2[gr] = l2;
-      in.delta[gr] = ok ? delta[row] : 0.f;
-      in.tpos[gr] = d.q_off + (ok ? tq : 0);
-      in.blkmask[gr] = (ok && l2 != -INFINITY) ? bit : 0;
-      fence_proxy_async_smem();
-      mbar_arrive(&bars->gathered[bu]);
+      in.nlse2[gr] = -l2;
+      in.ndelta[gr] = -dl;
+      in.klo[0][gr] = lo0;
+      in.span[0][gr] = sp0;
+      in.klo[1][gr] = lo1;
+      in.span[1][gr] = sp1;
+      // rows 32c .. 32c+31 are this warp's: flag the halves they reach
+      const int kb0 = kbase, kb1 = kbase + kKeys;
+      const bool r0 = lo0 <= kb0 + kKeys - 1 && lo0 + sp0 >= kb0;
+      const bool r1 = lo1 <= kb1 + kKeys - 1 && lo1 + sp1 >= kb1;
+      const unsigned m0 = __ballot_sync(0xffffffffu, r0), m1 = __ballot_sync(0xffffffffu, r1);
+      if (lane == 0) in.chunk[warp - 10] = (m0 ? 1 : 0) | (m1 ? 2 : 0);
+      if (u >= 1) {
+        cp_async_wait<1>();        // tile u - 1 has landed
+        fence_proxy_async_smem();  // the MMAs read it through the async proxy
+        mbar_arrive(&bars->gathered[(u - 1) % kNBuf]);
+      }
     }
-  } else if (warp == 4) {
+    cp_async_wait<0>();  // no copy outlives the CTA
+    if (ok && ntiles > 0) {
+      fence_proxy_async_smem();
+      mbar_arrive(&bars->gathered[(ntiles - 1) % kNBuf]);
+    }
+  } else if (warp == 8) {
     // ---- S^T / dP^T issue (and the pair's K/V by TMA) ---------------------------------
     if (lane == 0) {
       constexpr uint32_t idesc_st = idesc_bf16(128, 128, false, false);
+      constexpr uint32_t idesc_dp = idesc_f16(128, 128, false, false);
       const uint32_t k_addr = smem_u32(smem + KV_OFF_K), v_addr = smem_u32(smem + KV_OFF_V);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
@@ -617,10 +696,11 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         tma_load_3d(smem + KV_OFF_K + h * kTileBytes, &tm_k, &bars->kv, 0, g, b * nkeys + kbase + h * kKeys);
         tma_load_3d(smem + KV_OFF_V + h * kTileBytes, &tm_v, &bars->kv, 0, g, b * nkeys + kbase + h * kKeys);
       }
-      const bool ok = wait_bar(&bars->kv, 0, abort_flag, err);
+      const bool ok = wait_bar(&bars->kv, 0, abort_flag, err) &&
+                      (ntiles == 0 || wait_bar(&bars->vready, 0, abort_flag, err));
       for (int u = 0; ok && u < ntiles; ++u) {
-        const int bu = u & 1;
-        if (!wait_bar(&bars->gathered[bu], (u >> 1) & 1, abort_flag, err)) break;
+        const int bu = u % kNBuf;
+        if (!wait_bar(&bars->gathered[bu], (u / kNBuf) & 1, abort_flag, err)) break;
         // S^T / dP^T are single-buffered: the key threads must have loaded tile u-1's
         if (u >= 1 && !wait_bar(&bars->sfree, (u - 1) & 1, abort_flag, err)) break;
         tc_fence_after();
@@ -634,11 +714,11 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_bf16(tmem + kvColDP, desc_sw128(v_addr + kk * 32, 16), desc_sw128(do_addr + kk * 32, 16),
-                   idesc_st, kk > 0);
+                   idesc_dp, kk > 0);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)  // dO lo: dP^T keeps about fp32 accuracy
-          mma_bf16(tmem + kvColDP, desc_sw128(v_addr + kk * 32, 16), desc_sw128(dol_addr + kk * 32, 16),
-                   idesc_st, 1u);
+          mma_bf16(tmem + kvColDP, desc_sw128(v_addr + kk * 32, 16),
+                   desc_sw128(dol_addr + kk * 32, 16), idesc_dp, 1u);
         mma_commit(&bars->s);
       }
       mma_commit(&bars->sdone);
@@ -648,28 +728,22 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
   } else if (warp == 9) {
     // ---- dV += P^T dO, dK += dS^T Q issue ----------------------------------------------
     if (lane == 0) {
-      constexpr uint32_t idesc_kv = idesc_bf16(128, 64, false, true);  // dK (hi, A in TMEM)
-      constexpr uint32_t idesc_kl = idesc_bf16(128, 64, false, true);  // dK (lo, A from smem)
-      constexpr uint32_t idesc_v16 = idesc_f16(128, 64, false, true);  // dV (fp16)
-      const uint32_t dsl_addr = smem_u32(smem + KV_OFF_DSL);
+      constexpr uint32_t idesc_kv = idesc_bf16(128, 64, false, true);  // A in TMEM, B MN-major
+      constexpr uint32_t idesc_v16 = idesc_f16(128, 64, false, true);   // dV: fp16 P^T, dO
       for (int u = 0; u < ntiles; ++u) {
-        // A operands in TMEM (and dS^T lo in smem); the gathered tiles read
-        // MN-major: K dimension = rows
+        // A operands in TMEM; the gathered tiles read MN-major: K dimension = rows
         if (!wait_bar(&bars->p, u & 1, abort_flag, err)) break;
         tc_fence_after();
-        const int bu = u & 1;
+        const int bu = u % kNBuf;
         const uint32_t q_addr = smem_u32(smem + KV_OFF_Q + bu * kRowTile);
-        const uint32_t doh_addr = smem_u32(smem + KV_OFF_DOH + bu * kRowTile);
+        const uint32_t do_addr = smem_u32(smem + KV_OFF_DO + bu * kRowTile);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t acc = (u > 0 || kk > 0) ? 1u : 0u;
-          const uint64_t qb = desc_sw128(q_addr + kk * 2048, 8192);
           mma_bf16_ts(tmem + kvColDV, tmem + kvColP + kk * 8,
-                      desc_sw128(doh_addr + kk * 2048, 8192), idesc_v16, acc);
-          mma_bf16_ts(tmem + kvColDK, tmem + kvColDS + kk * 8, qb, idesc_kv, acc);
-          // dS^T lo: 128 keys x 128 rows, K-major, two 64-row swizzle atoms
-          mma_bf16(tmem + kvColDK, desc_sw128(dsl_addr + (kk >> 2) * kKTile2 + (kk & 3) * 32, 16),
-                   qb, idesc_kl, 1u);
+                      desc_sw128(do_addr + kk * 2048, 8192), idesc_v16, acc);
+          mma_bf16_ts(tmem + kvColDK, tmem + kvColDS + kk * 8,
+                      desc_sw128(q_addr + kk * 2048, 8192), idesc_kv, acc);
         }
         mma_commit(&bars->bfree[bu]);  // frees the row buffer and the P^T / dS^T columns
       }
@@ -677,15 +751,40 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
       drain_bar(&bars->fin, 0);
     }
   } else {
-    // ---- key threads: thread k owns key kbase + k (TMEM lane k) -------------------------
-    const int k = tid;
+    // ---- key threads: key kbase + k (TMEM lane k), k = 32 (warp % 4) + lane -----------
+    const int k = 32 * (warp & 3) + lane;
+    const int csel = warp >> 2;  // this warp's chunks: csel and csel + 2
     const int key = kbase + k;
-    const int kbit = 1 << (k >> 6);  // which block of the pair
-    const uint32_t lane_tmem = tmem + ((uint32_t)(warp * 32) << 16);
+    const int half = k >> 6;  // which block of the pair
+    const uint32_t lane_tmem = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const float sl2 = d.scale * kLog2e;
+    const uint64_t sl2x2 = f2_pack(sl2, sl2);
     bool ok = true;
+    if (ntiles > 0) {
+      // V of the pair (bf16, landed by TMA) -> fp16 in place, for dP^T
+      ok = wait_bar_warp(&bars->kv, 0, abort_flag, err);
+      if (ok) {
+        uint4* vv = reinterpret_cast<uint4*>(smem + KV_OFF_V);
+        bool range_ok = true;
+        for (int i = tid; i < (int)(kKTile2 / 16); i += kKeyThreads) {
+          uint4 x = vv[i];
+          uint32_t* w = reinterpret_cast<uint32_t*>(&x);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+            range_ok = range_ok && fabsf(f.x) <= 65504.f && fabsf(f.y) <= 65504.f;
+            w[e] = pack_f16(f.x, f.y);
+          }
+          vv[i] = x;
+        }
+        if (!range_ok) record_error(err, kDevRange);
+        fence_proxy_async_smem();  // the MMA reads V through the async proxy
+        mbar_arrive(&bars->vready);
+      }
+    }
+    int dirty = 3;  // bit i: P^T / dS^T columns of chunk csel + 2i may hold nonzero values
     for (int u = 0; u < ntiles; ++u) {
-      const KvRowInfo& in = info[u & 1];
+      const KvRowInfo& in = info[u % kNBuf];
       if (!wait_bar_warp(&bars->s, u & 1, abort_flag, err)) {
         ok = false;
         break;
@@ -693,91 +792,106 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
       tc_fence_after();
       bool stop = false;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {  // 32 rows at a time
-        float sv[32], pv[32];
-        tmem_ld32(lane_tmem + kvColS + 32u * c, sv);
-        tmem_ld32(lane_tmem + kvColDP + 32u * c, pv);
-        tmem_wait_ld();
-        if (c == 3) {  // S^T and dP^T of this tile are in registers: release them
-          tc_fence_before();
-          mbar_arrive(&bars->sfree);
-        }
-        uint32_t pp[16], dd[16], dl[16];
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float p2[2], d2[2];
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int r = 32 * c + e + h;
-            const int t = in.tpos[r];
-            bool vis = (in.blkmask[r] & kbit) &&
-                       (MODE == 2 ? key * d.l + d.l - 1 <= t : key <= t);
-            if (MODE == 1) vis = vis && key >= t - d.window + 1;
-            const float pr = vis ? fast_exp2(fmaf(sv[e + h], sl2, -in.lse2[r])) : 0.f;
-            p2[h] = pr;
-            d2[h] = pr * (pv[e + h] - in.delta[r]);
+      for (int i = 0; i < 2; ++i) {  // 32 rows at a time, in halves of 16
+        const int c = csel + 2 * i;
+        const bool any = (in.chunk[c] >> half) & 1;  // warp-uniform
+        if (!any) {
+          if (i == 1) {  // nothing to load: release S^T / dP^T now
+            tc_fence_before();
+            mbar_arrive(&bars->sfree);
           }
-          const float h0 = __bfloat162float(__float2bfloat16_rn(d2[0]));
-          const float h1 = __bfloat162float(__float2bfloat16_rn(d2[1]));
-          pp[e / 2] = pack_f16(p2[0], p2[1]);
-          dd[e / 2] = pack_bf16(h0, h1);
-          dl[e / 2] = pack_bf16(d2[0] - h0, d2[1] - h1);
+          if (!((dirty >> i) & 1)) continue;  // columns already zero
         }
-        if (c == 0 && u >= 1) {
-          // P^T / dS^T (TMEM and the dS lo tile): the dV/dK MMAs of tile u-1
-          // must have read them (waited for only now, after the first 32 rows)
-          if (!wait_bar_warp(&bars->bfree[(u - 1) & 1], ((u - 1) >> 1) & 1, abort_flag, err)) {
+        if (u >= 1 && (dirty & 4) == 0) {
+          // P^T / dS^T (TMEM): the dV/dK MMAs of tile u-1 must have read them
+          // (waited for before this warp's first store of the tile; bit 2 of
+          // dirty records that it has been)
+          if (!wait_bar_warp(&bars->bfree[(u - 1) % kNBuf], ((u - 1) / kNBuf) & 1, abort_flag,
+                             err)) {
             stop = true;
+            if (any && i == 1) mbar_arrive(&bars->sfree);
             break;
           }
           tc_fence_after();
         }
-        tmem_st16u(lane_tmem + kvColP + 16u * c, pp);
-        tmem_st16u(lane_tmem + kvColDS + 16u * c, dd);
-        // dS lo into the K-major smem tile: row k, rows 32c .. 32c+31 of the
-        // tile are 16-byte chunks 4(c&1) .. 4(c&1)+3 of swizzle atom c >> 1
-        const uint32_t lrow = smem_u32(smem + KV_OFF_DSL) + (uint32_t)(c >> 1) * kKTile2 +
-                              (uint32_t)(k >> 3) * 1024u + (uint32_t)(k & 7) * 128u;
+        dirty |= 4;
+        if (!any) {
+          uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          const int cc = 4 * (c & 1) + q4;
-          st_shared_v4(lrow + ((uint32_t)(cc ^ (k & 7)) << 4), dl[4 * q4], dl[4 * q4 + 1],
-                       dl[4 * q4 + 2], dl[4 * q4 + 3]);
+          for (int hf = 0; hf < 2; ++hf) {
+            tmem_st8u(lane_tmem + kvColP + 16u * c + 8u * hf, z);
+            tmem_st8u(lane_tmem + kvColDS + 16u * c + 8u * hf, z);
+          }
+          dirty &= ~(1 << i);
+          continue;
         }
+#pragma unroll 1
+        for (int hf = 0; hf < 2; ++hf) {
+          float sv[16], pv[16];
+          tmem_ld16(lane_tmem + kvColS + 32u * c + 16u * hf, sv);
+          tmem_ld16(lane_tmem + kvColDP + 32u * c + 16u * hf, pv);
+          tmem_wait_ld();
+          if (i == 1 && hf == 1) {  // S^T and dP^T of this tile are in registers: release them
+            tc_fence_before();
+            mbar_arrive(&bars->sfree);
+          }
+          uint32_t pp[8], dd[8];
+#pragma unroll
+          for (int e = 0; e < 16; e += 2) {
+            const int r = 32 * c + 16 * hf + e;
+            const int2 lo = *reinterpret_cast<const int2*>(&in.klo[half][r]);
+            const int2 sp = *reinterpret_cast<const int2*>(&in.span[half][r]);
+            const uint64_t nl = *reinterpret_cast<const uint64_t*>(&in.nlse2[r]);
+            const uint64_t nd = *reinterpret_cast<const uint64_t*>(&in.ndelta[r]);
+            const float2 x = f2_unpack(f2_fma(f2_pack(sv[e], sv[e + 1]), sl2x2, nl));
+            const bool v0 = (unsigned)(key - lo.x) <= (unsigned)sp.x;
+            const bool v1 = (unsigned)(key - lo.y) <= (unsigned)sp.y;
+            const float p0 = v0 ? fast_exp2(x.x) : 0.f;
+            const float p1 = v1 ? fast_exp2(x.y) : 0.f;
+            const uint64_t pq = f2_pack(p0, p1);
+            const float2 ds = f2_unpack(f2_mul(pq, f2_add(f2_pack(pv[e], pv[e + 1]), nd)));
+            pp[e / 2] = pack_f16(p0, p1);
+            dd[e / 2] = pack_bf16(ds.x, ds.y);
+          }
+          tmem_st8u(lane_tmem + kvColP + 16u * c + 8u * hf, pp);
+          tmem_st8u(lane_tmem + kvColDS + 16u * c + 8u * hf, dd);
+        }
+        dirty |= 1 << i;
       }
+      dirty &= 3;
       if (stop) {
         ok = false;
         break;
       }
-      fence_proxy_async_smem();  // dS lo is read by the MMA (async proxy)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars->p);
     }
-    // epilogue: dk += scale * dK, dv += dV for this key (fp32, accumulated)
+    // epilogue: dv += dV (warps 0-3), dk += scale * dK (warps 4-7) for this key
     bool have = false;
     if (ok && ntiles > 0) have = wait_bar_warp(&bars->fin, 0, abort_flag, err);
     float a[32];
     const size_t krow = ((size_t)b * nkeys + key) * d.Hkv * 64 + (size_t)g * 64;
     const bool kin = key < nkeys;
     const size_t nk_all = (size_t)d.B * nkeys * d.Hkv * 64;  // one share of dK (or dV)
+    const bool isk = csel == 1;
 #pragma unroll 1
-    for (int h = 0; h < 4; ++h) {  // dV [0,64), dK [64,128) in halves of 32
+    for (int h = 0; h < 2; ++h) {  // columns [32h, 32h + 32) of dV or dK
       if (have) {
         tc_fence_after();
-        tmem_ld32(lane_tmem + kvColDV + 32u * h, a);
+        tmem_ld32(lane_tmem + (isk ? kvColDK : kvColDV) + 32u * h, a);
         tmem_wait_ld();
       }
-      const float sc = h < 2 ? 1.f : d.scale;
+      const float sc = isk ? d.scale : 1.f;
       if (MODE == 2 && kin) {  // this share's partial (zeros when it had no rows)
-        float* dst = part + ((size_t)seg * 2 + (h < 2 ? 1 : 0)) * nk_all + krow + 32 * (h & 1);
+        float* dst = part + ((size_t)seg * 2 + (isk ? 0 : 1)) * nk_all + krow + 32 * h;
 #pragma unroll
         for (int c = 0; c < 32; c += 4)
           *reinterpret_cast<float4*>(dst + c) =
               have ? make_float4(a[c] * sc, a[c + 1] * sc, a[c + 2] * sc, a[c + 3] * sc)
                    : make_float4(0.f, 0.f, 0.f, 0.f);
       } else if (have && kin) {
-        float* dst = (h < 2 ? dv : dk) + krow + 32 * (h & 1);
+        float* dst = (isk ? dk : dv) + krow + 32 * h;
 #pragma unroll
         for (int c = 0; c < 32; c += 4) {
           float4 x = *reinterpret_cast<float4*>(dst + c);
@@ -792,10 +906,35 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     tc_fence_before();
   }
   __syncthreads();
-  if (warp == 4) {
+  if (warp == 8) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+}
+
+// dO (fp32) split into an fp16 pair for the gathered dK/dV tiles: hi = dO
+// rounded to nearest even, lo = (dO - hi) rounded likewise; n a multiple
+// of 8.  A finite element beyond fp16's range is recorded as a range error.
+__global__ void dO_split_f16_kernel(const float* __restrict__ src, __half* __restrict__ hi,
+                                    __half* __restrict__ lo, size_t n, int* err) {
+  const size_t i = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) * 8;
+  if (i >= n) return;
+  const float4 a = *reinterpret_cast<const float4*>(src + i);
+  const float4 c = *reinterpret_cast<const float4*>(src + i + 4);
+  const float x[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+  uint32_t h[4], l[4];
+  bool range_ok = true;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float h0 = __half2float(__float2half_rn(x[2 * e]));
+    const float h1 = __half2float(__float2half_rn(x[2 * e + 1]));
+    range_ok = range_ok && fabsf(x[2 * e]) <= 65504.f && fabsf(x[2 * e + 1]) <= 65504.f;
+    h[e] = pack_f16(h0, h1);
+    l[e] = pack_f16(x[2 * e] - h0, x[2 * e + 1] - h1);
+  }
+  if (!range_ok) record_error(err, kDevRange);
+  *reinterpret_cast<uint4*>(hi + i) = make_uint4(h[0], h[1], h[2], h[3]);
+  *reinterpret_cast<uint4*>(lo + i) = make_uint4(l[0], l[1], l[2], l[3]);
 }
 
 // dk += sum over shares of part[s][0], dv += sum of part[s][1], in share order.
@@ -822,12 +961,15 @@ __global__ void dkdv_share_sum_kernel(const float* __restrict__ part, float* __r
 template <int MODE>
 cudaError_t launch_dkdv_tc_t(const Dims& d, const void* q, const void* k, const void* v,
                              const float* lse, const float* delta, const float* dO,
-                             const int* offsets, const int* list, float* dk, float* dv,
-                             float* part, int* err, cudaStream_t s) {
+                             void* dO16, const int* offsets, const int* list, float* dk,
+                             float* dv, float* part, int* err, cudaStream_t s) {
   const int nkeys = MODE == 2 ? d.Nc : d.T;
   const int nchunk = (nkeys + kKeys - 1) / kKeys;
   const int npairs = (nchunk + 1) / 2;
   if (npairs == 0) return cudaSuccess;
+  const size_t nel = (size_t)d.B * d.Tq * d.Hq * 64;
+  dO_split_f16_kernel<<<(unsigned)((nel / 8 + 255) / 256), 256, 0, s>>>(
+      dO, (__half*)dO16, (__half*)dO16 + nel, nel, err);
   const int nseg = MODE == 2 ? kCmpShares : 1;
   CUtensorMap mk, mv;
   if (!make_tmap_bf16(&mk, k, d.Hkv, (long)d.B * nkeys, 1, kKeys) ||
@@ -840,7 +982,8 @@ cudaError_t launch_dkdv_tc_t(const Dims& d, const void* q, const void* k, const 
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   bwd_dkdv_tc_kernel<MODE><<<dim3(npairs * nseg, d.Hkv, d.B), kKvThreads, smem, s>>>(
-      mk, mv, (const bf16*)q, lse, delta, dO, offsets, list, dk, dv, part, nseg, d, err);
+      mk, mv, (const bf16*)q, lse, delta, (const __half*)dO16, (const __half*)dO16 + nel, offsets,
+      list, dk, dv, part, nseg, d, err);
   e = cudaGetLastError();
   if (e != cudaSuccess || MODE != 2) return e;
   const size_t n = (size_t)d.B * nkeys * d.Hkv * 64;
@@ -887,14 +1030,15 @@ size_t dkdv_cmp_part_bytes(const Dims& d) {
 }
 
 cudaError_t launch_dkdv_tc(const Dims& d, int mode, const void* q, const void* k, const void* v,
-                           const float* lse, const float* delta, const float* dO,
+                           const float* lse, const float* delta, const float* dO, void* dO16,
                            const int* offsets, const int* list, float* dk, float* dv, float* part,
                            int* err, cudaStream_t s) {
+  void* o16 = dO16;
   if (mode == 0)
-    return launch_dkdv_tc_t<0>(d, q, k, v, lse, delta, dO, offsets, list, dk, dv, part, err, s);
+    return launch_dkdv_tc_t<0>(d, q, k, v, lse, delta, dO, o16, offsets, list, dk, dv, part, err, s);
   if (mode == 1)
-    return launch_dkdv_tc_t<1>(d, q, k, v, lse, delta, dO, offsets, list, dk, dv, part, err, s);
-  return launch_dkdv_tc_t<2>(d, q, k, v, lse, delta, dO, offsets, list, dk, dv, part, err, s);
+    return launch_dkdv_tc_t<1>(d, q, k, v, lse, delta, dO, o16, offsets, list, dk, dv, part, err, s);
+  return launch_dkdv_tc_t<2>(d, q, k, v, lse, delta, dO, o16, offsets, list, dk, dv, part, err, s);
 }
 
 cudaError_t launch_dq_tc(const Dims& d, int mode, const void* q, const void* k, const void* v,

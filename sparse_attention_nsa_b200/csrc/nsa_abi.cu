@@ -586,9 +586,10 @@ namespace {
 //   delta [B*Tq*Hq] f32 | dO_cmp, dO_sel, dO_swa [B*Tq*Hq*64] f32 |
 //   dkc, dvc [B*Nc*Hkv*64] f32 | reverse-map chunk positions
 //   [B*Hkv*ceil(Tq/256)*Nb] i32 | offsets [B*Hkv*(Nb+1)] i32 |
-//   list [B*Hkv*Tq*topk] i32 | compression dK/dV row shares (tensor-core path)
+//   list [B*Hkv*Tq*topk] i32 | compression dK/dV row shares (tensor-core path) |
+//   dO split into fp16 hi, lo [2*B*Tq*Hq*64] (tensor-core dK/dV path)
 struct BwdCarve {
-  size_t delta, dO[3], dkc, dvc, counts, offsets, list, part, total;
+  size_t delta, dO[3], dkc, dvc, counts, offsets, list, part, dO16, total;
 };
 
 BwdCarve bwd_carve(const Dims& d) {
@@ -608,6 +609,7 @@ BwdCarve bwd_carve(const Dims& d) {
   c.offsets = take((size_t)d.B * d.Hkv * (d.Nb + 1) * 4);
   c.list = take((size_t)d.B * d.Hkv * d.Tq * d.topk * 4);
   c.part = take(nsa::dkdv_tc_eligible(d, 2) ? nsa::dkdv_cmp_part_bytes(d) : 0);
+  c.dO16 = take(nsa::dkdv_tc_eligible(d, 0) ? 2 * rows * 64 * 2 : 0);
   c.total = at;
   return c;
 }
@@ -626,8 +628,8 @@ nsa_status sel_bwd_body(const Dims& d, const void* q, const void* k, const void*
   int* list = (int*)(w + c.list);
   NSA_TRY_CUDA(nsa::launch_dq(d, 0, q, k, v, idx, o_sel, lse_sel, dO_sel, dq, delta, err_word(), s));
   NSA_TRY_CUDA(nsa::launch_revmap(d, idx, counts, offsets, list, s));
-  NSA_TRY_CUDA(nsa::launch_dkdv(d, 0, q, k, v, lse_sel, delta, dO_sel, offsets, list, dk, dv, nullptr,
-                                err_word(), s));
+  NSA_TRY_CUDA(nsa::launch_dkdv(d, 0, q, k, v, lse_sel, delta, dO_sel, w + c.dO16, offsets, list,
+                                dk, dv, nullptr, err_word(), s));
   return NSA_OK;
 }
 
@@ -637,8 +639,8 @@ nsa_status swa_bwd_body(const Dims& d, const void* q, const void* k, const void*
                         cudaStream_t s) {
   float* delta = (float*)(w + c.delta);
   NSA_TRY_CUDA(nsa::launch_dq(d, 1, q, k, v, nullptr, o_swa, lse_swa, dO_swa, dq, delta, nullptr, s));
-  NSA_TRY_CUDA(nsa::launch_dkdv(d, 1, q, k, v, lse_swa, delta, dO_swa, nullptr, nullptr, dk, dv, nullptr,
-                                err_word(), s));
+  NSA_TRY_CUDA(nsa::launch_dkdv(d, 1, q, k, v, lse_swa, delta, dO_swa, w + c.dO16, nullptr, nullptr,
+                                dk, dv, nullptr, err_word(), s));
   return NSA_OK;
 }
 
@@ -654,7 +656,8 @@ nsa_status cmp_bwd_body(const Dims& d, const void* q, const void* kc, const void
   NSA_TRY_CUDA(cudaMemsetAsync(dkc, 0, nkc, s));
   NSA_TRY_CUDA(cudaMemsetAsync(dvc, 0, nkc, s));
   NSA_TRY_CUDA(nsa::launch_dq(d, 2, q, kc, vc, nullptr, o_cmp, lse_cmp, dO_cmp, dq, delta, nullptr, s));
-  NSA_TRY_CUDA(nsa::launch_dkdv(d, 2, q, kc, vc, lse_cmp, delta, dO_cmp, nullptr, nullptr, dkc, dvc,
+  NSA_TRY_CUDA(nsa::launch_dkdv(d, 2, q, kc, vc, lse_cmp, delta, dO_cmp, w + c.dO16, nullptr, nullptr,
+                                dkc, dvc,
                                 (float*)(w + c.part), err_word(), s));
   NSA_TRY_CUDA(nsa::launch_pool_bwd(d, dkc, dvc, dk, dv, s));
   return NSA_OK;

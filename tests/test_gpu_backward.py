@@ -1,12 +1,12 @@
 """GPU parity of the backward: every branch's two-pass backward, the gate
 backward and the whole nsa_backward against the fp64 oracle.
 
-Small cases are compared element by element.  The training shape (B=8,
-T=8192, GQA-4) is compared on sampled dq rows (dq is local to its row) and
-on two identities that hold exactly at any size: per KV group the key
-gradients sum to zero (softmax is invariant to a constant shift of the
-logits), and the value gradients sum to the gated upstream gradient summed
-over every row that has at least one key in the branch.
+Small cases are compared element by element.  One 340M-shape
+sequence (T=8192) is compared element by element; the B=8 training shape on
+sampled dq rows (dq is local to its row) and on an identity that holds
+exactly at any size: the value gradients of a KV group sum to the gated
+upstream gradient summed over every row that has at least one key in the
+branch.
 """
 import numpy as np
 import pytest
@@ -16,7 +16,8 @@ import oracle as orc
 import sparse_attention_nsa_b200 as nsa
 from sparse_attention_nsa_b200 import inputs as W
 
-from helpers import TOL, assert_close, ocfg, to_np
+from helpers import (TOL, assert_close, assert_dgates_close, idx_mismatch_rows, ocfg,
+                     oracle_backward_given_idx, to_np)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -171,44 +172,34 @@ def test_backward_small(cuda_lib, w):
     tol = TOL[w.dtype]
     for got, ref, name in zip((dq, dk, dv), want[:3], ("dq", "dk", "dv")):
         assert_close(to_np(got), ref, tol, name)
-    # dgates = dout . o_branch is formed from the forward's STORED branch
-    # output (dtype); rounding it (RNE, relative error <= 2^-9 per element)
-    # moves the dot product by at most 2^-9 sum|dout * o|.  Bound: the
-    # dtype tolerance plus twice that.
-    do = dout.double().numpy()
-    err = np.abs(to_np(dg) - want[3])
-    for i, name in enumerate(("o_cmp", "o_sel", "o_swa")):
-        if not w.branch_mask & (1 << i):
-            assert np.all(to_np(dg)[..., i] == 0)
-            continue
-        bound = tol + (2.0 ** -8 if w.dtype == torch.bfloat16 else 2.0 ** -23) * \
-            np.abs(do * r[name]).sum(-1)
-        assert np.all(err[..., i] <= bound), f"dgates[{i}]: {float((err[..., i] - bound).max())}"
+    # dgates = dout . o_i reads the forward's stored branch outputs; the
+    # oracle reads its own outputs rounded the same way (reading R15)
+    assert_dgates_close(to_np(dg), want[3], dout.double().numpy(),
+                        (r["o_cmp"], r["o_sel"], r["o_swa"]), w, tol)
 
 
 def test_backward_training_shape_sampled(cuda_lib):
+    """B=8 training shape: dq on sampled rows.  Every sampled (row, group)
+    whose selection differs from the oracle's must be a near-tie with a
+    valid selection (its dq is then a different correct answer and is
+    excluded; at most 2 % of the sampled rows)."""
     w = W.TRAIN_340M
     inp = W.make_inputs(w, seed=0, with_dout=True)
     saved, (dq, dk, dv, dg) = gpu_fwd_bwd(w, inp, inp["dout"])
     c = ocfg(w)
     rng = np.random.default_rng(40)
     ts = sorted(set([0, 63, 64, 511, 512, 1023, 1024, 4095, w.T - 1] +
-                    list(rng.integers(0, w.T, 12))))
+                    list(rng.integers(0, w.T, 40))))
     rows = np.array([[int(rng.integers(0, w.B)), t] for t in ts])
     fr = orc.forward_rows(c, inp["q"], inp["k"], inp["v"], inp["gates"], rows)
     gi = to_np(saved["idx"])[rows[:, 0], rows[:, 1]]
-    same = np.all(gi == fr["idx"], axis=(1, 2))  # rows whose selection agrees exactly
-    assert same.mean() > 0.8
+    diff = idx_mismatch_rows(gi, fr["idx"], fr["score"], np.repeat(rows[:, 1], w.Hkv),
+                             w.topk, w.sel_block).reshape(len(rows), w.Hkv)
+    same = ~diff.any(axis=1)
+    assert (~same).sum() <= max(1, int(0.02 * len(rows))), f"{(~same).sum()} near-tie rows"
     rows = rows[same]
     want = orc.backward_dq_rows(c, inp["q"], inp["k"], inp["v"], inp["gates"], inp["dout"], rows)
     assert_close(to_np(dq)[rows[:, 0], rows[:, 1]], want, TOL[w.dtype], "dq rows")
-    # sum over keys of dk is zero for every branch, per (sequence, KV group);
-    # delta uses the stored bf16 branch output (as the ABI defines), which
-    # perturbs each row's sum by about 2^-9 of delta, hence the loose bound
-    dk_np = to_np(dk)
-    s = np.abs(dk_np.sum(axis=1))
-    scale = np.abs(dk_np).sum(axis=1)
-    assert np.all(s <= 3e-2 * scale + 1e-3), float((s / (scale + 1e-30)).max())
     # sum over keys of dv is the gated upstream gradient of every row with keys
     gates = inp["gates"].double()
     t = torch.arange(w.T)
@@ -218,3 +209,27 @@ def test_backward_training_shape_sampled(cuda_lib):
     want_dv = want_dv.sum(dim=(1, 3)).numpy()
     assert_close(to_np(dv).sum(axis=1), want_dv, 5e-2 * max(1.0, np.abs(want_dv).max()) / 10,
                  "sum dv")
+
+
+def test_backward_t8192_elementwise(cuda_lib):
+    """One 340M-shape sequence (T=8192, GQA-4, bf16): dq, dk, dv and dgates
+    element by element against the oracle's whole backward.  The GPU's
+    selection must equal the oracle's except at validated near-ties; the
+    oracle's backward is then taken on the GPU's (valid) selection, which
+    the backward holds constant, so nothing is excluded."""
+    w = W.TRAIN_340M.replace(name="bwd_340m_b1_t8192", B=1)
+    inp = W.make_inputs(w, seed=3, with_dout=True)
+    saved, (dq, dk, dv, dg) = gpu_fwd_bwd(w, inp, inp["dout"])
+    c = ocfg(w)
+    r = orc.forward(c, inp["q"], inp["k"], inp["v"], inp["gates"])
+    gi = to_np(saved["idx"])
+    t_of_row = np.broadcast_to(np.arange(w.T)[None, :, None], gi.shape[:3])
+    diff = idx_mismatch_rows(gi, r["idx"], r["score"], t_of_row, w.topk, w.sel_block)
+    assert diff.sum() <= 0.01 * diff.size, f"{diff.sum()} near-tie (token, group) rows"
+    want = oracle_backward_given_idx(c, w, inp, inp["dout"], gi)
+    tol = TOL[w.dtype]
+    for got, ref, name in zip((dq, dk, dv), want, ("dq", "dk", "dv")):
+        assert_close(to_np(got), ref, tol, name)
+    o_sel, _ = orc.sel_attn_fwd(c, inp["q"], inp["k"], inp["v"], gi)
+    assert_dgates_close(to_np(dg), want[3], inp["dout"].double().numpy(),
+                        (r["o_cmp"], o_sel, r["o_swa"]), w, tol)
