@@ -28,8 +28,10 @@
  *   queries are the LAST Tq positions of the T-key sequence: query i sits at
  *   position T - Tq + i; prefill has Tq = T, decode Tq = 1), Hq query heads,
  *   Hkv key/value heads, G = Hq / Hkv query heads per KV group (query head h
- *   reads KV head h / G), D head dim (64).  l = block size.
- *   Nc = number of compressed blocks = floor(T / l) (complete blocks only).
+ *   reads KV head h / G), D head dim (64).  l' = selection block size,
+ *   Nb = ceil(T / l') selection blocks; compressed blocks of l tokens every
+ *   d tokens (block j covers tokens [j d, j d + l)), Nc = (T - l) / d + 1
+ *   of them (complete blocks only; 0 if T < l).
  * Layouts (row-major):
  *   q, o_*, out          [B, Tq, Hq, D]   dtype
  *   k, v                 [B, T, Hkv, D]   dtype
@@ -43,7 +45,10 @@
  *   argument returns NSA_ERR_INVALID_ARG and a valid but unimplemented
  *   geometry NSA_ERR_UNSUPPORTED, with nothing launched.  A failed launch
  *   returns NSA_ERR_CUDA.  Device-side bounded waits and checks never trap:
- *   they record a code read back by nsa_last_device_error.
+ *   they record a code read back by nsa_last_device_error.  When that
+ *   returns anything but NSA_OK, the outputs of every call enqueued since
+ *   the previous check are undefined (a kernel that gave up on a wait
+ *   leaves its part of the result unwritten).
  */
 #ifndef NSA_H_
 #define NSA_H_
@@ -78,14 +83,16 @@ enum {
 
 /* Problem description.  The block geometry follows the pages' problem
  * statement: compression block size l and stride d, selection block size l',
- * top-k n, window w.  This build runs l = d = l' (the geometry used in
- * "Sparsity is Cool", Method: block 64 for both, stride = block); other
- * combinations return NSA_ERR_UNSUPPORTED. */
+ * top-k n, window w ("Sparsity is Cool", Method, uses l = d = l' = 64).
+ * Any l, d, l' >= 1 run, up to 1024 selection blocks and 1024 compressed
+ * blocks per sequence (NSA_ERR_UNSUPPORTED beyond); the bf16 tensor-core
+ * selection, window and backward kernels take l' = 64, other l' the CUDA-core
+ * kernels. */
 typedef struct {
   int B, T, Tq, Hq, Hkv, D;
   int cmp_block;   /* l  : tokens per compressed block              */
-  int cmp_stride;  /* d  : stride between compressed blocks (= l)   */
-  int sel_block;   /* l' : tokens per selection block (= l)         */
+  int cmp_stride;  /* d  : stride between compressed blocks          */
+  int sel_block;   /* l' : tokens per selection block               */
   int topk;        /* n  : selected blocks per (query, KV group), >= 2 */
   int window;      /* w  : sliding-window length in keys, >= 1      */
   float scale;     /* softmax scale, finite and > 0, normally 1/sqrt(D) */
@@ -125,8 +132,8 @@ nsa_status nsa_workspace_size(const nsa_params* p, size_t* bytes);
  * the synchronisation itself failed). */
 nsa_status nsa_last_device_error(void* stream);
 
-/* ---- compression: mean-pool consecutive blocks --------------------------
- * kc[b, j, g, :] = (1/l) * sum_{i<l} k[b, j*l + i, g, :], same for vc.
+/* ---- compression: mean-pool blocks of l tokens every d tokens ------------
+ * kc[b, j, g, :] = (1/l) * sum_{i<l} k[b, j*d + i, g, :], same for vc.
  * Passage: "Sparsity is Cool", Method and Key claims (mean-pooling replaces
  * NSA's MLP); "DeepSeek's Native Sparse Attention", COMPRESSION.
  * k, v [B, T, Hkv, D] -> kc, vc [B, Nc, Hkv, D].  The sum is exact (fp64)
@@ -136,7 +143,7 @@ nsa_status nsa_compress(const nsa_params* p, const void* k, const void* v,
 
 /* ---- compression branch and block importance ----------------------------
  * For query position t: compressed block j is visible iff its last token
- * j*l + l - 1 <= t.  P[t,h,:] = softmax over visible j of scale*q.kc_j;
+ * j*d + l - 1 <= t.  P[t,h,:] = softmax over visible j of scale*q.kc_j;
  * o_cmp = sum_j P v c_j (0 and lse = -inf when nothing is visible);
  * score[t,g,j] = sum over the G heads h of group g of P[t,h,j] (0 for
  * invisible j).  Passage: "DeepSeek's Native Sparse Attention", COMPRESSION
@@ -151,9 +158,14 @@ nsa_status nsa_cmp_attn_scores(const nsa_params* p, const void* q,
  * cur = t / l'.  If cur + 1 <= topk, idx = 0..cur then -1 padding.  Else
  * blocks 0 and cur are forced and the topk - 2 highest-scoring blocks of
  * 1..cur-1 are added (equal scores: lower block index first); idx is
- * ascending.  Passage: "DeepSeek's Native Sparse Attention", SELECTION;
- * "Sparsity is Cool", Method (block 64 / top-k 16) and Key claims (always
- * include the first block).  score [B,Tq,Hkv,Nc] -> idx [B,Tq,Hkv,topk]. */
+ * ascending.  The score of selection block j (tokens [j l', (j+1) l')) is
+ * the sum, in ascending order, of score[.., i] over the compressed blocks i
+ * whose tokens [i d, i d + l) overlap it (the pages give no rule for
+ * mapping compressed blocks onto selection blocks of another geometry; this
+ * is the plainest one, and with l = d = l' it is score[.., j] itself).
+ * Passage: "DeepSeek's Native Sparse Attention", SELECTION; "Sparsity is
+ * Cool", Method (block 64 / top-k 16) and Key claims (always include the
+ * first block).  score [B,Tq,Hkv,Nc] -> idx [B,Tq,Hkv,topk]. */
 nsa_status nsa_select_topk(const nsa_params* p, const float* score,
                            int32_t* idx, void* stream);
 
@@ -360,13 +372,15 @@ nsa_status nsa_backward(const nsa_params* p, const void* q, const void* k,
  * that loads the library until the process exits).  It allocates nothing.
  * A problem whose scratch would not fit returns NSA_ERR_SCRATCH_TOO_SMALL
  * before anything is launched (B=64 sequences, 16 heads on one KV head,
- * 32768-token caches, top-k 16, window 512 need about 11 MiB).  The first
- * call on a device looks up the array's device
- * address (with that device current) and caches it; make that first call
- * before any stream capture.  All calls on a device share the array and it
- * keeps the previous call's contents (every element is written before it
- * is read, so nothing needs clearing); calls that overlap on the GPU race
- * on it, so order them on one stream. */
+ * 32768-token caches, top-k 16, window 512 need about 11 MiB).  Every call
+ * looks up the array's device address in the current context (the caller's
+ * device must be current); the first lookup on a device may load the
+ * library's device code, so make the first call before any stream capture.
+ * All calls on a device share the array and it keeps the previous call's
+ * contents (a call reads only scratch it has written itself, so nothing
+ * needs clearing); calls that overlap on the GPU race on it, so order them
+ * on one stream.  As for every entry point, out and idx_out are undefined
+ * if nsa_last_device_error() then reports an error. */
 nsa_status nsa_decode_noalloc(const nsa_params* p, const void* q,
                               const void* k_cache, const void* v_cache,
                               const void* kc_cache, const void* vc_cache,

@@ -133,6 +133,18 @@ def cmp_attn_scores(cfg: Cfg, q, kc, vc):
     return o, lse, score
 
 
+def sel_block_scores(cfg: Cfg, score):
+    """Importance of every selection block [B, T, Hkv, Nb] from the
+    compressed-block scores [B, T, Hkv, Nc] (the ranking top-k uses)."""
+    lib = _load()
+    score = _f64(score)
+    nb = -(-cfg.T // cfg.sel_block)
+    out = np.zeros((cfg.B, cfg.T, cfg.Hkv, nb))
+    cc = cfg.c()
+    lib.orc_sel_scores(C.byref(cc), _p(score), _p(out))
+    return out
+
+
 def select_topk(cfg: Cfg, score):
     """Per-(token, KV group) block indices [B, T, Hkv, topk], -1 padded."""
     lib = _load()

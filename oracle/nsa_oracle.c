@@ -267,6 +267,31 @@ static void orc_scores_token(const orc_cfg* c, const double* q_tok,
 /* (always include the first block); "DeepSeek's Native Sparse         */
 /* Attention", SELECTION.                                              */
 /* ------------------------------------------------------------------ */
+/* Importance of selection block j for one (token, KV group): the sum of
+ * the importances of the compressed blocks whose tokens overlap it
+ * (compressed block i covers [i*d, i*d + l), selection block j covers
+ * [j*l', (j+1)*l')); blocks not yet complete have importance 0. */
+static double sel_block_importance(const orc_cfg* c, const double* cmp_score_row, int j) {
+  const int nc = orc_num_cmp_blocks(c);
+  const long lo = (long)j * c->sel_block, hi = lo + c->sel_block; /* [lo, hi) */
+  double acc = 0.0;
+  for (int i = 0; i < nc; ++i) {
+    const long clo = (long)i * c->cmp_stride, chi = clo + c->cmp_block;
+    if (clo < hi && chi > lo) acc += cmp_score_row[i];
+  }
+  return acc;
+}
+
+/* The selection-block importances of every row: score [B, T, Hkv, Nc] ->
+ * out [B, T, Hkv, Nb] (Nb = ceil(T / l')). */
+void orc_sel_scores(const orc_cfg* c, const double* score, double* out) {
+  const int nc = orc_num_cmp_blocks(c), nb = orc_num_sel_blocks(c);
+  const long rows = (long)c->B * c->T * c->Hkv;
+  for (long r = 0; r < rows; ++r)
+    for (int j = 0; j < nb; ++j)
+      out[(size_t)r * nb + j] = sel_block_importance(c, score + (size_t)r * nc, j);
+}
+
 static void orc_topk_row(const orc_cfg* c, const double* cmp_score_row, int t,
                          int* idx_row) {
   const int n = c->topk;
@@ -278,17 +303,8 @@ static void orc_topk_row(const orc_cfg* c, const double* cmp_score_row, int t,
   }
   /* selection-block importances from the compressed blocks that overlap
      each selection block (blocks not yet complete have importance 0) */
-  const int nc = orc_num_cmp_blocks(c);
   double* score_row = (double*)malloc(sizeof(double) * (size_t)(cur + 1));
-  for (int j = 0; j <= cur; ++j) {
-    const long lo = (long)j * c->sel_block, hi = lo + c->sel_block; /* [lo, hi) */
-    double acc = 0.0;
-    for (int i = 0; i < nc; ++i) {
-      const long clo = (long)i * c->cmp_stride, chi = clo + c->cmp_block;
-      if (clo < hi && chi > lo) acc += cmp_score_row[i];
-    }
-    score_row[j] = acc;
-  }
+  for (int j = 0; j <= cur; ++j) score_row[j] = sel_block_importance(c, cmp_score_row, j);
   /* rank the non-forced causal blocks 1..cur-1 by (score desc, index asc)
      with a plain selection sort; keep the first n-2. */
   const int m = cur - 1;

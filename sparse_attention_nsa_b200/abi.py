@@ -52,7 +52,9 @@ class Params(C.Structure):
 
     @property
     def Nc(self) -> int:
-        return self.T // self.cmp_block
+        if self.T < self.cmp_block:
+            return 0
+        return (self.T - self.cmp_block) // self.cmp_stride + 1
 
     @property
     def G(self) -> int:

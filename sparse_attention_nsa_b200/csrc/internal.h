@@ -10,8 +10,10 @@ namespace nsa {
 // Validated, derived problem sizes (see nsa.h for the meaning of each).
 struct Dims {
   int B, T, Tq, Hq, Hkv, D, G;
-  int l;       // block size (compression = selection = stride)
-  int Nc;      // complete compressed blocks: T / l
+  int l;       // selection block size l'
+  int lc;      // compression block size l
+  int dc;      // compression stride d
+  int Nc;      // complete compressed blocks: (T - lc) / dc + 1 (0 if T < lc)
   int Nb;      // selection blocks: ceil(T / l)
   int topk;
   int window;
@@ -20,6 +22,20 @@ struct Dims {
   int branch_mask;
   int q_off;   // position of query 0: T - Tq
 };
+
+// Compressed blocks complete at position t: block c covers tokens
+// [c dc, c dc + lc) and is visible to the query at t once c dc + lc - 1 <= t.
+__host__ __device__ inline int cmp_nvis(const Dims& d, int t) {
+  if (t + 1 < d.lc) return 0;
+  const int n = (t + 1 - d.lc) / d.dc + 1;
+  return n < d.Nc ? n : d.Nc;
+}
+
+// Compression block = stride = selection block: compressed block j scores
+// selection block j directly (no remap of the scores).
+__host__ __device__ inline bool plain_geometry(const Dims& d) {
+  return d.lc == d.l && d.dc == d.l;
+}
 
 // Each launcher enqueues on `s` and returns the launch status.  `err` is
 // the device error word (may be NULL).

@@ -165,7 +165,7 @@ dq_kernel(const T* __restrict__ q, const T* __restrict__ keys, const T* __restri
     } else if (MODE == kBwdSwa) {
       fold(max(0, t - d.window + 1), t + 1);
     } else {
-      fold(0, min((t + 1) / d.l, d.Nc));
+      fold(0, cmp_nvis(d, t));
     }
   }
   dq[row * 64 + lane] += a0 * d.scale;
@@ -542,7 +542,7 @@ dkdv_kernel(const T* __restrict__ q, const T* __restrict__ keys, const T* __rest
     tq_lo = max(0, t_lo - d.q_off);
     n_tok = max(0, t_hi - d.q_off - tq_lo + 1);
   } else {
-    const int t_lo = (j * kKB) * d.l + d.l - 1;  // first query that sees the chunk
+    const int t_lo = (j * kKB) * d.dc + d.lc - 1;  // first query that sees the chunk
     tq_lo = max(0, t_lo - d.q_off);
     n_tok = max(0, d.Tq - tq_lo);
   }
@@ -583,7 +583,7 @@ dkdv_kernel(const T* __restrict__ q, const T* __restrict__ keys, const T* __rest
       bool vis;
       if (MODE == kBwdSel) vis = s <= t;
       else if (MODE == kBwdSwa) vis = s <= t && s >= t - d.window + 1;
-      else vis = s * d.l + d.l - 1 <= t;
+      else vis = s * d.dc + d.lc - 1 <= t;
       vis = vis && key_ok && lse_s[rr] != -INFINITY;
       const float p = vis ? exp2f(qk * sl2 - lse_s[rr]) : 0.f;
       const float ds = p * (dp - del_s[rr]);
@@ -605,23 +605,32 @@ dkdv_kernel(const T* __restrict__ q, const T* __restrict__ keys, const T* __rest
   }
 }
 
-// dk[t] += dkc[t / l] / l for the tokens of complete blocks (mean-pool backward)
+// Mean-pool backward: compressed block c covers tokens [c dc, c dc + lc), so
+// dk[t] += sum over the blocks c covering t of dkc[c] / lc (ascending c),
+// same for dv; tokens that no complete block covers get nothing.
 __global__ void pool_bwd_kernel(const float* __restrict__ dkc, const float* __restrict__ dvc,
                                 float* __restrict__ dk, float* __restrict__ dv, Dims d) {
   const long e = (long)blockIdx.x * blockDim.x + threadIdx.x;
   const long row_elems = (long)d.Hkv * 64;
-  const long n = (long)d.B * d.Nc * d.l * row_elems;
+  const long n = (long)d.B * d.T * row_elems;
   if (e >= n) return;
   const long c = e % row_elems;
-  const long tok = e / row_elems;  // b * (Nc * l) + t
-  const int t = (int)(tok % ((long)d.Nc * d.l));
-  const int b = (int)(tok / ((long)d.Nc * d.l));
-  const int jc = t / d.l;
-  const float inv = 1.f / (float)d.l;
-  const size_t src = ((size_t)b * d.Nc + jc) * row_elems + c;
+  const long tok = e / row_elems;  // b * T + t
+  const int t = (int)(tok % d.T);
+  const int b = (int)(tok / d.T);
+  const int chi = min(t / d.dc, d.Nc - 1);                       // last block starting <= t
+  const int clo = t < d.lc ? 0 : (t - d.lc) / d.dc + 1;          // first block ending after t
+  if (clo > chi) return;
+  float sk = 0.f, sv = 0.f;
+  for (int jc = clo; jc <= chi; ++jc) {
+    const size_t src = ((size_t)b * d.Nc + jc) * row_elems + c;
+    sk += dkc[src];
+    sv += dvc[src];
+  }
+  const float inv = 1.f / (float)d.lc;
   const size_t dst = ((size_t)b * d.T + t) * row_elems + c;
-  dk[dst] += dkc[src] * inv;
-  dv[dst] += dvc[src] * inv;
+  dk[dst] += sk * inv;
+  dv[dst] += sv * inv;
 }
 
 // ---- launchers ----------------------------------------------------------------------
@@ -736,7 +745,7 @@ cudaError_t launch_dkdv(const Dims& d, int mode, const void* q, const void* keys
 
 cudaError_t launch_pool_bwd(const Dims& d, const float* dkc, const float* dvc, float* dk,
                             float* dv, cudaStream_t s) {
-  const long n = (long)d.B * d.Nc * d.l * d.Hkv * 64;
+  const long n = d.Nc == 0 ? 0 : (long)d.B * d.T * d.Hkv * 64;
   if (n == 0) return cudaSuccess;
   pool_bwd_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(dkc, dvc, dk, dv, d);
   return cudaGetLastError();

@@ -179,7 +179,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       blk[0] = jlo;
       *nblk_s = tlast / d.l - jlo + 1;
     } else {  // compressed keys 0 .. (tlast + 1) / l - 1, in 64-key chunks
-      const int cmax = min((tlast + 1) / d.l, d.Nc) - 1;
+      const int cmax = cmp_nvis(d, tlast) - 1;
       blk[0] = 0;
       *nblk_s = cmax < 0 ? 0 : cmax / kKeys + 1;
     }
@@ -298,7 +298,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       mbar_arrive(&bars->dorows);
     }
     const int lo = MODE == 1 ? max(0, t - d.window + 1) : 0;
-    const int khi = MODE == 2 ? min((t + 1) / d.l, d.Nc) - 1 : t;  // last visible key
+    const int khi = MODE == 2 ? cmp_nvis(d, t) - 1 : t;  // last visible key
     const int* lst = SEL ? toks + tl * (d.topk + 1) : nullptr;
     int ptr = 0;
     int nxt = SEL && valid ? lst[0] : INT_MAX;
@@ -542,7 +542,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
       tq_lo = max(0, t_lo - d.q_off);
       ntok = max(0, t_hi - d.q_off - tq_lo + 1);
     } else {  // every query from the one that completes compressed block kbase on
-      tq_lo = max(0, (kbase + 1) * d.l - 1 - d.q_off);
+      tq_lo = max(0, kbase * d.dc + d.lc - 1 - d.q_off);
       ntok = max(0, d.Tq - tq_lo);
     }
     ntiles_all = (int)(((long)ntok * d.G + 127) / 128);
@@ -652,7 +652,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
           lo0 = lo1 = max(0, t - d.window + 1);
           sp0 = sp1 = t - lo0;
         } else {
-          const int khi = (t + 1) / d.l - 1;  // last complete compressed block
+          const int khi = cmp_nvis(d, t) - 1;  // last complete compressed block
           if (khi >= 0) {
             lo0 = lo1 = 0;
             sp0 = sp1 = khi;

@@ -34,7 +34,7 @@ cmp_scores_kernel(const T* __restrict__ q, const T* __restrict__ kc,
   const int g = blockIdx.y, b = blockIdx.z;
   if (tq >= d.Tq) return;
   const int t = d.q_off + tq;
-  const int nvis = min((t + 1) / d.l, d.Nc);
+  const int nvis = cmp_nvis(d, t);
   const float sl2 = d.scale * kLog2e;
   for (int j = lane; j < d.Nc; j += 32) sacc[j] = 0.f;
   const size_t row = (size_t)d.Hkv * 64;  // elements between consecutive kc rows

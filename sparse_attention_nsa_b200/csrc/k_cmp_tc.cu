@@ -90,7 +90,7 @@ cmp_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   const int g = blockIdx.y, b = blockIdx.z;
   const int nvalid = min(TQ, d.Tq - t0);
   const int pos0 = d.q_off + t0;
-  const int nvis_max = min((pos0 + nvalid) / d.l, d.Nc);  // of the tile's last token
+  const int nvis_max = nvalid > 0 ? cmp_nvis(d, pos0 + nvalid - 1) : 0;  // of the tile's last token
   const int n = (nvis_max + kChunk - 1) / kChunk;
   // with at most two chunks both S tiles stay in TMEM: pass 2 re-reads them
   // instead of recomputing, and each chunk's Kc and Vc are loaded once
@@ -194,7 +194,7 @@ cmp_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const int tl = r / d.G, hh = r % d.G;
     const bool valid = tl < nvalid;
     const int t = pos0 + tl;
-    const int nvis = valid ? min((t + 1) / d.l, d.Nc) : 0;
+    const int nvis = valid ? cmp_nvis(d, t) : 0;
     const float sl2 = d.scale * kLog2e;
     const uint32_t lane_tmem = tmem + ((uint32_t)(warp * 32) << 16);
     float m = -INFINITY, lsum = 0.f;
@@ -406,7 +406,7 @@ cudaError_t launch_cmp_tc(const Dims& d, const void* q, const void* kc, const vo
 cudaError_t launch_cmp_scores(const Dims& d, const void* q, const void* kc, const void* vc,
                               void* o_cmp, float* lse_cmp, float* score, int* err,
                               cudaStream_t s) {
-  const bool tc = d.dtype == 1 && d.l == 64 && d.Nc > 0 && kRows % d.G == 0 &&
+  const bool tc = d.dtype == 1 && d.Nc > 0 && kRows % d.G == 0 &&
                   tmap_encode_fn() != nullptr;
   if (!tc) return launch_cmp_scores_simt(d, q, kc, vc, o_cmp, lse_cmp, score, s);
   if (o_cmp) return launch_cmp_tc<true>(d, q, kc, vc, o_cmp, lse_cmp, score, err, s);

@@ -19,7 +19,7 @@ namespace nsa {
 template <typename T>
 __global__ void compress_kernel(const T* __restrict__ k, const T* __restrict__ v,
                                 T* __restrict__ kc, T* __restrict__ vc, int T_,
-                                int Hkv, int l, int Nc) {
+                                int Hkv, int l, int stride, int Nc) {
   constexpr int VEC = 16 / sizeof(T);
   extern __shared__ double part[];  // [R][row_elems]
   const int row_elems = Hkv * 64;
@@ -33,7 +33,7 @@ __global__ void compress_kernel(const T* __restrict__ k, const T* __restrict__ v
   double acc[VEC];
 #pragma unroll
   for (int i = 0; i < VEC; ++i) acc[i] = 0.0;
-  const T* base = src + ((size_t)b * T_ + (size_t)j * l) * row_elems + (size_t)col * VEC;
+  const T* base = src + ((size_t)b * T_ + (size_t)j * stride) * row_elems + (size_t)col * VEC;
   // all of this thread's rows are loaded before any is summed
   constexpr int kMaxRows = 8;
   uint4 raw[kMaxRows];
@@ -81,7 +81,7 @@ static cudaError_t launch_compress_t(const Dims& d, const void* k, const void* v
     if (e != cudaSuccess) return e;
   }
   compress_kernel<T><<<dim3(d.Nc, d.B, 2), threads, smem, s>>>(
-      (const T*)k, (const T*)v, (T*)kc, (T*)vc, d.T, d.Hkv, d.l, d.Nc);
+      (const T*)k, (const T*)v, (T*)kc, (T*)vc, d.T, d.Hkv, d.lc, d.dc, d.Nc);
   return cudaGetLastError();
 }
 

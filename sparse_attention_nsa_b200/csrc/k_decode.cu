@@ -575,7 +575,8 @@ int window_blocks(const Dims& d, int* jlo) {
 // group (the 16 MMA rows), up to 1024 compressed blocks (the top-k warp's
 // registers) and one query.
 bool decode_split_eligible(const Dims& d) {
-  if (!(d.Tq == 1 && d.dtype == 1 && d.l == 64 && d.D == 64 && d.G <= 16 && d.Nc <= 1024 &&
+  if (!(d.Tq == 1 && d.dtype == 1 && d.l == 64 && plain_geometry(d) && d.D == 64 && d.G <= 16 &&
+        d.Nc <= 1024 &&
         tmap_encode_fn() != nullptr))
     return false;
   int jlo = 0;

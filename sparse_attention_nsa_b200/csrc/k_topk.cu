@@ -10,7 +10,14 @@
 // output is ascending and padded with -1.
 //
 // One warp per row, no shared memory: the radix select of topk.cuh over the
-// row's fp32 scores read straight from global memory.
+// row's fp32 scores read straight from global memory.  With a compression
+// block or stride other than the selection block ("Sparsity is Cool",
+// Method, and "DeepSeek's Native Sparse Attention", COMPRESSION, give block
+// size and stride as parameters), the importance of selection block j is
+// the sum, in ascending order, of the scores of the compressed blocks whose
+// tokens overlap it (compressed block i covers [i dc, i dc + lc), selection
+// block j covers [j l, (j + 1) l)); the sum is formed as each candidate's
+// key is loaded.
 #include <climits>
 
 #include "common.cuh"
@@ -31,7 +38,20 @@ topk_kernel(const float* __restrict__ score, int32_t* __restrict__ idx, Dims d) 
   for (int b = blockIdx.y; b < d.B; b += gridDim.y) {
     const size_t r = (size_t)b * d.Tq * d.Hkv + rb;
     // candidates are blocks 1..cur-1 (all complete, so all have scores)
-    warp_select_blocks<QMAX>(score + r * d.Nc, t / d.l, d.topk, idx + r * d.topk, lane);
+    const float* row = score + r * d.Nc;
+    if (plain_geometry(d)) {
+      warp_select_blocks<QMAX>(row, t / d.l, d.topk, idx + r * d.topk, lane);
+    } else {
+      auto remap = [row, &d](int j) {
+        const int lo = j * d.l;  // selection block j: tokens [lo, lo + l)
+        const int ilo = lo < d.lc ? 0 : (lo - d.lc) / d.dc + 1;
+        const int ihi = min((lo + d.l - 1) / d.dc, d.Nc - 1);
+        float acc = 0.f;
+        for (int i = ilo; i <= ihi; ++i) acc += row[i];
+        return acc;
+      };
+      warp_select_blocks_fn<QMAX>(remap, t / d.l, d.topk, idx + r * d.topk, lane);
+    }
   }
 }
 

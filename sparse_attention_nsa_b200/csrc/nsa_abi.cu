@@ -52,14 +52,13 @@ nsa_status fill_dims(const nsa_params* p, Dims* d) {
   if (!(p->scale > 0.f) || p->scale == INFINITY) return NSA_ERR_INVALID_ARG;
   // valid NSA geometry, but outside what this build runs
   if (p->D != 64) return NSA_ERR_UNSUPPORTED;
-  if (p->cmp_stride != p->cmp_block || p->sel_block != p->cmp_block)
-    return NSA_ERR_UNSUPPORTED;
   const int G = p->Hq / p->Hkv;
   if (G > 32 || (G & (G - 1)) != 0) return NSA_ERR_UNSUPPORTED;
   if (p->Hkv > 64 || p->topk > 64) return NSA_ERR_UNSUPPORTED;
-  const int l = p->cmp_block;
+  const int l = p->sel_block;
   const int Nb = (p->T + l - 1) / l;
-  if (Nb > 1024) return NSA_ERR_UNSUPPORTED;
+  const int Nc = p->T < p->cmp_block ? 0 : (p->T - p->cmp_block) / p->cmp_stride + 1;
+  if (Nb > 1024 || Nc > 1024) return NSA_ERR_UNSUPPORTED;
   d->B = p->B;
   d->T = p->T;
   d->Tq = p->Tq;
@@ -68,7 +67,9 @@ nsa_status fill_dims(const nsa_params* p, Dims* d) {
   d->D = p->D;
   d->G = G;
   d->l = l;
-  d->Nc = p->T / l;
+  d->lc = p->cmp_block;
+  d->dc = p->cmp_stride;
+  d->Nc = Nc;
   d->Nb = Nb;
   d->topk = p->topk;
   d->window = p->window;

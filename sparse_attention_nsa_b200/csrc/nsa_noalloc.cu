@@ -12,11 +12,10 @@
 // The array (kNoAllocScratchBytes) is a file-scope __device__ object: every
 // GPU that loads the library holds it until the process exits.  All calls
 // on a device share it and it keeps the previous call's contents; decode
-// writes every scratch element before reading it, so nothing needs
-// clearing.  Calls whose executions overlap on the GPU (different streams,
-// or different host threads without ordering) race on the array.
-#include <mutex>
-
+// writes every scratch element it reads in the same call (stale values from
+// an earlier call are never read), so nothing needs clearing.  Calls whose
+// executions overlap on the GPU (different streams, or different host
+// threads without ordering) race on the array.
 #include "common.cuh"
 #include "internal.h"
 #include "nsa.h"
@@ -31,23 +30,17 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 
 namespace {
 
-constexpr int kMaxDev = 64;
-std::mutex g_scratch_mu;
-void* g_scratch_ptr[kMaxDev] = {};
-
-// Device address of the scratch array on the current device.  In host code
-// the array's name only stands for it; the real address is looked up once
-// per device, with that device current, and cached.
+// Device address of the scratch array in the current context.  In host code
+// the array's name only stands for it: the address is looked up on every
+// call, with the caller's device current, so a call never uses an address
+// taken in another context (another device, a context the caller made
+// current itself, or one created again after a device reset).  Only the
+// first lookup in a context does real work (it may load the library's
+// device code): make the first call on a device before any stream capture.
 nsa_status scratch_ptr(void** out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return NSA_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return NSA_ERR_CUDA;
-    g_scratch_ptr[dev] = p;
-  }
-  *out = g_scratch_ptr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return NSA_ERR_CUDA;
+  *out = p;
   return NSA_OK;
 }
 

@@ -27,11 +27,11 @@ __device__ __forceinline__ uint32_t order_key(float x) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// score[j] for j in 1..cur-1 must be readable (global or shared memory);
+// score(j) gives the importance of selection block j for j in 1..cur-1;
 // QMAX * 32 must cover cur.  All 32 lanes call; out receives topk entries.
-template <int QMAX>
-__device__ __forceinline__ void warp_select_blocks(const float* score, int cur, int topk,
-                                                   int32_t* out, int lane) {
+template <int QMAX, typename Score>
+__device__ __forceinline__ void warp_select_blocks_fn(Score score, int cur, int topk,
+                                                      int32_t* out, int lane) {
   if (cur + 1 <= topk) {
     for (int s = lane; s < topk; s += 32) out[s] = s <= cur ? s : -1;
     return;
@@ -40,7 +40,7 @@ __device__ __forceinline__ void warp_select_blocks(const float* score, int cur, 
 #pragma unroll
   for (int q = 0; q < QMAX; ++q) {
     const int j = 1 + lane + 32 * q;
-    key[q] = j < cur ? order_key(score[j]) : 0u;
+    key[q] = j < cur ? order_key(score(j)) : 0u;
   }
   const int K2 = topk - 2;
   // tau = the largest value with at least K2 keys >= tau.  Absent slots hold
@@ -92,6 +92,13 @@ __device__ __forceinline__ void warp_select_blocks(const float* score, int cur, 
     out[0] = 0;
     out[K2 + 1] = cur;
   }
+}
+
+// score[j] for j in 1..cur-1 readable (global or shared memory).
+template <int QMAX>
+__device__ __forceinline__ void warp_select_blocks(const float* score, int cur, int topk,
+                                                   int32_t* out, int lane) {
+  warp_select_blocks_fn<QMAX>([score](int j) { return score[j]; }, cur, topk, out, lane);
 }
 
 }  // namespace nsa

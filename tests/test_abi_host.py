@@ -54,9 +54,25 @@ BAD = [
     (dict(topk=1), 1), (dict(window=0), 1), (dict(dtype=7), 1), (dict(branch_mask=0), 1),
     (dict(branch_mask=9), 1), (dict(scale=float("nan")), 1), (dict(scale=-0.125), 1), (dict(scale=0.0), 1),
     (dict(scale=float("inf")), 1),
-    (dict(D=128), 2), (dict(cmp_stride=32), 2), (dict(sel_block=32), 2),
+    (dict(D=128), 2), (dict(cmp_stride=2), 2), (dict(sel_block=2), 2),
     (dict(Hq=24, Hkv=4), 2), (dict(topk=65), 2), (dict(T=200000), 2),
 ]
+
+
+@pytest.mark.parametrize("change", [dict(cmp_stride=32), dict(sel_block=32),
+                                    dict(cmp_block=128, cmp_stride=64, sel_block=64),
+                                    dict(cmp_block=32, cmp_stride=16, sel_block=64),
+                                    dict(cmp_block=16, cmp_stride=8, sel_block=32)])
+def test_general_block_geometry_accepted(change):
+    """Compression block and stride other than the selection block run
+    (reading R14: a selection block's importance is summed over the
+    compressed blocks that overlap it)."""
+    p = nsa.make_params(1, 4096, 16, 4)
+    for k, v in change.items():
+        setattr(p, k, v)
+    assert nsa.nsa_check_params(p) == 0
+    assert nsa.nsa_workspace_size(p) > 0
+    assert nsa.nsa_backward_workspace_size(p) > 0
 
 
 @pytest.mark.parametrize("change,code", BAD)

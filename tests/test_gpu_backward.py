@@ -43,6 +43,14 @@ BWD = [
           sel_block=128, topk=3, window=200),
     small("bwd_pruned_mqa_t500_bf16", T=500, Hkv=1, topk=4, window=64,
           branch_mask=W.BR_SEL | W.BR_SWA, cmp_gate_zero=True, qk_norm=False),
+    # general geometry: overlapping compressed blocks (stride < block), and
+    # compression blocks of another size than the selection block
+    small("bwd_geo_l32_d16_s64_t700_bf16", T=700, cmp_block=32, cmp_stride=16, topk=5,
+          window=150),
+    small("bwd_geo_l128_d64_s64_mqa_t900_bf16", T=900, Hkv=1, cmp_block=128, cmp_stride=64,
+          topk=4, window=100, qk_norm=False),
+    small("bwd_geo_l16_d8_s32_t300_f32", T=300, Hq=4, Hkv=2, cmp_block=16, cmp_stride=8,
+          sel_block=32, topk=4, window=50, dtype=torch.float32, qk_norm=False, qkv_std=0.5),
 ]
 
 
@@ -106,7 +114,8 @@ def test_swa_bwd(cuda_lib, w):
         assert_close(to_np(got), ref, TOL[w.dtype], name)
 
 
-@pytest.mark.parametrize("w", BWD[:7] + [small("bwd_short_T40", T=40)], ids=lambda w: w.name)
+@pytest.mark.parametrize("w", BWD[:7] + BWD[8:] + [small("bwd_short_T40", T=40)],
+                         ids=lambda w: w.name)
 def test_cmp_bwd(cuda_lib, w):
     inp = W.make_inputs(w, seed=35)
     c = ocfg(w)

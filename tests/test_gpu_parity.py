@@ -84,7 +84,8 @@ def compare_forward(w, r, out, saved, t0=0):
         gi = to_np(saved["idx"])
         t_rows = np.broadcast_to((np.arange(gi.shape[1]) + t0)[None, :, None],
                                  gi.shape[:3])
-        diff = idx_mismatch_rows(gi, r["idx"][:, sl], r["score"][:, sl], t_rows, w.topk,
+        ssel = orc.sel_block_scores(ocfg(w), r["score"])  # ranking the top-k uses
+        diff = idx_mismatch_rows(gi, r["idx"][:, sl], ssel[:, sl], t_rows, w.topk,
                                  w.sel_block)
         bad = diff.reshape(gi.shape[:3]).any(-1)
         assert bad.mean() < 0.01
@@ -287,6 +288,11 @@ def check_decode(w, inp, seqs):
     o_ref, i_ref, s_ref = orc.decode(c, inp["q"][seqs], kcache, vcache, okc, ovc,
                                      inp["gates"][seqs], with_score=True)
     if w.branch_mask & W.BR_SEL:  # idx_out is written when selection runs
+        if (w.cmp_block, w.cmp_stride) != (w.sel_block, w.sel_block):
+            # the selection-block importances the top-k ranks (query at T-1)
+            full = np.zeros((len(seqs), w.T, w.Hkv, w.Nc))
+            full[:, w.T - 1] = s_ref
+            s_ref = orc.sel_block_scores(c, full)[:, w.T - 1]
         diff = idx_mismatch_rows(to_np(idx)[seqs], i_ref, s_ref,
                                  np.full(len(seqs) * w.Hkv, w.T - 1), w.topk, w.sel_block)
         keep = ~diff.reshape(len(seqs), w.Hkv).any(-1)
@@ -310,6 +316,76 @@ def check_decode(w, inp, seqs):
 ], ids=lambda w: w.name)
 def test_decode_small(cuda_lib, w):
     inp = W.make_decode_inputs(w, seed=13)
+    check_decode(w, inp, list(range(w.B)))
+
+
+# ------------------------------------------------------------------ general geometry
+# Compression block l and stride d other than the selection block l' (the
+# pages give block size and stride as parameters): overlapping compressed
+# blocks, and a selection block's importance summed over the compressed
+# blocks that overlap it (reading R14).
+GEOM = [
+    small("geo_l32_d16_s64_gqa4_t900_bf16", T=900, cmp_block=32, cmp_stride=16, topk=5,
+          window=150),
+    small("geo_l64_d32_s64_gqa4_t1000_bf16", T=1000, cmp_block=64, cmp_stride=32, topk=5,
+          window=200),
+    small("geo_l128_d64_s64_mqa_t1300_bf16", T=1300, Hkv=1, cmp_block=128, cmp_stride=64,
+          topk=6, window=100, qk_norm=False),
+    small("geo_l16_d8_s32_gqa2_t300_f32", T=300, Hq=4, Hkv=2, cmp_block=16, cmp_stride=8,
+          sel_block=32, topk=4, window=50, dtype=torch.float32, qk_norm=False, qkv_std=0.5),
+    # block-major selection (Nb >= 8 top-k) with stride < block
+    small("geo_l64_d32_s64_gqa4_t4200_k4_bf16", T=4200, cmp_block=64, cmp_stride=32, topk=4,
+          window=128),
+]
+
+
+@pytest.mark.parametrize("w", GEOM, ids=lambda w: w.name)
+def test_compress_general_geometry(cuda_lib, w):
+    inp = W.make_inputs(w, seed=41)
+    d = dev(inp)
+    kc = torch.empty((w.B, w.Nc, w.Hkv, w.D), dtype=w.dtype, device=DEV)
+    vc = torch.empty_like(kc)
+    nsa.nsa_compress(nsa.params_for(w), d["k"], d["v"], kc, vc)
+    okc, ovc = orc.compress(ocfg(w), inp["k"], inp["v"])
+    if w.dtype == torch.bfloat16:
+        np.testing.assert_array_equal(to_np(kc), okc)
+        np.testing.assert_array_equal(to_np(vc), ovc)
+    else:
+        assert_close(to_np(kc), okc, 1e-6, "kc")
+        assert_close(to_np(vc), ovc, 1e-6, "vc")
+
+
+@pytest.mark.parametrize("w", GEOM, ids=lambda w: w.name)
+def test_forward_general_geometry(cuda_lib, w):
+    inp = W.make_inputs(w, seed=42)
+    r = orc.forward(ocfg(w), inp["q"], inp["k"], inp["v"], inp["gates"])
+    out, saved = gpu_forward(w, inp)
+    compare_forward(w, r, out, saved)
+
+
+def test_topk_general_geometry_on_oracle_scores(cuda_lib):
+    """The top-k's score remap alone, on scores drawn in fp32: the GPU sums
+    the overlapping compressed blocks in fp32, so only near-ties may differ."""
+    w = small("geo_topk_l32_d16", T=2000, cmp_block=32, cmp_stride=16, topk=8)
+    c = ocfg(w)
+    g = np.random.default_rng(43)
+    score = g.random((w.B, w.T, w.Hkv, w.Nc)).astype(np.float32).astype(np.float64)
+    want = orc.select_topk(c, score)
+    idx = torch.empty((w.B, w.T, w.Hkv, w.topk), dtype=torch.int32, device=DEV)
+    nsa.nsa_select_topk(nsa.params_for(w), torch.from_numpy(score).float().to(DEV), idx)
+    t_rows = np.broadcast_to(np.arange(w.T)[None, :, None], (w.B, w.T, w.Hkv))
+    diff = idx_mismatch_rows(to_np(idx), want, orc.sel_block_scores(c, score), t_rows, w.topk,
+                             w.sel_block)
+    assert diff.mean() < 0.01
+
+
+@pytest.mark.parametrize("w", [
+    W.DECODE_32K.replace(name="decode_geo_l32_d16", B=3, T=2500, cmp_block=32, cmp_stride=16),
+    W.DECODE_32K.replace(name="decode_geo_l128_d64_gqa4", B=2, T=3001, Hq=16, Hkv=4,
+                         cmp_block=128, cmp_stride=64),
+], ids=lambda w: w.name)
+def test_decode_general_geometry(cuda_lib, w):
+    inp = W.make_decode_inputs(w, seed=44)
     check_decode(w, inp, list(range(w.B)))
 
 

@@ -228,6 +228,26 @@ def test_topk_general_geometry_brute_force(l, d, ls):
                 assert idx[b, t, h].tolist() == want, (b, t, h)
 
 
+@pytest.mark.parametrize("l,d,ls", [(4, 2, 8), (8, 8, 8), (6, 4, 8), (32, 16, 64)])
+def test_sel_block_scores_are_token_overlap_sums(l, d, ls):
+    """The exported selection-block importances equal the token-set
+    intersection sums (for l = d = l' the compressed scores themselves,
+    and 0 for a selection block with no complete compressed block)."""
+    c = cfg_small(T=130, cmp_block=l, cmp_stride=d, sel_block=ls, topk=4, Hkv=2)
+    g = np.random.default_rng(9)
+    score = g.random((c.B, c.T, c.Hkv, c.Nc))
+    got = orc.sel_block_scores(c, score)
+    nb = -(-c.T // ls)
+    assert got.shape == (c.B, c.T, c.Hkv, nb)
+    cmp_tokens = [set(range(i * d, i * d + l)) for i in range(c.Nc)]
+    for j in range(nb):
+        over = [i for i in range(c.Nc) if cmp_tokens[i] & set(range(j * ls, (j + 1) * ls))]
+        want = score[..., over].sum(-1) if over else np.zeros(score.shape[:3])
+        np.testing.assert_allclose(got[..., j], want, rtol=1e-15, atol=0)
+    if l == d == ls:
+        np.testing.assert_array_equal(got[..., :c.Nc], score)
+
+
 def test_topk_general_geometry_hand_cases():
     """Hand-derived: with l = 4, d = 2 a compressed block i covers tokens
     [2i, 2i + 4), so for selection blocks of 4 tokens block j collects the
