@@ -333,3 +333,17 @@ def backward_dq_rows(cfg: Cfg, q, k, v, gates, dout, rows, kc=None, vc=None):
     lib.orc_backward_dq_rows(C.byref(cc), _p(q), _p(k), _p(v), _p(gates), _p(dout), _p(kc),
                              _p(vc), C.c_int(rows.shape[0]), _p(rows), _p(dq))
     return dq
+
+
+def moba_fwd(cfg: Cfg, q, k, v):
+    """MoBA block attention (cfg.cmp_block = cfg.cmp_stride = cfg.sel_block =
+    the MoBA block size, cfg.topk = k): (o [B,T,Hq,D], lse [B,T,Hq],
+    idx [B,T,Hkv,k] MoBA block indices)."""
+    lib = _load()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    o = np.zeros((cfg.B, cfg.T, cfg.Hq, cfg.D))
+    lse = np.zeros((cfg.B, cfg.T, cfg.Hq))
+    idx = np.zeros((cfg.B, cfg.T, cfg.Hkv, cfg.topk), dtype=np.int32)
+    cc = cfg.c()
+    lib.orc_moba_fwd(C.byref(cc), _p(q), _p(k), _p(v), _p(idx), _p(o), _p(lse))
+    return o, lse, idx

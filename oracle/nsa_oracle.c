@@ -857,3 +857,90 @@ void orc_decode(const orc_cfg* c, const double* q_last, const double* kcache,
     free(sc);
   }
 }
+
+/* ================================================================== */
+/* MoBA block attention.  "Sparsity is Cool", Method (MoBA with block  */
+/* size 512 and top-k 3) and Key claims (MoBA does not always read the */
+/* first block; dense below ~1.5k tokens); "DeepSeek's Native Sparse   */
+/* Attention" newsletter, MoBA section (blocks, top-k gating that sends */
+/* each query to its most relevant blocks, causal protection).          */
+/* Readings taken where the pages are silent:                           */
+/*   - the gate of block j for query t is q . (mean of block j's keys), */
+/*     summed over the query heads of the KV group, so one selection    */
+/*     serves the group (as NSA's selection does);                      */
+/*   - the query's own block is always selected and counts toward k;    */
+/*     the complete past blocks 0 .. cur-1 compete for the other k-1;   */
+/*     with at most k causal blocks all are selected; equal gates go to */
+/*     the lower block; keys after the query are masked.                */
+/* cfg: cmp_block = cmp_stride = sel_block = the MoBA block size L;     */
+/* topk = k; kv_round rounds the mean-pooled keys as stored.            */
+/* idx [B, T, Hkv, k] MoBA block indices (ascending, -1 padded),        */
+/* o [B, T, Hq, D], lse [B, T, Hq].                                     */
+/* ================================================================== */
+static void orc_moba_select_row(const orc_cfg* c, const double* q, const double* kc, int nc,
+                                int b, int t, int g, int* idx_row) {
+  const int n = c->topk, G = c->Hq / c->Hkv, D = c->D;
+  const int cur = t / c->sel_block;
+  for (int s = 0; s < n; ++s) idx_row[s] = -1;
+  if (cur + 1 <= n) {
+    for (int j = 0; j <= cur; ++j) idx_row[j] = j;
+    return;
+  }
+  /* gates of the complete past blocks */
+  double* gate = (double*)malloc(sizeof(double) * (size_t)cur);
+  for (int j = 0; j < cur; ++j) {
+    double acc = 0.0;
+    for (int h = g * G; h < (g + 1) * G; ++h)
+      acc += dot(q + QI(c, b, t, h), kc + CI(c, nc, b, j, g), D);
+    gate[j] = acc;
+  }
+  /* the n-1 best of 0 .. cur-1 by (gate desc, index asc), selection sort */
+  int* cand = (int*)malloc(sizeof(int) * (size_t)cur);
+  for (int i = 0; i < cur; ++i) cand[i] = i;
+  for (int i = 0; i < n - 1; ++i) {
+    int best = i;
+    for (int r = i + 1; r < cur; ++r) {
+      const double gr = gate[cand[r]], gb = gate[cand[best]];
+      if (gr > gb || (gr == gb && cand[r] < cand[best])) best = r;
+    }
+    int tmp = cand[i];
+    cand[i] = cand[best];
+    cand[best] = tmp;
+  }
+  for (int i = 0; i < n - 1; ++i) idx_row[i] = cand[i];
+  idx_row[n - 1] = cur;
+  for (int i = 1; i < n; ++i) /* insertion sort, ascending */
+    for (int r = i; r > 0 && idx_row[r - 1] > idx_row[r]; --r) {
+      int tmp = idx_row[r];
+      idx_row[r] = idx_row[r - 1];
+      idx_row[r - 1] = tmp;
+    }
+  free(gate);
+  free(cand);
+}
+
+void orc_moba_fwd(const orc_cfg* c, const double* q, const double* k, const double* v,
+                  int* idx, double* o, double* lse) {
+  const int nc = orc_num_cmp_blocks(c);
+  const int G = c->Hq / c->Hkv;
+  const size_t nkc = (size_t)c->B * (nc + 1) * c->Hkv * c->D;
+  double* kc = (double*)malloc(nkc * sizeof(double));
+  double* vc = (double*)malloc(nkc * sizeof(double)); /* pooled values: unused */
+  orc_compress(c, k, v, kc, vc);
+#pragma omp parallel for collapse(2) schedule(dynamic, 16)
+  for (int b = 0; b < c->B; ++b)
+    for (int t = 0; t < c->T; ++t) {
+      int* pos = (int*)malloc(sizeof(int) * (size_t)(c->topk * c->sel_block + 1));
+      for (int g = 0; g < c->Hkv; ++g) {
+        int* ir = idx + XI(c, b, t, g);
+        orc_moba_select_row(c, q, kc, nc, b, t, g, ir);
+        const int n = sel_keys(c, ir, t, pos);
+        for (int h = g * G; h < (g + 1) * G; ++h)
+          orc_list_row(c, q + QI(c, b, t, h), k, v, b, g, pos, n, o + QI(c, b, t, h),
+                       lse + RI(c, b, t, h));
+      }
+      free(pos);
+    }
+  free(kc);
+  free(vc);
+}

@@ -43,6 +43,10 @@ MUTANTS = {
     "bf16_round_truncates": ("double r = nearbyint(ldexp(m, 8));", "double r = trunc(ldexp(m, 8));"),
     "gate_grad_reads_exact_outputs": ("    o_sel[i] = round_store(o_sel[i], c->o_round);\n",
                                       "    o_sel[i] = o_sel[i];\n"),
+    "moba_gate_first_head_only": ("      acc += dot(q + QI(c, b, t, h), kc + CI(c, nc, b, j, g), D);",
+                                  "      if (h == g * G) acc += dot(q + QI(c, b, t, h), kc + CI(c, nc, b, j, g), D);"),
+    "moba_own_block_not_forced": ("  idx_row[n - 1] = cur;\n", "  idx_row[n - 1] = cand[n - 1];\n"),
+    "moba_ties_to_higher_block": ("(gr == gb && cand[r] < cand[best])", "(gr == gb && cand[r] > cand[best])"),
     "remap_overlap_off_by_one": ("if (clo < hi && chi > lo) acc += cmp_score_row[i];",
                                  "if (clo <= hi && chi > lo) acc += cmp_score_row[i];"),
     "remap_first_block_only": ("if (clo < hi && chi > lo) acc += cmp_score_row[i];",

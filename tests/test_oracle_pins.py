@@ -604,3 +604,81 @@ def test_backward_composed_on_own_selection_equals_backward():
     want = orc.backward(c, inp["q"], inp["k"], inp["v"], inp["gates"], inp["dout"])
     for a, b in zip(got, want):
         np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- MoBA
+def moba_cfg(**kw):
+    base = dict(B=2, T=48, Hq=4, Hkv=2, D=8, cmp_block=8, cmp_stride=8, sel_block=8,
+                topk=3, window=1)
+    base.update(kw)
+    return orc.Cfg(**base)
+
+
+def test_moba_with_every_block_selected_is_full_causal_attention():
+    """k >= the number of blocks: every causal block is read, so MoBA is
+    dense causal attention (library SDPA)."""
+    c = moba_cfg(topk=6)
+    q, k, v = qkv(c, 161)
+    o, lse, idx = orc.moba_fwd(c, q, k, v)
+    o_ref, lse_ref = sdpa(q, k, v, causal(c.T), 1 / math.sqrt(c.D))
+    np.testing.assert_allclose(o, o_ref, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, lse_ref, rtol=0, atol=1e-12)
+
+
+def test_moba_dense_below_k_blocks():
+    """The pages' short-context claim in miniature: with block L and top-3,
+    a sequence of 3 L tokens is dense attention (1.5k tokens at L = 512)."""
+    c = moba_cfg(T=24, topk=3)
+    q, k, v = qkv(c, 162)
+    o, _, idx = orc.moba_fwd(c, q, k, v)
+    o_ref, _ = sdpa(q, k, v, causal(c.T), 1 / math.sqrt(c.D))
+    np.testing.assert_allclose(o, o_ref, rtol=0, atol=1e-12)
+    assert np.all(idx[:, 23, :, :].tolist() == np.array([0, 1, 2]))
+
+
+def test_moba_equals_block_masked_attention():
+    """Given its selection, MoBA is SDPA under the block mask of the
+    selected blocks (and causal)."""
+    c = moba_cfg(T=64, topk=3)
+    q, k, v = qkv(c, 163)
+    o, lse, idx = orc.moba_fwd(c, q, k, v)
+    blk = torch.arange(c.T) // c.sel_block
+    mask = torch.zeros(c.B, c.Hq, c.T, c.T, dtype=torch.bool)
+    for b in range(c.B):
+        for t in range(c.T):
+            for h in range(c.Hq):
+                chosen = torch.tensor([j for j in idx[b, t, h // c.G] if j >= 0])
+                mask[b, h, t] = torch.isin(blk, chosen) & (torch.arange(c.T) <= t)
+    o_ref, lse_ref = sdpa(q, k, v, mask, 1 / math.sqrt(c.D))
+    np.testing.assert_allclose(o, o_ref, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, lse_ref, rtol=0, atol=1e-12)
+    # the query's own block is always selected, the rest are complete past blocks
+    for b in range(c.B):
+        for t in range(c.T):
+            cur = t // c.sel_block
+            for g in range(c.Hkv):
+                sel = [j for j in idx[b, t, g] if j >= 0]
+                assert cur in sel and all(j <= cur for j in sel)
+                assert sel == sorted(sel) and len(sel) == min(cur + 1, c.topk)
+
+
+def test_moba_gate_hand_cases():
+    """Hand-built gates: keys constant inside each block (so the block mean
+    is that constant) along one axis, queries along the same axis; head
+    gates are summed over the KV group.  Block 5 is the query's own."""
+    c = moba_cfg(B=1, T=48, Hq=2, Hkv=1, topk=3)
+    t = 47  # cur = 5: blocks 0..4 compete for two places
+    k = np.zeros((1, c.T, 1, c.D))
+    v = np.zeros_like(k)
+    a = [0.1, 0.9, 0.4, 0.9, 0.2, 0.0]   # block j's key value on axis 0
+    b_ = [0.0, 0.0, 0.5, 0.0, 0.8, 0.0]  # ... on axis 1
+    for j in range(6):
+        k[0, j * 8:(j + 1) * 8, 0, 0] = a[j]
+        k[0, j * 8:(j + 1) * 8, 0, 1] = b_[j]
+    q = np.zeros((1, c.T, 2, c.D))
+    q[0, t, 0, 0] = 1.0  # head 0 reads axis 0: gates a
+    _, _, idx = orc.moba_fwd(c, q, k, v)
+    assert idx[0, t, 0].tolist() == [1, 3, 5]  # 0.9 and 0.9 tie: both taken
+    q[0, t, 1, 1] = 1.0  # head 1 adds axis 1: sums 0.1, 0.9, 0.9, 0.9, 1.0
+    _, _, idx = orc.moba_fwd(c, q, k, v)
+    assert idx[0, t, 0].tolist() == [1, 4, 5]  # 1.0 first, then the lowest of three 0.9
