@@ -424,6 +424,10 @@ def run_gpu(args, rank: int, world: int, dist_on: bool) -> None:
     long_ctx = run_long(dev, flush, stream, max(3, args.steps // 4), peaks)
     # the 1.3B-shape forward (B=4, GQA-4 with 8 KV heads)
     onep3b = run_1p3b(dev, flush, stream, max(3, args.steps // 2), peaks)
+    # MoBA block attention (block 512, top-3) on the selection kernels
+    moba = run_moba(dev, flush, stream, max(3, args.steps // 2), peaks)
+    # selection backward, two-pass against single-pass atomic
+    selbwd = run_sel_bwd_compare(dev, flush, stream, 3, peaks)
     sampler.__exit__(None, None, None)
 
     barrier_sync(dist_on)
@@ -471,6 +475,8 @@ def run_gpu(args, rank: int, world: int, dist_on: bool) -> None:
         "train": train,
         "long_context": long_ctx,
         "nsa_1p3b": onep3b,
+        "moba": moba,
+        "sel_bwd_two_pass_vs_atomic": selbwd,
         "e2e": {"value": job_tokens_per_s(tokens_per_step, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": kernels_per_forward(w) * args.steps,
@@ -524,6 +530,49 @@ def run_train(dev, flush, stream, steps, peaks, batch=None) -> dict:
             "flops_note": "algorithmic: forward + backward counted as 2.5x forward"}
 
 
+def run_sel_bwd_compare(dev, flush, stream, steps, peaks, batch=8) -> dict:
+    """The selection backward at the training shape (B=8, T=8192, GQA-4) two
+    ways on the same forward: the two-pass kernels (query-stationary dQ, then
+    key-stationary dK/dV over the reverse map) and the single pass that adds
+    dK/dV with atomics from the query-stationary pass; the pages compare
+    these two designs and find the two-pass one faster."""
+    w = W.TRAIN_340M.replace(B=batch)
+    inp = W.make_inputs(w, seed=6, with_dout=True)
+    q, k, v, g = (inp[n].to(dev) for n in ("q", "k", "v", "gates"))
+    p = nsa.params_for(w)
+    out = torch.empty_like(q)
+    f32 = torch.float32
+    saved = {"idx": torch.empty((w.B, w.T, w.Hkv, w.topk), dtype=torch.int32, device=dev),
+             "o_sel": torch.empty_like(q),
+             "lse_sel": torch.empty((w.B, w.T, w.Hq), dtype=f32, device=dev)}
+    nsa.nsa_forward(p, q, k, v, g, out, saved, nsa.alloc_workspace(p, dev))
+    dO = inp["dout"].to(dev).float()
+    dq = torch.zeros((w.B, w.T, w.Hq, w.D), dtype=f32, device=dev)
+    dk = torch.zeros((w.B, w.T, w.Hkv, w.D), dtype=f32, device=dev)
+    dv = torch.zeros_like(dk)
+    ws = torch.empty(nsa.nsa_backward_workspace_size(p), dtype=torch.uint8, device=dev)
+    args = (p, q, k, v, saved["idx"], saved["o_sel"], saved["lse_sel"], dO, dq, dk, dv, ws)
+
+    def two_pass():
+        nsa.nsa_sel_attn_bwd(*args)
+
+    def single_pass():
+        nsa.nsa_sel_attn_bwd_atomic(*args)
+
+    for _ in range(2):
+        two_pass()
+        single_pass()
+    t2 = statistics.mean(timed_steps(two_pass, steps, flush, stream))
+    t1 = statistics.mean(timed_steps(single_pass, steps, flush, stream))
+    if nsa.nsa_last_device_error() != 0:
+        raise RuntimeError("device-side check failed in the selection-backward comparison")
+    flops = 2.5 * fwd_flops(w)["sel"]
+    return {"workload": w.name, "two_pass_ms": t2, "single_pass_atomic_ms": t1,
+            "two_pass_tflops": flops / (t2 * 1e-3) / 1e12,
+            "atomic_over_two_pass": t1 / t2,
+            "flops_note": "algorithmic selection backward counted as 2.5x its forward"}
+
+
 def run_1p3b(dev, flush, stream, steps, peaks) -> dict:
     """The 1.3B-shape forward: B=4 x 8192 tokens, 32 query heads on 8 KV
     heads (GQA-4), block 64, top-k 16, window 512, bf16."""
@@ -547,6 +596,33 @@ def run_1p3b(dev, flush, stream, steps, peaks) -> dict:
     return {"workload": w.name, "fwd_ms": ms, "tokens_per_s": w.B * w.T / (ms * 1e-3),
             "tflops": tf, "frac_bf16_peak": tf / peaks["bf16_tflops"],
             "flops_per_step": flops}
+
+
+def run_moba(dev, flush, stream, steps, peaks) -> dict:
+    """MoBA block attention at the 340M shape (B=1, T=8192, GQA-4; block 512,
+    top-k 3, the pages' MoBA setting) through nsa_moba_forward: gate and
+    top-k, then the selection attention kernels on the chosen blocks."""
+    w = W.NSA_340M.replace(name="moba_340m_gqa4_t8192_L512_k3_bf16")
+    L, k = 512, 3
+    inp = W.make_inputs(w, seed=5)
+    q, kk, v = (inp[n].to(dev) for n in ("q", "k", "v"))
+    p = nsa.make_moba_params(w.B, w.T, w.Hq, w.Hkv, block=L, topk=k, dtype=w.dtype)
+    out = torch.empty_like(q)
+    ws = torch.empty(nsa.nsa_moba_workspace_size(p), dtype=torch.uint8, device=dev)
+
+    def fwd():
+        nsa.nsa_moba_forward(p, q, kk, v, out, None, None, ws)
+
+    for _ in range(3):
+        fwd()
+    ms = statistics.mean(timed_steps(fwd, steps, flush, stream))
+    if nsa.nsa_last_device_error() != 0:
+        raise RuntimeError("device-side check failed in the MoBA leg")
+    keys = sum(min(t + 1, (k - 1) * L + t % L + 1) for t in range(w.T))
+    flops = 4 * w.D * keys * w.B * w.Hq
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"workload": w.name, "fwd_ms": ms, "tokens_per_s": w.B * w.T / (ms * 1e-3),
+            "tflops": tf, "frac_bf16_peak": tf / peaks["bf16_tflops"], "flops_per_step": flops}
 
 
 def run_long(dev, flush, stream, steps, peaks) -> dict:
@@ -639,13 +715,14 @@ def main():
     ap.add_argument("--impl", default="nsa", choices=["nsa", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--leg", default="all",
-                    choices=["all", "forward", "decode", "train", "long", "onep3b"],
-                    help="forward / decode / train / long / onep3b: run only that leg on one GPU "
+                    choices=["all", "forward", "decode", "train", "long", "onep3b", "moba",
+                             "selbwd"],
+                    help="forward / decode / train / long / onep3b / moba / selbwd: run only that leg on one GPU "
                          "and print its numbers (for profiling that leg alone); all: the "
                          "benchmark")
     ap.add_argument("--batch", type=int, default=None,
-                    help="--leg train only: batch size instead of 8 (a smaller case of the "
-                         "same kernels, for profiling)")
+                    help="--leg train / selbwd only: batch size instead of 8 (a smaller case "
+                         "of the same kernels, for profiling)")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -663,6 +740,12 @@ def main():
             print(json.dumps({"decode": run_decode(dev, flush, stream, args.steps, peaks)}))
         elif args.leg == "long":
             print(json.dumps({"long_context": run_long(dev, flush, stream, args.steps, peaks)}))
+        elif args.leg == "selbwd":
+            print(json.dumps({"sel_bwd_two_pass_vs_atomic": run_sel_bwd_compare(
+                dev, flush, stream, args.steps, peaks,
+                batch=args.batch if args.batch else 8)}))
+        elif args.leg == "moba":
+            print(json.dumps({"moba": run_moba(dev, flush, stream, args.steps, peaks)}))
         elif args.leg == "onep3b":
             print(json.dumps({"nsa_1p3b": run_1p3b(dev, flush, stream, args.steps, peaks)}))
         else:

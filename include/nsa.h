@@ -325,6 +325,23 @@ nsa_status nsa_sel_attn_bwd(const nsa_params* p, const void* q, const void* k,
                             float* dk, float* dv, void* workspace,
                             size_t workspace_bytes, void* stream);
 
+/* ---- selection backward, single pass with atomics ----------------------------
+ * The alternative "Sparsity is Cool", Method and Key claims, compare the
+ * two-pass kernel against: one query-stationary pass computes dQ over each
+ * query's selected blocks and, in the same kernel, each block's dK / dV
+ * contribution from the query tile, added to dk / dv with atomics
+ * (contention where many queries share a key: the pages report the two-pass
+ * form faster).  Same arguments and results as nsa_sel_attn_bwd (dq, dk, dv
+ * accumulated, +=), except that dk / dv depend on the order in which the
+ * atomics land (equal to the two-pass results up to fp32 rounding, not bit
+ * for bit).  bf16, 64-key blocks only (NSA_ERR_UNSUPPORTED otherwise);
+ * workspace: nsa_backward_workspace_size(p) bytes, 256-byte aligned. */
+nsa_status nsa_sel_attn_bwd_atomic(const nsa_params* p, const void* q, const void* k,
+                                   const void* v, const int32_t* idx, const void* o_sel,
+                                   const float* lse_sel, const float* dO_sel, float* dq,
+                                   float* dk, float* dv, void* workspace,
+                                   size_t workspace_bytes, void* stream);
+
 /* ---- sliding-window backward (same two-pass shape; the reverse map of key
  * s is the query range [s, s + w - 1]).  Passage: "DeepSeek's Native Sparse
  * Attention", SLIDING WINDOW. */
@@ -359,6 +376,52 @@ nsa_status nsa_backward(const nsa_params* p, const void* q, const void* k,
                         const nsa_saved* saved, float* dq, float* dk, float* dv,
                         float* dgates, void* workspace, size_t workspace_bytes,
                         void* stream);
+
+/* ========================================================================
+ * MoBA block attention on the same selection kernels.
+ * "Sparsity is Cool: Reverse-Engineering MoBA and NSA", Method (MoBA with
+ * block 512 and top-k 3) and Key claims (dense below about 1.5k tokens);
+ * "DeepSeek's Native Sparse Attention" newsletter, MoBA section (the
+ * context in blocks, a top-k gate sending each query to its most relevant
+ * past blocks, causal protection).  Per (query at t, KV group g):
+ *   cur = t / L.  With cur + 1 <= k all blocks 0..cur are read.  Otherwise
+ *   the gate of each complete past block j < cur is the sum over the
+ *   group's query heads h of q_h . mean(k of block j); the k - 1 best gates
+ *   (equal gates: lower block) and the query's own block are read.  The
+ *   pages do not say how the gate is formed or shared under GQA: this is the
+ *   plainest reading (the block's mean-pooled key, one selection per KV
+ *   group as in NSA's selection).
+ * out[t, h] = softmax attention of q_h over the keys s <= t of the chosen
+ * blocks (no gates, no other branch); lse its log-sum-exp.
+ * ======================================================================== */
+typedef struct {
+  int B, T, Tq, Hq, Hkv, D; /* as in nsa_params (D = 64)                      */
+  int block;                /* L: tokens per MoBA block, a multiple of 64     */
+  int topk;                 /* k: blocks per (query, KV group), own included  */
+  float scale;              /* softmax scale, finite and > 0                  */
+  int dtype;                /* nsa_dtype of q, k, v, out                      */
+} nsa_moba_params;
+
+/* Workspace bytes of nsa_moba_forward and nsa_moba_backward.  Limits: T / L
+ * <= 128 MoBA blocks, k L / 64 <= 64, T <= 65536 (else NSA_ERR_UNSUPPORTED). */
+nsa_status nsa_moba_workspace_size(const nsa_moba_params* p, size_t* bytes);
+
+/* q [B, Tq, Hq, D], k, v [B, T, Hkv, D] -> out [B, Tq, Hq, D] (dtype),
+ * lse [B, Tq, Hq] f32 (may be NULL), idx [B, Tq, Hkv, k] int32 (the chosen
+ * MoBA blocks, ascending, -1 padded; may be NULL).  The blocks are read as
+ * 64-key selection blocks by the selection attention kernels. */
+nsa_status nsa_moba_forward(const nsa_moba_params* p, const void* q, const void* k,
+                            const void* v, void* out, float* lse, int32_t* idx,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/* Gradients (float32, overwritten) of out for upstream dout [B, Tq, Hq, D]
+ * (float32), the forward's idx, out and lse held fixed (no gradient through
+ * the discrete gate): the two-pass selection backward on the chosen blocks. */
+nsa_status nsa_moba_backward(const nsa_moba_params* p, const void* q, const void* k,
+                             const void* v, const int32_t* idx, const void* out,
+                             const float* lse, const float* dout, float* dq, float* dk,
+                             float* dv, void* workspace, size_t workspace_bytes,
+                             void* stream);
 
 /* ---- decode without any allocation by the caller ---------------------------
  * No counterpart in the paper: this is a deployment variant of nsa_decode.

@@ -33,7 +33,9 @@ EXPORTS = ("nsa_status_string", "nsa_check_params", "nsa_workspace_size",
            "nsa_gate_combine_bwd", "nsa_sel_attn_bwd", "nsa_swa_bwd", "nsa_cmp_bwd",
            "nsa_backward", "nsa_decode_noalloc", "nsa_decode_noalloc_max_scratch",
            "nsa_sel_workspace_size", "nsa_sel_attn_fwd_ws", "nsa_set_kernel_events",
-           "nsa_forward_host_workspace_size", "nsa_forward_host")
+           "nsa_forward_host_workspace_size", "nsa_forward_host",
+           "nsa_moba_workspace_size", "nsa_moba_forward", "nsa_moba_backward",
+           "nsa_sel_attn_bwd_atomic")
 
 
 class NsaError(RuntimeError):
@@ -105,6 +107,7 @@ def load():
             "nsa_backward_workspace_size": ([P, C.POINTER(C.c_size_t)], C.c_int),
             "nsa_gate_combine_bwd": ([P] + [vp] * 10, C.c_int),
             "nsa_sel_attn_bwd": ([P] + [vp] * 11 + [C.c_size_t, vp], C.c_int),
+            "nsa_sel_attn_bwd_atomic": ([P] + [vp] * 11 + [C.c_size_t, vp], C.c_int),
             "nsa_swa_bwd": ([P] + [vp] * 10 + [C.c_size_t, vp], C.c_int),
             "nsa_cmp_bwd": ([P] + [vp] * 10 + [C.c_size_t, vp], C.c_int),
             "nsa_backward": ([P, vp, vp, vp, vp, vp, C.POINTER(Saved), vp, vp, vp, vp, vp,
@@ -113,6 +116,12 @@ def load():
             "nsa_sel_workspace_size": ([P, C.POINTER(C.c_size_t)], C.c_int),
             "nsa_sel_attn_fwd_ws": ([P, vp, vp, vp, vp, vp, vp, vp, C.c_size_t, vp], C.c_int),
             "nsa_set_kernel_events": ([vp, vp], C.c_int),
+            "nsa_moba_workspace_size": ([C.POINTER(MobaParams), C.POINTER(C.c_size_t)],
+                                        C.c_int),
+            "nsa_moba_forward": ([C.POINTER(MobaParams)] + [vp] * 7 + [C.c_size_t, vp],
+                                 C.c_int),
+            "nsa_moba_backward": ([C.POINTER(MobaParams)] + [vp] * 11 + [C.c_size_t, vp],
+                                  C.c_int),
         }
         for name, (args, res) in sig.items():
             f = getattr(lib, name)
@@ -120,6 +129,21 @@ def load():
             f.restype = res
         _lib = lib
     return _lib
+
+
+class MobaParams(C.Structure):
+    """Mirror of nsa_moba_params."""
+    _fields_ = [("B", C.c_int), ("T", C.c_int), ("Tq", C.c_int), ("Hq", C.c_int),
+                ("Hkv", C.c_int), ("D", C.c_int), ("block", C.c_int), ("topk", C.c_int),
+                ("scale", C.c_float), ("dtype", C.c_int)]
+
+
+def make_moba_params(B, T, Hq, Hkv, D=64, *, Tq=None, block=512, topk=3, scale=None,
+                     dtype=NSA_BF16) -> MobaParams:
+    if isinstance(dtype, torch.dtype):
+        dtype = NSA_BF16 if dtype == torch.bfloat16 else NSA_F32
+    return MobaParams(B, T, T if Tq is None else Tq, Hq, Hkv, D, block, topk,
+                      float(D ** -0.5 if scale is None else scale), dtype)
 
 
 def make_params(B, T, Hq, Hkv, D=64, *, Tq=None, cmp_block=64, cmp_stride=None,
@@ -384,6 +408,20 @@ def nsa_sel_attn_bwd(p: Params, q, k, v, idx, o_sel, lse_sel, dO_sel, dq, dk, dv
         wp, wb, _stream(stream)), "nsa_sel_attn_bwd")
 
 
+def nsa_sel_attn_bwd_atomic(p: Params, q, k, v, idx, o_sel, lse_sel, dO_sel, dq, dk, dv,
+                            workspace, stream=None):
+    """Single-pass selection backward (dK / dV by atomics); arguments as
+    nsa_sel_attn_bwd."""
+    s, dt, f = _shapes(p), p.torch_dtype, torch.float32
+    wp, wb = _ws(workspace)
+    _check(load().nsa_sel_attn_bwd_atomic(
+        C.byref(p), _ptr(q, s["q"], dt, "q"), _ptr(k, s["k"], dt, "k"), _ptr(v, s["k"], dt, "v"),
+        _ptr(idx, s["idx"], torch.int32, "idx"), _ptr(o_sel, s["o"], dt, "o_sel"),
+        _ptr(lse_sel, s["lse"], f, "lse_sel"), _ptr(dO_sel, s["o"], f, "dO_sel"),
+        _ptr(dq, s["q"], f, "dq"), _ptr(dk, s["k"], f, "dk"), _ptr(dv, s["k"], f, "dv"),
+        wp, wb, _stream(stream)), "nsa_sel_attn_bwd_atomic")
+
+
 def nsa_swa_bwd(p: Params, q, k, v, o_swa, lse_swa, dO_swa, dq, dk, dv, workspace,
                 stream=None):
     s, dt, f = _shapes(p), p.torch_dtype, torch.float32
@@ -486,3 +524,45 @@ def forward(p: Params, q, k, v, gates, keep: bool = False, workspace=None, strea
         workspace = alloc_workspace(p, dev)
     nsa_forward(p, q, k, v, gates, out, saved, workspace, stream)
     return (out, saved) if keep else out
+
+
+# ------------------------------------------------------------------ MoBA
+def nsa_moba_workspace_size(p: MobaParams) -> int:
+    n = C.c_size_t(0)
+    _check(load().nsa_moba_workspace_size(C.byref(p), C.byref(n)), "nsa_moba_workspace_size")
+    return n.value
+
+
+def _moba_shapes(p: MobaParams) -> dict:
+    return {"q": (p.B, p.Tq, p.Hq, p.D), "k": (p.B, p.T, p.Hkv, p.D),
+            "lse": (p.B, p.Tq, p.Hq), "idx": (p.B, p.Tq, p.Hkv, p.topk)}
+
+
+def nsa_moba_forward(p: MobaParams, q, k, v, out, lse=None, idx=None, workspace=None,
+                     stream=None):
+    s = _moba_shapes(p)
+    dt = torch.bfloat16 if p.dtype == NSA_BF16 else torch.float32
+    if workspace is None:
+        workspace = torch.empty(max(nsa_moba_workspace_size(p), 1), dtype=torch.uint8,
+                                device=q.device)
+    _check(load().nsa_moba_forward(
+        C.byref(p), _ptr(q, s["q"], dt, "q"), _ptr(k, s["k"], dt, "k"), _ptr(v, s["k"], dt, "v"),
+        _ptr(out, s["q"], dt, "out"), _ptr(lse, s["lse"], torch.float32, "lse", True),
+        _ptr(idx, s["idx"], torch.int32, "idx", True), _ptr(workspace, name="workspace"),
+        workspace.numel() * workspace.element_size(), _stream(stream)), "nsa_moba_forward")
+
+
+def nsa_moba_backward(p: MobaParams, q, k, v, idx, out, lse, dout, dq, dk, dv, workspace=None,
+                      stream=None):
+    s = _moba_shapes(p)
+    dt = torch.bfloat16 if p.dtype == NSA_BF16 else torch.float32
+    f = torch.float32
+    if workspace is None:
+        workspace = torch.empty(max(nsa_moba_workspace_size(p), 1), dtype=torch.uint8,
+                                device=q.device)
+    _check(load().nsa_moba_backward(
+        C.byref(p), _ptr(q, s["q"], dt, "q"), _ptr(k, s["k"], dt, "k"), _ptr(v, s["k"], dt, "v"),
+        _ptr(idx, s["idx"], torch.int32, "idx"), _ptr(out, s["q"], dt, "out"),
+        _ptr(lse, s["lse"], f, "lse"), _ptr(dout, s["q"], f, "dout"), _ptr(dq, s["q"], f, "dq"),
+        _ptr(dk, s["k"], f, "dk"), _ptr(dv, s["k"], f, "dv"), _ptr(workspace, name="workspace"),
+        workspace.numel() * workspace.element_size(), _stream(stream)), "nsa_moba_backward")

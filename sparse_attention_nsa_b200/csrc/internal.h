@@ -37,6 +37,14 @@ __host__ __device__ inline bool plain_geometry(const Dims& d) {
   return d.lc == d.l && d.dc == d.l;
 }
 
+// MoBA (k_moba.cu): gate + top-k per (query, KV group) over MoBA blocks of
+// L tokens (d.lc = d.dc = L pooled into kc; d.l = 64), writing the chosen
+// blocks (idx_m, may be NULL) and their 64-key blocks (idx64, top-k n L/64).
+cudaError_t launch_moba_select(const Dims& d, const void* q, const void* kc, int32_t* idx_m,
+                               int32_t* idx64, int L, int n, cudaStream_t s);
+cudaError_t launch_moba_expand(const Dims& d, const int32_t* idx_m, int32_t* idx64, int L, int n,
+                               cudaStream_t s);
+
 // Each launcher enqueues on `s` and returns the launch status.  `err` is
 // the device error word (may be NULL).
 cudaError_t launch_compress(const Dims& d, const void* k, const void* v,
@@ -99,6 +107,12 @@ cudaError_t launch_dq(const Dims& d, int mode, const void* q, const void* keys,
                       const float* dO, float* dq, float* delta, int* err, cudaStream_t s);
 // tensor-core dQ pass (k_bwd_tc.cu); modes 0 selection, 1 window
 bool dq_tc_eligible(const Dims& d, int mode);
+// single-pass selection backward (dQ query-stationary, dK / dV by atomics in
+// the same kernel); tensor-core geometry as dq_tc_eligible(d, 0)
+cudaError_t launch_sel_bwd_atomic(const Dims& d, const void* q, const void* k, const void* v,
+                                  const int32_t* idx, const void* o, const float* lse,
+                                  const float* dO, float* dq, float* delta, float* dk, float* dv,
+                                  int* err, cudaStream_t s);
 cudaError_t launch_dq_tc(const Dims& d, int mode, const void* q, const void* keys,
                          const void* vals, const int32_t* idx, const void* o, const float* lse,
                          const float* dO, float* dq, float* delta, int* err, cudaStream_t s);

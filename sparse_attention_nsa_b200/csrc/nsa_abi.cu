@@ -711,6 +711,26 @@ nsa_status nsa_sel_attn_bwd(const nsa_params* p, const void* q, const void* k, c
                       (cudaStream_t)stream);
 }
 
+nsa_status nsa_sel_attn_bwd_atomic(const nsa_params* p, const void* q, const void* k,
+                                   const void* v, const int32_t* idx, const void* o_sel,
+                                   const float* lse_sel, const float* dO_sel, float* dq,
+                                   float* dk, float* dv, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
+  Dims d;
+  nsa_status st = fill_dims(p, &d);
+  if (st != NSA_OK) return st;
+  for (const void* ptr : {q, k, v, (const void*)idx, o_sel, (const void*)lse_sel,
+                          (const void*)dO_sel, (const void*)dq, (const void*)dk, (const void*)dv})
+    if (!aligned16(ptr)) return NSA_ERR_INVALID_ARG;
+  if (!nsa::dq_tc_eligible(d, 0)) return NSA_ERR_UNSUPPORTED;
+  const BwdCarve c = bwd_carve(d);
+  if (!ws_ok(workspace, workspace_bytes, c.total)) return NSA_ERR_WORKSPACE;
+  float* delta = (float*)((char*)workspace + c.delta);
+  NSA_TRY_CUDA(nsa::launch_sel_bwd_atomic(d, q, k, v, idx, o_sel, lse_sel, dO_sel, dq, delta, dk,
+                                          dv, err_word(), (cudaStream_t)stream));
+  return NSA_OK;
+}
+
 nsa_status nsa_swa_bwd(const nsa_params* p, const void* q, const void* k, const void* v,
                        const void* o_swa, const float* lse_swa, const float* dO_swa, float* dq,
                        float* dk, float* dv, void* workspace, size_t workspace_bytes,
@@ -788,6 +808,129 @@ nsa_status nsa_backward(const nsa_params* p, const void* q, const void* k, const
     if (st != NSA_OK) return st;
   }
   return NSA_OK;
+}
+
+}  // extern "C"
+
+// ============================================================================
+// MoBA block attention on the selection kernels
+// ============================================================================
+namespace {
+
+// Dims of the selection attention that runs MoBA: 64-key selection blocks,
+// top-k = k L / 64; compression (pooling) over MoBA blocks of L tokens.
+nsa_status fill_moba_dims(const nsa_moba_params* p, Dims* d) {
+  if (!p) return NSA_ERR_INVALID_ARG;
+  if (p->block < 1 || p->topk < 1) return NSA_ERR_INVALID_ARG;
+  nsa_params q{};
+  q.B = p->B;
+  q.T = p->T;
+  q.Tq = p->Tq;
+  q.Hq = p->Hq;
+  q.Hkv = p->Hkv;
+  q.D = p->D;
+  q.cmp_block = p->block;
+  q.cmp_stride = p->block;
+  q.sel_block = 64;
+  q.topk = 2;  // validated below
+  q.window = 1;
+  q.scale = p->scale;
+  q.dtype = p->dtype;
+  q.branch_mask = NSA_BRANCH_SEL;
+  nsa_status st = fill_dims(&q, d);
+  if (st != NSA_OK) return st;
+  if (p->block % 64 != 0 || p->T / p->block > 128 || p->topk * (p->block / 64) > 64)
+    return NSA_ERR_UNSUPPORTED;
+  d->topk = p->topk * (p->block / 64);
+  if (d->topk < 2) return NSA_ERR_UNSUPPORTED;  // the selection kernels take >= 2 blocks
+  return NSA_OK;
+}
+
+struct MobaCarve {
+  size_t kc, vc, idx64, idxm, selbm, total;
+};
+
+MobaCarve moba_carve(const Dims& d, int n) {
+  MobaCarve c{};
+  size_t at = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = at;
+    at += align256(bytes);
+    return o;
+  };
+  const size_t rows = (size_t)d.B * d.Tq * d.Hkv;
+  c.kc = take((size_t)d.B * d.Nc * d.Hkv * 64 * esize(d));
+  c.vc = take((size_t)d.B * d.Nc * d.Hkv * 64 * esize(d));
+  c.idx64 = take(rows * d.topk * 4);
+  c.idxm = take(rows * (size_t)n * 4);
+  c.selbm = take(use_sel_bm(d) ? nsa::sel_bm_ws_bytes(d) : 0);
+  c.total = at;
+  return c;
+}
+
+}  // namespace
+
+extern "C" {
+
+nsa_status nsa_moba_workspace_size(const nsa_moba_params* p, size_t* bytes) {
+  Dims d;
+  nsa_status st = fill_moba_dims(p, &d);
+  if (st != NSA_OK) return st;
+  if (!bytes) return NSA_ERR_INVALID_ARG;
+  const size_t rows = (size_t)d.B * d.Tq * d.Hkv;
+  *bytes = std::max(moba_carve(d, p->topk).total,
+                    bwd_carve(d).total + align256(rows * d.topk * 4));
+  return NSA_OK;
+}
+
+nsa_status nsa_moba_forward(const nsa_moba_params* p, const void* q, const void* k, const void* v,
+                            void* out, float* lse, int32_t* idx, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  Dims d;
+  nsa_status st = fill_moba_dims(p, &d);
+  if (st != NSA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+      (lse && !aligned16(lse)) || (idx && !aligned16(idx)))
+    return NSA_ERR_INVALID_ARG;
+  const MobaCarve c = moba_carve(d, p->topk);
+  if (!ws_ok(workspace, workspace_bytes, c.total)) return NSA_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  char* w = (char*)workspace;
+  int32_t* idx64 = (int32_t*)(w + c.idx64);
+  if (d.Nc > 0) NSA_TRY_CUDA(nsa::launch_compress(d, k, v, w + c.kc, w + c.vc, s));
+  NSA_TRY_CUDA(nsa::launch_moba_select(d, q, w + c.kc, idx ? idx : (int32_t*)(w + c.idxm), idx64,
+                                       p->block, p->topk, s));
+  if (use_sel_bm(d))
+    NSA_TRY_CUDA(nsa::launch_sel_bm(d, q, k, v, idx64, out, lse, err_word(), nullptr,
+                                    w + c.selbm, s));
+  else
+    NSA_TRY_CUDA(nsa::launch_sel_fwd(d, q, k, v, idx64, out, lse, err_word(), s));
+  return NSA_OK;
+}
+
+nsa_status nsa_moba_backward(const nsa_moba_params* p, const void* q, const void* k,
+                             const void* v, const int32_t* idx, const void* out, const float* lse,
+                             const float* dout, float* dq, float* dk, float* dv, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  Dims d;
+  nsa_status st = fill_moba_dims(p, &d);
+  if (st != NSA_OK) return st;
+  for (const void* ptr : {q, k, v, (const void*)idx, out, (const void*)lse, (const void*)dout,
+                          (const void*)dq, (const void*)dk, (const void*)dv})
+    if (!aligned16(ptr)) return NSA_ERR_INVALID_ARG;
+  // the selection backward's workspace, then the expanded indices after it
+  const BwdCarve c = bwd_carve(d);
+  const size_t rows = (size_t)d.B * d.Tq * d.Hkv;
+  const size_t need = c.total + align256(rows * d.topk * 4);
+  if (!ws_ok(workspace, workspace_bytes, need)) return NSA_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  char* w = (char*)workspace;
+  int32_t* idx64 = (int32_t*)(w + c.total);
+  NSA_TRY_CUDA(nsa::launch_moba_expand(d, idx, idx64, p->block, p->topk, s));
+  NSA_TRY_CUDA(cudaMemsetAsync(dq, 0, (size_t)d.B * d.Tq * d.Hq * 64 * 4, s));
+  NSA_TRY_CUDA(cudaMemsetAsync(dk, 0, (size_t)d.B * d.T * d.Hkv * 64 * 4, s));
+  NSA_TRY_CUDA(cudaMemsetAsync(dv, 0, (size_t)d.B * d.T * d.Hkv * 64 * 4, s));
+  return sel_bwd_body(d, q, k, v, idx64, out, lse, dout, dq, dk, dv, w, c, s);
 }
 
 }  // extern "C"
