@@ -59,9 +59,28 @@ struct Bars {
   uint64_t sfree;   // the 128 row threads have loaded them
   uint64_t ds;      // the 128 row threads have written dS
   uint64_t fin;
+  // single-pass variant only
+  uint64_t pfree;   // dV/dK MMAs of a block pair done: P / dS tiles free
+  uint64_t kvfull;  // dV/dK of a block pair are in TMEM
+  uint64_t kvfree;  // the 128 epilogue threads have loaded them
 };
 constexpr uint32_t OFF_MISC = OFF_BAR + ((sizeof(Bars) + 15) / 16) * 16;
 constexpr uint32_t OFF_LIST = OFF_MISC + 16;
+
+// Shared-memory layout of the single-pass (atomic) variant: three K/V
+// stages, then the P and dS tiles of a pair of blocks (each 128 rows x 64
+// keys, 128-byte swizzle: P of block 2m, P of block 2m+1 (fp16), dS of 2m,
+// dS of 2m+1 (bf16)), the dO lo tile (bf16: dO - bf16(dO)) and the dO tile
+// in fp16, then the barriers and the block list.
+constexpr int kAtStages = 3;
+constexpr uint32_t AT_OFF_P = OFF_KV + kAtStages * 2 * kTileBytes;
+constexpr uint32_t AT_OFF_DOL = AT_OFF_P + 4 * kQBytes;
+constexpr uint32_t AT_OFF_DOH = AT_OFF_DOL + kQBytes;
+constexpr uint32_t AT_OFF_BAR = AT_OFF_DOH + kQBytes;
+constexpr uint32_t AT_OFF_MISC = AT_OFF_BAR + ((sizeof(Bars) + 15) / 16) * 16;
+constexpr uint32_t AT_OFF_LIST = AT_OFF_MISC + 16;
+constexpr int kAtThreads = 320;
+constexpr uint32_t kColDV = 256, kColDK = 320;  // TMEM columns of a pair's dV / dK
 
 __host__ __device__ inline int tokens_per_tile(int G) { return kRows / G; }
 
@@ -72,23 +91,45 @@ __host__ __device__ inline size_t list_ints(const Dims& d) {
 
 // MODE 0 selection, 1 window, 2 compression (keys = the compressed cache;
 // key c is visible to the query at t when its block is complete:
-// (c + 1) l - 1 <= t).
-template <int MODE>
-__global__ void __launch_bounds__(kThreads, 2)
+// c d + l - 1 <= t).
+//
+// ATOMIC (selection only): the single-pass query-stationary backward that
+// "Sparsity is Cool", Method, sets against the two-pass one: the same pass
+// also forms each block's dK and dV from this tile's rows and adds them to
+// dk / dv with atomics.  dK and dV sum over many rows, so they need what
+// the two-pass kernel needs: dP = V (dO_hi + dO_lo)^T to about fp32 (dS =
+// P (dP - delta) cancels when the softmax is peaked) and dV in fp16.  The
+// row threads write P (fp16) and dS (bf16) of each union block into shared
+// memory as well; once two blocks' tiles are there (or the last block is),
+// one MMA per gradient covers both blocks' 128 keys:
+//   dV = P^T dO (fp16), dK = dS^T Q (bf16)  (M128 N64 K128: A the P / dS
+//   tiles read MN-major, the second block's tiles 16 KB after the first's;
+//   B the dO (fp16) / Q tiles read MN-major), fp32 in TMEM [256, 384);
+// warps 6-9 (thread = key of the pair) load them and add them to dk, dv
+// with float4 atomics (so dk / dv depend on the order the atomics land in:
+// equal to the two-pass results up to fp32 rounding, not bit for bit).
+template <int MODE, bool ATOMIC = false>
+__global__ void __launch_bounds__(ATOMIC ? kAtThreads : kThreads, ATOMIC ? 1 : 2)
 bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const bf16* __restrict__ o,
                  const float* __restrict__ lse, const float* __restrict__ dO,
                  const int32_t* __restrict__ idx, float* __restrict__ dq,
-                 float* __restrict__ delta, Dims d, int* err) {
+                 float* __restrict__ delta, Dims d, int* err, float* __restrict__ dk_at = nullptr,
+                 float* __restrict__ dv_at = nullptr) {
   constexpr bool SEL = MODE == 0;
+  constexpr int NST = ATOMIC ? kAtStages : kStages;
+  constexpr uint32_t O_BAR = ATOMIC ? AT_OFF_BAR : OFF_BAR;
+  constexpr uint32_t O_MISC = ATOMIC ? AT_OFF_MISC : OFF_MISC;
+  constexpr uint32_t O_LIST = ATOMIC ? AT_OFF_LIST : OFF_LIST;
+  constexpr uint32_t TMEM_COLS = ATOMIC ? 512 : 256;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  Bars* bars = (Bars*)(smem + OFF_BAR);
+  Bars* bars = (Bars*)(smem + O_BAR);
   const int nkeys = MODE == 2 ? d.Nc : d.T;  // key rows per sequence
-  uint32_t* tmem_slot = (uint32_t*)(smem + OFF_MISC);
-  volatile int* abort_flag = (volatile int*)(smem + OFF_MISC + 4);
-  int* nblk_s = (int*)(smem + OFF_MISC + 8);
-  int* blk = (int*)(smem + OFF_LIST);
+  uint32_t* tmem_slot = (uint32_t*)(smem + O_MISC);
+  volatile int* abort_flag = (volatile int*)(smem + O_MISC + 4);
+  int* nblk_s = (int*)(smem + O_MISC + 8);
+  int* blk = (int*)(smem + O_LIST);
   const int words = (d.Nb + 31) / 32;
   uint32_t* bits = (uint32_t*)(blk + d.Nb);
   int* toks = (int*)(bits + words);
@@ -104,7 +145,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   if (tid == 0) {
     mbar_init(&bars->q, 1);
     mbar_init(&bars->dorows, 128);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < NST; ++s) {
       mbar_init(&bars->full[s], 1);
       mbar_init(&bars->empty[s], 1);
     }
@@ -112,11 +153,14 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     mbar_init(&bars->sfree, 128);
     mbar_init(&bars->ds, 128);
     mbar_init(&bars->fin, 1);
+    mbar_init(&bars->pfree, 1);
+    mbar_init(&bars->kvfull, 1);
+    mbar_init(&bars->kvfree, 128);
     fence_barrier_init();
     fence_proxy_async_smem();
     *abort_flag = 0;
   }
-  if (warp == 4) tmem_alloc(tmem_slot, 256);
+  if (warp == 4) tmem_alloc(tmem_slot, TMEM_COLS);
   if (warp == 5 && lane == 0) {
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
@@ -125,9 +169,9 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
   // ---- block list (as in the forward kernel) ---------------------------------------
   if (SEL) {
-    for (int w = tid; w < words; w += kThreads) bits[w] = 0u;
+    for (int w = tid; w < words; w += blockDim.x) bits[w] = 0u;
     __syncthreads();
-    for (int tl = tid; tl < TQ; tl += kThreads) {
+    for (int tl = tid; tl < TQ; tl += blockDim.x) {
       int* lst = toks + tl * (d.topk + 1);
       int cnt = 0;
       if (tl < nvalid) {
@@ -197,9 +241,9 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       tma_load_3d(smem + OFF_Q, &tm_q, &bars->q, 0, g * d.G, b * d.Tq + t0);
       int issued = 0;
       for (int i = 0; i < n; ++i) {
-        const int st = i % kStages;
-        if (i >= kStages &&
-            !wait_bar(&bars->empty[st], ((i / kStages) & 1) ^ 1, abort_flag, err))
+        const int st = i % NST;
+        if (i >= NST &&
+            !wait_bar(&bars->empty[st], ((i / NST) & 1) ^ 1, abort_flag, err))
           break;
         const int j = SEL ? blk[i] : blk0 + i;
         const int row = b * nkeys + j * kKeys;
@@ -211,8 +255,8 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       }
       if (*abort_flag) {  // let the copies already issued land before exit
         drain_bar(&bars->q, 0);
-        for (int i = max(0, issued - kStages); i < issued; ++i)
-          drain_bar(&bars->full[i % kStages], (i / kStages) & 1);
+        for (int i = max(0, issued - NST); i < issued; ++i)
+          drain_bar(&bars->full[i % NST], (i / NST) & 1);
       }
     }
   } else if (warp == 4) {
@@ -227,20 +271,40 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         // dS of block i (TMEM) times K of block i read MN-major
         if (!wait_bar(&bars->ds, i & 1, abort_flag, err)) return false;
         tc_fence_after();
-        const int st = i % kStages;
+        const int st = i % NST;
         const uint32_t k_addr = smem_u32(smem + OFF_KV + st * 2 * kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_bf16_ts(tmem + kColDQ, tmem + kColDS + kk * 8, desc_sw128(k_addr + kk * 2048, 8192),
                       idesc_q, (i > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&bars->empty[st]);  // frees the stage and the dS columns
+        if constexpr (ATOMIC) {
+          if ((i & 1) || i == n - 1) {  // blocks 2m and 2m+1 (or the last alone)
+            const int pi = i >> 1;
+            if (pi >= 1 && !wait_bar(&bars->kvfree, (pi - 1) & 1, abort_flag, err)) return false;
+            tc_fence_after();
+            constexpr uint32_t idesc_kv = idesc_bf16(128, 64, true, true);  // A, B MN-major
+            constexpr uint32_t idesc_v16 = idesc_f16(128, 64, true, true);  // dV: fp16
+            const uint32_t p_addr = smem_u32(smem + AT_OFF_P), s_addr = p_addr + 2 * kQBytes;
+            const uint32_t doh_addr = smem_u32(smem + AT_OFF_DOH);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {  // K = the tile's 128 rows, 16 at a time
+              mma_bf16(tmem + kColDV, desc_sw128(p_addr + kk * 2048, kQBytes),
+                       desc_sw128(doh_addr + kk * 2048, 8192), idesc_v16, kk > 0);
+              mma_bf16(tmem + kColDK, desc_sw128(s_addr + kk * 2048, kQBytes),
+                       desc_sw128(q_addr + kk * 2048, 8192), idesc_kv, kk > 0);
+            }
+            mma_commit(&bars->pfree);
+            mma_commit(&bars->kvfull);
+          }
+        }
         return true;
       };
       for (int i = 0; ok && i < n; ++i) {
         // S and dP are single-buffered: the rows must have loaded block i-1's
         if (i >= 1 && !wait_bar(&bars->sfree, (i - 1) & 1, abort_flag, err)) break;
-        const int st = i % kStages;
-        if (!wait_bar(&bars->full[st], (i / kStages) & 1, abort_flag, err)) break;
+        const int st = i % NST;
+        if (!wait_bar(&bars->full[st], (i / NST) & 1, abort_flag, err)) break;
         tc_fence_after();
         const uint32_t k_addr = smem_u32(smem + OFF_KV + st * 2 * kTileBytes);
         const uint32_t v_addr = k_addr + kTileBytes;
@@ -252,6 +316,13 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         for (int kk = 0; kk < 4; ++kk)
           mma_bf16(tmem + kColDP, desc_sw128(do_addr + kk * 32, 16),
                    desc_sw128(v_addr + kk * 32, 16), idesc_s, kk > 0);
+        if constexpr (ATOMIC) {  // dO lo: dP to about fp32 for dS = P (dP - delta)
+          const uint32_t dol_addr = smem_u32(smem + AT_OFF_DOL);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16(tmem + kColDP, desc_sw128(dol_addr + kk * 32, 16),
+                     desc_sw128(v_addr + kk * 32, 16), idesc_s, 1u);
+        }
         mma_commit(&bars->s);
         if (i >= 1 && !issue_dq(i - 1)) break;
         if (i == n - 1) issue_dq(i);
@@ -260,7 +331,37 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       mma_commit(&bars->fin);
       drain_bar(&bars->fin, 0);
     }
-  } else {
+  } else if (ATOMIC && warp >= 6) {
+    // ---- single pass: dK / dV of each block pair into dk, dv with atomics --------------
+    const int k = 32 * (warp & 3) + lane;  // key of the pair (TMEM lane k)
+    const uint32_t lane_tmem = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    const int npairs = (n + 1) / 2;
+    for (int pi = 0; pi < npairs; ++pi) {
+      if (!wait_bar_warp(&bars->kvfull, pi & 1, abort_flag, err)) break;
+      tc_fence_after();
+      float av[64], ak[64];
+      tmem_ld32(lane_tmem + kColDV, av);
+      tmem_ld32(lane_tmem + kColDV + 32u, av + 32);
+      tmem_ld32(lane_tmem + kColDK, ak);
+      tmem_ld32(lane_tmem + kColDK + 32u, ak + 32);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&bars->kvfree);
+      const int bi = 2 * pi + (k >> 6);
+      if (bi >= n) continue;
+      const int key = blk[bi] * kKeys + (k & 63);
+      if (key >= nkeys) continue;
+      const size_t krow = (((size_t)b * nkeys + key) * d.Hkv + g) * 64;
+      float4* pv4 = reinterpret_cast<float4*>(dv_at + krow);
+      float4* pk4 = reinterpret_cast<float4*>(dk_at + krow);
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        atomicAdd(pv4 + c, make_float4(av[4 * c], av[4 * c + 1], av[4 * c + 2], av[4 * c + 3]));
+        atomicAdd(pk4 + c, make_float4(ak[4 * c] * d.scale, ak[4 * c + 1] * d.scale,
+                                       ak[4 * c + 2] * d.scale, ak[4 * c + 3] * d.scale));
+      }
+    }
+  } else if (warp < 4) {
     // ---- rows: thread r owns query row r -----------------------------------------------
     const int r = tid;
     const int tl = r / d.G, hh = r % d.G;
@@ -287,6 +388,26 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           w[1] = pack_bf16(a.z, a.w);
           w[2] = pack_bf16(a2.x, a2.y);
           w[3] = pack_bf16(a2.z, a2.w);
+          if constexpr (ATOMIC) {
+            const float x[8] = {a.x, a.y, a.z, a.w, a2.x, a2.y, a2.z, a2.w};
+            uint32_t wl[4], wh[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float h0 = __bfloat162float(__float2bfloat16_rn(x[2 * e]));
+              const float h1 = __bfloat162float(__float2bfloat16_rn(x[2 * e + 1]));
+              wl[e] = pack_bf16(x[2 * e] - h0, x[2 * e + 1] - h1);
+              wh[e] = pack_f16(x[2 * e], x[2 * e + 1]);
+            }
+            const uint32_t sw = (uint32_t)(c ^ (r & 7)) << 4;
+            const uint32_t base = (uint32_t)(r >> 3) * 1024u + (uint32_t)(r & 7) * 128u + sw;
+            st_shared_v4(smem_u32(smem + AT_OFF_DOL) + base, wl[0], wl[1], wl[2], wl[3]);
+            st_shared_v4(smem_u32(smem + AT_OFF_DOH) + base, wh[0], wh[1], wh[2], wh[3]);
+          }
+        } else if constexpr (ATOMIC) {
+          const uint32_t sw = (uint32_t)(c ^ (r & 7)) << 4;
+          const uint32_t base = (uint32_t)(r >> 3) * 1024u + (uint32_t)(r & 7) * 128u + sw;
+          st_shared_v4(smem_u32(smem + AT_OFF_DOL) + base, 0u, 0u, 0u, 0u);
+          st_shared_v4(smem_u32(smem + AT_OFF_DOH) + base, 0u, 0u, 0u, 0u);
         }
         st_shared_v4(drow + ((uint32_t)(c ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
       }
@@ -321,6 +442,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       }
       tc_fence_after();
       uint32_t dsk[32];
+      uint32_t ppk[ATOMIC ? 32 : 1];
 #pragma unroll
       for (int h2 = 0; h2 < 2; ++h2) {
         float sv[32], pv[32];
@@ -343,15 +465,44 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
               if (key + 1 > khi || key + 1 < lo) p1 = 0.f;
             }
             dsk[16 * h2 + c / 2] = pack_bf16(p0 * (pv[c] - dl), p1 * (pv[c + 1] - dl));
+            if constexpr (ATOMIC) ppk[16 * h2 + c / 2] = pack_f16(p0, p1);
           }
         } else {
 #pragma unroll
-          for (int c = 0; c < 16; ++c) dsk[16 * h2 + c] = 0u;
+          for (int c = 0; c < 16; ++c) {
+            dsk[16 * h2 + c] = 0u;
+            if constexpr (ATOMIC) ppk[16 * h2 + c] = 0u;
+          }
         }
+      }
+      if constexpr (ATOMIC) {
+        // P and dS of this row for the pair's dV / dK MMAs: row r of the
+        // tiles of half i & 1 (the pair's previous MMAs must be done with them)
+        const int hf = i & 1;
+        if (hf == 0 && i >= 2) {
+          if (!wait_bar_warp(&bars->pfree, ((i >> 1) - 1) & 1, abort_flag, err)) {
+            ok = false;
+            break;
+          }
+        }
+        const uint32_t line = (uint32_t)(r >> 3) * 1024u + (uint32_t)(r & 7) * 128u;
+        const uint32_t pa = smem_u32(smem + AT_OFF_P) + hf * kQBytes + line;
+        const uint32_t sa = pa + 2 * kQBytes;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint32_t sw = (uint32_t)(c ^ (r & 7)) << 4;
+          st_shared_v4(pa + sw, ppk[4 * c], ppk[4 * c + 1], ppk[4 * c + 2], ppk[4 * c + 3]);
+          st_shared_v4(sa + sw, dsk[4 * c], dsk[4 * c + 1], dsk[4 * c + 2], dsk[4 * c + 3]);
+          if (hf == 0 && i == n - 1) {  // a last block alone: its pair half is zero
+            st_shared_v4(pa + kQBytes + sw, 0u, 0u, 0u, 0u);
+            st_shared_v4(sa + kQBytes + sw, 0u, 0u, 0u, 0u);
+          }
+        }
+        fence_proxy_async_smem();  // the MMA reads the tiles through the async proxy
       }
       // the dQ MMA of block i-1 reads the dS columns: wait for it
       if (i >= 1) {
-        if (!wait_bar_warp(&bars->empty[(i - 1) % kStages], ((i - 1) / kStages) & 1, abort_flag,
+        if (!wait_bar_warp(&bars->empty[(i - 1) % NST], ((i - 1) / NST) & 1, abort_flag,
                            err)) {
           ok = false;
           break;
@@ -393,7 +544,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   __syncthreads();
   if (warp == 4) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, TMEM_COLS);
   }
 }
 
@@ -1039,6 +1190,29 @@ cudaError_t launch_dkdv_tc(const Dims& d, int mode, const void* q, const void* k
   if (mode == 1)
     return launch_dkdv_tc_t<1>(d, q, k, v, lse, delta, dO, o16, offsets, list, dk, dv, part, err, s);
   return launch_dkdv_tc_t<2>(d, q, k, v, lse, delta, dO, o16, offsets, list, dk, dv, part, err, s);
+}
+
+// The single-pass selection backward: dQ as launch_dq_tc (mode 0), dK and
+// dV added into dk, dv by atomics in the same kernel.
+cudaError_t launch_sel_bwd_atomic(const Dims& d, const void* q, const void* k, const void* v,
+                                  const int32_t* idx, const void* o, const float* lse,
+                                  const float* dO, float* dq, float* delta, float* dk, float* dv,
+                                  int* err, cudaStream_t s) {
+  const int TQ = tokens_per_tile(d.G);
+  if ((long)d.B * d.T == 0) return cudaSuccess;
+  CUtensorMap mq, mk, mv;
+  if (!make_tmap_bf16(&mq, q, d.Hq, (long)d.B * d.Tq, d.G, TQ) ||
+      !make_tmap_bf16(&mk, k, d.Hkv, (long)d.B * d.T, 1, kKeys) ||
+      !make_tmap_bf16(&mv, v, d.Hkv, (long)d.B * d.T, 1, kKeys))
+    return cudaErrorInvalidValue;
+  const size_t smem = AT_OFF_LIST + list_ints(d) * sizeof(int) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(bwd_dq_tc_kernel<0, true>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((d.Tq + TQ - 1) / TQ, d.Hkv, d.B);
+  bwd_dq_tc_kernel<0, true><<<grid, kAtThreads, smem, s>>>(
+      mq, mk, mv, (const bf16*)o, lse, dO, idx, dq, delta, d, err, dk, dv);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_dq_tc(const Dims& d, int mode, const void* q, const void* k, const void* v,

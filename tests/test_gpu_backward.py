@@ -96,6 +96,34 @@ def test_sel_attn_bwd_two_pass(cuda_lib, w):
     assert_close(to_np(dk), 2 * want[1], 2 * TOL[w.dtype], "dk twice")
 
 
+@pytest.mark.parametrize("w", [BWD[1], BWD[2], BWD[5], BWD[7],
+                               small("bwd_atomic_gqa4_t2100_k6_bf16", T=2100, topk=6)],
+                         ids=lambda w: w.name)
+def test_sel_attn_bwd_single_pass_atomic(cuda_lib, w):
+    """The single-pass variant (dK / dV by atomics from the query-stationary
+    pass) against the oracle, like the two-pass backward; union block counts
+    odd and even occur across the tiles of these cases."""
+    inp = W.make_inputs(w, seed=31)
+    c = ocfg(w)
+    r = orc.forward(c, inp["q"], inp["k"], inp["v"], inp["gates"])
+    g = torch.Generator().manual_seed(32)
+    dO = torch.randn((w.B, w.T, w.Hq, w.D), generator=g)
+    want = orc.sel_attn_bwd(c, inp["q"], inp["k"], inp["v"], r["idx"], dO)
+    p = nsa.params_for(w)
+    d = {k_: v_.to(DEV) for k_, v_ in inp.items()}
+    idx = torch.from_numpy(r["idx"]).to(DEV)
+    o = torch.empty((w.B, w.T, w.Hq, w.D), dtype=w.dtype, device=DEV)
+    lse = torch.empty((w.B, w.T, w.Hq), dtype=torch.float32, device=DEV)
+    nsa.nsa_sel_attn_fwd(p, d["q"], d["k"], d["v"], idx, o, lse)
+    dq, dk, dv = zeros_grads(w)
+    nsa.nsa_sel_attn_bwd_atomic(p, d["q"], d["k"], d["v"], idx, o, lse, dO.to(DEV), dq, dk, dv,
+                                bwd_ws(p))
+    torch.cuda.synchronize()
+    assert nsa.nsa_last_device_error() == 0
+    for got, ref, name in zip((dq, dk, dv), want, ("dq", "dk", "dv")):
+        assert_close(to_np(got), ref, TOL[w.dtype], name)
+
+
 @pytest.mark.parametrize("w", BWD[:7], ids=lambda w: w.name)
 def test_swa_bwd(cuda_lib, w):
     inp = W.make_inputs(w, seed=33)
