@@ -28,7 +28,7 @@ namespace nsa {
 
 constexpr int kTopkWarps = 8;
 
-template <int QMAX>
+template <int QMAX, bool REMAP>
 __global__ void __launch_bounds__(kTopkWarps * 32)
 topk_kernel(const float* __restrict__ score, int32_t* __restrict__ idx, Dims d) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -39,7 +39,7 @@ topk_kernel(const float* __restrict__ score, int32_t* __restrict__ idx, Dims d) 
     const size_t r = (size_t)b * d.Tq * d.Hkv + rb;
     // candidates are blocks 1..cur-1 (all complete, so all have scores)
     const float* row = score + r * d.Nc;
-    if (plain_geometry(d)) {
+    if (!REMAP) {
       warp_select_blocks<QMAX>(row, t / d.l, d.topk, idx + r * d.topk, lane);
     } else {
       auto remap = [row, &d](int j) {
@@ -55,6 +55,15 @@ topk_kernel(const float* __restrict__ score, int32_t* __restrict__ idx, Dims d) 
   }
 }
 
+template <bool REMAP>
+static void launch_topk_t(const Dims& d, const float* score, int32_t* idx, dim3 blocks, int q,
+                          cudaStream_t s) {
+  if (q <= 4) topk_kernel<4, REMAP><<<blocks, kTopkWarps * 32, 0, s>>>(score, idx, d);
+  else if (q <= 8) topk_kernel<8, REMAP><<<blocks, kTopkWarps * 32, 0, s>>>(score, idx, d);
+  else if (q <= 16) topk_kernel<16, REMAP><<<blocks, kTopkWarps * 32, 0, s>>>(score, idx, d);
+  else topk_kernel<32, REMAP><<<blocks, kTopkWarps * 32, 0, s>>>(score, idx, d);
+}
+
 cudaError_t launch_topk(const Dims& d, const float* score, int32_t* idx,
                         cudaStream_t s) {
   const long rows = (long)d.Tq * d.Hkv;  // per sequence (< 2^31: Tq < 2^24, Hkv <= 128)
@@ -62,10 +71,8 @@ cudaError_t launch_topk(const Dims& d, const float* score, int32_t* idx,
   if (rows > INT_MAX - kTopkWarps) return cudaErrorInvalidValue;
   const dim3 blocks((unsigned)((rows + kTopkWarps - 1) / kTopkWarps), (unsigned)min(d.B, 65535));
   const int q = (d.Nb + 31) / 32;  // candidate slots per lane
-  if (q <= 4) topk_kernel<4><<<blocks, kTopkWarps * 32, 0, s>>>(score, idx, d);
-  else if (q <= 8) topk_kernel<8><<<blocks, kTopkWarps * 32, 0, s>>>(score, idx, d);
-  else if (q <= 16) topk_kernel<16><<<blocks, kTopkWarps * 32, 0, s>>>(score, idx, d);
-  else topk_kernel<32><<<blocks, kTopkWarps * 32, 0, s>>>(score, idx, d);
+  if (plain_geometry(d)) launch_topk_t<false>(d, score, idx, blocks, q, s);
+  else launch_topk_t<true>(d, score, idx, blocks, q, s);
   return cudaGetLastError();
 }
 
