@@ -347,3 +347,27 @@ def moba_fwd(cfg: Cfg, q, k, v):
     cc = cfg.c()
     lib.orc_moba_fwd(C.byref(cc), _p(q), _p(k), _p(v), _p(idx), _p(o), _p(lse))
     return o, lse, idx
+
+
+def compress_mlp(cfg: Cfg, k, v, wk, wv):
+    """Parametric compression: one linear layer over each block's l rows
+    flattened in token order, wk, wv [l D, D] (reading R17)."""
+    lib = _load()
+    k, v, wk, wv = _f64(k), _f64(v), _f64(wk), _f64(wv)
+    kc = np.zeros((cfg.B, cfg.Nc, cfg.Hkv, cfg.D))
+    vc = np.zeros_like(kc)
+    cc = cfg.c()
+    lib.orc_compress_mlp(C.byref(cc), _p(k), _p(v), _p(wk), _p(wv), _p(kc), _p(vc))
+    return kc, vc
+
+
+def compress_mlp_bwd(cfg: Cfg, k, v, wk, wv, dkc, dvc):
+    """(dk, dv, dwk, dwv) of compress_mlp for upstream dkc, dvc."""
+    lib = _load()
+    k, v, wk, wv, dkc, dvc = (_f64(x) for x in (k, v, wk, wv, dkc, dvc))
+    dk, dv = np.zeros_like(k), np.zeros_like(v)
+    dwk, dwv = np.zeros_like(wk), np.zeros_like(wv)
+    cc = cfg.c()
+    lib.orc_compress_mlp_bwd(C.byref(cc), _p(k), _p(v), _p(wk), _p(wv), _p(dkc), _p(dvc),
+                             _p(dk), _p(dv), _p(dwk), _p(dwv))
+    return dk, dv, dwk, dwv

@@ -944,3 +944,67 @@ void orc_moba_fwd(const orc_cfg* c, const double* q, const double* k, const doub
   free(kc);
   free(vc);
 }
+
+/* ================================================================== */
+/* Parametric compression (the NSA original that "Sparsity is Cool",    */
+/* Method and Key claims, replaces with mean-pooling; "DeepSeek's       */
+/* Native Sparse Attention", COMPRESSION: a small neural layer          */
+/* summarises the block into one key and one value).  Reading taken:    */
+/* one linear layer over the block's l rows of D values flattened in    */
+/* token order, weights shared by every head and block:                 */
+/*   kc[b, j, g, n] = sum_{i<l} sum_{e<D} k[b, j d + i, g, e] Wk[i D + e, n] */
+/* (same for vc with Wv).  Mean-pooling is the special case             */
+/* W[i D + e, n] = (e == n) / l.  Wk, Wv [l D, D]; kv_round rounds the  */
+/* outputs as stored.                                                   */
+/* ================================================================== */
+void orc_compress_mlp(const orc_cfg* c, const double* k, const double* v, const double* wk,
+                      const double* wv, double* kc, double* vc) {
+  const int nc = orc_num_cmp_blocks(c);
+  const int l = c->cmp_block, dstr = c->cmp_stride, D = c->D;
+  for (int b = 0; b < c->B; ++b)
+    for (int j = 0; j < nc; ++j)
+      for (int g = 0; g < c->Hkv; ++g)
+        for (int n = 0; n < D; ++n) {
+          double sk = 0.0, sv = 0.0;
+          for (int i = 0; i < l; ++i)
+            for (int e = 0; e < D; ++e) {
+              sk += k[KI(c, b, j * dstr + i, g) + e] * wk[((size_t)i * D + e) * D + n];
+              sv += v[KI(c, b, j * dstr + i, g) + e] * wv[((size_t)i * D + e) * D + n];
+            }
+          kc[CI(c, nc, b, j, g) + n] = round_store(sk, c->kv_round);
+          vc[CI(c, nc, b, j, g) + n] = round_store(sv, c->kv_round);
+        }
+}
+
+/* Its gradient for upstream dkc, dvc [B, Nc, Hkv, D]: the weights'
+ *   dWk[i D + e, n] = sum over (b, j, g) of k[b, j d + i, g, e] dkc[b, j, g, n]
+ * and the raw rows' dk[b, j d + i, g, e] += sum_n Wk[i D + e, n] dkc[b, j, g, n]
+ * summed over every block j whose tokens include the row (same for v).
+ * dk, dv, dwk, dwv are overwritten. */
+void orc_compress_mlp_bwd(const orc_cfg* c, const double* k, const double* v,
+                          const double* wk, const double* wv, const double* dkc,
+                          const double* dvc, double* dk, double* dv, double* dwk, double* dwv) {
+  const int nc = orc_num_cmp_blocks(c);
+  const int l = c->cmp_block, dstr = c->cmp_stride, D = c->D;
+  memset(dk, 0, (size_t)c->B * c->T * c->Hkv * D * sizeof(double));
+  memset(dv, 0, (size_t)c->B * c->T * c->Hkv * D * sizeof(double));
+  memset(dwk, 0, (size_t)l * D * D * sizeof(double));
+  memset(dwv, 0, (size_t)l * D * D * sizeof(double));
+  for (int b = 0; b < c->B; ++b)
+    for (int j = 0; j < nc; ++j)
+      for (int g = 0; g < c->Hkv; ++g)
+        for (int i = 0; i < l; ++i)
+          for (int e = 0; e < D; ++e) {
+            const size_t rowi = KI(c, b, j * dstr + i, g) + e;
+            double ak = 0.0, av = 0.0;
+            for (int n = 0; n < D; ++n) {
+              const double gk = dkc[CI(c, nc, b, j, g) + n], gv = dvc[CI(c, nc, b, j, g) + n];
+              dwk[((size_t)i * D + e) * D + n] += k[rowi] * gk;
+              dwv[((size_t)i * D + e) * D + n] += v[rowi] * gv;
+              ak += wk[((size_t)i * D + e) * D + n] * gk;
+              av += wv[((size_t)i * D + e) * D + n] * gv;
+            }
+            dk[rowi] += ak;
+            dv[rowi] += av;
+          }
+}

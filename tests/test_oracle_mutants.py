@@ -47,6 +47,12 @@ MUTANTS = {
                                   "      if (h == g * G) acc += dot(q + QI(c, b, t, h), kc + CI(c, nc, b, j, g), D);"),
     "moba_own_block_not_forced": ("  idx_row[n - 1] = cur;\n", "  idx_row[n - 1] = cand[n - 1];\n"),
     "moba_ties_to_higher_block": ("(gr == gb && cand[r] < cand[best])", "(gr == gb && cand[r] > cand[best])"),
+    "mlp_ignores_stride": ("              sk += k[KI(c, b, j * dstr + i, g) + e] * wk[((size_t)i * D + e) * D + n];",
+                           "              sk += k[KI(c, b, j * l + i, g) + e] * wk[((size_t)i * D + e) * D + n];"),
+    "mlp_weight_transposed": ("              sv += v[KI(c, b, j * dstr + i, g) + e] * wv[((size_t)i * D + e) * D + n];",
+                              "              sv += v[KI(c, b, j * dstr + i, g) + e] * wv[((size_t)i * D + n) * D + e];"),
+    "mlp_bwd_drops_weight_grad_row": ("              dwk[((size_t)i * D + e) * D + n] += k[rowi] * gk;",
+                                      "              dwk[((size_t)i * D + e) * D + n] += k[rowi] * gk * (i > 0);"),
     "remap_overlap_off_by_one": ("if (clo < hi && chi > lo) acc += cmp_score_row[i];",
                                  "if (clo <= hi && chi > lo) acc += cmp_score_row[i];"),
     "remap_first_block_only": ("if (clo < hi && chi > lo) acc += cmp_score_row[i];",

@@ -682,3 +682,72 @@ def test_moba_gate_hand_cases():
     q[0, t, 1, 1] = 1.0  # head 1 adds axis 1: sums 0.1, 0.9, 0.9, 0.9, 1.0
     _, _, idx = orc.moba_fwd(c, q, k, v)
     assert idx[0, t, 0].tolist() == [1, 4, 5]  # 1.0 first, then the lowest of three 0.9
+
+
+# ---------------------------------------------------------------- parametric compression
+def unfold_blocks(x, l, d):
+    """[B, T, H, D] -> [B, Nc, H, l*D]: each block's l rows flattened in
+    token order (torch's unfold; independent of the oracle)."""
+    t = torch.from_numpy(x)
+    u = t.unfold(1, l, d)                 # [B, Nc, H, D, l]
+    return u.permute(0, 1, 2, 4, 3).reshape(u.shape[0], u.shape[1], u.shape[2], -1)
+
+
+@pytest.mark.parametrize("l,d", [(8, 8), (8, 4), (4, 2), (6, 3)])
+def test_compress_mlp_is_unfold_matmul(l, d):
+    """One linear layer over the flattened block (reading R17) equals torch
+    unfold + matmul."""
+    c = cfg_small(T=40, cmp_block=l, cmp_stride=d, D=8)
+    _, k, v = qkv(c, 171)
+    g = np.random.default_rng(172)
+    wk, wv = g.standard_normal((l * c.D, c.D)), g.standard_normal((l * c.D, c.D))
+    kc, vc = orc.compress_mlp(c, k, v, wk, wv)
+    want_k = (unfold_blocks(k, l, d) @ torch.from_numpy(wk)).numpy()
+    want_v = (unfold_blocks(v, l, d) @ torch.from_numpy(wv)).numpy()
+    np.testing.assert_allclose(kc, want_k, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(vc, want_v, rtol=0, atol=1e-12)
+
+
+def test_compress_mlp_with_mean_weights_is_mean_pooling():
+    """W[i D + e, n] = (e == n) / l makes the layer mean-pooling (the pages'
+    replacement of the MLP is its special case): torch avg_pool1d."""
+    c = cfg_small(T=40, cmp_block=8, cmp_stride=4, D=8)
+    _, k, v = qkv(c, 173)
+    w = np.tile(np.eye(c.D) / c.cmp_block, (c.cmp_block, 1))
+    kc, vc = orc.compress_mlp(c, k, v, w, w)
+    pool = F.avg_pool1d(torch.from_numpy(k).permute(0, 2, 3, 1).reshape(-1, 1, c.T),
+                        c.cmp_block, c.cmp_stride)
+    want = pool.reshape(c.B, c.Hkv, c.D, -1).permute(0, 3, 1, 2).numpy()
+    np.testing.assert_allclose(kc, want, rtol=0, atol=1e-14)
+
+
+@pytest.mark.parametrize("l,d", [(4, 4), (4, 2)])
+def test_compress_mlp_backward_matches_autograd_and_differences(l, d):
+    c = cfg_small(B=1, T=14, Hkv=2, Hq=2, cmp_block=l, cmp_stride=d, D=3)
+    _, k, v = qkv(c, 174)
+    g = np.random.default_rng(175)
+    wk, wv = g.standard_normal((l * c.D, c.D)), g.standard_normal((l * c.D, c.D))
+    gk, gv = g.standard_normal((c.B, c.Nc, c.Hkv, c.D)), g.standard_normal((c.B, c.Nc, c.Hkv, c.D))
+    dk, dv, dwk, dwv = orc.compress_mlp_bwd(c, k, v, wk, wv, gk, gv)
+    tk, tv = torch.from_numpy(k).requires_grad_(), torch.from_numpy(v).requires_grad_()
+    twk, twv = torch.from_numpy(wk).requires_grad_(), torch.from_numpy(wv).requires_grad_()
+    uk = tk.unfold(1, l, d).permute(0, 1, 2, 4, 3).reshape(c.B, c.Nc, c.Hkv, -1)
+    uv = tv.unfold(1, l, d).permute(0, 1, 2, 4, 3).reshape(c.B, c.Nc, c.Hkv, -1)
+    loss = ((uk @ twk) * torch.from_numpy(gk)).sum() + ((uv @ twv) * torch.from_numpy(gv)).sum()
+    loss.backward()
+    for got, t in ((dk, tk), (dv, tv), (dwk, twk), (dwv, twv)):
+        np.testing.assert_allclose(got, t.grad.numpy(), rtol=0, atol=1e-12)
+    # and central differences of the oracle's own forward, on a few entries
+    def lossf(kk, vv, wkk, wvv):
+        a, b = orc.compress_mlp(c, kk, vv, wkk, wvv)
+        return float((a * gk).sum() + (b * gv).sum())
+    eps = 1e-6
+    for arr, grad in ((k, dk), (wk, dwk), (wv, dwv)):
+        for i in (0, arr.size // 2, arr.size - 1):
+            xp, xm = arr.copy(), arr.copy()
+            xp.flat[i] += eps
+            xm.flat[i] -= eps
+            args_p = [xp if a is arr else a for a in (k, v, wk, wv)]
+            args_m = [xm if a is arr else a for a in (k, v, wk, wv)]
+            fd = (lossf(*args_p) - lossf(*args_m)) / (2 * eps)
+            assert abs(fd - grad.flat[i]) <= 1e-7 * max(1.0, abs(fd))
