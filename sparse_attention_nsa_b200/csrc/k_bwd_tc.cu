@@ -22,8 +22,11 @@
 // S/dP as soon as they have loaded them, so the next block's MMAs overlap
 // this block's arithmetic; dS is single-buffered.
 // TMEM columns (256 per CTA): S [0,64), dP [64,128), dQ [128,192),
-// dS [192,224).  Warp roles (192 threads): warps 0-3 rows, warp 4 MMA issue
-// and TMEM owner, warp 5 TMA producer.
+// dS [192,224).  Warp roles (320 threads, two CTAs per SM): warps 0-7 rows
+// (warps w and w + 4 share the rows of TMEM lane quarter w, warp w the
+// first 32 keys of every block and warp w + 4 the last 32: P = exp(S - lse)
+// needs no statistics shared between them), warp 8 MMA issue and TMEM
+// owner, warp 9 TMA producer.
 #include <climits>
 
 #include "common.cuh"
@@ -39,7 +42,7 @@ using namespace sm100;
 constexpr int kRows = 128;
 constexpr int kKeys = 64;
 constexpr int kStages = 4;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;  // 8 row warps, the MMA warp, the TMA warp
 constexpr uint32_t kTileBytes = kKeys * 64 * 2;
 constexpr uint32_t kQBytes = kRows * 64 * 2;
 
@@ -79,7 +82,7 @@ constexpr uint32_t AT_OFF_DOH = AT_OFF_DOL + kQBytes;
 constexpr uint32_t AT_OFF_BAR = AT_OFF_DOH + kQBytes;
 constexpr uint32_t AT_OFF_MISC = AT_OFF_BAR + ((sizeof(Bars) + 15) / 16) * 16;
 constexpr uint32_t AT_OFF_LIST = AT_OFF_MISC + 16;
-constexpr int kAtThreads = 320;
+constexpr int kAtThreads = 448;  // plus 4 epilogue warps
 constexpr uint32_t kColDV = 256, kColDK = 320;  // TMEM columns of a pair's dV / dK
 
 __host__ __device__ inline int tokens_per_tile(int G) { return kRows / G; }
@@ -105,7 +108,7 @@ __host__ __device__ inline size_t list_ints(const Dims& d) {
 //   dV = P^T dO (fp16), dK = dS^T Q (bf16)  (M128 N64 K128: A the P / dS
 //   tiles read MN-major, the second block's tiles 16 KB after the first's;
 //   B the dO (fp16) / Q tiles read MN-major), fp32 in TMEM [256, 384);
-// warps 6-9 (thread = key of the pair) load them and add them to dk, dv
+// warps 10-13 (thread = key of the pair) load them and add them to dk, dv
 // with float4 atomics (so dk / dv depend on the order the atomics land in:
 // equal to the two-pass results up to fp32 rounding, not bit for bit).
 template <int MODE, bool ATOMIC = false>
@@ -150,8 +153,8 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       mbar_init(&bars->empty[s], 1);
     }
     mbar_init(&bars->s, 1);
-    mbar_init(&bars->sfree, 128);
-    mbar_init(&bars->ds, 128);
+    mbar_init(&bars->sfree, 256);
+    mbar_init(&bars->ds, 256);
     mbar_init(&bars->fin, 1);
     mbar_init(&bars->pfree, 1);
     mbar_init(&bars->kvfull, 1);
@@ -160,8 +163,8 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     fence_proxy_async_smem();
     *abort_flag = 0;
   }
-  if (warp == 4) tmem_alloc(tmem_slot, TMEM_COLS);
-  if (warp == 5 && lane == 0) {
+  if (warp == 8) tmem_alloc(tmem_slot, TMEM_COLS);
+  if (warp == 9 && lane == 0) {
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
@@ -234,7 +237,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const int n = *nblk_s;
   const int blk0 = blk[0];
 
-  if (warp == 5) {
+  if (warp == 9) {
     // ---- TMA producer --------------------------------------------------------------
     if (lane == 0) {
       mbar_expect_tx(&bars->q, kQBytes);
@@ -259,7 +262,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           drain_bar(&bars->full[i % NST], (i / NST) & 1);
       }
     }
-  } else if (warp == 4) {
+  } else if (warp == 8) {
     // ---- MMA issue: S, dP of block i, then dQ of block i-1 ------------------------------
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16(kRows, kKeys, false, false);
@@ -331,46 +334,53 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       mma_commit(&bars->fin);
       drain_bar(&bars->fin, 0);
     }
-  } else if (ATOMIC && warp >= 6) {
+  } else if (ATOMIC && warp >= 10) {
     // ---- single pass: dK / dV of each block pair into dk, dv with atomics --------------
     const int k = 32 * (warp & 3) + lane;  // key of the pair (TMEM lane k)
     const uint32_t lane_tmem = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const int npairs = (n + 1) / 2;
     for (int pi = 0; pi < npairs; ++pi) {
       if (!wait_bar_warp(&bars->kvfull, pi & 1, abort_flag, err)) break;
-      tc_fence_after();
-      float av[64], ak[64];
-      tmem_ld32(lane_tmem + kColDV, av);
-      tmem_ld32(lane_tmem + kColDV + 32u, av + 32);
-      tmem_ld32(lane_tmem + kColDK, ak);
-      tmem_ld32(lane_tmem + kColDK + 32u, ak + 32);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&bars->kvfree);
       const int bi = 2 * pi + (k >> 6);
-      if (bi >= n) continue;
-      const int key = blk[bi] * kKeys + (k & 63);
-      if (key >= nkeys) continue;
-      const size_t krow = (((size_t)b * nkeys + key) * d.Hkv + g) * 64;
-      float4* pv4 = reinterpret_cast<float4*>(dv_at + krow);
-      float4* pk4 = reinterpret_cast<float4*>(dk_at + krow);
+      const int key = bi < n ? blk[bi] * kKeys + (k & 63) : nkeys;
+      const size_t krow = (((size_t)b * nkeys + min(key, nkeys - 1)) * d.Hkv + g) * 64;
+#pragma unroll 1
+      for (int hc = 0; hc < 2; ++hc) {  // columns [32 hc, 32 hc + 32) of dV and dK
+        tc_fence_after();
+        float av[32], ak[32];
+        tmem_ld32(lane_tmem + kColDV + 32u * hc, av);
+        tmem_ld32(lane_tmem + kColDK + 32u * hc, ak);
+        tmem_wait_ld();
+        if (hc == 1) {  // both halves loaded: the next pair's MMAs may overwrite them
+          tc_fence_before();
+          mbar_arrive(&bars->kvfree);
+        }
+        if (key >= nkeys) continue;
+        float4* pv4 = reinterpret_cast<float4*>(dv_at + krow + 32 * hc);
+        float4* pk4 = reinterpret_cast<float4*>(dk_at + krow + 32 * hc);
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        atomicAdd(pv4 + c, make_float4(av[4 * c], av[4 * c + 1], av[4 * c + 2], av[4 * c + 3]));
-        atomicAdd(pk4 + c, make_float4(ak[4 * c] * d.scale, ak[4 * c + 1] * d.scale,
-                                       ak[4 * c + 2] * d.scale, ak[4 * c + 3] * d.scale));
+        for (int c = 0; c < 8; ++c) {
+          atomicAdd(pv4 + c, make_float4(av[4 * c], av[4 * c + 1], av[4 * c + 2], av[4 * c + 3]));
+          atomicAdd(pk4 + c, make_float4(ak[4 * c] * d.scale, ak[4 * c + 1] * d.scale,
+                                         ak[4 * c + 2] * d.scale, ak[4 * c + 3] * d.scale));
+        }
       }
     }
-  } else if (warp < 4) {
-    // ---- rows: thread r owns query row r -----------------------------------------------
-    const int r = tid;
+  } else if (warp < 8) {
+    // ---- rows: thread r owns query row r; warps w and w + 4 share row r = 32 (w % 4) +
+    // lane (TMEM lane quarter w % 4), warp w taking keys 0..31 of every block and warp
+    // w + 4 keys 32..63 (P needs no per-block statistics here: lse is known) ------------
+    const int qw = warp & 3, ch = warp >> 2;
+    const int r = 32 * qw + lane;
     const int tl = r / d.G, hh = r % d.G;
     const bool valid = tl < nvalid;
     const int t = pos0 + tl;
     const size_t row = ((size_t)b * d.Tq + t0 + tl) * d.Hq + (size_t)g * d.G + hh;
-    const uint32_t lane_tmem = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t lane_tmem = tmem + ((uint32_t)(qw * 32) << 16);
+    float* row_lse2 = (float*)(toks + (SEL ? TQ * (d.topk + 1) : 0));  // [128], then delta [128]
+    float* row_dl = row_lse2 + kRows;
     float dl = 0.f, lse2 = -INFINITY;
-    {  // delta = dO . o, and dO rounded to bf16 into the swizzled A tile
+    if (ch == 0) {  // delta = dO . o, and dO rounded to bf16 into the swizzled A tile
       const uint32_t drow = smem_u32(smem + OFF_DO) + (uint32_t)(r >> 3) * 1024u + (uint32_t)(r & 7) * 128u;
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
@@ -415,8 +425,16 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         delta[row] = dl;
         lse2 = lse[row] * kLog2e;
       }
+      row_lse2[r] = lse2;
+      row_dl[r] = dl;
       fence_proxy_async_smem();
-      mbar_arrive(&bars->dorows);
+      mbar_arrive(&bars->dorows);  // also publishes lse2 and delta of the row
+    }
+    bool ok = true;
+    if (ch == 1) {
+      ok = wait_bar_warp(&bars->dorows, 0, abort_flag, err);
+      lse2 = row_lse2[r];
+      dl = row_dl[r];
     }
     const int lo = MODE == 1 ? max(0, t - d.window + 1) : 0;
     const int khi = MODE == 2 ? cmp_nvis(d, t) - 1 : t;  // last visible key
@@ -424,60 +442,64 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     int ptr = 0;
     int nxt = SEL && valid ? lst[0] : INT_MAX;
     const float sl2 = d.scale * kLog2e;
-    bool ok = true;
-    for (int i = 0; i < n; ++i) {
+    const float nl2 = -lse2;
+    for (int i = 0; ok && i < n; ++i) {
       const int j = SEL ? blk[i] : blk0 + i;
-      const int k0 = j * kKeys;
+      const int k0 = j * kKeys + 32 * ch;  // this warp's first key of the block
       bool rowsel = valid && k0 <= khi && lse2 != -INFINITY;
       if (SEL) {
         const bool hit = nxt == j;
         if (hit) nxt = lst[++ptr];
         rowsel = rowsel && hit;
       } else {
-        rowsel = rowsel && (k0 + kKeys - 1 >= lo);
+        rowsel = rowsel && (k0 + 31 >= lo);
       }
       if (!wait_bar_warp(&bars->s, i & 1, abort_flag, err)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      uint32_t dsk[32];
-      uint32_t ppk[ATOMIC ? 32 : 1];
+      const bool any = __any_sync(0xffffffffu, rowsel);
+      uint32_t dsk[16];
+      uint32_t ppk[ATOMIC ? 16 : 1];
 #pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
-        float sv[32], pv[32];
-        tmem_ld32(lane_tmem + kColS + 32u * h2, sv);
-        tmem_ld32(lane_tmem + kColDP + 32u * h2, pv);
-        tmem_wait_ld();
+      for (int h2 = 0; h2 < 2; ++h2) {  // 16 keys at a time
+        float sv[16], pv[16];
+        if (any) {
+          tmem_ld16(lane_tmem + kColS + 32u * ch + 16u * h2, sv);
+          tmem_ld16(lane_tmem + kColDP + 32u * ch + 16u * h2, pv);
+          tmem_wait_ld();
+        }
         if (h2 == 1) {  // S and dP of this block are in registers: release them
           tc_fence_before();
           mbar_arrive(&bars->sfree);
         }
         if (rowsel) {
-          const bool part = !((k0 + kKeys - 1 <= khi) && (k0 >= lo));
+          const bool part = !((k0 + 31 <= khi) && (k0 >= lo));
 #pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            const int key = k0 + 32 * h2 + c;
-            float p0 = fast_exp2(fmaf(sv[c], sl2, -lse2));
-            float p1 = fast_exp2(fmaf(sv[c + 1], sl2, -lse2));
+          for (int c = 0; c < 16; c += 2) {
+            const int key = k0 + 16 * h2 + c;
+            float p0 = fast_exp2(fmaf(sv[c], sl2, nl2));
+            float p1 = fast_exp2(fmaf(sv[c + 1], sl2, nl2));
             if (part) {
               if (key > khi || key < lo) p0 = 0.f;
               if (key + 1 > khi || key + 1 < lo) p1 = 0.f;
             }
-            dsk[16 * h2 + c / 2] = pack_bf16(p0 * (pv[c] - dl), p1 * (pv[c + 1] - dl));
-            if constexpr (ATOMIC) ppk[16 * h2 + c / 2] = pack_f16(p0, p1);
+            dsk[8 * h2 + c / 2] = pack_bf16(p0 * (pv[c] - dl), p1 * (pv[c + 1] - dl));
+            if constexpr (ATOMIC) ppk[8 * h2 + c / 2] = pack_f16(p0, p1);
           }
         } else {
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            dsk[16 * h2 + c] = 0u;
-            if constexpr (ATOMIC) ppk[16 * h2 + c] = 0u;
+          for (int c = 0; c < 8; ++c) {
+            dsk[8 * h2 + c] = 0u;
+            if constexpr (ATOMIC) ppk[8 * h2 + c] = 0u;
           }
         }
       }
       if constexpr (ATOMIC) {
-        // P and dS of this row for the pair's dV / dK MMAs: row r of the
-        // tiles of half i & 1 (the pair's previous MMAs must be done with them)
+        // P and dS of this row's 32 keys for the pair's dV / dK MMAs: chunks
+        // 4 ch .. 4 ch + 3 of row r of the tiles of half i & 1 (the pair's
+        // previous MMAs must be done with them)
         const int hf = i & 1;
         if (hf == 0 && i >= 2) {
           if (!wait_bar_warp(&bars->pfree, ((i >> 1) - 1) & 1, abort_flag, err)) {
@@ -489,8 +511,8 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const uint32_t pa = smem_u32(smem + AT_OFF_P) + hf * kQBytes + line;
         const uint32_t sa = pa + 2 * kQBytes;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint32_t sw = (uint32_t)(c ^ (r & 7)) << 4;
+        for (int c = 0; c < 4; ++c) {
+          const uint32_t sw = (uint32_t)((4 * ch + c) ^ (r & 7)) << 4;
           st_shared_v4(pa + sw, ppk[4 * c], ppk[4 * c + 1], ppk[4 * c + 2], ppk[4 * c + 3]);
           st_shared_v4(sa + sw, dsk[4 * c], dsk[4 * c + 1], dsk[4 * c + 2], dsk[4 * c + 3]);
           if (hf == 0 && i == n - 1) {  // a last block alone: its pair half is zero
@@ -509,29 +531,26 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         tc_fence_after();
       }
-      tmem_st32u(lane_tmem + kColDS, dsk);
+      tmem_st16u(lane_tmem + kColDS + 16u * ch, dsk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars->ds);
     }
-    // epilogue: dq += scale * dQ (fp32, accumulated across branches)
-    float acc[64];
+    // epilogue: dq += scale * dQ (fp32, accumulated across branches), this
+    // warp's 32 of the row's 64 columns
+    float acc[32];
     bool have = false;
     if (ok && n > 0) have = wait_bar_warp(&bars->fin, 0, abort_flag, err);
     if (have) {
       tc_fence_after();
-      tmem_ld32(lane_tmem + kColDQ, acc);
-      tmem_ld32(lane_tmem + kColDQ + 32u, acc + 32);
+      tmem_ld32(lane_tmem + kColDQ + 32u * ch, acc);
       tmem_wait_ld();
-    } else {
-#pragma unroll
-      for (int c = 0; c < 64; ++c) acc[c] = 0.f;
     }
     tc_fence_before();
     if (valid && have) {
-      float4* dst = reinterpret_cast<float4*>(dq + row * 64);
+      float4* dst = reinterpret_cast<float4*>(dq + row * 64 + 32 * ch);
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
+      for (int c = 0; c < 8; ++c) {
         float4 x = dst[c];
         x.x = fmaf(acc[4 * c], d.scale, x.x);
         x.y = fmaf(acc[4 * c + 1], d.scale, x.y);
@@ -542,7 +561,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
   }
   __syncthreads();
-  if (warp == 4) {
+  if (warp == 8) {
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
@@ -1154,7 +1173,7 @@ cudaError_t launch_dq_tc_t(const Dims& d, const void* q, const void* k, const vo
       !make_tmap_bf16(&mk, k, d.Hkv, key_rows, 1, kKeys) ||
       !make_tmap_bf16(&mv, v, d.Hkv, key_rows, 1, kKeys))
     return cudaErrorInvalidValue;
-  const size_t smem = OFF_LIST + list_ints(d) * sizeof(int) + 1024;
+  const size_t smem = OFF_LIST + (list_ints(d) + 2 * kRows) * sizeof(int) + 1024;
   cudaError_t e = cudaFuncSetAttribute(bwd_dq_tc_kernel<MODE>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -1205,7 +1224,7 @@ cudaError_t launch_sel_bwd_atomic(const Dims& d, const void* q, const void* k, c
       !make_tmap_bf16(&mk, k, d.Hkv, (long)d.B * d.T, 1, kKeys) ||
       !make_tmap_bf16(&mv, v, d.Hkv, (long)d.B * d.T, 1, kKeys))
     return cudaErrorInvalidValue;
-  const size_t smem = AT_OFF_LIST + list_ints(d) * sizeof(int) + 1024;
+  const size_t smem = AT_OFF_LIST + (list_ints(d) + 2 * kRows) * sizeof(int) + 1024;
   cudaError_t e = cudaFuncSetAttribute(bwd_dq_tc_kernel<0, true>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
