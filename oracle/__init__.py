@@ -274,6 +274,17 @@ def cmp_bwd(cfg: Cfg, q, kc, vc, dO_cmp):
     return dq, dk, dv
 
 
+def cmp_bwd_kc(cfg: Cfg, q, kc, vc, dO_cmp):
+    """Compression-branch gradients stopped at the compressed tensors:
+    (dq, dkc, dvc), dkc/dvc [B, Nc, Hkv, D]."""
+    lib = _load()
+    q, kc, vc, dO = _f64(q), _f64(kc), _f64(vc), _f64(dO_cmp)
+    dq, dkc, dvc = np.zeros_like(q), np.zeros_like(kc), np.zeros_like(vc)
+    cc = cfg.c()
+    lib.orc_cmp_bwd_kc(C.byref(cc), _p(q), _p(kc), _p(vc), _p(dO), _p(dq), _p(dkc), _p(dvc))
+    return dq, dkc, dvc
+
+
 def gate_combine_bwd(cfg: Cfg, gates, dout, o_cmp, o_sel, o_swa):
     """(dgates, dO_cmp, dO_sel, dO_swa) of the gated combination."""
     lib = _load()

@@ -672,6 +672,41 @@ void orc_cmp_bwd(const orc_cfg* c, const double* q, const double* kc,
   }
 }
 
+/* The same backward stopped at the compressed keys and values: dq gets the
+ * branch's share and dkc, dvc [B, Nc, Hkv, D] the gradient of kc, vc
+ * (accumulated).  With a parametric compressor this is what flows into
+ * orc_compress_mlp_bwd. */
+void orc_cmp_bwd_kc(const orc_cfg* c, const double* q, const double* kc, const double* vc,
+                    const double* dO_cmp, double* dq, double* dkc, double* dvc) {
+  const int nc = orc_num_cmp_blocks(c);
+  const int G = c->Hq / c->Hkv;
+  const long ngrp = (long)c->B * c->Hkv;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (long bg = 0; bg < ngrp; ++bg) {
+    const int b = (int)(bg / c->Hkv), g = (int)(bg % c->Hkv);
+    const double** kr = (const double**)malloc(sizeof(double*) * (size_t)(nc + 1));
+    const double** vr = (const double**)malloc(sizeof(double*) * (size_t)(nc + 1));
+    double** dkr = (double**)malloc(sizeof(double*) * (size_t)(nc + 1));
+    double** dvr = (double**)malloc(sizeof(double*) * (size_t)(nc + 1));
+    for (int j = 0; j < nc; ++j) {
+      kr[j] = kc + CI(c, nc, b, j, g);
+      vr[j] = vc + CI(c, nc, b, j, g);
+      dkr[j] = dkc + CI(c, nc, b, j, g);
+      dvr[j] = dvc + CI(c, nc, b, j, g);
+    }
+    for (int t = 0; t < c->T; ++t) {
+      const int n = cmp_visible(c, t);
+      for (int h = g * G; h < (g + 1) * G; ++h)
+        attend_bwd(q + QI(c, b, t, h), c->D, c->scale, n, kr, vr, dO_cmp + QI(c, b, t, h),
+                   dq + QI(c, b, t, h), dkr, dvr);
+    }
+    free(kr);
+    free(vr);
+    free(dkr);
+    free(dvr);
+  }
+}
+
 /* Gradient of the gated combination: dgates[..., i] = dO . o_i for the
  * enabled branches (0 for disabled ones), and dO_i = gate_i * dO. */
 void orc_gate_combine_bwd(const orc_cfg* c, const double* gates,

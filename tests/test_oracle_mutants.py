@@ -53,6 +53,8 @@ MUTANTS = {
                               "              sv += v[KI(c, b, j * dstr + i, g) + e] * wv[((size_t)i * D + n) * D + e];"),
     "mlp_bwd_drops_weight_grad_row": ("              dwk[((size_t)i * D + e) * D + n] += k[rowi] * gk;",
                                       "              dwk[((size_t)i * D + e) * D + n] += k[rowi] * gk * (i > 0);"),
+    "cmp_bwd_kc_swaps_key_value_grads": ("      dkr[j] = dkc + CI(c, nc, b, j, g);\n      dvr[j] = dvc + CI(c, nc, b, j, g);",
+                                         "      dkr[j] = dvc + CI(c, nc, b, j, g);\n      dvr[j] = dkc + CI(c, nc, b, j, g);"),
     "remap_overlap_off_by_one": ("if (clo < hi && chi > lo) acc += cmp_score_row[i];",
                                  "if (clo <= hi && chi > lo) acc += cmp_score_row[i];"),
     "remap_first_block_only": ("if (clo < hi && chi > lo) acc += cmp_score_row[i];",

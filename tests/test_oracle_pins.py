@@ -751,3 +751,47 @@ def test_compress_mlp_backward_matches_autograd_and_differences(l, d):
             args_m = [xm if a is arr else a for a in (k, v, wk, wv)]
             fd = (lossf(*args_p) - lossf(*args_m)) / (2 * eps)
             assert abs(fd - grad.flat[i]) <= 1e-7 * max(1.0, abs(fd))
+
+
+@pytest.mark.parametrize("l,d", [(4, 4), (4, 2)])
+def test_cmp_bwd_kc_matches_central_differences(l, d):
+    """dkc, dvc, dq of the compression branch against central differences of
+    sum(dO . o_cmp) computed by the oracle's forward."""
+    c = cfg_small(B=1, T=20, Hq=4, Hkv=2, D=4, cmp_block=l, cmp_stride=d)
+    q, k, v = qkv(c, 176)
+    kc, vc = orc.compress(c, k, v)
+    g = np.random.default_rng(177)
+    kc, vc = kc + 0.3 * g.standard_normal(kc.shape), vc + 0.3 * g.standard_normal(vc.shape)
+    dO = g.standard_normal((c.B, c.T, c.Hq, c.D))
+    dq, dkc, dvc = orc.cmp_bwd_kc(c, q, kc, vc, dO)
+
+    def lossf(qq, a, b):
+        o, _, _ = orc.cmp_attn_scores(c, qq, a, b)
+        return float((o * dO).sum())
+    eps = 1e-6
+    for which, grad in ((0, dq), (1, dkc), (2, dvc)):
+        base = (q, kc, vc)[which]
+        for i in range(0, base.size, max(1, base.size // 9)):
+            xp, xm = base.copy(), base.copy()
+            xp.flat[i] += eps
+            xm.flat[i] -= eps
+            ap = [xp if j == which else (q, kc, vc)[j] for j in range(3)]
+            am = [xm if j == which else (q, kc, vc)[j] for j in range(3)]
+            fd = (lossf(*ap) - lossf(*am)) / (2 * eps)
+            assert abs(fd - grad.flat[i]) <= 1e-7 * max(1.0, abs(fd)), (which, i)
+
+
+def test_cmp_bwd_kc_through_mean_weights_is_cmp_bwd():
+    """Stopping at kc / vc and going on through the linear layer with mean
+    weights gives the mean-pool branch gradient on the raw rows."""
+    c = cfg_small(B=2, T=48, cmp_block=8, cmp_stride=4, D=8)
+    q, k, v = qkv(c, 178)
+    kc, vc = orc.compress(c, k, v)
+    dO = rand((c.B, c.T, c.Hq, c.D), 179)
+    dq_ref, dk_ref, dv_ref = orc.cmp_bwd(c, q, kc, vc, dO)
+    dq, dkc, dvc = orc.cmp_bwd_kc(c, q, kc, vc, dO)
+    w = np.tile(np.eye(c.D) / c.cmp_block, (c.cmp_block, 1))
+    dk, dv, _, _ = orc.compress_mlp_bwd(c, k, v, w, w, dkc, dvc)
+    np.testing.assert_allclose(dq, dq_ref, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(dk, dk_ref, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(dv, dv_ref, rtol=0, atol=1e-13)
