@@ -426,6 +426,8 @@ def run_gpu(args, rank: int, world: int, dist_on: bool) -> None:
     onep3b = run_1p3b(dev, flush, stream, max(3, args.steps // 2), peaks)
     # MoBA block attention (block 512, top-3) on the selection kernels
     moba = run_moba(dev, flush, stream, max(3, args.steps // 2), peaks)
+    # NSA on its parametric compressor (blocks of 32 every 16 tokens)
+    mlp = run_mlp(dev, flush, stream, max(3, args.steps // 2), peaks)
     # selection backward, two-pass against single-pass atomic
     selbwd = run_sel_bwd_compare(dev, flush, stream, 3, peaks)
     sampler.__exit__(None, None, None)
@@ -476,6 +478,7 @@ def run_gpu(args, rank: int, world: int, dist_on: bool) -> None:
         "long_context": long_ctx,
         "nsa_1p3b": onep3b,
         "moba": moba,
+        "mlp_compression": mlp,
         "sel_bwd_two_pass_vs_atomic": selbwd,
         "e2e": {"value": job_tokens_per_s(tokens_per_step, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
@@ -625,6 +628,77 @@ def run_moba(dev, flush, stream, steps, peaks) -> dict:
             "tflops": tf, "frac_bf16_peak": tf / peaks["bf16_tflops"], "flops_per_step": flops}
 
 
+def run_mlp(dev, flush, stream, steps, peaks) -> dict:
+    """NSA with its own parametric compressor (one linear layer over each
+    block's rows) at the 340M shape with NSA's original compression geometry
+    (blocks of 32 every 16 tokens; selection block 64, top-k 16, window
+    512), B=1 x 8192 tokens: the compressor forward and backward alone, the
+    whole forward and a training step (forward + backward), beside the same
+    forward on the mean pool."""
+    w = W.NSA_340M.replace(name="nsa_mlp_340m_gqa4_t8192_l32_d16_bf16", cmp_block=32,
+                           cmp_stride=16)
+    inp = W.make_inputs(w, seed=7, with_dout=True)
+    q, k, v, g, dout = (inp[n].to(dev) for n in ("q", "k", "v", "gates", "dout"))
+    wk, wv = (t.to(dev) for t in W.make_mlp_weights(w, seed=8))
+    p = nsa.params_for(w)
+    out = torch.empty_like(q)
+    ws = torch.empty(nsa.nsa_forward_mlp_workspace_size(p), dtype=torch.uint8, device=dev)
+    mws = nsa.alloc_workspace(p, dev)
+    fws = torch.empty(max(nsa.nsa_compress_mlp_workspace_size(p), 1), dtype=torch.uint8,
+                      device=dev)
+    f32 = torch.float32
+    kc = torch.empty((w.B, w.Nc, w.Hkv, w.D), dtype=w.dtype, device=dev)
+    vc = torch.empty_like(kc)
+    dkc = torch.randn((w.B, w.Nc, w.Hkv, w.D), dtype=f32, device=dev)
+    dvc = torch.randn_like(dkc)
+    dk = torch.zeros((w.B, w.T, w.Hkv, w.D), dtype=f32, device=dev)
+    dv = torch.zeros_like(dk)
+    dwk = torch.empty((w.cmp_block * w.D, w.D), dtype=f32, device=dev)
+    dwv = torch.empty_like(dwk)
+    cws = torch.empty(nsa.nsa_compress_mlp_bwd_workspace_size(p), dtype=torch.uint8, device=dev)
+    saved = nsa.alloc_saved(p, dev)
+    bws = torch.empty(nsa.nsa_backward_mlp_workspace_size(p), dtype=torch.uint8, device=dev)
+    dq = torch.empty((w.B, w.T, w.Hq, w.D), dtype=f32, device=dev)
+    dkk, dvv = torch.empty_like(dk), torch.empty_like(dk)
+    dg = torch.empty((w.B, w.T, w.Hq, 3), dtype=f32, device=dev)
+
+    def cfwd():
+        nsa.nsa_compress_mlp(p, k, v, wk, wv, kc, vc, fws)
+
+    def cbwd():
+        nsa.nsa_compress_mlp_bwd(p, k, v, wk, wv, dkc, dvc, dk, dv, dwk, dwv, cws)
+
+    def fwd_mlp():
+        nsa.nsa_forward_mlp(p, q, k, v, wk, wv, g, out, None, ws)
+
+    def fwd_mean():
+        nsa.nsa_forward(p, q, k, v, g, out, None, mws)
+
+    def train():
+        nsa.nsa_forward_mlp(p, q, k, v, wk, wv, g, out, saved, ws)
+        nsa.nsa_backward_mlp(p, q, k, v, wk, wv, g, dout, saved, dq, dkk, dvv, dwk, dwv, dg, bws)
+
+    for fn in (cfwd, cbwd, fwd_mlp, fwd_mean, train, train):
+        fn()
+    res = {}
+    for name, fn in (("compress_fwd_ms", cfwd), ("compress_bwd_ms", cbwd),
+                     ("fwd_ms", fwd_mlp), ("fwd_mean_pool_ms", fwd_mean), ("train_step_ms", train)):
+        res[name] = statistics.mean(timed_steps(fn, steps, flush, stream))
+    if nsa.nsa_last_device_error() != 0:
+        raise RuntimeError("device-side check failed in the parametric-compression leg")
+    # the compressor's GEMM work: kc and vc, one (l*D) x D product per block row
+    rows = w.B * w.Nc * w.Hkv
+    cflops = 2 * 2 * rows * (w.cmp_block * w.D) * w.D
+    ctf = cflops / (res["compress_fwd_ms"] * 1e-3) / 1e12
+    btf = 2 * cflops / (res["compress_bwd_ms"] * 1e-3) / 1e12
+    res.update({"workload": w.name, "tokens_per_s": w.B * w.T / (res["fwd_ms"] * 1e-3),
+                "compress_fwd_tflops": ctf, "compress_bwd_tflops": btf,
+                "compress_flops": cflops,
+                "note": "compressor FLOPs 2 x (kc, vc) x rows x (l D) x D; its backward "
+                        "(dW and the rows' gradient) twice that"})
+    return res
+
+
 def run_long(dev, flush, stream, steps, peaks) -> dict:
     """Long-context forward: the pruned MQA workload (B=1, 32768 tokens,
     selection + window).  Its selection runs block-major (Nb = 32 top-k);
@@ -716,8 +790,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--leg", default="all",
                     choices=["all", "forward", "decode", "train", "long", "onep3b", "moba",
-                             "selbwd"],
-                    help="forward / decode / train / long / onep3b / moba / selbwd: run only that leg on one GPU "
+                             "selbwd", "mlp"],
+                    help="forward / decode / train / long / onep3b / moba / selbwd / mlp: run only that leg on one GPU "
                          "and print its numbers (for profiling that leg alone); all: the "
                          "benchmark")
     ap.add_argument("--batch", type=int, default=None,
@@ -746,6 +820,8 @@ def main():
                 batch=args.batch if args.batch else 8)}))
         elif args.leg == "moba":
             print(json.dumps({"moba": run_moba(dev, flush, stream, args.steps, peaks)}))
+        elif args.leg == "mlp":
+            print(json.dumps({"mlp_compression": run_mlp(dev, flush, stream, args.steps, peaks)}))
         elif args.leg == "onep3b":
             print(json.dumps({"nsa_1p3b": run_1p3b(dev, flush, stream, args.steps, peaks)}))
         else:

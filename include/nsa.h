@@ -378,6 +378,69 @@ nsa_status nsa_backward(const nsa_params* p, const void* q, const void* k,
                         void* stream);
 
 /* ========================================================================
+ * Parametric compression: NSA's own compressor.
+ * "DeepSeek's Native Sparse Attention", COMPRESSION (a small learned layer
+ * turns each block of keys / values into one compressed key / value; blocks
+ * of length l every d tokens) and "Sparsity is Cool", Method and Key claims
+ * (the study replaces it with mean-pooling).  The pages give no shape for
+ * the layer: this is the plainest reading, one linear map over the block's
+ * l rows flattened in token order, shared by every sequence, block and KV
+ * group:
+ *   kc[b, j, g, n] = sum_{i<l} sum_{e<D} k[b, j*d + i, g, e] * wk[i*D + e, n]
+ * and vc likewise with wv.  wk, wv: [l*D, D] row-major, the dtype of k
+ * (bf16 only here; NSA_ERR_UNSUPPORTED otherwise).  Mean-pooling is the
+ * special case wk[i*D + e, n] = (e == n) / l.  The products accumulate in
+ * fp32 on the tensor cores; kc, vc are stored as bf16.  The whole-path
+ * entries below run NSA with this compressor in place of the mean pool.
+ * ======================================================================== */
+
+/* kc, vc [B, Nc, Hkv, D] from k, v [B, T, Hkv, D] and the weights.
+ * workspace: nsa_compress_mlp_workspace_size(p) bytes, 256-byte aligned
+ * (fp32 partial sums when the blocks alone would leave SMs idle; it may be
+ * 0, and then workspace may be NULL). */
+nsa_status nsa_compress_mlp_workspace_size(const nsa_params* p, size_t* bytes);
+nsa_status nsa_compress_mlp(const nsa_params* p, const void* k, const void* v,
+                            const void* wk, const void* wv, void* kc, void* vc,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/* Gradient of nsa_compress_mlp for upstream dkc, dvc (fp32 [B, Nc, Hkv, D]):
+ *   dwk[i*D + e, n] = sum over (b, j, g) of k[b, j*d + i, g, e] dkc[b, j, g, n]
+ * (overwritten; dwv likewise, both fp32 [l*D, D]) and the raw rows'
+ *   dk[b, j*d + i, g, e] += sum_n wk[i*D + e, n] dkc[b, j, g, n]
+ * summed, in block order, over every block j holding the row (dk, dv fp32
+ * [B, T, Hkv, D], ADDED to).  dkc, dvc enter the tensor cores as a bf16
+ * pair (value and remainder), so they are carried to about 16 bits.
+ * workspace: nsa_compress_mlp_bwd_workspace_size(p) bytes, 256-byte aligned. */
+nsa_status nsa_compress_mlp_bwd_workspace_size(const nsa_params* p, size_t* bytes);
+nsa_status nsa_compress_mlp_bwd(const nsa_params* p, const void* k, const void* v,
+                                const void* wk, const void* wv, const float* dkc,
+                                const float* dvc, float* dk, float* dv, float* dwk,
+                                float* dwv, void* workspace, size_t workspace_bytes,
+                                void* stream);
+
+/* nsa_forward with kc, vc from nsa_compress_mlp.  Same arguments and saved
+ * tensors as nsa_forward; workspace: nsa_forward_mlp_workspace_size(p)
+ * bytes, 256-byte aligned (nsa_forward's plus the compressor's). */
+nsa_status nsa_forward_mlp_workspace_size(const nsa_params* p, size_t* bytes);
+nsa_status nsa_forward_mlp(const nsa_params* p, const void* q, const void* k,
+                           const void* v, const void* wk, const void* wv,
+                           const float* gates, void* out, const nsa_saved* saved,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/* nsa_backward for nsa_forward_mlp: also overwrites dwk, dwv (fp32 [l*D, D];
+ * zero when the compression branch is off, as top-k passes no gradient) and
+ * adds the compressor's share to dk, dv.  saved must hold the kc, vc that
+ * nsa_forward_mlp wrote.  workspace: nsa_backward_mlp_workspace_size(p)
+ * bytes, 256-byte aligned. */
+nsa_status nsa_backward_mlp_workspace_size(const nsa_params* p, size_t* bytes);
+nsa_status nsa_backward_mlp(const nsa_params* p, const void* q, const void* k,
+                            const void* v, const void* wk, const void* wv,
+                            const float* gates, const void* dout,
+                            const nsa_saved* saved, float* dq, float* dk, float* dv,
+                            float* dwk, float* dwv, float* dgates, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
+/* ========================================================================
  * MoBA block attention on the same selection kernels.
  * "Sparsity is Cool: Reverse-Engineering MoBA and NSA", Method (MoBA with
  * block 512 and top-k 3) and Key claims (dense below about 1.5k tokens);

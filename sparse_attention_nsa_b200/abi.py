@@ -35,7 +35,10 @@ EXPORTS = ("nsa_status_string", "nsa_check_params", "nsa_workspace_size",
            "nsa_sel_workspace_size", "nsa_sel_attn_fwd_ws", "nsa_set_kernel_events",
            "nsa_forward_host_workspace_size", "nsa_forward_host",
            "nsa_moba_workspace_size", "nsa_moba_forward", "nsa_moba_backward",
-           "nsa_sel_attn_bwd_atomic")
+           "nsa_sel_attn_bwd_atomic", "nsa_compress_mlp_workspace_size", "nsa_compress_mlp",
+           "nsa_compress_mlp_bwd_workspace_size", "nsa_compress_mlp_bwd",
+           "nsa_forward_mlp_workspace_size", "nsa_forward_mlp", "nsa_backward_mlp_workspace_size",
+           "nsa_backward_mlp")
 
 
 class NsaError(RuntimeError):
@@ -122,6 +125,16 @@ def load():
                                  C.c_int),
             "nsa_moba_backward": ([C.POINTER(MobaParams)] + [vp] * 11 + [C.c_size_t, vp],
                                   C.c_int),
+            "nsa_compress_mlp_workspace_size": ([P, C.POINTER(C.c_size_t)], C.c_int),
+            "nsa_compress_mlp": ([P] + [vp] * 7 + [C.c_size_t, vp], C.c_int),
+            "nsa_forward_mlp_workspace_size": ([P, C.POINTER(C.c_size_t)], C.c_int),
+            "nsa_compress_mlp_bwd_workspace_size": ([P, C.POINTER(C.c_size_t)], C.c_int),
+            "nsa_compress_mlp_bwd": ([P] + [vp] * 11 + [C.c_size_t, vp], C.c_int),
+            "nsa_forward_mlp": ([P, vp, vp, vp, vp, vp, vp, vp, C.POINTER(Saved), vp,
+                                 C.c_size_t, vp], C.c_int),
+            "nsa_backward_mlp_workspace_size": ([P, C.POINTER(C.c_size_t)], C.c_int),
+            "nsa_backward_mlp": ([P, vp, vp, vp, vp, vp, vp, vp, C.POINTER(Saved)] + [vp] * 7
+                                 + [C.c_size_t, vp], C.c_int),
         }
         for name, (args, res) in sig.items():
             f = getattr(lib, name)
@@ -499,31 +512,66 @@ def alloc_workspace(p: Params, device=None) -> torch.Tensor:
     return torch.empty(max(n, 1), dtype=torch.uint8, device=device or "cuda")
 
 
+def alloc_saved(p: Params, dev) -> dict:
+    s, dt = _shapes(p), p.torch_dtype
+    saved = {"kc": torch.empty(s["kc"], dtype=dt, device=dev),
+             "vc": torch.empty(s["kc"], dtype=dt, device=dev),
+             "o_cmp": torch.zeros(s["o"], dtype=dt, device=dev),
+             "lse_cmp": torch.zeros(s["lse"], dtype=torch.float32, device=dev),
+             "score": torch.zeros(s["score"], dtype=torch.float32, device=dev),
+             "idx": torch.zeros(s["idx"], dtype=torch.int32, device=dev),
+             "o_sel": torch.zeros(s["o"], dtype=dt, device=dev),
+             "lse_sel": torch.zeros(s["lse"], dtype=torch.float32, device=dev),
+             "o_swa": torch.zeros(s["o"], dtype=dt, device=dev),
+             "lse_swa": torch.zeros(s["lse"], dtype=torch.float32, device=dev)}
+    return {k_: t for k_, t in saved.items() if t.numel() > 0}
+
+
 def forward(p: Params, q, k, v, gates, keep: bool = False, workspace=None, stream=None):
     """Allocate outputs with torch and run nsa_forward.
 
     Returns out, or (out, saved-dict) with every intermediate when keep=True.
     """
-    s, dt = _shapes(p), p.torch_dtype
     dev = q.device
-    out = torch.empty(s["o"], dtype=dt, device=dev)
-    saved = None
-    if keep:
-        saved = {"kc": torch.empty(s["kc"], dtype=dt, device=dev),
-                 "vc": torch.empty(s["kc"], dtype=dt, device=dev),
-                 "o_cmp": torch.zeros(s["o"], dtype=dt, device=dev),
-                 "lse_cmp": torch.zeros(s["lse"], dtype=torch.float32, device=dev),
-                 "score": torch.zeros(s["score"], dtype=torch.float32, device=dev),
-                 "idx": torch.zeros(s["idx"], dtype=torch.int32, device=dev),
-                 "o_sel": torch.zeros(s["o"], dtype=dt, device=dev),
-                 "lse_sel": torch.zeros(s["lse"], dtype=torch.float32, device=dev),
-                 "o_swa": torch.zeros(s["o"], dtype=dt, device=dev),
-                 "lse_swa": torch.zeros(s["lse"], dtype=torch.float32, device=dev)}
-        saved = {k_: t for k_, t in saved.items() if t.numel() > 0}
+    out = torch.empty(_shapes(p)["o"], dtype=p.torch_dtype, device=dev)
+    saved = alloc_saved(p, dev) if keep else None
     if workspace is None:
         workspace = alloc_workspace(p, dev)
     nsa_forward(p, q, k, v, gates, out, saved, workspace, stream)
     return (out, saved) if keep else out
+
+
+def forward_mlp(p: Params, q, k, v, wk, wv, gates, keep: bool = False, workspace=None,
+                stream=None):
+    """forward() with the parametric compressor (nsa_forward_mlp)."""
+    dev = q.device
+    out = torch.empty(_shapes(p)["o"], dtype=p.torch_dtype, device=dev)
+    saved = alloc_saved(p, dev) if keep else None
+    if workspace is None:
+        workspace = torch.empty(max(nsa_forward_mlp_workspace_size(p), 1), dtype=torch.uint8,
+                                device=dev)
+    nsa_forward_mlp(p, q, k, v, wk, wv, gates, out, saved, workspace, stream)
+    return (out, saved) if keep else out
+
+
+def backward_mlp(p: Params, q, k, v, wk, wv, gates, dout, saved: dict, workspace=None,
+                 stream=None):
+    """Allocate fp32 gradients with torch and run nsa_backward_mlp:
+    (dq, dk, dv, dwk, dwv, dgates)."""
+    s, dev = _shapes(p), q.device
+    f = torch.float32
+    dq = torch.empty(s["q"], dtype=f, device=dev)
+    dk = torch.empty(s["k"], dtype=f, device=dev)
+    dv = torch.empty(s["k"], dtype=f, device=dev)
+    dwk = torch.empty(_w_shape(p), dtype=f, device=dev)
+    dwv = torch.empty(_w_shape(p), dtype=f, device=dev)
+    dg = torch.empty(s["gates"], dtype=f, device=dev)
+    if workspace is None:
+        workspace = torch.empty(max(nsa_backward_mlp_workspace_size(p), 1), dtype=torch.uint8,
+                                device=dev)
+    nsa_backward_mlp(p, q, k, v, wk, wv, gates, dout, saved, dq, dk, dv, dwk, dwv, dg,
+                     workspace, stream)
+    return dq, dk, dv, dwk, dwv, dg
 
 
 # ------------------------------------------------------------------ MoBA
@@ -566,3 +614,110 @@ def nsa_moba_backward(p: MobaParams, q, k, v, idx, out, lse, dout, dq, dk, dv, w
         _ptr(lse, s["lse"], f, "lse"), _ptr(dout, s["q"], f, "dout"), _ptr(dq, s["q"], f, "dq"),
         _ptr(dk, s["k"], f, "dk"), _ptr(dv, s["k"], f, "dv"), _ptr(workspace, name="workspace"),
         workspace.numel() * workspace.element_size(), _stream(stream)), "nsa_moba_backward")
+
+
+# ------------------------------------------------------------------ parametric compression
+def _w_shape(p: Params):
+    return (p.cmp_block * p.D, p.D)
+
+
+def nsa_compress_mlp_workspace_size(p: Params) -> int:
+    n = C.c_size_t(0)
+    _check(load().nsa_compress_mlp_workspace_size(C.byref(p), C.byref(n)),
+           "nsa_compress_mlp_workspace_size")
+    return n.value
+
+
+def nsa_compress_mlp(p: Params, k, v, wk, wv, kc, vc, workspace=None, stream=None):
+    """workspace: None allocates nsa_compress_mlp_workspace_size(p) bytes."""
+    s, dt = _shapes(p), p.torch_dtype
+    if workspace is None:
+        n = nsa_compress_mlp_workspace_size(p)
+        workspace = torch.empty(n, dtype=torch.uint8, device=k.device) if n else None
+    wp, wb = _ws(workspace)
+    _check(load().nsa_compress_mlp(
+        C.byref(p), _ptr(k, s["k"], dt, "k"), _ptr(v, s["k"], dt, "v"),
+        _ptr(wk, _w_shape(p), dt, "wk"), _ptr(wv, _w_shape(p), dt, "wv"),
+        _ptr(kc, s["kc"], dt, "kc", p.Nc == 0), _ptr(vc, s["kc"], dt, "vc", p.Nc == 0),
+        wp, wb, _stream(stream)), "nsa_compress_mlp")
+
+
+def nsa_compress_mlp_bwd_workspace_size(p: Params) -> int:
+    n = C.c_size_t(0)
+    _check(load().nsa_compress_mlp_bwd_workspace_size(C.byref(p), C.byref(n)),
+           "nsa_compress_mlp_bwd_workspace_size")
+    return n.value
+
+
+def nsa_compress_mlp_bwd(p: Params, k, v, wk, wv, dkc, dvc, dk, dv, dwk, dwv, workspace,
+                         stream=None):
+    s, dt, f = _shapes(p), p.torch_dtype, torch.float32
+    wp, wb = _ws(workspace)
+    _check(load().nsa_compress_mlp_bwd(
+        C.byref(p), _ptr(k, s["k"], dt, "k"), _ptr(v, s["k"], dt, "v"),
+        _ptr(wk, _w_shape(p), dt, "wk"), _ptr(wv, _w_shape(p), dt, "wv"),
+        _ptr(dkc, s["kc"], f, "dkc", p.Nc == 0), _ptr(dvc, s["kc"], f, "dvc", p.Nc == 0),
+        _ptr(dk, s["k"], f, "dk"), _ptr(dv, s["k"], f, "dv"),
+        _ptr(dwk, _w_shape(p), f, "dwk"), _ptr(dwv, _w_shape(p), f, "dwv"), wp, wb,
+        _stream(stream)), "nsa_compress_mlp_bwd")
+
+
+def _saved_struct(p: Params, saved: dict | None) -> "Saved":
+    s, dt = _shapes(p), p.torch_dtype
+    sv = Saved()
+    if saved:
+        want = {"kc": (s["kc"], dt), "vc": (s["kc"], dt), "o_cmp": (s["o"], dt),
+                "lse_cmp": (s["lse"], torch.float32), "score": (s["score"], torch.float32),
+                "idx": (s["idx"], torch.int32), "o_sel": (s["o"], dt),
+                "lse_sel": (s["lse"], torch.float32), "o_swa": (s["o"], dt),
+                "lse_swa": (s["lse"], torch.float32)}
+        for name, t in saved.items():
+            if t is None or t.numel() == 0:
+                continue
+            shp, tdt = want[name]
+            setattr(sv, name, _ptr(t, shp, tdt, name).value)
+    return sv
+
+
+def nsa_forward_mlp_workspace_size(p: Params) -> int:
+    n = C.c_size_t(0)
+    _check(load().nsa_forward_mlp_workspace_size(C.byref(p), C.byref(n)),
+           "nsa_forward_mlp_workspace_size")
+    return n.value
+
+
+def nsa_forward_mlp(p: Params, q, k, v, wk, wv, gates, out, saved: dict | None = None,
+                    workspace=None, stream=None):
+    """nsa_forward with the parametric compressor (weights wk, wv [l D, D])."""
+    s, dt = _shapes(p), p.torch_dtype
+    sv = _saved_struct(p, saved)
+    wp, wb = _ws(workspace)
+    _check(load().nsa_forward_mlp(
+        C.byref(p), _ptr(q, s["q"], dt, "q"), _ptr(k, s["k"], dt, "k"), _ptr(v, s["k"], dt, "v"),
+        _ptr(wk, _w_shape(p), dt, "wk"), _ptr(wv, _w_shape(p), dt, "wv"),
+        _ptr(gates, s["gates"], torch.float32, "gates"), _ptr(out, s["o"], dt, "out"),
+        C.byref(sv), wp, wb, _stream(stream)), "nsa_forward_mlp")
+
+
+def nsa_backward_mlp_workspace_size(p: Params) -> int:
+    n = C.c_size_t(0)
+    _check(load().nsa_backward_mlp_workspace_size(C.byref(p), C.byref(n)),
+           "nsa_backward_mlp_workspace_size")
+    return n.value
+
+
+def nsa_backward_mlp(p: Params, q, k, v, wk, wv, gates, dout, saved: dict, dq, dk, dv, dwk,
+                     dwv, dgates, workspace, stream=None):
+    s, dt, f = _shapes(p), p.torch_dtype, torch.float32
+    sv = Saved()
+    for name, t in saved.items():
+        if t is not None and t.numel() > 0:
+            setattr(sv, name, _ptr(t, name=name).value)
+    wp, wb = _ws(workspace)
+    _check(load().nsa_backward_mlp(
+        C.byref(p), _ptr(q, s["q"], dt, "q"), _ptr(k, s["k"], dt, "k"), _ptr(v, s["k"], dt, "v"),
+        _ptr(wk, _w_shape(p), dt, "wk"), _ptr(wv, _w_shape(p), dt, "wv"),
+        _ptr(gates, s["gates"], f, "gates"), _ptr(dout, s["o"], dt, "dout"), C.byref(sv),
+        _ptr(dq, s["q"], f, "dq"), _ptr(dk, s["k"], f, "dk"), _ptr(dv, s["k"], f, "dv"),
+        _ptr(dwk, _w_shape(p), f, "dwk"), _ptr(dwv, _w_shape(p), f, "dwv"),
+        _ptr(dgates, s["gates"], f, "dgates"), wp, wb, _stream(stream)), "nsa_backward_mlp")

@@ -94,6 +94,14 @@ size_t sel_bm_ws_bytes(const Dims& d);
 cudaError_t launch_sel_bm(const Dims& d, const void* q, const void* k, const void* v,
                           const int32_t* idx, void* o_sel, float* lse_sel, int* err,
                           const EpilogueFuse* fz, void* ws, cudaStream_t s);
+// launch_sel_bm in two steps: the reverse map and work units (prep), then the
+// block-major kernel and the merge (run), so that other work can be ordered
+// between them
+cudaError_t launch_sel_bm_prep(const Dims& d, const int32_t* idx, int* err, void* ws,
+                               cudaStream_t s);
+cudaError_t launch_sel_bm_run(const Dims& d, const void* q, const void* k, const void* v,
+                              const int32_t* idx, void* o_sel, float* lse_sel, int* err,
+                              const EpilogueFuse* fz, void* ws, cudaStream_t s);
 cudaError_t launch_combine(const Dims& d, const float* gates, const void* o_cmp,
                            const void* o_sel, const void* o_swa, void* out,
                            cudaStream_t s);
@@ -121,11 +129,12 @@ size_t revmap_chunk_ints(const Dims& d);
 cudaError_t launch_revmap(const Dims& d, const int32_t* idx, int* chunk, int* offsets,
                           int* list, cudaStream_t s);
 // the same map for the block-major selection forward: entries are
-// query << 6 | slot in no particular order within a block's list, indices
-// that break the forward's rule are reported in err, and per (sequence,
-// group) the lists are cut into work units of at most tpu entries
-// (units[bg * umax + u] = (block, first, end) for u < ucount[bg]).
-// cursor: B * Hkv * Nb ints.
+// query << 6 | slot, in ascending query order within a block's list (the
+// same lists on every run), indices that break the forward's rule are
+// reported in err, and per (sequence, group) the lists are cut into work
+// units of at most tpu entries (units[bg * umax + u] = (block, first, end)
+// for u < ucount[bg]).  cursor: B * Hkv * Nb ints (each block's first
+// position).
 // Reverse map of the forward's selection plus its work units: per (sequence,
 // group) at most umax units of at most tpu = k * tq list entries (k <= 4
 // tiles of tq entries), written sorted by size (units of k tiles first, then
@@ -147,6 +156,22 @@ cudaError_t launch_dkdv_tc(const Dims& d, int mode, const void* q, const void* k
                            const void* vals, const float* lse, const float* delta,
                            const float* dO, void* dO16, const int* offsets, const int* list,
                            float* dk, float* dv, float* part, int* err, cudaStream_t s);
+
+// Parametric (one linear layer) compression, bf16, D = 64: kc = sum_i k rows
+// j d + i times W[i], same for vc (k_cmp_mlp.cu).  The backward overwrites
+// dwk / dwv and adds the raw rows' gradient into dk / dv; ws holds
+// cmp_mlp_bwd_ws_bytes(d) bytes, 256-byte aligned.
+bool cmp_mlp_eligible(const Dims& d);
+size_t cmp_mlp_fwd_ws_bytes(const Dims& d);  // 256-byte aligned, may be 0
+size_t cmp_mlp_bwd_ws_bytes(const Dims& d);
+cudaError_t launch_cmp_mlp_fwd(const Dims& d, const void* k, const void* v, const void* wk,
+                               const void* wv, void* kc, void* vc, void* ws, int* err,
+                               cudaStream_t s);
+cudaError_t launch_cmp_mlp_bwd(const Dims& d, const void* k, const void* v, const void* wk,
+                               const void* wv, const float* dkc, const float* dvc, float* dk,
+                               float* dv, float* dwk, float* dwv, void* ws, int* err,
+                               cudaStream_t s);
+
 cudaError_t launch_pool_bwd(const Dims& d, const float* dkc, const float* dvc, float* dk,
                             float* dv, cudaStream_t s);
 

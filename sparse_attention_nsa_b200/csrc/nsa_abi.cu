@@ -4,6 +4,7 @@
 // workspace, and enqueues kernels on the caller's stream.  It allocates no
 // device memory and never synchronises except in nsa_last_device_error.
 #include <algorithm>
+#include <initializer_list>
 #include <mutex>
 
 #include "common.cuh"
@@ -308,9 +309,13 @@ nsa_status nsa_gate_combine(const nsa_params* p, const float* gates, const void*
   return NSA_OK;
 }
 
-// Library-owned side stream per device for running the window branch
-// concurrently with compression -> top-k -> selection inside one forward.
-// Created on first use (with that device current) and kept until exit.
+// Library-owned side stream per device, at the device's highest stream
+// priority, for the dependent chain compression -> top-k -> reverse map of a
+// forward while the window branch runs on the caller's stream: the block
+// scheduler gives the chain's blocks the SMs first as they free up, and the
+// window's fill the rest (launched the other way round, the window's blocks
+// took every SM before the chain could start).  Created on first use (with
+// that device current) and kept until exit.
 struct SideStream {
   cudaStream_t s2 = nullptr;
   cudaEvent_t fork = nullptr, join = nullptr;
@@ -323,7 +328,10 @@ static SideStream* side_stream_locked() {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
   SideStream& ss = g_side[dev];
   if (!ss.s2) {
-    if (cudaStreamCreateWithFlags(&ss.s2, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    int least = 0, greatest = 0;
+    if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess) greatest = 0;
+    if (cudaStreamCreateWithPriority(&ss.s2, cudaStreamNonBlocking, greatest) != cudaSuccess)
+      return nullptr;
     if (cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
         cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess)
       return nullptr;
@@ -362,24 +370,27 @@ static nsa_status run_forward(const Dims& d, const void* q, const void* k, const
   const bool bm = use_sel_bm(d);
   if (sel && swa && nsa::swa_combine_fusable(d)) {
     // The window branch does not depend on compression, top-k or selection:
-    // it runs on the side stream while those run here, and the selection
-    // kernel, last on this stream, applies the gates in its epilogue.
+    // those run as a high-priority chain on the side stream while the window
+    // runs here, and the selection kernel, last on this stream, applies the
+    // gates in its epilogue.
     std::lock_guard<std::mutex> lock(g_side_mu);
     SideStream* ss = side_stream_locked();
     if (ss) {
       if (cudaEventRecord(ss->fork, s) != cudaSuccess ||
           cudaStreamWaitEvent(ss->s2, ss->fork, 0) != cudaSuccess)
         return NSA_ERR_CUDA;
-      const cudaError_t ew = nsa::launch_swa_fwd(d, q, k, v, o_swa, S.lse_swa, ss->s2);
+      cudaError_t em = cudaSuccess;
+      if (!kc_given) em = nsa::launch_compress(d, k, v, kc, vc, ss->s2);
+      if (em == cudaSuccess)
+        em = nsa::launch_cmp_scores(d, q, kc, vc, cmp ? o_cmp : nullptr, cmp ? lse_cmp : nullptr,
+                                    score, err_word(), ss->s2);
+      if (em == cudaSuccess) em = nsa::launch_topk(d, score, idx, ss->s2);
+      if (em == cudaSuccess && bm)
+        em = nsa::launch_sel_bm_prep(d, idx, err_word(), w + c.off[W_SELBM], ss->s2);
       // the join is enqueued whatever happens, so no side-stream work can
       // outlive this call's ordering on the caller's stream
       const cudaError_t ej = cudaEventRecord(ss->join, ss->s2);
-      cudaError_t em = cudaSuccess;
-      if (!kc_given) em = nsa::launch_compress(d, k, v, kc, vc, s);
-      if (em == cudaSuccess)
-        em = nsa::launch_cmp_scores(d, q, kc, vc, cmp ? o_cmp : nullptr, cmp ? lse_cmp : nullptr,
-                                    score, err_word(), s);
-      if (em == cudaSuccess) em = nsa::launch_topk(d, score, idx, s);
+      const cudaError_t ew = nsa::launch_swa_fwd(d, q, k, v, o_swa, S.lse_swa, s);
       const cudaError_t ewait = cudaStreamWaitEvent(s, ss->join, 0);
       if (ew != cudaSuccess || ej != cudaSuccess || em != cudaSuccess || ewait != cudaSuccess)
         return NSA_ERR_CUDA;
@@ -389,8 +400,8 @@ static nsa_status run_forward(const Dims& d, const void* q, const void* k, const
                                    {0, 2},
                                    1,
                                    out};
-        NSA_TRY_CUDA(nsa::launch_sel_bm(d, q, k, v, idx, S.o_sel, S.lse_sel, err_word(), &fz,
-                                        w + c.off[W_SELBM], s));
+        NSA_TRY_CUDA(nsa::launch_sel_bm_run(d, q, k, v, idx, S.o_sel, S.lse_sel, err_word(), &fz,
+                                            w + c.off[W_SELBM], s));
         return NSA_OK;
       }
       NSA_TRY_CUDA(nsa::launch_sel_fwd_combine(d, q, k, v, idx, S.o_sel, S.lse_sel, err_word(),
@@ -645,14 +656,27 @@ nsa_status swa_bwd_body(const Dims& d, const void* q, const void* k, const void*
   return NSA_OK;
 }
 
+// The parametric compressor of nsa_backward_mlp: its inputs, its weights'
+// gradients and its own workspace.
+struct MlpGrad {
+  const void *k, *v, *wk, *wv;
+  float *dwk, *dwv;
+  void* ws;
+};
+
 nsa_status cmp_bwd_body(const Dims& d, const void* q, const void* kc, const void* vc,
                         const void* o_cmp, const float* lse_cmp, const float* dO_cmp,
                         float* dq, float* dk, float* dv, char* w, const BwdCarve& c,
-                        cudaStream_t s) {
+                        cudaStream_t s, const MlpGrad* mlp = nullptr) {
   float* delta = (float*)(w + c.delta);
   float* dkc = (float*)(w + c.dkc);
   float* dvc = (float*)(w + c.dvc);
-  if (d.Nc == 0) return NSA_OK;  // nothing visible anywhere: no gradient
+  if (d.Nc == 0) {  // nothing visible anywhere: no gradient
+    if (mlp)
+      NSA_TRY_CUDA(nsa::launch_cmp_mlp_bwd(d, mlp->k, mlp->v, mlp->wk, mlp->wv, dkc, dvc, dk, dv,
+                                           mlp->dwk, mlp->dwv, mlp->ws, err_word(), s));
+    return NSA_OK;
+  }
   const size_t nkc = (size_t)d.B * d.Nc * d.Hkv * 64 * 4;
   NSA_TRY_CUDA(cudaMemsetAsync(dkc, 0, nkc, s));
   NSA_TRY_CUDA(cudaMemsetAsync(dvc, 0, nkc, s));
@@ -660,7 +684,11 @@ nsa_status cmp_bwd_body(const Dims& d, const void* q, const void* kc, const void
   NSA_TRY_CUDA(nsa::launch_dkdv(d, 2, q, kc, vc, lse_cmp, delta, dO_cmp, w + c.dO16, nullptr, nullptr,
                                 dkc, dvc,
                                 (float*)(w + c.part), err_word(), s));
-  NSA_TRY_CUDA(nsa::launch_pool_bwd(d, dkc, dvc, dk, dv, s));
+  if (mlp)
+    NSA_TRY_CUDA(nsa::launch_cmp_mlp_bwd(d, mlp->k, mlp->v, mlp->wk, mlp->wv, dkc, dvc, dk, dv,
+                                         mlp->dwk, mlp->dwv, mlp->ws, err_word(), s));
+  else
+    NSA_TRY_CUDA(nsa::launch_pool_bwd(d, dkc, dvc, dk, dv, s));
   return NSA_OK;
 }
 
@@ -764,13 +792,15 @@ nsa_status nsa_cmp_bwd(const nsa_params* p, const void* q, const void* kc, const
                       (cudaStream_t)stream);
 }
 
-nsa_status nsa_backward(const nsa_params* p, const void* q, const void* k, const void* v,
-                        const float* gates, const void* dout, const nsa_saved* sv, float* dq,
-                        float* dk, float* dv, float* dgates, void* workspace,
-                        size_t workspace_bytes, void* stream) {
-  Dims d;
-  nsa_status st = fill_dims(p, &d);
-  if (st != NSA_OK) return st;
+}  // extern "C"
+
+namespace {
+
+nsa_status backward_body(const Dims& d, const void* q, const void* k, const void* v,
+                         const float* gates, const void* dout, const nsa_saved* sv, float* dq,
+                         float* dk, float* dv, float* dgates, void* workspace,
+                         size_t workspace_bytes, cudaStream_t s, MlpGrad* mlp) {
+  nsa_status st = NSA_OK;
   if (!sv) return NSA_ERR_INVALID_ARG;
   for (const void* ptr : {q, k, v, (const void*)gates, dout, (const void*)dq, (const void*)dk,
                           (const void*)dv, (const void*)dgates})
@@ -785,9 +815,10 @@ nsa_status nsa_backward(const nsa_params* p, const void* q, const void* k, const
     return NSA_ERR_INVALID_ARG;
   if (swa && (!aligned16(sv->o_swa) || !aligned16(sv->lse_swa))) return NSA_ERR_INVALID_ARG;
   const BwdCarve c = bwd_carve(d);
-  if (!ws_ok(workspace, workspace_bytes, c.total)) return NSA_ERR_WORKSPACE;
-  cudaStream_t s = (cudaStream_t)stream;
+  const size_t need = c.total + (mlp ? nsa::cmp_mlp_bwd_ws_bytes(d) : 0);
+  if (!ws_ok(workspace, workspace_bytes, need)) return NSA_ERR_WORKSPACE;
   char* w = (char*)workspace;
+  if (mlp) mlp->ws = w + c.total;
   float* dO[3] = {(float*)(w + c.dO[0]), (float*)(w + c.dO[1]), (float*)(w + c.dO[2])};
   NSA_TRY_CUDA(nsa::launch_gate_bwd(d, gates, dout, sv->o_cmp, sv->o_sel, sv->o_swa, dgates,
                                     cmp ? dO[0] : nullptr, sel ? dO[1] : nullptr,
@@ -796,8 +827,14 @@ nsa_status nsa_backward(const nsa_params* p, const void* q, const void* k, const
   NSA_TRY_CUDA(cudaMemsetAsync(dk, 0, (size_t)d.B * d.T * d.Hkv * 64 * 4, s));
   NSA_TRY_CUDA(cudaMemsetAsync(dv, 0, (size_t)d.B * d.T * d.Hkv * 64 * 4, s));
   if (cmp) {
-    st = cmp_bwd_body(d, q, sv->kc, sv->vc, sv->o_cmp, sv->lse_cmp, dO[0], dq, dk, dv, w, c, s);
+    st = cmp_bwd_body(d, q, sv->kc, sv->vc, sv->o_cmp, sv->lse_cmp, dO[0], dq, dk, dv, w, c, s,
+                      mlp);
     if (st != NSA_OK) return st;
+  } else if (mlp) {
+    // compressed keys reach only the selection scores, and top-k passes no gradient
+    const size_t wbytes = (size_t)d.lc * 64 * 64 * sizeof(float);
+    NSA_TRY_CUDA(cudaMemsetAsync(mlp->dwk, 0, wbytes, s));
+    NSA_TRY_CUDA(cudaMemsetAsync(mlp->dwv, 0, wbytes, s));
   }
   if (sel) {
     st = sel_bwd_body(d, q, k, v, sv->idx, sv->o_sel, sv->lse_sel, dO[1], dq, dk, dv, w, c, s);
@@ -808,6 +845,145 @@ nsa_status nsa_backward(const nsa_params* p, const void* q, const void* k, const
     if (st != NSA_OK) return st;
   }
   return NSA_OK;
+}
+
+// d, the parametric compressor's pointers: bf16, D = 64, 16-byte aligned
+nsa_status mlp_args_ok(const Dims& d, std::initializer_list<const void*> ptrs) {
+  if (!nsa::cmp_mlp_eligible(d)) return NSA_ERR_UNSUPPORTED;
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return NSA_ERR_INVALID_ARG;
+  return NSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+nsa_status nsa_backward(const nsa_params* p, const void* q, const void* k, const void* v,
+                        const float* gates, const void* dout, const nsa_saved* sv, float* dq,
+                        float* dk, float* dv, float* dgates, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  Dims d;
+  nsa_status st = fill_dims(p, &d);
+  if (st != NSA_OK) return st;
+  return backward_body(d, q, k, v, gates, dout, sv, dq, dk, dv, dgates, workspace,
+                       workspace_bytes, (cudaStream_t)stream, nullptr);
+}
+
+// ---- parametric compression ----------------------------------------------------
+
+nsa_status nsa_compress_mlp_workspace_size(const nsa_params* p, size_t* bytes) {
+  Dims d;
+  nsa_status st = fill_dims(p, &d);
+  if (st != NSA_OK) return st;
+  if (!bytes) return NSA_ERR_INVALID_ARG;
+  *bytes = nsa::cmp_mlp_fwd_ws_bytes(d);
+  return NSA_OK;
+}
+
+nsa_status nsa_compress_mlp(const nsa_params* p, const void* k, const void* v, const void* wk,
+                            const void* wv, void* kc, void* vc, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  Dims d;
+  nsa_status st = fill_dims(p, &d);
+  if (st != NSA_OK) return st;
+  st = mlp_args_ok(d, {k, v, wk, wv});
+  if (st != NSA_OK) return st;
+  if (d.Nc > 0 && (!aligned16(kc) || !aligned16(vc))) return NSA_ERR_INVALID_ARG;
+  const size_t need = nsa::cmp_mlp_fwd_ws_bytes(d);
+  if (need > 0 && !ws_ok(workspace, workspace_bytes, need)) return NSA_ERR_WORKSPACE;
+  NSA_TRY_CUDA(nsa::launch_cmp_mlp_fwd(d, k, v, wk, wv, kc, vc, workspace, err_word(),
+                                       (cudaStream_t)stream));
+  return NSA_OK;
+}
+
+nsa_status nsa_compress_mlp_bwd_workspace_size(const nsa_params* p, size_t* bytes) {
+  Dims d;
+  nsa_status st = fill_dims(p, &d);
+  if (st != NSA_OK) return st;
+  if (!bytes) return NSA_ERR_INVALID_ARG;
+  *bytes = nsa::cmp_mlp_bwd_ws_bytes(d);
+  return NSA_OK;
+}
+
+nsa_status nsa_compress_mlp_bwd(const nsa_params* p, const void* k, const void* v,
+                                const void* wk, const void* wv, const float* dkc,
+                                const float* dvc, float* dk, float* dv, float* dwk, float* dwv,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  Dims d;
+  nsa_status st = fill_dims(p, &d);
+  if (st != NSA_OK) return st;
+  st = mlp_args_ok(d, {k, v, wk, wv, dk, dv, dwk, dwv});
+  if (st != NSA_OK) return st;
+  if (d.Nc > 0 && (!aligned16(dkc) || !aligned16(dvc))) return NSA_ERR_INVALID_ARG;
+  if (!ws_ok(workspace, workspace_bytes, nsa::cmp_mlp_bwd_ws_bytes(d))) return NSA_ERR_WORKSPACE;
+  NSA_TRY_CUDA(nsa::launch_cmp_mlp_bwd(d, k, v, wk, wv, dkc, dvc, dk, dv, dwk, dwv, workspace,
+                                       err_word(), (cudaStream_t)stream));
+  return NSA_OK;
+}
+
+nsa_status nsa_forward_mlp(const nsa_params* p, const void* q, const void* k, const void* v,
+                           const void* wk, const void* wv, const float* gates, void* out,
+                           const nsa_saved* saved, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+  Dims d;
+  nsa_status st = fill_dims(p, &d);
+  if (st != NSA_OK) return st;
+  st = mlp_args_ok(d, {q, k, v, wk, wv, gates, out});
+  if (st != NSA_OK) return st;
+  nsa_saved sv = saved ? *saved : nsa_saved{};
+  const void* ptrs[10] = {sv.kc, sv.vc, sv.o_cmp, sv.lse_cmp, sv.score,
+                          sv.idx, sv.o_sel, sv.lse_sel, sv.o_swa, sv.lse_swa};
+  for (const void* ptr : ptrs)
+    if (ptr && (((uintptr_t)ptr) & 15u)) return NSA_ERR_INVALID_ARG;
+  const Carve c = carve(d, saved);
+  const size_t need = c.total + nsa::cmp_mlp_fwd_ws_bytes(d);
+  if (need > 0 && !ws_ok(workspace, workspace_bytes, need)) return NSA_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  char* w = (char*)workspace;
+  // kc / vc take the first two slots, the compressor's partial sums the end;
+  // the rest of the forward carves what lies between
+  if (!sv.kc) sv.kc = w + c.off[W_KC];
+  if (!sv.vc) sv.vc = w + c.off[W_VC];
+  const bool need_kc = d.branch_mask & (NSA_BRANCH_CMP | NSA_BRANCH_SEL);
+  if (need_kc)
+    NSA_TRY_CUDA(nsa::launch_cmp_mlp_fwd(d, k, v, wk, wv, sv.kc, sv.vc, w + c.total, err_word(), s));
+  const size_t used = c.off[W_OCMP];
+  return run_forward(d, q, k, v, true, gates, out, &sv, used ? w + used : workspace,
+                     c.total - used, s);
+}
+
+nsa_status nsa_forward_mlp_workspace_size(const nsa_params* p, size_t* bytes) {
+  Dims d;
+  nsa_status st = fill_dims(p, &d);
+  if (st != NSA_OK) return st;
+  if (!bytes) return NSA_ERR_INVALID_ARG;
+  *bytes = carve(d, nullptr).total + nsa::cmp_mlp_fwd_ws_bytes(d);
+  return NSA_OK;
+}
+
+nsa_status nsa_backward_mlp_workspace_size(const nsa_params* p, size_t* bytes) {
+  Dims d;
+  nsa_status st = fill_dims(p, &d);
+  if (st != NSA_OK) return st;
+  if (!bytes) return NSA_ERR_INVALID_ARG;
+  *bytes = bwd_carve(d).total + nsa::cmp_mlp_bwd_ws_bytes(d);
+  return NSA_OK;
+}
+
+nsa_status nsa_backward_mlp(const nsa_params* p, const void* q, const void* k, const void* v,
+                            const void* wk, const void* wv, const float* gates, const void* dout,
+                            const nsa_saved* sv, float* dq, float* dk, float* dv, float* dwk,
+                            float* dwv, float* dgates, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  Dims d;
+  nsa_status st = fill_dims(p, &d);
+  if (st != NSA_OK) return st;
+  st = mlp_args_ok(d, {wk, wv, dwk, dwv});
+  if (st != NSA_OK) return st;
+  MlpGrad mlp{k, v, wk, wv, dwk, dwv, nullptr};
+  return backward_body(d, q, k, v, gates, dout, sv, dq, dk, dv, dgates, workspace,
+                       workspace_bytes, (cudaStream_t)stream, &mlp);
 }
 
 }  // extern "C"

@@ -124,6 +124,19 @@ def make_inputs(w: Workload, seed: int = 0, with_dout: bool = False) -> dict:
     return out
 
 
+def make_mlp_weights(w: Workload, seed: int = 0) -> tuple:
+    """Draw the parametric compressor's weights wk, wv [cmp_block * D, D] in
+    w.dtype: Gaussian with variance 1 / (cmp_block * D), the usual fan-in
+    initialisation of a linear layer (the pages train theirs; no trained
+    weights exist here)."""
+    g = torch.Generator().manual_seed(seed)
+    fan_in = w.cmp_block * w.D
+    std = 1.0 / math.sqrt(fan_in)
+    wk = torch.randn((fan_in, w.D), generator=g, dtype=torch.float32) * std
+    wv = torch.randn((fan_in, w.D), generator=g, dtype=torch.float32) * std
+    return wk.to(w.dtype), wv.to(w.dtype)
+
+
 def make_decode_inputs(w: Workload, seed: int = 0) -> dict:
     """Draw one decode step: the query of position T-1 of each sequence and
     caches of T keys/values that already hold that position.
