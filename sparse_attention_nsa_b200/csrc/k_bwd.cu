@@ -238,14 +238,34 @@ rev_chunk_scan_kernel(int* __restrict__ chunk, int* __restrict__ offsets, Dims d
   __shared__ int utotal;
   const int bg = blockIdx.x;
   int* cc = chunk + (size_t)bg * nchunk * d.Nb;
-  for (int j = threadIdx.x; j < d.Nb; j += blockDim.x) {
-    int run = 0;
-    for (int c = 0; c < nchunk; ++c) {
-      const int v = cc[(size_t)c * d.Nb + j];
-      cc[(size_t)c * d.Nb + j] = run;
-      run += v;
+  // each block's counts over the chunks -> the chunks' first positions
+  // within it: P lanes of a warp share a block (P a power of two, so a
+  // group never straddles warps), each sums a contiguous range of chunks,
+  // a shuffle scan over the group places the ranges
+  int P = 1;
+  while (P < 32 && P * 2 * d.Nb <= (int)blockDim.x && P < nchunk) P *= 2;
+  const int sub = threadIdx.x & (P - 1);
+  const int c0 = (int)((long)nchunk * sub / P), c1 = (int)((long)nchunk * (sub + 1) / P);
+  for (int jb = 0; jb < d.Nb; jb += (int)blockDim.x / P) {
+    const int j = jb + (int)threadIdx.x / P;
+    const bool ok = j < d.Nb;
+    int part = 0;
+    if (ok)
+      for (int c = c0; c < c1; ++c) part += cc[(size_t)c * d.Nb + j];
+    int incl = part;
+    for (int o = 1; o < P; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o, P);
+      if (sub >= o) incl += y;
     }
-    tot[j] = run;
+    if (ok) {
+      int run = incl - part;
+      for (int c = c0; c < c1; ++c) {
+        const int v = cc[(size_t)c * d.Nb + j];
+        cc[(size_t)c * d.Nb + j] = run;
+        run += v;
+      }
+      if (sub == P - 1) tot[j] = incl;
+    }
   }
   __syncthreads();
   // exclusive scan of tot over j: each thread a contiguous range
@@ -287,8 +307,7 @@ rev_chunk_scan_kernel(int* __restrict__ chunk, int* __restrict__ offsets, Dims d
     if (units) tot[d.Nb] = run;  // with units tot holds Nb + 1 offsets
   }
   __syncthreads();
-  for (int j = threadIdx.x; j < d.Nb; j += blockDim.x)
-    for (int c = 0; c < nchunk; ++c) cc[(size_t)c * d.Nb + j] += tot[j];
+  for (int x = threadIdx.x; x < nchunk * d.Nb; x += blockDim.x) cc[x] += tot[x % d.Nb];
   if (!units) return;
   // Work units of at most tpu list entries (tpu = kseg tiles of tq entries):
   // block j's list [off[j], off[j+1]) in consecutive pieces.  The group's
@@ -404,90 +423,67 @@ rev_chunk_scan_kernel(int* __restrict__ chunk, int* __restrict__ offsets, Dims d
   }
 }
 
-// one warp per (chunk, group, sequence)
-__global__ void __launch_bounds__(32)
-rev_chunk_fill_kernel(const int32_t* __restrict__ idx, const int* __restrict__ chunk,
-                      int* __restrict__ list, Dims d) {
-  extern __shared__ int sm[];  // run[Nb], bits[Nb]
-  int* run = sm;
-  unsigned* bits = (unsigned*)(sm + d.Nb);
+// The list fill of the forward (entries query << 6 | slot, topk <= 64) and
+// of the backward (entries query): per chunk of kRevChunk queries, one
+// thread per query, a block's entries in ascending query order from the
+// chunk's scanned first position for that block, so the lists are the same
+// on every run.  Warp w marks in bits[w][j] the lanes whose query chose
+// block j (atomicOr: the result does not depend on the order of the
+// updates); thread j turns the warps' counts into each warp's first
+// position; a (query, slot) pair lands at pos[w][j] + the number of lower
+// lanes of its warp that chose j.
+constexpr int kRevWarps = kRevChunk / 32;
+template <bool SLOT>
+__global__ void __launch_bounds__(kRevChunk)
+rev_fill_kernel(const int32_t* __restrict__ idx, const int* __restrict__ chunk,
+                int* __restrict__ list, Dims d) {
+  extern __shared__ int sm[];  // bits[kRevWarps][Nb], pos[kRevWarps][Nb]
+  unsigned* bits = reinterpret_cast<unsigned*>(sm);
+  int* pos = sm + kRevWarps * d.Nb;
   const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int nchunk = gridDim.x;
-  const int lane = threadIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const size_t bg = (size_t)b * d.Hkv + g;
-  const int* base = chunk + (bg * nchunk + c) * d.Nb;
-  for (int j = lane; j < d.Nb; j += 32) {
-    run[j] = base[j];
-    bits[j] = 0u;
-  }
-  __syncwarp();
-  int* lst = list + bg * (size_t)d.Tq * d.topk;
-  const unsigned lt = (1u << lane) - 1u;
-  for (int grp = 0; grp < kRevChunk / 32; ++grp) {
-    const int tq = c * kRevChunk + grp * 32 + lane;
-    const bool q_ok = tq < d.Tq;
-    const int32_t* ir = idx + (((size_t)b * d.Tq + (q_ok ? tq : 0)) * d.Hkv + g) * d.topk;
-    const int cur = (d.q_off + tq) / d.l;
-    for (int s = 0; s < d.topk; ++s)
-      if (q_ok && rev_valid(ir, s, cur)) atomicOr(&bits[ir[s]], 1u << lane);
-    __syncwarp();
-    for (int s = 0; s < d.topk; ++s)
-      if (q_ok && rev_valid(ir, s, cur)) {
-        const int j = ir[s];
-        lst[run[j] + __popc(bits[j] & lt)] = tq;
-      }
-    __syncwarp();
-    for (int s = 0; s < d.topk; ++s)
-      if (q_ok && rev_valid(ir, s, cur)) {
-        const int j = ir[s];
-        const unsigned m = bits[j];
-        if ((m & lt) == 0u) {  // the lowest lane that chose j advances its position
-          run[j] += __popc(m);
-          bits[j] = 0u;
-        }
-      }
-    __syncwarp();
-  }
-}
-
-// The forward's fill, entries query << 6 | slot (topk <= 64).  The order
-// inside a block's list is free (each (query, slot) pair is computed on its
-// own), so a CTA of kRevChunk queries counts its pairs per block in shared
-// memory, reserves each block's range with one global atomic on the block's
-// cursor (started at its scanned offset), and places its pairs with shared
-// atomics.  One thread per query.
-__global__ void __launch_bounds__(kRevChunk)
-rev_atomic_fill_kernel(const int32_t* __restrict__ idx, int* __restrict__ cursor,
-                       int* __restrict__ list, Dims d) {
-  extern __shared__ int sh[];  // count[Nb], base[Nb]
-  int* cnt = sh;
-  int* base = sh + d.Nb;
-  const int tq = blockIdx.x * kRevChunk + threadIdx.x;
-  const int g = blockIdx.y, b = blockIdx.z;
+  for (int x = threadIdx.x; x < kRevWarps * d.Nb; x += blockDim.x) bits[x] = 0u;
+  __syncthreads();
+  const int tq = c * kRevChunk + threadIdx.x;
   const bool q_ok = tq < d.Tq;
-  const size_t bg = (size_t)b * d.Hkv + g;
   const int32_t* ir = idx + (((size_t)b * d.Tq + (q_ok ? tq : 0)) * d.Hkv + g) * d.topk;
   const int cur = (d.q_off + tq) / d.l;
-  for (int j = threadIdx.x; j < d.Nb; j += blockDim.x) cnt[j] = 0;
-  __syncthreads();
+  unsigned* mine = bits + warp * d.Nb;
   if (q_ok)
     for (int s = 0; s < d.topk; ++s)
-      if (rev_valid(ir, s, cur)) atomicAdd(&cnt[ir[s]], 1);
+      if (rev_valid(ir, s, cur)) atomicOr(&mine[ir[s]], 1u << lane);
   __syncthreads();
-  int* cb = cursor + bg * d.Nb;
+  const int* base = chunk + (bg * nchunk + c) * d.Nb;
   for (int j = threadIdx.x; j < d.Nb; j += blockDim.x) {
-    const int c = cnt[j];
-    base[j] = c ? atomicAdd(cb + j, c) : 0;
-    cnt[j] = 0;
+    int run = base[j];
+#pragma unroll
+    for (int w = 0; w < kRevWarps; ++w) {
+      pos[w * d.Nb + j] = run;
+      run += __popc(bits[w * d.Nb + j]);
+    }
   }
   __syncthreads();
   int* lst = list + bg * (size_t)d.Tq * d.topk;
+  const unsigned lt = (1u << lane) - 1u;
+  const int* mpos = pos + warp * d.Nb;
   if (q_ok)
     for (int s = 0; s < d.topk; ++s)
       if (rev_valid(ir, s, cur)) {
         const int j = ir[s];
-        lst[base[j] + atomicAdd(&cnt[j], 1)] = (tq << 6) | s;
+        lst[mpos[j] + __popc(mine[j] & lt)] = SLOT ? ((tq << 6) | s) : tq;
       }
+}
+
+cudaError_t launch_rev_fill(const Dims& d, bool slot, const int32_t* idx, const int* chunk,
+                            int* list, int nchunk, cudaStream_t s) {
+  const size_t smem = 2 * (size_t)kRevWarps * d.Nb * sizeof(int);
+  auto kern = slot ? rev_fill_kernel<true> : rev_fill_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<dim3(nchunk, d.Hkv, d.B), kRevChunk, smem, s>>>(idx, chunk, list, d);
+  return cudaGetLastError();
 }
 
 // ---- pass 2: dK, dV, key-stationary ----------------------------------------------
@@ -687,9 +683,9 @@ cudaError_t launch_revmap(const Dims& d, const int32_t* idx, int* chunk, int* of
                                                                               nullptr, nullptr);
   rev_chunk_scan_kernel<<<d.B * d.Hkv, 1024, nb_bytes, s>>>(chunk, offsets, d, nchunk, nullptr,
                                                            nullptr, nullptr, 0, 1, 0);
-  rev_chunk_fill_kernel<<<dim3(nchunk, d.Hkv, d.B), 32, 2 * nb_bytes, s>>>(idx, chunk,
-                                                                                  list, d);
-  return cudaGetLastError();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_rev_fill(d, false, idx, chunk, list, nchunk, s);
 }
 
 cudaError_t launch_revmap_units(const Dims& d, const int32_t* idx, int* chunk, int* offsets,
@@ -700,17 +696,15 @@ cudaError_t launch_revmap_units(const Dims& d, const int32_t* idx, int* chunk, i
   const int nchunk = (d.Tq + kRevChunk - 1) / kRevChunk;
   if (nchunk == 0 || d.Nb == 0) return cudaSuccess;
   const size_t nb_bytes = (size_t)d.Nb * sizeof(int);
-  // per-(sequence, group, block) totals (chunk holds them: B * Hkv * Nb ints)
-  cudaError_t e = cudaMemsetAsync(chunk, 0, (size_t)d.B * d.Hkv * nb_bytes, s);
-  if (e != cudaSuccess) return e;
-  // with totals given the count kernel writes only them (its chunk output is unused)
-  rev_chunk_count_kernel<<<dim3(nchunk, d.Hkv, d.B), kRevChunk, nb_bytes, s>>>(idx, nullptr, d,
-                                                                              err, chunk);
+  // per-(chunk, block) counts -> each chunk's first position per block, the
+  // offsets and the work units -> the entries in ascending query order
+  rev_chunk_count_kernel<<<dim3(nchunk, d.Hkv, d.B), kRevChunk, nb_bytes, s>>>(idx, chunk, d,
+                                                                              err, nullptr);
   rev_chunk_scan_kernel<<<d.B * d.Hkv, 1024, (kMaxUnitClasses + 1) * nb_bytes + sizeof(int), s>>>(
-      chunk, offsets, d, 1, units, ucount, cursor, tpu, tq, umax);
-  rev_atomic_fill_kernel<<<dim3(nchunk, d.Hkv, d.B), kRevChunk, 2 * nb_bytes, s>>>(idx, cursor,
-                                                                                   list, d);
-  return cudaGetLastError();
+      chunk, offsets, d, nchunk, units, ucount, cursor, tpu, tq, umax);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_rev_fill(d, true, idx, chunk, list, nchunk, s);
 }
 
 template <typename T, int MODE>

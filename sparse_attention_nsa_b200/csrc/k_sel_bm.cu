@@ -803,9 +803,27 @@ bool sel_bm_eligible(const Dims& d) {
 
 size_t sel_bm_ws_bytes(const Dims& d) { return bm_carve(d).total; }
 
+cudaError_t launch_sel_bm_prep(const Dims& d, const int32_t* idx, int* err, void* ws,
+                               cudaStream_t s) {
+  const BmCarve c = bm_carve(d);
+  char* w = (char*)ws;
+  return launch_revmap_units(d, idx, (int*)(w + c.chunk), (int*)(w + c.offsets),
+                             (int*)(w + c.cursor), (int*)(w + c.list), (int4*)(w + c.units),
+                             (int*)(w + c.ucount), kSeg * tile_tokens(d.G), tile_tokens(d.G),
+                             units_per_group(d), err, s);
+}
+
 cudaError_t launch_sel_bm(const Dims& d, const void* q, const void* k, const void* v,
                           const int32_t* idx, void* o_sel, float* lse_sel, int* err,
                           const EpilogueFuse* fz, void* ws, cudaStream_t s) {
+  const cudaError_t e = launch_sel_bm_prep(d, idx, err, ws, s);
+  if (e != cudaSuccess) return e;
+  return launch_sel_bm_run(d, q, k, v, idx, o_sel, lse_sel, err, fz, ws, s);
+}
+
+cudaError_t launch_sel_bm_run(const Dims& d, const void* q, const void* k, const void* v,
+                              const int32_t* idx, void* o_sel, float* lse_sel, int* err,
+                              const EpilogueFuse* fz, void* ws, cudaStream_t s) {
   const BmCarve c = bm_carve(d);
   char* w = (char*)ws;
   int* list = (int*)(w + c.list);
@@ -814,10 +832,7 @@ cudaError_t launch_sel_bm(const Dims& d, const void* q, const void* k, const voi
   __half* part_o = (__half*)(w + c.part_o);
   float* part_lse = (float*)(w + c.part_lse);
   const int umax = units_per_group(d);
-  cudaError_t e = launch_revmap_units(d, idx, (int*)(w + c.chunk), (int*)(w + c.offsets),
-                                      (int*)(w + c.cursor), list, units, ucount,
-                                      kSeg * tile_tokens(d.G), tile_tokens(d.G), umax, err, s);
-  if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
   CUtensorMap mk, mv;
   if (!make_tmap_bf16(&mk, k, d.Hkv, (long)d.B * d.T, 1, kKeys) ||
       !make_tmap_bf16(&mv, v, d.Hkv, (long)d.B * d.T, 1, kKeys))
