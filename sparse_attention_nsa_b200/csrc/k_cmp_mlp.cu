@@ -62,6 +62,20 @@ __device__ __forceinline__ void split8(const float* src, uint32_t h[4], uint32_t
   }
 }
 
+// dkc, dvc (fp32 [nq, 64]) -> bf16 pairs hi[2][nq][64], lo[2][nq][64] (keys, values), the
+// operands of the dW and dA GEMMs; 8 values a thread
+__global__ void cmp_mlp_split_kernel(const float* __restrict__ dkc, const float* __restrict__ dvc,
+                                     bf16* __restrict__ hi, bf16* __restrict__ lo, long n8) {
+  const long e = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= 2 * n8) return;
+  const int which = (int)(e / n8);
+  const long o = e - which * n8;
+  uint32_t h[4], l[4];
+  split8((which ? dvc : dkc) + o * 8, h, l);
+  reinterpret_cast<uint4*>(hi)[e] = make_uint4(h[0], h[1], h[2], h[3]);
+  reinterpret_cast<uint4*>(lo)[e] = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
 __device__ __forceinline__ void setup(MlpBars* bars, volatile int* abort_flag) {
   for (int s = 0; s < kMlpStages; ++s) {
     mbar_init(&bars->full[s], 128);
@@ -230,6 +244,7 @@ __global__ void cmp_mlp_fwd_reduce_kernel(const float* __restrict__ part, bf16* 
 // ---- dW: rows (i, e) of token offsets i = 2m, 2m + 1 against a range of blocks q --------
 // Stage: X [64 K rows q][two 64-wide atoms: offsets 2m, 2m + 1] read MN-major (the second
 // atom 8 KB after the first), dXc hi, lo [64 q][64 n] read MN-major.  D: TMEM [0, 64).
+// Every operand arrives by cp.async, two stages ahead of the MMAs.
 // CTA z of S takes the chunks u = z, z + S, ...; with S > 1 it writes its partial sum
 // to part[z] for a fixed-order reduction.
 constexpr uint32_t MW_STAGE = 4 * kW64;
@@ -238,7 +253,7 @@ constexpr uint32_t MW_SMEM = MW_OFF_BAR + kBarBytes + 16;
 
 __global__ void __launch_bounds__(kMlpThreads, 1)
 cmp_mlp_dw_kernel(const bf16* __restrict__ xk, const bf16* __restrict__ xv,
-                  const float* __restrict__ dkc, const float* __restrict__ dvc,
+                  const bf16* __restrict__ ghi, const bf16* __restrict__ glo,
                   float* __restrict__ dwk, float* __restrict__ dwv, float* __restrict__ part,
                   Dims d, int* err) {
   extern __shared__ uint8_t smem_raw[];
@@ -249,8 +264,9 @@ cmp_mlp_dw_kernel(const bf16* __restrict__ xk, const bf16* __restrict__ xv,
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
   const int m = blockIdx.x, which = blockIdx.y, z = blockIdx.z, S = gridDim.z;
   const bf16* x = which ? xv : xk;
-  const float* dxc = which ? dvc : dkc;
   const long nq = (long)d.B * d.Nc * d.Hkv;  // contraction length
+  const bf16* gh = ghi + which * nq * 64;
+  const bf16* gl = glo + which * nq * 64;
   const int nchunk = (int)((nq + 63) / 64);
   const int mine = nchunk > z ? (nchunk - z + S - 1) / S : 0;
   if (tid == 0) setup(bars, abort_flag);
@@ -261,15 +277,9 @@ cmp_mlp_dw_kernel(const bf16* __restrict__ xk, const bf16* __restrict__ xv,
 
   if (warp < 4) {
     bool ok = true;
-    for (int it = 0; it < mine; ++it) {
+    auto issue = [&](int it) {  // chunk it's operands into its stage, one cp.async group
       const int st = it % kMlpStages;
       const long u = z + (long)it * S;
-      if (it >= kMlpStages &&
-          !wait_bar_warp(&bars->empty[st], ((it - kMlpStages) / kMlpStages) & 1, abort_flag,
-                         err)) {
-        ok = false;
-        break;
-      }
       const uint32_t a0 = smem_u32(smem + st * MW_STAGE), a1 = a0 + kW64;
       const uint32_t bh = a1 + kW64, bl = bh + kW64;
       // X: 64 K rows x 2 atoms x 8 chunks = 1024 chunks, 8 per thread
@@ -289,21 +299,37 @@ cmp_mlp_dw_kernel(const bf16* __restrict__ xk, const bf16* __restrict__ xv,
         }
         cp_async16((atom ? a1 : a0) + swz_off(r, c), x + row * 64 + 8 * c, present ? 16u : 0u);
       }
-      cp_async_commit();
-      // dXc rows as bf16 hi + lo: 64 rows x 8 chunks, 4 per thread
+      // dXc hi, lo rows: 64 rows x 8 chunks each, 4 + 4 per thread
 #pragma unroll
       for (int t4 = 0; t4 < 4; ++t4) {
         const int idx = tid + 128 * t4, r = idx >> 3, c = idx & 7;
         const long q = u * 64 + r;
-        uint32_t h[4] = {0u, 0u, 0u, 0u}, lo[4] = {0u, 0u, 0u, 0u};
-        if (q < nq) split8(dxc + q * 64 + 8 * c, h, lo);
-        st_shared_v4(bh + swz_off(r, c), h[0], h[1], h[2], h[3]);
-        st_shared_v4(bl + swz_off(r, c), lo[0], lo[1], lo[2], lo[3]);
+        const bool present = q < nq;
+        const size_t off = (size_t)(present ? q : 0) * 64 + 8 * c;
+        cp_async16(bh + swz_off(r, c), gh + off, present ? 16u : 0u);
+        cp_async16(bl + swz_off(r, c), gl + off, present ? 16u : 0u);
       }
-      cp_async_wait<0>();
+      cp_async_commit();
+    };
+    // chunks 0 and 1 in flight before the loop; chunk it + 2 issued once chunk it landed
+    for (int it = 0; it < 2 && it < mine; ++it) issue(it);
+    for (int it = 0; it < mine; ++it) {
+      if (it + 1 < mine) cp_async_wait<1>();
+      else cp_async_wait<0>();
       fence_proxy_async_smem();
-      mbar_arrive(&bars->full[st]);
+      mbar_arrive(&bars->full[it % kMlpStages]);
+      const int nx = it + 2;
+      if (nx < mine) {
+        if (nx >= kMlpStages &&
+            !wait_bar_warp(&bars->empty[nx % kMlpStages], ((nx - kMlpStages) / kMlpStages) & 1,
+                           abort_flag, err)) {
+          ok = false;
+          break;
+        }
+        issue(nx);
+      }
     }
+    cp_async_wait<0>();  // no copy outlives the CTA
     // epilogue: thread r holds row (i, e) = (2m + r / 64, r % 64) of dW
     const bool have = ok && mine > 0 && wait_bar_warp(&bars->fin, 0, abort_flag, err);
     const int i = 2 * m + (tid >> 6), e = tid & 63;
@@ -373,7 +399,7 @@ constexpr uint32_t MA_OFF_BAR = MA_OFF_W + kMlpStages * kW64;
 constexpr uint32_t MA_SMEM = MA_OFF_BAR + kBarBytes + 16;
 
 __global__ void __launch_bounds__(kMlpThreads, 1)
-cmp_mlp_da_kernel(const float* __restrict__ dkc, const float* __restrict__ dvc,
+cmp_mlp_da_kernel(const bf16* __restrict__ ghi, const bf16* __restrict__ glo,
                   const bf16* __restrict__ wk, const bf16* __restrict__ wv,
                   float* __restrict__ dak, float* __restrict__ dav, Dims d, int* err) {
   extern __shared__ uint8_t smem_raw[];
@@ -383,10 +409,11 @@ cmp_mlp_da_kernel(const float* __restrict__ dkc, const float* __restrict__ dvc,
   volatile int* abort_flag = (volatile int*)(smem + MA_OFF_BAR + kBarBytes + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
   const int which = blockIdx.y;
-  const float* dxc = which ? dvc : dkc;
   const bf16* w = which ? wv : wk;
   float* da = which ? dav : dak;
   const long nq = (long)d.B * d.Nc * d.Hkv;
+  const bf16* gh = ghi + which * nq * 64;
+  const bf16* gl = glo + which * nq * 64;
   const long q = (long)blockIdx.x * 128 + tid;  // this thread's row (warps 0-3)
   const int Z = (int)gridDim.z, z = (int)blockIdx.z;
   const int u0 = (int)(((long)d.lc * z) / Z);
@@ -399,32 +426,39 @@ cmp_mlp_da_kernel(const float* __restrict__ dkc, const float* __restrict__ dvc,
 
   if (warp < 4) {
     const uint32_t ah = smem_u32(smem), al = ah + kRowTile;
+    // A (once, with W_0's group): row r = dXc[q] as the bf16 pair, 8 + 8 chunks per thread
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
-      uint32_t h[4] = {0u, 0u, 0u, 0u}, lo[4] = {0u, 0u, 0u, 0u};
-      if (q < nq) split8(dxc + q * 64 + 8 * c, h, lo);
-      st_shared_v4(ah + swz_off(tid, c), h[0], h[1], h[2], h[3]);
-      st_shared_v4(al + swz_off(tid, c), lo[0], lo[1], lo[2], lo[3]);
+      const bool present = q < nq;
+      const size_t off = (size_t)(present ? q : 0) * 64 + 8 * c;
+      cp_async16(ah + swz_off(tid, c), gh + off, present ? 16u : 0u);
+      cp_async16(al + swz_off(tid, c), gl + off, present ? 16u : 0u);
     }
-    // W_i stages by cp.async (the first arrival also publishes A); the epilogue of offset
-    // u - 1 follows the arrival for offset u
+    auto issue = [&](int u) {  // W of offset u into its stage, one cp.async group
+      const uint32_t wb = smem_u32(smem + MA_OFF_W + (u % kMlpStages) * kW64);
+#pragma unroll
+      for (int m4 = 0; m4 < 4; ++m4) {
+        const int idx = tid + 128 * m4, e = idx >> 3, c = idx & 7;
+        cp_async16(wb + swz_off(e, c), w + ((size_t)(u0 + u) * 64 + e) * 64 + 8 * c, 16u);
+      }
+      cp_async_commit();
+    };
+    for (int u = 0; u < 2 && u < L; ++u) issue(u);
+    // offset u's stage is published once it landed; the epilogue of offset u - 1 follows
     for (int u = 0; u <= L; ++u) {
       if (u < L) {
-        const int st = u % kMlpStages;
-        if (u >= kMlpStages &&
-            !wait_bar_warp(&bars->empty[st], ((u - kMlpStages) / kMlpStages) & 1, abort_flag,
-                           err))
-          break;
-        const uint32_t wb = smem_u32(smem + MA_OFF_W + st * kW64);
-#pragma unroll
-        for (int m4 = 0; m4 < 4; ++m4) {
-          const int idx = tid + 128 * m4, e = idx >> 3, c = idx & 7;
-          cp_async16(wb + swz_off(e, c), w + ((size_t)(u0 + u) * 64 + e) * 64 + 8 * c, 16u);
-        }
-        cp_async_commit();
-        cp_async_wait<0>();
+        if (u + 1 < L) cp_async_wait<1>();
+        else cp_async_wait<0>();
         fence_proxy_async_smem();
-        mbar_arrive(&bars->full[st]);
+        mbar_arrive(&bars->full[u % kMlpStages]);
+        const int nx = u + 2;
+        if (nx < L) {
+          if (nx >= kMlpStages &&
+              !wait_bar_warp(&bars->empty[nx % kMlpStages], ((nx - kMlpStages) / kMlpStages) & 1,
+                             abort_flag, err))
+            break;
+          issue(nx);
+        }
       }
       if (u >= 1) {
         const int pu = u - 1, bu = pu & 1;
@@ -442,6 +476,7 @@ cmp_mlp_da_kernel(const float* __restrict__ dkc, const float* __restrict__ dvc,
         }
       }
     }
+    cp_async_wait<0>();  // no copy outlives the CTA
   } else if (lane == 0) {
     constexpr uint32_t idesc = idesc_bf16(128, 64, false, false);  // A, B K-major
     const uint32_t ah = smem_u32(smem), al = ah + kRowTile;
@@ -473,27 +508,33 @@ cmp_mlp_da_kernel(const float* __restrict__ dkc, const float* __restrict__ dvc,
 }
 
 // dx[b, t, g, :] += sum over the blocks j covering t, ascending, of
-// dA[(b Nc + j) Hkv + g, t - j d, :]  (one thread per element)
+// dA[(b Nc + j) Hkv + g, t - j d, :]  (4 values a thread)
 __global__ void cmp_mlp_gather_kernel(const float* __restrict__ dak, const float* __restrict__ dav,
                                       float* __restrict__ dk, float* __restrict__ dv, Dims d) {
-  const long e = (long)blockIdx.x * blockDim.x + threadIdx.x;
-  const long row_elems = (long)d.Hkv * 64;
-  const long n = (long)d.B * d.T * row_elems;
-  if (e >= n) return;
-  const int c = (int)(e % 64), g = (int)((e / 64) % d.Hkv);
-  const long tok = e / row_elems;
+  const long e4 = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long n4 = (long)d.B * d.T * d.Hkv * 16;
+  if (e4 >= n4) return;
+  const int c4 = (int)(e4 & 15), g = (int)((e4 >> 4) % d.Hkv);
+  const long tok = (e4 >> 4) / d.Hkv;
   const int t = (int)(tok % d.T), b = (int)(tok / d.T);
   const int chi = min(t / d.dc, d.Nc - 1);
   const int clo = t < d.lc ? 0 : (t - d.lc) / d.dc + 1;
   if (clo > chi) return;
-  float sk = 0.f, sv = 0.f;
+  float4 sk = make_float4(0.f, 0.f, 0.f, 0.f), sv = sk;
   for (int j = clo; j <= chi; ++j) {
-    const size_t src = ((((size_t)b * d.Nc + j) * d.Hkv + g) * d.lc + (t - j * d.dc)) * 64 + c;
-    sk += dak[src];
-    sv += dav[src];
+    const size_t src = ((((size_t)b * d.Nc + j) * d.Hkv + g) * d.lc + (t - j * d.dc)) * 16 + c4;
+    const float4 a = reinterpret_cast<const float4*>(dak)[src];
+    const float4 v = reinterpret_cast<const float4*>(dav)[src];
+    sk.x += a.x; sk.y += a.y; sk.z += a.z; sk.w += a.w;
+    sv.x += v.x; sv.y += v.y; sv.z += v.z; sv.w += v.w;
   }
-  dk[e] += sk;
-  dv[e] += sv;
+  float4* pk = reinterpret_cast<float4*>(dk) + e4;
+  float4* pv = reinterpret_cast<float4*>(dv) + e4;
+  float4 ok = *pk, ov = *pv;
+  ok.x += sk.x; ok.y += sk.y; ok.z += sk.z; ok.w += sk.w;
+  ov.x += sv.x; ov.y += sv.y; ov.z += sv.z; ov.w += sv.w;
+  *pk = ok;
+  *pv = ov;
 }
 
 // CTAs per output tile when the tiles alone would leave SMs idle (at most one per offset)
@@ -527,12 +568,25 @@ size_t cmp_mlp_fwd_ws_bytes(const Dims& d) {
   return S > 1 ? (size_t)S * 2 * d.B * d.Nc * d.Hkv * 64 * sizeof(float) : 0;
 }
 
-size_t cmp_mlp_bwd_ws_bytes(const Dims& d) {
-  const size_t da = 2 * (size_t)d.B * d.Nc * d.Hkv * d.lc * 64 * sizeof(float);
+// backward workspace: dA scratch [2][nq][l][64] fp32, the dW partial sums, the
+// upstream gradient's bf16 pairs hi, lo [2][nq][64] each (each part 256-byte aligned)
+struct BwdWs {
+  size_t da, part, hi, lo, total;
+};
+BwdWs bwd_ws(const Dims& d) {
+  const size_t nq = (size_t)d.B * d.Nc * d.Hkv;
+  auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  BwdWs w{};
+  w.da = 0;
+  w.part = al(2 * nq * d.lc * 64 * sizeof(float));
   const int S = dw_splits(d);
-  const size_t part = S > 1 ? (size_t)S * 2 * d.lc * 64 * 64 * sizeof(float) : 0;
-  return ((da + 255) & ~(size_t)255) + part;
+  w.hi = w.part + al(S > 1 ? (size_t)S * 2 * d.lc * 64 * 64 * sizeof(float) : 0);
+  w.lo = w.hi + al(2 * nq * 64 * sizeof(bf16));
+  w.total = w.lo + al(2 * nq * 64 * sizeof(bf16));
+  return w;
 }
+
+size_t cmp_mlp_bwd_ws_bytes(const Dims& d) { return bwd_ws(d).total; }
 
 cudaError_t launch_cmp_mlp_fwd(const Dims& d, const void* k, const void* v, const void* wk,
                                const void* wv, void* kc, void* vc, void* ws, int* err,
@@ -571,13 +625,19 @@ cudaError_t launch_cmp_mlp_bwd(const Dims& d, const void* k, const void* v, cons
   e = cudaFuncSetAttribute(cmp_mlp_da_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, sma);
   if (e != cudaSuccess) return e;
   const long nq = (long)d.B * d.Nc * d.Hkv;
-  float* dak = (float*)ws;
+  const BwdWs L = bwd_ws(d);
+  float* dak = (float*)((char*)ws + L.da);
   float* dav = dak + (size_t)nq * d.lc * 64;
-  const size_t da_bytes = 2 * (size_t)nq * d.lc * 64 * sizeof(float);
-  float* part = (float*)((char*)ws + ((da_bytes + 255) & ~(size_t)255));
+  float* part = (float*)((char*)ws + L.part);
+  bf16* ghi = (bf16*)((char*)ws + L.hi);
+  bf16* glo = (bf16*)((char*)ws + L.lo);
+  const long n8 = nq * 8;
+  cmp_mlp_split_kernel<<<(unsigned)((2 * n8 + 255) / 256), 256, 0, s>>>(dkc, dvc, ghi, glo, n8);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
   const int S = dw_splits(d);
   cmp_mlp_dw_kernel<<<dim3((d.lc + 1) / 2, 2, S), kMlpThreads, smw, s>>>(
-      (const bf16*)k, (const bf16*)v, dkc, dvc, dwk, dwv, part, d, err);
+      (const bf16*)k, (const bf16*)v, ghi, glo, dwk, dwv, part, d, err);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (S > 1) {
@@ -588,11 +648,11 @@ cudaError_t launch_cmp_mlp_bwd(const Dims& d, const void* k, const void* v, cons
     if (e != cudaSuccess) return e;
   }
   cmp_mlp_da_kernel<<<dim3((unsigned)((nq + 127) / 128), 2, da_splits(d)), kMlpThreads, sma, s>>>(
-      dkc, dvc, (const bf16*)wk, (const bf16*)wv, dak, dav, d, err);
+      ghi, glo, (const bf16*)wk, (const bf16*)wv, dak, dav, d, err);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const long n = (long)d.B * d.T * d.Hkv * 64;
-  cmp_mlp_gather_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(dak, dav, dk, dv, d);
+  const long n4 = (long)d.B * d.T * d.Hkv * 16;
+  cmp_mlp_gather_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, s>>>(dak, dav, dk, dv, d);
   return cudaGetLastError();
 }
 
