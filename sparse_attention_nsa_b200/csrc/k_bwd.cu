@@ -25,30 +25,68 @@ enum BwdMode { kBwdSel = 0, kBwdSwa = 1, kBwdCmp = 2 };
 
 // ---- gated combination ---------------------------------------------------------
 // dgates[r, i] = dout_r . o_i,r (enabled branches, else 0); dO_i = gate_i dout.
+// 8 consecutive values of a row as fp32 (one 16-byte load for bf16, two for fp32)
+__device__ __forceinline__ void load8(const bf16* p, float* x) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 f = __bfloat1622float2(h[e]);
+    x[2 * e] = f.x;
+    x[2 * e + 1] = f.y;
+  }
+}
+__device__ __forceinline__ void load8(const float* p, float* x) {
+  const float4 a = *reinterpret_cast<const float4*>(p);
+  const float4 c = *reinterpret_cast<const float4*>(p + 4);
+  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+  x[4] = c.x; x[5] = c.y; x[6] = c.z; x[7] = c.w;
+}
+
+// Eight threads per row, eight values each: every load of the row (dout and
+// the enabled branches' outputs) is issued before any is used, the three dot
+// products are reduced over the row's eight lanes.
 template <typename T>
-__global__ void gate_bwd_kernel(const float* __restrict__ gates, const T* __restrict__ dout,
-                                const T* __restrict__ oc, const T* __restrict__ os,
-                                const T* __restrict__ ow, float* __restrict__ dgates,
-                                float* __restrict__ dOc, float* __restrict__ dOs,
-                                float* __restrict__ dOw, long nrows, int mask) {
-  const long warp = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (warp >= nrows) return;
-  const size_t base = (size_t)warp * 64;
-  const float g0 = to_f32(dout[base + lane]), g1 = to_f32(dout[base + lane + 32]);
+__global__ void __launch_bounds__(256)
+gate_bwd_kernel(const float* __restrict__ gates, const T* __restrict__ dout,
+                const T* __restrict__ oc, const T* __restrict__ os, const T* __restrict__ ow,
+                float* __restrict__ dgates, float* __restrict__ dOc, float* __restrict__ dOs,
+                float* __restrict__ dOw, long nrows, int mask) {
+  const long t = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long row0 = t >> 3;
+  const int sub = (int)(t & 7);
+  const bool live = row0 < nrows;  // every lane stays for the shuffles
+  const long row = live ? row0 : nrows - 1;
+  const size_t base = (size_t)row * 64 + 8 * sub;
   const T* br[3] = {oc, os, ow};
   float* dst[3] = {dOc, dOs, dOw};
+  float g[8], x[3][8];
+  load8(dout + base, g);
 #pragma unroll
   for (int i = 0; i < 3; ++i) {
-    const bool on = (mask >> i) & 1;
+    if ((mask >> i) & 1) load8(br[i] + base, x[i]);
+    else
+#pragma unroll
+      for (int e = 0; e < 8; ++e) x[i][e] = 0.f;
+  }
+  float gi[3];
+#pragma unroll
+  for (int i = 0; i < 3; ++i) gi[i] = ((mask >> i) & 1) ? gates[row * 3 + i] : 0.f;
+#pragma unroll
+  for (int i = 0; i < 3; ++i) {
     float dg = 0.f;
-    if (on) dg = warp_sum(g0 * to_f32(br[i][base + lane]) + g1 * to_f32(br[i][base + lane + 32]));
-    const float gi = on ? gates[warp * 3 + i] : 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) dg = fmaf(g[e], x[i][e], dg);
+    dg += __shfl_xor_sync(0xffffffffu, dg, 1);
+    dg += __shfl_xor_sync(0xffffffffu, dg, 2);
+    dg += __shfl_xor_sync(0xffffffffu, dg, 4);
+    if (!live) continue;
     if (dst[i]) {
-      dst[i][base + lane] = gi * g0;
-      dst[i][base + lane + 32] = gi * g1;
+      float4* o = reinterpret_cast<float4*>(dst[i] + base);
+      o[0] = make_float4(gi[i] * g[0], gi[i] * g[1], gi[i] * g[2], gi[i] * g[3]);
+      o[1] = make_float4(gi[i] * g[4], gi[i] * g[5], gi[i] * g[6], gi[i] * g[7]);
     }
-    if (lane == 0) dgates[warp * 3 + i] = dg;
+    if (sub == 0) dgates[row * 3 + i] = ((mask >> i) & 1) ? dg : 0.f;
   }
 }
 
@@ -606,27 +644,34 @@ dkdv_kernel(const T* __restrict__ q, const T* __restrict__ keys, const T* __rest
 // same for dv; tokens that no complete block covers get nothing.
 __global__ void pool_bwd_kernel(const float* __restrict__ dkc, const float* __restrict__ dvc,
                                 float* __restrict__ dk, float* __restrict__ dv, Dims d) {
-  const long e = (long)blockIdx.x * blockDim.x + threadIdx.x;
-  const long row_elems = (long)d.Hkv * 64;
-  const long n = (long)d.B * d.T * row_elems;
-  if (e >= n) return;
-  const long c = e % row_elems;
-  const long tok = e / row_elems;  // b * T + t
+  // four consecutive values a thread (16-byte loads and stores)
+  const long e4 = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long row4 = (long)d.Hkv * 16;
+  const long n4 = (long)d.B * d.T * row4;
+  if (e4 >= n4) return;
+  const long c4 = e4 % row4;
+  const long tok = e4 / row4;  // b * T + t
   const int t = (int)(tok % d.T);
   const int b = (int)(tok / d.T);
   const int chi = min(t / d.dc, d.Nc - 1);                       // last block starting <= t
   const int clo = t < d.lc ? 0 : (t - d.lc) / d.dc + 1;          // first block ending after t
   if (clo > chi) return;
-  float sk = 0.f, sv = 0.f;
+  float4 sk = make_float4(0.f, 0.f, 0.f, 0.f), sv = sk;
   for (int jc = clo; jc <= chi; ++jc) {
-    const size_t src = ((size_t)b * d.Nc + jc) * row_elems + c;
-    sk += dkc[src];
-    sv += dvc[src];
+    const size_t src = ((size_t)b * d.Nc + jc) * row4 + c4;
+    const float4 a = reinterpret_cast<const float4*>(dkc)[src];
+    const float4 v = reinterpret_cast<const float4*>(dvc)[src];
+    sk.x += a.x; sk.y += a.y; sk.z += a.z; sk.w += a.w;
+    sv.x += v.x; sv.y += v.y; sv.z += v.z; sv.w += v.w;
   }
   const float inv = 1.f / (float)d.lc;
-  const size_t dst = ((size_t)b * d.T + t) * row_elems + c;
-  dk[dst] += sk * inv;
-  dv[dst] += sv * inv;
+  float4* pk = reinterpret_cast<float4*>(dk) + e4;
+  float4* pv = reinterpret_cast<float4*>(dv) + e4;
+  float4 ok = *pk, ov = *pv;
+  ok.x += sk.x * inv; ok.y += sk.y * inv; ok.z += sk.z * inv; ok.w += sk.w * inv;
+  ov.x += sv.x * inv; ov.y += sv.y * inv; ov.z += sv.z * inv; ov.w += sv.w * inv;
+  *pk = ok;
+  *pv = ov;
 }
 
 // ---- launchers ----------------------------------------------------------------------
@@ -634,7 +679,7 @@ cudaError_t launch_gate_bwd(const Dims& d, const float* gates, const void* dout,
                             const void* o_cmp, const void* o_sel, const void* o_swa,
                             float* dgates, float* dOc, float* dOs, float* dOw, cudaStream_t s) {
   const long nrows = (long)d.B * d.Tq * d.Hq;
-  const unsigned blocks = (unsigned)((nrows * 32 + 255) / 256);
+  const unsigned blocks = (unsigned)((nrows * 8 + 255) / 256);
   if (d.dtype == 1)
     gate_bwd_kernel<bf16><<<blocks, 256, 0, s>>>(gates, (const bf16*)dout, (const bf16*)o_cmp,
                                                  (const bf16*)o_sel, (const bf16*)o_swa, dgates,
@@ -739,9 +784,9 @@ cudaError_t launch_dkdv(const Dims& d, int mode, const void* q, const void* keys
 
 cudaError_t launch_pool_bwd(const Dims& d, const float* dkc, const float* dvc, float* dk,
                             float* dv, cudaStream_t s) {
-  const long n = d.Nc == 0 ? 0 : (long)d.B * d.T * d.Hkv * 64;
-  if (n == 0) return cudaSuccess;
-  pool_bwd_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(dkc, dvc, dk, dv, d);
+  const long n4 = d.Nc == 0 ? 0 : (long)d.B * d.T * d.Hkv * 16;
+  if (n4 == 0) return cudaSuccess;
+  pool_bwd_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, s>>>(dkc, dvc, dk, dv, d);
   return cudaGetLastError();
 }
 

@@ -124,14 +124,6 @@ __device__ __forceinline__ void pv_tile(float o[8][4], const float p[8][4], uint
   }
 }
 
-// Programmatic dependent launch: the next kernel in the stream may start its
-// prologue early; it waits for this grid's completion (and memory) with
-// griddepcontrol.wait before touching this grid's outputs.
-__device__ __forceinline__ void pdl_launch_dependents() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-
 __device__ __forceinline__ float quad_max(float x) {
   x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 1));
   return fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 2));

@@ -650,13 +650,20 @@ sel_merge_kernel(const int32_t* __restrict__ idx, const __half* __restrict__ par
   const int cur = (d.q_off + tq) / d.l;
   const int32_t* ir = idx + (bt * d.Hkv + h / d.G) * d.topk;
   const float* ls = part_lse + row * d.topk;
+  // the slots' lse values are read with their indices, not after them (an
+  // unused slot's value is read but dropped), so the partial loads below
+  // wait for one memory latency instead of two
   float wk[kMergeSlots];
+#pragma unroll
+  for (int k = 0; k < kMergeSlots; ++k) {
+    const int s = sub + 8 * k;
+    wk[k] = s < d.topk ? ls[s] : -INFINITY;
+  }
   float m = -INFINITY;
 #pragma unroll
   for (int k = 0; k < kMergeSlots; ++k) {
     const int s = sub + 8 * k;
-    wk[k] = -INFINITY;
-    if (s < d.topk && slot_used(ir, s, cur)) wk[k] = ls[s];
+    if (!(s < d.topk && slot_used(ir, s, cur))) wk[k] = -INFINITY;
     m = fmaxf(m, wk[k]);
   }
   m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
