@@ -428,6 +428,8 @@ def run_gpu(args, rank: int, world: int, dist_on: bool) -> None:
     moba = run_moba(dev, flush, stream, max(3, args.steps // 2), peaks)
     # NSA on its parametric compressor (blocks of 32 every 16 tokens)
     mlp = run_mlp(dev, flush, stream, max(3, args.steps // 2), peaks)
+    # the pages' branch pruning: sel + window, cmp + window, window alone
+    pruned = run_pruned(dev, flush, stream, max(3, args.steps // 2), peaks)
     # selection backward, two-pass against single-pass atomic
     selbwd = run_sel_bwd_compare(dev, flush, stream, 3, peaks)
     sampler.__exit__(None, None, None)
@@ -479,6 +481,7 @@ def run_gpu(args, rank: int, world: int, dist_on: bool) -> None:
         "nsa_1p3b": onep3b,
         "moba": moba,
         "mlp_compression": mlp,
+        "pruned_branches": pruned,
         "sel_bwd_two_pass_vs_atomic": selbwd,
         "e2e": {"value": job_tokens_per_s(tokens_per_step, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
@@ -699,6 +702,36 @@ def run_mlp(dev, flush, stream, steps, peaks) -> dict:
     return res
 
 
+def run_pruned(dev, flush, stream, steps, peaks) -> dict:
+    """The pages' branch pruning at the 340M shape (B=1, T=8192, GQA-4): the
+    same forward with every branch, with selection + window (compression
+    gate 0), and with the window alone, as later layers run once their
+    unused branches are pruned; speedups are against the full forward."""
+    res = {}
+    for name, mask in (("all", W.BR_ALL), ("sel_swa", W.BR_SEL | W.BR_SWA),
+                       ("cmp_swa", W.BR_CMP | W.BR_SWA), ("swa", W.BR_SWA)):
+        w = W.NSA_340M.replace(name=f"nsa_340m_gqa4_t8192_{name}_bf16", branch_mask=mask,
+                               cmp_gate_zero=not (mask & W.BR_CMP))
+        inp = W.make_inputs(w, seed=9)
+        q, k, v, g = (inp[n].to(dev) for n in ("q", "k", "v", "gates"))
+        p = nsa.params_for(w)
+        out = torch.empty_like(q)
+        ws = nsa.alloc_workspace(p, dev)
+
+        def fwd():
+            nsa.nsa_forward(p, q, k, v, g, out, None, ws)
+
+        for _ in range(3):
+            fwd()
+        ms = statistics.mean(timed_steps(fwd, steps, flush, stream))
+        res[name] = {"fwd_ms": ms, "tokens_per_s": w.B * w.T / (ms * 1e-3)}
+    if nsa.nsa_last_device_error() != 0:
+        raise RuntimeError("device-side check failed in the pruned-branch leg")
+    for name in res:
+        res[name]["speedup_vs_all"] = res["all"]["fwd_ms"] / res[name]["fwd_ms"]
+    return res
+
+
 def run_long(dev, flush, stream, steps, peaks) -> dict:
     """Long-context forward: the pruned MQA workload (B=1, 32768 tokens,
     selection + window).  Its selection runs block-major (Nb = 32 top-k);
@@ -790,8 +823,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--leg", default="all",
                     choices=["all", "forward", "decode", "train", "long", "onep3b", "moba",
-                             "selbwd", "mlp"],
-                    help="forward / decode / train / long / onep3b / moba / selbwd / mlp: run only that leg on one GPU "
+                             "selbwd", "mlp", "pruned"],
+                    help="forward / decode / train / long / onep3b / moba / selbwd / mlp / pruned: run only that leg on one GPU "
                          "and print its numbers (for profiling that leg alone); all: the "
                          "benchmark")
     ap.add_argument("--batch", type=int, default=None,
@@ -822,6 +855,8 @@ def main():
             print(json.dumps({"moba": run_moba(dev, flush, stream, args.steps, peaks)}))
         elif args.leg == "mlp":
             print(json.dumps({"mlp_compression": run_mlp(dev, flush, stream, args.steps, peaks)}))
+        elif args.leg == "pruned":
+            print(json.dumps({"pruned_branches": run_pruned(dev, flush, stream, args.steps, peaks)}))
         elif args.leg == "onep3b":
             print(json.dumps({"nsa_1p3b": run_1p3b(dev, flush, stream, args.steps, peaks)}))
         else:
