@@ -52,8 +52,13 @@ cudaError_t launch_compress(const Dims& d, const void* k, const void* v,
 cudaError_t launch_cmp_scores(const Dims& d, const void* q, const void* kc,
                               const void* vc, void* o_cmp, float* lse_cmp,
                               float* score, int* err, cudaStream_t s);
-cudaError_t launch_topk(const Dims& d, const float* score, int32_t* idx,
-                        cudaStream_t s);
+// Queries per chunk of the reverse map (its count, scan and fill passes).
+constexpr int kRevChunkQueries = 256;
+// rev_counts (optional, revmap_chunk_ints(d) ints): also produce the block-major
+// reverse map's per-(chunk, block) counts, so its own count pass is skipped
+// (launch_sel_bm_prep with counted = true).
+cudaError_t launch_topk(const Dims& d, const float* score, int32_t* idx, cudaStream_t s,
+                        int* rev_counts = nullptr);
 cudaError_t launch_sel_fwd(const Dims& d, const void* q, const void* k,
                            const void* v, const int32_t* idx, void* o,
                            float* lse, int* err, cudaStream_t s);
@@ -98,7 +103,9 @@ cudaError_t launch_sel_bm(const Dims& d, const void* q, const void* k, const voi
 // block-major kernel and the merge (run), so that other work can be ordered
 // between them
 cudaError_t launch_sel_bm_prep(const Dims& d, const int32_t* idx, int* err, void* ws,
-                               cudaStream_t s);
+                               cudaStream_t s, bool counted = false);
+// where launch_sel_bm_prep expects the counts of a counted top-k
+int* sel_bm_rev_counts(const Dims& d, void* ws);
 cudaError_t launch_sel_bm_run(const Dims& d, const void* q, const void* k, const void* v,
                               const int32_t* idx, void* o_sel, float* lse_sel, int* err,
                               const EpilogueFuse* fz, void* ws, cudaStream_t s);
@@ -140,9 +147,11 @@ cudaError_t launch_revmap(const Dims& d, const int32_t* idx, int* chunk, int* of
 // tiles of tq entries), written sorted by size (units of k tiles first, then
 // tails of k - 1, ..., 1 tiles, each class in block order); ucount holds the
 // four class sizes of each (sequence, group) as an int4.
+// counted: chunk already holds the per-(chunk, block) counts (a counted
+// launch_topk), so the count pass is skipped.
 cudaError_t launch_revmap_units(const Dims& d, const int32_t* idx, int* chunk, int* offsets,
                                 int* cursor, int* list, int4* units, int* ucount, int tpu, int tq,
-                                int umax, int* err, cudaStream_t s);
+                                int umax, int* err, cudaStream_t s, bool counted = false);
 // dO16: scratch of 2*B*Tq*Hq*64 16-bit values (the tensor-core path splits
 // dO into an fp16 pair hi, lo there)
 cudaError_t launch_dkdv(const Dims& d, int mode, const void* q, const void* keys,

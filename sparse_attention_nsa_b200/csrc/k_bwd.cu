@@ -221,7 +221,7 @@ dq_kernel(const T* __restrict__ q, const T* __restrict__ keys, const T* __restri
 // selection at its block's running position plus its rank among the lanes
 // that chose the same block.  A selection counts when it is a real,
 // causal block that does not repeat or go back (the forward's rule).
-constexpr int kRevChunk = 256;
+constexpr int kRevChunk = kRevChunkQueries;
 constexpr int kMaxUnitClasses = 4;  // work-unit sizes of 1 .. 4 tiles
 
 __device__ __forceinline__ bool rev_valid(const int32_t* ir, int s, int cur) {
@@ -735,7 +735,7 @@ cudaError_t launch_revmap(const Dims& d, const int32_t* idx, int* chunk, int* of
 
 cudaError_t launch_revmap_units(const Dims& d, const int32_t* idx, int* chunk, int* offsets,
                                 int* cursor, int* list, int4* units, int* ucount, int tpu, int tq,
-                                int umax, int* err, cudaStream_t s) {
+                                int umax, int* err, cudaStream_t s, bool counted) {
   if (tq < 1 || (tq & (tq - 1)) || (tpu & (tpu - 1)) || tpu < tq || tpu / tq > kMaxUnitClasses)
     return cudaErrorInvalidValue;  // powers of two, at most four tiles a unit
   const int nchunk = (d.Tq + kRevChunk - 1) / kRevChunk;
@@ -743,8 +743,9 @@ cudaError_t launch_revmap_units(const Dims& d, const int32_t* idx, int* chunk, i
   const size_t nb_bytes = (size_t)d.Nb * sizeof(int);
   // per-(chunk, block) counts -> each chunk's first position per block, the
   // offsets and the work units -> the entries in ascending query order
-  rev_chunk_count_kernel<<<dim3(nchunk, d.Hkv, d.B), kRevChunk, nb_bytes, s>>>(idx, chunk, d,
-                                                                              err, nullptr);
+  if (!counted)
+    rev_chunk_count_kernel<<<dim3(nchunk, d.Hkv, d.B), kRevChunk, nb_bytes, s>>>(idx, chunk, d,
+                                                                                err, nullptr);
   rev_chunk_scan_kernel<<<d.B * d.Hkv, 1024, (kMaxUnitClasses + 1) * nb_bytes + sizeof(int), s>>>(
       chunk, offsets, d, nchunk, units, ucount, cursor, tpu, tq, umax);
   cudaError_t e = cudaGetLastError();

@@ -811,13 +811,17 @@ bool sel_bm_eligible(const Dims& d) {
 size_t sel_bm_ws_bytes(const Dims& d) { return bm_carve(d).total; }
 
 cudaError_t launch_sel_bm_prep(const Dims& d, const int32_t* idx, int* err, void* ws,
-                               cudaStream_t s) {
+                               cudaStream_t s, bool counted) {
   const BmCarve c = bm_carve(d);
   char* w = (char*)ws;
   return launch_revmap_units(d, idx, (int*)(w + c.chunk), (int*)(w + c.offsets),
                              (int*)(w + c.cursor), (int*)(w + c.list), (int4*)(w + c.units),
                              (int*)(w + c.ucount), kSeg * tile_tokens(d.G), tile_tokens(d.G),
-                             units_per_group(d), err, s);
+                             units_per_group(d), err, s, counted);
+}
+
+int* sel_bm_rev_counts(const Dims& d, void* ws) {
+  return (int*)((char*)ws + bm_carve(d).chunk);
 }
 
 cudaError_t launch_sel_bm(const Dims& d, const void* q, const void* k, const void* v,

@@ -384,9 +384,12 @@ static nsa_status run_forward(const Dims& d, const void* q, const void* k, const
       if (em == cudaSuccess)
         em = nsa::launch_cmp_scores(d, q, kc, vc, cmp ? o_cmp : nullptr, cmp ? lse_cmp : nullptr,
                                     score, err_word(), ss->s2);
-      if (em == cudaSuccess) em = nsa::launch_topk(d, score, idx, ss->s2);
+      // with the block-major kernel, the top-k also counts the reverse map's
+      // entries (the map then has no count pass of its own)
+      int* rc = bm ? nsa::sel_bm_rev_counts(d, w + c.off[W_SELBM]) : nullptr;
+      if (em == cudaSuccess) em = nsa::launch_topk(d, score, idx, ss->s2, rc);
       if (em == cudaSuccess && bm)
-        em = nsa::launch_sel_bm_prep(d, idx, err_word(), w + c.off[W_SELBM], ss->s2);
+        em = nsa::launch_sel_bm_prep(d, idx, err_word(), w + c.off[W_SELBM], ss->s2, true);
       // the join is enqueued whatever happens, so no side-stream work can
       // outlive this call's ordering on the caller's stream
       const cudaError_t ej = cudaEventRecord(ss->join, ss->s2);
