@@ -240,7 +240,13 @@ nsa_status nsa_gate_combine(const nsa_params* p, const float* gates,
  * Attention Work? (three key/value sets per query, three attention outputs
  * merged by gates); "Sparsity is Cool", Method (mean-pool compression,
  * block 64, top-k 16, window 512) and Key claims (later layers pruned to
- * fewer branches at inference: the branch mask). */
+ * fewer branches at inference: the branch mask).
+ * With selection and window both enabled, the steps up to the reverse map
+ * run on a library-owned stream of the current device (highest stream
+ * priority, created on first use) while the window runs on `stream`; the
+ * call forks from and joins back into `stream` with events, so to the
+ * caller everything is ordered on `stream` as usual (graph capture
+ * included).  Concurrent calls serialise their enqueueing on a lock. */
 nsa_status nsa_forward(const nsa_params* p, const void* q, const void* k,
                        const void* v, const float* gates, void* out,
                        const nsa_saved* saved, void* workspace,

@@ -650,9 +650,14 @@ sel_merge_kernel(const int32_t* __restrict__ idx, const __half* __restrict__ par
   const int cur = (d.q_off + tq) / d.l;
   const int32_t* ir = idx + (bt * d.Hkv + h / d.G) * d.topk;
   const float* ls = part_lse + row * d.topk;
-  // the slots' lse values are read with their indices, not after them (an
-  // unused slot's value is read but dropped), so the partial loads below
-  // wait for one memory latency instead of two
+  // the first 8 slots' partials and the slots' lse values are read with the
+  // indices, not after them (an unused slot's bytes are read but dropped: its
+  // weight is 0), so a row's loads wait for one memory latency, not three
+  const uint4* po = reinterpret_cast<const uint4*>(part_o + row * d.topk * 64) + sub;
+  uint4 u0[8];
+#pragma unroll
+  for (int q2 = 0; q2 < 8; ++q2)
+    if (q2 < d.topk) u0[q2] = po[q2 * 8];
   float wk[kMergeSlots];
 #pragma unroll
   for (int k = 0; k < kMergeSlots; ++k) {
@@ -679,14 +684,13 @@ sel_merge_kernel(const int32_t* __restrict__ idx, const __half* __restrict__ par
   L += __shfl_xor_sync(0xffffffffu, L, 2);
   L += __shfl_xor_sync(0xffffffffu, L, 4);
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  const uint4* po = reinterpret_cast<const uint4*>(part_o + row * d.topk * 64) + sub;
 #pragma unroll
   for (int k = 0; k < kMergeSlots; ++k) {
     if (8 * k >= d.topk) break;
     uint4 u[8];
 #pragma unroll
     for (int q2 = 0; q2 < 8; ++q2)
-      if (8 * k + q2 < d.topk) u[q2] = po[(8 * k + q2) * 8];
+      if (8 * k + q2 < d.topk) u[q2] = k == 0 ? u0[q2] : po[(8 * k + q2) * 8];
 #pragma unroll
     for (int q2 = 0; q2 < 8; ++q2) {
       if (8 * k + q2 >= d.topk) break;
