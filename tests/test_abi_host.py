@@ -135,3 +135,37 @@ def test_forward_host_workspace_and_argument_checks():
     bad = nsa.make_params(2, 1000, 16, 4, scale=-1.0)
     assert lib.nsa_forward_host(C.byref(bad), host, host, host, host, host, host, need,
                                 None) == 1
+
+
+def test_parametric_compression_checks_before_launch():
+    """The parametric compressor runs bf16 only (NSA_ERR_UNSUPPORTED for
+    fp32), rejects NULL or misaligned pointers, a missing workspace and a
+    missing saved-tensor block before anything is enqueued, and sizes its
+    workspaces as the mean-pool path's plus its own."""
+    lib = nsa.load()
+    ptr = C.c_void_p(4096)  # aligned, never dereferenced: the checks come first
+    f32 = nsa.make_params(1, 1000, 16, 4, cmp_block=32, cmp_stride=16, dtype=nsa.NSA_F32)
+    assert lib.nsa_compress_mlp(C.byref(f32), *([ptr] * 6), ptr, 1 << 30, None) == 2
+    assert lib.nsa_forward_mlp(C.byref(f32), *([ptr] * 7), None, ptr, 1 << 30, None) == 2
+    p = nsa.make_params(1, 1000, 16, 4, cmp_block=32, cmp_stride=16)
+    assert lib.nsa_compress_mlp(C.byref(p), None, ptr, ptr, ptr, ptr, ptr, ptr, 1 << 30,
+                                None) == 1
+    assert lib.nsa_compress_mlp(C.byref(p), ptr, ptr, C.c_void_p(4100), ptr, ptr, ptr, ptr,
+                                1 << 30, None) == 1  # misaligned wk
+    fws = nsa.nsa_compress_mlp_workspace_size(p)
+    assert fws > 0  # 61 blocks x 4 groups: the token offsets are split over CTAs
+    assert lib.nsa_compress_mlp(C.byref(p), *([ptr] * 6), None, 0, None) == 6
+    assert lib.nsa_compress_mlp(C.byref(p), *([ptr] * 6), ptr, fws - 1, None) == 6
+    assert nsa.nsa_forward_mlp_workspace_size(p) >= nsa.nsa_workspace_size(p) + fws
+    bws = nsa.nsa_compress_mlp_bwd_workspace_size(p)
+    nq = 1 * p.Nc * 4
+    assert bws >= 2 * nq * 32 * 64 * 4  # the per-block row gradients, fp32
+    assert nsa.nsa_backward_mlp_workspace_size(p) == nsa.nsa_backward_workspace_size(p) + bws
+    args = [ptr] * 4 + [ptr] * 6
+    assert lib.nsa_compress_mlp_bwd(C.byref(p), *args, None, 0, None) == 6
+    # nsa_backward_mlp: q k v wk wv gates dout saved dq dk dv dwk dwv dgates
+    assert lib.nsa_backward_mlp(C.byref(p), *([ptr] * 7), None, *([ptr] * 6), ptr,
+                                1 << 30, None) == 1  # no saved tensors
+    # enough output tiles: one CTA per tile, no partial sums
+    wide = nsa.make_params(1, 2400, 64, 64, cmp_block=32, cmp_stride=16, window=64)
+    assert nsa.nsa_compress_mlp_workspace_size(wide) == 0
