@@ -114,9 +114,13 @@ cudaError_t launch_combine(const Dims& d, const float* gates, const void* o_cmp,
                            cudaStream_t s);
 
 // ---- backward (k_bwd.cu); mode 0 selection, 1 window, 2 compression ----
+// h16[i] (optional): also write branch i's dO as the fp16 pair the tensor-core
+// dK/dV kernel takes (hi at h16[i], lo nel halves after it, nel = B Tq Hq 64),
+// so that kernel can skip its own split (launch_dkdv with dO16_ready)
 cudaError_t launch_gate_bwd(const Dims& d, const float* gates, const void* dout,
                             const void* o_cmp, const void* o_sel, const void* o_swa,
-                            float* dgates, float* dOc, float* dOs, float* dOw, cudaStream_t s);
+                            float* dgates, float* dOc, float* dOs, float* dOw, cudaStream_t s,
+                            void* const* h16 = nullptr, int* err = nullptr);
 cudaError_t launch_dq(const Dims& d, int mode, const void* q, const void* keys,
                       const void* vals, const int32_t* idx, const void* o, const float* lse,
                       const float* dO, float* dq, float* delta, int* err, cudaStream_t s);
@@ -154,17 +158,20 @@ cudaError_t launch_revmap_units(const Dims& d, const int32_t* idx, int* chunk, i
                                 int umax, int* err, cudaStream_t s, bool counted = false);
 // dO16: scratch of 2*B*Tq*Hq*64 16-bit values (the tensor-core path splits
 // dO into an fp16 pair hi, lo there)
+// dO16_ready: dO16 already holds dO's fp16 pair (written by launch_gate_bwd)
 cudaError_t launch_dkdv(const Dims& d, int mode, const void* q, const void* keys,
                         const void* vals, const float* lse, const float* delta,
                         const float* dO, void* dO16, const int* offsets, const int* list,
-                        float* dk, float* dv, float* part, int* err, cudaStream_t s);
+                        float* dk, float* dv, float* part, int* err, cudaStream_t s,
+                        bool dO16_ready = false);
 bool dkdv_tc_eligible(const Dims& d, int mode);
 // workspace of the compression branch's row shares (tensor-core dK/dV)
 size_t dkdv_cmp_part_bytes(const Dims& d);
 cudaError_t launch_dkdv_tc(const Dims& d, int mode, const void* q, const void* keys,
                            const void* vals, const float* lse, const float* delta,
                            const float* dO, void* dO16, const int* offsets, const int* list,
-                           float* dk, float* dv, float* part, int* err, cudaStream_t s);
+                           float* dk, float* dv, float* part, int* err, cudaStream_t s,
+                           bool dO16_ready = false);
 
 // Parametric (one linear layer) compression, bf16, D = 64: kc = sum_i k rows
 // j d + i times W[i], same for vc (k_cmp_mlp.cu).  The backward overwrites

@@ -46,12 +46,16 @@ __device__ __forceinline__ void load8(const float* p, float* x) {
 // Eight threads per row, eight values each: every load of the row (dout and
 // the enabled branches' outputs) is issued before any is used, the three dot
 // products are reduced over the row's eight lanes.
+struct Half3 {
+  __half* p[3];  // per branch: the fp16 pair's hi half (lo follows nel later), or null
+};
+
 template <typename T>
 __global__ void __launch_bounds__(256)
 gate_bwd_kernel(const float* __restrict__ gates, const T* __restrict__ dout,
                 const T* __restrict__ oc, const T* __restrict__ os, const T* __restrict__ ow,
                 float* __restrict__ dgates, float* __restrict__ dOc, float* __restrict__ dOs,
-                float* __restrict__ dOw, long nrows, int mask) {
+                float* __restrict__ dOw, long nrows, int mask, Half3 h16, int* err) {
   const long t = (long)blockIdx.x * blockDim.x + threadIdx.x;
   const long row0 = t >> 3;
   const int sub = (int)(t & 7);
@@ -85,6 +89,25 @@ gate_bwd_kernel(const float* __restrict__ gates, const T* __restrict__ dout,
       float4* o = reinterpret_cast<float4*>(dst[i] + base);
       o[0] = make_float4(gi[i] * g[0], gi[i] * g[1], gi[i] * g[2], gi[i] * g[3]);
       o[1] = make_float4(gi[i] * g[4], gi[i] * g[5], gi[i] * g[6], gi[i] * g[7]);
+    }
+    if (h16.p[i]) {  // the same fp32 values as the fp16 pair hi + lo
+      uint32_t hw[4], lw[4];
+      bool range_ok = true;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float x0 = gi[i] * g[2 * e], x1 = gi[i] * g[2 * e + 1];
+        const float h0 = __half2float(__float2half_rn(x0));
+        const float h1 = __half2float(__float2half_rn(x1));
+        range_ok = range_ok && fabsf(x0) <= 65504.f && fabsf(x1) <= 65504.f;
+        const __half2 hh = __floats2half2_rn(h0, h1);
+        const __half2 ll = __floats2half2_rn(x0 - h0, x1 - h1);
+        hw[e] = *reinterpret_cast<const uint32_t*>(&hh);
+        lw[e] = *reinterpret_cast<const uint32_t*>(&ll);
+      }
+      if (!range_ok) record_error(err, kDevRange);
+      const size_t nel = (size_t)nrows * 64;
+      *reinterpret_cast<uint4*>(h16.p[i] + base) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      *reinterpret_cast<uint4*>(h16.p[i] + nel + base) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
     }
     if (sub == 0) dgates[row * 3 + i] = ((mask >> i) & 1) ? dg : 0.f;
   }
@@ -677,17 +700,22 @@ __global__ void pool_bwd_kernel(const float* __restrict__ dkc, const float* __re
 // ---- launchers ----------------------------------------------------------------------
 cudaError_t launch_gate_bwd(const Dims& d, const float* gates, const void* dout,
                             const void* o_cmp, const void* o_sel, const void* o_swa,
-                            float* dgates, float* dOc, float* dOs, float* dOw, cudaStream_t s) {
+                            float* dgates, float* dOc, float* dOs, float* dOw, cudaStream_t s,
+                            void* const* h16, int* err) {
+  Half3 hp{{nullptr, nullptr, nullptr}};
+  if (h16)
+    for (int i = 0; i < 3; ++i) hp.p[i] = (__half*)h16[i];
   const long nrows = (long)d.B * d.Tq * d.Hq;
   const unsigned blocks = (unsigned)((nrows * 8 + 255) / 256);
   if (d.dtype == 1)
     gate_bwd_kernel<bf16><<<blocks, 256, 0, s>>>(gates, (const bf16*)dout, (const bf16*)o_cmp,
                                                  (const bf16*)o_sel, (const bf16*)o_swa, dgates,
-                                                 dOc, dOs, dOw, nrows, d.branch_mask);
+                                                 dOc, dOs, dOw, nrows, d.branch_mask, hp, err);
   else
     gate_bwd_kernel<float><<<blocks, 256, 0, s>>>(gates, (const float*)dout, (const float*)o_cmp,
                                                   (const float*)o_sel, (const float*)o_swa,
-                                                  dgates, dOc, dOs, dOw, nrows, d.branch_mask);
+                                                  dgates, dOc, dOs, dOw, nrows, d.branch_mask, hp,
+                                                  err);
   return cudaGetLastError();
 }
 
@@ -769,10 +797,10 @@ static cudaError_t dkdv_t(const Dims& d, const void* q, const void* keys, const 
 cudaError_t launch_dkdv(const Dims& d, int mode, const void* q, const void* keys,
                         const void* vals, const float* lse, const float* delta, const float* dO,
                         void* dO16, const int* offsets, const int* list, float* dk, float* dv,
-                        float* part, int* err, cudaStream_t s) {
+                        float* part, int* err, cudaStream_t s, bool dO16_ready) {
   if (dkdv_tc_eligible(d, mode))
     return launch_dkdv_tc(d, mode, q, keys, vals, lse, delta, dO, dO16, offsets, list, dk, dv,
-                          part, err, s);
+                          part, err, s, dO16_ready);
   if (d.dtype == 1) {
     if (mode == kBwdSel) return dkdv_t<bf16, kBwdSel>(d, q, keys, vals, lse, delta, dO, offsets, list, dk, dv, s);
     if (mode == kBwdSwa) return dkdv_t<bf16, kBwdSwa>(d, q, keys, vals, lse, delta, dO, offsets, list, dk, dv, s);

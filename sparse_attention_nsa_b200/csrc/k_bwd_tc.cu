@@ -1132,14 +1132,15 @@ template <int MODE>
 cudaError_t launch_dkdv_tc_t(const Dims& d, const void* q, const void* k, const void* v,
                              const float* lse, const float* delta, const float* dO,
                              void* dO16, const int* offsets, const int* list, float* dk,
-                             float* dv, float* part, int* err, cudaStream_t s) {
+                             float* dv, float* part, int* err, cudaStream_t s, bool ready) {
   const int nkeys = MODE == 2 ? d.Nc : d.T;
   const int nchunk = (nkeys + kKeys - 1) / kKeys;
   const int npairs = (nchunk + 1) / 2;
   if (npairs == 0) return cudaSuccess;
   const size_t nel = (size_t)d.B * d.Tq * d.Hq * 64;
-  dO_split_f16_kernel<<<(unsigned)((nel / 8 + 255) / 256), 256, 0, s>>>(
-      dO, (__half*)dO16, (__half*)dO16 + nel, nel, err);
+  if (!ready)
+    dO_split_f16_kernel<<<(unsigned)((nel / 8 + 255) / 256), 256, 0, s>>>(
+        dO, (__half*)dO16, (__half*)dO16 + nel, nel, err);
   const int nseg = MODE == 2 ? kCmpShares : 1;
   CUtensorMap mk, mv;
   if (!make_tmap_bf16(&mk, k, d.Hkv, (long)d.B * nkeys, 1, kKeys) ||
@@ -1202,13 +1203,14 @@ size_t dkdv_cmp_part_bytes(const Dims& d) {
 cudaError_t launch_dkdv_tc(const Dims& d, int mode, const void* q, const void* k, const void* v,
                            const float* lse, const float* delta, const float* dO, void* dO16,
                            const int* offsets, const int* list, float* dk, float* dv, float* part,
-                           int* err, cudaStream_t s) {
+                           int* err, cudaStream_t s, bool dO16_ready) {
   void* o16 = dO16;
+  const bool r = dO16_ready;
   if (mode == 0)
-    return launch_dkdv_tc_t<0>(d, q, k, v, lse, delta, dO, o16, offsets, list, dk, dv, part, err, s);
+    return launch_dkdv_tc_t<0>(d, q, k, v, lse, delta, dO, o16, offsets, list, dk, dv, part, err, s, r);
   if (mode == 1)
-    return launch_dkdv_tc_t<1>(d, q, k, v, lse, delta, dO, o16, offsets, list, dk, dv, part, err, s);
-  return launch_dkdv_tc_t<2>(d, q, k, v, lse, delta, dO, o16, offsets, list, dk, dv, part, err, s);
+    return launch_dkdv_tc_t<1>(d, q, k, v, lse, delta, dO, o16, offsets, list, dk, dv, part, err, s, r);
+  return launch_dkdv_tc_t<2>(d, q, k, v, lse, delta, dO, o16, offsets, list, dk, dv, part, err, s, r);
 }
 
 // The single-pass selection backward: dQ as launch_dq_tc (mode 0), dK and

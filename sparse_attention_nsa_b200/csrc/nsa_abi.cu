@@ -602,9 +602,11 @@ namespace {
 //   dkc, dvc [B*Nc*Hkv*64] f32 | reverse-map chunk positions
 //   [B*Hkv*ceil(Tq/256)*Nb] i32 | offsets [B*Hkv*(Nb+1)] i32 |
 //   list [B*Hkv*Tq*topk] i32 | compression dK/dV row shares (tensor-core path) |
-//   dO split into fp16 hi, lo [2*B*Tq*Hq*64] (tensor-core dK/dV path)
+//   dO split into fp16 hi, lo [2*B*Tq*Hq*64] (tensor-core dK/dV path) |
+//   the whole backward's per-branch fp16 pairs, written by the gate backward
+//   [3][2*B*Tq*Hq*64] (tensor-core dK/dV path)
 struct BwdCarve {
-  size_t delta, dO[3], dkc, dvc, counts, offsets, list, part, dO16, total;
+  size_t delta, dO[3], dkc, dvc, counts, offsets, list, part, dO16, dO16b[3], total;
 };
 
 BwdCarve bwd_carve(const Dims& d) {
@@ -625,6 +627,8 @@ BwdCarve bwd_carve(const Dims& d) {
   c.list = take((size_t)d.B * d.Hkv * d.Tq * d.topk * 4);
   c.part = take(nsa::dkdv_tc_eligible(d, 2) ? nsa::dkdv_cmp_part_bytes(d) : 0);
   c.dO16 = take(nsa::dkdv_tc_eligible(d, 0) ? 2 * rows * 64 * 2 : 0);
+  for (int i = 0; i < 3; ++i)  // branch i: compression (mode 2), selection (0), window (1)
+    c.dO16b[i] = take(nsa::dkdv_tc_eligible(d, i == 0 ? 2 : i - 1) ? 2 * rows * 64 * 2 : 0);
   c.total = at;
   return c;
 }
@@ -636,26 +640,27 @@ bool ws_ok(const void* ws, size_t bytes, size_t need) {
 nsa_status sel_bwd_body(const Dims& d, const void* q, const void* k, const void* v,
                         const int32_t* idx, const void* o_sel, const float* lse_sel,
                         const float* dO_sel, float* dq, float* dk, float* dv, char* w,
-                        const BwdCarve& c, cudaStream_t s) {
+                        const BwdCarve& c, cudaStream_t s, void* pre16 = nullptr) {
   float* delta = (float*)(w + c.delta);
   int* counts = (int*)(w + c.counts);
   int* offsets = (int*)(w + c.offsets);
   int* list = (int*)(w + c.list);
   NSA_TRY_CUDA(nsa::launch_dq(d, 0, q, k, v, idx, o_sel, lse_sel, dO_sel, dq, delta, err_word(), s));
   NSA_TRY_CUDA(nsa::launch_revmap(d, idx, counts, offsets, list, s));
-  NSA_TRY_CUDA(nsa::launch_dkdv(d, 0, q, k, v, lse_sel, delta, dO_sel, w + c.dO16, offsets, list,
-                                dk, dv, nullptr, err_word(), s));
+  NSA_TRY_CUDA(nsa::launch_dkdv(d, 0, q, k, v, lse_sel, delta, dO_sel, pre16 ? pre16 : w + c.dO16,
+                                offsets, list, dk, dv, nullptr, err_word(), s, pre16 != nullptr));
   return NSA_OK;
 }
 
 nsa_status swa_bwd_body(const Dims& d, const void* q, const void* k, const void* v,
                         const void* o_swa, const float* lse_swa, const float* dO_swa,
                         float* dq, float* dk, float* dv, char* w, const BwdCarve& c,
-                        cudaStream_t s) {
+                        cudaStream_t s, void* pre16 = nullptr) {
   float* delta = (float*)(w + c.delta);
   NSA_TRY_CUDA(nsa::launch_dq(d, 1, q, k, v, nullptr, o_swa, lse_swa, dO_swa, dq, delta, nullptr, s));
-  NSA_TRY_CUDA(nsa::launch_dkdv(d, 1, q, k, v, lse_swa, delta, dO_swa, w + c.dO16, nullptr, nullptr,
-                                dk, dv, nullptr, err_word(), s));
+  NSA_TRY_CUDA(nsa::launch_dkdv(d, 1, q, k, v, lse_swa, delta, dO_swa, pre16 ? pre16 : w + c.dO16,
+                                nullptr, nullptr, dk, dv, nullptr, err_word(), s,
+                                pre16 != nullptr));
   return NSA_OK;
 }
 
@@ -670,7 +675,7 @@ struct MlpGrad {
 nsa_status cmp_bwd_body(const Dims& d, const void* q, const void* kc, const void* vc,
                         const void* o_cmp, const float* lse_cmp, const float* dO_cmp,
                         float* dq, float* dk, float* dv, char* w, const BwdCarve& c,
-                        cudaStream_t s, const MlpGrad* mlp = nullptr) {
+                        cudaStream_t s, const MlpGrad* mlp = nullptr, void* pre16 = nullptr) {
   float* delta = (float*)(w + c.delta);
   float* dkc = (float*)(w + c.dkc);
   float* dvc = (float*)(w + c.dvc);
@@ -684,9 +689,9 @@ nsa_status cmp_bwd_body(const Dims& d, const void* q, const void* kc, const void
   NSA_TRY_CUDA(cudaMemsetAsync(dkc, 0, nkc, s));
   NSA_TRY_CUDA(cudaMemsetAsync(dvc, 0, nkc, s));
   NSA_TRY_CUDA(nsa::launch_dq(d, 2, q, kc, vc, nullptr, o_cmp, lse_cmp, dO_cmp, dq, delta, nullptr, s));
-  NSA_TRY_CUDA(nsa::launch_dkdv(d, 2, q, kc, vc, lse_cmp, delta, dO_cmp, w + c.dO16, nullptr, nullptr,
-                                dkc, dvc,
-                                (float*)(w + c.part), err_word(), s));
+  NSA_TRY_CUDA(nsa::launch_dkdv(d, 2, q, kc, vc, lse_cmp, delta, dO_cmp, pre16 ? pre16 : w + c.dO16,
+                                nullptr, nullptr, dkc, dvc, (float*)(w + c.part), err_word(), s,
+                                pre16 != nullptr));
   if (mlp)
     NSA_TRY_CUDA(nsa::launch_cmp_mlp_bwd(d, mlp->k, mlp->v, mlp->wk, mlp->wv, dkc, dvc, dk, dv,
                                          mlp->dwk, mlp->dwv, mlp->ws, err_word(), s));
@@ -823,15 +828,21 @@ nsa_status backward_body(const Dims& d, const void* q, const void* k, const void
   char* w = (char*)workspace;
   if (mlp) mlp->ws = w + c.total;
   float* dO[3] = {(float*)(w + c.dO[0]), (float*)(w + c.dO[1]), (float*)(w + c.dO[2])};
+  // the gate backward also writes each tensor-core branch's dO as the fp16
+  // pair its dK/dV kernel reads, so those kernels skip their own split
+  const bool on[3] = {cmp && d.Nc > 0, sel, swa};
+  void* pre16[3];
+  for (int i = 0; i < 3; ++i)
+    pre16[i] = on[i] && nsa::dkdv_tc_eligible(d, i == 0 ? 2 : i - 1) ? w + c.dO16b[i] : nullptr;
   NSA_TRY_CUDA(nsa::launch_gate_bwd(d, gates, dout, sv->o_cmp, sv->o_sel, sv->o_swa, dgates,
                                     cmp ? dO[0] : nullptr, sel ? dO[1] : nullptr,
-                                    swa ? dO[2] : nullptr, s));
+                                    swa ? dO[2] : nullptr, s, pre16, err_word()));
   NSA_TRY_CUDA(cudaMemsetAsync(dq, 0, (size_t)d.B * d.Tq * d.Hq * 64 * 4, s));
   NSA_TRY_CUDA(cudaMemsetAsync(dk, 0, (size_t)d.B * d.T * d.Hkv * 64 * 4, s));
   NSA_TRY_CUDA(cudaMemsetAsync(dv, 0, (size_t)d.B * d.T * d.Hkv * 64 * 4, s));
   if (cmp) {
     st = cmp_bwd_body(d, q, sv->kc, sv->vc, sv->o_cmp, sv->lse_cmp, dO[0], dq, dk, dv, w, c, s,
-                      mlp);
+                      mlp, pre16[0]);
     if (st != NSA_OK) return st;
   } else if (mlp) {
     // compressed keys reach only the selection scores, and top-k passes no gradient
@@ -840,11 +851,12 @@ nsa_status backward_body(const Dims& d, const void* q, const void* k, const void
     NSA_TRY_CUDA(cudaMemsetAsync(mlp->dwv, 0, wbytes, s));
   }
   if (sel) {
-    st = sel_bwd_body(d, q, k, v, sv->idx, sv->o_sel, sv->lse_sel, dO[1], dq, dk, dv, w, c, s);
+    st = sel_bwd_body(d, q, k, v, sv->idx, sv->o_sel, sv->lse_sel, dO[1], dq, dk, dv, w, c, s,
+                      pre16[1]);
     if (st != NSA_OK) return st;
   }
   if (swa) {
-    st = swa_bwd_body(d, q, k, v, sv->o_swa, sv->lse_swa, dO[2], dq, dk, dv, w, c, s);
+    st = swa_bwd_body(d, q, k, v, sv->o_swa, sv->lse_swa, dO[2], dq, dk, dv, w, c, s, pre16[2]);
     if (st != NSA_OK) return st;
   }
   return NSA_OK;
