@@ -312,3 +312,22 @@ def test_backward_mlp_without_compression_branch_zeroes_weight_grads(cuda_lib):
     assert torch.count_nonzero(dwk) == 0 and torch.count_nonzero(dwv) == 0
     for a, b in zip((dq, dk, dv, dg), ref):
         assert torch.equal(a, b)
+
+
+def test_forward_mlp_chunked_queries_equal_the_full_forward_tail(cuda_lib):
+    """Queries as the last Tq positions (chunked prefill) see the same
+    compressed keys (the layer runs over all T keys), so their outputs are
+    the full forward's last Tq rows, bit for bit."""
+    w = CASES[0]
+    inp = W.make_inputs(w, seed=70)
+    wk, wv = (t.to(DEV) for t in weights(w))
+    d = dev(inp)
+    p = nsa.params_for(w)
+    full = nsa.forward_mlp(p, d["q"], d["k"], d["v"], wk, wv, d["gates"])
+    tq = w.T - 300
+    pc = nsa.params_for(w, Tq=tq)
+    part = nsa.forward_mlp(pc, d["q"][:, w.T - tq:].contiguous(), d["k"], d["v"], wk, wv,
+                           d["gates"][:, w.T - tq:].contiguous())
+    torch.cuda.synchronize()
+    assert nsa.nsa_last_device_error() == 0
+    assert torch.equal(part, full[:, w.T - tq:])
