@@ -45,13 +45,13 @@ DECODE = W.DECODE_32K
 
 def kernels_per_forward(w) -> int:
     """Kernels one nsa_forward of workload w launches (as its ncu launch list
-    shows): pooling, compression branch + scores, top-k, window (side
-    stream), then either the query-tiled selection with the combination, or
-    (block-major, from Nb >= 8 top-k and Tq >= 64) the reverse map's count,
-    scan and fill, the selection kernel and the merge with the combination."""
+    shows): pooling, compression branch + scores, top-k, window, then either
+    the query-tiled selection with the combination, or (block-major, from Nb
+    >= 8 top-k and Tq >= 64) the reverse map's scan and fill (the top-k does
+    its counting), the selection kernel and the merge with the combination."""
     nb = -(-w.T // w.sel_block)
     block_major = w.dtype == torch.bfloat16 and nb >= 8 * w.topk and w.T >= 64
-    return 4 + (5 if block_major else 1)
+    return 4 + (4 if block_major else 1)
 
 
 # ------------------------------------------------------------------ work model
