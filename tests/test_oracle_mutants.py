@@ -59,6 +59,25 @@ MUTANTS = {
                                  "if (clo <= hi && chi > lo) acc += cmp_score_row[i];"),
     "remap_first_block_only": ("if (clo < hi && chi > lo) acc += cmp_score_row[i];",
                                "if (clo >= lo && clo < hi) { acc += cmp_score_row[i]; break; }"),
+    "current_block_not_forced": ("idx_row[cnt++] = cur;", "idx_row[cnt++] = cur - 1;"),
+    "dq_uses_query_not_key": ("dq[d] += scale * ds * krows[s][d];", "dq[d] += scale * ds * qrow[d];"),
+    "softmax_not_normalised": ("double p = logit[s] / sum;", "double p = logit[s];"),
+    "delta_uses_first_value_row": ("double delta = dot(dO, o, D);",
+                                   "double delta = dot(dO, vrows[0], D);"),
+    "pool_key_ignores_stride": ("sk += k[KI(c, b, j * dstr + i, g) + d];",
+                                "sk += k[KI(c, b, j * l + i, g) + d];"),
+    "window_excludes_query": ("for (int p = lo; p <= t; ++p) pos[n++] = p;",
+                              "for (int p = lo; p < t; ++p) pos[n++] = p;"),
+    "decode_reads_previous_row": ("b, L - 1, oc,", "b, L - 2, oc,"),
+    "gate_bwd_ignores_branch_mask": ("dob[i][d] = on ? gates[(size_t)r * 3 + i] * dO[d] : 0.0;",
+                                     "dob[i][d] = gates[(size_t)r * 3 + i] * dO[d];"),
+    "dgates_scaled_by_gate": ("dgates[(size_t)r * 3 + i] = on ? dot(dO, ob[i], D) : 0.0;",
+                              "dgates[(size_t)r * 3 + i] = on ? gates[(size_t)r * 3 + i] * dot(dO, ob[i], D) : 0.0;"),
+    "moba_prefers_lowest_gate": ("    gate[j] = acc;", "    gate[j] = -acc;"),
+    "mlp_bwd_row_grad_transposed": ("ak += wk[((size_t)i * D + e) * D + n] * gk;",
+                                    "ak += wk[((size_t)i * D + n) * D + e] * gk;"),
+    "mlp_bwd_row_grad_first_block_only": ("            dk[rowi] += ak;",
+                                          "            if (j == 0) dk[rowi] += ak;"),
 }
 
 

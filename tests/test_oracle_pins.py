@@ -393,6 +393,30 @@ def test_gate_combine_is_linear_and_respects_branch_mask():
     np.testing.assert_allclose(r["out"], want, rtol=0, atol=1e-15)
 
 
+@pytest.mark.parametrize("mask", [7, 6, 5, 3, 4, 1])
+def test_gate_combine_bwd_is_autograd_of_the_masked_sum(mask):
+    """The combination's backward against torch autograd of
+    out = sum over the kept branches of gate_i * o_i: a pruned branch gets
+    neither a gate gradient nor an output gradient ("Sparsity is Cool",
+    Key claims: unused branches are dropped)."""
+    c = cfg_small(branch_mask=mask)
+    rng = np.random.default_rng(40 + mask)
+    shp = (c.B, c.T, c.Hq, c.D)
+    gates = rng.random((c.B, c.T, c.Hq, 3))
+    o3 = [rng.standard_normal(shp) for _ in range(3)]
+    dout = rng.standard_normal(shp)
+    gt = torch.from_numpy(gates).requires_grad_()
+    ot = [torch.from_numpy(o).requires_grad_() for o in o3]
+    bits = (orc.BR_CMP, orc.BR_SEL, orc.BR_SWA)
+    out = sum(gt[..., i:i + 1] * ot[i] for i in range(3) if mask & bits[i])
+    (out * torch.from_numpy(dout)).sum().backward()
+    dg, *dO = orc.gate_combine_bwd(c, gates, dout, *o3)
+    np.testing.assert_allclose(dg, gt.grad.numpy(), rtol=1e-13, atol=1e-13)
+    for i in range(3):
+        want = ot[i].grad.numpy() if ot[i].grad is not None else np.zeros(shp)
+        np.testing.assert_allclose(dO[i], want, rtol=0, atol=1e-15)
+
+
 def test_dense_degeneration_at_short_context():
     """With block 64, top-k 16 and window 512, a 1024-token sequence selects
     every causal block, so the selection branch is dense causal attention,
