@@ -169,3 +169,53 @@ def test_parametric_compression_checks_before_launch():
     # enough output tiles: one CTA per tile, no partial sums
     wide = nsa.make_params(1, 2400, 64, 64, cmp_block=32, cmp_stride=16, window=64)
     assert nsa.nsa_compress_mlp_workspace_size(wide) == 0
+
+
+MOBA_CASES = [
+    (dict(), 0),                                  # block 512, top-3 at T 8192
+    (dict(block=64, topk=16), 0),                 # 128 blocks of 64
+    (dict(block=0), 1), (dict(topk=0), 1), (dict(Hkv=3), 1), (dict(scale=float("nan")), 1),
+    (dict(block=100), 2),                         # not a multiple of 64
+    (dict(block=64, topk=1), 2),                  # one 64-key block: below the kernels' two
+    (dict(block=64, T=16384), 2),                 # 256 MoBA blocks > 128
+    (dict(topk=9), 2),                            # 9 x 8 = 72 selection blocks > 64
+    (dict(T=131072, block=1024), 2),              # 2048 64-key blocks > 1024
+    (dict(D=128), 2),
+]
+
+
+@pytest.mark.parametrize("change,code", MOBA_CASES)
+def test_moba_params_checked_before_launch(change, code):
+    """MoBA's limits (MoBA blocks of a multiple of 64 tokens, at most 128 of
+    them, k L / 64 <= 64 selection blocks) and the shared parameter checks,
+    all answered by the workspace query without a device."""
+    base = dict(B=1, T=8192, Hq=16, Hkv=4, block=512, topk=3)
+    base.update({k: v for k, v in change.items() if k in base})
+    p = nsa.make_moba_params(**base)
+    for k, v in change.items():
+        if k not in base:
+            setattr(p, k, v)
+    n = C.c_size_t(0)
+    assert nsa.load().nsa_moba_workspace_size(C.byref(p), C.byref(n)) == code
+    if code == 0:
+        assert n.value > 0
+
+
+def test_moba_pointer_and_workspace_checks():
+    """Every case fails a check before anything is enqueued (the pointers
+    are never dereferenced)."""
+    lib = nsa.load()
+    p = nsa.make_moba_params(1, 8192, 16, 4)
+    need = nsa.nsa_moba_workspace_size(p)
+    ptr = C.c_void_p(4096)  # aligned, never dereferenced: the checks come first
+    assert lib.nsa_moba_forward(C.byref(p), None, ptr, ptr, ptr, None, None, ptr, need,
+                                None) == 1
+    assert lib.nsa_moba_forward(C.byref(p), ptr, ptr, ptr, ptr, C.c_void_p(4100), None, ptr,
+                                need, None) == 1  # misaligned lse
+    assert lib.nsa_moba_forward(C.byref(p), ptr, ptr, ptr, ptr, None, None, ptr, 0,
+                                None) == 6  # NSA_ERR_WORKSPACE
+    assert lib.nsa_moba_forward(C.byref(p), ptr, ptr, ptr, ptr, None, None, None, need,
+                                None) == 6
+    assert lib.nsa_moba_backward(C.byref(p), *([ptr] * 6), None, *([ptr] * 3), ptr, need,
+                                 None) == 1  # no dout
+    assert lib.nsa_moba_backward(C.byref(p), *([ptr] * 10), None, 0, None) == 6
