@@ -315,8 +315,19 @@ def oracle_tokens_per_s(budget_s: float, seed: int = 0) -> dict:
                       f"precomputed; {dt:.1f} s"}
 
 
+def workload_config(w, world: int) -> dict:
+    """The JSON line's config, the same for both arms: the workload, the L2
+    treatment between timed GPU steps, and how the ranks divide the work."""
+    return {"workload": w.name, "B": w.B, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
+            "block": w.sel_block, "topk": w.topk, "window": w.window,
+            "l2": "flushed between GPU steps (256 MiB write); the CPU oracle reads a "
+                  "fresh sample each step",
+            "parallelism": f"replicas x{world} (independent sequences, no collective "
+                           "on the data path)"}
+
+
 # ------------------------------------------------------------------ main legs
-def run_reference(args, rank: int) -> None:
+def run_reference(args, rank: int, world: int) -> None:
     if rank != 0:
         return
     budget = max(2.0, min(20.0, 25.0 / max(args.steps, 1)))
@@ -333,9 +344,7 @@ def run_reference(args, rank: int) -> None:
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": WORK.B * WORK.T / v * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": WORK.name, "B": WORK.B, "T": WORK.T, "Hq": WORK.Hq,
-                       "Hkv": WORK.Hkv, "D": WORK.D, "block": WORK.sel_block,
-                       "topk": WORK.topk, "window": WORK.window},
+            "config": workload_config(WORK, world),
             "cpu_baseline": cb,
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -443,10 +452,7 @@ def run_gpu(args, rank: int, world: int, dist_on: bool) -> None:
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv,
-                   "D": w.D, "block": w.sel_block, "topk": w.topk, "window": w.window,
-                   "l2": "flushed between steps (256 MiB write)",
-                   "parallelism": f"replicas x{world}"},
+        "config": workload_config(w, world),
         "tflops": flops["total"] * world / (ms * 1e-3) / 1e12,
         "frac_bf16_peak": flops["total"] / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
         "flops_per_step": flops,
@@ -836,7 +842,7 @@ def main():
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
-        run_reference(args, rank)
+        run_reference(args, rank, world)
         return
     if args.leg not in ("all", "forward"):
         dev = torch.device("cuda", 0)

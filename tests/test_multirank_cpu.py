@@ -74,3 +74,31 @@ def test_fwd_flops_matches_the_counting_rule():
     assert f["sel"] == 31_289_507_840
     assert f["swa"] == 16_644_046_848
     assert f["cmp"] == 2_131_230_720
+
+
+def test_reference_arm_line_matches_the_gpu_arm_config(monkeypatch, capsys):
+    """The reference arm (the fp64 oracle on the host cores) prints one line
+    on rank 0 only, with the GPU arm's config; the oracle timing itself is
+    stubbed here (bench's cpu_baseline leg runs it for real)."""
+    import argparse
+    import json
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    calls = []
+
+    def fake(budget_s, seed=0):
+        calls.append(budget_s)
+        return {"value": 1000.0 + len(calls), "unit": "tokens/s", "cores": 4,
+                "kind": "oracle", "sample": "stub"}
+
+    monkeypatch.setattr(bench, "oracle_tokens_per_s", fake)
+    args = argparse.Namespace(gpus=2, steps=2, warmup=3)
+    bench.run_reference(args, rank=1, world=2)
+    assert capsys.readouterr().out == "" and not calls
+    bench.run_reference(args, rank=0, world=2)
+    line = json.loads(capsys.readouterr().out.strip())
+    assert len(calls) == 5 and calls[:3] == [1.0] * 3
+    assert line["impl"] == "reference" and line["config"] == bench.workload_config(bench.WORK, 2)
+    assert line["value"] == 1004.5 and line["e2e"]["value"] == line["value"]
+    assert line["cpu_baseline"]["value"] == line["value"]
