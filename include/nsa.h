@@ -85,9 +85,9 @@ enum {
  * statement: compression block size l and stride d, selection block size l',
  * top-k n, window w ("Sparsity is Cool", Method, uses l = d = l' = 64).
  * Any l, d, l' >= 1 run, up to 1024 selection blocks and 1024 compressed
- * blocks per sequence (NSA_ERR_UNSUPPORTED beyond); the bf16 tensor-core
- * selection, window and backward kernels take l' = 64, other l' the CUDA-core
- * kernels. */
+ * blocks per sequence and B T < 2^31 key rows (NSA_ERR_UNSUPPORTED beyond);
+ * the bf16 tensor-core selection, window and backward kernels take l' = 64,
+ * other l' the CUDA-core kernels. */
 typedef struct {
   int B, T, Tq, Hq, Hkv, D;
   int cmp_block;   /* l  : tokens per compressed block              */

@@ -57,9 +57,12 @@ nsa_status fill_dims(const nsa_params* p, Dims* d) {
   if (G > 32 || (G & (G - 1)) != 0) return NSA_ERR_UNSUPPORTED;
   if (p->Hkv > 64 || p->topk > 64) return NSA_ERR_UNSUPPORTED;
   const int l = p->sel_block;
-  const int Nb = (p->T + l - 1) / l;
+  const long long Nb = ((long long)p->T + l - 1) / l;  // T + l - 1 may pass INT_MAX
   const int Nc = p->T < p->cmp_block ? 0 : (p->T - p->cmp_block) / p->cmp_stride + 1;
   if (Nb > 1024 || Nc > 1024) return NSA_ERR_UNSUPPORTED;
+  // key / value rows (b T + t) are addressed by signed 32-bit tensor-map
+  // coordinates
+  if ((long long)p->B * p->T >= (1LL << 31)) return NSA_ERR_UNSUPPORTED;
   d->B = p->B;
   d->T = p->T;
   d->Tq = p->Tq;
@@ -71,7 +74,7 @@ nsa_status fill_dims(const nsa_params* p, Dims* d) {
   d->lc = p->cmp_block;
   d->dc = p->cmp_stride;
   d->Nc = Nc;
-  d->Nb = Nb;
+  d->Nb = (int)Nb;
   d->topk = p->topk;
   d->window = p->window;
   d->scale = p->scale;

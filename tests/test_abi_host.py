@@ -56,6 +56,10 @@ BAD = [
     (dict(scale=float("inf")), 1),
     (dict(D=128), 2), (dict(cmp_stride=2), 2), (dict(sel_block=2), 2),
     (dict(Hq=24, Hkv=4), 2), (dict(topk=65), 2), (dict(T=200000), 2),
+    # T + l' - 1 past INT_MAX: the block count must not wrap to a negative number
+    (dict(T=2**31 - 1, cmp_block=2**31 - 1, cmp_stride=1, sel_block=2), 2),
+    # B T >= 2^31 key rows (32-bit tensor-map coordinates), geometry otherwise valid
+    (dict(B=2**15, T=2**16, cmp_block=2**16, sel_block=2**10), 2),
 ]
 
 
