@@ -1033,7 +1033,8 @@ nsa_status fill_moba_dims(const nsa_moba_params* p, Dims* d) {
   q.branch_mask = NSA_BRANCH_SEL;
   nsa_status st = fill_dims(&q, d);
   if (st != NSA_OK) return st;
-  if (p->block % 64 != 0 || p->T / p->block > 128 || p->topk * (p->block / 64) > 64)
+  if (p->block % 64 != 0 || p->T / p->block > 128 ||
+      (long long)p->topk * (p->block / 64) > 64)  // k <= 64 also bounds the MoBA index rows
     return NSA_ERR_UNSUPPORTED;
   d->topk = p->topk * (p->block / 64);
   if (d->topk < 2) return NSA_ERR_UNSUPPORTED;  // the selection kernels take >= 2 blocks

@@ -184,6 +184,7 @@ MOBA_CASES = [
     (dict(block=64, T=16384), 2),                 # 256 MoBA blocks > 128
     (dict(topk=9), 2),                            # 9 x 8 = 72 selection blocks > 64
     (dict(T=131072, block=1024), 2),              # 2048 64-key blocks > 1024
+    (dict(block=256, topk=2**30 + 4), 2),         # k L / 64 wraps to 16 in 32 bits
     (dict(D=128), 2),
 ]
 
