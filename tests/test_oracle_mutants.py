@@ -9,6 +9,7 @@ never in the CUDA library.
 import os
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 import pytest
 
@@ -81,18 +82,41 @@ MUTANTS = {
 }
 
 
-@pytest.mark.parametrize("name", sorted(MUTANTS))
-def test_pins_reject_mutant(name, tmp_path):
+def _run_mutant(name: str, workdir: str) -> tuple:
+    """Build the oracle with mutant `name` planted and run the pin suite on
+    it; returns (pin-suite exit code, the end of its output)."""
     old, new = MUTANTS[name]
     src = open(SRC).read()
-    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
-    mut = tmp_path / "mutant.c"
-    mut.write_text(src.replace(old, new))
-    lib = tmp_path / "libmutant.so"
-    subprocess.run(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-o",
-                    str(lib), str(mut), "-lm"], check=True)
-    env = dict(os.environ, NSA_ORACLE_LIB=str(lib), OMP_NUM_THREADS="2")
+    if src.count(old) != 1:
+        return None, f"mutation site for {name} not found exactly once"
+    mut = os.path.join(workdir, f"{name}.c")
+    with open(mut, "w") as f:
+        f.write(src.replace(old, new))
+    lib = os.path.join(workdir, f"lib{name}.so")
+    subprocess.run(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-o", lib, mut,
+                    "-lm"], check=True)
+    env = dict(os.environ, NSA_ORACLE_LIB=lib, OMP_NUM_THREADS="2")
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
                         os.path.join(ROOT, "tests", "test_oracle_pins.py")],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
-    assert r.returncode != 0, f"pins accepted mutant {name}:\n{r.stdout[-2000:]}"
+    return r.returncode, r.stdout[-2000:]
+
+
+@pytest.fixture(scope="module")
+def mutant_results(request, tmp_path_factory):
+    """The selected mutants, run a few at a time (each pin run is one
+    process with two OpenMP threads)."""
+    names = sorted({item.callspec.params["name"] for item in request.session.items
+                    if item.originalname == "test_pins_reject_mutant"})
+    workdir = str(tmp_path_factory.mktemp("mutants"))
+    workers = max(1, min(4, (os.cpu_count() or 2) // 2))
+    with ThreadPoolExecutor(max_workers=workers) as ex:
+        futs = {n: ex.submit(_run_mutant, n, workdir) for n in names}
+        return {n: f.result() for n, f in futs.items()}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_reject_mutant(name, mutant_results):
+    code, out = mutant_results[name]
+    assert code is not None, out
+    assert code != 0, f"pins accepted mutant {name}:\n{out}"
