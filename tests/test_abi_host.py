@@ -224,3 +224,28 @@ def test_moba_pointer_and_workspace_checks():
     assert lib.nsa_moba_backward(C.byref(p), *([ptr] * 6), None, *([ptr] * 3), ptr, need,
                                  None) == 1  # no dout
     assert lib.nsa_moba_backward(C.byref(p), *([ptr] * 10), None, 0, None) == 6
+
+
+def test_binding_checks_tensors_before_calling_the_library():
+    """The binding's marshalling refuses host tensors where the library
+    wants device pointers (and the reverse for the host-buffer forward),
+    non-contiguous tensors, wrong dtypes and wrong shapes, before any call
+    into the library."""
+    import torch
+    p = nsa.make_params(1, 256, 4, 1, cmp_block=32, topk=4, window=64, dtype=nsa.NSA_F32)
+    q = torch.zeros(1, 256, 4, 64)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        nsa.nsa_swa_fwd(p, q, q[:, :, :1], q[:, :, :1], q, torch.zeros(1, 256, 4))
+    with pytest.raises(ValueError, match="required"):
+        abi._ptr(None, name="q")
+    assert abi._ptr(None, name="lse", nullable=True) is None
+    with pytest.raises(TypeError):
+        abi._ptr([0.0], name="q")
+    s = abi._shapes(p)
+    with pytest.raises(ValueError, match="contiguous"):
+        abi._host_ptr(torch.zeros(1, 4, 256, 64).transpose(1, 2), s["q"], torch.float32, "q")
+    with pytest.raises(ValueError, match="float32"):
+        abi._host_ptr(torch.zeros(s["q"], dtype=torch.float64), s["q"], torch.float32, "q")
+    with pytest.raises(ValueError, match="shape"):
+        abi._host_ptr(torch.zeros(1, 255, 4, 64), s["q"], torch.float32, "q")
+    assert abi._host_ptr(q, s["q"], torch.float32, "q").value == q.data_ptr()
